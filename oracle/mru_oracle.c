@@ -1,0 +1,368 @@
+/*
+ * mru_oracle.c -- plain, slow, fp64 CPU oracle for the Matrix Recurrent Unit
+ * (MRU) prefix-product scan.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the CPU
+ * baseline leg of the benchmark load this library.  It shares no code, header,
+ * table or helper with the CUDA library; it reads the same input bytes and
+ * nothing else.
+ *
+ * What it computes (sources are the web pages the method is described on):
+ *
+ *   "MRU Update: An independent developer's alternative to Attention is now
+ *    running successfully", section "What MRU Actually Does":
+ *     1. each token's embedding is reshaped into an input state matrix X_t;
+ *     2. the matrices are multiplied together along the sequence, the state
+ *        being multiplied by the new input matrix at every step, i.e.
+ *        S_t = S_{t-1} . X_t with S_0 = I (right multiplication);
+ *     3. the state matrix is mapped back to a vector.
+ *   "Improving Matrix Recurrent Units as an Attention Alternative", section
+ *   "Key Points" and "Technical Deep Dive": two construction variants,
+ *     - determinant correction: a scalar keeps det(X) at unit magnitude;
+ *       read here as X = Xr / |det Xr|^(1/n) (sign of det kept);
+ *     - LDU factor filling: X = L . D . U with L unit lower, U unit upper,
+ *       D diagonal; read here as L = I + a*strict_lower(M),
+ *       U = I + a*strict_upper(M), D = diag(exp(d*tanh(M_ii))).
+ *
+ * The oracle is the plain definition written out: every X_t is built in fp64
+ * from the widened input, and S_t is the serial left-to-right product with a
+ * textbook triple loop.  No blocking, no reordering, no library BLAS.  The
+ * determinant uses textbook LU with partial pivoting.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    int64_t B, H, L;
+    int32_t n;
+    int32_t x_dtype;      /* 0: float32, 1: bfloat16 (raw 16-bit patterns) */
+    int32_t mode;         /* 0: reshape, 1: determinant-corrected, 2: LDU fill */
+    float alpha;          /* Xr = add_identity*I + alpha*M (modes 0 and 1) */
+    int32_t add_identity;
+    float ldu_offdiag;    /* a in L = I + a*strict_lower(M), U = I + a*strict_upper(M) */
+    float ldu_diag;       /* d in D = diag(exp(d*tanh(M_ii))) */
+} mro_problem;
+
+enum { MRO_OK = 0, MRO_ERR_ARG = 1, MRO_ERR_SINGULAR = 5 };
+
+/* ---- input widening -------------------------------------------------- */
+
+/* bfloat16 is the top half of an IEEE binary32 pattern: widening is exact. */
+double mro_bf16_to_double(uint16_t bits)
+{
+    uint32_t w = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &w, sizeof f);
+    return (double)f;
+}
+
+static double widen(const mro_problem* p, const void* x, int64_t idx)
+{
+    if (p->x_dtype == 1)
+        return mro_bf16_to_double(((const uint16_t*)x)[idx]);
+    return (double)((const float*)x)[idx];
+}
+
+/* ---- textbook dense helpers (row-major n x n) ------------------------ */
+
+static void matmul(int n, const double* A, const double* Bm, double* C)
+{
+    for (int i = 0; i < n; ++i)
+        for (int j = 0; j < n; ++j) {
+            double s = 0.0;
+            for (int k = 0; k < n; ++k)
+                s += A[i * n + k] * Bm[k * n + j];
+            C[i * n + j] = s;
+        }
+}
+
+static void set_identity(int n, double* A)
+{
+    for (int i = 0; i < n * n; ++i) A[i] = 0.0;
+    for (int i = 0; i < n; ++i) A[i * n + i] = 1.0;
+}
+
+/* log|det A| and sign(det A) by LU with partial pivoting (A is destroyed).
+ * Returns 0 when det A == 0 (an exact zero pivot). */
+static int log_abs_det(int n, double* A, double* logabs, int* sign)
+{
+    double acc = 0.0;
+    int sg = 1;
+    for (int k = 0; k < n; ++k) {
+        int piv = k;
+        double best = fabs(A[k * n + k]);
+        for (int i = k + 1; i < n; ++i)
+            if (fabs(A[i * n + k]) > best) { best = fabs(A[i * n + k]); piv = i; }
+        if (best == 0.0) return 0;
+        if (piv != k) {
+            for (int j = 0; j < n; ++j) {
+                double t = A[k * n + j]; A[k * n + j] = A[piv * n + j]; A[piv * n + j] = t;
+            }
+            sg = -sg;
+        }
+        double pk = A[k * n + k];
+        if (pk < 0) sg = -sg;
+        acc += log(fabs(pk));
+        for (int i = k + 1; i < n; ++i) {
+            double l = A[i * n + k] / pk;
+            for (int j = k + 1; j < n; ++j)
+                A[i * n + j] -= l * A[k * n + j];
+        }
+    }
+    *logabs = acc;
+    *sign = sg;
+    return 1;
+}
+
+/* ---- step 1: lift one token-head embedding slice to X_t ----------------
+ * The slice of head h is x[b, t, h*n*n : (h+1)*n*n], viewed row-major as
+ * n x n: M[i][j] = x[... + i*n + j].  work must hold 3*n*n doubles. */
+int mro_lift(const mro_problem* p, const void* x, int64_t b, int64_t t, int64_t h,
+             double* X, double* work)
+{
+    const int n = p->n;
+    const int64_t nn = (int64_t)n * n;
+    const int64_t base = ((b * p->L + t) * p->H + h) * nn;
+    double* M = work;
+    for (int64_t e = 0; e < nn; ++e) M[e] = widen(p, x, base + e);
+
+    if (p->mode == 0 || p->mode == 1) {
+        const double a = (double)p->alpha;
+        for (int64_t e = 0; e < nn; ++e) X[e] = a * M[e];
+        if (p->add_identity)
+            for (int i = 0; i < n; ++i) X[i * n + i] += 1.0;
+        if (p->mode == 1) {
+            double* A = work + nn;
+            memcpy(A, X, (size_t)nn * sizeof(double));
+            double la; int sg;
+            if (!log_abs_det(n, A, &la, &sg) || !isfinite(la)) return MRO_ERR_SINGULAR;
+            const double c = exp(-la / n);   /* |det X|^(-1/n) */
+            for (int64_t e = 0; e < nn; ++e) X[e] *= c;
+        }
+        return MRO_OK;
+    }
+    if (p->mode == 2) {
+        const double a = (double)p->ldu_offdiag, d = (double)p->ldu_diag;
+        double* Lm = work + nn;
+        double* DU = work + 2 * nn;
+        set_identity(n, Lm);
+        set_identity(n, DU);
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j) {
+                if (i > j) Lm[i * n + j] = a * M[i * n + j];
+                if (i < j) DU[i * n + j] = a * M[i * n + j];
+            }
+        /* DU = D . U (row i of U scaled by D_i), then X = L . DU */
+        for (int i = 0; i < n; ++i) {
+            const double Di = exp(d * tanh(M[i * n + i]));
+            for (int j = 0; j < n; ++j) DU[i * n + j] *= Di;
+        }
+        matmul(n, Lm, DU, X);
+        return MRO_OK;
+    }
+    return MRO_ERR_ARG;
+}
+
+/* ---- step 2: the serial left-to-right product ------------------------- */
+
+typedef struct {
+    const mro_problem* p;
+    const void* x;
+    const double* S0;        /* [B,H,n,n] or NULL (identity) */
+    double* S_all;           /* [B,L,H,n,n] or NULL */
+    /* comparison targets (all optional) */
+    const float* S_gpu;      /* [B,L,H,n,n] */
+    const double* u;         /* [n] readout vector */
+    const float* o_gpu;      /* [B,L,H,n] */
+    double* o_all;           /* [B,L,H,n] oracle readout, optional */
+    int64_t snap_every;      /* 0: none */
+    const float* snap_gpu;   /* [B,L/snap_every,H,n,n] */
+    double* snap_all;        /* oracle snapshots, optional */
+    double* dS;              /* [B,L,H] squared Frobenius norm of the difference */
+    double* rS;              /* [B,L,H] squared Frobenius norm of the oracle S_t */
+    double* dO;              /* [B,L,H] */
+    double* rO;
+    double* dP;              /* [B,L/snap_every,H] */
+    double* rP;
+    int64_t t_end;           /* process t in [0, t_end) */
+    const int64_t* bh;       /* list of (b*H + h) */
+    int64_t n_bh;
+    int64_t next;            /* work counter (under lock) */
+    pthread_mutex_t lock;
+    int status;
+} job_t;
+
+static void run_sequence(job_t* J, int64_t bh_idx)
+{
+    const mro_problem* p = J->p;
+    const int n = p->n;
+    const int64_t nn = (int64_t)n * n;
+    const int64_t b = bh_idx / p->H, h = bh_idx % p->H;
+    double* S = malloc(sizeof(double) * nn);
+    double* Sn = malloc(sizeof(double) * nn);
+    double* X = malloc(sizeof(double) * nn);
+    double* work = malloc(sizeof(double) * 3 * nn);
+    if (!S || !Sn || !X || !work) { J->status = MRO_ERR_ARG; goto done; }
+
+    if (J->S0) memcpy(S, J->S0 + (b * p->H + h) * nn, sizeof(double) * nn);
+    else set_identity(n, S);
+
+    for (int64_t t = 0; t < J->t_end; ++t) {
+        int rc = mro_lift(p, J->x, b, t, h, X, work);
+        if (rc != MRO_OK) { J->status = rc; goto done; }
+        matmul(n, S, X, Sn);                       /* S_t = S_{t-1} . X_t */
+        double* sw = S; S = Sn; Sn = sw;
+
+        const int64_t row = (b * p->L + t) * p->H + h;   /* index of (b,t,h) */
+        if (J->S_all) memcpy(J->S_all + row * nn, S, sizeof(double) * nn);
+        if (J->S_gpu) {
+            double d2 = 0.0, r2 = 0.0;
+            const float* g = J->S_gpu + row * nn;
+            for (int64_t e = 0; e < nn; ++e) {
+                double df = (double)g[e] - S[e];
+                d2 += df * df;
+                r2 += S[e] * S[e];
+            }
+            J->dS[row] = d2;
+            J->rS[row] = r2;
+        }
+        if (J->u && (J->o_gpu || J->o_all)) {
+            double d2 = 0.0, r2 = 0.0;
+            for (int i = 0; i < n; ++i) {
+                double o = 0.0;                    /* o_t = S_t . u */
+                for (int j = 0; j < n; ++j) o += S[i * n + j] * J->u[j];
+                if (J->o_all) J->o_all[row * n + i] = o;
+                if (J->o_gpu) {
+                    double df = (double)J->o_gpu[row * n + i] - o;
+                    d2 += df * df;
+                    r2 += o * o;
+                }
+            }
+            if (J->o_gpu) { J->dO[row] = d2; J->rO[row] = r2; }
+        }
+        if (J->snap_every > 0 && ((t + 1) % J->snap_every) == 0) {
+            const int64_t k = (t + 1) / J->snap_every - 1;     /* 1-based t = (k+1)*every */
+            const int64_t L_s = p->L / J->snap_every;
+            const int64_t srow = (b * L_s + k) * p->H + h;
+            if (J->snap_all) memcpy(J->snap_all + srow * nn, S, sizeof(double) * nn);
+            if (J->snap_gpu) {
+                double d2 = 0.0, r2 = 0.0;
+                const float* g = J->snap_gpu + srow * nn;
+                for (int64_t e = 0; e < nn; ++e) {
+                    double df = (double)g[e] - S[e];
+                    d2 += df * df;
+                    r2 += S[e] * S[e];
+                }
+                J->dP[srow] = d2;
+                J->rP[srow] = r2;
+            }
+        }
+    }
+done:
+    free(S); free(Sn); free(X); free(work);
+}
+
+static void* worker(void* arg)
+{
+    job_t* J = (job_t*)arg;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int64_t i = J->next++;
+        int st = J->status;
+        pthread_mutex_unlock(&J->lock);
+        if (i >= J->n_bh || st != MRO_OK) break;
+        run_sequence(J, J->bh[i]);
+    }
+    return NULL;
+}
+
+static int run_job(job_t* J, int nthreads)
+{
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > J->n_bh) nthreads = (int)(J->n_bh > 0 ? J->n_bh : 1);
+    pthread_mutex_init(&J->lock, NULL);
+    J->next = 0;
+    J->status = MRO_OK;
+    pthread_t* th = malloc(sizeof(pthread_t) * nthreads);
+    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, worker, J);
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&J->lock);
+    return J->status;
+}
+
+static int check_problem(const mro_problem* p)
+{
+    if (!p || p->B < 0 || p->H < 0 || p->L < 0 || p->n < 1) return MRO_ERR_ARG;
+    if (p->x_dtype != 0 && p->x_dtype != 1) return MRO_ERR_ARG;
+    if (p->mode < 0 || p->mode > 2) return MRO_ERR_ARG;
+    return MRO_OK;
+}
+
+/* All states S_t (fp64) for every (b, t, h): S_all is [B, L, H, n, n]. */
+int mro_scan(const mro_problem* p, const void* x, const double* S0, double* S_all,
+             int nthreads)
+{
+    if (check_problem(p) != MRO_OK) return MRO_ERR_ARG;
+    const int64_t nbh = p->B * p->H;
+    int64_t* bh = malloc(sizeof(int64_t) * (nbh > 0 ? nbh : 1));
+    for (int64_t i = 0; i < nbh; ++i) bh[i] = i;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.p = p; J.x = x; J.S0 = S0; J.S_all = S_all;
+    J.t_end = p->L; J.bh = bh; J.n_bh = nbh;
+    int rc = run_job(&J, nthreads);
+    free(bh);
+    return rc;
+}
+
+/* Readout o_t = S_t . u for every (b,t,h) ([B,L,H,n]) and snapshots S_t at
+ * 1-based t = every, 2*every, ... ([B, L/every, H, n, n]); either may be NULL. */
+int mro_readout(const mro_problem* p, const void* x, const double* S0, const double* u,
+                double* o_all, int64_t snap_every, double* snap_all, int nthreads)
+{
+    if (check_problem(p) != MRO_OK || !u) return MRO_ERR_ARG;
+    const int64_t nbh = p->B * p->H;
+    int64_t* bh = malloc(sizeof(int64_t) * (nbh > 0 ? nbh : 1));
+    for (int64_t i = 0; i < nbh; ++i) bh[i] = i;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.p = p; J.x = x; J.S0 = S0; J.u = u; J.o_all = o_all;
+    J.snap_every = snap_every; J.snap_all = snap_all;
+    J.t_end = p->L; J.bh = bh; J.n_bh = nbh;
+    int rc = run_job(&J, nthreads);
+    free(bh);
+    return rc;
+}
+
+/* Streaming comparison for sizes too large to hold in fp64: for each listed
+ * sequence (b*H + h), recompute S_t for t < t_end and accumulate, per
+ * (b,t,h), the squared Frobenius norm of (gpu - oracle) and of the oracle.
+ * Any of the gpu arrays may be NULL; with all of them NULL the call only
+ * runs the product (used to time the oracle). */
+int mro_compare(const mro_problem* p, const void* x, const double* S0,
+                const int64_t* bh, int64_t n_bh, int64_t t_end,
+                const float* S_gpu, double* dS, double* rS,
+                const double* u, const float* o_gpu, double* dO, double* rO,
+                int64_t snap_every, const float* snap_gpu, double* dP, double* rP,
+                int nthreads)
+{
+    if (check_problem(p) != MRO_OK) return MRO_ERR_ARG;
+    if (t_end < 0 || t_end > p->L) return MRO_ERR_ARG;
+    if (S_gpu && (!dS || !rS)) return MRO_ERR_ARG;
+    if (o_gpu && (!u || !dO || !rO)) return MRO_ERR_ARG;
+    if (snap_gpu && (snap_every <= 0 || !dP || !rP)) return MRO_ERR_ARG;
+    for (int64_t i = 0; i < n_bh; ++i)
+        if (bh[i] < 0 || bh[i] >= p->B * p->H) return MRO_ERR_ARG;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.p = p; J.x = x; J.S0 = S0;
+    J.S_gpu = S_gpu; J.dS = dS; J.rS = rS;
+    J.u = u; J.o_gpu = o_gpu; J.dO = dO; J.rO = rO;
+    J.snap_every = snap_gpu ? snap_every : 0; J.snap_gpu = snap_gpu; J.dP = dP; J.rP = rP;
+    J.t_end = t_end; J.bh = bh; J.n_bh = n_bh;
+    return run_job(&J, nthreads);
+}
