@@ -1,0 +1,469 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the MRU prefix-product scan on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = one call of mru_scan_fused over the whole workload (lift + chunk
+prefixes + chunk-total scan + fix-up, every kernel of the path) with the
+embeddings already resident in HBM.  The default workload is the n = 16,
+B8 H8 L4096 determinant-corrected scan (x [8, 4096, 2048] fp32 in, every
+S_t [8, 4096, 8, 16, 16] fp32 out).  Rank 0 prints one JSON line.
+
+Multi-GPU (torchrun, one process per GPU): the (b, h) sequences are
+independent, so every rank scans its own replica of the workload with no
+data-path collective ("scaling": "weak"); NCCL is used only for the barrier
+and the max over ranks of the timed region.
+
+--impl reference times the fp64 CPU oracle on the host cores, on a bounded
+sample of the same workload per step (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_rnn_scan_b200 import inputs as gen  # noqa: E402
+
+METRIC = "MRU scan tokens·heads/s and achieved % of HBM/tensor roofline, 1×B200"
+UNIT = "token·heads/s"
+DEFAULT_WORKLOAD = "n16_detnorm_b8h8l4096"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+# ------------------------------------------------------------ bookkeeping ---
+
+def step_bytes(w: gen.Workload) -> dict:
+    """Algorithmic HBM bytes of one step: embeddings in, results out."""
+    nn = w.n * w.n
+    xb = 2 if w.x_dtype == "bf16" else 4
+    x_bytes = w.token_heads * nn * xb
+    if w.readout:
+        out = w.token_heads * w.n * 4
+        if w.snapshot_every:
+            out += w.B * (w.L // w.snapshot_every) * w.H * nn * 4
+    else:
+        out = w.token_heads * nn * 4
+    return {"in": x_bytes, "out": out, "total": x_bytes + out}
+
+
+KERNELS = ["k_chunk_prefix", "k_carry_local", "k_carry_groups", "k_carry_final", "k_fixup"]
+
+
+def kernel_bytes(name: str, w: gen.Workload, chunk: int) -> int:
+    """Algorithmic bytes one launch of a kernel must move (per launch = the
+    whole workload).  Chunk prefixes: embeddings in, local prefixes Q_t out
+    (where S_t goes); fix-up: Q_t in, S_t out; carry kernels: chunk totals."""
+    nn = w.n * w.n
+    sb = step_bytes(w)
+    K = -(-w.L // chunk)
+    tot = w.B * w.H * K * nn
+    if name == "k_chunk_prefix":
+        return sb["in"] + sb["out"] + tot * 4
+    if name == "k_fixup":
+        return 2 * sb["out"] + tot * 4
+    if name == "k_carry_local":
+        return tot * (4 + 8)
+    if name == "k_carry_groups":
+        G = max(1, math.isqrt(K - 1) + 1) if K > 1 else 1
+        return w.B * w.H * (-(-K // G)) * nn * 16
+    if name == "k_carry_final":
+        return tot * (8 + 8 + 4)
+    return 0
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "linear_rnn_scan_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rows = json.load(f)
+    except Exception:
+        return None
+    cur = csrc_hash()
+    for r in rows:
+        if r.get("workload") == workload and r.get("kernel") == kernel and r.get("csrc_sha256") == cur:
+            return float(r["dram_bytes_per_launch"])
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML during a region."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.stop_ev = threading.Event()
+        self.thread = None
+        self.max_mhz = None
+        self.err = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = device_index
+            if vis:
+                ids = [v.strip() for v in vis.split(",") if v.strip()]
+                if device_index < len(ids) and ids[device_index].isdigit():
+                    idx = int(ids[device_index])
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report the absence
+            self.nv = None
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.time(), sm, rs))
+            except Exception as e:
+                self.err = str(e)
+            self.stop_ev.wait(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self.stop_ev.set()
+        if self.thread:
+            self.thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": self.err or "no samples"}
+        mhz = [s[1] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= int(s[2])
+        reasons = [name for b, name in sorted(self.REASONS.items()) if bits & b and name != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(mhz)), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz), "sm_mhz_min": min(mhz)}
+
+
+# ------------------------------------------------------------- CPU oracle ---
+
+def oracle_rate(w: gen.Workload, x_np, target_s: float, nthreads: int):
+    """Times the fp64 oracle (as it stands) on a bounded sample of the
+    workload: the first t_end tokens of a set of (b, h) sequences."""
+    import oracle
+    p = oracle.make_problem(w.B, w.H, w.L, w.n, x_dtype=w.x_dtype, mode=w.mode, alpha=w.alpha,
+                            add_identity=w.add_identity, ldu_offdiag=w.ldu_offdiag, ldu_diag=w.ldu_diag)
+    nbh = w.B * w.H
+    seqs = min(nbh, max(1, nthreads))
+    bh = np.linspace(0, nbh - 1, seqs).round().astype(np.int64)
+    # calibrate on a short prefix
+    t_cal = min(w.L, 16)
+    t0 = time.perf_counter()
+    oracle.compare(p, x_np, bh=bh, t_end=t_cal, nthreads=nthreads)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    per_token = dt / t_cal
+    t_end = int(min(w.L, max(t_cal, target_s / per_token)))
+    t0 = time.perf_counter()
+    oracle.compare(p, x_np, bh=bh, t_end=t_end, nthreads=nthreads)
+    el = time.perf_counter() - t0
+    units = len(bh) * t_end
+    sample = f"first {t_end} of {w.L} tokens of {len(bh)} of {nbh} (b,h) sequences, fp64, {nthreads} threads"
+    return units / el, units, el, sample
+
+
+def run_reference(args, w):
+    rank = env_int("RANK", 0)
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    nthreads = os.cpu_count() or 1
+    x_np = gen.make_x(w)
+    per_step = float(os.environ.get("MRU_REF_STEP_SECONDS", "3.0"))
+    for _ in range(args.warmup):
+        oracle_rate(w, x_np, 0.2, nthreads)
+    rates, units_all, secs_all, sample = [], 0, 0.0, ""
+    for _ in range(args.steps):
+        r, u, s, sample = oracle_rate(w, x_np, per_step, nthreads)
+        rates.append(r)
+        units_all += u
+        secs_all += s
+    value = units_all / secs_all
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * secs_all / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, None),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                         "sample": f"per step: {sample}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, chunk):
+    sb = step_bytes(w)
+    return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "n": w.n, "x_dtype": w.x_dtype,
+            "mode": ["reshape", "detnorm", "ldu"][w.mode], "readout": w.readout,
+            "snapshot_every": w.snapshot_every, "chunk": chunk,
+            "l2": ("inputs larger than L2: x %.0f MiB in, %.0f MiB out per step" %
+                   (sb["in"] / 2 ** 20, sb["out"] / 2 ** 20)) if sb["total"] > L2_BYTES
+            else "inputs smaller than L2 (no flush)",
+            "parallelism": "single GPU; replicas across GPUs (independent (b,h) sequences)"}
+
+
+# ------------------------------------------------------------------- ours ---
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from linear_rnn_scan_b200 import mru
+
+    rank, world, local = env_int("RANK", 0), env_int("WORLD_SIZE", 1), env_int("LOCAL_RANK", 0)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # CPU baseline first (rank 0, one GPU), before any CUDA work.
+    x_np = gen.make_x(w, seed=w.seed + rank)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        nthreads = os.cpu_count() or 1
+        r, units, el, sample = oracle_rate(w, x_np, args.cpu_seconds, nthreads)
+        cpu = {"value": r, "unit": UNIT, "cores": nthreads, "kind": "oracle", "sample": sample,
+               "seconds": round(el, 2)}
+
+    p = mru.problem_from_workload(w)
+    chunk = mru.chosen_chunk(p)
+    stream = torch.cuda.current_stream()
+    s_handle = stream.cuda_stream
+    if w.x_dtype == "bf16":
+        x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16)
+    else:
+        x_host = torch.from_numpy(x_np)
+    x_pin = x_host.pin_memory()
+    x_dev = x_pin.to(dev)
+    ws = mru.workspace_t(p, dev)
+    if w.readout:
+        u = torch.from_numpy(gen.make_u(w)).to(dev)
+        o = torch.empty((w.B, w.L, w.H, w.n), dtype=torch.float32, device=dev)
+        snaps = (torch.empty((w.B, w.L // w.snapshot_every, w.H, w.n, w.n), dtype=torch.float32, device=dev)
+                 if w.snapshot_every else None)
+        ro = mru.Readout(u.data_ptr(), w.snapshot_every, snaps.data_ptr() if snaps is not None else None)
+        out_main = o
+        outs_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True)]
+        outs_dev = [o]
+        if snaps is not None:
+            outs_host.append(torch.empty(snaps.shape, dtype=snaps.dtype, pin_memory=True))
+            outs_dev.append(snaps)
+
+        def call(xd):
+            return mru.scan_fused(p, xd.data_ptr(), None, ro, None, o.data_ptr(), ws.data_ptr(), ws.numel(),
+                                  s_handle)
+    else:
+        S = torch.empty((w.B, w.L, w.H, w.n, w.n), dtype=torch.float32, device=dev)
+        out_main = S
+        outs_host = [torch.empty(S.shape, dtype=S.dtype, pin_memory=True)]
+        outs_dev = [S]
+
+        def call(xd):
+            return mru.scan_fused(p, xd.data_ptr(), None, None, S.data_ptr(), None, ws.data_ptr(), ws.numel(),
+                                  s_handle)
+
+    launches_per_step = mru.launch_count(p, w.readout)
+
+    def step():
+        rc = call(x_dev)
+        if rc != mru.OK:
+            raise mru.MruError(rc, "mru_scan_fused")
+
+    # warm-up
+    for _ in range(args.warmup):
+        step()
+    st = mru.last_device_status(ws.data_ptr(), s_handle)
+    if st != mru.OK:
+        raise mru.MruError(st, "device status after warm-up")
+
+    # timed region: exactly K steps, device-resident inputs
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        ev1.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms = max_over_ranks(ms)
+    value = world * w.token_heads / (ms / 1e3)
+
+    # per-kernel durations: the same K steps again with the library's event hook
+    n_k = launches_per_step
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_k)] for _ in range(args.steps)]
+    for row in evs:
+        for e in row:
+            e.record(stream)           # creates the handles
+    torch.cuda.synchronize()
+    for row in evs:
+        mru.set_profile_events([e.cuda_event for e in row])
+        step()
+    mru.set_profile_events(None)
+    torch.cuda.synchronize()
+    per_kernel = []
+    for i in range(n_k):
+        per_kernel.append(statistics.mean(row[2 * i].elapsed_time(row[2 * i + 1]) for row in evs))
+    dom = int(np.argmax(per_kernel))
+    dom_name = KERNELS[dom] if dom < len(KERNELS) else f"kernel{dom}"
+    peaks = read_peaks()
+    dom_bytes = kernel_bytes(dom_name, w, chunk)
+    achieved = dom_bytes / (per_kernel[dom] / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "traffic": recorded_traffic(w.name, dom_name),
+                "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_ms": per_kernel[dom],
+                "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] == "measured"
+                else "fallback 6.65 TB/s"}
+    sb = step_bytes(w)
+    path = {"algorithmic_bytes_per_step": sb["total"], "achieved_gbs": sb["total"] / (ms / 1e3) / 1e9}
+    path["frac_of_hbm_peak"] = path["achieved_gbs"] / peaks["hbm_gbs"]
+    kernels_ms = {KERNELS[i] if i < len(KERNELS) else f"kernel{i}": round(per_kernel[i], 5) for i in range(n_k)}
+
+    # e2e: public API with host buffers; H2D of x and D2H of every output inside the region
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    h2d = x_pin.numel() * x_pin.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in outs_host)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_pin, non_blocking=True)
+        rc = call(x_dev)
+        if rc != mru.OK:
+            raise mru.MruError(rc, "mru_scan_fused")
+        for hd, dd in zip(outs_host, outs_dev):
+            hd.copy_(dd, non_blocking=True)
+    e1.record(stream)
+    e1.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+    st = mru.last_device_status(ws.data_ptr(), s_handle)
+    if st != mru.OK:
+        raise mru.MruError(st, "device status after timing")
+
+    if rank == 0:
+        cfg = workload_config(w, chunk)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded N(0,1) embeddings)",
+            "config": cfg, "clocks": clocks.summary(),
+            "e2e": {"value": world * w.token_heads / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "roofline": roofline, "path_roofline": path, "kernels_ms": kernels_ms,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    del out_main
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(gen.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)      # at least 3 untimed warm-up steps, always
+    w = gen.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,140 @@
+/*
+ * mru.h -- C-ABI of libmru.so, the B200 (sm_100a) Matrix Recurrent Unit
+ * prefix-product scan.
+ *
+ * The operation ("MRU Update: An independent developer's alternative to
+ * Attention is now running successfully", section "What MRU Actually Does"):
+ * every token's embedding slice is lifted to an n x n input state matrix X_t,
+ * and the states are the cumulative products along the sequence,
+ *
+ *     S_t = S_{t-1} . X_t,     S_0 = I (or a caller-given S0),
+ *
+ * computed as a parallel scan because matrix multiplication is associative.
+ * Construction modes ("Improving Matrix Recurrent Units as an Attention
+ * Alternative", "Key Points" / "Technical Deep Dive"):
+ *   RESHAPE  Xr = add_identity*I + alpha*M, X = Xr;
+ *   DETNORM  X = Xr / |det Xr|^(1/n)   (determinant-correcting scalar; the
+ *            sign of det Xr is kept; det Xr = 0 or not finite is an error);
+ *   LDU      X = L D U, L = I + ldu_offdiag*strict_lower(M),
+ *            U = I + ldu_offdiag*strict_upper(M),
+ *            D = diag(exp(ldu_diag*tanh(M_ii))).
+ * M is the head's slice x[b, t, h*n*n : (h+1)*n*n] viewed row-major as n x n.
+ *
+ * Layouts (all row-major, contiguous, C order):
+ *   x        [B, L, H*n*n]   float32 or bfloat16 (per x_dtype)      device
+ *   X, F     [B, L, H, n, n] float32                                 device
+ *   S0       [B, H, n, n]    float32, or NULL for the identity       device
+ *   S_out    [B, L, H, n, n] float32; memory position t holds S_{t+1} device
+ *   u        [n]             float32, shared by every (b, h)          device
+ *   o_out    [B, L, H, n]    float32, o_t = S_t . u                   device
+ *   snapshots [B, L/every, H, n, n] float32, S_t at 1-based t = k*every device
+ *
+ * Ownership and execution: the caller owns every buffer (the library never
+ * allocates or frees device memory); calls are asynchronous on `stream`
+ * (a cudaStream_t passed as void*; NULL is the legacy default stream).
+ * Buffers must be 16-byte aligned and x/X must not alias any output.
+ *
+ * Errors: argument problems are returned synchronously and nothing is
+ * launched.  Conditions found on the device (a singular matrix in DETNORM
+ * mode) are recorded in a status word inside the workspace and read with
+ * mru_last_device_status(), which synchronises the stream.  Nothing throws
+ * across this boundary.
+ */
+#ifndef MRU_H_
+#define MRU_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MRU_OK = 0,
+    MRU_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misaligned buffer, bad enum */
+    MRU_ERR_UNSUPPORTED = 2,  /* n not in {4, 8, 16, 32, 64}, or an unsupported combination */
+    MRU_ERR_WORKSPACE = 3,    /* workspace smaller than mru_workspace_size() */
+    MRU_ERR_CUDA = 4,         /* a CUDA launch or copy failed */
+    MRU_ERR_SINGULAR = 5,     /* DETNORM met det = 0 or a non-finite determinant */
+    MRU_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up */
+} mru_status;
+
+typedef enum { MRU_MODE_RESHAPE = 0, MRU_MODE_DETNORM = 1, MRU_MODE_LDU = 2 } mru_mode;
+typedef enum { MRU_F32 = 0, MRU_BF16 = 1 } mru_dtype;
+typedef enum {
+    MRU_MATH_AUTO = 0,    /* library choice per n and dtype */
+    MRU_MATH_FP32 = 1,    /* fp32 FMA throughout */
+    MRU_MATH_TF32 = 2,    /* tensor-core products with tf32 operands, fp32 accumulate */
+    MRU_MATH_TF32X3 = 3,  /* split-tf32 (hi/lo, three products), fp32 accumulate */
+    MRU_MATH_BF16X3 = 4   /* split-bf16 (hi/lo, three products), fp32 accumulate */
+} mru_math;
+
+typedef struct {
+    int64_t B, H, L;            /* batch, heads, sequence length (>= 0) */
+    int32_t n;                  /* matrix side: 4, 8, 16, 32 or 64 */
+    int32_t x_dtype;            /* mru_dtype of x */
+    int32_t mode;               /* mru_mode */
+    int32_t math;               /* mru_math */
+    float alpha;                /* RESHAPE / DETNORM: Xr = add_identity*I + alpha*M */
+    int32_t add_identity;       /* 0 or 1 */
+    float ldu_offdiag;          /* LDU: off-diagonal scale of L and U */
+    float ldu_diag;             /* LDU: D_ii = exp(ldu_diag * tanh(M_ii)) */
+    int32_t store_minus_identity; /* mru_build_states writes F = X - I; mru_scan reads F */
+    int32_t chunk;              /* tokens per scan chunk; 0 = library choice, else >= 1 */
+} mru_problem;
+
+typedef struct {
+    const float* u;             /* [n] readout vector (device) */
+    int64_t snapshot_every;     /* 0: no snapshots; else > 0, floor(L/every) snapshots per (b, h) */
+    float* snapshots;           /* [B, L/every, H, n, n] (device), ignored when every == 0 */
+} mru_readout;
+
+/* Bytes of device workspace a call on this problem needs (>= 256: the first
+ * 256 bytes hold the device status word).  Returns 0 for an invalid problem. */
+size_t mru_workspace_size(const mru_problem* p);
+
+/* Lift only: X_out[b,t,h] = X_t (or F = X_t - I when store_minus_identity).
+ * Construction as listed above.  ws: at least mru_workspace_size(p) bytes. */
+mru_status mru_build_states(const mru_problem* p, const void* x, float* X_out,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Scan only: S_out[b,t,h] = S0[b,h] . X_1 ... X_{t+1} from given matrices X
+ * (or F = X - I when store_minus_identity; the identity-split form keeps the
+ * product accurate for near-identity inputs).  x_dtype/mode are ignored. */
+mru_status mru_scan(const mru_problem* p, const float* X, const float* S0, float* S_out,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* Lift + scan fused: construction from x happens inside the scan.  With
+ * ro == NULL every state is written to S_out (o_out unused, may be NULL).
+ * With ro != NULL the states are reduced instead: o_out[b,t,h] = S_t . u, and
+ * S_t is stored to ro->snapshots at t = every, 2*every, ... (S_out unused). */
+mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0,
+                          const mru_readout* ro, float* S_out, float* o_out,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream` and returns the device-detected status of the last
+ * call that used this workspace (MRU_OK, MRU_ERR_SINGULAR, MRU_ERR_TIMEOUT). */
+mru_status mru_last_device_status(const void* ws, void* stream);
+
+/* Static string for a status code. */
+const char* mru_status_string(mru_status s);
+
+/* Chunk length the library would use for this problem (0 if invalid). */
+int32_t mru_chosen_chunk(const mru_problem* p);
+
+/* Number of kernel launches one call of mru_scan_fused makes for p. */
+int32_t mru_launch_count(const mru_problem* p, int32_t readout);
+
+/* Benchmark hook.  With count > 0, every later mru_scan / mru_scan_fused call
+ * records events[2*i] just before and events[2*i+1] just after its i-th
+ * kernel launch (for i < count/2), on the call's stream, so that the caller
+ * can time each kernel with cudaEventElapsedTime.  The cudaEvent_t handles
+ * are created and owned by the caller; count <= 64.  events == NULL or
+ * count == 0 switches the hook off.  Process-wide; not thread-safe. */
+mru_status mru_set_profile_events(void* const* events, int32_t count);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MRU_H_ */

@@ -1,0 +1,220 @@
+// mru_api.cu -- the extern "C" boundary of libmru: argument checks, workspace
+// layout, kernel selection and launch.  No allocation happens here: every
+// buffer, the workspace included, belongs to the caller.
+#include <string.h>
+
+#include "mru_internal.cuh"
+
+namespace mru {
+namespace {
+
+bool supported_n(int n) { return n == 4 || n == 8 || n == 16 || n == 32 || n == 64; }
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Tokens per chunk: aim at about 4096 chains (b, h, chunk) so that a
+// generic-path launch fills 148 SMs several times over; a power of two in
+// [16, 1024].
+int32_t choose_chunk(const mru_problem& p)
+{
+    if (p.chunk > 0) return p.chunk;
+    const int64_t th = p.B * p.H * p.L;
+    int64_t c = 16;
+    while (c < 1024 && c * 4096 < th) c *= 2;
+    return (int32_t)c;
+}
+
+int32_t choose_group(int64_t K)
+{
+    int64_t g = 1;
+    while (g * g < K) ++g;
+    return (int32_t)(g < 1 ? 1 : g);
+}
+
+mru_status check_problem(const mru_problem* p)
+{
+    if (!p) return MRU_ERR_INVALID_ARG;
+    if (p->B < 0 || p->H < 0 || p->L < 0 || p->chunk < 0) return MRU_ERR_INVALID_ARG;
+    if (p->x_dtype != MRU_F32 && p->x_dtype != MRU_BF16) return MRU_ERR_INVALID_ARG;
+    if (p->mode < MRU_MODE_RESHAPE || p->mode > MRU_MODE_LDU) return MRU_ERR_INVALID_ARG;
+    if (p->math < MRU_MATH_AUTO || p->math > MRU_MATH_BF16X3) return MRU_ERR_INVALID_ARG;
+    if (p->add_identity != 0 && p->add_identity != 1) return MRU_ERR_INVALID_ARG;
+    if (!supported_n(p->n)) return MRU_ERR_UNSUPPORTED;
+    return MRU_OK;
+}
+
+KParams make_params(const mru_problem& p, int32_t src)
+{
+    KParams k;
+    memset(&k, 0, sizeof k);
+    k.B = p.B; k.H = p.H; k.L = p.L; k.n = p.n;
+    k.x_dtype = p.x_dtype; k.mode = p.mode; k.src = src;
+    k.alpha = p.alpha; k.add_identity = p.add_identity;
+    k.ldu_a = p.ldu_offdiag; k.ldu_d = p.ldu_diag;
+    k.chunk = choose_chunk(p);
+    k.K = ceil_div(p.L, k.chunk);
+    k.group = choose_group(k.K);
+    k.NG = k.K > 0 ? ceil_div(k.K, k.group) : 0;
+    return k;
+}
+
+Workspace layout(const KParams& k)
+{
+    Workspace W;
+    const size_t nn = (size_t)k.n * k.n;
+    const size_t BH = (size_t)(k.B * k.H);
+    size_t off = 0;
+    W.status = off; off += 256;
+    W.totals = off; off = round_up(off + BH * k.K * nn * sizeof(float), 256);
+    W.local = off;  off = round_up(off + BH * k.K * nn * sizeof(double), 256);
+    W.gcarry = off; off = round_up(off + BH * k.NG * nn * sizeof(double), 256);
+    W.carry = off;  off = round_up(off + BH * k.K * nn * sizeof(float), 256);
+    W.bytes = off;
+    return W;
+}
+
+cudaEvent_t g_prof_events[64];
+int g_prof_count = 0;
+
+mru_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MRU_OK : MRU_ERR_CUDA; }
+
+mru_status reset_status(void* ws, cudaStream_t s)
+{
+    return from_cuda(cudaMemsetAsync(ws, 0, sizeof(uint32_t), s));
+}
+
+}  // namespace
+
+void profile_mark(int kernel, int after, cudaStream_t s)
+{
+    const int slot = 2 * kernel + after;
+    if (slot < g_prof_count) cudaEventRecord(g_prof_events[slot], s);
+}
+
+}  // namespace mru
+
+using namespace mru;
+
+extern "C" {
+
+size_t mru_workspace_size(const mru_problem* p)
+{
+    if (check_problem(p) != MRU_OK) return 0;
+    return layout(make_params(*p, SRC_EMBEDDING)).bytes;
+}
+
+int32_t mru_chosen_chunk(const mru_problem* p)
+{
+    if (check_problem(p) != MRU_OK) return 0;
+    return choose_chunk(*p);
+}
+
+int32_t mru_launch_count(const mru_problem* p, int32_t readout)
+{
+    (void)readout;
+    if (check_problem(p) != MRU_OK) return 0;
+    if (p->B * p->H * p->L == 0) return 0;
+    return 5;
+}
+
+mru_status mru_build_states(const mru_problem* p, const void* x, float* X_out, void* ws, size_t ws_bytes,
+                            void* stream)
+{
+    mru_status st = check_problem(p);
+    if (st != MRU_OK) return st;
+    if (!x || !X_out || !ws || !aligned16(x) || !aligned16(X_out) || !aligned16(ws)) return MRU_ERR_INVALID_ARG;
+    KParams k = make_params(*p, SRC_EMBEDDING);
+    Workspace W = layout(k);
+    if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = reset_status(ws, s)) != MRU_OK) return st;
+    if (p->B * p->H * p->L == 0) return MRU_OK;
+    return from_cuda(launch_build_states(k, x, X_out, p->store_minus_identity, ws, W, s));
+}
+
+mru_status mru_scan(const mru_problem* p, const float* X, const float* S0, float* S_out, void* ws,
+                    size_t ws_bytes, void* stream)
+{
+    mru_status st = check_problem(p);
+    if (st != MRU_OK) return st;
+    if (!X || !S_out || !ws || !aligned16(X) || !aligned16(S_out) || !aligned16(ws)) return MRU_ERR_INVALID_ARG;
+    if (S0 && !aligned16(S0)) return MRU_ERR_INVALID_ARG;
+    if ((const void*)X == (const void*)S_out) return MRU_ERR_INVALID_ARG;
+    KParams k = make_params(*p, p->store_minus_identity ? SRC_F : SRC_X);
+    Workspace W = layout(k);
+    if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = reset_status(ws, s)) != MRU_OK) return st;
+    if (p->B * p->H * p->L == 0) return MRU_OK;
+    return from_cuda(launch_scan(k, X, S0, nullptr, 0, S_out, nullptr, nullptr, ws, W, s, nullptr));
+}
+
+mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0, const mru_readout* ro,
+                          float* S_out, float* o_out, void* ws, size_t ws_bytes, void* stream)
+{
+    mru_status st = check_problem(p);
+    if (st != MRU_OK) return st;
+    if (!x || !ws || !aligned16(x) || !aligned16(ws)) return MRU_ERR_INVALID_ARG;
+    if (S0 && !aligned16(S0)) return MRU_ERR_INVALID_ARG;
+    int64_t every = 0;
+    float* snaps = nullptr;
+    if (ro) {
+        if (!ro->u || !o_out || !aligned16(o_out) || ro->snapshot_every < 0) return MRU_ERR_INVALID_ARG;
+        every = ro->snapshot_every;
+        if (every > 0) {
+            snaps = ro->snapshots;
+            if (!snaps || !aligned16(snaps)) return MRU_ERR_INVALID_ARG;
+        }
+        if ((const void*)o_out == x) return MRU_ERR_INVALID_ARG;
+    } else {
+        if (!S_out || !aligned16(S_out) || (const void*)S_out == x) return MRU_ERR_INVALID_ARG;
+    }
+    KParams k = make_params(*p, SRC_EMBEDDING);
+    Workspace W = layout(k);
+    if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = reset_status(ws, s)) != MRU_OK) return st;
+    if (p->B * p->H * p->L == 0) return MRU_OK;
+    return from_cuda(launch_scan(k, x, S0, ro ? ro->u : nullptr, every, ro ? nullptr : S_out,
+                                 ro ? o_out : nullptr, snaps, ws, W, s, nullptr));
+}
+
+mru_status mru_last_device_status(const void* ws, void* stream)
+{
+    if (!ws) return MRU_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MRU_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, ws, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess) return MRU_ERR_CUDA;
+    if (word & STATUS_TIMEOUT) return MRU_ERR_TIMEOUT;
+    if (word & STATUS_SINGULAR) return MRU_ERR_SINGULAR;
+    return MRU_OK;
+}
+
+mru_status mru_set_profile_events(void* const* events, int32_t count)
+{
+    if (count < 0 || count > 64 || (count > 0 && !events)) return MRU_ERR_INVALID_ARG;
+    for (int i = 0; i < count; ++i)
+        if (!events[i]) return MRU_ERR_INVALID_ARG;
+    for (int i = 0; i < count; ++i) g_prof_events[i] = reinterpret_cast<cudaEvent_t>(events[i]);
+    g_prof_count = count;
+    return MRU_OK;
+}
+
+const char* mru_status_string(mru_status s)
+{
+    switch (s) {
+        case MRU_OK: return "ok";
+        case MRU_ERR_INVALID_ARG: return "invalid argument";
+        case MRU_ERR_UNSUPPORTED: return "unsupported problem (n must be 4, 8, 16, 32 or 64)";
+        case MRU_ERR_WORKSPACE: return "workspace too small";
+        case MRU_ERR_CUDA: return "CUDA error";
+        case MRU_ERR_SINGULAR: return "singular input matrix (det = 0 or not finite)";
+        case MRU_ERR_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

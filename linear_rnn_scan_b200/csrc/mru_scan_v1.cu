@@ -1,0 +1,606 @@
+// mru_scan_v1.cu -- generic (every supported n) chunked prefix-product scan.
+//
+// The scan follows the method's associativity argument ("MRU Update: An
+// independent developer's alternative to Attention is now running
+// successfully", section "What MRU Actually Does"): the sequence of each
+// (b, h) is cut into chunks of C tokens; every chunk forms its local prefix
+// products independently, the chunk totals are scanned, and every local
+// prefix is then multiplied on the left by its chunk's carry.
+//
+// Numerics.  Every matrix is carried in identity-split form, X = I + F,
+// P = I + Q, so that the near-identity inputs of the determinant-corrected
+// workloads lose nothing to the implicit 1 on the diagonal:
+//     Q_t = Q_{t-1} + F_t + Q_{t-1} F_t            (in-chunk, fp32)
+//     carry_{k+1} = carry_k + carry_k Q_k          (chunk totals, fp64)
+//     S_t = carry + carry Q_t                      (fix-up, fp32)
+// The chunk-total scan is two-level (groups of G totals, then the group
+// totals) so that no serial chain is longer than max(G, K/G).
+//
+// Kernels (one call of mru_scan_fused):
+//   k_chunk_prefix  one CTA per (b, h, chunk): lift + in-chunk prefix; writes
+//                   Q_t where S_t (or o_t = S_t u, snapshots) will go, and
+//                   the chunk total to the workspace
+//   k_carry_local   one CTA per (b, h, group): in-group inclusive prefixes
+//   k_carry_groups  one CTA per (b, h): exclusive group carries (serial)
+//   k_carry_final   one CTA per (b, h, chunk): exclusive chunk carries
+//   k_fixup         one CTA per (b, h, chunk): S_t = carry (I + Q_t) in place
+#include "mru_internal.cuh"
+
+namespace mru {
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float load_elem(const void* base, int64_t idx, int dtype)
+{
+    if (dtype == MRU_BF16)
+        return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[idx]);
+    return reinterpret_cast<const float*>(base)[idx];
+}
+
+// Trailing-submatrix update of one elimination step on an N x N matrix in
+// shared memory: W[i][j] -= W[i][k] * r * W[k][j] for i, j > k.
+template <int N>
+__device__ __forceinline__ void eliminate_step(float* sW, int k, float r)
+{
+    const int m = N - k - 1;
+    for (int idx = threadIdx.x; idx < m * m; idx += kThreads) {
+        const int i = k + 1 + idx / m, j = k + 1 + idx % m;
+        sW[i * N + j] = fmaf(-sW[i * N + k] * r, sW[k * N + j], sW[i * N + j]);
+    }
+}
+
+// Per-token scalars in shared memory, after the 4N floats of per-row
+// scratch: [4N] pivot row (int), [4N+1] flag, [4N+2..4N+3] log|det| (fp64),
+// [4N+4] c, [4N+5] c - 1.  (The scratch area holds 4N + 8 floats.)
+template <int N> __device__ __forceinline__ int* aux_piv(float* a) { return reinterpret_cast<int*>(a + 4 * N); }
+template <int N> __device__ __forceinline__ float* aux_flag(float* a) { return a + 4 * N + 1; }
+template <int N> __device__ __forceinline__ double* aux_logdet(float* a) { return reinterpret_cast<double*>(a + 4 * N + 2); }
+template <int N> __device__ __forceinline__ float* aux_c(float* a) { return a + 4 * N + 4; }
+
+// log|det W| by LU with partial pivoting on the full matrix in sW (destroyed),
+// accumulated in fp64 into the logdet slot; the flag slot is set when a pivot
+// column is entirely zero.  Called by the whole CTA.
+template <int N>
+__device__ void cta_logabsdet_pivoted(float* sW, float* sAux)
+{
+    int* sPiv = aux_piv<N>(sAux);
+    if (threadIdx.x == 0) { *aux_logdet<N>(sAux) = 0.0; *aux_flag<N>(sAux) = 0.0f; }
+    __syncthreads();
+    for (int k = 0; k < N; ++k) {
+        if (threadIdx.x < 32) {
+            float best = -1.0f;
+            int bi = k;
+            for (int i = k + threadIdx.x; i < N; i += 32) {
+                const float a = fabsf(sW[i * N + k]);
+                if (a > best) { best = a; bi = i; }
+            }
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ob = __shfl_down_sync(0xffffffffu, best, o);
+                const int oi = __shfl_down_sync(0xffffffffu, bi, o);
+                if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+            }
+            if (threadIdx.x == 0) {
+                *sPiv = bi;
+                if (!(best > 0.0f)) *aux_flag<N>(sAux) = 1.0f;
+            }
+        }
+        __syncthreads();
+        const int piv = *sPiv;
+        if (piv != k) {
+            for (int j = threadIdx.x; j < N; j += kThreads) {
+                const float a = sW[k * N + j];
+                sW[k * N + j] = sW[piv * N + j];
+                sW[piv * N + j] = a;
+            }
+        }
+        __syncthreads();
+        const float pk = sW[k * N + k];
+        if (threadIdx.x == 0) *aux_logdet<N>(sAux) += log(fabs((double)pk));
+        const float r = (pk != 0.0f) ? 1.0f / pk : 0.0f;
+        eliminate_step<N>(sW, k, r);
+        __syncthreads();
+    }
+}
+
+// Lift one token-head slice into F = X - I (shared memory, sF).  The whole
+// CTA calls it; it ends with a barrier.  sM, sW: N*N floats of scratch;
+// sAux: 4N + 8 floats of scratch.
+//
+// The per-token scalars that every later step multiplies into the product
+// (the determinant scale c and c - 1, the LDU diagonal D_i - 1) are formed in
+// fp64 and rounded once: a bias of one fp32 ulp in them would otherwise add
+// up coherently over thousands of tokens.
+template <int N>
+__device__ void cta_construct(const KParams& p, const void* src, int64_t off, float* sF,
+                              float* sM, float* sW, float* sAux, uint32_t* status)
+{
+    constexpr int NN = N * N;
+    const int tid = threadIdx.x;
+    if (p.src != SRC_EMBEDDING) {
+        const float* f = reinterpret_cast<const float*>(src) + off;
+        for (int e = tid; e < NN; e += kThreads) {
+            float v = f[e];
+            if (p.src == SRC_X && (e / N) == (e % N)) v -= 1.0f;
+            sF[e] = v;
+        }
+        __syncthreads();
+        return;
+    }
+    for (int e = tid; e < NN; e += kThreads) sM[e] = load_elem(src, off + e, p.x_dtype);
+    __syncthreads();
+
+    if (p.mode == MRU_MODE_RESHAPE) {
+        for (int e = tid; e < NN; e += kThreads) {
+            float v = p.alpha * sM[e];
+            if (!p.add_identity && (e / N) == (e % N)) v -= 1.0f;
+            sF[e] = v;
+        }
+        __syncthreads();
+        return;
+    }
+
+    if (p.mode == MRU_MODE_LDU) {
+        // D_k and D_k - 1 (the latter without cancellation), fp64 then rounded.
+        for (int k = tid; k < N; k += kThreads) {
+            const double z = (double)p.ldu_d * tanh((double)sM[k * N + k]);
+            sAux[k] = (float)exp(z);
+            sAux[N + k] = (float)expm1(z);
+        }
+        __syncthreads();
+        const float a = p.ldu_a;
+        // X_ij = sum_{k <= min(i,j)} L_ik D_k U_kj with unit diagonals.
+        for (int e = tid; e < NN; e += kThreads) {
+            const int i = e / N, j = e % N;
+            const int m = i < j ? i : j;
+            float acc = 0.0f;
+            for (int k = 0; k < m; ++k)
+                acc = fmaf(a * sM[i * N + k] * sAux[k], a * sM[k * N + j], acc);
+            if (i < j) acc = fmaf(sAux[i], a * sM[i * N + j], acc);
+            else if (i > j) acc = fmaf(a * sM[i * N + j], sAux[j], acc);
+            else acc += sAux[N + i];
+            sF[e] = acc;
+        }
+        __syncthreads();
+        return;
+    }
+
+    // DETNORM: X = Xr * c, c = |det Xr|^(-1/N).
+    bool need_pivot = !p.add_identity;
+    if (p.add_identity) {
+        // Near-identity fast path: eliminate W = I + E keeping only E, so the
+        // pivots 1 + delta_k are known through delta_k to full precision;
+        // |det| = prod |1 + delta_k| is formed in fp64.  Falls back to
+        // pivoting when a pivot is small.
+        for (int e = tid; e < NN; e += kThreads) sW[e] = p.alpha * sM[e];
+        __syncthreads();
+        for (int k = 0; k < N; ++k) {
+            const float r = 1.0f / (1.0f + sW[k * N + k]);
+            eliminate_step<N>(sW, k, r);
+            __syncthreads();
+        }
+        if (tid == 0) {
+            double prod = 1.0;
+            float bad = 0.0f;
+            for (int k = 0; k < N; ++k) {
+                const float d = sW[k * N + k];
+                if (!(fabsf(1.0f + d) >= 0.5f)) bad = 1.0f;
+                prod *= 1.0 + (double)d;
+            }
+            *aux_logdet<N>(sAux) = log(fabs(prod));
+            *aux_flag<N>(sAux) = bad;
+        }
+        __syncthreads();
+        need_pivot = *aux_flag<N>(sAux) != 0.0f;
+        __syncthreads();
+    }
+    if (need_pivot) {
+        for (int e = tid; e < NN; e += kThreads) {
+            float v = p.alpha * sM[e];
+            if (p.add_identity && (e / N) == (e % N)) v += 1.0f;
+            sW[e] = v;
+        }
+        __syncthreads();
+        cta_logabsdet_pivoted<N>(sW, sAux);
+    }
+    if (tid == 0) {
+        const double ld = *aux_logdet<N>(sAux);
+        const bool singular = need_pivot && *aux_flag<N>(sAux) != 0.0f;
+        const double cm1 = expm1(-ld / N);
+        float c = (float)(1.0 + cm1);
+        float cm1f = (float)cm1;
+        if (singular || !isfinite(ld) || !isfinite(c) || c == 0.0f) {
+            atomicOr(status, STATUS_SINGULAR);
+            c = 0.0f;        // output unspecified; keep it finite (X = I)
+            cm1f = 0.0f;
+        }
+        aux_c<N>(sAux)[0] = c;
+        aux_c<N>(sAux)[1] = cm1f;
+    }
+    __syncthreads();
+    const float c = aux_c<N>(sAux)[0];
+    const float cm1 = aux_c<N>(sAux)[1];
+    for (int e = tid; e < NN; e += kThreads) {
+        const bool diag = (e / N) == (e % N);
+        float v = c * (p.alpha * sM[e]);
+        if (diag) v += p.add_identity ? cm1 : -1.0f;
+        if (c == 0.0f) v = 0.0f;
+        sF[e] = v;
+    }
+    __syncthreads();
+}
+
+// ----------------------------------------------------------------------------
+template <int N>
+__global__ void __launch_bounds__(kThreads)
+k_build_states(KParams p, const void* src, float* X_out, int store_minus_identity, uint32_t* status)
+{
+    constexpr int NN = N * N;
+    extern __shared__ float smem[];
+    float* sF = smem;
+    float* sM = sF + NN;
+    float* sW = sM + NN;
+    float* sAux = sW + NN;
+    const int64_t rows = p.B * p.L * p.H;
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+        cta_construct<N>(p, src, row * NN, sF, sM, sW, sAux, status);
+        for (int e = threadIdx.x; e < NN; e += kThreads) {
+            float v = sF[e];
+            if (!store_minus_identity && (e / N) == (e % N)) v += 1.0f;
+            X_out[row * NN + e] = v;
+        }
+        __syncthreads();
+    }
+}
+
+template <int N>
+__global__ void __launch_bounds__(kThreads)
+k_chunk_prefix(KParams p, const void* src, const float* u, int64_t snap_every, float* S_out,
+               float* o_out, float* snaps, float* totals, uint32_t* status)
+{
+    constexpr int NN = N * N;
+    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    extern __shared__ float smem[];
+    float* sQ = smem;
+    float* sF = sQ + NN;
+    float* sM = sF + NN;
+    float* sW = sM + NN;
+    float* sAux = sW + NN;
+    float* sU = sAux + 4 * N + 8;
+    const int tid = threadIdx.x;
+    const int64_t chain = blockIdx.x;
+    const int64_t k = chain % p.K;
+    const int64_t bh = chain / p.K;
+    const int64_t h = bh % p.H, b = bh / p.H;
+    const int64_t t0 = k * p.chunk;
+    const int64_t t1 = (t0 + p.chunk < p.L) ? t0 + p.chunk : p.L;
+    const bool readout = o_out != nullptr;
+
+    for (int e = tid; e < NN; e += kThreads) sQ[e] = 0.0f;
+    if (readout)
+        for (int i = tid; i < N; i += kThreads) sU[i] = u[i];
+    __syncthreads();
+
+    for (int64_t t = t0; t < t1; ++t) {
+        const int64_t row = (b * p.L + t) * p.H + h;
+        cta_construct<N>(p, src, row * NN, sF, sM, sW, sAux, status);
+        float acc[PER];
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            if (e < NN) {
+                const int i = e / N, j = e % N;
+                float a = sQ[e] + sF[e];
+#pragma unroll 8
+                for (int q = 0; q < N; ++q) a = fmaf(sQ[i * N + q], sF[q * N + j], a);
+                acc[r] = a;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            if (e < NN) {
+                sQ[e] = acc[r];
+                if (!readout) S_out[row * NN + e] = acc[r];
+            }
+        }
+        __syncthreads();
+        if (readout) {
+            for (int i = tid; i < N; i += kThreads) {
+                float v = 0.0f;
+                for (int j = 0; j < N; ++j) v = fmaf(sQ[i * N + j], sU[j], v);
+                o_out[row * N + i] = v;                    // Q_t u, fixed up later
+            }
+            if (snap_every > 0 && ((t + 1) % snap_every) == 0) {
+                const int64_t srow = (b * (p.L / snap_every) + (t + 1) / snap_every - 1) * p.H + h;
+                for (int e = tid; e < NN; e += kThreads) snaps[srow * NN + e] = sQ[e];
+            }
+        }
+    }
+    for (int e = tid; e < NN; e += kThreads) totals[chain * NN + e] = sQ[e];
+}
+
+// In-group inclusive prefixes of the chunk totals, fp64, split form:
+// R_j = R_{j-1} + T_j + R_{j-1} T_j.
+template <int N>
+__global__ void __launch_bounds__(kThreads)
+k_carry_local(KParams p, const float* totals, double* local)
+{
+    constexpr int NN = N * N;
+    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    extern __shared__ double dsm[];
+    double* sR = dsm;
+    double* sT = sR + NN;
+    const int tid = threadIdx.x;
+    const int64_t bh = blockIdx.x / p.NG, g = blockIdx.x % p.NG;
+    const int64_t j0 = g * p.group;
+    const int64_t j1 = (j0 + p.group < p.K) ? j0 + p.group : p.K;
+    for (int e = tid; e < NN; e += kThreads) sR[e] = 0.0;
+    for (int64_t j = j0; j < j1; ++j) {
+        const int64_t base = (bh * p.K + j) * NN;
+        for (int e = tid; e < NN; e += kThreads) sT[e] = (double)totals[base + e];
+        __syncthreads();
+        double acc[PER];
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            if (e < NN) {
+                const int i = e / N, c = e % N;
+                double a = sR[e] + sT[e];
+                for (int q = 0; q < N; ++q) a = fma(sR[i * N + q], sT[q * N + c], a);
+                acc[r] = a;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            if (e < NN) { sR[e] = acc[r]; local[base + e] = acc[r]; }
+        }
+    }
+}
+
+// Exclusive group carries (full matrices, fp64): GC_0 = S0 (or I),
+// GC_{g+1} = GC_g + GC_g R_{g,last}.  Serial over the groups of a sequence.
+template <int N>
+__global__ void __launch_bounds__(kThreads)
+k_carry_groups(KParams p, const float* S0, const double* local, double* gcarry)
+{
+    constexpr int NN = N * N;
+    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    extern __shared__ double dsm[];
+    double* sG = dsm;
+    double* sT = sG + NN;
+    const int tid = threadIdx.x;
+    const int64_t bh = blockIdx.x;
+    for (int e = tid; e < NN; e += kThreads)
+        sG[e] = S0 ? (double)S0[bh * NN + e] : ((e / N) == (e % N) ? 1.0 : 0.0);
+    for (int64_t g = 0; g < p.NG; ++g) {
+        const int64_t last = ((g + 1) * p.group < p.K ? (g + 1) * p.group : p.K) - 1;
+        __syncthreads();
+        for (int e = tid; e < NN; e += kThreads) {
+            gcarry[(bh * p.NG + g) * NN + e] = sG[e];
+            sT[e] = local[(bh * p.K + last) * NN + e];
+        }
+        __syncthreads();
+        double acc[PER];
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            if (e < NN) {
+                const int i = e / N, c = e % N;
+                double a = sG[e];
+                for (int q = 0; q < N; ++q) a = fma(sG[i * N + q], sT[q * N + c], a);
+                acc[r] = a;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            if (e < NN) sG[e] = acc[r];
+        }
+    }
+}
+
+// Exclusive chunk carries: carry_k = GC_g (I + R_{g,k-1}), rounded to fp32.
+template <int N>
+__global__ void __launch_bounds__(kThreads)
+k_carry_final(KParams p, const double* local, const double* gcarry, float* carry)
+{
+    constexpr int NN = N * N;
+    extern __shared__ double dsm[];
+    double* sG = dsm;
+    double* sT = sG + NN;
+    const int tid = threadIdx.x;
+    const int64_t bh = blockIdx.x / p.K, k = blockIdx.x % p.K;
+    const int64_t g = k / p.group;
+    const bool first = (k == g * p.group);
+    for (int e = tid; e < NN; e += kThreads) {
+        sG[e] = gcarry[(bh * p.NG + g) * NN + e];
+        sT[e] = first ? 0.0 : local[(bh * p.K + k - 1) * NN + e];
+    }
+    __syncthreads();
+    for (int e = tid; e < NN; e += kThreads) {
+        const int i = e / N, c = e % N;
+        double a = sG[e];
+        if (!first)
+            for (int q = 0; q < N; ++q) a = fma(sG[i * N + q], sT[q * N + c], a);
+        carry[(bh * p.K + k) * NN + e] = (float)a;
+    }
+}
+
+// S_t = carry (I + Q_t) = carry + carry Q_t, in place; readout: o_t = carry (u + Q_t u).
+template <int N>
+__global__ void __launch_bounds__(kThreads)
+k_fixup(KParams p, const float* carry, const float* u, int64_t snap_every, float* S_out,
+        float* o_out, float* snaps)
+{
+    constexpr int NN = N * N;
+    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    extern __shared__ float smem[];
+    float* sC = smem;
+    float* sQ = sC + NN;
+    float* sCu = sQ + NN;
+    float* sV = sCu + N;
+    const int tid = threadIdx.x;
+    const int64_t chain = blockIdx.x;
+    const int64_t k = chain % p.K;
+    const int64_t bh = chain / p.K;
+    const int64_t h = bh % p.H, b = bh / p.H;
+    const int64_t t0 = k * p.chunk;
+    const int64_t t1 = (t0 + p.chunk < p.L) ? t0 + p.chunk : p.L;
+    for (int e = tid; e < NN; e += kThreads) sC[e] = carry[chain * NN + e];
+    __syncthreads();
+
+    auto fix_matrix = [&](float* g) {       // g[e] <- (C + C Q)[e], Q = g
+        for (int e = tid; e < NN; e += kThreads) sQ[e] = g[e];
+        __syncthreads();
+        float acc[PER];
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            if (e < NN) {
+                const int i = e / N, j = e % N;
+                float a = sC[e];
+#pragma unroll 8
+                for (int q = 0; q < N; ++q) a = fmaf(sC[i * N + q], sQ[q * N + j], a);
+                acc[r] = a;
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            if (e < NN) g[e] = acc[r];
+        }
+        __syncthreads();
+    };
+
+    if (o_out == nullptr) {
+        for (int64_t t = t0; t < t1; ++t) fix_matrix(S_out + ((b * p.L + t) * p.H + h) * NN);
+        return;
+    }
+    for (int i = tid; i < N; i += kThreads) {
+        float a = 0.0f;
+        for (int j = 0; j < N; ++j) a = fmaf(sC[i * N + j], u[j], a);
+        sCu[i] = a;
+    }
+    __syncthreads();
+    for (int64_t t = t0; t < t1; ++t) {
+        float* o = o_out + ((b * p.L + t) * p.H + h) * N;
+        for (int j = tid; j < N; j += kThreads) sV[j] = o[j];
+        __syncthreads();
+        for (int i = tid; i < N; i += kThreads) {
+            float a = sCu[i];
+            for (int j = 0; j < N; ++j) a = fmaf(sC[i * N + j], sV[j], a);
+            o[i] = a;
+        }
+        __syncthreads();
+    }
+    if (snap_every > 0) {
+        const int64_t first = ((t0 + snap_every) / snap_every) * snap_every;   // 1-based
+        for (int64_t t1b = first; t1b <= t1; t1b += snap_every) {
+            const int64_t srow = (b * (p.L / snap_every) + t1b / snap_every - 1) * p.H + h;
+            fix_matrix(snaps + srow * NN);
+        }
+    }
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes)
+{
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int N>
+cudaError_t build_states_n(const KParams& p, const void* x, float* X_out, int smi, uint32_t* status,
+                           cudaStream_t s)
+{
+    constexpr int NN = N * N;
+    const size_t sm = sizeof(float) * (3 * NN + 4 * N + 8);
+    cudaError_t e = set_smem(k_build_states<N>, sm);
+    if (e != cudaSuccess) return e;
+    const int64_t rows = p.B * p.L * p.H;
+    const int64_t grid = rows < 148 * 64 ? rows : 148 * 64;
+    if (grid > 0) k_build_states<N><<<(unsigned)grid, kThreads, sm, s>>>(p, x, X_out, smi, status);
+    return cudaGetLastError();
+}
+
+template <int N>
+cudaError_t scan_n(const KParams& p, const void* src, const float* S0, const float* u, int64_t snap_every,
+                   float* S_out, float* o_out, float* snaps, char* ws, const Workspace& W, cudaStream_t s,
+                   int* launches)
+{
+    constexpr int NN = N * N;
+    uint32_t* status = reinterpret_cast<uint32_t*>(ws + W.status);
+    float* totals = reinterpret_cast<float*>(ws + W.totals);
+    double* local = reinterpret_cast<double*>(ws + W.local);
+    double* gcarry = reinterpret_cast<double*>(ws + W.gcarry);
+    float* carry = reinterpret_cast<float*>(ws + W.carry);
+    const int64_t BH = p.B * p.H;
+    const int64_t chains = BH * p.K;
+    if (chains == 0) return cudaSuccess;
+    cudaError_t e;
+
+    const size_t sm_chunk = sizeof(float) * (4 * NN + 5 * N + 8);
+    const size_t sm_d = sizeof(double) * 2 * NN;
+    const size_t sm_fix = sizeof(float) * (2 * NN + 2 * N);
+    if ((e = set_smem(k_chunk_prefix<N>, sm_chunk)) != cudaSuccess) return e;
+    if ((e = set_smem(k_carry_local<N>, sm_d)) != cudaSuccess) return e;
+    if ((e = set_smem(k_carry_groups<N>, sm_d)) != cudaSuccess) return e;
+    if ((e = set_smem(k_carry_final<N>, sm_d)) != cudaSuccess) return e;
+    if ((e = set_smem(k_fixup<N>, sm_fix)) != cudaSuccess) return e;
+    profile_mark(0, 0, s);
+    k_chunk_prefix<N><<<(unsigned)chains, kThreads, sm_chunk, s>>>(p, src, u, snap_every, S_out, o_out,
+                                                                    snaps, totals, status);
+    profile_mark(0, 1, s);
+    profile_mark(1, 0, s);
+    k_carry_local<N><<<(unsigned)(BH * p.NG), kThreads, sm_d, s>>>(p, totals, local);
+    profile_mark(1, 1, s);
+    profile_mark(2, 0, s);
+    k_carry_groups<N><<<(unsigned)BH, kThreads, sm_d, s>>>(p, S0, local, gcarry);
+    profile_mark(2, 1, s);
+    profile_mark(3, 0, s);
+    k_carry_final<N><<<(unsigned)chains, kThreads, sm_d, s>>>(p, local, gcarry, carry);
+    profile_mark(3, 1, s);
+    profile_mark(4, 0, s);
+    k_fixup<N><<<(unsigned)chains, kThreads, sm_fix, s>>>(p, carry, u, snap_every, S_out, o_out, snaps);
+    profile_mark(4, 1, s);
+    if (launches) *launches = 5;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_build_states(const KParams& p, const void* x, float* X_out, int store_minus_identity,
+                                void* ws_base, const Workspace& W, cudaStream_t s)
+{
+    uint32_t* status = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws_base) + W.status);
+    switch (p.n) {
+        case 4: return build_states_n<4>(p, x, X_out, store_minus_identity, status, s);
+        case 8: return build_states_n<8>(p, x, X_out, store_minus_identity, status, s);
+        case 16: return build_states_n<16>(p, x, X_out, store_minus_identity, status, s);
+        case 32: return build_states_n<32>(p, x, X_out, store_minus_identity, status, s);
+        case 64: return build_states_n<64>(p, x, X_out, store_minus_identity, status, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_scan(const KParams& p, const void* src, const float* S0, const float* u,
+                        int64_t snap_every, float* S_out, float* o_out, float* snaps,
+                        void* ws_base, const Workspace& W, cudaStream_t s, int* launches)
+{
+    char* ws = reinterpret_cast<char*>(ws_base);
+    switch (p.n) {
+        case 4: return scan_n<4>(p, src, S0, u, snap_every, S_out, o_out, snaps, ws, W, s, launches);
+        case 8: return scan_n<8>(p, src, S0, u, snap_every, S_out, o_out, snaps, ws, W, s, launches);
+        case 16: return scan_n<16>(p, src, S0, u, snap_every, S_out, o_out, snaps, ws, W, s, launches);
+        case 32: return scan_n<32>(p, src, S0, u, snap_every, S_out, o_out, snaps, ws, W, s, launches);
+        case 64: return scan_n<64>(p, src, S0, u, snap_every, S_out, o_out, snaps, ws, W, s, launches);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace mru

@@ -1,0 +1,240 @@
+"""ctypes binding of libmru.so (declared in include/mru.h).
+
+Argument marshalling only: every step of the scan runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  There is no
+CPU fallback: if libmru.so has not been built, the first call raises.
+
+Low level (same names as the C-ABI; pointers are ints, streams are ints):
+    workspace_size, build_states, scan, scan_fused, last_device_status,
+    status_string, chosen_chunk, launch_count
+Tensor level:
+    problem(...)                 -> Problem
+    scan_fused_t(p, x, ...)      -> S [B, L, H, n, n]  or  (o, snapshots)
+    scan_t(p, X, ...)            -> S
+    build_states_t(p, x, ...)    -> X (or F)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmru.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_SINGULAR, ERR_TIMEOUT = range(7)
+MODE_RESHAPE, MODE_DETNORM, MODE_LDU = 0, 1, 2
+F32, BF16 = 0, 1
+MATH = {"auto": 0, "fp32": 1, "tf32": 2, "tf32x3": 3, "bf16x3": 4}
+
+# Every symbol include/mru.h declares.
+EXPORTS = ["mru_workspace_size", "mru_build_states", "mru_scan", "mru_scan_fused",
+           "mru_last_device_status", "mru_status_string", "mru_chosen_chunk", "mru_launch_count",
+           "mru_set_profile_events"]
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int64), ("H", ctypes.c_int64), ("L", ctypes.c_int64),
+        ("n", ctypes.c_int32), ("x_dtype", ctypes.c_int32), ("mode", ctypes.c_int32),
+        ("math", ctypes.c_int32), ("alpha", ctypes.c_float), ("add_identity", ctypes.c_int32),
+        ("ldu_offdiag", ctypes.c_float), ("ldu_diag", ctypes.c_float),
+        ("store_minus_identity", ctypes.c_int32), ("chunk", ctypes.c_int32),
+    ]
+
+
+class Readout(ctypes.Structure):
+    _fields_ = [("u", ctypes.c_void_p), ("snapshot_every", ctypes.c_int64), ("snapshots", ctypes.c_void_p)]
+
+
+class MruError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libmru.so (once).  Raises when it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise ImportError(f"{path} is missing: build it with `python -m linear_rnn_scan_b200.build`")
+            lib = ctypes.CDLL(path)
+            P = ctypes.POINTER(Problem)
+            vp, sz = ctypes.c_void_p, ctypes.c_size_t
+            lib.mru_workspace_size.argtypes = [P]
+            lib.mru_workspace_size.restype = sz
+            lib.mru_build_states.argtypes = [P, vp, vp, vp, sz, vp]
+            lib.mru_build_states.restype = ctypes.c_int
+            lib.mru_scan.argtypes = [P, vp, vp, vp, vp, sz, vp]
+            lib.mru_scan.restype = ctypes.c_int
+            lib.mru_scan_fused.argtypes = [P, vp, vp, ctypes.POINTER(Readout), vp, vp, vp, sz, vp]
+            lib.mru_scan_fused.restype = ctypes.c_int
+            lib.mru_last_device_status.argtypes = [vp, vp]
+            lib.mru_last_device_status.restype = ctypes.c_int
+            lib.mru_status_string.argtypes = [ctypes.c_int]
+            lib.mru_status_string.restype = ctypes.c_char_p
+            lib.mru_chosen_chunk.argtypes = [P]
+            lib.mru_chosen_chunk.restype = ctypes.c_int32
+            lib.mru_launch_count.argtypes = [P, ctypes.c_int32]
+            lib.mru_launch_count.restype = ctypes.c_int32
+            lib.mru_set_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
+            lib.mru_set_profile_events.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def problem(B, H, L, n, *, x_dtype="f32", mode=MODE_RESHAPE, math="auto", alpha=1.0, add_identity=1,
+            ldu_offdiag=0.02, ldu_diag=0.1, store_minus_identity=0, chunk=0) -> Problem:
+    dt = {"f32": F32, "bf16": BF16}[x_dtype] if isinstance(x_dtype, str) else int(x_dtype)
+    mt = MATH[math] if isinstance(math, str) else int(math)
+    return Problem(int(B), int(H), int(L), int(n), dt, int(mode), mt, float(alpha), int(add_identity),
+                   float(ldu_offdiag), float(ldu_diag), int(store_minus_identity), int(chunk))
+
+
+def problem_from_workload(w, **over) -> Problem:
+    kw = dict(x_dtype=w.x_dtype, mode=w.mode, math=w.math, alpha=w.alpha, add_identity=w.add_identity,
+              ldu_offdiag=w.ldu_offdiag, ldu_diag=w.ldu_diag)
+    kw.update(over)
+    return problem(w.B, w.H, w.L, w.n, **kw)
+
+
+# ---------------------------------------------------------------- C-ABI ---
+
+def workspace_size(p: Problem) -> int:
+    return int(load().mru_workspace_size(ctypes.byref(p)))
+
+
+def chosen_chunk(p: Problem) -> int:
+    return int(load().mru_chosen_chunk(ctypes.byref(p)))
+
+
+def launch_count(p: Problem, readout: bool = False) -> int:
+    return int(load().mru_launch_count(ctypes.byref(p), int(bool(readout))))
+
+
+def status_string(status: int) -> str:
+    return load().mru_status_string(int(status)).decode()
+
+
+def build_states(p: Problem, x: int, X_out: int, ws: int, ws_bytes: int, stream: int = 0) -> int:
+    return load().mru_build_states(ctypes.byref(p), x, X_out, ws, ws_bytes, stream)
+
+
+def scan(p: Problem, X: int, S0: int | None, S_out: int, ws: int, ws_bytes: int, stream: int = 0) -> int:
+    return load().mru_scan(ctypes.byref(p), X, S0, S_out, ws, ws_bytes, stream)
+
+
+def scan_fused(p: Problem, x: int, S0: int | None, readout: Readout | None, S_out: int | None,
+               o_out: int | None, ws: int, ws_bytes: int, stream: int = 0) -> int:
+    ro = ctypes.byref(readout) if readout is not None else None
+    return load().mru_scan_fused(ctypes.byref(p), x, S0, ro, S_out, o_out, ws, ws_bytes, stream)
+
+
+def last_device_status(ws: int, stream: int = 0) -> int:
+    return load().mru_last_device_status(ws, stream)
+
+
+def set_profile_events(handles) -> int:
+    """handles: list of cudaEvent_t values (ints), or None/[] to switch off."""
+    if not handles:
+        return load().mru_set_profile_events(None, 0)
+    arr = (ctypes.c_void_p * len(handles))(*handles)
+    return load().mru_set_profile_events(arr, len(handles))
+
+
+# --------------------------------------------------------- tensor level ---
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev_ptr(t, name):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _check(rc, what):
+    if rc != OK:
+        raise MruError(rc, what)
+
+
+def workspace_t(p: Problem, device="cuda"):
+    torch = _torch()
+    nbytes = workspace_size(p)
+    if nbytes == 0:
+        raise MruError(ERR_INVALID_ARG, "workspace_size")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def check_device_status(ws, stream=None):
+    _check(last_device_status(ws.data_ptr(), _stream(stream)), "device status")
+
+
+def scan_fused_t(p: Problem, x, *, S0=None, u=None, snapshot_every: int = 0, out=None, o_out=None,
+                 snapshots=None, ws=None, stream=None):
+    """x: CUDA tensor [B, L, H*n*n] (float32, or bfloat16 when x_dtype is bf16).
+    Without u: returns S [B, L, H, n, n].  With u: returns (o, snapshots)."""
+    torch = _torch()
+    dev = x.device
+    if ws is None:
+        ws = workspace_t(p, dev)
+    B, L, H, n = p.B, p.L, p.H, p.n
+    s = _stream(stream)
+    if u is None:
+        if out is None:
+            out = torch.empty((B, L, H, n, n), dtype=torch.float32, device=dev)
+        rc = scan_fused(p, _dev_ptr(x, "x"), _dev_ptr(S0, "S0"), None, _dev_ptr(out, "out"), None,
+                        ws.data_ptr(), ws.numel(), s)
+        _check(rc, "mru_scan_fused")
+        return out
+    if o_out is None:
+        o_out = torch.empty((B, L, H, n), dtype=torch.float32, device=dev)
+    if snapshot_every > 0 and snapshots is None:
+        snapshots = torch.empty((B, L // snapshot_every, H, n, n), dtype=torch.float32, device=dev)
+    ro = Readout(_dev_ptr(u, "u"), int(snapshot_every), _dev_ptr(snapshots, "snapshots") if snapshot_every > 0 else None)
+    rc = scan_fused(p, _dev_ptr(x, "x"), _dev_ptr(S0, "S0"), ro, None, _dev_ptr(o_out, "o_out"),
+                    ws.data_ptr(), ws.numel(), s)
+    _check(rc, "mru_scan_fused")
+    return o_out, snapshots
+
+
+def scan_t(p: Problem, X, *, S0=None, out=None, ws=None, stream=None):
+    torch = _torch()
+    if ws is None:
+        ws = workspace_t(p, X.device)
+    if out is None:
+        out = torch.empty((p.B, p.L, p.H, p.n, p.n), dtype=torch.float32, device=X.device)
+    rc = scan(p, _dev_ptr(X, "X"), _dev_ptr(S0, "S0"), _dev_ptr(out, "out"), ws.data_ptr(), ws.numel(),
+              _stream(stream))
+    _check(rc, "mru_scan")
+    return out
+
+
+def build_states_t(p: Problem, x, *, out=None, ws=None, stream=None):
+    torch = _torch()
+    if ws is None:
+        ws = workspace_t(p, x.device)
+    if out is None:
+        out = torch.empty((p.B, p.L, p.H, p.n, p.n), dtype=torch.float32, device=x.device)
+    rc = build_states(p, _dev_ptr(x, "x"), _dev_ptr(out, "out"), ws.data_ptr(), ws.numel(), _stream(stream))
+    _check(rc, "mru_build_states")
+    return out

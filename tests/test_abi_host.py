@@ -1,0 +1,115 @@
+"""Host-side checks of the C-ABI library (no GPU needed, no kernel launched):
+libmru.so loads, exports every entry point include/mru.h declares, sizes its
+workspace, and rejects bad arguments synchronously before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_rnn_scan_b200 import inputs as gen
+from linear_rnn_scan_b200 import mru
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_rnn_scan_b200 import build
+    build.build()
+    return mru.load()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "mru.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mru_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 8
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(mru.EXPORTS) == names
+
+
+def test_problem_struct_matches_header():
+    # field order and widths of mru_problem as declared in include/mru.h
+    text = open(os.path.join(ROOT, "include", "mru.h")).read()
+    body = re.search(r"typedef struct \{(.*?)\} mru_problem;", text, re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if not decl:
+            continue
+        typ, names = decl.split(None, 1)
+        for nm in names.split(","):
+            fields.append((nm.strip(), typ))
+    widths = {"int64_t": 8, "int32_t": 4, "float": 4}
+    assert [f for f, _ in fields] == [f for f, _ in mru.Problem._fields_]
+    for (f, typ), (f2, ct) in zip(fields, mru.Problem._fields_):
+        assert widths[typ] == ctypes.sizeof(ct), f
+
+
+def test_workspace_size(lib):
+    w = gen.WORKLOADS["n16_detnorm_b8h8l4096"]
+    p = mru.problem_from_workload(w)
+    ws = mru.workspace_size(p)
+    assert ws >= 256 and ws % 256 == 0
+    C = mru.chosen_chunk(p)
+    assert C >= 1 and (C & (C - 1)) == 0
+    K = -(-w.L // C)
+    assert ws >= 256 + w.B * w.H * K * 256 * (4 + 8 + 4)
+    for n in (4, 8, 16, 32, 64):
+        assert mru.workspace_size(mru.problem(1, 1, 7, n)) >= 256
+    assert mru.workspace_size(mru.problem(1, 1, 7, 12)) == 0          # unsupported n
+    assert mru.workspace_size(mru.problem(-1, 1, 7, 16)) == 0         # negative size
+    assert mru.workspace_size(mru.problem(0, 0, 0, 16)) >= 256        # empty is valid
+
+
+def test_chunk_override(lib):
+    p = mru.problem(2, 3, 100, 16, chunk=7)
+    assert mru.chosen_chunk(p) == 7
+    assert mru.launch_count(p) >= 1
+    assert mru.launch_count(mru.problem(0, 3, 100, 16)) == 0
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert isinstance(mru.status_string(s), str) and mru.status_string(s)
+    assert "unknown" in mru.status_string(99)
+
+
+def test_invalid_arguments_rejected_before_any_launch(lib):
+    p = mru.problem(1, 1, 8, 16)
+    nb = mru.workspace_size(p)
+    fake = 1 << 20  # never dereferenced: every call below fails its checks first
+    assert mru.scan_fused(p, 0, None, None, fake, None, fake, nb) == mru.ERR_INVALID_ARG       # x null
+    assert mru.scan_fused(p, fake, None, None, 0, None, fake, nb) == mru.ERR_INVALID_ARG       # S_out null
+    assert mru.scan_fused(p, fake + 4, None, None, fake, None, fake, nb) == mru.ERR_INVALID_ARG  # misaligned
+    assert mru.scan_fused(p, fake, None, None, fake, None, fake, nb) == mru.ERR_INVALID_ARG    # alias
+    assert mru.scan_fused(p, fake, None, None, 2 * fake, None, 3 * fake, nb - 1) == mru.ERR_WORKSPACE
+    bad = mru.problem(1, 1, 8, 12)
+    assert mru.scan_fused(bad, fake, None, None, 2 * fake, None, 3 * fake, nb) == mru.ERR_UNSUPPORTED
+    bad = mru.problem(1, 1, 8, 16, mode=7)
+    assert mru.scan_fused(bad, fake, None, None, 2 * fake, None, 3 * fake, nb) == mru.ERR_INVALID_ARG
+    ro = mru.Readout(None, 0, None)
+    assert mru.scan_fused(p, fake, None, ro, None, 2 * fake, 3 * fake, nb) == mru.ERR_INVALID_ARG  # u null
+    ro = mru.Readout(4 * fake, 4, None)
+    assert mru.scan_fused(p, fake, None, ro, None, 2 * fake, 3 * fake, nb) == mru.ERR_INVALID_ARG  # snaps null
+    assert mru.scan(p, fake, None, fake, 3 * fake, nb) == mru.ERR_INVALID_ARG                  # X aliases S
+    assert mru.build_states(p, 0, fake, 3 * fake, nb) == mru.ERR_INVALID_ARG
+    assert mru.last_device_status(0) == mru.ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    missing = str(tmp_path / "libmru.so")
+    saved = mru._lib
+    try:
+        mru._lib = None
+        with pytest.raises(ImportError):
+            mru.load(missing)
+    finally:
+        mru._lib = saved

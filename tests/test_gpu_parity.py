@@ -1,0 +1,223 @@
+"""GPU parity: the CUDA path (through the C-ABI) against the fp64 oracle on
+the same seeded inputs.  Bit-exact where the arithmetic is exact (integer
+permutation and shear products check indexing, layout, chunking and carries),
+within the relative Frobenius gate elsewhere (1e-4 fp32, 1e-2 tensor-core
+paths), over several chunks and ragged tails, every n, every construction
+mode, both input dtypes, with and without S0, and with the readout."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+from linear_rnn_scan_b200 import inputs as gen
+from linear_rnn_scan_b200 import mru
+
+from gpu_helpers import (TOL_FP32, compare_readout, compare_S, oracle_problem, run_fused, to_device_x,
+                         torch)
+
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+NS = [4, 8, 16, 32, 64]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    t = torch()
+    if not t.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    mru.load()
+    yield
+
+
+def small(n, mode, *, B=1, H=1, L=37, x_dtype="f32", alpha=None, add_identity=1, seed=7):
+    if alpha is None:
+        alpha = 0.3 / np.sqrt(n)
+    return gen.Workload(f"t{n}", B=B, H=H, L=L, n=n, x_dtype=x_dtype, mode=mode, alpha=float(alpha),
+                        add_identity=add_identity, seed=seed)
+
+
+# ---------------------------------------------------------------- exact ---
+
+def _perm_inputs(B, H, L, n, seed):
+    r = np.random.default_rng(seed)
+    x = np.zeros((B, L, H, n, n), np.float32)
+    for b in range(B):
+        for t in range(L):
+            for h in range(H):
+                x[b, t, h, np.arange(n), r.permutation(n)] = 1.0
+    return x.reshape(B, L, H * n * n)
+
+
+def _shear_inputs(B, H, L, n, seed):
+    r = np.random.default_rng(seed)
+    x = np.zeros((B, L, H, n, n), np.float32)
+    for b in range(B):
+        for t in range(L):
+            for h in range(H):
+                x[b, t, h] = np.eye(n, dtype=np.float32)
+                i, j = sorted(r.choice(n, 2, replace=False))
+                if t % 2:
+                    i, j = j, i
+                x[b, t, h, i, j] = r.choice([-1.0, 1.0])
+    return x.reshape(B, L, H * n * n)
+
+
+@pytest.mark.parametrize("n", NS)
+@pytest.mark.parametrize("kind", ["perm", "shear"])
+@pytest.mark.parametrize("chunk", [1, 5, 16, 0])
+def test_exact_integer_products(n, kind, chunk):
+    B, H, L = 2, 3, 41
+    w = small(n, gen.MODE_RESHAPE, B=B, H=H, L=L, alpha=1.0, add_identity=0)
+    x = (_perm_inputs if kind == "perm" else _shear_inputs)(B, H, L, n, seed=n + chunk)
+    S_ref = oracle.scan(oracle_problem(w), x)
+    assert np.abs(S_ref).max() < 2 ** 22
+    S, st = run_fused(w, x, chunk=chunk)
+    assert st == mru.OK
+    assert np.array_equal(S.astype(np.float64), S_ref), np.argwhere(S.astype(np.float64) != S_ref)[:5]
+
+
+@pytest.mark.parametrize("n", [4, 16, 64])
+def test_exact_with_initial_state(n):
+    B, H, L = 1, 2, 23
+    w = small(n, gen.MODE_RESHAPE, B=B, H=H, L=L, alpha=1.0, add_identity=0)
+    x = _perm_inputs(B, H, L, n, seed=3)
+    S0 = _perm_inputs(B, 1, H, n, seed=4).reshape(B, H, n, n) * 2.0 - np.eye(n, dtype=np.float32)
+    S_ref = oracle.scan(oracle_problem(w), x, S0.astype(np.float64))
+    S, st = run_fused(w, x, S0=S0, chunk=4)
+    assert st == mru.OK and np.array_equal(S.astype(np.float64), S_ref)
+
+
+# --------------------------------------------------------------- parity ---
+
+MODES = [gen.MODE_RESHAPE, gen.MODE_DETNORM, gen.MODE_LDU]
+
+
+@pytest.mark.parametrize("n", NS)
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("L,chunk", [(1, 0), (15, 16), (16, 16), (17, 16), (53, 16), (97, 0)])
+def test_parity_small(n, mode, L, chunk):
+    w = small(n, mode, B=2, H=3, L=L, seed=100 + n + L)
+    x = gen.make_x(w)
+    S, st = run_fused(w, x, chunk=chunk)
+    assert st == mru.OK
+    e = compare_S(w, x, S)
+    assert e["count"] == w.B * w.L * w.H
+    assert e["max"] <= TOL_FP32, e
+
+
+@pytest.mark.parametrize("n", NS)
+@pytest.mark.parametrize("mode", MODES)
+def test_parity_bf16_and_initial_state(n, mode):
+    w = small(n, mode, B=1, H=2, L=29, x_dtype="bf16", seed=300 + n)
+    x = gen.make_x(w)
+    S0 = gen.make_S0(w, seed=301 + n)
+    S, st = run_fused(w, x, S0=S0, chunk=8)
+    assert st == mru.OK
+    e = compare_S(w, x, S, S0=S0)
+    assert e["max"] <= TOL_FP32, e
+
+
+@pytest.mark.parametrize("n", [4, 16, 64])
+def test_parity_far_from_identity(n):
+    """Reshape without the identity and determinant correction of a matrix
+    that needs pivoting: the general (not near-identity) construction."""
+    for mode, add_id, alpha in ((gen.MODE_RESHAPE, 0, 1.0 / np.sqrt(n)), (gen.MODE_DETNORM, 0, 1.0),
+                                (gen.MODE_DETNORM, 1, 3.0)):
+        w = small(n, mode, B=1, H=2, L=19, alpha=alpha, add_identity=add_id, seed=400 + n)
+        x = gen.make_x(w)
+        S, st = run_fused(w, x, chunk=4)
+        assert st == mru.OK
+        e = compare_S(w, x, S, t_end=19)
+        assert e["max"] <= TOL_FP32, (mode, add_id, e)
+
+
+@pytest.mark.parametrize("chunk", [1, 2, 3, 31, 64, 1024])
+def test_chunk_sizes_agree(chunk):
+    w = small(16, gen.MODE_DETNORM, B=2, H=2, L=200, alpha=0.05 / 4, seed=500)
+    x = gen.make_x(w)
+    S, st = run_fused(w, x, chunk=chunk)
+    assert st == mru.OK
+    assert compare_S(w, x, S)["max"] <= TOL_FP32
+
+
+@pytest.mark.parametrize("n", NS)
+def test_readout_and_snapshots(n):
+    w = small(n, gen.MODE_DETNORM, B=2, H=2, L=70, seed=600 + n).with_(readout=True, snapshot_every=8)
+    x = gen.make_x(w)
+    u = gen.make_u(w)
+    S0 = gen.make_S0(w, seed=601)
+    for s0 in (None, S0):
+        (o, snaps), st = run_fused(w, x, S0=s0, u=u, every=8, chunk=16)
+        assert st == mru.OK and snaps.shape == (2, 8, 2, n, n)
+        e = compare_readout(w, x, o, snaps, u, 8, S0=s0)
+        assert e["o"]["max"] <= TOL_FP32 and e["snap"]["max"] <= TOL_FP32, e
+    (o, snaps), st = run_fused(w, x, u=u, every=0, chunk=16)
+    assert snaps is None and compare_readout(w, x, o, None, u, 0)["o"]["max"] <= TOL_FP32
+
+
+@pytest.mark.parametrize("n", [4, 16, 32])
+@pytest.mark.parametrize("mode", MODES)
+def test_unfused_build_then_scan(n, mode):
+    t = torch()
+    w = small(n, mode, B=1, H=3, L=45, seed=700 + n)
+    x = gen.make_x(w)
+    S_fused, _ = run_fused(w, x, chunk=8)
+    for smi in (0, 1):
+        p = mru.problem_from_workload(w, chunk=8, store_minus_identity=smi)
+        X = mru.build_states_t(p, to_device_x(x))
+        t.cuda.synchronize()
+        # lifted matrices against the oracle's X_t
+        Xh = X.cpu().numpy().astype(np.float64)
+        for (tt, h) in ((0, 0), (17, 2), (44, 1)):
+            ref = oracle.lift(oracle_problem(w), x, 0, tt, h)
+            got = Xh[0, tt, h] + (np.eye(n) if smi else 0.0)
+            assert np.abs(got - ref).max() <= 2e-6 * max(1.0, np.abs(ref).max())
+        S = mru.scan_t(p, X).cpu().numpy()
+        assert compare_S(w, x, S)["max"] <= TOL_FP32
+        np.testing.assert_allclose(S, S_fused, rtol=0, atol=5e-5 * np.abs(S_fused).max())
+
+
+def test_empty_and_degenerate_shapes():
+    t = torch()
+    for B, H, L in ((0, 2, 5), (2, 0, 5), (2, 2, 0)):
+        p = mru.problem(B, H, L, 16, mode=gen.MODE_DETNORM, alpha=0.01)
+        x = t.zeros((max(B, 1), max(L, 1), max(H, 1) * 256), device="cuda")
+        out = t.empty((max(B, 1), max(L, 1), max(H, 1), 16, 16), device="cuda")
+        ws = mru.workspace_t(p)
+        assert mru.scan_fused(p, x.data_ptr(), None, None, out.data_ptr(), None, ws.data_ptr(), ws.numel(),
+                              t.cuda.current_stream().cuda_stream) == mru.OK
+        assert mru.last_device_status(ws.data_ptr(), t.cuda.current_stream().cuda_stream) == mru.OK
+
+
+def test_singular_matrix_reported():
+    w = small(16, gen.MODE_DETNORM, B=1, H=2, L=9, alpha=1.0, add_identity=0)
+    x = gen.make_x(w)
+    x[0, 4, 256:512] = 0.0                      # head 1, token 4: X~ = 0
+    S, st = run_fused(w, x, chunk=4)
+    assert st == mru.ERR_SINGULAR
+    assert np.isfinite(S).all()
+    # the other head is unaffected
+    e = compare_S(w, x, S, bh=[0])
+    assert e["max"] <= TOL_FP32
+
+
+def test_status_resets_between_calls():
+    w = small(16, gen.MODE_DETNORM, B=1, H=1, L=5, alpha=1.0, add_identity=0)
+    x = gen.make_x(w)
+    x0 = x.copy()
+    x0[0, 2] = 0.0
+    _, st = run_fused(w, x0)
+    assert st == mru.ERR_SINGULAR
+    _, st = run_fused(w, x)
+    assert st == mru.OK
+
+
+def test_repeated_calls_are_deterministic():
+    w = small(32, gen.MODE_LDU, B=2, H=4, L=300, x_dtype="bf16", seed=800)
+    x = gen.make_x(w)
+    first, _ = run_fused(w, x)
+    for _ in range(5):
+        again, _ = run_fused(w, x)
+        assert np.array_equal(first, again)
