@@ -10,7 +10,7 @@
 // Numerics.  Every matrix is carried in identity-split form, X = I + F,
 // P = I + Q, so that the near-identity inputs of the determinant-corrected
 // workloads lose nothing to the implicit 1 on the diagonal:
-//     Q_t = Q_{t-1} + F_t + Q_{t-1} F_t            (in-chunk, fp32)
+//     Q_t = Q_{t-1} + (F_t + Q_{t-1} F_t)          (in-chunk, fp32)
 //     carry_{k+1} = carry_k + carry_k Q_k          (chunk totals, fp64)
 //     S_t = carry + carry Q_t                      (fix-up, fp32)
 // The chunk-total scan is two-level (groups of G totals, then the group
@@ -290,10 +290,13 @@ k_chunk_prefix(KParams p, const void* src, const float* u, int64_t snap_every, f
             const int e = tid + r * kThreads;
             if (e < NN) {
                 const int i = e / N, j = e % N;
-                float a = sQ[e] + sF[e];
+                // The product term is accumulated on its own (its magnitude is
+                // that of F) and only then added to Q: accumulating on top of
+                // Q + F would round every partial sum at the scale of Q.
+                float a = 0.0f;
 #pragma unroll 8
                 for (int q = 0; q < N; ++q) a = fmaf(sQ[i * N + q], sF[q * N + j], a);
-                acc[r] = a;
+                acc[r] = sQ[e] + (sF[e] + a);
             }
         }
         __syncthreads();
@@ -347,9 +350,9 @@ k_carry_local(KParams p, const float* totals, double* local)
             const int e = tid + r * kThreads;
             if (e < NN) {
                 const int i = e / N, c = e % N;
-                double a = sR[e] + sT[e];
+                double a = 0.0;
                 for (int q = 0; q < N; ++q) a = fma(sR[i * N + q], sT[q * N + c], a);
-                acc[r] = a;
+                acc[r] = sR[e] + (sT[e] + a);
             }
         }
         __syncthreads();
@@ -390,9 +393,9 @@ k_carry_groups(KParams p, const float* S0, const double* local, double* gcarry)
             const int e = tid + r * kThreads;
             if (e < NN) {
                 const int i = e / N, c = e % N;
-                double a = sG[e];
+                double a = 0.0;
                 for (int q = 0; q < N; ++q) a = fma(sG[i * N + q], sT[q * N + c], a);
-                acc[r] = a;
+                acc[r] = sG[e] + a;
             }
         }
         __syncthreads();
@@ -424,10 +427,10 @@ k_carry_final(KParams p, const double* local, const double* gcarry, float* carry
     __syncthreads();
     for (int e = tid; e < NN; e += kThreads) {
         const int i = e / N, c = e % N;
-        double a = sG[e];
+        double a = 0.0;
         if (!first)
             for (int q = 0; q < N; ++q) a = fma(sG[i * N + q], sT[q * N + c], a);
-        carry[(bh * p.K + k) * NN + e] = (float)a;
+        carry[(bh * p.K + k) * NN + e] = (float)(sG[e] + a);
     }
 }
 
@@ -463,10 +466,10 @@ k_fixup(KParams p, const float* carry, const float* u, int64_t snap_every, float
             const int e = tid + r * kThreads;
             if (e < NN) {
                 const int i = e / N, j = e % N;
-                float a = sC[e];
+                float a = 0.0f;
 #pragma unroll 8
                 for (int q = 0; q < N; ++q) a = fmaf(sC[i * N + q], sQ[q * N + j], a);
-                acc[r] = a;
+                acc[r] = sC[e] + a;
             }
         }
 #pragma unroll
@@ -492,9 +495,9 @@ k_fixup(KParams p, const float* carry, const float* u, int64_t snap_every, float
         for (int j = tid; j < N; j += kThreads) sV[j] = o[j];
         __syncthreads();
         for (int i = tid; i < N; i += kThreads) {
-            float a = sCu[i];
+            float a = 0.0f;
             for (int j = 0; j < N; ++j) a = fmaf(sC[i * N + j], sV[j], a);
-            o[i] = a;
+            o[i] = sCu[i] + a;
         }
         __syncthreads();
     }
