@@ -134,6 +134,40 @@ int32_t mru_launch_count(const mru_problem* p, int32_t readout);
  * count == 0 switches the hook off.  Process-wide; not thread-safe. */
 mru_status mru_set_profile_events(void* const* events, int32_t count);
 
+/* Size of the fixed device scratch that mru_scan_fused_noalloc uses (16 MiB). */
+#define MRU_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/* mru_scan_fused without a workspace argument, for callers that may not
+ * allocate device memory at all: a plugin inside a host framework that owns
+ * every device allocation, or a service that reserves its whole memory budget
+ * at start-up and forbids allocation afterwards.  The method's pages have no
+ * counterpart to this entry point; it exists for such callers only.
+ *
+ * Arguments and results are those of mru_scan_fused; the caller still owns
+ * x, S0, the readout buffers, S_out and o_out.  The scratch is one
+ * file-scope device array of MRU_NOALLOC_SCRATCH_BYTES, held by every GPU
+ * whose context loads this library until the process exits.  The call
+ * allocates nothing (no cudaMalloc, no cudaFree, no allocating library call).
+ *
+ *   - Size limit: with p->chunk == 0 the chunk is the library's choice,
+ *     doubled until the workspace (mru_workspace_size) fits the scratch; a
+ *     problem that does not fit even then, or whose explicit p->chunk does not
+ *     fit, is rejected with MRU_ERR_WORKSPACE before anything is launched.
+ *   - Set-up: the first call on each device looks up the scratch's device
+ *     address (cudaGetSymbolAddress, with that device current) and caches
+ *     it; make that first call before any stream capture.
+ *   - Sharing: every call on a device uses the same scratch, which keeps the
+ *     last call's contents; the call clears what must start at zero itself.
+ *     Calls whose executions overlap on the GPU (on different streams, or
+ *     from different host threads) race on the scratch: serialise them.
+ *   - Status: when status_out (a device pointer to one uint32, 4-byte
+ *     aligned) is not NULL, the device status word is copied there on the
+ *     stream after the scan: 0 ok, bit 0 singular matrix, bit 1 timeout.
+ */
+mru_status mru_scan_fused_noalloc(const mru_problem* p, const void* x, const float* S0,
+                                  const mru_readout* ro, float* S_out, float* o_out,
+                                  uint32_t* status_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

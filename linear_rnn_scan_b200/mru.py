@@ -30,7 +30,8 @@ MATH = {"auto": 0, "fp32": 1, "tf32": 2, "tf32x3": 3, "bf16x3": 4}
 # Every symbol include/mru.h declares.
 EXPORTS = ["mru_workspace_size", "mru_build_states", "mru_scan", "mru_scan_fused",
            "mru_last_device_status", "mru_status_string", "mru_chosen_chunk", "mru_launch_count",
-           "mru_set_profile_events"]
+           "mru_set_profile_events", "mru_scan_fused_noalloc"]
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class Problem(ctypes.Structure):
@@ -85,6 +86,8 @@ def load(path: str = LIB_PATH):
             lib.mru_launch_count.restype = ctypes.c_int32
             lib.mru_set_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
             lib.mru_set_profile_events.restype = ctypes.c_int
+            lib.mru_scan_fused_noalloc.argtypes = [P, vp, vp, ctypes.POINTER(Readout), vp, vp, vp, vp]
+            lib.mru_scan_fused_noalloc.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -134,6 +137,14 @@ def scan_fused(p: Problem, x: int, S0: int | None, readout: Readout | None, S_ou
                o_out: int | None, ws: int, ws_bytes: int, stream: int = 0) -> int:
     ro = ctypes.byref(readout) if readout is not None else None
     return load().mru_scan_fused(ctypes.byref(p), x, S0, ro, S_out, o_out, ws, ws_bytes, stream)
+
+
+def scan_fused_noalloc(p: Problem, x: int, S0: int | None, readout: Readout | None, S_out: int | None,
+                       o_out: int | None, status_out: int | None = None, stream: int = 0) -> int:
+    """mru_scan_fused without a workspace: scratch is the library's fixed
+    device array (for callers that may not allocate device memory)."""
+    ro = ctypes.byref(readout) if readout is not None else None
+    return load().mru_scan_fused_noalloc(ctypes.byref(p), x, S0, ro, S_out, o_out, status_out, stream)
 
 
 def last_device_status(ws: int, stream: int = 0) -> int:
