@@ -63,11 +63,13 @@ typedef enum {
 typedef enum { MRU_MODE_RESHAPE = 0, MRU_MODE_DETNORM = 1, MRU_MODE_LDU = 2 } mru_mode;
 typedef enum { MRU_F32 = 0, MRU_BF16 = 1 } mru_dtype;
 typedef enum {
-    MRU_MATH_AUTO = 0,    /* library choice per n and dtype */
-    MRU_MATH_FP32 = 1,    /* fp32 FMA throughout */
+    MRU_MATH_AUTO = 0,    /* library choice per n and dtype (fp32-accurate) */
+    MRU_MATH_FP32 = 1,    /* fp32 FMA throughout (the generic kernels) */
     MRU_MATH_TF32 = 2,    /* tensor-core products with tf32 operands, fp32 accumulate */
     MRU_MATH_TF32X3 = 3,  /* split-tf32 (hi/lo, three products), fp32 accumulate */
     MRU_MATH_BF16X3 = 4   /* split-bf16 (hi/lo, three products), fp32 accumulate */
+    /* A mode without a specialised kernel for the problem's n and dtype runs
+     * the fp32 kernels, which are at least as accurate. */
 } mru_math;
 
 typedef struct {
@@ -125,6 +127,10 @@ int32_t mru_chosen_chunk(const mru_problem* p);
 
 /* Number of kernel launches one call of mru_scan_fused makes for p. */
 int32_t mru_launch_count(const mru_problem* p, int32_t readout);
+
+/* Name of the i-th kernel one call of mru_scan_fused launches for p (with the
+ * readout when readout != 0); "" when i is out of range or p is invalid. */
+const char* mru_kernel_name(const mru_problem* p, int32_t readout, int32_t i);
 
 /* Benchmark hook.  With count > 0, every later mru_scan / mru_scan_fused call
  * records events[2*i] just before and events[2*i+1] just after its i-th

@@ -14,16 +14,32 @@ bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Tokens per chunk: aim at about 4096 chains (b, h, chunk) so that a
-// generic-path launch fills 148 SMs several times over; a power of two in
-// [16, 1024].
-int32_t choose_chunk(const mru_problem& p)
+// Tokens per chunk of the generic path: aim at about 4096 chains (b, h,
+// chunk) so that a launch fills 148 SMs several times over; a power of two
+// in [16, 1024].
+int32_t generic_chunk(const mru_problem& p)
 {
-    if (p.chunk > 0) return p.chunk;
     const int64_t th = p.B * p.H * p.L;
     int64_t c = 16;
     while (c < 1024 && c * 4096 < th) c *= 2;
     return (int32_t)c;
+}
+
+// Whether the fused scan of this problem (with or without the readout) runs
+// on the specialised n = 16 kernels, given the chunk they need.
+bool fast16_eligible(const mru_problem& p, bool readout)
+{
+    return p.n == 16 && p.x_dtype == MRU_F32 && !readout &&
+           (p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM) &&
+           (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32X3) &&
+           (p.chunk == 0 || p.chunk == n16::chunk_tokens());
+}
+
+int32_t choose_chunk(const mru_problem& p, int32_t src, bool readout)
+{
+    if (p.chunk > 0) return p.chunk;
+    if (src == SRC_EMBEDDING && fast16_eligible(p, readout)) return n16::chunk_tokens();
+    return generic_chunk(p);
 }
 
 int32_t choose_group(int64_t K)
@@ -45,7 +61,7 @@ mru_status check_problem(const mru_problem* p)
     return MRU_OK;
 }
 
-KParams make_params(const mru_problem& p, int32_t src)
+KParams make_params(const mru_problem& p, int32_t src, bool readout)
 {
     KParams k;
     memset(&k, 0, sizeof k);
@@ -53,7 +69,8 @@ KParams make_params(const mru_problem& p, int32_t src)
     k.x_dtype = p.x_dtype; k.mode = p.mode; k.src = src;
     k.alpha = p.alpha; k.add_identity = p.add_identity;
     k.ldu_a = p.ldu_offdiag; k.ldu_d = p.ldu_diag;
-    k.chunk = choose_chunk(p);
+    k.math = p.math;
+    k.chunk = choose_chunk(p, src, readout);
     k.K = ceil_div(p.L, k.chunk);
     k.group = choose_group(k.K);
     k.NG = k.K > 0 ? ceil_div(k.K, k.group) : 0;
@@ -102,13 +119,26 @@ extern "C" {
 size_t mru_workspace_size(const mru_problem* p)
 {
     if (check_problem(p) != MRU_OK) return 0;
-    return layout(make_params(*p, SRC_EMBEDDING)).bytes;
+    // large enough for every entry point and for both output forms
+    size_t b = 0;
+    for (int32_t src : {SRC_EMBEDDING, SRC_X})
+        for (bool ro : {false, true}) {
+            const size_t w = layout(make_params(*p, src, ro)).bytes;
+            if (w > b) b = w;
+        }
+    return b;
 }
 
 int32_t mru_chosen_chunk(const mru_problem* p)
 {
     if (check_problem(p) != MRU_OK) return 0;
-    return choose_chunk(*p);
+    return choose_chunk(*p, SRC_EMBEDDING, false);
+}
+
+const char* mru_kernel_name(const mru_problem* p, int32_t readout, int32_t i)
+{
+    if (check_problem(p) != MRU_OK) return "";
+    return kernel_name(make_params(*p, SRC_EMBEDDING, readout != 0), readout != 0, i);
 }
 
 int32_t mru_launch_count(const mru_problem* p, int32_t readout)
@@ -125,7 +155,7 @@ mru_status mru_build_states(const mru_problem* p, const void* x, float* X_out, v
     mru_status st = check_problem(p);
     if (st != MRU_OK) return st;
     if (!x || !X_out || !ws || !aligned16(x) || !aligned16(X_out) || !aligned16(ws)) return MRU_ERR_INVALID_ARG;
-    KParams k = make_params(*p, SRC_EMBEDDING);
+    KParams k = make_params(*p, SRC_EMBEDDING, false);
     Workspace W = layout(k);
     if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -142,7 +172,7 @@ mru_status mru_scan(const mru_problem* p, const float* X, const float* S0, float
     if (!X || !S_out || !ws || !aligned16(X) || !aligned16(S_out) || !aligned16(ws)) return MRU_ERR_INVALID_ARG;
     if (S0 && !aligned16(S0)) return MRU_ERR_INVALID_ARG;
     if ((const void*)X == (const void*)S_out) return MRU_ERR_INVALID_ARG;
-    KParams k = make_params(*p, p->store_minus_identity ? SRC_F : SRC_X);
+    KParams k = make_params(*p, p->store_minus_identity ? SRC_F : SRC_X, false);
     Workspace W = layout(k);
     if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -171,7 +201,7 @@ mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0, 
     } else {
         if (!S_out || !aligned16(S_out) || (const void*)S_out == x) return MRU_ERR_INVALID_ARG;
     }
-    KParams k = make_params(*p, SRC_EMBEDDING);
+    KParams k = make_params(*p, SRC_EMBEDDING, ro != nullptr);
     Workspace W = layout(k);
     if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

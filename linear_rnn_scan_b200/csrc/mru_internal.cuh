@@ -30,6 +30,7 @@ struct KParams {
     int32_t add_identity;
     float ldu_a;
     float ldu_d;
+    int32_t math;        // mru_math requested
     int32_t chunk;       // tokens per chunk (C)
     int64_t K;           // chunks per sequence, ceil(L / C)
     int32_t group;       // chunk totals per carry group (G)
@@ -53,11 +54,22 @@ __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + 
 // no events are registered.
 void profile_mark(int kernel, int after, cudaStream_t s);
 
+// n = 16 tensor-core kernels (mru_n16.cu).
+namespace n16 {
+int chunk_tokens();
+bool supports(const KParams& p, bool readout);
+cudaError_t launch_chunk(const KParams& p, const float* x, float* S_out, float* totals, uint32_t* status,
+                         cudaStream_t s);
+cudaError_t launch_fixup(const KParams& p, const float* carry, float* S_out, cudaStream_t s);
+}  // namespace n16
+
 // Launchers (mru_scan_v1.cu).
 cudaError_t launch_build_states(const KParams& p, const void* x, float* X_out, int store_minus_identity,
                                 void* ws_base, const Workspace& W, cudaStream_t s);
 cudaError_t launch_scan(const KParams& p, const void* src, const float* S0, const float* u,
                         int64_t snap_every, float* S_out, float* o_out, float* snaps,
                         void* ws_base, const Workspace& W, cudaStream_t s, int* launches);
+// Name of the i-th kernel one launch_scan call starts for this problem.
+const char* kernel_name(const KParams& p, bool readout, int i);
 
 }  // namespace mru

@@ -30,7 +30,7 @@ MATH = {"auto": 0, "fp32": 1, "tf32": 2, "tf32x3": 3, "bf16x3": 4}
 # Every symbol include/mru.h declares.
 EXPORTS = ["mru_workspace_size", "mru_build_states", "mru_scan", "mru_scan_fused",
            "mru_last_device_status", "mru_status_string", "mru_chosen_chunk", "mru_launch_count",
-           "mru_set_profile_events", "mru_scan_fused_noalloc"]
+           "mru_set_profile_events", "mru_scan_fused_noalloc", "mru_kernel_name"]
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -88,6 +88,8 @@ def load(path: str = LIB_PATH):
             lib.mru_set_profile_events.restype = ctypes.c_int
             lib.mru_scan_fused_noalloc.argtypes = [P, vp, vp, ctypes.POINTER(Readout), vp, vp, vp, vp]
             lib.mru_scan_fused_noalloc.restype = ctypes.c_int
+            lib.mru_kernel_name.argtypes = [P, ctypes.c_int32, ctypes.c_int32]
+            lib.mru_kernel_name.restype = ctypes.c_char_p
             _lib = lib
     return _lib
 
@@ -119,6 +121,11 @@ def chosen_chunk(p: Problem) -> int:
 
 def launch_count(p: Problem, readout: bool = False) -> int:
     return int(load().mru_launch_count(ctypes.byref(p), int(bool(readout))))
+
+
+def kernel_names(p: Problem, readout: bool = False) -> list:
+    n = launch_count(p, readout)
+    return [load().mru_kernel_name(ctypes.byref(p), int(bool(readout)), i).decode() for i in range(n)]
 
 
 def status_string(status: int) -> str:
