@@ -31,14 +31,13 @@ bool fast16_eligible(const mru_problem& p, bool readout)
 {
     return p.n == 16 && p.x_dtype == MRU_F32 && !readout &&
            (p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM) &&
-           (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32X3) &&
-           (p.chunk == 0 || p.chunk == n16::chunk_tokens());
+           (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32X3) && p.chunk % n16::kSub == 0;
 }
 
 int32_t choose_chunk(const mru_problem& p, int32_t src, bool readout)
 {
     if (p.chunk > 0) return p.chunk;
-    if (src == SRC_EMBEDDING && fast16_eligible(p, readout)) return n16::chunk_tokens();
+    if (src == SRC_EMBEDDING && fast16_eligible(p, readout)) return n16::preferred_chunk(p.B * p.H * p.L);
     return generic_chunk(p);
 }
 
@@ -77,13 +76,22 @@ KParams make_params(const mru_problem& p, int32_t src, bool readout)
     return k;
 }
 
-Workspace layout(const KParams& k)
+Workspace layout(const KParams& k, bool readout)
 {
     Workspace W;
+    memset(&W, 0, sizeof W);
     const size_t nn = (size_t)k.n * k.n;
     const size_t BH = (size_t)(k.B * k.H);
     size_t off = 0;
     W.status = off; off += 256;
+    if (n16::supports(k, readout)) {
+        W.fast = true;
+        W.totals = off; off = round_up(off + BH * k.K * nn * sizeof(float), 256);
+        W.cd = off; off = round_up(off + BH * (size_t)k.L * sizeof(float2), 256);
+        W.plan = carry::plan((int64_t)BH, k.K, (int)nn, off);
+        W.bytes = W.plan.end > off ? W.plan.end : off;
+        return W;
+    }
     W.totals = off; off = round_up(off + BH * k.K * nn * sizeof(float), 256);
     W.local = off;  off = round_up(off + BH * k.K * nn * sizeof(double), 256);
     W.gcarry = off; off = round_up(off + BH * k.NG * nn * sizeof(double), 256);
@@ -123,7 +131,7 @@ size_t mru_workspace_size(const mru_problem* p)
     size_t b = 0;
     for (int32_t src : {SRC_EMBEDDING, SRC_X})
         for (bool ro : {false, true}) {
-            const size_t w = layout(make_params(*p, src, ro)).bytes;
+            const size_t w = layout(make_params(*p, src, ro), ro).bytes;
             if (w > b) b = w;
         }
     return b;
@@ -138,15 +146,25 @@ int32_t mru_chosen_chunk(const mru_problem* p)
 const char* mru_kernel_name(const mru_problem* p, int32_t readout, int32_t i)
 {
     if (check_problem(p) != MRU_OK) return "";
-    return kernel_name(make_params(*p, SRC_EMBEDDING, readout != 0), readout != 0, i);
+    const KParams k = make_params(*p, SRC_EMBEDDING, readout != 0);
+    const Workspace W = layout(k, readout != 0);
+    if (!W.fast) return kernel_name(k, readout != 0, i);
+    const int lv = W.plan.levels;
+    if (i == 0) return "k16_reduce";
+    if (i >= 1 && i <= lv) return "k_level";
+    if (i == lv + 1) return "k_top";
+    if (i >= lv + 2 && i <= 2 * lv) return "k_down";
+    if (i == 2 * lv + 1) return "k16_apply";
+    return "";
 }
 
 int32_t mru_launch_count(const mru_problem* p, int32_t readout)
 {
-    (void)readout;
     if (check_problem(p) != MRU_OK) return 0;
     if (p->B * p->H * p->L == 0) return 0;
-    return 5;
+    const KParams k = make_params(*p, SRC_EMBEDDING, readout != 0);
+    const Workspace W = layout(k, readout != 0);
+    return W.fast ? 2 + carry::launches(W.plan) : 5;
 }
 
 mru_status mru_build_states(const mru_problem* p, const void* x, float* X_out, void* ws, size_t ws_bytes,
@@ -156,7 +174,7 @@ mru_status mru_build_states(const mru_problem* p, const void* x, float* X_out, v
     if (st != MRU_OK) return st;
     if (!x || !X_out || !ws || !aligned16(x) || !aligned16(X_out) || !aligned16(ws)) return MRU_ERR_INVALID_ARG;
     KParams k = make_params(*p, SRC_EMBEDDING, false);
-    Workspace W = layout(k);
+    Workspace W = layout(k, false);
     if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = reset_status(ws, s)) != MRU_OK) return st;
@@ -173,7 +191,7 @@ mru_status mru_scan(const mru_problem* p, const float* X, const float* S0, float
     if (S0 && !aligned16(S0)) return MRU_ERR_INVALID_ARG;
     if ((const void*)X == (const void*)S_out) return MRU_ERR_INVALID_ARG;
     KParams k = make_params(*p, p->store_minus_identity ? SRC_F : SRC_X, false);
-    Workspace W = layout(k);
+    Workspace W = layout(k, false);
     if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = reset_status(ws, s)) != MRU_OK) return st;
@@ -202,7 +220,7 @@ mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0, 
         if (!S_out || !aligned16(S_out) || (const void*)S_out == x) return MRU_ERR_INVALID_ARG;
     }
     KParams k = make_params(*p, SRC_EMBEDDING, ro != nullptr);
-    Workspace W = layout(k);
+    Workspace W = layout(k, ro != nullptr);
     if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = reset_status(ws, s)) != MRU_OK) return st;

@@ -38,12 +38,33 @@ struct KParams {
 };
 
 // Workspace carve-up (byte offsets from the workspace base).
+// Multi-level fp64 scan of chunk totals (mru_carry.cu).
+namespace carry {
+constexpr int kMaxLevels = 8;
+struct Plan {
+    int64_t nseq;                 // independent sequences (B * H)
+    int G;                        // group size at every level
+    int levels;                   // levels below the top
+    int64_t cnt[kMaxLevels + 1];  // matrices per sequence at each level
+    size_t R[kMaxLevels];         // local prefixes of level l (fp32 for l = 0, else fp64)
+    size_t Tot[kMaxLevels];       // group totals of level l (fp64)
+    size_t E[kMaxLevels + 1];     // exclusive carries of level l >= 1 (fp64)
+    size_t end;                   // first byte after the plan's buffers
+};
+Plan plan(int64_t nseq, int64_t K, int nn, size_t off);
+int launches(const Plan& pl);
+cudaError_t run_n16(const Plan& pl, const float* totals, const float* S0, char* ws, cudaStream_t s, int& slot);
+}  // namespace carry
+
 struct Workspace {
     size_t status;       // uint32 status word
     size_t totals;       // float  [B*H, K, n, n]   chunk totals, split form (T - I)
     size_t local;        // double [B*H, K, n, n]   inclusive in-group prefixes of totals, split form
     size_t gcarry;       // double [B*H, NG, n, n]  exclusive group carries (full matrices)
     size_t carry;        // float  [B*H, K, n, n]   exclusive chunk carries (full matrices)
+    bool fast;           // specialised kernels: chunk totals, per-token scalars, carry plan
+    size_t cd;           // float2 [B, L, H] per-token scalars (c alpha, diagonal of F)
+    carry::Plan plan;
     size_t bytes;        // total
 };
 
@@ -56,11 +77,13 @@ void profile_mark(int kernel, int after, cudaStream_t s);
 
 // n = 16 tensor-core kernels (mru_n16.cu).
 namespace n16 {
-int chunk_tokens();
+constexpr int kSub = 8;           // tokens per LU pass; chunks are multiples of it
 bool supports(const KParams& p, bool readout);
-cudaError_t launch_chunk(const KParams& p, const float* x, float* S_out, float* totals, uint32_t* status,
-                         cudaStream_t s);
-cudaError_t launch_fixup(const KParams& p, const float* carry, float* S_out, cudaStream_t s);
+int32_t preferred_chunk(int64_t token_heads);
+cudaError_t launch_reduce(const KParams& p, const float* x, float* totals, float2* cd, uint32_t* status,
+                          cudaStream_t s);
+cudaError_t launch_apply(const KParams& p, const float* x, const float2* cd, const carry::Plan& pl,
+                         const char* ws, float* S_out, cudaStream_t s);
 }  // namespace n16
 
 // Launchers (mru_scan_v1.cu).

@@ -1,30 +1,30 @@
 // mru_n16.cu -- n = 16 scan kernels on the tensor cores (fp32 embeddings,
-// reshape and determinant-corrected modes).
+// reshape and determinant-corrected modes), two passes over the embeddings:
 //
-// Same three phases and numerics as the generic path (identity split,
-// product term accumulated apart, fp64 per-token scalars, fp64 chunk-total
-// scan), mapped onto the B200 this way:
-//
-//  * chunk kernel  one warp per chain (b, h, chunk of 8 tokens), 8 chains per
-//                  CTA.  Phase 1: the CTA copies its 64 token-head slices to
-//                  shared memory (cp.async, rows padded to 20 words) and runs
-//                  64 LU factorisations at once, 4 lanes per token (each lane
-//                  owns rows r, r+4, r+8, r+12 in registers; the pivot row is
-//                  broadcast by shuffles inside the 4-lane group).  Phase 2:
-//                  each warp runs its chain Q_t = Q_{t-1} + (F_t + Q_{t-1} F_t)
-//                  with mma.sync m16n8k8 tf32 in split precision (hi + lo
-//                  operands, three products), the state staying in the
-//                  accumulator registers from step to step: the contraction
+//  * reduce pass   one warp per chain (b, h, chunk of C = 8m tokens); warps
+//                  never wait for each other.  Per pass of 8 tokens the warp
+//                  copies the 8 token-head slices to its shared memory
+//                  (cp.async, rows padded to 20 words), factorises the 8
+//                  matrices at once with 4 lanes per token (lane r owns rows
+//                  r, r+4, r+8, r+12 in registers; the pivot row is broadcast
+//                  by shuffles inside the 4-lane group), records the token's
+//                  scalars (c alpha, diagonal of F) and advances the chunk
+//                  product Q_t = Q_{t-1} + (F_t + Q_{t-1} F_t) with mma.sync
+//                  m16n8k8 tf32 in split precision.  The state stays in the
+//                  accumulator registers from token to token: the contraction
 //                  index of the next product is permuted so that the
 //                  accumulator fragment of column tile j is exactly the A
-//                  fragment of k-tile j.
-//  * fix-up kernel one warp per chain: S_t = C + C Q_t with the carry C as the
-//                  split A operand (loaded once) and Q_t streamed in.
+//                  fragment of k-tile j.  Only the chunk total is written.
+//  * (the fp64 scan of chunk totals, mru_carry.cu)
+//  * apply pass    one warp per chain: forms the chunk's exact carry from the
+//                  carry scan (fp64), then runs the chain again from it,
+//                  S_t = S_{t-1} + S_{t-1} F_t, and writes every S_t.  No local
+//                  prefix ever goes to memory: per token·head the path moves
+//                  x twice and S once.
 //
 // Split-tf32 ("3xTF32", after Ootomo and Yokota, 2022): x = hi + lo with hi
 // the top 19 bits of x (sign, exponent, 10 mantissa bits) and lo = x - hi
-// exact in fp32; a b ~ a_hi b_hi + a_hi b_lo + a_lo b_hi, the small terms
-// first.
+// exact in fp32; a b ~ a_lo b_hi + a_hi b_lo + a_hi b_hi.
 #include "mru_internal.cuh"
 
 namespace mru {
@@ -35,13 +35,13 @@ constexpr int N = 16;
 constexpr int NN = N * N;
 constexpr int ROWW = 20;            // padded shared-memory row stride, in words
 constexpr int SLICE = N * ROWW;     // one token-head slice in shared memory
-constexpr int CT = 8;               // tokens per chunk
+constexpr int SUB = kSub;           // tokens per pass
 constexpr int WARPS = 8;            // chains per CTA
 constexpr int THREADS = 32 * WARPS;
 
-struct Smem {
-    float x[WARPS][CT][SLICE];      // 81,920 bytes
-    float c[WARPS][CT][2];          // c_t and c_t - 1
+struct WarpSmem {
+    float x[SUB][SLICE];            // 10,240 bytes
+    float2 cd[SUB];                 // (c * alpha, diagonal term of F) per token
 };
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
@@ -68,7 +68,6 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// acc += A B in split precision for one (k-tile, n-tile) pair.
 __device__ __forceinline__ void mma_3xtf32(float (&acc)[4], const uint32_t (&ah)[4], const uint32_t (&al)[4],
                                            const uint32_t (&bh)[2], const uint32_t (&bl)[2])
 {
@@ -77,11 +76,12 @@ __device__ __forceinline__ void mma_3xtf32(float (&acc)[4], const uint32_t (&ah)
     mma_tf32(acc, ah, bh);
 }
 
-// log|det(W)| of one 16 x 16 matrix held by a group of 4 lanes (lane r of
-// the group owns rows r, r+4, r+8, r+12 in e[0..3][0..15]).  near_identity:
-// W = I + e, eliminated on e alone without pivoting; returns false (and
-// nothing useful) when a pivot |1 + delta_k| < 0.5.  Otherwise W = e with
-// partial pivoting.  The determinant magnitude is accumulated in fp64.
+// log|det(W)| of one 16 x 16 matrix held by a group of 4 lanes (lane r owns
+// rows r, r+4, r+8, r+12 in e[0..3][0..15]).  near_identity: W = I + e,
+// eliminated on e alone without pivoting, |det| = prod |1 + delta_k| in fp64;
+// returns false when a pivot |1 + delta_k| < 0.5.  Otherwise W = e with
+// partial pivoting, log|det| summed in fp64.  Every lane of the warp must
+// call it with the same near_identity (the shuffles span the warp).
 __device__ __forceinline__ bool group_logabsdet(float (&e)[4][N], int r, bool near_identity, double& logabs,
                                                 bool& singular)
 {
@@ -94,7 +94,6 @@ __device__ __forceinline__ bool group_logabsdet(float (&e)[4][N], int r, bool ne
     for (int k = 0; k < N; ++k) {
         const int kr = k >> 2, owner = k & 3;
         if (!near_identity) {
-            // partial pivoting: largest |W[i][k]| over rows i >= k of the group
             float best = -1.0f;
             int bi = k;
 #pragma unroll
@@ -110,41 +109,29 @@ __device__ __forceinline__ bool group_logabsdet(float (&e)[4][N], int r, bool ne
                 if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
             }
             if (!(best > 0.0f)) singular = true;
-            {
-                // swap rows k and bi (row i lives in lane i & 3, slot i >> 2);
-                // executed unconditionally (a no-op when bi == k) so that the
-                // shuffles stay converged across the warp
-                const int pr = bi >> 2, powner = bi & 3;
+            // swap rows k and bi (row i lives in lane i & 3, slot i >> 2);
+            // unconditional (a no-op when bi == k) to keep the warp converged
+            const int pr = bi >> 2, powner = bi & 3;
 #pragma unroll
-                for (int j = 0; j < N; ++j) {
-                    float vk = 0.0f, vp = 0.0f;
+            for (int j = 0; j < N; ++j) {
+                float vk = 0.0f, vp = 0.0f;
 #pragma unroll
-                    for (int lr = 0; lr < 4; ++lr) {
-                        if (lr == kr) vk = e[lr][j];
-                        if (lr == pr) vp = e[lr][j];
-                    }
-                    const float rowk = __shfl_sync(full, vk, owner, 4);
-                    const float rowp = __shfl_sync(full, vp, powner, 4);
+                for (int lr = 0; lr < 4; ++lr) {
+                    if (lr == kr) vk = e[lr][j];
+                    if (lr == pr) vp = e[lr][j];
+                }
+                const float rowk = __shfl_sync(full, vk, owner, 4);
+                const float rowp = __shfl_sync(full, vp, powner, 4);
 #pragma unroll
-                    for (int lr = 0; lr < 4; ++lr) {
-                        if (lr == kr && r == owner) e[lr][j] = rowp;
-                        if (lr == pr && r == powner) e[lr][j] = rowk;
-                    }
+                for (int lr = 0; lr < 4; ++lr) {
+                    if (lr == kr && r == owner) e[lr][j] = rowp;
+                    if (lr == pr && r == powner) e[lr][j] = rowk;
                 }
             }
         }
-        // broadcast pivot row k from its owner lane
         float prow[N];
 #pragma unroll
-        for (int j = 0; j < N; ++j) {
-            if (j >= k) {
-                float v = 0.0f;
-#pragma unroll
-                for (int lr = 0; lr < 4; ++lr)
-                    if (lr == kr) v = e[lr][j];
-                prow[j] = __shfl_sync(full, v, owner, 4);
-            }
-        }
+        for (int j = k; j < N; ++j) prow[j] = __shfl_sync(full, e[kr][j], owner, 4);
         float pk;
         if (near_identity) {
             const float d = prow[k];
@@ -155,15 +142,15 @@ __device__ __forceinline__ bool group_logabsdet(float (&e)[4][N], int r, bool ne
             pk = prow[k];
             lsum += log(fabs((double)pk));
         }
-        const float rk = (pk != 0.0f) ? 1.0f / pk : 0.0f;
+        const float rk = (pk != 0.0f) ? __frcp_rn(pk) : 0.0f;
 #pragma unroll
         for (int lr = 0; lr < 4; ++lr) {
+            if (4 * lr + 3 <= k) continue;        // no row of this slot is below k
             const int i = 4 * lr + r;
             if (i > k) {
                 const float l = e[lr][k] * rk;
 #pragma unroll
-                for (int j = 0; j < N; ++j)
-                    if (j > k) e[lr][j] = fmaf(-l, prow[j], e[lr][j]);
+                for (int j = k + 1; j < N; ++j) e[lr][j] = fmaf(-l, prow[j], e[lr][j]);
             }
         }
     }
@@ -171,253 +158,346 @@ __device__ __forceinline__ bool group_logabsdet(float (&e)[4][N], int r, bool ne
     return ok;
 }
 
-__global__ void __launch_bounds__(THREADS, 2)
-k16_chunk(KParams p, const float* __restrict__ x, float* __restrict__ S_out, float* __restrict__ totals,
-          uint32_t* status)
+// Copies the slices of tokens [t0, t0 + nt) of one (b, h) into the warp's
+// shared memory (16-byte granules, rows padded to ROWW words).
+__device__ __forceinline__ void load_pass(WarpSmem& ws, const float* xb, int64_t tok, int64_t t0, int nt, int lane)
 {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t nchains = p.B * p.H * p.K;
-    const int64_t chain0 = (int64_t)blockIdx.x * WARPS;
-
-    // chain id -> (b, k, h), h fastest, so that a CTA's chains are the heads of
-    // one token range: their slices are contiguous in memory.
-    auto decode = [&](int64_t chain, int64_t& b, int64_t& k, int64_t& h) {
-        h = chain % p.H;
-        const int64_t bk = chain / p.H;
-        k = bk % p.K;
-        b = bk / p.K;
-    };
-
-    // ---- phase 1a: copy the CTA's slices into shared memory ----------------
-    for (int g = tid; g < WARPS * CT * 64; g += THREADS) {
-        const int w = g / (CT * 64), j = (g / 64) % CT, q16 = g % 64;
-        const int64_t chain = chain0 + w;
-        if (chain >= nchains) continue;
-        int64_t b, k, h;
-        decode(chain, b, k, h);
-        const int64_t t = k * CT + j;
-        if (t >= p.L) continue;
-        const int row = q16 >> 2, col4 = q16 & 3;
-        const float* src = x + (((b * p.L + t) * p.H + h) * NN) + row * N + col4 * 4;
-        cp_async16(&sm.x[w][j][row * ROWW + col4 * 4], src);
+#pragma unroll
+    for (int i = 0; i < SUB * 64 / 32; ++i) {
+        const int gi = lane + 32 * i;
+        const int j = gi >> 6, q16 = gi & 63, row = q16 >> 2, col4 = q16 & 3;
+        if (j < nt) cp_async16(&ws.x[j][row * ROWW + col4 * 4], xb + (t0 + j) * tok + row * N + col4 * 4);
     }
     cp_async_wait_all();
-    __syncthreads();
+    __syncwarp();
+}
 
-    // ---- phase 1b: per-token scalars (determinant scale) -------------------
-    {
-        const int grp = tid >> 2, r = tid & 3;       // 64 groups of 4 lanes
-        const int w = grp / CT, j = grp % CT;
-        const int64_t chain = chain0 + w;
-        bool live = chain < nchains;
-        int64_t b = 0, k = 0, h = 0;
-        if (live) {
-            decode(chain, b, k, h);
-            live = k * CT + j < p.L;
+// The per-token scalars of F = ca * M + dv * I for the 8 tokens of a pass:
+// 4-lane LU groups for the determinant-corrected mode.  Lane r == 0 of each
+// group writes ws.cd[group].
+__device__ __forceinline__ void pass_scalars(const KParams& p, WarpSmem& ws, int nt, int lane, uint32_t* status)
+{
+    const int grp = lane >> 2, r = lane & 3;
+    const bool live = grp < nt;
+    float ca = p.alpha, dv = p.add_identity ? 0.0f : -1.0f;
+    if (p.mode == MRU_MODE_DETNORM) {
+        float e[4][N];
+        const float* xs = ws.x[grp];
+#pragma unroll
+        for (int lr = 0; lr < 4; ++lr) {
+            const float4* row4 = reinterpret_cast<const float4*>(xs + (4 * lr + r) * ROWW);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const float4 v = live ? row4[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+                e[lr][4 * c4 + 0] = p.alpha * v.x;
+                e[lr][4 * c4 + 1] = p.alpha * v.y;
+                e[lr][4 * c4 + 2] = p.alpha * v.z;
+                e[lr][4 * c4 + 3] = p.alpha * v.w;
+            }
         }
-        float c = 1.0f, cm1 = 0.0f;
-        if (p.mode == MRU_MODE_DETNORM) {
-            float e[4][N];
-            const float* xs = sm.x[w][j];
+        double ld = 0.0;
+        bool singular = false, ok = true;
+        if (p.add_identity) ok = group_logabsdet(e, r, true, ld, singular);
+        if (__any_sync(0xffffffffu, !p.add_identity || !ok)) {
+            const bool need = !p.add_identity || !ok;
 #pragma unroll
             for (int lr = 0; lr < 4; ++lr) {
                 const int i = 4 * lr + r;
 #pragma unroll
-                for (int jj = 0; jj < N; ++jj) e[lr][jj] = live ? p.alpha * xs[i * ROWW + jj] : 0.0f;
+                for (int jj = 0; jj < N; ++jj)
+                    e[lr][jj] = live ? p.alpha * xs[i * ROWW + jj] + ((p.add_identity && i == jj) ? 1.0f : 0.0f)
+                                     : (i == jj ? 1.0f : 0.0f);
             }
-            double ld = 0.0;
-            bool singular = false;
-            bool ok = true;
-            if (p.add_identity) ok = group_logabsdet(e, r, true, ld, singular);
-            // every group of the warp must agree before the pivoted retry, as
-            // the shuffles inside span the whole warp
-            const bool retry = __any_sync(0xffffffffu, !p.add_identity || !ok);
-            if (retry) {
-                const bool need = !p.add_identity || !ok;
-#pragma unroll
-                for (int lr = 0; lr < 4; ++lr) {
-                    const int i = 4 * lr + r;
-#pragma unroll
-                    for (int jj = 0; jj < N; ++jj)
-                        e[lr][jj] = live ? p.alpha * xs[i * ROWW + jj] + ((p.add_identity && i == jj) ? 1.0f : 0.0f)
-                                         : (i == jj ? 1.0f : 0.0f);
-                }
-                double ld2 = 0.0;
-                bool sing2 = false;
-                group_logabsdet(e, r, false, ld2, sing2);
-                if (need) { ld = ld2; singular = sing2; }
-            }
-            const double cm1d = expm1(-ld / N);
-            c = (float)(1.0 + cm1d);
-            cm1 = (float)cm1d;
-            if (live && (singular || !isfinite(ld) || !isfinite(c) || c == 0.0f)) {
-                if (r == 0) atomicOr(status, STATUS_SINGULAR);
-                c = 0.0f;
-                cm1 = 0.0f;
-            }
+            double ld2 = 0.0;
+            bool sing2 = false;
+            group_logabsdet(e, r, false, ld2, sing2);
+            if (need) { ld = ld2; singular = sing2; }
         }
-        if (r == 0) {
-            sm.c[w][j][0] = c;
-            sm.c[w][j][1] = cm1;
+        const double cm1d = expm1(-ld / N);
+        const float c = (float)(1.0 + cm1d);
+        if (singular || !isfinite(ld) || !isfinite(c) || c == 0.0f) {
+            if (live && r == 0) atomicOr(status, STATUS_SINGULAR);
+            ca = 0.0f;                       // output unspecified; keep X = I
+            dv = 0.0f;
+        } else {
+            ca = c * p.alpha;
+            dv = p.add_identity ? (float)cm1d : -1.0f;
         }
     }
-    __syncthreads();
+    if (r == 0) ws.cd[grp] = make_float2(ca, dv);
+    __syncwarp();
+}
 
-    // ---- phase 2: the chain of warp `warp` ---------------------------------
-    const int64_t chain = chain0 + warp;
-    if (chain >= nchains) return;
-    int64_t b, k, h;
-    decode(chain, b, k, h);
+// B fragments (split) of F = ca * M + dv * I for one token, with the
+// contraction index permuted (slot q <-> row 8kt + 2q, slot q + 4 <-> row
+// 8kt + 2q + 1), and F at this lane's accumulator positions.
+struct FragF {
+    uint32_t bh[2][2][2], bl[2][2][2];
+    float fd[2][4];
+};
+
+__device__ __forceinline__ void make_frag_f(const float* xs, float ca, float d0, float d1, int g, int q, FragF& f,
+                                            bool want_fd)
+{
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const float* base = xs + (8 * kt + 2 * q) * ROWW + 8 * nt + g;
+            const float v0 = fmaf(ca, base[0], kt == nt ? d0 : 0.0f);
+            const float v1 = fmaf(ca, base[ROWW], kt == nt ? d1 : 0.0f);
+            split_tf32(v0, f.bh[kt][nt][0], f.bl[kt][nt][0]);
+            split_tf32(v1, f.bh[kt][nt][1], f.bl[kt][nt][1]);
+        }
+    if (want_fd) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+                const float2 xv = *reinterpret_cast<const float2*>(xs + (g + 8 * h8) * ROWW + 8 * nt + 2 * q);
+                f.fd[nt][2 * h8 + 0] = fmaf(ca, xv.x, h8 == nt ? d0 : 0.0f);
+                f.fd[nt][2 * h8 + 1] = fmaf(ca, xv.y, h8 == nt ? d1 : 0.0f);
+            }
+    }
+}
+
+// acc = A F with A the 16 x 16 state held in accumulator layout (Ad).
+__device__ __forceinline__ void chain_product(const float (&Ad)[2][4], const FragF& f, float (&acc)[2][4])
+{
+    uint32_t ah[2][4], al[2][4];
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt) {
+        split_tf32(Ad[kt][0], ah[kt][0], al[kt][0]);
+        split_tf32(Ad[kt][2], ah[kt][1], al[kt][1]);
+        split_tf32(Ad[kt][1], ah[kt][2], al[kt][2]);
+        split_tf32(Ad[kt][3], ah[kt][3], al[kt][3]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+#pragma unroll
+        for (int kt = 0; kt < 2; ++kt) mma_3xtf32(acc[nt], ah[kt], al[kt], f.bh[kt][nt], f.bl[kt][nt]);
+    }
+}
+
+__device__ __forceinline__ void store_d(float* out, const float (&Ad)[2][4], int g, int q)
+{
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8)
+            *reinterpret_cast<float2*>(out + (g + 8 * h8) * N + 8 * nt + 2 * q) =
+                make_float2(Ad[nt][2 * h8], Ad[nt][2 * h8 + 1]);
+}
+
+// chain id -> (b, k, h), h fastest: a CTA's chains are neighbouring heads of
+// one token range (their slices are contiguous in memory).
+struct ChainIx {
+    int64_t b, h, k, tbeg, tend;
+};
+__device__ __forceinline__ ChainIx chain_ix(const KParams& p, int64_t chain)
+{
+    ChainIx c;
+    c.h = chain % p.H;
+    const int64_t bk = chain / p.H;
+    c.k = bk % p.K;
+    c.b = bk / p.K;
+    c.tbeg = c.k * p.chunk;
+    c.tend = (c.tbeg + p.chunk < p.L) ? c.tbeg + p.chunk : p.L;
+    return c;
+}
+
+// ---- chain bodies, shared by the two-pass kernels and the fused kernel ----
+
+// The reduce chain of one warp over tokens [tbeg, tend): per-token scalars to
+// cdb[t * H] and the chunk total (split form) left in Qd.
+__device__ __forceinline__ void reduce_chain(const KParams& p, WarpSmem& ws, const float* xb, int64_t tok,
+                                             float2* cdb, int64_t tbeg, int64_t tend, int lane, uint32_t* status,
+                                             float (&Qd)[2][4])
+{
     const int g = lane >> 2, q = lane & 3;
-    float Qd[2][4];                                  // accumulator layout, 2 column tiles
+    const float m0 = (g == 2 * q) ? 1.0f : 0.0f;         // diagonal positions of this lane's fragments
+    const float m1 = (g == 2 * q + 1) ? 1.0f : 0.0f;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) Qd[nt][i] = 0.0f;
-
-    const float dconst = p.add_identity ? 0.0f : -1.0f;   // diagonal of F besides c-1
-    for (int j = 0; j < CT; ++j) {
-        const int64_t t = k * CT + j;
-        if (t >= p.L) break;
-        const float* xs = sm.x[warp][j];
-        const float c = sm.c[warp][j][0];
-        const float ca = c * p.alpha;
-        const float dval = p.add_identity ? sm.c[warp][j][1] : dconst;
-        auto F = [&](int rr, int cc) {
-            const float v = ca * xs[rr * ROWW + cc];
-            return (c == 0.0f) ? 0.0f : (rr == cc ? v + dval : v);
-        };
-        // B fragments of F with the permuted contraction index:
-        // slot q <-> logical row 8kt + 2q, slot q + 4 <-> 8kt + 2q + 1.
-        uint32_t bh[2][2][2], bl[2][2][2];
+    for (int64_t t0 = tbeg; t0 < tend; t0 += SUB) {
+        const int nt_pass = (tend - t0 < SUB) ? (int)(tend - t0) : SUB;
+        load_pass(ws, xb, tok, t0, nt_pass, lane);
+        pass_scalars(p, ws, nt_pass, lane, status);
+        if (lane < nt_pass) cdb[(t0 + lane) * p.H] = ws.cd[lane];
+        for (int j = 0; j < nt_pass; ++j) {
+            const float2 cdj = ws.cd[j];
+            FragF f;
+            make_frag_f(ws.x[j], cdj.x, m0 * cdj.y, m1 * cdj.y, g, q, f, true);
+            float acc[2][4];
+            chain_product(Qd, f, acc);
 #pragma unroll
-        for (int kt = 0; kt < 2; ++kt)
+            for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                split_tf32(F(8 * kt + 2 * q, 8 * nt + g), bh[kt][nt][0], bl[kt][nt][0]);
-                split_tf32(F(8 * kt + 2 * q + 1, 8 * nt + g), bh[kt][nt][1], bl[kt][nt][1]);
-            }
-        // A fragments straight from the state registers
-        uint32_t ah[2][4], al[2][4];
-#pragma unroll
-        for (int kt = 0; kt < 2; ++kt) {
-            split_tf32(Qd[kt][0], ah[kt][0], al[kt][0]);
-            split_tf32(Qd[kt][2], ah[kt][1], al[kt][1]);
-            split_tf32(Qd[kt][1], ah[kt][2], al[kt][2]);
-            split_tf32(Qd[kt][3], ah[kt][3], al[kt][3]);
+                for (int i = 0; i < 4; ++i) Qd[nt][i] += f.fd[nt][i] + acc[nt][i];
         }
-        float acc[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
-#pragma unroll
-            for (int kt = 0; kt < 2; ++kt) mma_3xtf32(acc[nt], ah[kt], al[kt], bh[kt][nt], bl[kt][nt]);
-        }
-        float* out = S_out + (((b * p.L + t) * p.H + h) * NN);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int c0 = 8 * nt + 2 * q;
-            Qd[nt][0] += F(g, c0) + acc[nt][0];
-            Qd[nt][1] += F(g, c0 + 1) + acc[nt][1];
-            Qd[nt][2] += F(g + 8, c0) + acc[nt][2];
-            Qd[nt][3] += F(g + 8, c0 + 1) + acc[nt][3];
-            *reinterpret_cast<float2*>(out + g * N + c0) = make_float2(Qd[nt][0], Qd[nt][1]);
-            *reinterpret_cast<float2*>(out + (g + 8) * N + c0) = make_float2(Qd[nt][2], Qd[nt][3]);
-        }
-    }
-    // chunk total, indexed (b*H + h)*K + k like the generic path
-    float* tot = totals + ((b * p.H + h) * p.K + k) * NN;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        const int c0 = 8 * nt + 2 * q;
-        *reinterpret_cast<float2*>(tot + g * N + c0) = make_float2(Qd[nt][0], Qd[nt][1]);
-        *reinterpret_cast<float2*>(tot + (g + 8) * N + c0) = make_float2(Qd[nt][2], Qd[nt][3]);
+        __syncwarp();
     }
 }
 
-// S_t = C + C Q_t in place, one warp per chain.
-__global__ void __launch_bounds__(THREADS)
-k16_fixup(KParams p, const float* __restrict__ carry, float* __restrict__ S_out)
+// The chain's carry C = E (I + R) in fp64 (R may be null: C = E), rounded to
+// fp32, into accumulator layout Sd.  Uses the warp's x buffer as scratch.
+__device__ __forceinline__ void form_carry(WarpSmem& ws, const double* E, const float* R, int lane,
+                                           float (&Sd)[2][4])
 {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t nchains = p.B * p.H * p.K;
-    const int64_t chain = (int64_t)blockIdx.x * WARPS + warp;
-    if (chain >= nchains) return;
-    const int64_t h = chain % p.H, bk = chain / p.H, k = bk % p.K, b = bk / p.K;
-    const int g = lane >> 2, q = lane & 3;
-    const float* C = carry + ((b * p.H + h) * p.K + k) * NN;
-    uint32_t ah[2][4], al[2][4];
+    double* sE = reinterpret_cast<double*>(&ws.x[0][0]);      // 2 KB
+    float* sC = reinterpret_cast<float*>(&ws.x[2][0]);        // 1 KB
+    for (int e = lane; e < NN; e += 32) sE[e] = E[e];
+    __syncwarp();
+    const int r0 = (lane >> 2) * 2, c0 = (lane & 3) * 4;
+    double acc[2][4];
 #pragma unroll
-    for (int kt = 0; kt < 2; ++kt) {
-        split_tf32(C[g * N + 8 * kt + q], ah[kt][0], al[kt][0]);
-        split_tf32(C[(g + 8) * N + 8 * kt + q], ah[kt][1], al[kt][1]);
-        split_tf32(C[g * N + 8 * kt + q + 4], ah[kt][2], al[kt][2]);
-        split_tf32(C[(g + 8) * N + 8 * kt + q + 4], ah[kt][3], al[kt][3]);
-    }
-    float Cd[2][4];
+    for (int i = 0; i < 2; ++i)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        const int c0 = 8 * nt + 2 * q;
-        Cd[nt][0] = C[g * N + c0];
-        Cd[nt][1] = C[g * N + c0 + 1];
-        Cd[nt][2] = C[(g + 8) * N + c0];
-        Cd[nt][3] = C[(g + 8) * N + c0 + 1];
-    }
-    for (int j = 0; j < CT; ++j) {
-        const int64_t t = k * CT + j;
-        if (t >= p.L) break;
-        float* Sq = S_out + (((b * p.L + t) * p.H + h) * NN);
-        uint32_t bh[2][2][2], bl[2][2][2];
+        for (int cc = 0; cc < 4; ++cc) acc[i][cc] = 0.0;
+    if (R) {
+#pragma unroll 4
+        for (int kk = 0; kk < N; ++kk) {
+            const double a0 = sE[r0 * N + kk], a1 = sE[(r0 + 1) * N + kk];
+            const float4 rv = *reinterpret_cast<const float4*>(R + kk * N + c0);
+            const double bv[4] = {(double)rv.x, (double)rv.y, (double)rv.z, (double)rv.w};
 #pragma unroll
-        for (int kt = 0; kt < 2; ++kt)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                split_tf32(Sq[(8 * kt + q) * N + 8 * nt + g], bh[kt][nt][0], bl[kt][nt][0]);
-                split_tf32(Sq[(8 * kt + q + 4) * N + 8 * nt + g], bh[kt][nt][1], bl[kt][nt][1]);
+            for (int cc = 0; cc < 4; ++cc) {
+                acc[0][cc] = fma(a0, bv[cc], acc[0][cc]);
+                acc[1][cc] = fma(a1, bv[cc], acc[1][cc]);
             }
-        __syncwarp();
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-            for (int kt = 0; kt < 2; ++kt) mma_3xtf32(acc, ah[kt], al[kt], bh[kt][nt], bl[kt][nt]);
-            const int c0 = 8 * nt + 2 * q;
-            *reinterpret_cast<float2*>(Sq + g * N + c0) = make_float2(Cd[nt][0] + acc[0], Cd[nt][1] + acc[1]);
-            *reinterpret_cast<float2*>(Sq + (g + 8) * N + c0) = make_float2(Cd[nt][2] + acc[2], Cd[nt][3] + acc[3]);
         }
     }
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+            sC[(r0 + i) * N + c0 + cc] = (float)(sE[(r0 + i) * N + c0 + cc] + acc[i][cc]);
+    __syncwarp();
+    const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+            const float2 v = *reinterpret_cast<const float2*>(sC + (g + 8 * h8) * N + 8 * nt + 2 * q);
+            Sd[nt][2 * h8] = v.x;
+            Sd[nt][2 * h8 + 1] = v.y;
+        }
+    __syncwarp();
+}
+
+// The apply chain of one warp: S_t = S_{t-1} + S_{t-1} F_t from Sd, every
+// S_t written to ob + t * tok.
+__device__ __forceinline__ void apply_chain(WarpSmem& ws, const float* xb, float* ob, int64_t tok, int64_t H,
+                                            const float2* cdb, int64_t tbeg, int64_t tend, int lane,
+                                            float (&Sd)[2][4])
+{
+    const int g = lane >> 2, q = lane & 3;
+    const float m0 = (g == 2 * q) ? 1.0f : 0.0f;
+    const float m1 = (g == 2 * q + 1) ? 1.0f : 0.0f;
+    for (int64_t t0 = tbeg; t0 < tend; t0 += SUB) {
+        const int nt_pass = (tend - t0 < SUB) ? (int)(tend - t0) : SUB;
+        load_pass(ws, xb, tok, t0, nt_pass, lane);
+        for (int j = 0; j < nt_pass; ++j) {
+            const float2 cdj = cdb[(t0 + j) * H];
+            FragF f;
+            make_frag_f(ws.x[j], cdj.x, m0 * cdj.y, m1 * cdj.y, g, q, f, false);
+            float acc[2][4];
+            chain_product(Sd, f, acc);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) Sd[nt][i] += acc[nt][i];
+            store_d(ob + (t0 + j) * tok, Sd, g, q);
+        }
+        __syncwarp();
+    }
+}
+
+// Reduce pass: chunk totals (split form) and per-token scalars.
+__global__ void __launch_bounds__(THREADS, 2)
+k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, float2* __restrict__ cd_out,
+           uint32_t* status)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    WarpSmem& ws = reinterpret_cast<WarpSmem*>(smem_raw)[warp];
+    const int64_t chain = (int64_t)blockIdx.x * WARPS + warp;
+    if (chain >= p.B * p.H * p.K) return;
+    const ChainIx c = chain_ix(p, chain);
+    const int64_t tok = p.H * NN;
+    const float* xb = x + (c.b * p.L * p.H + c.h) * NN;
+    float2* cdb = cd_out + c.b * p.L * p.H + c.h;
+    float Qd[2][4];
+    reduce_chain(p, ws, xb, tok, cdb, c.tbeg, c.tend, lane, status, Qd);
+    store_d(totals + ((c.b * p.H + c.h) * p.K + c.k) * NN, Qd, lane >> 2, lane & 3);
+}
+
+// Apply pass: the chunk's carry C = E1 (I + R0[k-1]) in fp64, then
+// S_t = S_{t-1} + S_{t-1} F_t from S = C, every S_t written.
+__global__ void __launch_bounds__(THREADS, 2)
+k16_apply(KParams p, const float* __restrict__ x, const float2* __restrict__ cd_in, const float* __restrict__ R0,
+          const double* __restrict__ E1, int G, float* __restrict__ S_out)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    WarpSmem& ws = reinterpret_cast<WarpSmem*>(smem_raw)[warp];
+    const int64_t chain = (int64_t)blockIdx.x * WARPS + warp;
+    if (chain >= p.B * p.H * p.K) return;
+    const ChainIx c = chain_ix(p, chain);
+    const int64_t seq = c.b * p.H + c.h;
+    const int64_t n1 = (p.K + G - 1) / G;
+    float Sd[2][4];
+    form_carry(ws, E1 + (seq * n1 + c.k / G) * NN, (c.k % G) ? R0 + (seq * p.K + c.k - 1) * NN : nullptr, lane, Sd);
+    const int64_t tok = p.H * NN;
+    apply_chain(ws, x + (c.b * p.L * p.H + c.h) * NN, S_out + (c.b * p.L * p.H + c.h) * NN, tok, p.H,
+                cd_in + c.b * p.L * p.H + c.h, c.tbeg, c.tend, lane, Sd);
 }
 
 }  // namespace
 
-int chunk_tokens() { return CT; }
-
 bool supports(const KParams& p, bool readout)
 {
     return p.n == N && p.src == SRC_EMBEDDING && p.x_dtype == MRU_F32 && !readout &&
-           (p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM) && p.chunk == CT;
+           (p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM) &&
+           (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32X3) && p.chunk > 0 && p.chunk % SUB == 0;
 }
 
-cudaError_t launch_chunk(const KParams& p, const float* x, float* S_out, float* totals, uint32_t* status,
-                         cudaStream_t s)
+// Chunk length: 8 tokens per pass, m passes per chain, m a power of two that
+// keeps at least 16384 chains (about 7 waves of 16 warps per SM) when the
+// workload allows, so that long sequences get long chunks (few chunk totals).
+int32_t preferred_chunk(int64_t token_heads)
+{
+    int32_t m = 1;
+    while (m < 16 && token_heads / ((int64_t)SUB * 2 * m) >= 16384) m *= 2;
+    return SUB * m;
+}
+
+cudaError_t launch_reduce(const KParams& p, const float* x, float* totals, float2* cd, uint32_t* status,
+                          cudaStream_t s)
 {
     const int64_t nchains = p.B * p.H * p.K;
     const unsigned grid = (unsigned)((nchains + WARPS - 1) / WARPS);
-    const size_t sm = sizeof(Smem);
-    cudaError_t e = cudaFuncSetAttribute(k16_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    const size_t sm = sizeof(WarpSmem) * WARPS;
+    cudaError_t e = cudaFuncSetAttribute(k16_reduce, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    k16_chunk<<<grid, THREADS, sm, s>>>(p, x, S_out, totals, status);
+    k16_reduce<<<grid, THREADS, sm, s>>>(p, x, totals, cd, status);
     return cudaGetLastError();
 }
 
-cudaError_t launch_fixup(const KParams& p, const float* carry, float* S_out, cudaStream_t s)
+cudaError_t launch_apply(const KParams& p, const float* x, const float2* cd, const carry::Plan& pl,
+                         const char* ws, float* S_out, cudaStream_t s)
 {
     const int64_t nchains = p.B * p.H * p.K;
     const unsigned grid = (unsigned)((nchains + WARPS - 1) / WARPS);
-    k16_fixup<<<grid, THREADS, 0, s>>>(p, carry, S_out);
+    const size_t sm = sizeof(WarpSmem) * WARPS;
+    cudaError_t e = cudaFuncSetAttribute(k16_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    k16_apply<<<grid, THREADS, sm, s>>>(p, x, cd, reinterpret_cast<const float*>(ws + pl.R[0]),
+                                        reinterpret_cast<const double*>(ws + pl.E[1]), pl.G, S_out);
     return cudaGetLastError();
 }
 

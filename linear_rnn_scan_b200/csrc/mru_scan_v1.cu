@@ -578,34 +578,21 @@ cudaError_t scan_n(const KParams& p, const void* src, const float* S0, const flo
 cudaError_t scan_fast16(const KParams& p, const void* src, const float* S0, float* S_out, char* ws,
                         const Workspace& W, cudaStream_t s, int* launches)
 {
-    constexpr int N = 16, NN = N * N;
     uint32_t* status = reinterpret_cast<uint32_t*>(ws + W.status);
     float* totals = reinterpret_cast<float*>(ws + W.totals);
-    double* local = reinterpret_cast<double*>(ws + W.local);
-    double* gcarry = reinterpret_cast<double*>(ws + W.gcarry);
-    float* carry = reinterpret_cast<float*>(ws + W.carry);
-    const int64_t BH = p.B * p.H;
-    const int64_t chains = BH * p.K;
-    if (chains == 0) return cudaSuccess;
+    float2* cd = reinterpret_cast<float2*>(ws + W.cd);
+    const float* x = reinterpret_cast<const float*>(src);
+    if (p.B * p.H * p.K == 0) return cudaSuccess;
     cudaError_t e;
-    const size_t sm_d = sizeof(double) * 2 * NN;
-    profile_mark(0, 0, s);
-    if ((e = n16::launch_chunk(p, reinterpret_cast<const float*>(src), S_out, totals, status, s)) != cudaSuccess)
-        return e;
-    profile_mark(0, 1, s);
-    profile_mark(1, 0, s);
-    k_carry_local<N><<<(unsigned)(BH * p.NG), kThreads, sm_d, s>>>(p, totals, local);
-    profile_mark(1, 1, s);
-    profile_mark(2, 0, s);
-    k_carry_groups<N><<<(unsigned)BH, kThreads, sm_d, s>>>(p, S0, local, gcarry);
-    profile_mark(2, 1, s);
-    profile_mark(3, 0, s);
-    k_carry_final<N><<<(unsigned)chains, kThreads, sm_d, s>>>(p, local, gcarry, carry);
-    profile_mark(3, 1, s);
-    profile_mark(4, 0, s);
-    if ((e = n16::launch_fixup(p, carry, S_out, s)) != cudaSuccess) return e;
-    profile_mark(4, 1, s);
-    if (launches) *launches = 5;
+    int slot = 0;
+    profile_mark(slot, 0, s);
+    if ((e = n16::launch_reduce(p, x, totals, cd, status, s)) != cudaSuccess) return e;
+    profile_mark(slot++, 1, s);
+    if ((e = carry::run_n16(W.plan, totals, S0, ws, s, slot)) != cudaSuccess) return e;
+    profile_mark(slot, 0, s);
+    if ((e = n16::launch_apply(p, x, cd, W.plan, ws, S_out, s)) != cudaSuccess) return e;
+    profile_mark(slot++, 1, s);
+    if (launches) *launches = slot;
     return cudaGetLastError();
 }
 
@@ -613,12 +600,12 @@ cudaError_t scan_fast16(const KParams& p, const void* src, const float* S0, floa
 
 const char* kernel_name(const KParams& p, bool readout, int i)
 {
+    (void)p;
+    (void)readout;
     static const char* generic[] = {"k_chunk_prefix", "k_carry_local", "k_carry_groups", "k_carry_final",
                                     "k_fixup"};
-    static const char* fast16[] = {"k16_chunk", "k_carry_local", "k_carry_groups", "k_carry_final",
-                                   "k16_fixup"};
     if (i < 0 || i >= 5) return "";
-    return n16::supports(p, readout) ? fast16[i] : generic[i];
+    return generic[i];
 }
 
 cudaError_t launch_build_states(const KParams& p, const void* x, float* X_out, int store_minus_identity,
@@ -640,8 +627,7 @@ cudaError_t launch_scan(const KParams& p, const void* src, const float* S0, cons
                         void* ws_base, const Workspace& W, cudaStream_t s, int* launches)
 {
     char* ws = reinterpret_cast<char*>(ws_base);
-    if (n16::supports(p, o_out != nullptr))
-        return scan_fast16(p, src, S0, S_out, ws, W, s, launches);
+    if (W.fast) return scan_fast16(p, src, S0, S_out, ws, W, s, launches);
     switch (p.n) {
         case 4: return scan_n<4>(p, src, S0, u, snap_every, S_out, o_out, snaps, ws, W, s, launches);
         case 8: return scan_n<8>(p, src, S0, u, snap_every, S_out, o_out, snaps, ws, W, s, launches);

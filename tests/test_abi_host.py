@@ -61,7 +61,7 @@ def test_workspace_size(lib):
     C = mru.chosen_chunk(p)
     assert C >= 1 and (C & (C - 1)) == 0
     K = -(-w.L // C)
-    assert ws >= 256 + w.B * w.H * K * 256 * (4 + 8 + 4)
+    assert ws >= 256 + w.B * w.H * K * 256 * 4          # at least the fp32 chunk totals
     for n in (4, 8, 16, 32, 64):
         assert mru.workspace_size(mru.problem(1, 1, 7, n)) >= 256
     assert mru.workspace_size(mru.problem(1, 1, 7, 12)) == 0          # unsupported n
