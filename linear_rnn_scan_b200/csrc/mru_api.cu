@@ -1,12 +1,25 @@
 // mru_api.cu -- the extern "C" boundary of libmru: argument checks, workspace
 // layout, kernel selection and launch.  No allocation happens here: every
 // buffer, the workspace included, belongs to the caller.
+#include <stdlib.h>
 #include <string.h>
 
 #include "mru_internal.cuh"
 
 namespace mru {
 namespace {
+
+// The two-pass n = 16 kernels are the default; MRU_N16_FUSED=1 in the
+// environment selects the fused persistent kernel instead (experimental: it
+// is correct but its per-window scans still serialise the windows).
+bool fused_enabled()
+{
+    static const bool on = [] {
+        const char* v = getenv("MRU_N16_FUSED");
+        return v && v[0] == '1';
+    }();
+    return on;
+}
 
 bool supported_n(int n) { return n == 4 || n == 8 || n == 16 || n == 32 || n == 64; }
 
@@ -37,7 +50,8 @@ bool fast16_eligible(const mru_problem& p, bool readout)
 int32_t choose_chunk(const mru_problem& p, int32_t src, bool readout)
 {
     if (p.chunk > 0) return p.chunk;
-    if (src == SRC_EMBEDDING && fast16_eligible(p, readout)) return n16::preferred_chunk(p.B * p.H * p.L);
+    if (src == SRC_EMBEDDING && fast16_eligible(p, readout))
+        return fused_enabled() ? 16 : n16::preferred_chunk(p.B * p.H * p.L);
     return generic_chunk(p);
 }
 
@@ -84,6 +98,13 @@ Workspace layout(const KParams& k, bool readout)
     const size_t BH = (size_t)(k.B * k.H);
     size_t off = 0;
     W.status = off; off += 256;
+    if (n16::supports(k, readout) && k.chunk == 16 && fused_enabled()) {
+        W.fast = true;
+        W.fused = true;
+        W.fl = n16::fused_layout(k, off);
+        W.bytes = W.fl.end;
+        return W;
+    }
     if (n16::supports(k, readout)) {
         W.fast = true;
         W.totals = off; off = round_up(off + BH * k.K * nn * sizeof(float), 256);
@@ -148,6 +169,7 @@ const char* mru_kernel_name(const mru_problem* p, int32_t readout, int32_t i)
     if (check_problem(p) != MRU_OK) return "";
     const KParams k = make_params(*p, SRC_EMBEDDING, readout != 0);
     const Workspace W = layout(k, readout != 0);
+    if (W.fused) return i == 0 ? "k16_fused" : "";
     if (!W.fast) return kernel_name(k, readout != 0, i);
     const int lv = W.plan.levels;
     if (i == 0) return "k16_reduce";
@@ -164,6 +186,7 @@ int32_t mru_launch_count(const mru_problem* p, int32_t readout)
     if (p->B * p->H * p->L == 0) return 0;
     const KParams k = make_params(*p, SRC_EMBEDDING, readout != 0);
     const Workspace W = layout(k, readout != 0);
+    if (W.fused) return 1;
     return W.fast ? 2 + carry::launches(W.plan) : 5;
 }
 

@@ -56,6 +56,16 @@ int launches(const Plan& pl);
 cudaError_t run_n16(const Plan& pl, const float* totals, const float* S0, char* ws, cudaStream_t s, int& slot);
 }  // namespace carry
 
+namespace n16 {
+// The fused persistent kernel: one launch, reduce / carry / apply as a
+// dataflow over L2-sized windows.
+struct FusedLayout {
+    int G, Kw;
+    int64_t NW, NG;
+    size_t counters, counters_bytes, totals, cd, R0, Tot, E1, cstate, end;
+};
+}  // namespace n16
+
 struct Workspace {
     size_t status;       // uint32 status word
     size_t totals;       // float  [B*H, K, n, n]   chunk totals, split form (T - I)
@@ -63,6 +73,8 @@ struct Workspace {
     size_t gcarry;       // double [B*H, NG, n, n]  exclusive group carries (full matrices)
     size_t carry;        // float  [B*H, K, n, n]   exclusive chunk carries (full matrices)
     bool fast;           // specialised kernels: chunk totals, per-token scalars, carry plan
+    bool fused;          // the fused persistent kernel with its own layout below
+    n16::FusedLayout fl;
     size_t cd;           // float2 [B, L, H] per-token scalars (c alpha, diagonal of F)
     carry::Plan plan;
     size_t bytes;        // total
@@ -84,6 +96,9 @@ cudaError_t launch_reduce(const KParams& p, const float* x, float* totals, float
                           cudaStream_t s);
 cudaError_t launch_apply(const KParams& p, const float* x, const float2* cd, const carry::Plan& pl,
                          const char* ws, float* S_out, cudaStream_t s);
+FusedLayout fused_layout(const KParams& p, size_t off);
+cudaError_t launch_fused(const KParams& p, const FusedLayout& L, char* ws, uint32_t* status, const float* x,
+                         const float* S0, float* S_out, cudaStream_t s);
 }  // namespace n16
 
 // Launchers (mru_scan_v1.cu).

@@ -25,6 +25,8 @@
 // Split-tf32 ("3xTF32", after Ootomo and Yokota, 2022): x = hi + lo with hi
 // the top 19 bits of x (sign, exponent, 10 mantissa bits) and lo = x - hi
 // exact in fp32; a b ~ a_lo b_hi + a_hi b_lo + a_hi b_hi.
+#include <string.h>
+
 #include "mru_internal.cuh"
 
 namespace mru {
@@ -457,6 +459,257 @@ k16_apply(KParams p, const float* __restrict__ x, const float2* __restrict__ cd_
                 cd_in + c.b * p.L * p.H + c.h, c.tbeg, c.tend, lane, Sd);
 }
 
+// ---- fused persistent kernel --------------------------------------------
+//
+// One launch runs the whole scan as a dataflow of work items over windows of
+// Kw chunks (all sequences), taken in ticket order from a global counter:
+//     R(0) .. R(lag-1), then per window w:  R(w+lag), S1(w), S2(w), A(w)
+//   R(w)   reduce chains of window w: chunk totals + per-token scalars
+//   S1(w)  per (sequence, group of G chunks): fp64 inclusive local prefixes
+//          R0 (kept fp32) and the group total Tot (fp64)
+//   S2(w)  per sequence: exclusive group carries E1 from the running carry
+//          (fp64), which it hands on to S2(w+1)
+//   A(w)   apply chains of window w from their exact carries, S_t written
+// An item only waits for items with smaller tickets (S1(w) for all R(w),
+// S2(w) for all S1(w) and S2(w-1), A(w) for S2(w)); those are held by CTAs
+// that are running, so the waits end.  Each wait is bounded: past the limit
+// the kernel records STATUS_TIMEOUT, raises the abort flag and returns.
+// Windows are sized so that the embeddings of the lag + 1 windows in flight
+// stay in L2, where the apply pass reads them the second time.
+
+constexpr unsigned kSpinLimit = 4u << 20;     // x up to ~1 us of back-off: a few seconds
+
+struct FusedCfg {
+    int G;              // chunks per group
+    int Kw;             // chunks per window (multiple of G)
+    int lag;            // windows the reduce items run ahead
+    int64_t NW;         // windows
+    int64_t nR, nS1, nS2, nA;
+    int64_t total;      // tickets
+    int64_t NG;         // groups per sequence
+};
+
+struct FusedBufs {
+    unsigned* ticket;
+    unsigned* abort_flag;
+    unsigned* cntR;     // [NW]
+    unsigned* cntS1;    // [NW]
+    unsigned* cntS2;    // [NW]
+    float* totals;      // [seq][K]
+    float2* cd;         // [B][L][H]
+    float* R0;          // [seq][K]
+    double* Tot;        // [seq][NG]
+    double* E1;         // [seq][NG]
+    double* cstate;     // [seq]
+    uint32_t* status;
+};
+
+__device__ __forceinline__ unsigned ld_volatile(const unsigned* p)
+{
+    return *reinterpret_cast<const volatile unsigned*>(p);
+}
+
+// Called by thread 0 only.  True once *ctr >= target; false on timeout or
+// when another CTA has aborted.
+__device__ bool wait_geq(const unsigned* ctr, unsigned target, const FusedBufs& fb)
+{
+    unsigned ns = 32;
+    for (unsigned spins = 0;; ++spins) {
+        if (ld_volatile(ctr) >= target) {
+            __threadfence();
+            return true;
+        }
+        if (ld_volatile(fb.abort_flag)) return false;
+        if (spins >= kSpinLimit) {
+            atomicOr(fb.status, STATUS_TIMEOUT);
+            atomicExch(fb.abort_flag, 1u);
+            return false;
+        }
+        __nanosleep(ns);
+        if (ns < 1024) ns <<= 1;
+    }
+}
+
+// C = A B for 16 x 16 fp64 matrices in shared memory; lane owns a 2 x 4 block.
+__device__ __forceinline__ void warp_gemm16_f64(const double* A, const double* B, int lane, double (&acc)[2][4])
+{
+    const int r0 = (lane >> 2) * 2, c0 = (lane & 3) * 4;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[i][c] = 0.0;
+#pragma unroll 4
+    for (int k = 0; k < N; ++k) {
+        const double a0 = A[r0 * N + k], a1 = A[(r0 + 1) * N + k];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const double b = B[k * N + c0 + c];
+            acc[0][c] = fma(a0, b, acc[0][c]);
+            acc[1][c] = fma(a1, b, acc[1][c]);
+        }
+    }
+}
+
+// chain index inside window w -> global chain coordinates (h fastest, then
+// the chunk within the window, then b); false when outside the problem.
+__device__ __forceinline__ bool window_chain(const KParams& p, const FusedCfg& fc, int64_t w, int64_t ci, ChainIx& c)
+{
+    if (ci >= p.B * (int64_t)fc.Kw * p.H) return false;
+    c.h = ci % p.H;
+    const int64_t kk = (ci / p.H) % fc.Kw;
+    c.b = ci / (p.H * (int64_t)fc.Kw);
+    c.k = w * fc.Kw + kk;
+    if (c.k >= p.K) return false;
+    c.tbeg = c.k * p.chunk;
+    c.tend = (c.tbeg + p.chunk < p.L) ? c.tbeg + p.chunk : p.L;
+    return true;
+}
+
+__global__ void __launch_bounds__(THREADS, 2)
+k16_fused(KParams p, FusedCfg fc, FusedBufs fb, const float* __restrict__ x, const float* __restrict__ S0,
+          float* __restrict__ S_out)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ int64_t s_ticket;
+    __shared__ int s_go;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    WarpSmem& ws = reinterpret_cast<WarpSmem*>(smem_raw)[warp];
+    const int64_t tok = p.H * NN;
+    const int64_t nseq = p.B * p.H;
+    const int gpw = fc.Kw / fc.G;                    // groups per window
+
+    for (;;) {
+        if (tid == 0) s_ticket = ld_volatile(fb.abort_flag) ? fc.total : (int64_t)atomicAdd(fb.ticket, 1u);
+        __syncthreads();
+        const int64_t t = s_ticket;
+        __syncthreads();
+        if (t >= fc.total) return;
+
+        int kind;                                    // 0 R, 1 S1, 2 S2, 3 A
+        int64_t w, idx;
+        if (t < fc.lag * fc.nR) {
+            kind = 0; w = t / fc.nR; idx = t % fc.nR;
+        } else {
+            const int64_t bs = fc.nR + fc.nS1 + fc.nS2 + fc.nA;
+            const int64_t u = t - fc.lag * fc.nR;
+            w = u / bs;
+            int64_t r = u % bs;
+            if (r < fc.nR) { kind = 0; w += fc.lag; idx = r; }
+            else if ((r -= fc.nR) < fc.nS1) { kind = 1; idx = r; }
+            else if ((r -= fc.nS1) < fc.nS2) { kind = 2; idx = r; }
+            else { kind = 3; idx = r - fc.nS2; }
+        }
+        if (kind == 0 && w >= fc.NW) continue;       // past the last window: nothing to do
+
+        // ---- wait for this item's inputs ----
+        if (tid == 0) {
+            bool ok = true;
+            if (kind == 1) ok = wait_geq(fb.cntR + w, (unsigned)fc.nR, fb);
+            if (kind == 2) {
+                ok = wait_geq(fb.cntS1 + w, (unsigned)fc.nS1, fb);
+                if (ok && w > 0) ok = wait_geq(fb.cntS2 + w - 1, (unsigned)fc.nS2, fb);
+            }
+            if (kind == 3) ok = wait_geq(fb.cntS2 + w, (unsigned)fc.nS2, fb);
+            s_go = ok;
+        }
+        __syncthreads();
+        if (!s_go) return;
+
+        if (kind == 0) {
+            ChainIx c;
+            if (window_chain(p, fc, w, idx * WARPS + warp, c)) {
+                float Qd[2][4];
+                reduce_chain(p, ws, x + (c.b * p.L * p.H + c.h) * NN, tok, fb.cd + c.b * p.L * p.H + c.h,
+                             c.tbeg, c.tend, lane, fb.status, Qd);
+                store_d(fb.totals + ((c.b * p.H + c.h) * p.K + c.k) * NN, Qd, lane >> 2, lane & 3);
+            }
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) atomicAdd(fb.cntR + w, 1u);
+        } else if (kind == 1) {
+            const int64_t gi = idx * WARPS + warp;
+            const int64_t seq = gi / gpw;
+            const int64_t gg = w * gpw + gi % gpw;
+            if (seq < nseq && gg * fc.G < p.K) {
+                double* sR = reinterpret_cast<double*>(&ws.x[0][0]);
+                double* sT = sR + NN;
+                const int r0 = (lane >> 2) * 2, c0 = (lane & 3) * 4;
+                for (int e = lane; e < NN; e += 32) sR[e] = 0.0;
+                const int64_t k1 = (gg + 1) * fc.G < p.K ? (gg + 1) * fc.G : p.K;
+                for (int64_t k = gg * fc.G; k < k1; ++k) {
+                    const float* tk = fb.totals + (seq * p.K + k) * NN;
+                    for (int e = lane; e < NN; e += 32) sT[e] = (double)tk[e];
+                    __syncwarp();
+                    double acc[2][4];
+                    warp_gemm16_f64(sR, sT, lane, acc);
+                    __syncwarp();
+                    float* rk = fb.R0 + (seq * p.K + k) * NN;
+#pragma unroll
+                    for (int i = 0; i < 2; ++i)
+#pragma unroll
+                        for (int cc = 0; cc < 4; ++cc) {
+                            const int e = (r0 + i) * N + c0 + cc;
+                            const double v = sR[e] + (sT[e] + acc[i][cc]);
+                            sR[e] = v;
+                            rk[e] = (float)v;
+                        }
+                    __syncwarp();
+                }
+                double* tot = fb.Tot + (seq * fc.NG + gg) * NN;
+                for (int e = lane; e < NN; e += 32) tot[e] = sR[e];
+            }
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) atomicAdd(fb.cntS1 + w, 1u);
+        } else if (kind == 2) {
+            const int64_t seq = idx * WARPS + warp;
+            if (seq < nseq) {
+                double* sG = reinterpret_cast<double*>(&ws.x[0][0]);
+                double* sT = sG + NN;
+                const int r0 = (lane >> 2) * 2, c0 = (lane & 3) * 4;
+                for (int e = lane; e < NN; e += 32)
+                    sG[e] = (w > 0) ? fb.cstate[seq * NN + e]
+                                    : (S0 ? (double)S0[seq * NN + e] : ((e / N) == (e % N) ? 1.0 : 0.0));
+                __syncwarp();
+                for (int gw = 0; gw < gpw; ++gw) {
+                    const int64_t gg = w * gpw + gw;
+                    if (gg >= fc.NG) break;
+                    double* e1 = fb.E1 + (seq * fc.NG + gg) * NN;
+                    const double* tg = fb.Tot + (seq * fc.NG + gg) * NN;
+                    for (int e = lane; e < NN; e += 32) {
+                        e1[e] = sG[e];
+                        sT[e] = tg[e];
+                    }
+                    __syncwarp();
+                    double acc[2][4];
+                    warp_gemm16_f64(sG, sT, lane, acc);
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 2; ++i)
+#pragma unroll
+                        for (int cc = 0; cc < 4; ++cc) sG[(r0 + i) * N + c0 + cc] += acc[i][cc];
+                    __syncwarp();
+                }
+                for (int e = lane; e < NN; e += 32) fb.cstate[seq * NN + e] = sG[e];
+            }
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) atomicAdd(fb.cntS2 + w, 1u);
+        } else {
+            ChainIx c;
+            if (window_chain(p, fc, w, idx * WARPS + warp, c)) {
+                const int64_t seq = c.b * p.H + c.h;
+                float Sd[2][4];
+                form_carry(ws, fb.E1 + (seq * fc.NG + c.k / fc.G) * NN,
+                           (c.k % fc.G) ? fb.R0 + (seq * p.K + c.k - 1) * NN : nullptr, lane, Sd);
+                apply_chain(ws, x + (c.b * p.L * p.H + c.h) * NN, S_out + (c.b * p.L * p.H + c.h) * NN, tok, p.H,
+                            fb.cd + c.b * p.L * p.H + c.h, c.tbeg, c.tend, lane, Sd);
+            }
+            __syncthreads();
+        }
+    }
+}
+
 }  // namespace
 
 bool supports(const KParams& p, bool readout)
@@ -498,6 +751,85 @@ cudaError_t launch_apply(const KParams& p, const float* x, const float2* cd, con
     if (e != cudaSuccess) return e;
     k16_apply<<<grid, THREADS, sm, s>>>(p, x, cd, reinterpret_cast<const float*>(ws + pl.R[0]),
                                         reinterpret_cast<const double*>(ws + pl.E[1]), pl.G, S_out);
+    return cudaGetLastError();
+}
+
+// Layout of the fused kernel's workspace from byte offset `off` (the first
+// bytes, counters and flags, must be zeroed before every launch).
+FusedLayout fused_layout(const KParams& p, size_t off)
+{
+    FusedLayout L;
+    memset(&L, 0, sizeof L);
+    const int64_t nseq = p.B * p.H;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = (off + bytes + 255) / 256 * 256;
+        return o;
+    };
+    L.G = 16;
+    const int64_t unit = nseq * (int64_t)p.chunk * L.G * NN * (int64_t)sizeof(float);  // x bytes per group of chunks
+    int64_t groups = (16ll << 20) / (unit > 0 ? unit : 1);
+    if (groups < 1) groups = 1;
+    if (groups > 64) groups = 64;
+    L.Kw = (int)(groups * L.G);
+    L.NW = p.K > 0 ? (p.K + L.Kw - 1) / L.Kw : 0;
+    L.NG = (p.K + L.G - 1) / L.G;
+    L.counters = take(sizeof(unsigned) * (2 + 3 * (size_t)L.NW));
+    L.counters_bytes = sizeof(unsigned) * (2 + 3 * (size_t)L.NW);
+    L.totals = take(sizeof(float) * nseq * p.K * NN);
+    L.cd = take(sizeof(float2) * nseq * p.L);
+    L.R0 = take(sizeof(float) * nseq * p.K * NN);
+    L.Tot = take(sizeof(double) * nseq * L.NG * NN);
+    L.E1 = take(sizeof(double) * nseq * L.NG * NN);
+    L.cstate = take(sizeof(double) * nseq * NN);
+    L.end = off;
+    return L;
+}
+
+cudaError_t launch_fused(const KParams& p, const FusedLayout& L, char* ws, uint32_t* status, const float* x,
+                         const float* S0, float* S_out, cudaStream_t s)
+{
+    const int64_t nseq = p.B * p.H;
+    if (nseq * p.K == 0) return cudaSuccess;
+    FusedCfg fc;
+    fc.G = L.G;
+    fc.Kw = L.Kw;
+    fc.lag = 2;
+    fc.NW = L.NW;
+    fc.NG = L.NG;
+    const int64_t chains_w = p.B * (int64_t)L.Kw * p.H;
+    fc.nR = (chains_w + WARPS - 1) / WARPS;
+    fc.nA = fc.nR;
+    fc.nS1 = (nseq * (L.Kw / L.G) + WARPS - 1) / WARPS;
+    fc.nS2 = (nseq + WARPS - 1) / WARPS;
+    fc.total = fc.lag * fc.nR + fc.NW * (fc.nR + fc.nS1 + fc.nS2 + fc.nA);
+    FusedBufs fb;
+    unsigned* ctr = reinterpret_cast<unsigned*>(ws + L.counters);
+    fb.ticket = ctr;
+    fb.abort_flag = ctr + 1;
+    fb.cntR = ctr + 2;
+    fb.cntS1 = ctr + 2 + L.NW;
+    fb.cntS2 = ctr + 2 + 2 * L.NW;
+    fb.totals = reinterpret_cast<float*>(ws + L.totals);
+    fb.cd = reinterpret_cast<float2*>(ws + L.cd);
+    fb.R0 = reinterpret_cast<float*>(ws + L.R0);
+    fb.Tot = reinterpret_cast<double*>(ws + L.Tot);
+    fb.E1 = reinterpret_cast<double*>(ws + L.E1);
+    fb.cstate = reinterpret_cast<double*>(ws + L.cstate);
+    fb.status = status;
+    cudaError_t e = cudaMemsetAsync(ws + L.counters, 0, L.counters_bytes, s);
+    if (e != cudaSuccess) return e;
+    const size_t sm = sizeof(WarpSmem) * WARPS;
+    e = cudaFuncSetAttribute(k16_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k16_fused, THREADS, sm)) != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    int64_t grid = (int64_t)sms * per_sm;
+    if (grid > fc.total) grid = fc.total;
+    k16_fused<<<(unsigned)grid, THREADS, sm, s>>>(p, fc, fb, x, S0, S_out);
     return cudaGetLastError();
 }
 

@@ -627,6 +627,14 @@ cudaError_t launch_scan(const KParams& p, const void* src, const float* S0, cons
                         void* ws_base, const Workspace& W, cudaStream_t s, int* launches)
 {
     char* ws = reinterpret_cast<char*>(ws_base);
+    if (W.fused) {
+        profile_mark(0, 0, s);
+        cudaError_t e = n16::launch_fused(p, W.fl, ws, reinterpret_cast<uint32_t*>(ws + W.status),
+                                          reinterpret_cast<const float*>(src), S0, S_out, s);
+        profile_mark(0, 1, s);
+        if (launches) *launches = 1;
+        return e;
+    }
     if (W.fast) return scan_fast16(p, src, S0, S_out, ws, W, s, launches);
     switch (p.n) {
         case 4: return scan_n<4>(p, src, S0, u, snap_every, S_out, o_out, snaps, ws, W, s, launches);
