@@ -122,6 +122,11 @@ mru_status mru_last_device_status(const void* ws, void* stream);
 /* Static string for a status code. */
 const char* mru_status_string(mru_status s);
 
+/* The mru_math the kernels chosen for this problem compute in
+ * (MRU_MATH_FP32 for the generic fp32 kernels, MRU_MATH_TF32X3 or
+ * MRU_MATH_BF16X3 for the tensor-core kernels); -1 if p is invalid. */
+int32_t mru_effective_math(const mru_problem* p, int32_t readout);
+
 /* Chunk length the library would use for this problem (0 if invalid). */
 int32_t mru_chosen_chunk(const mru_problem* p);
 

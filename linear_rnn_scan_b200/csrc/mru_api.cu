@@ -47,9 +47,16 @@ bool fast16_eligible(const mru_problem& p, bool readout)
            (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32X3) && p.chunk % n16::kSub == 0;
 }
 
+bool fast32_eligible(const mru_problem& p, bool readout)
+{
+    return p.n == 32 && p.x_dtype == MRU_BF16 && !readout && p.mode == MRU_MODE_LDU &&
+           (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_BF16X3) && p.chunk % n16::kSub == 0;
+}
+
 int32_t choose_chunk(const mru_problem& p, int32_t src, bool readout)
 {
     if (p.chunk > 0) return p.chunk;
+    if (src == SRC_EMBEDDING && fast32_eligible(p, readout)) return n32::preferred_chunk(p.B * p.H * p.L);
     if (src == SRC_EMBEDDING && fast16_eligible(p, readout))
         return fused_enabled() ? 16 : n16::preferred_chunk(p.B * p.H * p.L);
     return generic_chunk(p);
@@ -105,10 +112,11 @@ Workspace layout(const KParams& k, bool readout)
         W.bytes = W.fl.end;
         return W;
     }
-    if (n16::supports(k, readout)) {
+    if (n16::supports(k, readout) || n32::supports(k, readout)) {
         W.fast = true;
+        W.fast_n = k.n;
         W.totals = off; off = round_up(off + BH * k.K * nn * sizeof(float), 256);
-        W.cd = off; off = round_up(off + BH * (size_t)k.L * sizeof(float2), 256);
+        if (k.n == 16) { W.cd = off; off = round_up(off + BH * (size_t)k.L * sizeof(float2), 256); }
         W.plan = carry::plan((int64_t)BH, k.K, (int)nn, off);
         W.bytes = W.plan.end > off ? W.plan.end : off;
         return W;
@@ -158,6 +166,13 @@ size_t mru_workspace_size(const mru_problem* p)
     return b;
 }
 
+int32_t mru_effective_math(const mru_problem* p, int32_t readout)
+{
+    if (check_problem(p) != MRU_OK) return -1;
+    const KParams k = make_params(*p, SRC_EMBEDDING, readout != 0);
+    return effective_math(k, readout != 0);
+}
+
 int32_t mru_chosen_chunk(const mru_problem* p)
 {
     if (check_problem(p) != MRU_OK) return 0;
@@ -172,11 +187,12 @@ const char* mru_kernel_name(const mru_problem* p, int32_t readout, int32_t i)
     if (W.fused) return i == 0 ? "k16_fused" : "";
     if (!W.fast) return kernel_name(k, readout != 0, i);
     const int lv = W.plan.levels;
-    if (i == 0) return "k16_reduce";
+    const bool n32k = W.fast_n == 32;
+    if (i == 0) return n32k ? "k32_reduce" : "k16_reduce";
     if (i >= 1 && i <= lv) return "k_level";
     if (i == lv + 1) return "k_top";
     if (i >= lv + 2 && i <= 2 * lv) return "k_down";
-    if (i == 2 * lv + 1) return "k16_apply";
+    if (i == 2 * lv + 1) return n32k ? "k32_apply" : "k16_apply";
     return "";
 }
 

@@ -21,7 +21,9 @@ namespace mru {
 namespace carry {
 namespace {
 
-constexpr int WARPS = 4;
+// warps per CTA of the carry kernels: the staged inputs of a warp take
+// (G + 1) N^2 doubles of shared memory
+template <int N> struct Warps { static constexpr int value = N <= 16 ? 4 : 2; };
 
 // One warp computes the product A B of two N x N fp64 matrices in shared
 // memory; each lane owns a block of RB rows x CB columns of the result.
@@ -91,7 +93,7 @@ __device__ __forceinline__ void stage(double* dst, const void* src, int64_t base
 // group totals Tot (fp64) [seq][ceil(cnt / G)].  One warp per (seq, group);
 // the group's inputs are staged in shared memory first.
 template <int N>
-__global__ void __launch_bounds__(32 * WARPS)
+__global__ void __launch_bounds__(32 * Warps<N>::value)
 k_level(int64_t nseq, int64_t cnt, int G, const void* in, int in32, void* R, int out32, double* Tot)
 {
     constexpr int NN = N * N;
@@ -101,7 +103,7 @@ k_level(int64_t nseq, int64_t cnt, int G, const void* in, int in32, void* R, int
     double* sR = dyn + (size_t)warp * (G + 1) * NN;
     double* sIn = sR + NN;
     const int64_t ngroups = (cnt + G - 1) / G;
-    const int64_t item = (int64_t)blockIdx.x * WARPS + warp;
+    const int64_t item = (int64_t)blockIdx.x * Warps<N>::value + warp;
     if (item >= nseq * ngroups) return;
     const int64_t seq = item / ngroups, g = item % ngroups;
     const int64_t j0 = g * G, j1 = (j0 + G < cnt) ? j0 + G : cnt;
@@ -135,7 +137,7 @@ k_level(int64_t nseq, int64_t cnt, int G, const void* in, int in32, void* R, int
 // Top level: exclusive carries of at most G group totals per sequence,
 // starting from S0 (or I).  E[seq][i] = S0 prod_{m < i} (I + Tot_m).
 template <int N>
-__global__ void __launch_bounds__(32 * WARPS)
+__global__ void __launch_bounds__(32 * Warps<N>::value)
 k_top(int64_t nseq, int64_t cnt, int G, const double* Tot, const float* S0, double* E)
 {
     constexpr int NN = N * N;
@@ -144,7 +146,7 @@ k_top(int64_t nseq, int64_t cnt, int G, const double* Tot, const float* S0, doub
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     double* sG = dyn + (size_t)warp * (G + 1) * NN;
     double* sIn = sG + NN;
-    const int64_t seq = (int64_t)blockIdx.x * WARPS + warp;
+    const int64_t seq = (int64_t)blockIdx.x * Warps<N>::value + warp;
     if (seq >= nseq) return;
     stage<N>(sIn, Tot, seq * cnt * NN, (int)cnt, 0, lane);
     int r0, c0;
@@ -173,14 +175,14 @@ k_top(int64_t nseq, int64_t cnt, int G, const double* Tot, const float* S0, doub
 // Going down one level: E_l[i] = E_{l+1}[i / G] (I + R_l[i - 1]), with R_l
 // fp64.  One warp per matrix.
 template <int N>
-__global__ void __launch_bounds__(32 * WARPS)
+__global__ void __launch_bounds__(32 * Warps<N>::value)
 k_down(int64_t nseq, int64_t cnt, int G, const double* Eup, const double* R, double* E)
 {
     constexpr int NN = N * N;
     using WG = WarpGemm<N>;
-    __shared__ double sm[WARPS][2][NN];
+    __shared__ double sm[Warps<N>::value][2][NN];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t item = (int64_t)blockIdx.x * WARPS + warp;
+    const int64_t item = (int64_t)blockIdx.x * Warps<N>::value + warp;
     if (item >= nseq * cnt) return;
     const int64_t seq = item / cnt, i = item % cnt;
     const int64_t nup = (cnt + G - 1) / G;
@@ -214,6 +216,7 @@ k_down(int64_t nseq, int64_t cnt, int G, const double* Eup, const double* R, dou
 template <int N>
 cudaError_t run(const Plan& pl, const float* totals, const float* S0, char* ws, cudaStream_t s, int& slot)
 {
+    constexpr int WARPS = Warps<N>::value;
     const int64_t nseq = pl.nseq;
     // level 1: chunk totals (fp32) -> R1 (fp32), Tot1 (fp64)
     int64_t cnt = pl.cnt[0];
@@ -268,7 +271,7 @@ Plan plan(int64_t nseq, int64_t K, int nn, size_t off)
     Plan pl;
     memset(&pl, 0, sizeof pl);
     pl.nseq = nseq;
-    pl.G = 16;
+    pl.G = nn <= 256 ? 16 : 8;
     auto take = [&](size_t bytes) {
         const size_t o = off;
         off = (off + bytes + 255) / 256 * 256;
@@ -297,6 +300,11 @@ int launches(const Plan& pl) { return pl.levels + 1 + (pl.levels - 1); }
 cudaError_t run_n16(const Plan& pl, const float* totals, const float* S0, char* ws, cudaStream_t s, int& slot)
 {
     return run<16>(pl, totals, S0, ws, s, slot);
+}
+
+cudaError_t run_n32(const Plan& pl, const float* totals, const float* S0, char* ws, cudaStream_t s, int& slot)
+{
+    return run<32>(pl, totals, S0, ws, s, slot);
 }
 
 }  // namespace carry

@@ -54,6 +54,7 @@ struct Plan {
 Plan plan(int64_t nseq, int64_t K, int nn, size_t off);
 int launches(const Plan& pl);
 cudaError_t run_n16(const Plan& pl, const float* totals, const float* S0, char* ws, cudaStream_t s, int& slot);
+cudaError_t run_n32(const Plan& pl, const float* totals, const float* S0, char* ws, cudaStream_t s, int& slot);
 }  // namespace carry
 
 namespace n16 {
@@ -74,6 +75,7 @@ struct Workspace {
     size_t carry;        // float  [B*H, K, n, n]   exclusive chunk carries (full matrices)
     bool fast;           // specialised kernels: chunk totals, per-token scalars, carry plan
     bool fused;          // the fused persistent kernel with its own layout below
+    int fast_n;          // 16 or 32: which specialised kernels
     n16::FusedLayout fl;
     size_t cd;           // float2 [B, L, H] per-token scalars (c alpha, diagonal of F)
     carry::Plan plan;
@@ -101,6 +103,15 @@ cudaError_t launch_fused(const KParams& p, const FusedLayout& L, char* ws, uint3
                          const float* S0, float* S_out, cudaStream_t s);
 }  // namespace n16
 
+// n = 32 LDU tensor-core kernels (mru_n32.cu).
+namespace n32 {
+bool supports(const KParams& p, bool readout);
+int32_t preferred_chunk(int64_t token_heads);
+cudaError_t launch_reduce(const KParams& p, const void* x, float* totals, cudaStream_t s);
+cudaError_t launch_apply(const KParams& p, const void* x, const carry::Plan& pl, const char* ws, float* S_out,
+                         cudaStream_t s);
+}  // namespace n32
+
 // Launchers (mru_scan_v1.cu).
 cudaError_t launch_build_states(const KParams& p, const void* x, float* X_out, int store_minus_identity,
                                 void* ws_base, const Workspace& W, cudaStream_t s);
@@ -109,5 +120,8 @@ cudaError_t launch_scan(const KParams& p, const void* src, const float* S0, cons
                         void* ws_base, const Workspace& W, cudaStream_t s, int* launches);
 // Name of the i-th kernel one launch_scan call starts for this problem.
 const char* kernel_name(const KParams& p, bool readout, int i);
+// mru_math the kernels for this problem actually use (MRU_MATH_FP32 for the
+// generic kernels).
+int32_t effective_math(const KParams& p, bool readout);
 
 }  // namespace mru

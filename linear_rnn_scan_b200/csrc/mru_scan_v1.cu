@@ -596,7 +596,32 @@ cudaError_t scan_fast16(const KParams& p, const void* src, const float* S0, floa
     return cudaGetLastError();
 }
 
+cudaError_t scan_fast32(const KParams& p, const void* src, const float* S0, float* S_out, char* ws,
+                        const Workspace& W, cudaStream_t s, int* launches)
+{
+    float* totals = reinterpret_cast<float*>(ws + W.totals);
+    if (p.B * p.H * p.K == 0) return cudaSuccess;
+    cudaError_t e;
+    int slot = 0;
+    profile_mark(slot, 0, s);
+    if ((e = n32::launch_reduce(p, src, totals, s)) != cudaSuccess) return e;
+    profile_mark(slot++, 1, s);
+    if ((e = carry::run_n32(W.plan, totals, S0, ws, s, slot)) != cudaSuccess) return e;
+    profile_mark(slot, 0, s);
+    if ((e = n32::launch_apply(p, src, W.plan, ws, S_out, s)) != cudaSuccess) return e;
+    profile_mark(slot++, 1, s);
+    if (launches) *launches = slot;
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+int32_t effective_math(const KParams& p, bool readout)
+{
+    if (n16::supports(p, readout)) return MRU_MATH_TF32X3;
+    if (n32::supports(p, readout)) return MRU_MATH_BF16X3;
+    return MRU_MATH_FP32;
+}
 
 const char* kernel_name(const KParams& p, bool readout, int i)
 {
@@ -635,6 +660,7 @@ cudaError_t launch_scan(const KParams& p, const void* src, const float* S0, cons
         if (launches) *launches = 1;
         return e;
     }
+    if (W.fast && W.fast_n == 32) return scan_fast32(p, src, S0, S_out, ws, W, s, launches);
     if (W.fast) return scan_fast16(p, src, S0, S_out, ws, W, s, launches);
     switch (p.n) {
         case 4: return scan_n<4>(p, src, S0, u, snap_every, S_out, o_out, snaps, ws, W, s, launches);

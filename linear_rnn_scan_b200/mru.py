@@ -30,7 +30,7 @@ MATH = {"auto": 0, "fp32": 1, "tf32": 2, "tf32x3": 3, "bf16x3": 4}
 # Every symbol include/mru.h declares.
 EXPORTS = ["mru_workspace_size", "mru_build_states", "mru_scan", "mru_scan_fused",
            "mru_last_device_status", "mru_status_string", "mru_chosen_chunk", "mru_launch_count",
-           "mru_set_profile_events", "mru_scan_fused_noalloc", "mru_kernel_name"]
+           "mru_set_profile_events", "mru_scan_fused_noalloc", "mru_kernel_name", "mru_effective_math"]
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -90,6 +90,8 @@ def load(path: str = LIB_PATH):
             lib.mru_scan_fused_noalloc.restype = ctypes.c_int
             lib.mru_kernel_name.argtypes = [P, ctypes.c_int32, ctypes.c_int32]
             lib.mru_kernel_name.restype = ctypes.c_char_p
+            lib.mru_effective_math.argtypes = [P, ctypes.c_int32]
+            lib.mru_effective_math.restype = ctypes.c_int32
             _lib = lib
     return _lib
 
@@ -126,6 +128,14 @@ def launch_count(p: Problem, readout: bool = False) -> int:
 def kernel_names(p: Problem, readout: bool = False) -> list:
     n = launch_count(p, readout)
     return [load().mru_kernel_name(ctypes.byref(p), int(bool(readout)), i).decode() for i in range(n)]
+
+
+MATH_NAMES = {v: k for k, v in MATH.items()}
+
+
+def effective_math(p: Problem, readout: bool = False) -> str:
+    """Name of the arithmetic the chosen kernels use: "fp32", "tf32x3", "bf16x3"."""
+    return MATH_NAMES.get(int(load().mru_effective_math(ctypes.byref(p), int(bool(readout)))), "invalid")
 
 
 def status_string(status: int) -> str:

@@ -15,7 +15,14 @@ TOL_TENSOR = 1e-2
 
 
 def tol_for(math: str) -> float:
-    return TOL_TENSOR if math in ("tf32", "bf16") else TOL_FP32
+    """Gate by the arithmetic the chosen kernels use: split-tf32 keeps fp32
+    accuracy (1e-4); single tf32 and split-bf16 tensor paths get 1e-2."""
+    return TOL_TENSOR if math in ("tf32", "bf16", "bf16x3") else TOL_FP32
+
+
+def tol_for_problem(w, **over) -> float:
+    p = mru.problem_from_workload(w, **over)
+    return tol_for(mru.effective_math(p, w.readout))
 
 
 def torch():

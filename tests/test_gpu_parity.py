@@ -13,7 +13,7 @@ from linear_rnn_scan_b200 import inputs as gen
 from linear_rnn_scan_b200 import mru
 
 from gpu_helpers import (TOL_FP32, compare_readout, compare_S, oracle_problem, run_fused, to_device_x,
-                         torch)
+                         tol_for_problem, torch)
 
 import oracle
 
@@ -116,7 +116,7 @@ def test_parity_bf16_and_initial_state(n, mode):
     S, st = run_fused(w, x, S0=S0, chunk=8)
     assert st == mru.OK
     e = compare_S(w, x, S, S0=S0)
-    assert e["max"] <= TOL_FP32, e
+    assert e["max"] <= tol_for_problem(w, chunk=8), e
 
 
 @pytest.mark.parametrize("n", [4, 16, 64])
@@ -214,10 +214,42 @@ def test_status_resets_between_calls():
     assert st == mru.OK
 
 
-def test_repeated_calls_are_deterministic():
-    w = small(32, gen.MODE_LDU, B=2, H=4, L=300, x_dtype="bf16", seed=800)
+@pytest.mark.parametrize("n,mode,dtype", [(32, gen.MODE_LDU, "bf16"), (16, gen.MODE_DETNORM, "f32"),
+                                           (64, gen.MODE_DETNORM, "f32")])
+def test_repeated_calls_are_deterministic(n, mode, dtype):
+    w = small(n, mode, B=2, H=4, L=300, x_dtype=dtype, seed=800)
     x = gen.make_x(w)
     first, _ = run_fused(w, x)
     for _ in range(5):
         again, _ = run_fused(w, x)
         assert np.array_equal(first, again)
+
+
+@pytest.mark.parametrize("L,chunk", [(1, 0), (7, 8), (8, 8), (9, 8), (100, 0), (300, 64), (129, 16)])
+@pytest.mark.parametrize("add_s0", [False, True])
+def test_parity_n32_ldu_tensor_path(L, chunk, add_s0):
+    """The bf16 tensor-core LDU kernels at n = 32: ragged chunks, S0."""
+    w = small(32, gen.MODE_LDU, B=2, H=3, L=L, x_dtype="bf16", seed=900 + L)
+    x = gen.make_x(w)
+    S0 = gen.make_S0(w, seed=901) if add_s0 else None
+    p = mru.problem_from_workload(w, chunk=chunk)
+    assert mru.effective_math(p) == "bf16x3"
+    S, st = run_fused(w, x, S0=S0, chunk=chunk)
+    assert st == mru.OK
+    e = compare_S(w, x, S, S0=S0)
+    assert e["count"] == w.B * w.L * w.H
+    assert e["max"] <= tol_for_problem(w, chunk=chunk), e
+
+
+@pytest.mark.parametrize("L,chunk", [(1, 0), (7, 8), (16, 8), (17, 8), (100, 0), (333, 32)])
+def test_parity_n16_tensor_path(L, chunk):
+    """The split-tf32 tensor-core kernels at n = 16 (fp32-accurate gate)."""
+    w = small(16, gen.MODE_DETNORM, B=2, H=3, L=L, alpha=0.05 / 4, seed=950 + L)
+    x = gen.make_x(w)
+    S0 = gen.make_S0(w, seed=951)
+    p = mru.problem_from_workload(w, chunk=chunk)
+    assert mru.effective_math(p) == "tf32x3"
+    S, st = run_fused(w, x, S0=S0, chunk=chunk)
+    assert st == mru.OK
+    e = compare_S(w, x, S, S0=S0)
+    assert e["max"] <= TOL_FP32, e

@@ -11,7 +11,7 @@ import pytest
 from linear_rnn_scan_b200 import inputs as gen
 from linear_rnn_scan_b200 import mru
 
-from gpu_helpers import compare_readout, compare_S, run_fused, tol_for, torch
+from gpu_helpers import compare_readout, compare_S, run_fused, tol_for_problem, torch
 
 pytestmark = pytest.mark.gpu
 
@@ -30,7 +30,7 @@ def test_full_workload_against_oracle(name):
     nbh = w.B * w.H
     k = SAMPLE[name]
     bh = None if k is None else np.unique(np.linspace(0, nbh - 1, k).round().astype(np.int64))
-    tol = tol_for(w.math)
+    tol = tol_for_problem(w)
     if w.readout:
         u = gen.make_u(w)
         (o, snaps), st = run_fused(w, x, u=u, every=w.snapshot_every)
