@@ -112,6 +112,14 @@ cudaError_t launch_apply(const KParams& p, const void* x, const carry::Plan& pl,
                          cudaStream_t s);
 }  // namespace n32
 
+// n = 64 readout chunk kernel on the tensor cores (mru_n64.cu); the carry
+// scan and fix-up are the generic kernels.
+namespace n64 {
+bool supports(const KParams& p, bool readout);
+cudaError_t launch_chunk_readout(const KParams& p, const float* x, const float* u, int64_t snap_every,
+                                 float* o_out, float* snaps, float* totals, uint32_t* status, cudaStream_t s);
+}  // namespace n64
+
 // Launchers (mru_scan_v1.cu).
 cudaError_t launch_build_states(const KParams& p, const void* x, float* X_out, int store_minus_identity,
                                 void* ws_base, const Workspace& W, cudaStream_t s);

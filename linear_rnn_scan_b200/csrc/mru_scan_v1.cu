@@ -556,8 +556,14 @@ cudaError_t scan_n(const KParams& p, const void* src, const float* S0, const flo
     if ((e = set_smem(k_carry_final<N>, sm_d)) != cudaSuccess) return e;
     if ((e = set_smem(k_fixup<N>, sm_fix)) != cudaSuccess) return e;
     profile_mark(0, 0, s);
-    k_chunk_prefix<N><<<(unsigned)chains, kThreads, sm_chunk, s>>>(p, src, u, snap_every, S_out, o_out,
-                                                                    snaps, totals, status);
+    if (N == 64 && o_out != nullptr && n64::supports(p, true)) {
+        if ((e = n64::launch_chunk_readout(p, reinterpret_cast<const float*>(src), u, snap_every, o_out, snaps,
+                                           totals, status, s)) != cudaSuccess)
+            return e;
+    } else {
+        k_chunk_prefix<N><<<(unsigned)chains, kThreads, sm_chunk, s>>>(p, src, u, snap_every, S_out, o_out,
+                                                                        snaps, totals, status);
+    }
     profile_mark(0, 1, s);
     profile_mark(1, 0, s);
     k_carry_local<N><<<(unsigned)(BH * p.NG), kThreads, sm_d, s>>>(p, totals, local);
@@ -620,16 +626,16 @@ int32_t effective_math(const KParams& p, bool readout)
 {
     if (n16::supports(p, readout)) return MRU_MATH_TF32X3;
     if (n32::supports(p, readout)) return MRU_MATH_BF16X3;
+    if (n64::supports(p, readout)) return MRU_MATH_TF32;
     return MRU_MATH_FP32;
 }
 
 const char* kernel_name(const KParams& p, bool readout, int i)
 {
-    (void)p;
-    (void)readout;
     static const char* generic[] = {"k_chunk_prefix", "k_carry_local", "k_carry_groups", "k_carry_final",
                                     "k_fixup"};
     if (i < 0 || i >= 5) return "";
+    if (i == 0 && n64::supports(p, readout)) return "k64_chunk_readout";
     return generic[i];
 }
 
