@@ -1,5 +1,6 @@
 // mru_carry.cu -- multi-level fp64 scan of chunk totals for the specialised
-// kernels (one warp per group of G matrices).
+// kernels (one CTA per group of G matrices, every thread one output element
+// of each small product).
 //
 // Level 1 sees the chunk totals T_k = I + Q_k (fp32 Q_k from the chunk
 // kernel).  Each level cuts its sequence of matrices into groups of G and
@@ -21,56 +22,35 @@ namespace mru {
 namespace carry {
 namespace {
 
-// warps per CTA of the carry kernels: the staged inputs of a warp take
-// (G + 1) N^2 doubles of shared memory
-template <int N> struct Warps { static constexpr int value = N <= 16 ? 4 : 2; };
+constexpr int CT = 256;              // threads per CTA: one CTA per group / sequence / matrix
 
-// One warp computes the product A B of two N x N fp64 matrices in shared
-// memory; each lane owns a block of RB rows x CB columns of the result.
+// Cooperative fp64 product of two N x N matrices in shared memory: thread t
+// computes outputs (i, j) for e = t, t + CT, ... (i = e / N, j = e % N); the
+// whole CTA calls it.  PER = N*N / CT outputs per thread.
 template <int N>
-struct WarpGemm {
-    static constexpr int RB = N / 8;            // rows per lane
-    static constexpr int CB = N * N / 32 / RB;  // cols per lane
-    static constexpr int LANES_PER_ROWBLOCK = N / CB;
-    // lane -> (row0, col0)
-    __device__ static void owner(int lane, int& r0, int& c0)
+struct CtaGemm {
+    static constexpr int PER = (N * N + CT - 1) / CT;
+    __device__ static void mul(const double* A, const double* B, double (&acc)[PER])
     {
-        r0 = (lane / LANES_PER_ROWBLOCK) * RB;
-        c0 = (lane % LANES_PER_ROWBLOCK) * CB;
-    }
-    // acc[r][c] = sum_k A[r0 + r][k] B[k][c0 + c]
-    __device__ static void mul(const double* A, const double* B, int lane, double (&acc)[RB][CB])
-    {
-        int r0, c0;
-        owner(lane, r0, c0);
 #pragma unroll
-        for (int r = 0; r < RB; ++r)
-#pragma unroll
-            for (int c = 0; c < CB; ++c) acc[r][c] = 0.0;
-#pragma unroll 4
-        for (int k = 0; k < N; ++k) {
-            double a[RB], b[CB];
-#pragma unroll
-            for (int r = 0; r < RB; ++r) a[r] = A[(r0 + r) * N + k];
-#pragma unroll
-            for (int c = 0; c < CB; ++c) b[c] = B[k * N + c0 + c];
-#pragma unroll
-            for (int r = 0; r < RB; ++r)
-#pragma unroll
-                for (int c = 0; c < CB; ++c) acc[r][c] = fma(a[r], b[c], acc[r][c]);
+        for (int r = 0; r < PER; ++r) {
+            const int e = threadIdx.x + r * CT;
+            const int i = e / N, j = e % N;
+            double a = 0.0;
+#pragma unroll 8
+            for (int k = 0; k < N; ++k) a = fma(A[i * N + k], B[k * N + j], a);
+            acc[r] = a;
         }
     }
 };
 
-// Copies `count` matrices of N x N (fp32 when in32, else fp64) from global
-// memory to shared memory as fp64, all loads in flight at once.
-template <int N>
-__device__ __forceinline__ void stage(double* dst, const void* src, int64_t base, int count, int in32, int lane)
+// Copies `count` N x N matrices (fp32 when in32, else fp64) to shared memory
+// as fp64, every load in flight at once.
+__device__ __forceinline__ void stage(double* dst, const void* src, int64_t base, int64_t nvals, int in32)
 {
-    constexpr int NN = N * N;
     if (in32) {
         const float4* s4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(src) + base);
-        for (int e = lane; e < count * NN / 4; e += 32) {
+        for (int64_t e = threadIdx.x; e < nvals / 4; e += CT) {
             const float4 v = s4[e];
             dst[4 * e + 0] = v.x;
             dst[4 * e + 1] = v.y;
@@ -79,7 +59,7 @@ __device__ __forceinline__ void stage(double* dst, const void* src, int64_t base
         }
     } else {
         const double2* s2 = reinterpret_cast<const double2*>(reinterpret_cast<const double*>(src) + base);
-        for (int e = lane; e < count * NN / 2; e += 32) {
+        for (int64_t e = threadIdx.x; e < nvals / 2; e += CT) {
             const double2 v = s2[e];
             dst[2 * e + 0] = v.x;
             dst[2 * e + 1] = v.y;
@@ -90,170 +70,147 @@ __device__ __forceinline__ void stage(double* dst, const void* src, int64_t base
 // Inclusive local prefixes of one level.  Input: per sequence `cnt` matrices
 // (fp32 split form when in32, else fp64 split form), laid out
 // [seq][cnt][N][N].  Output: R (fp32 when out32, else fp64) [seq][cnt], and
-// group totals Tot (fp64) [seq][ceil(cnt / G)].  One warp per (seq, group);
+// group totals Tot (fp64) [seq][ceil(cnt / G)].  One CTA per (seq, group);
 // the group's inputs are staged in shared memory first.
 template <int N>
-__global__ void __launch_bounds__(32 * Warps<N>::value)
+__global__ void __launch_bounds__(CT)
 k_level(int64_t nseq, int64_t cnt, int G, const void* in, int in32, void* R, int out32, double* Tot)
 {
     constexpr int NN = N * N;
-    using WG = WarpGemm<N>;
+    using CG = CtaGemm<N>;
     extern __shared__ double dyn[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    double* sR = dyn + (size_t)warp * (G + 1) * NN;
+    double* sR = dyn;
     double* sIn = sR + NN;
     const int64_t ngroups = (cnt + G - 1) / G;
-    const int64_t item = (int64_t)blockIdx.x * Warps<N>::value + warp;
-    if (item >= nseq * ngroups) return;
-    const int64_t seq = item / ngroups, g = item % ngroups;
+    const int64_t seq = blockIdx.x / ngroups, g = blockIdx.x % ngroups;
     const int64_t j0 = g * G, j1 = (j0 + G < cnt) ? j0 + G : cnt;
-    stage<N>(sIn, in, (seq * cnt + j0) * NN, (int)(j1 - j0), in32, lane);
-    int r0, c0;
-    WG::owner(lane, r0, c0);
-    for (int e = lane; e < NN; e += 32) sR[e] = 0.0;
-    __syncwarp();
+    stage(sIn, in, (seq * cnt + j0) * NN, (j1 - j0) * NN, in32);
+    for (int e = threadIdx.x; e < NN; e += CT) sR[e] = 0.0;
+    __syncthreads();
     for (int64_t j = j0; j < j1; ++j) {
         const double* sT = sIn + (j - j0) * NN;
         const int64_t base = (seq * cnt + j) * NN;
-        double acc[WG::RB][WG::CB];
-        WG::mul(sR, sT, lane, acc);
-        __syncwarp();
+        double acc[CG::PER];
+        CG::mul(sR, sT, acc);
+        __syncthreads();
 #pragma unroll
-        for (int r = 0; r < WG::RB; ++r)
-#pragma unroll
-            for (int c = 0; c < WG::CB; ++c) {
-                const int e = (r0 + r) * N + c0 + c;
-                const double v = sR[e] + (sT[e] + acc[r][c]);
-                sR[e] = v;
-                if (out32) reinterpret_cast<float*>(R)[base + e] = (float)v;
-                else reinterpret_cast<double*>(R)[base + e] = v;
-            }
-        __syncwarp();
+        for (int r = 0; r < CG::PER; ++r) {
+            const int e = threadIdx.x + r * CT;
+            const double v = sR[e] + (sT[e] + acc[r]);
+            sR[e] = v;
+            if (out32) reinterpret_cast<float*>(R)[base + e] = (float)v;
+            else reinterpret_cast<double*>(R)[base + e] = v;
+        }
+        __syncthreads();
     }
     double* tot = Tot + (seq * ngroups + g) * NN;
-    for (int e = lane; e < NN; e += 32) tot[e] = sR[e];
+    for (int e = threadIdx.x; e < NN; e += CT) tot[e] = sR[e];
 }
 
 // Top level: exclusive carries of at most G group totals per sequence,
 // starting from S0 (or I).  E[seq][i] = S0 prod_{m < i} (I + Tot_m).
 template <int N>
-__global__ void __launch_bounds__(32 * Warps<N>::value)
+__global__ void __launch_bounds__(CT)
 k_top(int64_t nseq, int64_t cnt, int G, const double* Tot, const float* S0, double* E)
 {
     constexpr int NN = N * N;
-    using WG = WarpGemm<N>;
+    using CG = CtaGemm<N>;
     extern __shared__ double dyn[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    double* sG = dyn + (size_t)warp * (G + 1) * NN;
+    double* sG = dyn;
     double* sIn = sG + NN;
-    const int64_t seq = (int64_t)blockIdx.x * Warps<N>::value + warp;
-    if (seq >= nseq) return;
-    stage<N>(sIn, Tot, seq * cnt * NN, (int)cnt, 0, lane);
-    int r0, c0;
-    WG::owner(lane, r0, c0);
-    for (int e = lane; e < NN; e += 32)
+    const int64_t seq = blockIdx.x;
+    (void)G;
+    stage(sIn, Tot, seq * cnt * NN, cnt * NN, 0);
+    for (int e = threadIdx.x; e < NN; e += CT)
         sG[e] = S0 ? (double)S0[seq * NN + e] : ((e / N) == (e % N) ? 1.0 : 0.0);
-    __syncwarp();
+    __syncthreads();
     for (int64_t i = 0; i < cnt; ++i) {
         const double* sT = sIn + i * NN;
         const int64_t base = (seq * cnt + i) * NN;
-        for (int e = lane; e < NN; e += 32) E[base + e] = sG[e];
-        double acc[WG::RB][WG::CB];
-        WG::mul(sG, sT, lane, acc);
-        __syncwarp();
+        for (int e = threadIdx.x; e < NN; e += CT) E[base + e] = sG[e];
+        double acc[CG::PER];
+        CG::mul(sG, sT, acc);
+        __syncthreads();
 #pragma unroll
-        for (int r = 0; r < WG::RB; ++r)
-#pragma unroll
-            for (int c = 0; c < WG::CB; ++c) {
-                const int e = (r0 + r) * N + c0 + c;
-                sG[e] = sG[e] + acc[r][c];
-            }
-        __syncwarp();
+        for (int r = 0; r < CG::PER; ++r) {
+            const int e = threadIdx.x + r * CT;
+            sG[e] = sG[e] + acc[r];
+        }
+        __syncthreads();
     }
 }
 
 // Going down one level: E_l[i] = E_{l+1}[i / G] (I + R_l[i - 1]), with R_l
-// fp64.  One warp per matrix.
+// fp64.  One CTA per matrix.
 template <int N>
-__global__ void __launch_bounds__(32 * Warps<N>::value)
+__global__ void __launch_bounds__(CT)
 k_down(int64_t nseq, int64_t cnt, int G, const double* Eup, const double* R, double* E)
 {
     constexpr int NN = N * N;
-    using WG = WarpGemm<N>;
-    __shared__ double sm[Warps<N>::value][2][NN];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t item = (int64_t)blockIdx.x * Warps<N>::value + warp;
-    if (item >= nseq * cnt) return;
+    using CG = CtaGemm<N>;
+    __shared__ double sG[NN];
+    __shared__ double sT[NN];
+    const int64_t item = blockIdx.x;
     const int64_t seq = item / cnt, i = item % cnt;
     const int64_t nup = (cnt + G - 1) / G;
     const double* up = Eup + (seq * nup + i / G) * NN;
     double* out = E + item * NN;
     if (i % G == 0) {
-        for (int e = lane; e < NN; e += 32) out[e] = up[e];
+        for (int e = threadIdx.x; e < NN; e += CT) out[e] = up[e];
         return;
     }
-    double* sG = sm[warp][0];
-    double* sT = sm[warp][1];
     const double* rp = R + (item - 1) * NN;
-    for (int e = lane; e < NN; e += 32) {
+    for (int e = threadIdx.x; e < NN; e += CT) {
         sG[e] = up[e];
         sT[e] = rp[e];
     }
-    __syncwarp();
-    double acc[WG::RB][WG::CB];
-    WG::mul(sG, sT, lane, acc);
-    int r0, c0;
-    WG::owner(lane, r0, c0);
+    __syncthreads();
+    double acc[CG::PER];
+    CG::mul(sG, sT, acc);
 #pragma unroll
-    for (int r = 0; r < WG::RB; ++r)
-#pragma unroll
-        for (int c = 0; c < WG::CB; ++c) {
-            const int e = (r0 + r) * N + c0 + c;
-            out[e] = sG[e] + acc[r][c];
-        }
+    for (int r = 0; r < CG::PER; ++r) {
+        const int e = threadIdx.x + r * CT;
+        out[e] = sG[e] + acc[r];
+    }
 }
 
 template <int N>
 cudaError_t run(const Plan& pl, const float* totals, const float* S0, char* ws, cudaStream_t s, int& slot)
 {
-    constexpr int WARPS = Warps<N>::value;
+    constexpr int NN = N * N;
     const int64_t nseq = pl.nseq;
     // level 1: chunk totals (fp32) -> R1 (fp32), Tot1 (fp64)
     int64_t cnt = pl.cnt[0];
     const void* in = totals;
     int in32 = 1;
-    const size_t sm = sizeof(double) * WARPS * (pl.G + 1) * N * N;
+    const size_t sm = sizeof(double) * (size_t)(pl.G + 1) * NN;
     cudaError_t e = cudaFuncSetAttribute(k_level<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(k_top<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     for (int l = 0; l < pl.levels; ++l) {
         const int64_t ng = (cnt + pl.G - 1) / pl.G;
-        const unsigned grid = (unsigned)((nseq * ng + WARPS - 1) / WARPS);
         profile_mark(slot, 0, s);
-        k_level<N><<<grid, 32 * WARPS, sm, s>>>(nseq, cnt, pl.G, in, in32, ws + pl.R[l], l == 0 ? 1 : 0,
-                                                reinterpret_cast<double*>(ws + pl.Tot[l]));
+        k_level<N><<<(unsigned)(nseq * ng), CT, sm, s>>>(nseq, cnt, pl.G, in, in32, ws + pl.R[l], l == 0 ? 1 : 0,
+                                                         reinterpret_cast<double*>(ws + pl.Tot[l]));
         profile_mark(slot++, 1, s);
         in = ws + pl.Tot[l];
         in32 = 0;
         cnt = ng;
     }
     // top
-    {
-        const unsigned grid = (unsigned)((nseq + WARPS - 1) / WARPS);
-        profile_mark(slot, 0, s);
-        k_top<N><<<grid, 32 * WARPS, sm, s>>>(nseq, cnt, pl.G, reinterpret_cast<const double*>(in), S0,
-                                              reinterpret_cast<double*>(ws + pl.E[pl.levels]));
-        profile_mark(slot++, 1, s);
-    }
-    // down to level 2's carries (level-1 carries are formed by the fix-up)
+    profile_mark(slot, 0, s);
+    k_top<N><<<(unsigned)nseq, CT, sm, s>>>(nseq, cnt, pl.G, reinterpret_cast<const double*>(in), S0,
+                                            reinterpret_cast<double*>(ws + pl.E[pl.levels]));
+    profile_mark(slot++, 1, s);
+    // down to level 2's carries (level-1 carries are formed by the apply pass)
     for (int l = pl.levels - 1; l >= 1; --l) {
         const int64_t c = pl.cnt[l];
-        const unsigned grid = (unsigned)((nseq * c + WARPS - 1) / WARPS);
         profile_mark(slot, 0, s);
-        k_down<N><<<grid, 32 * WARPS, 0, s>>>(nseq, c, pl.G, reinterpret_cast<const double*>(ws + pl.E[l + 1]),
-                                              reinterpret_cast<const double*>(ws + pl.R[l]),
-                                              reinterpret_cast<double*>(ws + pl.E[l]));
+        k_down<N><<<(unsigned)(nseq * c), CT, 0, s>>>(nseq, c, pl.G,
+                                                      reinterpret_cast<const double*>(ws + pl.E[l + 1]),
+                                                      reinterpret_cast<const double*>(ws + pl.R[l]),
+                                                      reinterpret_cast<double*>(ws + pl.E[l]));
         profile_mark(slot++, 1, s);
     }
     return cudaGetLastError();

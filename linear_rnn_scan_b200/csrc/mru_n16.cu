@@ -402,9 +402,12 @@ __device__ __forceinline__ void apply_chain(WarpSmem& ws, const float* xb, float
     const float m1 = (g == 2 * q + 1) ? 1.0f : 0.0f;
     for (int64_t t0 = tbeg; t0 < tend; t0 += SUB) {
         const int nt_pass = (tend - t0 < SUB) ? (int)(tend - t0) : SUB;
+        // the pass's per-token scalars travel with the slice copies (they
+        // would otherwise be a dependent global load per token)
+        if (lane < nt_pass) ws.cd[lane] = cdb[(t0 + lane) * H];
         load_pass(ws, xb, tok, t0, nt_pass, lane);
         for (int j = 0; j < nt_pass; ++j) {
-            const float2 cdj = cdb[(t0 + j) * H];
+            const float2 cdj = ws.cd[j];
             FragF f;
             make_frag_f(ws.x[j], cdj.x, m0 * cdj.y, m1 * cdj.y, g, q, f, false);
             float acc[2][4];
