@@ -9,18 +9,6 @@
 namespace mru {
 namespace {
 
-// The two-pass n = 16 kernels are the default; MRU_N16_FUSED=1 in the
-// environment selects the fused persistent kernel instead (experimental: it
-// is correct but its per-window scans still serialise the windows).
-bool fused_enabled()
-{
-    static const bool on = [] {
-        const char* v = getenv("MRU_N16_FUSED");
-        return v && v[0] == '1';
-    }();
-    return on;
-}
-
 bool supported_n(int n) { return n == 4 || n == 8 || n == 16 || n == 32 || n == 64; }
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
@@ -58,7 +46,7 @@ int32_t choose_chunk(const mru_problem& p, int32_t src, bool readout)
     if (p.chunk > 0) return p.chunk;
     if (src == SRC_EMBEDDING && fast32_eligible(p, readout)) return n32::preferred_chunk(p.B * p.H * p.L);
     if (src == SRC_EMBEDDING && fast16_eligible(p, readout))
-        return fused_enabled() ? 16 : n16::preferred_chunk(p.B * p.H * p.L);
+        return n16::preferred_chunk(p.B * p.H * p.L);
     return generic_chunk(p);
 }
 
@@ -94,6 +82,8 @@ KParams make_params(const mru_problem& p, int32_t src, bool readout)
     k.K = ceil_div(p.L, k.chunk);
     k.group = choose_group(k.K);
     k.NG = k.K > 0 ? ceil_div(k.K, k.group) : 0;
+    fastdiv_magic(k.H, k.h_mul, k.h_shr);
+    fastdiv_magic(k.K, k.k_mul, k.k_shr);
     return k;
 }
 
@@ -105,18 +95,18 @@ Workspace layout(const KParams& k, bool readout)
     const size_t BH = (size_t)(k.B * k.H);
     size_t off = 0;
     W.status = off; off += 256;
-    if (n16::supports(k, readout) && k.chunk == 16 && fused_enabled()) {
+    if (n16::supports(k, readout)) {
         W.fast = true;
-        W.fused = true;
-        W.fl = n16::fused_layout(k, off);
-        W.bytes = W.fl.end;
+        W.fast_n = 16;
+        W.totals = off; off = round_up(off + BH * k.K * nn * sizeof(float), 256);
+        W.c16 = n16::carry_plan((int64_t)BH, k.K, off);
+        W.bytes = W.c16.end > off ? W.c16.end : off;
         return W;
     }
-    if (n16::supports(k, readout) || n32::supports(k, readout)) {
+    if (n32::supports(k, readout)) {
         W.fast = true;
-        W.fast_n = k.n;
+        W.fast_n = 32;
         W.totals = off; off = round_up(off + BH * k.K * nn * sizeof(float), 256);
-        if (k.n == 16) { W.cd = off; off = round_up(off + BH * (size_t)k.L * sizeof(float2), 256); }
         W.plan = carry::plan((int64_t)BH, k.K, (int)nn, off);
         W.bytes = W.plan.end > off ? W.plan.end : off;
         return W;
@@ -184,8 +174,8 @@ const char* mru_kernel_name(const mru_problem* p, int32_t readout, int32_t i)
     if (check_problem(p) != MRU_OK) return "";
     const KParams k = make_params(*p, SRC_EMBEDDING, readout != 0);
     const Workspace W = layout(k, readout != 0);
-    if (W.fused) return i == 0 ? "k16_fused" : "";
     if (!W.fast) return kernel_name(k, readout != 0, i);
+    if (W.fast_n == 16) return i == 0 ? "k16_reduce" : i == 1 ? "k16_carry" : i == 2 ? "k16_apply" : "";
     const int lv = W.plan.levels;
     const bool n32k = W.fast_n == 32;
     if (i == 0) return n32k ? "k32_reduce" : "k16_reduce";
@@ -202,8 +192,8 @@ int32_t mru_launch_count(const mru_problem* p, int32_t readout)
     if (p->B * p->H * p->L == 0) return 0;
     const KParams k = make_params(*p, SRC_EMBEDDING, readout != 0);
     const Workspace W = layout(k, readout != 0);
-    if (W.fused) return 1;
-    return W.fast ? 2 + carry::launches(W.plan) : 5;
+    if (W.fast) return W.fast_n == 16 ? 3 : 2 + carry::launches(W.plan);
+    return 5;
 }
 
 mru_status mru_build_states(const mru_problem* p, const void* x, float* X_out, void* ws, size_t ws_bytes,

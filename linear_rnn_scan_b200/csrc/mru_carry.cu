@@ -1,4 +1,4 @@
-// mru_carry.cu -- multi-level fp64 scan of chunk totals for the specialised
+// mru_carry.cu -- multi-level fp64 scan of chunk totals for the n = 32
 // kernels (one CTA per group of G matrices, every thread one output element
 // of each small product).
 //
@@ -253,11 +253,6 @@ Plan plan(int64_t nseq, int64_t K, int nn, size_t off)
 }
 
 int launches(const Plan& pl) { return pl.levels + 1 + (pl.levels - 1); }
-
-cudaError_t run_n16(const Plan& pl, const float* totals, const float* S0, char* ws, cudaStream_t s, int& slot)
-{
-    return run<16>(pl, totals, S0, ws, s, slot);
-}
 
 cudaError_t run_n32(const Plan& pl, const float* totals, const float* S0, char* ws, cudaStream_t s, int& slot)
 {

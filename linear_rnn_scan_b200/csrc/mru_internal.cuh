@@ -35,7 +35,26 @@ struct KParams {
     int64_t K;           // chunks per sequence, ceil(L / C)
     int32_t group;       // chunk totals per carry group (G)
     int64_t NG;          // carry groups per sequence, ceil(K / G)
+    // q = (umulhi(i, mul) + i) >> shr is i / H (i / K) for 0 <= i < 2^31
+    uint32_t h_mul, h_shr, k_mul, k_shr;
 };
+
+// Multiplier and shift of the division by d (>= 1) for 31-bit dividends:
+// l = ceil(log2 d), mul = floor(2^32 (2^l - d) / d) + 1 (Granlund and
+// Montgomery, 1994, unsigned division by invariant integers).
+inline void fastdiv_magic(int64_t d, uint32_t& mul, uint32_t& shr)
+{
+    if (d <= 1) { mul = 0; shr = 0; return; }
+    uint32_t l = 0;
+    while ((int64_t(1) << l) < d) ++l;
+    const unsigned __int128 num = ((unsigned __int128)1 << 32) * (((unsigned __int128)1 << l) - (unsigned __int128)d);
+    mul = (uint32_t)(num / (unsigned __int128)d + 1);
+    shr = l;
+}
+__device__ __forceinline__ uint32_t fastdiv(uint32_t i, uint32_t mul, uint32_t shr)
+{
+    return (__umulhi(i, mul) + i) >> shr;
+}
 
 // Workspace carve-up (byte offsets from the workspace base).
 // Multi-level fp64 scan of chunk totals (mru_carry.cu).
@@ -53,17 +72,26 @@ struct Plan {
 };
 Plan plan(int64_t nseq, int64_t K, int nn, size_t off);
 int launches(const Plan& pl);
-cudaError_t run_n16(const Plan& pl, const float* totals, const float* S0, char* ws, cudaStream_t s, int& slot);
 cudaError_t run_n32(const Plan& pl, const float* totals, const float* S0, char* ws, cudaStream_t s, int& slot);
 }  // namespace carry
 
+// n = 16 carry scan (one launch between the passes): a warp per group of G
+// chunk totals scans the group (fp64 tensor cores) and passes the group total
+// up a level; the last warp of a group there scans it, up to the top, which
+// is scanned from S0.
 namespace n16 {
-// The fused persistent kernel: one launch, reduce / carry / apply as a
-// dataflow over L2-sized windows.
-struct FusedLayout {
-    int G, Kw;
-    int64_t NW, NG;
-    size_t counters, counters_bytes, totals, cd, R0, Tot, E1, cstate, end;
+constexpr int kCarryLevels = 3;
+struct CarryPlan {
+    int64_t nseq;
+    int32_t G, gshift;                   // items per group, a power of two (G = 1 << gshift)
+    int32_t levels;                      // scanned levels below the top (<= kCarryLevels)
+    int64_t cnt[kCarryLevels + 1];       // items per sequence at level l (cnt[0] = K chunk totals)
+    size_t R[kCarryLevels];              // inclusive in-group prefixes of level l, [seq][cnt[l]] (fp32 at l = 0, else fp64)
+    size_t Tot[kCarryLevels];            // group totals of level l (fp64), [seq][cnt[l + 1]]
+    size_t Etop;                         // exclusive carries of the top level (fp64), [seq][cnt[levels]]
+    size_t ctr[kCarryLevels + 1];        // arrival counters (uint32): level l [seq][cnt[l + 1]], top [seq]
+    size_t ctr_begin, ctr_bytes;         // the counters (zeroed by every reduce launch)
+    size_t end;
 };
 }  // namespace n16
 
@@ -73,12 +101,10 @@ struct Workspace {
     size_t local;        // double [B*H, K, n, n]   inclusive in-group prefixes of totals, split form
     size_t gcarry;       // double [B*H, NG, n, n]  exclusive group carries (full matrices)
     size_t carry;        // float  [B*H, K, n, n]   exclusive chunk carries (full matrices)
-    bool fast;           // specialised kernels: chunk totals, per-token scalars, carry plan
-    bool fused;          // the fused persistent kernel with its own layout below
+    bool fast;           // specialised kernels: chunk totals and a carry plan
     int fast_n;          // 16 or 32: which specialised kernels
-    n16::FusedLayout fl;
-    size_t cd;           // float2 [B, L, H] per-token scalars (c alpha, diagonal of F)
-    carry::Plan plan;
+    carry::Plan plan;    // n = 32
+    n16::CarryPlan c16;  // n = 16
     size_t bytes;        // total
 };
 
@@ -91,16 +117,16 @@ void profile_mark(int kernel, int after, cudaStream_t s);
 
 // n = 16 tensor-core kernels (mru_n16.cu).
 namespace n16 {
-constexpr int kSub = 8;           // tokens per LU pass; chunks are multiples of it
+constexpr int kSub = 8;           // chunks of the specialised kernels are multiples of it
 bool supports(const KParams& p, bool readout);
 int32_t preferred_chunk(int64_t token_heads);
-cudaError_t launch_reduce(const KParams& p, const float* x, float* totals, float2* cd, uint32_t* status,
-                          cudaStream_t s);
-cudaError_t launch_apply(const KParams& p, const float* x, const float2* cd, const carry::Plan& pl,
-                         const char* ws, float* S_out, cudaStream_t s);
-FusedLayout fused_layout(const KParams& p, size_t off);
-cudaError_t launch_fused(const KParams& p, const FusedLayout& L, char* ws, uint32_t* status, const float* x,
-                         const float* S0, float* S_out, cudaStream_t s);
+CarryPlan carry_plan(int64_t nseq, int64_t K, size_t off);
+cudaError_t launch_reduce(const KParams& p, const float* x, float* totals, const CarryPlan& cp, char* ws,
+                          uint32_t* status, cudaStream_t s);
+cudaError_t launch_carry(const KParams& p, const float* totals, const CarryPlan& cp, char* ws, const float* S0,
+                         cudaStream_t s);
+cudaError_t launch_apply(const KParams& p, const float* x, const CarryPlan& cp, const char* ws, float* S_out,
+                         uint32_t* status, cudaStream_t s);
 }  // namespace n16
 
 // n = 32 LDU tensor-core kernels (mru_n32.cu).

@@ -1,31 +1,47 @@
 // mru_n16.cu -- n = 16 scan kernels on the tensor cores (fp32 embeddings,
-// reshape and determinant-corrected modes), two passes over the embeddings:
+// reshape and determinant-corrected modes): two launches, two passes over
+// the embeddings.
 //
-//  * reduce pass   one warp per chain (b, h, chunk of C = 8m tokens); warps
-//                  never wait for each other.  Per pass of 8 tokens the warp
-//                  copies the 8 token-head slices to its shared memory
-//                  (cp.async, rows padded to 20 words), factorises the 8
-//                  matrices at once with 4 lanes per token (lane r owns rows
-//                  r, r+4, r+8, r+12 in registers; the pivot row is broadcast
-//                  by shuffles inside the 4-lane group), records the token's
-//                  scalars (c alpha, diagonal of F) and advances the chunk
-//                  product Q_t = Q_{t-1} + (F_t + Q_{t-1} F_t) with mma.sync
-//                  m16n8k8 tf32 in split precision.  The state stays in the
-//                  accumulator registers from token to token: the contraction
-//                  index of the next product is permuted so that the
-//                  accumulator fragment of column tile j is exactly the A
-//                  fragment of k-tile j.  Only the chunk total is written.
-//  * (the fp64 scan of chunk totals, mru_carry.cu)
-//  * apply pass    one warp per chain: forms the chunk's exact carry from the
-//                  carry scan (fp64), then runs the chain again from it,
-//                  S_t = S_{t-1} + S_{t-1} F_t, and writes every S_t.  No local
-//                  prefix ever goes to memory: per token·head the path moves
-//                  x twice and S once.
+// Both passes run persistent warps: warp w of W takes the chains (b, h,
+// chunk of C tokens) w, w + W, w + 2W, ... (a CTA's warps hold neighbouring
+// heads of one token range, whose slices are contiguous) and streams their
+// token-head slices through a cp.async pipeline in its own shared memory,
+// across chain boundaries; while it computes on one stage the next ones are
+// in flight.  Warps never wait for each other.
+//
+//  * reduce pass   the chunk product Q_t = Q_{t-1} + (F_t + Q_{t-1} F_t)
+//                  (P = I + Q, X = I + F) on mma.sync m16n8k8 tf32 in split
+//                  precision; the state stays in the accumulator registers
+//                  from token to token (the contraction index of the next
+//                  product is permuted so that the accumulator fragment of
+//                  column tile j is exactly the A fragment of k-tile j).  In
+//                  the determinant-corrected mode with the identity added the
+//                  chain runs on the uncorrected matrices: the determinant is
+//                  multiplicative, so the product of the corrected matrices
+//                  is gamma P~ with gamma = |det P~|^(-1/16), one 16 x 16
+//                  factorisation per chunk.
+//                  Carry scan, in the same launch: after writing a chunk
+//                  total the warp counts itself in at the chunk's group of G
+//                  totals (an atomic counter); the last of a group scans the
+//                  group (inclusive in-group prefixes and the group total, in
+//                  fp64 on the tensor cores, mma.sync m8n8k4) and counts the
+//                  group total in one level up; the last at the top level
+//                  scans the top from S0 into exclusive carries.  No warp
+//                  waits for another: whoever completes a group does its scan.
+//  * apply pass    each chain's first stage brings the chain's carry factors
+//                  (the top carry and one in-group prefix per level), their
+//                  product is formed in fp64; per stage of 8 tokens the
+//                  determinant scales come from 8 LU factorisations at once
+//                  (4 lanes per token), then S_t = S_{t-1} + S_{t-1} F_t runs
+//                  from the carry and every S_t is written.  Per token·head
+//                  the path moves x twice and S once.
 //
 // Split-tf32 ("3xTF32", after Ootomo and Yokota, 2022): x = hi + lo with hi
-// the top 19 bits of x (sign, exponent, 10 mantissa bits) and lo = x - hi
-// exact in fp32; a b ~ a_lo b_hi + a_hi b_lo + a_hi b_hi.
+// x rounded to tf32 (sign, exponent, 10 mantissa bits) and lo = x - hi exact
+// in fp32; a b ~ a_lo b_hi + a_hi b_lo + a_hi b_hi.
 #include <string.h>
+
+#include <atomic>
 
 #include "mru_internal.cuh"
 
@@ -35,32 +51,73 @@ namespace {
 
 constexpr int N = 16;
 constexpr int NN = N * N;
-constexpr int ROWW = 20;            // padded shared-memory row stride, in words
-constexpr int SLICE = N * ROWW;     // one token-head slice in shared memory
-constexpr int SUB = kSub;           // tokens per pass
-constexpr int WARPS = 8;            // chains per CTA
-constexpr int THREADS = 32 * WARPS;
+constexpr unsigned FULL = 0xffffffffu;
 
+// Pipeline geometry.  Reduce: 4-token stages, three per warp, 8 warps a CTA
+// (2 CTAs per SM).  Apply: 8-token stages (one LU round per stage; a stage
+// also holds a chain's carry factors, at most 7 KB), two per warp, 4 warps a
+// CTA (3 CTAs per SM).
+constexpr int RST = 4, RNS = 3, RWARPS = 8;
+constexpr int AST = 8, ANS = 2, AWARPS = 4;
+
+template <int ST, int NS>
 struct WarpSmem {
-    float x[SUB][SLICE];            // 10,240 bytes
-    float2 cd[SUB];                 // (c * alpha, diagonal term of F) per token
+    float stage[NS][ST * NN];          // token slices (swizzled) or a chain's carry factors
+    float scratch[NN];                 // chunk product (reduce), carry (apply)
+    float2 cd[ST];                     // per token: (c alpha, diagonal term of F)
 };
+using RSmem = WarpSmem<RST, RNS>;      // 13,344 bytes
+using ASmem = WarpSmem<AST, ANS>;      // 17,472 bytes
+
+// Word offsets of the carry factors in an apply stage: top carry E (fp64),
+// then R_0 (fp32), R_1, R_2 (fp64).
+constexpr int CF_E = 0, CF_R0 = 2 * NN, CF_R1 = 3 * NN;
+static_assert(CF_R1 + 2 * 2 * NN <= AST * NN, "carry factors must fit one apply stage");
+
+// Word offset of element (row, col) of a token slice in shared memory: row
+// pairs form 128-byte lines of eight 16-byte granules, and granule j of line
+// l sits at j ^ 2 (l & 3).  The tensor-core fragment reads below are then
+// free of bank conflicts without padding the rows.
+__device__ __forceinline__ int swz(int row, int col)
+{
+    const int line = row >> 1;
+    const int gran = (((row & 1) << 2) | (col >> 2)) ^ ((line & 3) << 1);
+    return (line << 5) | (gran << 2) | (col & 3);
+}
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
 {
     const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int Pending>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(Pending));
+}
 
+// hi = v rounded to the nearest tf32 (ties away from zero: the magnitude
+// bits plus half a unit of the 10th mantissa bit, then truncated), lo = v - hi.
+// A truncated hi would leave every lo with the sign of v and bias the
+// dropped lo * lo terms; rounded, they average out.
 __device__ __forceinline__ void split_tf32(float v, uint32_t& hi, uint32_t& lo)
 {
-    const uint32_t h = __float_as_uint(v) & 0xffffe000u;
+    const uint32_t h = (__float_as_uint(v) + 0x1000u) & 0xffffe000u;
     hi = h;
     lo = __float_as_uint(v - __uint_as_float(h));
 }
 
-// D += A B, m16n8k8, tf32 operands, fp32 accumulate.
+// D = A B (+ 0), m16n8k8, tf32 operands, fp32 accumulate.
+__device__ __forceinline__ void mma_tf32_first(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2])
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};\n"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]), "f"(0.0f));
+}
+// D += A B.
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2])
 {
     asm volatile(
@@ -69,86 +126,70 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
-
-__device__ __forceinline__ void mma_3xtf32(float (&acc)[4], const uint32_t (&ah)[4], const uint32_t (&al)[4],
-                                           const uint32_t (&bh)[2], const uint32_t (&bl)[2])
+// D += A B, m8n8k4, fp64 throughout.
+__device__ __forceinline__ void mma_f64(double (&d)[2], double a, double b)
 {
-    mma_tf32(acc, al, bh);
-    mma_tf32(acc, ah, bl);
-    mma_tf32(acc, ah, bh);
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};\n"
+                 : "+d"(d[0]), "+d"(d[1])
+                 : "d"(a), "d"(b));
 }
 
-// log|det(W)| of one 16 x 16 matrix held by a group of 4 lanes (lane r owns
-// rows r, r+4, r+8, r+12 in e[0..3][0..15]).  near_identity: W = I + e,
-// eliminated on e alone without pivoting, |det| = prod |1 + delta_k| in fp64;
-// returns false when a pivot |1 + delta_k| < 0.5.  Otherwise W = e with
-// partial pivoting, log|det| summed in fp64.  Every lane of the warp must
-// call it with the same near_identity (the shuffles span the warp).
-__device__ __forceinline__ bool group_logabsdet(float (&e)[4][N], int r, bool near_identity, double& logabs,
-                                                bool& singular)
+// ---- per-token determinant scales ------------------------------------------
+
+// Rows r + (16 / R) lr of a 16 x 16 matrix, scale * value (+ I when
+// plus_i), from a swizzled token slice (stride 0) or rows `stride` words
+// apart.
+template <int R>
+__device__ __forceinline__ void load_rows(float (&e)[R][N], const float* src, int stride, int r, float scale,
+                                          bool plus_i)
 {
-    const unsigned full = 0xffffffffu;
+    constexpr int W = N / R;
+#pragma unroll
+    for (int lr = 0; lr < R; ++lr) {
+        const int i = W * lr + r;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+            const float4 v = *reinterpret_cast<const float4*>(src + (stride ? i * stride + 4 * c4 : swz(i, 4 * c4)));
+            e[lr][4 * c4 + 0] = scale * v.x + ((plus_i && i == 4 * c4 + 0) ? 1.0f : 0.0f);
+            e[lr][4 * c4 + 1] = scale * v.y + ((plus_i && i == 4 * c4 + 1) ? 1.0f : 0.0f);
+            e[lr][4 * c4 + 2] = scale * v.z + ((plus_i && i == 4 * c4 + 2) ? 1.0f : 0.0f);
+            e[lr][4 * c4 + 3] = scale * v.w + ((plus_i && i == 4 * c4 + 3) ? 1.0f : 0.0f);
+        }
+    }
+}
+
+__device__ __forceinline__ float rcp_approx(float v)
+{
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(r) : "f"(v));
+    return r;
+}
+
+// |det(I + e)| of one 16 x 16 matrix held by a group of 16 / R lanes (lane r
+// of the group owns rows r + (16 / R) lr, lr < R, in e[lr][0..15]),
+// eliminated on e alone without pivoting: prod |1 + delta_k| (fp64 product).
+// ok = false when a pivot |1 + delta_k| < 0.5.  All lanes of the warp call it
+// (the shuffles span the warp).
+template <int R>
+__device__ __forceinline__ double lu_near_identity(float (&e)[R][N], int r, bool& ok)
+{
+    constexpr int W = N / R;
     double prod = 1.0;
-    double lsum = 0.0;
-    bool ok = true;
-    singular = false;
+    ok = true;
 #pragma unroll
     for (int k = 0; k < N; ++k) {
-        const int kr = k >> 2, owner = k & 3;
-        if (!near_identity) {
-            float best = -1.0f;
-            int bi = k;
-#pragma unroll
-            for (int lr = 0; lr < 4; ++lr) {
-                const int i = 4 * lr + r;
-                const float a = fabsf(e[lr][k]);
-                if (i >= k && a > best) { best = a; bi = i; }
-            }
-#pragma unroll
-            for (int o = 1; o < 4; o <<= 1) {
-                const float ob = __shfl_xor_sync(full, best, o, 4);
-                const int oi = __shfl_xor_sync(full, bi, o, 4);
-                if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
-            }
-            if (!(best > 0.0f)) singular = true;
-            // swap rows k and bi (row i lives in lane i & 3, slot i >> 2);
-            // unconditional (a no-op when bi == k) to keep the warp converged
-            const int pr = bi >> 2, powner = bi & 3;
-#pragma unroll
-            for (int j = 0; j < N; ++j) {
-                float vk = 0.0f, vp = 0.0f;
-#pragma unroll
-                for (int lr = 0; lr < 4; ++lr) {
-                    if (lr == kr) vk = e[lr][j];
-                    if (lr == pr) vp = e[lr][j];
-                }
-                const float rowk = __shfl_sync(full, vk, owner, 4);
-                const float rowp = __shfl_sync(full, vp, powner, 4);
-#pragma unroll
-                for (int lr = 0; lr < 4; ++lr) {
-                    if (lr == kr && r == owner) e[lr][j] = rowp;
-                    if (lr == pr && r == powner) e[lr][j] = rowk;
-                }
-            }
-        }
+        const int kr = k / W, owner = k % W;
         float prow[N];
 #pragma unroll
-        for (int j = k; j < N; ++j) prow[j] = __shfl_sync(full, e[kr][j], owner, 4);
-        float pk;
-        if (near_identity) {
-            const float d = prow[k];
-            pk = 1.0f + d;
-            if (!(fabsf(pk) >= 0.5f)) ok = false;
-            prod *= 1.0 + (double)d;
-        } else {
-            pk = prow[k];
-            lsum += log(fabs((double)pk));
-        }
-        const float rk = (pk != 0.0f) ? __frcp_rn(pk) : 0.0f;
+        for (int j = k; j < N; ++j) prow[j] = __shfl_sync(FULL, e[kr][j], owner, W);
+        const float pk = 1.0f + prow[k];
+        if (!(fabsf(pk) >= 0.5f)) ok = false;
+        prod *= 1.0 + (double)prow[k];
+        const float rk = rcp_approx(pk);
 #pragma unroll
-        for (int lr = 0; lr < 4; ++lr) {
-            if (4 * lr + 3 <= k) continue;        // no row of this slot is below k
-            const int i = 4 * lr + r;
+        for (int lr = 0; lr < R; ++lr) {
+            if (W * lr + W - 1 <= k) continue;    // no row of this slot is below k
+            const int i = W * lr + r;
             if (i > k) {
                 const float l = e[lr][k] * rk;
 #pragma unroll
@@ -156,83 +197,150 @@ __device__ __forceinline__ bool group_logabsdet(float (&e)[4][N], int r, bool ne
             }
         }
     }
-    logabs = near_identity ? log(fabs(prod)) : lsum;
-    return ok;
+    return fabs(prod);
 }
 
-// Copies the slices of tokens [t0, t0 + nt) of one (b, h) into the warp's
-// shared memory (16-byte granules, rows padded to ROWW words).
-__device__ __forceinline__ void load_pass(WarpSmem& ws, const float* xb, int64_t tok, int64_t t0, int nt, int lane)
+struct LogDet {
+    double ld;        // log|det|, summed in fp64
+    bool singular;
+};
+
+// log|det(W)| with partial pivoting, W = scale * src (+ I when plus_i) loaded
+// here (same ownership of rows as lu_near_identity).  The fallback for
+// matrices far from the identity: kept out of line, off the hot path's
+// instruction footprint.
+template <int R>
+__device__ __noinline__ LogDet lu_pivoted(const float* src, int stride, int r, float scale, bool plus_i)
 {
+    constexpr int W = N / R;
+    float e[R][N];
+    load_rows<R>(e, src, stride, r, scale, plus_i);
+    LogDet out;
+    out.ld = 0.0;
+    out.singular = false;
 #pragma unroll
-    for (int i = 0; i < SUB * 64 / 32; ++i) {
-        const int gi = lane + 32 * i;
-        const int j = gi >> 6, q16 = gi & 63, row = q16 >> 2, col4 = q16 & 3;
-        if (j < nt) cp_async16(&ws.x[j][row * ROWW + col4 * 4], xb + (t0 + j) * tok + row * N + col4 * 4);
+    for (int k = 0; k < N; ++k) {
+        const int kr = k / W, owner = k % W;
+        float best = -1.0f;
+        int bi = k;
+#pragma unroll
+        for (int lr = 0; lr < R; ++lr) {
+            const int i = W * lr + r;
+            const float a = fabsf(e[lr][k]);
+            if (i >= k && a > best) { best = a; bi = i; }
+        }
+#pragma unroll
+        for (int o = 1; o < W; o <<= 1) {
+            const float ob = __shfl_xor_sync(FULL, best, o, W);
+            const int oi = __shfl_xor_sync(FULL, bi, o, W);
+            if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+        }
+        if (!(best > 0.0f)) out.singular = true;
+        // swap rows k and bi (row i lives in lane i % W, slot i / W);
+        // unconditional (a no-op when bi == k) to keep the warp converged
+        const int pr = bi / W, powner = bi % W;
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            float vk = 0.0f, vp = 0.0f;
+#pragma unroll
+            for (int lr = 0; lr < R; ++lr) {
+                if (lr == kr) vk = e[lr][j];
+                if (lr == pr) vp = e[lr][j];
+            }
+            const float rowk = __shfl_sync(FULL, vk, owner, W);
+            const float rowp = __shfl_sync(FULL, vp, powner, W);
+#pragma unroll
+            for (int lr = 0; lr < R; ++lr) {
+                if (lr == kr && r == owner) e[lr][j] = rowp;
+                if (lr == pr && r == powner) e[lr][j] = rowk;
+            }
+        }
+        float prow[N];
+#pragma unroll
+        for (int j = k; j < N; ++j) prow[j] = __shfl_sync(FULL, e[kr][j], owner, W);
+        const float pk = prow[k];
+        out.ld += log(fabs((double)pk));
+        const float rk = (pk != 0.0f) ? 1.0f / pk : 0.0f;
+#pragma unroll
+        for (int lr = 0; lr < R; ++lr) {
+            if (W * lr + W - 1 <= k) continue;
+            const int i = W * lr + r;
+            if (i > k) {
+                const float l = e[lr][k] * rk;
+#pragma unroll
+                for (int j = k + 1; j < N; ++j) e[lr][j] = fmaf(-l, prow[j], e[lr][j]);
+            }
+        }
     }
-    cp_async_wait_all();
-    __syncwarp();
+    return out;
 }
 
-// The per-token scalars of F = ca * M + dv * I for the 8 tokens of a pass:
-// 4-lane LU groups for the determinant-corrected mode.  Lane r == 0 of each
-// group writes ws.cd[group].
-__device__ __forceinline__ void pass_scalars(const KParams& p, WarpSmem& ws, int nt, int lane, uint32_t* status)
+// c - 1 = |det W|^(-1/16) - 1 for the matrix at src, W = scale * value
+// (+ I where plus_i), by the group of 16 / R lanes.  near (the same for the
+// whole warp: it selects code with full-warp shuffles) tries the
+// near-identity elimination first (W = I + e; fp32: |det| = 1 + u,
+// c - 1 = expm1(-log1p(u) / 16)); the pivoted one runs where any group of the
+// warp needs it.  singular: det W = 0 (or not finite).
+template <int R>
+__device__ __forceinline__ float det_scale_m1(const float* src, int stride, int r, float scale, bool near,
+                                              bool plus_i, bool& singular)
 {
-    const int grp = lane >> 2, r = lane & 3;
+    bool ok = false;
+    float cm1 = 0.0f;
+    singular = false;
+    if (near) {
+        float e[R][N];
+        load_rows<R>(e, src, stride, r, scale, false);
+        const double ad = lu_near_identity<R>(e, r, ok);
+        cm1 = expm1f(-log1pf((float)(ad - 1.0)) * (1.0f / N));
+    }
+    if (__any_sync(FULL, !ok)) {
+        __syncwarp();
+        const LogDet q = lu_pivoted<R>(src, stride, r, scale, plus_i);
+        if (!ok) {
+            singular = q.singular || !isfinite(q.ld);
+            cm1 = (float)expm1(-q.ld / N);
+        }
+    }
+    if (!isfinite(cm1) || cm1 <= -1.0f) singular = true;
+    return cm1;
+}
+
+// The per-token scalars of F = ca M + dv I for the nt (<= ST) tokens of a
+// stage, written to cd: one LU factorisation per token, 32 / ST lanes each,
+// in the determinant-corrected mode; the constants (alpha, 0 or -1)
+// otherwise.  A singular token sets the status bit and keeps X = I.
+template <int ST>
+__device__ __forceinline__ void stage_scalars(const KParams& p, float2* cd, const float* xs, int nt, int lane,
+                                              uint32_t* status)
+{
+    constexpr int R = N * ST / 32, W = N / R;
+    const int grp = lane / W, r = lane % W;
     const bool live = grp < nt;
     float ca = p.alpha, dv = p.add_identity ? 0.0f : -1.0f;
     if (p.mode == MRU_MODE_DETNORM) {
-        float e[4][N];
-        const float* xs = ws.x[grp];
-#pragma unroll
-        for (int lr = 0; lr < 4; ++lr) {
-            const float4* row4 = reinterpret_cast<const float4*>(xs + (4 * lr + r) * ROWW);
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                const float4 v = live ? row4[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
-                e[lr][4 * c4 + 0] = p.alpha * v.x;
-                e[lr][4 * c4 + 1] = p.alpha * v.y;
-                e[lr][4 * c4 + 2] = p.alpha * v.z;
-                e[lr][4 * c4 + 3] = p.alpha * v.w;
-            }
-        }
-        double ld = 0.0;
-        bool singular = false, ok = true;
-        if (p.add_identity) ok = group_logabsdet(e, r, true, ld, singular);
-        if (__any_sync(0xffffffffu, !p.add_identity || !ok)) {
-            const bool need = !p.add_identity || !ok;
-#pragma unroll
-            for (int lr = 0; lr < 4; ++lr) {
-                const int i = 4 * lr + r;
-#pragma unroll
-                for (int jj = 0; jj < N; ++jj)
-                    e[lr][jj] = live ? p.alpha * xs[i * ROWW + jj] + ((p.add_identity && i == jj) ? 1.0f : 0.0f)
-                                     : (i == jj ? 1.0f : 0.0f);
-            }
-            double ld2 = 0.0;
-            bool sing2 = false;
-            group_logabsdet(e, r, false, ld2, sing2);
-            if (need) { ld = ld2; singular = sing2; }
-        }
-        const double cm1d = expm1(-ld / N);
-        const float c = (float)(1.0 + cm1d);
-        if (singular || !isfinite(ld) || !isfinite(c) || c == 0.0f) {
+        // idle groups factorise I (scale 0, plus I)
+        bool singular = false;
+        const float cm1 = det_scale_m1<R>(xs + grp * NN, 0, r, live ? p.alpha : 0.0f, p.add_identity != 0,
+                                          p.add_identity || !live, singular);
+        if (singular) {
             if (live && r == 0) atomicOr(status, STATUS_SINGULAR);
             ca = 0.0f;                       // output unspecified; keep X = I
             dv = 0.0f;
         } else {
-            ca = c * p.alpha;
-            dv = p.add_identity ? (float)cm1d : -1.0f;
+            ca = (1.0f + cm1) * p.alpha;
+            dv = p.add_identity ? cm1 : -1.0f;
         }
     }
-    if (r == 0) ws.cd[grp] = make_float2(ca, dv);
+    if (r == 0) cd[grp] = make_float2(ca, dv);
     __syncwarp();
 }
 
-// B fragments (split) of F = ca * M + dv * I for one token, with the
-// contraction index permuted (slot q <-> row 8kt + 2q, slot q + 4 <-> row
-// 8kt + 2q + 1), and F at this lane's accumulator positions.
+// ---- the token chain (tf32 split, accumulator-resident state) -------------
+
+// B fragments (split) of F = ca M + dv I for one token, with the contraction
+// index permuted (slot q <-> row 8kt + 2q, slot q + 4 <-> row 8kt + 2q + 1),
+// and F at this lane's accumulator positions.
 struct FragF {
     uint32_t bh[2][2][2], bl[2][2][2];
     float fd[2][4];
@@ -245,9 +353,8 @@ __device__ __forceinline__ void make_frag_f(const float* xs, float ca, float d0,
     for (int kt = 0; kt < 2; ++kt)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-            const float* base = xs + (8 * kt + 2 * q) * ROWW + 8 * nt + g;
-            const float v0 = fmaf(ca, base[0], kt == nt ? d0 : 0.0f);
-            const float v1 = fmaf(ca, base[ROWW], kt == nt ? d1 : 0.0f);
+            const float v0 = fmaf(ca, xs[swz(8 * kt + 2 * q, 8 * nt + g)], kt == nt ? d0 : 0.0f);
+            const float v1 = fmaf(ca, xs[swz(8 * kt + 2 * q + 1, 8 * nt + g)], kt == nt ? d1 : 0.0f);
             split_tf32(v0, f.bh[kt][nt][0], f.bl[kt][nt][0]);
             split_tf32(v1, f.bh[kt][nt][1], f.bl[kt][nt][1]);
         }
@@ -256,14 +363,16 @@ __device__ __forceinline__ void make_frag_f(const float* xs, float ca, float d0,
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int h8 = 0; h8 < 2; ++h8) {
-                const float2 xv = *reinterpret_cast<const float2*>(xs + (g + 8 * h8) * ROWW + 8 * nt + 2 * q);
+                const float2 xv = *reinterpret_cast<const float2*>(xs + swz(g + 8 * h8, 8 * nt + 2 * q));
                 f.fd[nt][2 * h8 + 0] = fmaf(ca, xv.x, h8 == nt ? d0 : 0.0f);
                 f.fd[nt][2 * h8 + 1] = fmaf(ca, xv.y, h8 == nt ? d1 : 0.0f);
             }
     }
 }
 
-// acc = A F with A the 16 x 16 state held in accumulator layout (Ad).
+// acc = A F with A the 16 x 16 state held in accumulator layout (Ad).  The
+// four (column tile, k-tile) products accumulate separately and are summed
+// at the end, so that a token's dependent mma chain is three long, not six.
 __device__ __forceinline__ void chain_product(const float (&Ad)[2][4], const FragF& f, float (&acc)[2][4])
 {
     uint32_t ah[2][4], al[2][4];
@@ -274,13 +383,23 @@ __device__ __forceinline__ void chain_product(const float (&Ad)[2][4], const Fra
         split_tf32(Ad[kt][1], ah[kt][2], al[kt][2]);
         split_tf32(Ad[kt][3], ah[kt][3], al[kt][3]);
     }
+    float part[2][2][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+        for (int kt = 0; kt < 2; ++kt) mma_tf32_first(part[nt][kt], al[kt], f.bh[kt][nt]);
 #pragma unroll
-        for (int kt = 0; kt < 2; ++kt) mma_3xtf32(acc[nt], ah[kt], al[kt], f.bh[kt][nt], f.bl[kt][nt]);
-    }
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int kt = 0; kt < 2; ++kt) mma_tf32(part[nt][kt], ah[kt], f.bl[kt][nt]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int kt = 0; kt < 2; ++kt) mma_tf32(part[nt][kt], ah[kt], f.bh[kt][nt]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nt][i] = part[nt][0][i] + part[nt][1][i];
 }
 
 __device__ __forceinline__ void store_d(float* out, const float (&Ad)[2][4], int g, int q)
@@ -293,424 +412,581 @@ __device__ __forceinline__ void store_d(float* out, const float (&Ad)[2][4], int
                 make_float2(Ad[nt][2 * h8], Ad[nt][2 * h8 + 1]);
 }
 
-// chain id -> (b, k, h), h fastest: a CTA's chains are neighbouring heads of
-// one token range (their slices are contiguous in memory).
-struct ChainIx {
+// ---- fp64 16 x 16 products on the tensor cores (mma.sync m8n8k4) -----------
+//
+// A warp holds a 16 x 16 fp64 matrix in accumulator layout: lane (g, t)
+// (g = lane / 4, t = lane % 4) keeps M[8 mt + g][8 nb + 2 t + h] in
+// m[mt][nb][h] -- the same elements the tf32 accumulator layout gives the
+// lane.  As the A operand of the next product the contraction index is
+// permuted: k-tile kk = 2 nt + h, slot t <-> column 8 nt + 2 t + h.  The B
+// operand then holds, per k-tile kk and column tile nb, B[8 (kk / 2) + 2 t +
+// kk % 2][8 nb + g].
+
+template <typename T>
+struct M16 {
+    T m[2][2][2];
+};
+template <typename T>
+struct F16 {
+    T b[4][2];
+};
+using D16 = M16<double>;
+using B16 = F16<double>;
+
+__device__ __forceinline__ void d16_zero(D16& a)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) (&a.m[0][0][0])[i] = 0.0;
+}
+
+// acc += A B (B converted to fp64 as it is used).
+template <typename T>
+__device__ __forceinline__ void d16_mac(const D16& A, const F16<T>& B, D16& acc)
+{
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) mma_f64(acc.m[mt][nb], A.m[mt][kk >> 1][kk & 1], (double)B.b[kk][nb]);
+}
+
+// One row-major 16 x 16 matrix in shared memory as the B operand, in its own
+// precision.
+template <typename T>
+__device__ __forceinline__ void d16_load(const T* src, F16<T>& b, int lane)
+{
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) b.b[kk][nb] = src[(8 * (kk >> 1) + 2 * t + (kk & 1)) * N + 8 * nb + g];
+}
+
+// ---- carry scan (its own launch, between the passes) -----------------------
+//
+// One warp per group of G chunk totals.  The warp copies the group's items
+// into its shared memory (rows padded, one round of copies for up to 16
+// fp32 items or 8 fp64 ones), applies the per-chunk determinant correction
+// when the reduce pass left it (4-lane LU factorisations, 8 at once), and
+// scans them on the fp64 tensor cores.  Then it counts itself in at the
+// next level's group; the last warp of a group scans that one, and so on up
+// to the top, which is scanned from S0.  No warp waits for another.
+
+constexpr int CWARPS = 4;
+constexpr int CROW32 = 20;                  // padded row stride of staged fp32 items (words)
+constexpr int CROW64 = 18;                  // padded row stride of staged fp64 items (doubles)
+constexpr int CRB32 = 16, CRB64 = 8;        // items per staging round
+struct CSmem {
+    float buf[CRB32 * N * CROW32];          // 20,480 bytes
+    float2 gam[CRB32];                      // per staged item: (gamma, gamma - 1)
+};
+static_assert(CRB64 * N * CROW64 * sizeof(double) <= sizeof(float) * CRB32 * N * CROW32, "fp64 round fits");
+
+template <typename T> struct Stage;
+template <> struct Stage<float> {
+    static constexpr int RB = CRB32, ROW = CROW32;
+};
+template <> struct Stage<double> {
+    static constexpr int RB = CRB64, ROW = CROW64;
+};
+
+// Copies items [0, cnt) of src (row-major 16 x 16) into buf, rows padded.
+template <typename T>
+__device__ __forceinline__ void stage_items(T* buf, const T* src, int cnt, int lane)
+{
+    constexpr int GR = N * (int)sizeof(T) / 16;              // 16-byte granules per row
+    constexpr int ROW = Stage<T>::ROW;
+    for (int gi = lane; gi < cnt * N * GR; gi += 32) {
+        const int item = gi / (N * GR), rem = gi % (N * GR), row = rem / GR, c = rem % GR;
+        constexpr int PER = 16 / (int)sizeof(T);
+        cp_async16(buf + (item * N + row) * ROW + c * PER, src + (int64_t)item * NN + row * N + c * PER);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncwarp();
+}
+
+// gamma_j = |det(I + Q~_j)|^(-1/16) for the cnt staged fp32 items, 4 lanes
+// per item, 8 at once (a singular one gets gamma = 0: the apply pass flags
+// its token).
+__device__ __forceinline__ void stage_gammas(CSmem& sm, int cnt, int lane)
+{
+    const int grp = lane >> 2, r = lane & 3;
+    for (int b0 = 0; b0 < cnt; b0 += 8) {
+        const int item = b0 + grp;
+        const bool live = item < cnt;
+        bool singular = false;
+        const float gm1 = det_scale_m1<4>(sm.buf + (live ? item : 0) * N * CROW32, CROW32, r, live ? 1.0f : 0.0f,
+                                          true, true, singular);
+        if (live && r == 0) sm.gam[item] = singular ? make_float2(0.0f, -1.0f) : make_float2(1.0f + gm1, gm1);
+    }
+    __syncwarp();
+}
+
+// Staged item j as the B operand (and in accumulator layout), gamma T + (gamma - 1) I.
+template <typename T>
+__device__ __forceinline__ void load_staged(const T* buf, int j, double gm, double gm1, B16& b, D16& a, int lane)
+{
+    constexpr int ROW = Stage<T>::ROW;
+    const int g = lane >> 2, t = lane & 3;
+    const T* it = buf + j * N * ROW;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+            const int row = 8 * (kk >> 1) + 2 * t + (kk & 1), col = 8 * nb + g;
+            b.b[kk][nb] = gm * (double)it[row * ROW + col] + (row == col ? gm1 : 0.0);
+        }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int row = 8 * mt + g, col = 8 * nb + 2 * t + h;
+                a.m[mt][nb][h] = gm * (double)it[row * ROW + col] + (row == col ? gm1 : 0.0);
+            }
+}
+
+template <typename T>
+__device__ __forceinline__ void store_acc(T* dst, const D16& a, int lane)
+{
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) dst[(8 * mt + g) * N + 8 * nb + 2 * t + h] = (T)a.m[mt][nb][h];
+}
+
+// Scans the m split-form items at in: Top, the exclusive carries E_0 = S0
+// (or I), E_{j+1} = E_j (I + T_j) to E; otherwise the inclusive prefixes
+// R_j = R_{j-1} + (T_j + R_{j-1} T_j) to R and the last one to tot.
+// correct: the items still need their determinant correction (fp32 only).
+template <typename Tin, bool Top, typename Tout>
+__device__ __forceinline__ void staged_scan(CSmem& sm, const Tin* in, int m, bool correct, const float* S0,
+                                            double* E, Tout* R, double* tot, int lane)
+{
+    constexpr int RB = Stage<Tin>::RB;
+    Tin* buf = reinterpret_cast<Tin*>(sm.buf);
+    D16 st, acc, Ta;
+    B16 Bf;
+    if (Top) {
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int row = 8 * mt + g, col = 8 * nb + 2 * t + h;
+                    st.m[mt][nb][h] = S0 ? (double)S0[row * N + col] : (row == col ? 1.0 : 0.0);
+                }
+    } else {
+        d16_zero(st);
+    }
+    for (int j0 = 0; j0 < m; j0 += RB) {
+        const int cnt = (m - j0 < RB) ? m - j0 : RB;
+        __syncwarp();
+        stage_items(buf, in + (int64_t)j0 * NN, cnt, lane);
+        if (correct) stage_gammas(sm, cnt, lane);
+        for (int j = 0; j < cnt; ++j) {
+            double gm = 1.0, gm1 = 0.0;
+            if (correct) {
+                const float2 gg = sm.gam[j];
+                gm = (double)gg.x;
+                gm1 = (double)gg.y;
+            }
+            load_staged(buf, j, gm, gm1, Bf, Ta, lane);
+            if (Top) {
+                store_acc(E + (int64_t)(j0 + j) * NN, st, lane);
+                acc = st;                              // E_j + E_j T_j
+                d16_mac(st, Bf, acc);
+                st = acc;
+            } else {
+                acc = Ta;                              // T_j + R_{j-1} T_j
+                d16_mac(st, Bf, acc);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) (&st.m[0][0][0])[i] += (&acc.m[0][0][0])[i];
+                store_acc(R + (int64_t)(j0 + j) * NN, st, lane);
+            }
+        }
+    }
+    if (!Top) store_acc(tot, st, lane);
+}
+
+// Counts the warp in at a counter whose group has `target` members; true for
+// the last one.  The fences order this warp's earlier stores before the count
+// and the last one's later loads after it.
+__device__ __forceinline__ bool arrive(unsigned* ctr, unsigned target, int lane)
+{
+    __threadfence();
+    __syncwarp();
+    unsigned old = 0;
+    if (lane == 0) old = atomicAdd(ctr, 1u);
+    old = __shfl_sync(FULL, old, 0);
+    const bool last = old + 1 == target;
+    if (last) __threadfence();
+    return last;
+}
+
+// One warp per group of level 0 (per sequence when the chunk totals are the
+// top level already), then up the levels as the last arriver.
+__global__ void __launch_bounds__(CWARPS * 32)
+k16_carry(KParams p, const float* __restrict__ totals, CarryPlan cp, char* ws, const float* __restrict__ S0)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    CSmem& sm = reinterpret_cast<CSmem*>(smem_raw)[warp];
+    const bool correct = p.mode == MRU_MODE_DETNORM && p.add_identity;
+    const int64_t per_seq = cp.levels > 0 ? cp.cnt[1] : 1;
+    const int64_t unit = (int64_t)blockIdx.x * CWARPS + warp;
+    if (unit >= cp.nseq * per_seq) return;
+    const int64_t seq = unit / per_seq;
+    const float* s0 = S0 ? S0 + seq * NN : nullptr;
+    if (cp.levels == 0) {
+        const int64_t m = cp.cnt[0];
+        staged_scan<float, true, double>(sm, totals + seq * m * NN, (int)m, correct, s0,
+                                         reinterpret_cast<double*>(ws + cp.Etop) + seq * m * NN, nullptr, nullptr,
+                                         lane);
+        return;
+    }
+    int64_t gi = unit % per_seq;
+    for (int l = 0; l < cp.levels; ++l) {
+        if (l > 0) {
+            const int64_t item = gi;
+            gi = item >> cp.gshift;
+            const int64_t m = (cp.cnt[l] - (gi << cp.gshift) < cp.G) ? cp.cnt[l] - (gi << cp.gshift) : cp.G;
+            unsigned* ctr = reinterpret_cast<unsigned*>(ws + cp.ctr[l]) + seq * cp.cnt[l + 1] + gi;
+            if (!arrive(ctr, (unsigned)m, lane)) return;
+        }
+        const int64_t first = seq * cp.cnt[l] + (gi << cp.gshift);
+        const int64_t m = (cp.cnt[l] - (gi << cp.gshift) < cp.G) ? cp.cnt[l] - (gi << cp.gshift) : cp.G;
+        double* tot = reinterpret_cast<double*>(ws + cp.Tot[l]) + (seq * cp.cnt[l + 1] + gi) * NN;
+        if (l == 0)
+            staged_scan<float, false, float>(sm, totals + first * NN, (int)m, correct, nullptr, nullptr,
+                                             reinterpret_cast<float*>(ws + cp.R[0]) + first * NN, tot, lane);
+        else
+            staged_scan<double, false, double>(sm, reinterpret_cast<const double*>(ws + cp.Tot[l - 1]) + first * NN,
+                                               (int)m, false, nullptr, nullptr,
+                                               reinterpret_cast<double*>(ws + cp.R[l]) + first * NN, tot, lane);
+    }
+    const int64_t m = cp.cnt[cp.levels];
+    unsigned* ctr = reinterpret_cast<unsigned*>(ws + cp.ctr[cp.levels]) + seq;
+    if (!arrive(ctr, (unsigned)m, lane)) return;
+    staged_scan<double, true, double>(sm, reinterpret_cast<const double*>(ws + cp.Tot[cp.levels - 1]) + seq * m * NN,
+                                      (int)m, false, s0, reinterpret_cast<double*>(ws + cp.Etop) + seq * m * NN,
+                                      nullptr, nullptr, lane);
+}
+
+// ---- chains and the stage feed ---------------------------------------------
+
+// chain id -> (b, k, h), h fastest (chain ids stay below 2^31).
+struct Chain {
     int64_t b, h, k, tbeg, tend;
 };
-__device__ __forceinline__ ChainIx chain_ix(const KParams& p, int64_t chain)
+__device__ __forceinline__ Chain chain_at(const KParams& p, int64_t chain)
 {
-    ChainIx c;
-    c.h = chain % p.H;
-    const int64_t bk = chain / p.H;
-    c.k = bk % p.K;
-    c.b = bk / p.K;
+    Chain c;
+    const uint32_t ci = (uint32_t)chain;
+    const uint32_t bk = fastdiv(ci, p.h_mul, p.h_shr);
+    const uint32_t b = fastdiv(bk, p.k_mul, p.k_shr);
+    c.h = ci - bk * (uint32_t)p.H;
+    c.k = bk - b * (uint32_t)p.K;
+    c.b = b;
     c.tbeg = c.k * p.chunk;
     c.tend = (c.tbeg + p.chunk < p.L) ? c.tbeg + p.chunk : p.L;
     return c;
 }
 
-// ---- chain bodies, shared by the two-pass kernels and the fused kernel ----
+// The producer side of a warp's pipeline: the next stage to copy, along the
+// warp's chains.  Apply: a chain's first stage is its carry factors.
+template <bool Apply, int ST>
+struct Feed {
+    int64_t chain, stride, nchains, tok;
+    int64_t t, tend;
+    const float* xb;
+    // carry factors (apply): top carry, and per level the in-group prefix
+    // before this chain's item (null for the first item of a group)
+    const double* E;
+    const void* Rf[kCarryLevels];
+    bool carry_next;
 
-// The reduce chain of one warp over tokens [tbeg, tend): per-token scalars to
-// cdb[t * H] and the chunk total (split form) left in Qd.
-__device__ __forceinline__ void reduce_chain(const KParams& p, WarpSmem& ws, const float* xb, int64_t tok,
-                                             float2* cdb, int64_t tbeg, int64_t tend, int lane, uint32_t* status,
-                                             float (&Qd)[2][4])
+    __device__ __forceinline__ void set(const KParams& p, const float* x, const CarryPlan& cp, const char* ws)
+    {
+        if (chain >= nchains) return;
+        const Chain c = chain_at(p, chain);
+        xb = x + (c.b * p.L * p.H + c.h) * NN;
+        t = c.tbeg;
+        tend = c.tend;
+        if (Apply) {
+            const int64_t seq = c.b * p.H + c.h;
+            int64_t i = c.k;
+#pragma unroll
+            for (int l = 0; l < kCarryLevels; ++l) {
+                Rf[l] = nullptr;
+                if (l < cp.levels) {
+                    if (i & (cp.G - 1)) {
+                        const size_t esz = l == 0 ? sizeof(float) : sizeof(double);
+                        Rf[l] = ws + cp.R[l] + (size_t)((seq * cp.cnt[l] + i - 1) * NN) * esz;
+                    }
+                    i >>= cp.gshift;
+                }
+            }
+            E = reinterpret_cast<const double*>(ws + cp.Etop) + (seq * cp.cnt[cp.levels] + i) * NN;
+            carry_next = true;
+        }
+    }
+
+    // Copies the next stage into dst (nothing once the chains are done) and
+    // commits a cp.async group either way.
+    __device__ __forceinline__ void issue(float* dst, int lane, const KParams& p, const float* x,
+                                          const CarryPlan& cp, const char* ws)
+    {
+        if (chain < nchains) {
+            if (Apply && carry_next) {
+                const char* E8 = reinterpret_cast<const char*>(E);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) cp_async16(dst + CF_E + 4 * (lane + 32 * i), E8 + 16 * (lane + 32 * i));
+                if (Rf[0]) {
+                    const char* r8 = reinterpret_cast<const char*>(Rf[0]);
+#pragma unroll
+                    for (int i = 0; i < 2; ++i)
+                        cp_async16(dst + CF_R0 + 4 * (lane + 32 * i), r8 + 16 * (lane + 32 * i));
+                }
+#pragma unroll
+                for (int l = 1; l < kCarryLevels; ++l)
+                    if (Rf[l]) {
+                        const char* r8 = reinterpret_cast<const char*>(Rf[l]);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            cp_async16(dst + CF_R1 + 2 * NN * (l - 1) + 4 * (lane + 32 * i), r8 + 16 * (lane + 32 * i));
+                    }
+                carry_next = false;
+            } else {
+                const int nt = (tend - t < ST) ? (int)(tend - t) : ST;
+#pragma unroll
+                for (int i = 0; i < ST * 2; ++i) {     // 64 granules a slice, 2 per lane
+                    const int gi = lane + 32 * i;
+                    const int j = gi >> 6, gr = gi & 63, row = gr >> 2, c4 = gr & 3;
+                    if (j < nt) cp_async16(dst + j * NN + swz(row, 4 * c4), xb + (t + j) * tok + row * N + 4 * c4);
+                }
+                t += ST;
+                if (t >= tend) {
+                    chain += stride;
+                    set(p, x, cp, ws);
+                }
+            }
+        }
+        cp_async_commit();
+    }
+};
+
+// The chain's carry C = E (I + R_{levels-1}) ... (I + R_0) in fp64 (factors
+// absent for the first item of a group skipped), rounded to fp32 into
+// accumulator layout Sd; in = the carry stage.
+__device__ __forceinline__ void form_carry(const float* in, const CarryPlan& cp, int64_t k, int lane,
+                                           float (&Sd)[2][4])
 {
+    D16 C, acc;
+    {
+        const double* sE = reinterpret_cast<const double*>(in + CF_E);
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+                const double2 v = *reinterpret_cast<const double2*>(sE + (8 * mt + g) * N + 8 * nb + 2 * t);
+                C.m[mt][nb][0] = v.x;
+                C.m[mt][nb][1] = v.y;
+            }
+    }
+    for (int l = cp.levels - 1; l >= 0; --l) {
+        if (((k >> (cp.gshift * l)) & (cp.G - 1)) == 0) continue;
+        acc = C;                                   // C (I + R_l)
+        if (l == 0) {
+            F16<float> Bf;
+            d16_load(in + CF_R0, Bf, lane);
+            d16_mac(C, Bf, acc);
+        } else {
+            B16 Bf;
+            d16_load(reinterpret_cast<const double*>(in + CF_R1 + 2 * NN * (l - 1)), Bf, lane);
+            d16_mac(C, Bf, acc);
+        }
+        C = acc;
+    }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) Sd[nb][2 * mt + h] = (float)C.m[mt][nb][h];
+}
+
+// ---- kernels ----------------------------------------------------------------
+
+// Reduce pass: chunk totals (split form).  With PerToken (the corrected mode
+// without the identity, whose uncorrected products alpha M could leave the
+// fp32 range) the chain takes every token's scale as it goes; otherwise it
+// runs on the uncorrected matrices and the carry kernel applies the
+// determinant correction of each total.  CTA 0 also zeroes the carry scan's
+// counters (the carry kernel runs after this launch).
+template <bool PerToken>
+__global__ void __launch_bounds__(RWARPS * 32, 2)
+k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, unsigned* ctr, int64_t nctr,
+           uint32_t* status)
+{
+    if (blockIdx.x == 0)
+        for (int64_t i = threadIdx.x; i < nctr; i += blockDim.x) ctr[i] = 0u;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    RSmem& sm = reinterpret_cast<RSmem*>(smem_raw)[warp];
+    const int64_t nchains = p.B * p.H * p.K;
+    const int64_t first = (int64_t)blockIdx.x * RWARPS + warp, stride = (int64_t)gridDim.x * RWARPS;
     const int g = lane >> 2, q = lane & 3;
     const float m0 = (g == 2 * q) ? 1.0f : 0.0f;         // diagonal positions of this lane's fragments
     const float m1 = (g == 2 * q + 1) ? 1.0f : 0.0f;
+    Feed<false, RST> feed;
+    feed.chain = first;
+    feed.stride = stride;
+    feed.nchains = nchains;
+    feed.tok = p.H * NN;
+    const CarryPlan nocp = {};            // the reduce feed reads no carry factors
+    feed.set(p, x, nocp, nullptr);
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int s = 0; s < RNS - 1; ++s) feed.issue(sm.stage[s], lane, p, x, nocp, nullptr);
+    int cs = 0, ps = RNS - 1;
+    for (int64_t chain = first; chain < nchains; chain += stride) {
+        const Chain c = chain_at(p, chain);
+        float Qd[2][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) Qd[nt][i] = 0.0f;
-    for (int64_t t0 = tbeg; t0 < tend; t0 += SUB) {
-        const int nt_pass = (tend - t0 < SUB) ? (int)(tend - t0) : SUB;
-        load_pass(ws, xb, tok, t0, nt_pass, lane);
-        pass_scalars(p, ws, nt_pass, lane, status);
-        if (lane < nt_pass) cdb[(t0 + lane) * p.H] = ws.cd[lane];
-        for (int j = 0; j < nt_pass; ++j) {
-            const float2 cdj = ws.cd[j];
-            FragF f;
-            make_frag_f(ws.x[j], cdj.x, m0 * cdj.y, m1 * cdj.y, g, q, f, true);
-            float acc[2][4];
-            chain_product(Qd, f, acc);
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int i = 0; i < 4; ++i) Qd[nt][i] = 0.0f;
+        for (int64_t t0 = c.tbeg; t0 < c.tend; t0 += RST) {
+            feed.issue(sm.stage[ps], lane, p, x, nocp, nullptr);
+            ps = (ps + 1 == RNS) ? 0 : ps + 1;
+            cp_async_wait<RNS - 1>();
+            __syncwarp();
+            const float* xs = sm.stage[cs];
+            const int nt = (c.tend - t0 < RST) ? (int)(c.tend - t0) : RST;
+            float ca = p.alpha, dv = p.add_identity ? 0.0f : -1.0f;
+            if (PerToken) stage_scalars<RST>(p, sm.cd, xs, nt, lane, status);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) Qd[nt][i] += f.fd[nt][i] + acc[nt][i];
-        }
-        __syncwarp();
-    }
-}
-
-// The chain's carry C = E (I + R) in fp64 (R may be null: C = E), rounded to
-// fp32, into accumulator layout Sd.  Uses the warp's x buffer as scratch.
-__device__ __forceinline__ void form_carry(WarpSmem& ws, const double* E, const float* R, int lane,
-                                           float (&Sd)[2][4])
-{
-    double* sE = reinterpret_cast<double*>(&ws.x[0][0]);      // 2 KB
-    float* sC = reinterpret_cast<float*>(&ws.x[2][0]);        // 1 KB
-    for (int e = lane; e < NN; e += 32) sE[e] = E[e];
-    __syncwarp();
-    const int r0 = (lane >> 2) * 2, c0 = (lane & 3) * 4;
-    double acc[2][4];
+            for (int j = 0; j < RST; ++j) {
+                if (j < nt) {
+                    if (PerToken) {
+                        const float2 cdj = sm.cd[j];
+                        ca = cdj.x;
+                        dv = cdj.y;
+                    }
+                    FragF f;
+                    make_frag_f(xs + j * NN, ca, m0 * dv, m1 * dv, g, q, f, true);
+                    float acc[2][4];
+                    chain_product(Qd, f, acc);
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+                    for (int n2 = 0; n2 < 2; ++n2)
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) acc[i][cc] = 0.0;
-    if (R) {
-#pragma unroll 4
-        for (int kk = 0; kk < N; ++kk) {
-            const double a0 = sE[r0 * N + kk], a1 = sE[(r0 + 1) * N + kk];
-            const float4 rv = *reinterpret_cast<const float4*>(R + kk * N + c0);
-            const double bv[4] = {(double)rv.x, (double)rv.y, (double)rv.z, (double)rv.w};
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                acc[0][cc] = fma(a0, bv[cc], acc[0][cc]);
-                acc[1][cc] = fma(a1, bv[cc], acc[1][cc]);
+                        for (int i = 0; i < 4; ++i) Qd[n2][i] += f.fd[n2][i] + acc[n2][i];
+                }
             }
+            __syncwarp();
+            cs = (cs + 1 == RNS) ? 0 : cs + 1;
         }
+        store_d(totals + ((c.b * p.H + c.h) * p.K + c.k) * NN, Qd, g, q);
     }
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-            sC[(r0 + i) * N + c0 + cc] = (float)(sE[(r0 + i) * N + c0 + cc] + acc[i][cc]);
-    __syncwarp();
-    const int g = lane >> 2, q = lane & 3;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int h8 = 0; h8 < 2; ++h8) {
-            const float2 v = *reinterpret_cast<const float2*>(sC + (g + 8 * h8) * N + 8 * nt + 2 * q);
-            Sd[nt][2 * h8] = v.x;
-            Sd[nt][2 * h8 + 1] = v.y;
-        }
-    __syncwarp();
 }
 
-// The apply chain of one warp: S_t = S_{t-1} + S_{t-1} F_t from Sd, every
-// S_t written to ob + t * tok.
-__device__ __forceinline__ void apply_chain(WarpSmem& ws, const float* xb, float* ob, int64_t tok, int64_t H,
-                                            const float2* cdb, int64_t tbeg, int64_t tend, int lane,
-                                            float (&Sd)[2][4])
+// Apply pass: per chain the carry from the carry scan's factors, then
+// S_t = S_{t-1} + S_{t-1} F_t from S = carry, every S_t written, with the
+// per-token determinant scales factorised here.
+__global__ void __launch_bounds__(AWARPS * 32, 3)
+k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, float* __restrict__ S_out,
+          uint32_t* status)
 {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    ASmem& sm = reinterpret_cast<ASmem*>(smem_raw)[warp];
+    const int64_t nchains = p.B * p.H * p.K;
+    const int64_t first = (int64_t)blockIdx.x * AWARPS + warp, stride = (int64_t)gridDim.x * AWARPS;
+    const int64_t tok = p.H * NN;
     const int g = lane >> 2, q = lane & 3;
     const float m0 = (g == 2 * q) ? 1.0f : 0.0f;
     const float m1 = (g == 2 * q + 1) ? 1.0f : 0.0f;
-    for (int64_t t0 = tbeg; t0 < tend; t0 += SUB) {
-        const int nt_pass = (tend - t0 < SUB) ? (int)(tend - t0) : SUB;
-        // the pass's per-token scalars travel with the slice copies (they
-        // would otherwise be a dependent global load per token)
-        if (lane < nt_pass) ws.cd[lane] = cdb[(t0 + lane) * H];
-        load_pass(ws, xb, tok, t0, nt_pass, lane);
-        for (int j = 0; j < nt_pass; ++j) {
-            const float2 cdj = ws.cd[j];
-            FragF f;
-            make_frag_f(ws.x[j], cdj.x, m0 * cdj.y, m1 * cdj.y, g, q, f, false);
-            float acc[2][4];
-            chain_product(Sd, f, acc);
+    Feed<true, AST> feed;
+    feed.chain = first;
+    feed.stride = stride;
+    feed.nchains = nchains;
+    feed.tok = tok;
+    feed.set(p, x, cp, ws);
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) Sd[nt][i] += acc[nt][i];
-            store_d(ob + (t0 + j) * tok, Sd, g, q);
-        }
+    for (int s = 0; s < ANS - 1; ++s) feed.issue(sm.stage[s], lane, p, x, cp, ws);
+    int cs = 0, ps = ANS - 1;
+    for (int64_t chain = first; chain < nchains; chain += stride) {
+        const Chain c = chain_at(p, chain);
+        float Sd[2][4];
+        feed.issue(sm.stage[ps], lane, p, x, cp, ws);
+        ps = (ps + 1 == ANS) ? 0 : ps + 1;
+        cp_async_wait<ANS - 1>();
         __syncwarp();
-    }
-}
-
-// Reduce pass: chunk totals (split form) and per-token scalars.
-__global__ void __launch_bounds__(THREADS, 2)
-k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, float2* __restrict__ cd_out,
-           uint32_t* status)
-{
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    WarpSmem& ws = reinterpret_cast<WarpSmem*>(smem_raw)[warp];
-    const int64_t chain = (int64_t)blockIdx.x * WARPS + warp;
-    if (chain >= p.B * p.H * p.K) return;
-    const ChainIx c = chain_ix(p, chain);
-    const int64_t tok = p.H * NN;
-    const float* xb = x + (c.b * p.L * p.H + c.h) * NN;
-    float2* cdb = cd_out + c.b * p.L * p.H + c.h;
-    float Qd[2][4];
-    reduce_chain(p, ws, xb, tok, cdb, c.tbeg, c.tend, lane, status, Qd);
-    store_d(totals + ((c.b * p.H + c.h) * p.K + c.k) * NN, Qd, lane >> 2, lane & 3);
-}
-
-// Apply pass: the chunk's carry C = E1 (I + R0[k-1]) in fp64, then
-// S_t = S_{t-1} + S_{t-1} F_t from S = C, every S_t written.
-__global__ void __launch_bounds__(THREADS, 2)
-k16_apply(KParams p, const float* __restrict__ x, const float2* __restrict__ cd_in, const float* __restrict__ R0,
-          const double* __restrict__ E1, int G, float* __restrict__ S_out)
-{
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    WarpSmem& ws = reinterpret_cast<WarpSmem*>(smem_raw)[warp];
-    const int64_t chain = (int64_t)blockIdx.x * WARPS + warp;
-    if (chain >= p.B * p.H * p.K) return;
-    const ChainIx c = chain_ix(p, chain);
-    const int64_t seq = c.b * p.H + c.h;
-    const int64_t n1 = (p.K + G - 1) / G;
-    float Sd[2][4];
-    form_carry(ws, E1 + (seq * n1 + c.k / G) * NN, (c.k % G) ? R0 + (seq * p.K + c.k - 1) * NN : nullptr, lane, Sd);
-    const int64_t tok = p.H * NN;
-    apply_chain(ws, x + (c.b * p.L * p.H + c.h) * NN, S_out + (c.b * p.L * p.H + c.h) * NN, tok, p.H,
-                cd_in + c.b * p.L * p.H + c.h, c.tbeg, c.tend, lane, Sd);
-}
-
-// ---- fused persistent kernel --------------------------------------------
-//
-// One launch runs the whole scan as a dataflow of work items over windows of
-// Kw chunks (all sequences), taken in ticket order from a global counter:
-//     R(0) .. R(lag-1), then per window w:  R(w+lag), S1(w), S2(w), A(w)
-//   R(w)   reduce chains of window w: chunk totals + per-token scalars
-//   S1(w)  per (sequence, group of G chunks): fp64 inclusive local prefixes
-//          R0 (kept fp32) and the group total Tot (fp64)
-//   S2(w)  per sequence: exclusive group carries E1 from the running carry
-//          (fp64), which it hands on to S2(w+1)
-//   A(w)   apply chains of window w from their exact carries, S_t written
-// An item only waits for items with smaller tickets (S1(w) for all R(w),
-// S2(w) for all S1(w) and S2(w-1), A(w) for S2(w)); those are held by CTAs
-// that are running, so the waits end.  Each wait is bounded: past the limit
-// the kernel records STATUS_TIMEOUT, raises the abort flag and returns.
-// Windows are sized so that the embeddings of the lag + 1 windows in flight
-// stay in L2, where the apply pass reads them the second time.
-
-constexpr unsigned kSpinLimit = 4u << 20;     // x up to ~1 us of back-off: a few seconds
-
-struct FusedCfg {
-    int G;              // chunks per group
-    int Kw;             // chunks per window (multiple of G)
-    int lag;            // windows the reduce items run ahead
-    int64_t NW;         // windows
-    int64_t nR, nS1, nS2, nA;
-    int64_t total;      // tickets
-    int64_t NG;         // groups per sequence
-};
-
-struct FusedBufs {
-    unsigned* ticket;
-    unsigned* abort_flag;
-    unsigned* cntR;     // [NW]
-    unsigned* cntS1;    // [NW]
-    unsigned* cntS2;    // [NW]
-    float* totals;      // [seq][K]
-    float2* cd;         // [B][L][H]
-    float* R0;          // [seq][K]
-    double* Tot;        // [seq][NG]
-    double* E1;         // [seq][NG]
-    double* cstate;     // [seq]
-    uint32_t* status;
-};
-
-__device__ __forceinline__ unsigned ld_volatile(const unsigned* p)
-{
-    return *reinterpret_cast<const volatile unsigned*>(p);
-}
-
-// Called by thread 0 only.  True once *ctr >= target; false on timeout or
-// when another CTA has aborted.
-__device__ bool wait_geq(const unsigned* ctr, unsigned target, const FusedBufs& fb)
-{
-    unsigned ns = 32;
-    for (unsigned spins = 0;; ++spins) {
-        if (ld_volatile(ctr) >= target) {
-            __threadfence();
-            return true;
-        }
-        if (ld_volatile(fb.abort_flag)) return false;
-        if (spins >= kSpinLimit) {
-            atomicOr(fb.status, STATUS_TIMEOUT);
-            atomicExch(fb.abort_flag, 1u);
-            return false;
-        }
-        __nanosleep(ns);
-        if (ns < 1024) ns <<= 1;
-    }
-}
-
-// C = A B for 16 x 16 fp64 matrices in shared memory; lane owns a 2 x 4 block.
-__device__ __forceinline__ void warp_gemm16_f64(const double* A, const double* B, int lane, double (&acc)[2][4])
-{
-    const int r0 = (lane >> 2) * 2, c0 = (lane & 3) * 4;
+        form_carry(sm.stage[cs], cp, c.k, lane, Sd);
+        __syncwarp();
+        cs = (cs + 1 == ANS) ? 0 : cs + 1;
+        float* ob = S_out + (c.b * p.L * p.H + c.h) * NN;
+        for (int64_t t0 = c.tbeg; t0 < c.tend; t0 += AST) {
+            feed.issue(sm.stage[ps], lane, p, x, cp, ws);
+            ps = (ps + 1 == ANS) ? 0 : ps + 1;
+            cp_async_wait<ANS - 1>();
+            __syncwarp();
+            const float* xs = sm.stage[cs];
+            const int nt = (c.tend - t0 < AST) ? (int)(c.tend - t0) : AST;
+            stage_scalars<AST>(p, sm.cd, xs, nt, lane, status);
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+            for (int j = 0; j < AST; ++j) {
+                if (j < nt) {
+                    const float2 cdj = sm.cd[j];
+                    FragF f;
+                    make_frag_f(xs + j * NN, cdj.x, m0 * cdj.y, m1 * cdj.y, g, q, f, false);
+                    float acc[2][4];
+                    chain_product(Sd, f, acc);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[i][c] = 0.0;
-#pragma unroll 4
-    for (int k = 0; k < N; ++k) {
-        const double a0 = A[r0 * N + k], a1 = A[(r0 + 1) * N + k];
+                    for (int n2 = 0; n2 < 2; ++n2)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const double b = B[k * N + c0 + c];
-            acc[0][c] = fma(a0, b, acc[0][c]);
-            acc[1][c] = fma(a1, b, acc[1][c]);
-        }
-    }
-}
-
-// chain index inside window w -> global chain coordinates (h fastest, then
-// the chunk within the window, then b); false when outside the problem.
-__device__ __forceinline__ bool window_chain(const KParams& p, const FusedCfg& fc, int64_t w, int64_t ci, ChainIx& c)
-{
-    if (ci >= p.B * (int64_t)fc.Kw * p.H) return false;
-    c.h = ci % p.H;
-    const int64_t kk = (ci / p.H) % fc.Kw;
-    c.b = ci / (p.H * (int64_t)fc.Kw);
-    c.k = w * fc.Kw + kk;
-    if (c.k >= p.K) return false;
-    c.tbeg = c.k * p.chunk;
-    c.tend = (c.tbeg + p.chunk < p.L) ? c.tbeg + p.chunk : p.L;
-    return true;
-}
-
-__global__ void __launch_bounds__(THREADS, 2)
-k16_fused(KParams p, FusedCfg fc, FusedBufs fb, const float* __restrict__ x, const float* __restrict__ S0,
-          float* __restrict__ S_out)
-{
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    __shared__ int64_t s_ticket;
-    __shared__ int s_go;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    WarpSmem& ws = reinterpret_cast<WarpSmem*>(smem_raw)[warp];
-    const int64_t tok = p.H * NN;
-    const int64_t nseq = p.B * p.H;
-    const int gpw = fc.Kw / fc.G;                    // groups per window
-
-    for (;;) {
-        if (tid == 0) s_ticket = ld_volatile(fb.abort_flag) ? fc.total : (int64_t)atomicAdd(fb.ticket, 1u);
-        __syncthreads();
-        const int64_t t = s_ticket;
-        __syncthreads();
-        if (t >= fc.total) return;
-
-        int kind;                                    // 0 R, 1 S1, 2 S2, 3 A
-        int64_t w, idx;
-        if (t < fc.lag * fc.nR) {
-            kind = 0; w = t / fc.nR; idx = t % fc.nR;
-        } else {
-            const int64_t bs = fc.nR + fc.nS1 + fc.nS2 + fc.nA;
-            const int64_t u = t - fc.lag * fc.nR;
-            w = u / bs;
-            int64_t r = u % bs;
-            if (r < fc.nR) { kind = 0; w += fc.lag; idx = r; }
-            else if ((r -= fc.nR) < fc.nS1) { kind = 1; idx = r; }
-            else if ((r -= fc.nS1) < fc.nS2) { kind = 2; idx = r; }
-            else { kind = 3; idx = r - fc.nS2; }
-        }
-        if (kind == 0 && w >= fc.NW) continue;       // past the last window: nothing to do
-
-        // ---- wait for this item's inputs ----
-        if (tid == 0) {
-            bool ok = true;
-            if (kind == 1) ok = wait_geq(fb.cntR + w, (unsigned)fc.nR, fb);
-            if (kind == 2) {
-                ok = wait_geq(fb.cntS1 + w, (unsigned)fc.nS1, fb);
-                if (ok && w > 0) ok = wait_geq(fb.cntS2 + w - 1, (unsigned)fc.nS2, fb);
-            }
-            if (kind == 3) ok = wait_geq(fb.cntS2 + w, (unsigned)fc.nS2, fb);
-            s_go = ok;
-        }
-        __syncthreads();
-        if (!s_go) return;
-
-        if (kind == 0) {
-            ChainIx c;
-            if (window_chain(p, fc, w, idx * WARPS + warp, c)) {
-                float Qd[2][4];
-                reduce_chain(p, ws, x + (c.b * p.L * p.H + c.h) * NN, tok, fb.cd + c.b * p.L * p.H + c.h,
-                             c.tbeg, c.tend, lane, fb.status, Qd);
-                store_d(fb.totals + ((c.b * p.H + c.h) * p.K + c.k) * NN, Qd, lane >> 2, lane & 3);
-            }
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) atomicAdd(fb.cntR + w, 1u);
-        } else if (kind == 1) {
-            const int64_t gi = idx * WARPS + warp;
-            const int64_t seq = gi / gpw;
-            const int64_t gg = w * gpw + gi % gpw;
-            if (seq < nseq && gg * fc.G < p.K) {
-                double* sR = reinterpret_cast<double*>(&ws.x[0][0]);
-                double* sT = sR + NN;
-                const int r0 = (lane >> 2) * 2, c0 = (lane & 3) * 4;
-                for (int e = lane; e < NN; e += 32) sR[e] = 0.0;
-                const int64_t k1 = (gg + 1) * fc.G < p.K ? (gg + 1) * fc.G : p.K;
-                for (int64_t k = gg * fc.G; k < k1; ++k) {
-                    const float* tk = fb.totals + (seq * p.K + k) * NN;
-                    for (int e = lane; e < NN; e += 32) sT[e] = (double)tk[e];
-                    __syncwarp();
-                    double acc[2][4];
-                    warp_gemm16_f64(sR, sT, lane, acc);
-                    __syncwarp();
-                    float* rk = fb.R0 + (seq * p.K + k) * NN;
-#pragma unroll
-                    for (int i = 0; i < 2; ++i)
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) {
-                            const int e = (r0 + i) * N + c0 + cc;
-                            const double v = sR[e] + (sT[e] + acc[i][cc]);
-                            sR[e] = v;
-                            rk[e] = (float)v;
-                        }
-                    __syncwarp();
+                        for (int i = 0; i < 4; ++i) Sd[n2][i] += acc[n2][i];
+                    store_d(ob + (t0 + j) * tok, Sd, g, q);
                 }
-                double* tot = fb.Tot + (seq * fc.NG + gg) * NN;
-                for (int e = lane; e < NN; e += 32) tot[e] = sR[e];
             }
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) atomicAdd(fb.cntS1 + w, 1u);
-        } else if (kind == 2) {
-            const int64_t seq = idx * WARPS + warp;
-            if (seq < nseq) {
-                double* sG = reinterpret_cast<double*>(&ws.x[0][0]);
-                double* sT = sG + NN;
-                const int r0 = (lane >> 2) * 2, c0 = (lane & 3) * 4;
-                for (int e = lane; e < NN; e += 32)
-                    sG[e] = (w > 0) ? fb.cstate[seq * NN + e]
-                                    : (S0 ? (double)S0[seq * NN + e] : ((e / N) == (e % N) ? 1.0 : 0.0));
-                __syncwarp();
-                for (int gw = 0; gw < gpw; ++gw) {
-                    const int64_t gg = w * gpw + gw;
-                    if (gg >= fc.NG) break;
-                    double* e1 = fb.E1 + (seq * fc.NG + gg) * NN;
-                    const double* tg = fb.Tot + (seq * fc.NG + gg) * NN;
-                    for (int e = lane; e < NN; e += 32) {
-                        e1[e] = sG[e];
-                        sT[e] = tg[e];
-                    }
-                    __syncwarp();
-                    double acc[2][4];
-                    warp_gemm16_f64(sG, sT, lane, acc);
-                    __syncwarp();
-#pragma unroll
-                    for (int i = 0; i < 2; ++i)
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) sG[(r0 + i) * N + c0 + cc] += acc[i][cc];
-                    __syncwarp();
-                }
-                for (int e = lane; e < NN; e += 32) fb.cstate[seq * NN + e] = sG[e];
-            }
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) atomicAdd(fb.cntS2 + w, 1u);
-        } else {
-            ChainIx c;
-            if (window_chain(p, fc, w, idx * WARPS + warp, c)) {
-                const int64_t seq = c.b * p.H + c.h;
-                float Sd[2][4];
-                form_carry(ws, fb.E1 + (seq * fc.NG + c.k / fc.G) * NN,
-                           (c.k % fc.G) ? fb.R0 + (seq * p.K + c.k - 1) * NN : nullptr, lane, Sd);
-                apply_chain(ws, x + (c.b * p.L * p.H + c.h) * NN, S_out + (c.b * p.L * p.H + c.h) * NN, tok, p.H,
-                            fb.cd + c.b * p.L * p.H + c.h, c.tbeg, c.tend, lane, Sd);
-            }
-            __syncthreads();
+            __syncwarp();
+            cs = (cs + 1 == ANS) ? 0 : cs + 1;
         }
     }
+}
+
+// CTAs of a persistent launch: resident CTAs per SM times the SM count,
+// cached per device and kernel slot; no more than the chains need.
+std::atomic<int> g_resident[64][3];
+
+cudaError_t persistent_grid(int slot, const void* kern, int threads, size_t smem, int warps, int64_t nchains,
+                            unsigned& grid)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int res = (dev >= 0 && dev < 64) ? g_resident[dev][slot].load(std::memory_order_relaxed) : 0;
+    if (res <= 0) {
+        int sms = 0, per_sm = 0;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem)) != cudaSuccess)
+            return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+        res = sms * per_sm;
+        if (dev >= 0 && dev < 64) g_resident[dev][slot].store(res, std::memory_order_relaxed);
+    }
+    const int64_t need = (nchains + warps - 1) / warps;
+    grid = (unsigned)(need < res ? need : res);
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -719,120 +995,98 @@ bool supports(const KParams& p, bool readout)
 {
     return p.n == N && p.src == SRC_EMBEDDING && p.x_dtype == MRU_F32 && !readout &&
            (p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM) &&
-           (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32X3) && p.chunk > 0 && p.chunk % SUB == 0;
+           (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32X3) && p.chunk > 0 && p.chunk % kSub == 0;
 }
 
-// Chunk length: 8 tokens per pass, m passes per chain, m a power of two that
-// keeps at least 16384 chains (about 7 waves of 16 warps per SM) when the
-// workload allows, so that long sequences get long chunks (few chunk totals).
+// Chunk length: 8 m tokens, m a power of two that keeps at least 16384
+// chains when the workload allows (about seven per warp of a full persistent
+// grid), so that long sequences get long chunks (few chunk totals).
 int32_t preferred_chunk(int64_t token_heads)
 {
     int32_t m = 1;
-    while (m < 16 && token_heads / ((int64_t)SUB * 2 * m) >= 16384) m *= 2;
-    return SUB * m;
+    while (m < 16 && token_heads / ((int64_t)kSub * 2 * m) >= 16384) m *= 2;
+    return kSub * m;
 }
 
-cudaError_t launch_reduce(const KParams& p, const float* x, float* totals, float2* cd, uint32_t* status,
-                          cudaStream_t s)
+// Levels of the carry scan for nseq sequences of K chunk totals, laid out
+// from byte offset off.  G = 16 unless K > 16^4 (then the smallest power of
+// two with G^4 >= K), so that at most three levels sit below the top.
+CarryPlan carry_plan(int64_t nseq, int64_t K, size_t off)
 {
-    const int64_t nchains = p.B * p.H * p.K;
-    const unsigned grid = (unsigned)((nchains + WARPS - 1) / WARPS);
-    const size_t sm = sizeof(WarpSmem) * WARPS;
-    cudaError_t e = cudaFuncSetAttribute(k16_reduce, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (e != cudaSuccess) return e;
-    k16_reduce<<<grid, THREADS, sm, s>>>(p, x, totals, cd, status);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_apply(const KParams& p, const float* x, const float2* cd, const carry::Plan& pl,
-                         const char* ws, float* S_out, cudaStream_t s)
-{
-    const int64_t nchains = p.B * p.H * p.K;
-    const unsigned grid = (unsigned)((nchains + WARPS - 1) / WARPS);
-    const size_t sm = sizeof(WarpSmem) * WARPS;
-    cudaError_t e = cudaFuncSetAttribute(k16_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (e != cudaSuccess) return e;
-    k16_apply<<<grid, THREADS, sm, s>>>(p, x, cd, reinterpret_cast<const float*>(ws + pl.R[0]),
-                                        reinterpret_cast<const double*>(ws + pl.E[1]), pl.G, S_out);
-    return cudaGetLastError();
-}
-
-// Layout of the fused kernel's workspace from byte offset `off` (the first
-// bytes, counters and flags, must be zeroed before every launch).
-FusedLayout fused_layout(const KParams& p, size_t off)
-{
-    FusedLayout L;
-    memset(&L, 0, sizeof L);
-    const int64_t nseq = p.B * p.H;
+    CarryPlan cp;
+    memset(&cp, 0, sizeof cp);
+    cp.nseq = nseq;
+    cp.gshift = 4;
+    while (((int64_t)1 << (4 * cp.gshift)) < K) ++cp.gshift;
+    cp.G = 1 << cp.gshift;
     auto take = [&](size_t bytes) {
         const size_t o = off;
         off = (off + bytes + 255) / 256 * 256;
         return o;
     };
-    L.G = 16;
-    const int64_t unit = nseq * (int64_t)p.chunk * L.G * NN * (int64_t)sizeof(float);  // x bytes per group of chunks
-    int64_t groups = (16ll << 20) / (unit > 0 ? unit : 1);
-    if (groups < 1) groups = 1;
-    if (groups > 64) groups = 64;
-    L.Kw = (int)(groups * L.G);
-    L.NW = p.K > 0 ? (p.K + L.Kw - 1) / L.Kw : 0;
-    L.NG = (p.K + L.G - 1) / L.G;
-    L.counters = take(sizeof(unsigned) * (2 + 3 * (size_t)L.NW));
-    L.counters_bytes = sizeof(unsigned) * (2 + 3 * (size_t)L.NW);
-    L.totals = take(sizeof(float) * nseq * p.K * NN);
-    L.cd = take(sizeof(float2) * nseq * p.L);
-    L.R0 = take(sizeof(float) * nseq * p.K * NN);
-    L.Tot = take(sizeof(double) * nseq * L.NG * NN);
-    L.E1 = take(sizeof(double) * nseq * L.NG * NN);
-    L.cstate = take(sizeof(double) * nseq * NN);
-    L.end = off;
-    return L;
+    cp.cnt[0] = K;
+    int l = 0;
+    while (cp.cnt[l] > cp.G) {
+        cp.cnt[l + 1] = (cp.cnt[l] + cp.G - 1) / cp.G;
+        cp.R[l] = take((size_t)nseq * cp.cnt[l] * NN * (l == 0 ? sizeof(float) : sizeof(double)));
+        cp.Tot[l] = take((size_t)nseq * cp.cnt[l + 1] * NN * sizeof(double));
+        ++l;
+    }
+    cp.levels = l;
+    cp.Etop = take((size_t)nseq * cp.cnt[l] * NN * sizeof(double));
+    cp.ctr_begin = off;
+    for (int i = 0; i < l; ++i) cp.ctr[i] = take((size_t)nseq * cp.cnt[i + 1] * sizeof(unsigned));
+    cp.ctr[l] = take((size_t)nseq * sizeof(unsigned));
+    cp.ctr_bytes = off - cp.ctr_begin;
+    cp.end = off;
+    return cp;
 }
 
-cudaError_t launch_fused(const KParams& p, const FusedLayout& L, char* ws, uint32_t* status, const float* x,
-                         const float* S0, float* S_out, cudaStream_t s)
+cudaError_t launch_reduce(const KParams& p, const float* x, float* totals, const CarryPlan& cp, char* ws,
+                          uint32_t* status, cudaStream_t s)
 {
-    const int64_t nseq = p.B * p.H;
-    if (nseq * p.K == 0) return cudaSuccess;
-    FusedCfg fc;
-    fc.G = L.G;
-    fc.Kw = L.Kw;
-    fc.lag = 2;
-    fc.NW = L.NW;
-    fc.NG = L.NG;
-    const int64_t chains_w = p.B * (int64_t)L.Kw * p.H;
-    fc.nR = (chains_w + WARPS - 1) / WARPS;
-    fc.nA = fc.nR;
-    fc.nS1 = (nseq * (L.Kw / L.G) + WARPS - 1) / WARPS;
-    fc.nS2 = (nseq + WARPS - 1) / WARPS;
-    fc.total = fc.lag * fc.nR + fc.NW * (fc.nR + fc.nS1 + fc.nS2 + fc.nA);
-    FusedBufs fb;
-    unsigned* ctr = reinterpret_cast<unsigned*>(ws + L.counters);
-    fb.ticket = ctr;
-    fb.abort_flag = ctr + 1;
-    fb.cntR = ctr + 2;
-    fb.cntS1 = ctr + 2 + L.NW;
-    fb.cntS2 = ctr + 2 + 2 * L.NW;
-    fb.totals = reinterpret_cast<float*>(ws + L.totals);
-    fb.cd = reinterpret_cast<float2*>(ws + L.cd);
-    fb.R0 = reinterpret_cast<float*>(ws + L.R0);
-    fb.Tot = reinterpret_cast<double*>(ws + L.Tot);
-    fb.E1 = reinterpret_cast<double*>(ws + L.E1);
-    fb.cstate = reinterpret_cast<double*>(ws + L.cstate);
-    fb.status = status;
-    cudaError_t e = cudaMemsetAsync(ws + L.counters, 0, L.counters_bytes, s);
+    const int64_t nchains = p.B * p.H * p.K;
+    if (nchains == 0) return cudaSuccess;
+    if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    const size_t sm = sizeof(RSmem) * RWARPS;
+    const bool per_token = p.mode == MRU_MODE_DETNORM && !p.add_identity;
+    auto kern = per_token ? k16_reduce<true> : k16_reduce<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    const size_t sm = sizeof(WarpSmem) * WARPS;
-    e = cudaFuncSetAttribute(k16_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    unsigned grid = 0;
+    if ((e = persistent_grid(per_token ? 1 : 0, (const void*)kern, RWARPS * 32, sm, RWARPS, nchains, grid)) !=
+        cudaSuccess)
+        return e;
+    kern<<<grid, RWARPS * 32, sm, s>>>(p, x, totals, reinterpret_cast<unsigned*>(ws + cp.ctr_begin),
+                                       (int64_t)(cp.ctr_bytes / sizeof(unsigned)), status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_carry(const KParams& p, const float* totals, const CarryPlan& cp, char* ws, const float* S0,
+                         cudaStream_t s)
+{
+    const int64_t units = cp.nseq * (cp.levels > 0 ? cp.cnt[1] : 1);
+    if (p.B * p.H * p.K == 0 || units == 0) return cudaSuccess;
+    const size_t sm = sizeof(CSmem) * CWARPS;
+    cudaError_t e = cudaFuncSetAttribute(k16_carry, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0, per_sm = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k16_fused, THREADS, sm)) != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    int64_t grid = (int64_t)sms * per_sm;
-    if (grid > fc.total) grid = fc.total;
-    k16_fused<<<(unsigned)grid, THREADS, sm, s>>>(p, fc, fb, x, S0, S_out);
+    k16_carry<<<(unsigned)((units + CWARPS - 1) / CWARPS), CWARPS * 32, sm, s>>>(p, totals, cp, ws, S0);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_apply(const KParams& p, const float* x, const CarryPlan& cp, const char* ws, float* S_out,
+                         uint32_t* status, cudaStream_t s)
+{
+    const int64_t nchains = p.B * p.H * p.K;
+    if (nchains == 0) return cudaSuccess;
+    if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    const size_t sm = sizeof(ASmem) * AWARPS;
+    cudaError_t e = cudaFuncSetAttribute(k16_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    unsigned grid = 0;
+    if ((e = persistent_grid(2, (const void*)k16_apply, AWARPS * 32, sm, AWARPS, nchains, grid)) != cudaSuccess)
+        return e;
+    k16_apply<<<grid, AWARPS * 32, sm, s>>>(p, x, cp, ws, S_out, status);
     return cudaGetLastError();
 }
 

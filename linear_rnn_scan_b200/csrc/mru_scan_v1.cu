@@ -586,19 +586,19 @@ cudaError_t scan_fast16(const KParams& p, const void* src, const float* S0, floa
 {
     uint32_t* status = reinterpret_cast<uint32_t*>(ws + W.status);
     float* totals = reinterpret_cast<float*>(ws + W.totals);
-    float2* cd = reinterpret_cast<float2*>(ws + W.cd);
     const float* x = reinterpret_cast<const float*>(src);
     if (p.B * p.H * p.K == 0) return cudaSuccess;
     cudaError_t e;
-    int slot = 0;
-    profile_mark(slot, 0, s);
-    if ((e = n16::launch_reduce(p, x, totals, cd, status, s)) != cudaSuccess) return e;
-    profile_mark(slot++, 1, s);
-    if ((e = carry::run_n16(W.plan, totals, S0, ws, s, slot)) != cudaSuccess) return e;
-    profile_mark(slot, 0, s);
-    if ((e = n16::launch_apply(p, x, cd, W.plan, ws, S_out, s)) != cudaSuccess) return e;
-    profile_mark(slot++, 1, s);
-    if (launches) *launches = slot;
+    profile_mark(0, 0, s);
+    if ((e = n16::launch_reduce(p, x, totals, W.c16, ws, status, s)) != cudaSuccess) return e;
+    profile_mark(0, 1, s);
+    profile_mark(1, 0, s);
+    if ((e = n16::launch_carry(p, totals, W.c16, ws, S0, s)) != cudaSuccess) return e;
+    profile_mark(1, 1, s);
+    profile_mark(2, 0, s);
+    if ((e = n16::launch_apply(p, x, W.c16, ws, S_out, status, s)) != cudaSuccess) return e;
+    profile_mark(2, 1, s);
+    if (launches) *launches = 3;
     return cudaGetLastError();
 }
 
@@ -658,14 +658,6 @@ cudaError_t launch_scan(const KParams& p, const void* src, const float* S0, cons
                         void* ws_base, const Workspace& W, cudaStream_t s, int* launches)
 {
     char* ws = reinterpret_cast<char*>(ws_base);
-    if (W.fused) {
-        profile_mark(0, 0, s);
-        cudaError_t e = n16::launch_fused(p, W.fl, ws, reinterpret_cast<uint32_t*>(ws + W.status),
-                                          reinterpret_cast<const float*>(src), S0, S_out, s);
-        profile_mark(0, 1, s);
-        if (launches) *launches = 1;
-        return e;
-    }
     if (W.fast && W.fast_n == 32) return scan_fast32(p, src, S0, S_out, ws, W, s, launches);
     if (W.fast) return scan_fast16(p, src, S0, S_out, ws, W, s, launches);
     switch (p.n) {

@@ -90,7 +90,8 @@ def test_invalid_arguments_rejected_before_any_launch(lib):
     assert mru.scan_fused(p, fake, None, None, 0, None, fake, nb) == mru.ERR_INVALID_ARG       # S_out null
     assert mru.scan_fused(p, fake + 4, None, None, fake, None, fake, nb) == mru.ERR_INVALID_ARG  # misaligned
     assert mru.scan_fused(p, fake, None, None, fake, None, fake, nb) == mru.ERR_INVALID_ARG    # alias
-    assert mru.scan_fused(p, fake, None, None, 2 * fake, None, 3 * fake, nb - 1) == mru.ERR_WORKSPACE
+    # (the size is the largest any call of this problem needs; this call needs less, but more than 255 bytes)
+    assert mru.scan_fused(p, fake, None, None, 2 * fake, None, 3 * fake, 255) == mru.ERR_WORKSPACE
     bad = mru.problem(1, 1, 8, 12)
     assert mru.scan_fused(bad, fake, None, None, 2 * fake, None, 3 * fake, nb) == mru.ERR_UNSUPPORTED
     bad = mru.problem(1, 1, 8, 16, mode=7)

@@ -254,3 +254,29 @@ def test_parity_n16_tensor_path(L, chunk):
     assert st == mru.OK
     e = compare_S(w, x, S, S0=S0)
     assert e["max"] <= TOL_FP32, e
+
+
+@pytest.mark.parametrize("B,H,L,chunk,mode,add_identity", [
+    (1, 2, 2059, 8, gen.MODE_DETNORM, 1),       # 258 chunk totals: two levels below the top
+    (1, 1, 32800, 8, gen.MODE_DETNORM, 1),      # 4100 chunk totals: three levels
+    (2, 3, 41, 8, gen.MODE_DETNORM, 0),         # per-token scales in the reduce pass (short: these
+                                                # chains grow about e^0.4 a token)
+    (2, 2, 530, 16, gen.MODE_RESHAPE, 1),
+    (1, 3, 203, 8, gen.MODE_RESHAPE, 0),
+])
+def test_parity_n16_carry_levels(B, H, L, chunk, mode, add_identity):
+    """n = 16 tensor-core path: the in-launch carry scan over one to three
+    levels of groups, ragged last groups, both modes, with and without the
+    identity."""
+    # near identity with the identity added; alpha M of spectral radius about
+    # 1 without it (the determinant-corrected mode is scale free)
+    alpha = (0.05 / 4 if mode == gen.MODE_DETNORM else 0.01) if add_identity else 0.25
+    w = small(16, mode, B=B, H=H, L=L, alpha=alpha, add_identity=add_identity, seed=970 + L)
+    x = gen.make_x(w)
+    S0 = gen.make_S0(w, seed=971)
+    assert mru.effective_math(mru.problem_from_workload(w, chunk=chunk)) == "tf32x3"
+    S, st = run_fused(w, x, S0=S0, chunk=chunk)
+    assert st == mru.OK
+    e = compare_S(w, x, S, S0=S0)
+    assert e["count"] == B * H * L
+    assert e["max"] <= TOL_FP32, e
