@@ -167,14 +167,16 @@ __device__ __forceinline__ float rcp_approx(float v)
 
 // |det(I + e)| of one 16 x 16 matrix held by a group of 16 / R lanes (lane r
 // of the group owns rows r + (16 / R) lr, lr < R, in e[lr][0..15]),
-// eliminated on e alone without pivoting: prod |1 + delta_k| (fp64 product).
-// ok = false when a pivot |1 + delta_k| < 0.5.  All lanes of the warp call it
-// (the shuffles span the warp).
+// eliminated on e alone without pivoting: prod |1 + delta_k|, an fp32
+// product of 16 factors near 1 (relative error about 1e-7: the scale
+// c = |det|^(-1/16) it gives is good to about 1e-8).  ok = false when a
+// pivot |1 + delta_k| < 0.5.  All lanes of the warp call it (the shuffles
+// span the warp).
 template <int R>
-__device__ __forceinline__ double lu_near_identity(float (&e)[R][N], int r, bool& ok)
+__device__ __forceinline__ float lu_near_identity(float (&e)[R][N], int r, bool& ok)
 {
     constexpr int W = N / R;
-    double prod = 1.0;
+    float prod = 1.0f;
     ok = true;
 #pragma unroll
     for (int k = 0; k < N; ++k) {
@@ -184,7 +186,7 @@ __device__ __forceinline__ double lu_near_identity(float (&e)[R][N], int r, bool
         for (int j = k; j < N; ++j) prow[j] = __shfl_sync(FULL, e[kr][j], owner, W);
         const float pk = 1.0f + prow[k];
         if (!(fabsf(pk) >= 0.5f)) ok = false;
-        prod *= 1.0 + (double)prow[k];
+        prod *= pk;
         const float rk = rcp_approx(pk);
 #pragma unroll
         for (int lr = 0; lr < R; ++lr) {
@@ -197,7 +199,7 @@ __device__ __forceinline__ double lu_near_identity(float (&e)[R][N], int r, bool
             }
         }
     }
-    return fabs(prod);
+    return fabsf(prod);
 }
 
 struct LogDet {
@@ -291,8 +293,8 @@ __device__ __forceinline__ float det_scale_m1(const float* src, int stride, int 
     if (near) {
         float e[R][N];
         load_rows<R>(e, src, stride, r, scale, false);
-        const double ad = lu_near_identity<R>(e, r, ok);
-        cm1 = expm1f(-log1pf((float)(ad - 1.0)) * (1.0f / N));
+        const float ad = lu_near_identity<R>(e, r, ok);
+        cm1 = expm1f(-log1pf(ad - 1.0f) * (1.0f / N));
     }
     if (__any_sync(FULL, !ok)) {
         __syncwarp();
@@ -439,16 +441,23 @@ __device__ __forceinline__ void d16_zero(D16& a)
     for (int i = 0; i < 8; ++i) (&a.m[0][0][0])[i] = 0.0;
 }
 
-// acc += A B (B converted to fp64 as it is used).
+// acc += A B (B converted to fp64 as it is used).  The k-tiles 0-1 and 2-3
+// accumulate separately and are added at the end: two dependent mma steps
+// per product instead of four.
 template <typename T>
 __device__ __forceinline__ void d16_mac(const D16& A, const F16<T>& B, D16& acc)
 {
+    D16 hi;
+    d16_zero(hi);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-            for (int nb = 0; nb < 2; ++nb) mma_f64(acc.m[mt][nb], A.m[mt][kk >> 1][kk & 1], (double)B.b[kk][nb]);
+            for (int nb = 0; nb < 2; ++nb)
+                mma_f64(kk < 2 ? acc.m[mt][nb] : hi.m[mt][nb], A.m[mt][kk >> 1][kk & 1], (double)B.b[kk][nb]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) (&acc.m[0][0][0])[i] += (&hi.m[0][0][0])[i];
 }
 
 // One row-major 16 x 16 matrix in shared memory as the B operand, in its own
@@ -549,6 +558,9 @@ __device__ __forceinline__ void load_staged(const T* buf, int j, double gm, doub
             }
 }
 
+__device__ __forceinline__ void store_pair(float* p, double a, double b) { *reinterpret_cast<float2*>(p) = make_float2((float)a, (float)b); }
+__device__ __forceinline__ void store_pair(double* p, double a, double b) { *reinterpret_cast<double2*>(p) = make_double2(a, b); }
+
 template <typename T>
 __device__ __forceinline__ void store_acc(T* dst, const D16& a, int lane)
 {
@@ -556,9 +568,7 @@ __device__ __forceinline__ void store_acc(T* dst, const D16& a, int lane)
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) dst[(8 * mt + g) * N + 8 * nb + 2 * t + h] = (T)a.m[mt][nb][h];
+        for (int nb = 0; nb < 2; ++nb) store_pair(dst + (8 * mt + g) * N + 8 * nb + 2 * t, a.m[mt][nb][0], a.m[mt][nb][1]);
 }
 
 // Scans the m split-form items at in: Top, the exclusive carries E_0 = S0
@@ -592,14 +602,22 @@ __device__ __forceinline__ void staged_scan(CSmem& sm, const Tin* in, int m, boo
         __syncwarp();
         stage_items(buf, in + (int64_t)j0 * NN, cnt, lane);
         if (correct) stage_gammas(sm, cnt, lane);
-        for (int j = 0; j < cnt; ++j) {
+        // the next item's operands load (and convert) while this step's
+        // products run
+        B16 Bn;
+        D16 Tn;
+        auto operands = [&](int j, B16& b, D16& a) {
             double gm = 1.0, gm1 = 0.0;
             if (correct) {
                 const float2 gg = sm.gam[j];
                 gm = (double)gg.x;
                 gm1 = (double)gg.y;
             }
-            load_staged(buf, j, gm, gm1, Bf, Ta, lane);
+            load_staged(buf, j, gm, gm1, b, a, lane);
+        };
+        operands(0, Bf, Ta);
+        for (int j = 0; j < cnt; ++j) {
+            if (j + 1 < cnt) operands(j + 1, Bn, Tn);
             if (Top) {
                 store_acc(E + (int64_t)(j0 + j) * NN, st, lane);
                 acc = st;                              // E_j + E_j T_j
@@ -612,6 +630,8 @@ __device__ __forceinline__ void staged_scan(CSmem& sm, const Tin* in, int m, boo
                 for (int i = 0; i < 8; ++i) (&st.m[0][0][0])[i] += (&acc.m[0][0][0])[i];
                 store_acc(R + (int64_t)(j0 + j) * NN, st, lane);
             }
+            Bf = Bn;
+            Ta = Tn;
         }
     }
     if (!Top) store_acc(tot, st, lane);
