@@ -51,6 +51,50 @@ def env_int(name, default):
         return default
 
 
+class Ranks:
+    """One process per GPU, rank and world size from the launcher's
+    environment (RANK, WORLD_SIZE, LOCAL_RANK, MASTER_ADDR/PORT).  The only
+    collectives are the barrier around the timed regions and the max over
+    ranks of their durations; rank 0 prints."""
+
+    def __init__(self, backend: str = "nccl", device=None, timeout_s: float = 120.0):
+        self.rank, self.world = env_int("RANK", 0), env_int("WORLD_SIZE", 1)
+        self.local = env_int("LOCAL_RANK", 0)
+        self.device = device
+        self.dist = None
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+            self.dist = dist
+
+    @property
+    def printer(self) -> bool:
+        return self.rank == 0
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, v: float) -> float:
+        if self.dist is None:
+            return v
+        import torch
+        t = torch.tensor([v], device=self.device, dtype=torch.float64)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def aggregate_rate(world: int, units_per_rank: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank processed its units within the
+    slowest rank's time."""
+    return world * units_per_rank / (ms_max / 1e3)
+
+
 # ------------------------------------------------------------ bookkeeping ---
 
 def step_bytes(w: gen.Workload) -> dict:
@@ -69,22 +113,32 @@ def step_bytes(w: gen.Workload) -> dict:
 
 def kernel_bytes(name: str, w: gen.Workload, chunk: int) -> int:
     """Bytes one launch of a kernel must move by its own design (per launch =
-    the whole workload): chunk prefixes read the embeddings and write the
-    local prefixes Q_t where S_t goes plus the chunk totals; the fix-up reads
-    Q_t and writes S_t; the carry kernels touch only chunk totals."""
+    the whole workload).  Generic path: the chunk kernel reads the embeddings
+    and writes the local prefixes Q_t where S_t goes plus the chunk totals;
+    the fix-up reads Q_t and writes S_t.  Two-pass paths: the reduce pass
+    reads the embeddings and writes the chunk totals; the apply pass reads
+    the embeddings and each chain's carry factors and writes S_t; the carry
+    kernels touch only chunk totals, in-group prefixes and carries."""
     nn = w.n * w.n
     sb = step_bytes(w)
     K = -(-w.L // chunk)
-    tot = w.B * w.H * K * nn
-    scal = w.token_heads * 8 if w.n == 16 else 0     # per-token scalars of the n = 16 kernels
+    chains = w.B * w.H * K
+    tot = chains * nn                       # elements of all chunk totals
+    groups = -(-chains // 16)
     if "chunk" in name:
         return sb["in"] + sb["out"] + tot * 4
     if "fixup" in name:
         return 2 * sb["out"] + tot * 4
     if "reduce" in name:
-        return sb["in"] + tot * 4 + scal
+        return sb["in"] + tot * 4
     if "apply" in name:
-        return sb["in"] + sb["out"] + scal + tot * 4
+        return sb["in"] + sb["out"] + chains * nn * (8 + 4)
+    if name == "k16_carry":
+        return tot * (4 + 4) + groups * nn * (8 + 8)
+    if name == "k_level":
+        return tot * (4 + 4) + groups * nn * 8
+    if name in ("k_top", "k_down"):
+        return groups * nn * 16
     if name.endswith("carry_local"):
         return tot * (4 + 8)
     if name.endswith("carry_groups"):
@@ -275,7 +329,7 @@ def workload_config(w, chunk):
             "snapshot_every": w.snapshot_every, "chunk": chunk,
             "l2": ("inputs larger than L2: x %.0f MiB in, %.0f MiB out per step" %
                    (sb["in"] / 2 ** 20, sb["out"] / 2 ** 20)) if sb["total"] > L2_BYTES
-            else "inputs smaller than L2 (no flush)",
+            else "inputs smaller than L2: L2 flushed (252 MiB written) between timed steps, outside the events",
             "parallelism": "single GPU; replicas across GPUs (independent (b,h) sequences)"}
 
 
@@ -283,26 +337,15 @@ def workload_config(w, chunk):
 
 def run_ours(args, w):
     import torch
-    import torch.distributed as dist
 
     from linear_rnn_scan_b200 import mru
 
-    rank, world, local = env_int("RANK", 0), env_int("WORLD_SIZE", 1), env_int("LOCAL_RANK", 0)
+    local = env_int("LOCAL_RANK", 0)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks("nccl", dev)
+    rank, world = ranks.rank, ranks.world
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     # CPU baseline first (rank 0, one GPU), before any CUDA work.
     x_np = gen.make_x(w, seed=w.seed + rank)
@@ -367,22 +410,38 @@ def run_ours(args, w):
     if st != mru.OK:
         raise mru.MruError(st, "device status after warm-up")
 
-    # timed region: exactly K steps, device-resident inputs
+    # timed region: exactly K steps, device-resident inputs.  Workloads
+    # smaller than L2 get an L2 flush (a write of twice its size) between
+    # steps, outside the per-step events.
+    flush = None
+    if step_bytes(w)["total"] <= L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
-        ev0.record(stream)
-        for _ in range(args.steps):
-            step()
-        ev1.record(stream)
-        ev1.synchronize()
+        if flush is None:
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            for _ in range(args.steps):
+                step()
+            ev1.record(stream)
+            ev1.synchronize()
+            ms = ev0.elapsed_time(ev1) / args.steps
+        else:
+            pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(args.steps)]
+            for a, b in pairs:
+                flush.zero_()
+                a.record(stream)
+                step()
+                b.record(stream)
+            pairs[-1][1].synchronize()
+            ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
     torch.cuda.synchronize()
     barrier()
-    ms = ev0.elapsed_time(ev1) / args.steps
     ms = max_over_ranks(ms)
-    value = world * w.token_heads / (ms / 1e3)
+    value = aggregate_rate(world, w.token_heads, ms)
 
     # per-kernel durations: the same K steps again with the library's event hook
     n_k = launches_per_step
@@ -447,7 +506,7 @@ def run_ours(args, w):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded N(0,1) embeddings)",
             "config": cfg, "clocks": clocks.summary(),
-            "e2e": {"value": world * w.token_heads / (e2e_ms / 1e3), "unit": UNIT,
+            "e2e": {"value": aggregate_rate(world, w.token_heads, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                     "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
@@ -457,8 +516,7 @@ def run_ours(args, w):
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
     del out_main
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 

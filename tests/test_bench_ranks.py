@@ -1,0 +1,69 @@
+"""The bench's multi-process logic on CPU: two gloo ranks take the barrier
+and the max over ranks of their timings exactly as the NCCL ranks of
+`torchrun ... bench.py --gpus N` do; only rank 0 prints; the whole-job rate
+counts every rank's units over the slowest rank's time; the reference arm
+exits at once on ranks other than 0."""
+from __future__ import annotations
+
+import json
+import os
+import socket
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, outdir, per_rank_ms):
+    import torch
+    os.environ.update({"RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    r = bench.Ranks("gloo", torch.device("cpu"), timeout_s=60)
+    r.barrier()
+    ms = r.max(per_rank_ms[rank])
+    r.barrier()
+    out = {"rank": r.rank, "world": r.world, "printer": r.printer, "ms": ms,
+           "rate": bench.aggregate_rate(r.world, 1000, ms)}
+    r.close()
+    with open(os.path.join(outdir, f"rank{rank}.json"), "w") as f:
+        json.dump(out, f)
+
+
+def test_two_gloo_ranks_barrier_and_max(tmp_path):
+    import torch.multiprocessing as mp
+    world, port = 2, _free_port()
+    per_rank_ms = [1.25, 2.5]
+    mp.spawn(_rank_main, args=(world, port, str(tmp_path), per_rank_ms), nprocs=world, join=True)
+    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    assert [x["rank"] for x in res] == [0, 1]
+    assert all(x["world"] == 2 for x in res)
+    assert [x["printer"] for x in res] == [True, False]
+    assert all(x["ms"] == 2.5 for x in res)                    # slowest rank's time on every rank
+    assert all(x["rate"] == pytest.approx(2 * 1000 / 2.5e-3) for x in res)
+
+
+def test_single_process_needs_no_process_group(monkeypatch):
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    r = bench.Ranks("gloo")
+    assert (r.rank, r.world, r.printer) == (0, 1, True)
+    assert r.max(3.5) == 3.5
+    r.barrier()
+    r.close()
+
+
+def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+    args = bench.argparse.Namespace(gpus=2, steps=1, warmup=3, impl="reference")
+    assert bench.run_reference(args, bench.gen.WORKLOADS[bench.DEFAULT_WORKLOAD]) == 0
+    assert capsys.readouterr().out == ""
