@@ -372,9 +372,11 @@ __device__ __forceinline__ void make_frag_f(const float* xs, float ca, float d0,
     }
 }
 
-// acc = A F with A the 16 x 16 state held in accumulator layout (Ad).  The
-// four (column tile, k-tile) products accumulate separately and are summed
-// at the end, so that a token's dependent mma chain is three long, not six.
+// acc = init + A F with A the 16 x 16 state held in accumulator layout
+// (Ad); init is zero (Zero) or F itself at the accumulator positions (the
+// reduce pass's F + Q F).  One accumulator per column tile: the six split
+// products go in from the smallest (lo hi, hi lo) to the largest (hi hi).
+template <bool Zero>
 __device__ __forceinline__ void chain_product(const float (&Ad)[2][4], const FragF& f, float (&acc)[2][4])
 {
     uint32_t ah[2][4], al[2][4];
@@ -385,23 +387,26 @@ __device__ __forceinline__ void chain_product(const float (&Ad)[2][4], const Fra
         split_tf32(Ad[kt][1], ah[kt][2], al[kt][2]);
         split_tf32(Ad[kt][3], ah[kt][3], al[kt][3]);
     }
-    float part[2][2][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < 2; ++nt) {
+        if (Zero) {
+            mma_tf32_first(acc[nt], al[0], f.bh[0][nt]);
+        } else {
 #pragma unroll
-        for (int kt = 0; kt < 2; ++kt) mma_tf32_first(part[nt][kt], al[kt], f.bh[kt][nt]);
+            for (int i = 0; i < 4; ++i) acc[nt][i] = f.fd[nt][i];
+            mma_tf32(acc[nt], al[0], f.bh[0][nt]);
+        }
+    }
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < 2; ++nt) mma_tf32(acc[nt], al[1], f.bh[1][nt]);
 #pragma unroll
-        for (int kt = 0; kt < 2; ++kt) mma_tf32(part[nt][kt], ah[kt], f.bl[kt][nt]);
+    for (int kt = 0; kt < 2; ++kt)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < 2; ++nt) mma_tf32(acc[nt], ah[kt], f.bl[kt][nt]);
 #pragma unroll
-        for (int kt = 0; kt < 2; ++kt) mma_tf32(part[nt][kt], ah[kt], f.bh[kt][nt]);
+    for (int kt = 0; kt < 2; ++kt)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[nt][i] = part[nt][0][i] + part[nt][1][i];
+        for (int nt = 0; nt < 2; ++nt) mma_tf32(acc[nt], ah[kt], f.bh[kt][nt]);
 }
 
 __device__ __forceinline__ void store_d(float* out, const float (&Ad)[2][4], int g, int q)
@@ -905,11 +910,11 @@ k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, u
                     FragF f;
                     make_frag_f(xs + j * NN, ca, m0 * dv, m1 * dv, g, q, f, true);
                     float acc[2][4];
-                    chain_product(Qd, f, acc);
+                    chain_product<false>(Qd, f, acc);         // F + Q F
 #pragma unroll
                     for (int n2 = 0; n2 < 2; ++n2)
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) Qd[n2][i] += f.fd[n2][i] + acc[n2][i];
+                        for (int i = 0; i < 4; ++i) Qd[n2][i] += acc[n2][i];
                 }
             }
             __syncwarp();
@@ -970,7 +975,7 @@ k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, 
                     FragF f;
                     make_frag_f(xs + j * NN, cdj.x, m0 * cdj.y, m1 * cdj.y, g, q, f, false);
                     float acc[2][4];
-                    chain_product(Sd, f, acc);
+                    chain_product<true>(Sd, f, acc);
 #pragma unroll
                     for (int n2 = 0; n2 < 2; ++n2)
 #pragma unroll
