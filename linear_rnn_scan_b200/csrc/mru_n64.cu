@@ -9,8 +9,9 @@
 //     of E = alpha M in identity-split form (pivots 1 + delta_k), register
 //     blocked: thread (br, bc) owns rows 4br..4br+3, columns 8bc..8bc+7; the
 //     pivot row and column are exchanged through shared memory, one barrier
-//     per step; |det| = prod (1 + delta_k) in fp64.  A pivot below 1/2 in
-//     magnitude sends the token to a partially pivoted LU in shared memory,
+//     per step; |det| = prod (1 + delta_k) in fp32, c - 1 by log1p and expm1.
+//     A pivot below 1/2 in magnitude sends the token to a partially pivoted
+//     LU in shared memory,
 //   * Q_t = Q_{t-1} + (F_t + Q_{t-1} F_t) with F = c alpha M + (c - 1) I,
 //     the product on mma.sync m16n8k8 tf32 with fp32 accumulation (the
 //     workload's tf32 arithmetic; the identity split keeps the implicit 1 out
@@ -63,9 +64,12 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// log|det(I + alpha M)| (ok == true) by the register-blocked identity-split
+// |det(I + alpha M)| (ok == true) by the register-blocked identity-split
 // LU; ok == false when a pivot is below 1/2 in magnitude.  All threads call.
-__device__ double logdet_near_identity(Smem& sm, float alpha, bool& ok)
+// Thread (br, bc) updates its whole 4 x 8 block at every step where the block
+// reaches below and right of the pivot: entries in eliminated rows or columns
+// are never read again, so they need no masking.
+__device__ float absdet_near_identity(Smem& sm, float alpha, bool& ok)
 {
     const int t = threadIdx.x, br = t >> 3, bc = t & 7;
     float e[4][8];
@@ -76,7 +80,7 @@ __device__ double logdet_near_identity(Smem& sm, float alpha, bool& ok)
         e[r][0] = alpha * v0.x; e[r][1] = alpha * v0.y; e[r][2] = alpha * v0.z; e[r][3] = alpha * v0.w;
         e[r][4] = alpha * v1.x; e[r][5] = alpha * v1.y; e[r][6] = alpha * v1.z; e[r][7] = alpha * v1.w;
     }
-    double prod = 1.0;
+    float prod = 1.0f;
     bool good = true;
     // k = k0 + kk with kk unrolled, so that the register slots selected by
     // k & 3 and k & 7 are known at compile time (no local-memory arrays)
@@ -86,25 +90,24 @@ __device__ double logdet_near_identity(Smem& sm, float alpha, bool& ok)
             const int k = k0 + kk;
             const int par = kk & 1;
             if (br == (k >> 2)) {
-#pragma unroll
-                for (int c = 0; c < 8; ++c) sm.prow[par][8 * bc + c] = e[kk & 3][c];
+                float4* pr = reinterpret_cast<float4*>(sm.prow[par] + 8 * bc);
+                pr[0] = make_float4(e[kk & 3][0], e[kk & 3][1], e[kk & 3][2], e[kk & 3][3]);
+                pr[1] = make_float4(e[kk & 3][4], e[kk & 3][5], e[kk & 3][6], e[kk & 3][7]);
             }
-            if (bc == (k >> 3)) {
-#pragma unroll
-                for (int r = 0; r < 4; ++r) sm.pcol[par][4 * br + r] = e[r][kk];
-            }
+            if (bc == (k >> 3))
+                *reinterpret_cast<float4*>(sm.pcol[par] + 4 * br) = make_float4(e[0][kk], e[1][kk], e[2][kk], e[3][kk]);
             __syncthreads();
-            const float d = sm.prow[par][k];
-            const float pk = 1.0f + d;
+            const float pk = 1.0f + sm.prow[par][k];
             if (!(fabsf(pk) >= 0.5f)) good = false;
-            prod *= 1.0 + (double)d;
-            const float rk = __frcp_rn(pk);
+            prod *= pk;
             if (4 * br + 3 > k && 8 * bc + 7 > k) {
-                float l[4], pr[8];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) l[r] = (4 * br + r > k) ? sm.pcol[par][4 * br + r] * rk : 0.0f;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) pr[c] = (8 * bc + c > k) ? sm.prow[par][8 * bc + c] : 0.0f;
+                float rk;
+                asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(rk) : "f"(pk));
+                const float4 lc = *reinterpret_cast<const float4*>(sm.pcol[par] + 4 * br);
+                const float4 p0 = *reinterpret_cast<const float4*>(sm.prow[par] + 8 * bc);
+                const float4 p1 = *reinterpret_cast<const float4*>(sm.prow[par] + 8 * bc + 4);
+                const float l[4] = {lc.x * rk, lc.y * rk, lc.z * rk, lc.w * rk};
+                const float pr[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
                 for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -113,7 +116,7 @@ __device__ double logdet_near_identity(Smem& sm, float alpha, bool& ok)
         }
     }
     ok = good;
-    return log(fabs(prod));
+    return fabsf(prod);
 }
 
 // log|det(W)|, W = add_identity I + alpha M, by LU with partial pivoting on
@@ -222,24 +225,29 @@ k64_chunk_readout(KParams p, const float* __restrict__ x, const float* __restric
         // ---- determinant scale ----
         float ca = p.alpha, dv = p.add_identity ? 0.0f : -1.0f;
         if (p.mode == MRU_MODE_DETNORM) {
-            double ld = 0.0;
+            // near the identity: |det| = prod (1 + delta_k) in fp32 (64
+            // factors near 1, relative error about 2e-7), c - 1 =
+            // expm1(-log1p(|det| - 1) / 64); otherwise the pivoted LU's fp64 sum
+            float cm1 = 0.0f;
             bool ok = p.add_identity != 0;
-            if (ok) ld = logdet_near_identity(sm, p.alpha, ok);
+            if (ok) cm1 = expm1f(-log1pf(absdet_near_identity(sm, p.alpha, ok) - 1.0f) * (1.0f / N));
             __syncthreads();
             const bool retry = __syncthreads_or(!ok);
+            bool bad = false;
             if (retry) {
-                ld = logdet_pivoted(sm, p.alpha, p.add_identity);
+                const double ld = logdet_pivoted(sm, p.alpha, p.add_identity);
                 load_slice(sm, src);                 // the fallback overwrote the slice
+                bad = !isfinite(ld);
+                cm1 = (float)expm1(-ld / N);
             }
-            const double cm1d = expm1(-ld / N);
-            const float c = (float)(1.0 + cm1d);
-            if (!isfinite(ld) || !isfinite(c) || c == 0.0f) {
+            const float c = 1.0f + cm1;
+            if (bad || !isfinite(cm1) || !(c > 0.0f)) {
                 if (tid == 0) atomicOr(status, STATUS_SINGULAR);
                 ca = 0.0f;
                 dv = 0.0f;
             } else {
                 ca = c * p.alpha;
-                dv = p.add_identity ? (float)cm1d : -1.0f;
+                dv = p.add_identity ? cm1 : -1.0f;
             }
         }
         // ---- Q_t = Q + (F + Q F), 1xTF32 ----

@@ -446,7 +446,6 @@ k_fixup(KParams p, const float* carry, const float* u, int64_t snap_every, float
     float* sC = smem;
     float* sQ = sC + NN;
     float* sCu = sQ + NN;
-    float* sV = sCu + N;
     const int tid = threadIdx.x;
     const int64_t chain = blockIdx.x;
     const int64_t k = chain % p.K;
@@ -484,23 +483,45 @@ k_fixup(KParams p, const float* carry, const float* u, int64_t snap_every, float
         for (int64_t t = t0; t < t1; ++t) fix_matrix(S_out + ((b * p.L + t) * p.H + h) * NN);
         return;
     }
+    // readout: o_t = C u + C v_t for every token of the chunk, N tokens at a
+    // time as one small product with C transposed in shared memory
+    // (thread i reads column entries C[i][j] at consecutive addresses) and
+    // the v_t tile staged in sQ
+    float* sCt = sQ;                        // first C transposed, then reused
+    for (int e = tid; e < NN; e += kThreads) sCt[(e % N) * N + e / N] = sC[e];
+    __syncthreads();
     for (int i = tid; i < N; i += kThreads) {
         float a = 0.0f;
-        for (int j = 0; j < N; ++j) a = fmaf(sC[i * N + j], u[j], a);
+        for (int j = 0; j < N; ++j) a = fmaf(sCt[j * N + i], u[j], a);
         sCu[i] = a;
     }
     __syncthreads();
-    for (int64_t t = t0; t < t1; ++t) {
-        float* o = o_out + ((b * p.L + t) * p.H + h) * N;
-        for (int j = tid; j < N; j += kThreads) sV[j] = o[j];
+    for (int e = tid; e < NN; e += kThreads) sC[e] = sCt[e];     // sC now holds C transposed
+    __syncthreads();
+    constexpr int TT = NN / N;              // tokens per tile (sQ holds TT rows of N)
+    float* sVt = sQ;
+    for (int64_t tb = t0; tb < t1; tb += TT) {
+        const int nt = (int)((t1 - tb < TT) ? t1 - tb : TT);
+        for (int e = tid; e < nt * N; e += kThreads) {
+            const int tt = e / N, j = e % N;
+            sVt[e] = o_out[((b * p.L + tb + tt) * p.H + h) * N + j];
+        }
         __syncthreads();
-        for (int i = tid; i < N; i += kThreads) {
+        for (int e = tid; e < nt * N; e += kThreads) {
+            const int tt = e / N, i = e % N;
+            const float* v = sVt + tt * N;
             float a = 0.0f;
-            for (int j = 0; j < N; ++j) a = fmaf(sC[i * N + j], sV[j], a);
-            o[i] = sCu[i] + a;
+#pragma unroll 8
+            for (int j = 0; j < N; ++j) a = fmaf(sC[j * N + i], v[j], a);
+            o_out[((b * p.L + tb + tt) * p.H + h) * N + i] = sCu[i] + a;
         }
         __syncthreads();
     }
+    // snapshots need C itself again
+    for (int e = tid; e < NN; e += kThreads) sQ[e] = sC[e];
+    __syncthreads();
+    for (int e = tid; e < NN; e += kThreads) sC[(e % N) * N + e / N] = sQ[e];
+    __syncthreads();
     if (snap_every > 0) {
         const int64_t first = ((t0 + snap_every) / snap_every) * snap_every;   // 1-based
         for (int64_t t1b = first; t1b <= t1; t1b += snap_every) {
