@@ -17,6 +17,8 @@
 // expm1 so that the diagonal keeps its small deviation exactly.
 #include <string.h>
 
+#include <atomic>
+
 #include "mru_internal.cuh"
 
 namespace mru {
@@ -27,13 +29,15 @@ constexpr int N = 32;
 constexpr int NN = N * N;
 constexpr int ROWB = 80;             // padded shared-memory row stride in bytes (32 bf16 + 16 B)
 constexpr int SLICEB = N * ROWB;     // one token-head slice: 2,560 bytes
-constexpr int SUB = n16::kSub;       // tokens per pass (the chunk length is a multiple)
-constexpr int WARPS = 4;
+constexpr int SUB = n16::kSub;       // the chunk length is a multiple of it
+constexpr int ST = 2;                // tokens per pipeline stage
+constexpr int NS = 2;                // stages per warp: one in flight while one is consumed
+constexpr int WARPS = 4;             // warps per CTA (4 CTAs per SM)
 constexpr int THREADS = 32 * WARPS;
 
 struct WarpSmem {
-    unsigned char x[SUB][SLICEB];    // 20,480 bytes
-    float dd[SUB][2][N];             // D_i and D_i - 1 per token: 2,048 bytes
+    unsigned char x[NS][ST][SLICEB]; // 10,240 bytes
+    float dd[ST][2][N];              // D_i and D_i - 1 per token of the stage: 512 bytes
 };
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
@@ -41,7 +45,12 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
     const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int Pending>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(Pending));
+}
 
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* smem_row)
 {
@@ -240,143 +249,234 @@ __device__ __forceinline__ void store_state(float* out, const State& st, int g, 
                     make_float2(st[mt][nt][2 * h], st[mt][nt][2 * h + 1]);
 }
 
-// Copy the pass's slices (2 KB each, 128 granules) and form D, D - 1.
-__device__ __forceinline__ void load_pass(const KParams& p, WarpSmem& ws, const uint16_t* xb, int64_t tok, int64_t t0,
-                                          int nt, int lane)
+// D_i = exp(d tanh M_ii) and D_i - 1 (expm1) for the nt tokens of a stage
+// (lane i: diagonal entry i).
+__device__ __forceinline__ void stage_dd(const KParams& p, WarpSmem& ws, const unsigned char (*xs)[SLICEB], int nt,
+                                         int lane)
 {
-#pragma unroll
-    for (int i = 0; i < SUB * 128 / 32; ++i) {
-        const int gi = lane + 32 * i;
-        const int j = gi >> 7, q16 = gi & 127, row = q16 >> 2, c4 = q16 & 3;
-        if (j < nt) cp_async16(ws.x[j] + row * ROWB + c4 * 16, xb + (t0 + j) * tok + row * N + c4 * 8);
-    }
-    cp_async_wait_all();
-    __syncwarp();
     for (int j = 0; j < nt; ++j) {
-        const uint16_t mb = *reinterpret_cast<const uint16_t*>(ws.x[j] + lane * ROWB + lane * 2);
+        const uint16_t mb = *reinterpret_cast<const uint16_t*>(xs[j] + lane * ROWB + lane * 2);
         const float mii = __uint_as_float((uint32_t)mb << 16);
-        const float z = p.ldu_d * tanhf(mii);
-        const float dm1 = expm1f(z);
+        const float dm1 = expm1f(p.ldu_d * tanhf(mii));
         ws.dd[j][0][lane] = 1.0f + dm1;
         ws.dd[j][1][lane] = dm1;
     }
     __syncwarp();
 }
 
-struct ChainIx {
+// chain id -> (b, k, h), h fastest (chain ids stay below 2^31).
+struct Chain {
     int64_t b, h, k, tbeg, tend;
 };
-__device__ __forceinline__ ChainIx chain_ix(const KParams& p, int64_t chain)
+__device__ __forceinline__ Chain chain_at(const KParams& p, int64_t chain)
 {
-    ChainIx c;
-    c.h = chain % p.H;
-    const int64_t bk = chain / p.H;
-    c.k = bk % p.K;
-    c.b = bk / p.K;
+    Chain c;
+    const uint32_t ci = (uint32_t)chain;
+    const uint32_t bk = fastdiv(ci, p.h_mul, p.h_shr);
+    const uint32_t b = fastdiv(bk, p.k_mul, p.k_shr);
+    c.h = ci - bk * (uint32_t)p.H;
+    c.k = bk - b * (uint32_t)p.K;
+    c.b = b;
     c.tbeg = c.k * p.chunk;
     c.tend = (c.tbeg + p.chunk < p.L) ? c.tbeg + p.chunk : p.L;
     return c;
 }
 
-__global__ void __launch_bounds__(THREADS)
+// The producer side of a warp's pipeline: the next stage of ST token slices
+// (2 KB each, copied as 128 granules into rows padded to ROWB bytes) along
+// the warp's chains w, w + W, ...
+struct Feed {
+    int64_t chain, stride, nchains, tok;
+    int64_t t, tend;
+    const uint16_t* xb;
+
+    __device__ __forceinline__ void set(const KParams& p, const uint16_t* x)
+    {
+        if (chain >= nchains) return;
+        const Chain c = chain_at(p, chain);
+        xb = x + (c.b * p.L * p.H + c.h) * NN;
+        t = c.tbeg;
+        tend = c.tend;
+    }
+    // Copies the next stage into dst (nothing once the chains are done) and
+    // commits a cp.async group either way.
+    __device__ __forceinline__ void issue(unsigned char (*dst)[SLICEB], int lane, const KParams& p, const uint16_t* x)
+    {
+        if (chain < nchains) {
+            const int nt = (tend - t < ST) ? (int)(tend - t) : ST;
+#pragma unroll
+            for (int i = 0; i < ST * 128 / 32; ++i) {
+                const int gi = lane + 32 * i;
+                const int j = gi >> 7, g16 = gi & 127, row = g16 >> 2, c4 = g16 & 3;
+                if (j < nt) cp_async16(dst[j] + row * ROWB + c4 * 16, xb + (t + j) * tok + row * N + c4 * 8);
+            }
+            t += ST;
+            if (t >= tend) {
+                chain += stride;
+                set(p, x);
+            }
+        }
+        cp_async_commit();
+    }
+};
+
+__global__ void __launch_bounds__(THREADS, 4)
 k32_reduce(KParams p, const uint16_t* __restrict__ x, float* __restrict__ totals)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     WarpSmem& ws = reinterpret_cast<WarpSmem*>(smem_raw)[warp];
-    const int64_t chain = (int64_t)blockIdx.x * WARPS + warp;
-    if (chain >= p.B * p.H * p.K) return;
-    const ChainIx c = chain_ix(p, chain);
-    const int64_t tok = p.H * NN;
-    const uint16_t* xb = x + (c.b * p.L * p.H + c.h) * NN;
-    State st;
+    const int64_t nchains = p.B * p.H * p.K;
+    const int64_t first = (int64_t)blockIdx.x * WARPS + warp, stride = (int64_t)gridDim.x * WARPS;
+    Feed feed;
+    feed.chain = first;
+    feed.stride = stride;
+    feed.nchains = nchains;
+    feed.tok = p.H * NN;
+    feed.set(p, x);
+#pragma unroll
+    for (int s = 0; s < NS - 1; ++s) feed.issue(ws.x[s], lane, p, x);
+    int cs = 0, ps = NS - 1;
+    for (int64_t chain = first; chain < nchains; chain += stride) {
+        const Chain c = chain_at(p, chain);
+        State st;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) st[mt][nt][i] = 0.0f;
+        for (int64_t t0 = c.tbeg; t0 < c.tend; t0 += ST) {
+            feed.issue(ws.x[ps], lane, p, x);
+            ps = (ps + 1 == NS) ? 0 : ps + 1;
+            cp_async_wait<NS - 1>();
+            __syncwarp();
+            const int ntk = (c.tend - t0 < ST) ? (int)(c.tend - t0) : ST;
+            stage_dd(p, ws, ws.x[cs], ntk, lane);
+            for (int j = 0; j < ntk; ++j) apply_token<true>(st, ws.x[cs][j], ws.dd[j][0], ws.dd[j][1], p.ldu_a, lane);
+            __syncwarp();
+            cs = (cs + 1 == NS) ? 0 : cs + 1;
+        }
+        store_state(totals + ((c.b * p.H + c.h) * p.K + c.k) * NN, st, lane >> 2, lane & 3);
+    }
+}
+
+// The chain's carry C = E1 (I + R0[k-1]) in fp64 (E1 alone for the first
+// chunk of a group), computed straight into the accumulator layout from L2:
+// lane (g, q) forms rows 16 mt + g + 8 h, columns 8 nt + 2 q (+ 1).
+__device__ __forceinline__ void form_carry(const double* e1, const float* rp, int lane, State& st)
+{
+    const int g = lane >> 2, q = lane & 3;
+    double acc[2][2][4][2];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const double2 v = *reinterpret_cast<const double2*>(e1 + (16 * mt + g + 8 * h) * N + 8 * nt + 2 * q);
+                acc[mt][h][nt][0] = v.x;
+                acc[mt][h][nt][1] = v.y;
+            }
+    if (rp) {
+#pragma unroll 2
+        for (int kk = 0; kk < N; ++kk) {
+            double av[2][2];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) av[mt][h] = e1[(16 * mt + g + 8 * h) * N + kk];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const float2 r = *reinterpret_cast<const float2*>(rp + kk * N + 8 * nt + 2 * q);
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        acc[mt][h][nt][0] = fma(av[mt][h], (double)r.x, acc[mt][h][nt][0]);
+                        acc[mt][h][nt][1] = fma(av[mt][h], (double)r.y, acc[mt][h][nt][1]);
+                    }
+            }
+        }
+    }
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) st[mt][nt][i] = 0.0f;
-    for (int64_t t0 = c.tbeg; t0 < c.tend; t0 += SUB) {
-        const int ntk = (c.tend - t0 < SUB) ? (int)(c.tend - t0) : SUB;
-        load_pass(p, ws, xb, tok, t0, ntk, lane);
-        for (int j = 0; j < ntk; ++j) apply_token<true>(st, ws.x[j], ws.dd[j][0], ws.dd[j][1], p.ldu_a, lane);
-        __syncwarp();
-    }
-    store_state(totals + ((c.b * p.H + c.h) * p.K + c.k) * NN, st, lane >> 2, lane & 3);
+            for (int h = 0; h < 2; ++h) {
+                st[mt][nt][2 * h] = (float)acc[mt][h][nt][0];
+                st[mt][nt][2 * h + 1] = (float)acc[mt][h][nt][1];
+            }
 }
 
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, 4)
 k32_apply(KParams p, const uint16_t* __restrict__ x, const float* __restrict__ R0, const double* __restrict__ E1,
           int G, float* __restrict__ S_out)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     WarpSmem& ws = reinterpret_cast<WarpSmem*>(smem_raw)[warp];
-    const int64_t chain = (int64_t)blockIdx.x * WARPS + warp;
-    if (chain >= p.B * p.H * p.K) return;
-    const ChainIx c = chain_ix(p, chain);
-    const int64_t seq = c.b * p.H + c.h;
+    const int64_t nchains = p.B * p.H * p.K;
+    const int64_t first = (int64_t)blockIdx.x * WARPS + warp, stride = (int64_t)gridDim.x * WARPS;
     const int g = lane >> 2, q = lane & 3;
-    State st;
-    // carry C = E1 (I + R0[k-1]) in fp64, each lane a 4 x 8 block, staged in
-    // the x buffer (8 KB of E1, 4 KB of C)
-    {
-        double* sE = reinterpret_cast<double*>(ws.x[0]);
-        float* sC = reinterpret_cast<float*>(ws.x[4]);
-        const int64_t n1 = (p.K + G - 1) / G;
-        const double* e1 = E1 + (seq * n1 + c.k / G) * NN;
-        for (int e = lane; e < NN; e += 32) sE[e] = e1[e];
-        __syncwarp();
-        const int r0 = (lane >> 2) * 4, c0 = (lane & 3) * 8;
-        double acc[4][8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) acc[i][cc] = sE[(r0 + i) * N + c0 + cc];
-        if (c.k % G != 0) {
-            const float* rp = R0 + (seq * p.K + c.k - 1) * NN;
-#pragma unroll 2
-            for (int kk = 0; kk < N; ++kk) {
-                const float4 r1 = *reinterpret_cast<const float4*>(rp + kk * N + c0);
-                const float4 r2 = *reinterpret_cast<const float4*>(rp + kk * N + c0 + 4);
-                const double bv[8] = {r1.x, r1.y, r1.z, r1.w, r2.x, r2.y, r2.z, r2.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const double av = sE[(r0 + i) * N + kk];
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) acc[i][cc] = fma(av, bv[cc], acc[i][cc]);
-                }
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) sC[(r0 + i) * N + c0 + cc] = (float)acc[i][cc];
-        __syncwarp();
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const float2 v = *reinterpret_cast<const float2*>(sC + (16 * mt + g + 8 * h) * N + 8 * nt + 2 * q);
-                    st[mt][nt][2 * h] = v.x;
-                    st[mt][nt][2 * h + 1] = v.y;
-                }
-        __syncwarp();
-    }
     const int64_t tok = p.H * NN;
-    const uint16_t* xb = x + (c.b * p.L * p.H + c.h) * NN;
-    float* ob = S_out + (c.b * p.L * p.H + c.h) * NN;
-    for (int64_t t0 = c.tbeg; t0 < c.tend; t0 += SUB) {
-        const int ntk = (c.tend - t0 < SUB) ? (int)(c.tend - t0) : SUB;
-        load_pass(p, ws, xb, tok, t0, ntk, lane);
-        for (int j = 0; j < ntk; ++j) {
-            apply_token<false>(st, ws.x[j], ws.dd[j][0], ws.dd[j][1], p.ldu_a, lane);
-            store_state(ob + (t0 + j) * tok, st, g, q);
+    const int64_t n1 = (p.K + G - 1) / G;
+    Feed feed;
+    feed.chain = first;
+    feed.stride = stride;
+    feed.nchains = nchains;
+    feed.tok = tok;
+    feed.set(p, x);
+#pragma unroll
+    for (int s = 0; s < NS - 1; ++s) feed.issue(ws.x[s], lane, p, x);
+    int cs = 0, ps = NS - 1;
+    for (int64_t chain = first; chain < nchains; chain += stride) {
+        const Chain c = chain_at(p, chain);
+        const int64_t seq = c.b * p.H + c.h;
+        State st;
+        form_carry(E1 + (seq * n1 + c.k / G) * NN, (c.k % G) ? R0 + (seq * p.K + c.k - 1) * NN : nullptr, lane, st);
+        float* ob = S_out + (c.b * p.L * p.H + c.h) * NN;
+        for (int64_t t0 = c.tbeg; t0 < c.tend; t0 += ST) {
+            feed.issue(ws.x[ps], lane, p, x);
+            ps = (ps + 1 == NS) ? 0 : ps + 1;
+            cp_async_wait<NS - 1>();
+            __syncwarp();
+            const int ntk = (c.tend - t0 < ST) ? (int)(c.tend - t0) : ST;
+            stage_dd(p, ws, ws.x[cs], ntk, lane);
+            for (int j = 0; j < ntk; ++j) {
+                apply_token<false>(st, ws.x[cs][j], ws.dd[j][0], ws.dd[j][1], p.ldu_a, lane);
+                store_state(ob + (t0 + j) * tok, st, g, q);
+            }
+            __syncwarp();
+            cs = (cs + 1 == NS) ? 0 : cs + 1;
         }
-        __syncwarp();
     }
+}
+
+// CTAs of a persistent launch: resident CTAs per SM times the SM count,
+// cached per device and kernel slot; no more than the chains need.
+std::atomic<int> g_resident[64][2];
+
+cudaError_t persistent_grid(int slot, const void* kern, int64_t nchains, unsigned& grid)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int res = (dev >= 0 && dev < 64) ? g_resident[dev][slot].load(std::memory_order_relaxed) : 0;
+    if (res <= 0) {
+        int sms = 0, per_sm = 0;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, sizeof(WarpSmem) * WARPS)) !=
+            cudaSuccess)
+            return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+        res = sms * per_sm;
+        if (dev >= 0 && dev < 64) g_resident[dev][slot].store(res, std::memory_order_relaxed);
+    }
+    const int64_t need = (nchains + WARPS - 1) / WARPS;
+    grid = (unsigned)(need < res ? need : res);
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -397,10 +497,13 @@ int32_t preferred_chunk(int64_t token_heads)
 cudaError_t launch_reduce(const KParams& p, const void* x, float* totals, cudaStream_t s)
 {
     const int64_t nchains = p.B * p.H * p.K;
-    const unsigned grid = (unsigned)((nchains + WARPS - 1) / WARPS);
+    if (nchains == 0) return cudaSuccess;
+    if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const size_t sm = sizeof(WarpSmem) * WARPS;
     cudaError_t e = cudaFuncSetAttribute(k32_reduce, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
+    unsigned grid = 0;
+    if ((e = persistent_grid(0, (const void*)k32_reduce, nchains, grid)) != cudaSuccess) return e;
     k32_reduce<<<grid, THREADS, sm, s>>>(p, reinterpret_cast<const uint16_t*>(x), totals);
     return cudaGetLastError();
 }
@@ -409,10 +512,13 @@ cudaError_t launch_apply(const KParams& p, const void* x, const carry::Plan& pl,
                          cudaStream_t s)
 {
     const int64_t nchains = p.B * p.H * p.K;
-    const unsigned grid = (unsigned)((nchains + WARPS - 1) / WARPS);
+    if (nchains == 0) return cudaSuccess;
+    if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const size_t sm = sizeof(WarpSmem) * WARPS;
     cudaError_t e = cudaFuncSetAttribute(k32_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
+    unsigned grid = 0;
+    if ((e = persistent_grid(1, (const void*)k32_apply, nchains, grid)) != cudaSuccess) return e;
     k32_apply<<<grid, THREADS, sm, s>>>(p, reinterpret_cast<const uint16_t*>(x),
                                         reinterpret_cast<const float*>(ws + pl.R[0]),
                                         reinterpret_cast<const double*>(ws + pl.E[1]), pl.G, S_out);
