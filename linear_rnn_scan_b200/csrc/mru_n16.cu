@@ -1023,13 +1023,15 @@ bool supports(const KParams& p, bool readout)
            (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32X3) && p.chunk > 0 && p.chunk % kSub == 0;
 }
 
-// Chunk length: 8 m tokens, m a power of two that keeps at least 16384
-// chains when the workload allows (about seven per warp of a full persistent
-// grid), so that long sequences get long chunks (few chunk totals).
+// Chunk length: 8 m tokens, m a power of two (at most 16) that keeps at
+// least 8192 chains when the workload allows (about three per warp of a full
+// persistent grid), so that long sequences get long chunks (few chunk
+// totals, little carry work per token).  Measured on B200: 32 tokens for
+// 262,144 token-heads, 128 for 2,097,152.
 int32_t preferred_chunk(int64_t token_heads)
 {
     int32_t m = 1;
-    while (m < 16 && token_heads / ((int64_t)kSub * 2 * m) >= 16384) m *= 2;
+    while (m < 16 && token_heads / ((int64_t)kSub * 2 * m) >= 8192) m *= 2;
     return kSub * m;
 }
 
