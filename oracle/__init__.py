@@ -72,6 +72,8 @@ def _load():
                                         fp, dp, dp, dp, fp, dp, dp, ctypes.c_int64, fp, dp, dp,
                                         ctypes.c_int]
             lib.mro_compare.restype = ctypes.c_int
+            lib.mro_backward.argtypes = [P(Problem), vp, dp, dp, dp, dp, ctypes.c_int]
+            lib.mro_backward.restype = ctypes.c_int
             lib.mro_bf16_to_double.argtypes = [ctypes.c_uint16]
             lib.mro_bf16_to_double.restype = ctypes.c_double
             _lib = lib
@@ -131,6 +133,22 @@ def scan(p: Problem, x: np.ndarray, S0: np.ndarray | None = None, nthreads: int 
                           _ptr(S, ctypes.c_double), nthreads or os.cpu_count() or 1)
     _raise(rc, "scan")
     return S
+
+
+def backward(p: Problem, x: np.ndarray, dS: np.ndarray, S0: np.ndarray | None = None,
+             nthreads: int = 0):
+    """Vector-Jacobian product of the scan: (dx [B, L, H*n*n], dS0 [B, H, n, n]
+    or None) from upstream gradients dS [B, L, H, n, n] (fp64)."""
+    x = _check_x(p, x)
+    dS = np.ascontiguousarray(dS, np.float64).reshape(p.B, p.L, p.H, p.n, p.n)
+    S0 = None if S0 is None else np.ascontiguousarray(S0, np.float64).reshape(p.B, p.H, p.n, p.n)
+    dx = np.empty((p.B, p.L, p.H * p.n * p.n), np.float64)
+    dS0 = None if S0 is None else np.empty((p.B, p.H, p.n, p.n), np.float64)
+    rc = _load().mro_backward(ctypes.byref(p), x.ctypes.data, _ptr(S0, ctypes.c_double),
+                              _ptr(dS, ctypes.c_double), _ptr(dx, ctypes.c_double), _ptr(dS0, ctypes.c_double),
+                              nthreads or os.cpu_count() or 1)
+    _raise(rc, "backward")
+    return dx, dS0
 
 
 def readout(p: Problem, x: np.ndarray, u: np.ndarray, snapshot_every: int = 0,

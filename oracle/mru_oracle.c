@@ -366,3 +366,230 @@ int mro_compare(const mro_problem* p, const void* x, const double* S0,
     J.t_end = t_end; J.bh = bh; J.n_bh = n_bh;
     return run_job(&J, nthreads);
 }
+
+/* ---- backward: the vector-Jacobian product of the scan ------------------
+ *
+ * Not described on the pages (they train the MRU but print no gradient); this
+ * is the chain rule of the forward definition above, written out plainly.
+ * With G_t = dL/dS_t (all later states included) and upstream gradients dS_t:
+ *     G_L = dS_L,   G_{t-1} = dS_{t-1} + G_t X_t^T,
+ *     dL/dX_t = S_{t-1}^T G_t (S_0 = S0 or I),   dL/dS0 = G_1 X_1^T.
+ * Through the construction of X_t from the embedding slice M:
+ *   reshape:   X = add_identity I + alpha M          dM = alpha dX
+ *   det-corr.: X = c Xr, c = |det Xr|^(-1/n)         dXr = c (dX - <dX, Xr> Xr^-T / n)
+ *              (d log|det Xr| = tr(Xr^-1 dXr)),      dM = alpha dXr
+ *   LDU:       X = L D U                             dL = dX (D U)^T, d(DU) = L^T dX,
+ *              dU = D d(DU), dD_i = sum_j d(DU)_ij U_ij;
+ *              dM_ij = a dL_ij (i > j), a dU_ij (i < j),
+ *              dM_ii = dD_i D_i d (1 - tanh^2 M_ii).
+ * The inverse is textbook Gauss-Jordan with partial pivoting. */
+
+static void transpose(int n, const double* A, double* T)
+{
+    for (int i = 0; i < n; ++i)
+        for (int j = 0; j < n; ++j) T[j * n + i] = A[i * n + j];
+}
+
+/* A^-1 into Ai by Gauss-Jordan elimination with partial pivoting on [A | I]
+ * (A is destroyed).  Returns 0 when A is singular. */
+static int invert(int n, double* A, double* Ai)
+{
+    set_identity(n, Ai);
+    for (int k = 0; k < n; ++k) {
+        int piv = k;
+        double best = fabs(A[k * n + k]);
+        for (int i = k + 1; i < n; ++i)
+            if (fabs(A[i * n + k]) > best) { best = fabs(A[i * n + k]); piv = i; }
+        if (best == 0.0) return 0;
+        if (piv != k)
+            for (int j = 0; j < n; ++j) {
+                double t = A[k * n + j]; A[k * n + j] = A[piv * n + j]; A[piv * n + j] = t;
+                t = Ai[k * n + j]; Ai[k * n + j] = Ai[piv * n + j]; Ai[piv * n + j] = t;
+            }
+        const double pk = A[k * n + k];
+        for (int j = 0; j < n; ++j) { A[k * n + j] /= pk; Ai[k * n + j] /= pk; }
+        for (int i = 0; i < n; ++i) {
+            if (i == k) continue;
+            const double f = A[i * n + k];
+            if (f == 0.0) continue;
+            for (int j = 0; j < n; ++j) { A[i * n + j] -= f * A[k * n + j]; Ai[i * n + j] -= f * Ai[k * n + j]; }
+        }
+    }
+    return 1;
+}
+
+/* dM from dX for one token-head (the construction's chain rule above).
+ * work holds 6 n*n doubles. */
+static int lift_vjp(const mro_problem* p, const void* x, int64_t b, int64_t t, int64_t h,
+                    const double* dX, double* dM, double* work)
+{
+    const int n = p->n;
+    const int64_t nn = (int64_t)n * n;
+    const int64_t base = ((b * p->L + t) * p->H + h) * nn;
+    double* M = work;
+    for (int64_t e = 0; e < nn; ++e) M[e] = widen(p, x, base + e);
+    if (p->mode == 0) {
+        for (int64_t e = 0; e < nn; ++e) dM[e] = (double)p->alpha * dX[e];
+        return MRO_OK;
+    }
+    if (p->mode == 1) {
+        const double a = (double)p->alpha;
+        double* Xr = work + nn;
+        double* A = work + 2 * nn;
+        double* Ai = work + 3 * nn;
+        for (int64_t e = 0; e < nn; ++e) Xr[e] = a * M[e];
+        if (p->add_identity)
+            for (int i = 0; i < n; ++i) Xr[i * n + i] += 1.0;
+        memcpy(A, Xr, (size_t)nn * sizeof(double));
+        double la; int sg;
+        if (!log_abs_det(n, A, &la, &sg) || !isfinite(la)) return MRO_ERR_SINGULAR;
+        const double c = exp(-la / n);
+        memcpy(A, Xr, (size_t)nn * sizeof(double));
+        if (!invert(n, A, Ai)) return MRO_ERR_SINGULAR;
+        double inner = 0.0;                       /* <dX, Xr> */
+        for (int64_t e = 0; e < nn; ++e) inner += dX[e] * Xr[e];
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j) {
+                const double dXr = c * (dX[i * n + j] - inner * Ai[j * n + i] / n);   /* Xr^-T */
+                dM[i * n + j] = a * dXr;
+            }
+        return MRO_OK;
+    }
+    if (p->mode == 2) {
+        const double a = (double)p->ldu_offdiag, d = (double)p->ldu_diag;
+        double* Lm = work + nn;
+        double* U = work + 2 * nn;
+        double* DU = work + 3 * nn;
+        double* T = work + 4 * nn;
+        double* T2 = work + 5 * nn;
+        double D[64 * 8];                          /* n <= 512 */
+        set_identity(n, Lm);
+        set_identity(n, U);
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j) {
+                if (i > j) Lm[i * n + j] = a * M[i * n + j];
+                if (i < j) U[i * n + j] = a * M[i * n + j];
+            }
+        for (int i = 0; i < n; ++i) D[i] = exp(d * tanh(M[i * n + i]));
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j) DU[i * n + j] = D[i] * U[i * n + j];
+        /* dL = dX (DU)^T */
+        transpose(n, DU, T);
+        double* dL = T2;
+        matmul(n, dX, T, dL);
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < i; ++j) dM[i * n + j] = a * dL[i * n + j];
+        /* d(DU) = L^T dX */
+        transpose(n, Lm, T);
+        double* dDU = T2;
+        matmul(n, T, dX, dDU);
+        for (int i = 0; i < n; ++i) {
+            double dD = 0.0;
+            for (int j = 0; j < n; ++j) dD += dDU[i * n + j] * U[i * n + j];
+            const double th = tanh(M[i * n + i]);
+            dM[i * n + i] = dD * D[i] * d * (1.0 - th * th);
+            for (int j = i + 1; j < n; ++j) dM[i * n + j] = a * D[i] * dDU[i * n + j];
+        }
+        return MRO_OK;
+    }
+    return MRO_ERR_ARG;
+}
+
+/* Backward of one (b, h) sequence.  dS: [B,L,H,n,n]; dx: [B,L,H*n*n];
+ * dS0: [B,H,n,n] or NULL.  Holds every X_t and S_t of the sequence. */
+static int backward_sequence(const mro_problem* p, const void* x, const double* S0, const double* dS,
+                             double* dx, double* dS0, int64_t bh)
+{
+    const int n = p->n;
+    const int64_t nn = (int64_t)n * n, L = p->L;
+    const int64_t b = bh / p->H, h = bh % p->H;
+    double* X = malloc(sizeof(double) * (size_t)(L * nn + 1));
+    double* S = malloc(sizeof(double) * (size_t)((L + 1) * nn));
+    double* work = malloc(sizeof(double) * (size_t)(11 * nn));    /* 5 n*n here + 6 n*n for lift_vjp */
+    int rc = MRO_OK;
+    if (!X || !S || !work) { rc = MRO_ERR_ARG; goto done; }
+    /* forward: S[0] = S0 (or I), S[t+1] = S[t] X_{t+1} */
+    if (S0) memcpy(S, S0 + bh * nn, (size_t)nn * sizeof(double));
+    else set_identity(n, S);
+    for (int64_t t = 0; t < L; ++t) {
+        if ((rc = mro_lift(p, x, b, t, h, X + t * nn, work)) != MRO_OK) goto done;
+        matmul(n, S + t * nn, X + t * nn, S + (t + 1) * nn);
+    }
+    /* reverse */
+    double* G = work;              /* G_t */
+    double* Gn = work + nn;
+    double* Xt = work + 2 * nn;
+    double* dX = work + 3 * nn;
+    double* St = work + 4 * nn;
+    if (L > 0) memcpy(G, dS + ((b * L + (L - 1)) * p->H + h) * nn, (size_t)nn * sizeof(double));
+    for (int64_t t = L - 1; t >= 0; --t) {
+        transpose(n, S + t * nn, St);                 /* S_{t-1}^T (position t holds X_{t+1}) */
+        matmul(n, St, G, dX);
+        if ((rc = lift_vjp(p, x, b, t, h, dX, dx + ((b * L + t) * p->H + h) * nn, work + 5 * nn)) != MRO_OK)
+            goto done;
+        transpose(n, X + t * nn, Xt);
+        matmul(n, G, Xt, Gn);                         /* G_t X_t^T */
+        if (t > 0) {
+            const double* ds = dS + ((b * L + (t - 1)) * p->H + h) * nn;
+            for (int64_t e = 0; e < nn; ++e) G[e] = ds[e] + Gn[e];
+        } else if (dS0) {
+            memcpy(dS0 + bh * nn, Gn, (size_t)nn * sizeof(double));
+        }
+    }
+    if (L == 0 && dS0) memset(dS0 + bh * nn, 0, (size_t)nn * sizeof(double));
+done:
+    free(X);
+    free(S);
+    free(work);
+    return rc;
+}
+
+typedef struct {
+    const mro_problem* p;
+    const void* x;
+    const double* S0;
+    const double* dS;
+    double* dx;
+    double* dS0;
+    int64_t next;
+    pthread_mutex_t lock;
+    int status;
+} bwd_job_t;
+
+static void* bwd_worker(void* arg)
+{
+    bwd_job_t* J = arg;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        const int64_t i = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (i >= J->p->B * J->p->H) break;
+        const int rc = backward_sequence(J->p, J->x, J->S0, J->dS, J->dx, J->dS0, i);
+        if (rc != MRO_OK) {
+            pthread_mutex_lock(&J->lock);
+            J->status = rc;
+            pthread_mutex_unlock(&J->lock);
+        }
+    }
+    return NULL;
+}
+
+/* dx [B,L,H*n*n] (gradient with respect to the widened embedding values) and
+ * dS0 [B,H,n,n] (may be NULL) from upstream gradients dS [B,L,H,n,n]. */
+int mro_backward(const mro_problem* p, const void* x, const double* S0, const double* dS,
+                 double* dx, double* dS0, int nthreads)
+{
+    if (check_problem(p) != MRO_OK || !dS || !dx) return MRO_ERR_ARG;
+    if (p->mode == 2 && p->n > 512) return MRO_ERR_ARG;
+    bwd_job_t J;
+    memset(&J, 0, sizeof J);
+    J.p = p; J.x = x; J.S0 = S0; J.dS = dS; J.dx = dx; J.dS0 = dS0;
+    pthread_mutex_init(&J.lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    pthread_t th[256];
+    if (nthreads > 256) nthreads = 256;
+    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, bwd_worker, &J);
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    pthread_mutex_destroy(&J.lock);
+    return J.status;
+}
