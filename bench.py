@@ -520,6 +520,93 @@ def run_ours(args, w):
     return 0
 
 
+def run_backward(args, w):
+    """One step = one mru_scan_backward over the whole workload (gradients of
+    sum <dS, S> with respect to the embeddings), with x, the forward states
+    and the upstream gradients resident in HBM.  Not part of the default run."""
+    import torch
+
+    from linear_rnn_scan_b200 import mru
+
+    if w.readout:
+        print(json.dumps({"impl": "ours", "direction": "backward", "unavailable":
+                          "the backward covers the full-state output, not the readout"}), flush=True)
+        return 0
+    local = env_int("LOCAL_RANK", 0)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks("nccl", dev)
+    p = mru.problem_from_workload(w)
+    x_np = gen.make_x(w, seed=w.seed + ranks.rank)
+    if w.x_dtype == "bf16":
+        x = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(dev)
+    else:
+        x = torch.from_numpy(x_np).to(dev)
+    S = mru.scan_fused_t(p, x)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 17)
+    dS = torch.randn(S.shape, generator=g, device=dev, dtype=torch.float32)
+    dx = torch.empty((w.B, w.L, w.H * w.n * w.n), dtype=torch.float32, device=dev)
+    ws = torch.empty(mru.backward_workspace_size(p), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        rc = mru.scan_backward(p, x.data_ptr(), None, S.data_ptr(), dS.data_ptr(), dx.data_ptr(), None,
+                               ws.data_ptr(), ws.numel(), stream.cuda_stream)
+        if rc != mru.OK:
+            raise mru.MruError(rc, "mru_scan_backward")
+
+    for _ in range(args.warmup):
+        step()
+    st = mru.last_device_status(ws.data_ptr(), stream.cuda_stream)
+    if st != mru.OK:
+        raise mru.MruError(st, "device status after warm-up")
+    torch.cuda.synchronize()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        ev1.synchronize()
+    torch.cuda.synchronize()
+    ranks.barrier()
+    ms = ranks.max(ev0.elapsed_time(ev1) / args.steps)
+    names = ["k_bwd_local", "k_bwd_carry", "k_bwd_apply"]
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for e in evs:
+        e.record(stream)
+    torch.cuda.synchronize()
+    mru.set_profile_events([e.cuda_event for e in evs])
+    step()
+    mru.set_profile_events(None)
+    torch.cuda.synchronize()
+    kms = {names[i]: round(evs[2 * i].elapsed_time(evs[2 * i + 1]), 5) for i in range(3)}
+    # algorithmic bytes per token-head: x in, forward state in, upstream
+    # gradient in, embedding gradient out
+    nn = w.n * w.n
+    xb = 2 if w.x_dtype == "bf16" else 4
+    unit_bytes = nn * (xb + 4 + 4 + 4)
+    peaks = read_peaks()
+    dom = max(kms, key=kms.get)
+    achieved = unit_bytes * w.token_heads / (kms[dom] / 1e3) / 1e9
+    if ranks.printer:
+        print(json.dumps({
+            "metric": "MRU scan backward token·heads/s, 1×B200", "direction": "backward",
+            "value": aggregate_rate(ranks.world, w.token_heads, ms), "unit": UNIT, "n_gpus": ranks.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded N(0,1) embeddings "
+            "and upstream gradients)", "config": workload_config(w, None), "clocks": clocks.summary(),
+            "gpu_launches": 3 * args.steps, "kernels_ms": kms,
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "algorithmic_bytes_per_launch": unit_bytes * w.token_heads}}), flush=True)
+    ranks.close()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -530,11 +617,14 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true", help="time mru_scan_backward instead (not the default)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)      # at least 3 untimed warm-up steps, always
     w = gen.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.backward:
+        return run_backward(args, w)
     return run_ours(args, w)
 
 

@@ -115,6 +115,34 @@ mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0,
                           const mru_readout* ro, float* S_out, float* o_out,
                           void* ws, size_t ws_bytes, void* stream);
 
+/* Backward (vector-Jacobian product) of mru_scan_fused without the readout.
+ * The pages train the MRU but print no gradient: this is the chain rule of
+ * the forward definition ("MRU Update: An independent developer's
+ * alternative to Attention is now running successfully", section "What MRU
+ * Actually Does": S_t = S_{t-1} X_t; construction variants from "Improving
+ * Matrix Recurrent Units as an Attention Alternative", "Technical Deep
+ * Dive").  With G_t = dL/dS_t (later states included):
+ *   G_L = dS_L,  G_{t-1} = dS_{t-1} + G_t X_t^T,
+ *   dL/dX_t = S_{t-1}^T G_t,  dL/dS0 = G_1 X_1^T,
+ * then through the construction of X_t from the embedding slice M:
+ *   reshape: alpha dX;  determinant-corrected (X = c Xr):
+ *   alpha c (dX - <dX, Xr> Xr^-T / n);  LDU: through L, D and U.
+ *   x      [B, L, H*n*n] the forward's embeddings (f32 or bf16)
+ *   S0     [B, H, n, n] fp32 or NULL (identity), as in the forward
+ *   S_fwd  [B, L, H, n, n] fp32, the forward's states (mru_scan_fused output)
+ *   dS     [B, L, H, n, n] fp32 upstream gradients of every S_t
+ *   dx     [B, L, H*n*n] fp32 out: gradient with respect to the (widened)
+ *          embedding values
+ *   dS0    [B, H, n, n] fp32 out, or NULL
+ * Every pointer 16-byte aligned; dx and dS0 alias no input.  The workspace
+ * holds mru_backward_workspace_size(p) bytes.  fp32 arithmetic (fp64 for the
+ * right-to-left scan of the chunk gradients), for every n and mode; a
+ * singular matrix sets MRU_ERR_SINGULAR in the workspace status word. */
+size_t mru_backward_workspace_size(const mru_problem* p);
+mru_status mru_scan_backward(const mru_problem* p, const void* x, const float* S0, const float* S_fwd,
+                             const float* dS, float* dx, float* dS0, void* ws, size_t ws_bytes,
+                             void* stream);
+
 /* Synchronises `stream` and returns the device-detected status of the last
  * call that used this workspace (MRU_OK, MRU_ERR_SINGULAR, MRU_ERR_TIMEOUT). */
 mru_status mru_last_device_status(const void* ws, void* stream);

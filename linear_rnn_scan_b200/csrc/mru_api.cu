@@ -119,6 +119,31 @@ Workspace layout(const KParams& k, bool readout)
     return W;
 }
 
+// The backward's chunking: the generic chunk (or the caller's) and its
+// workspace.
+KParams make_bwd_params(const mru_problem& p)
+{
+    KParams k = make_params(p, SRC_EMBEDDING, false);
+    k.chunk = p.chunk > 0 ? p.chunk : generic_chunk(p);
+    k.K = ceil_div(p.L, k.chunk);
+    fastdiv_magic(k.K, k.k_mul, k.k_shr);
+    return k;
+}
+
+BwdWorkspace bwd_layout(const KParams& k)
+{
+    BwdWorkspace W;
+    memset(&W, 0, sizeof W);
+    const size_t nn = (size_t)k.n * k.n, chains = (size_t)(k.B * k.H * k.K);
+    size_t off = 0;
+    W.status = off; off += 256;
+    W.gloc = off; off = round_up(off + chains * nn * sizeof(float), 256);
+    W.wq = off;   off = round_up(off + chains * nn * sizeof(float), 256);
+    W.gin = off;  off = round_up(off + chains * nn * sizeof(float), 256);
+    W.bytes = off;
+    return W;
+}
+
 cudaEvent_t g_prof_events[64];
 int g_prof_count = 0;
 
@@ -292,6 +317,38 @@ const char* mru_status_string(mru_status s)
         case MRU_ERR_TIMEOUT: return "device-side wait timed out";
         default: return "unknown status";
     }
+}
+
+size_t mru_backward_workspace_size(const mru_problem* p)
+{
+    if (check_problem(p) != MRU_OK) return 0;
+    return bwd_layout(make_bwd_params(*p)).bytes;
+}
+
+mru_status mru_scan_backward(const mru_problem* p, const void* x, const float* S0, const float* S_fwd,
+                             const float* dS, float* dx, float* dS0, void* ws, size_t ws_bytes, void* stream)
+{
+    mru_status st = check_problem(p);
+    if (st != MRU_OK) return st;
+    if (!x || !S_fwd || !dS || !dx || !ws) return MRU_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(S_fwd) || !aligned16(dS) || !aligned16(dx) || !aligned16(ws))
+        return MRU_ERR_INVALID_ARG;
+    if ((S0 && !aligned16(S0)) || (dS0 && !aligned16(dS0))) return MRU_ERR_INVALID_ARG;
+    if ((const void*)dx == x || (const void*)dx == (const void*)S_fwd || (const void*)dx == (const void*)dS)
+        return MRU_ERR_INVALID_ARG;
+    if (dS0 && ((const void*)dS0 == (const void*)S0 || (const void*)dS0 == (const void*)dx)) return MRU_ERR_INVALID_ARG;
+    const KParams k = make_bwd_params(*p);
+    const BwdWorkspace W = bwd_layout(k);
+    if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = reset_status(ws, s)) != MRU_OK) return st;
+    if (p->B * p->H * p->L == 0) {
+        // no state depends on S0 when L = 0
+        if (dS0 && p->B * p->H > 0)
+            return from_cuda(cudaMemsetAsync(dS0, 0, sizeof(float) * (size_t)(p->B * p->H * p->n * p->n), s));
+        return MRU_OK;
+    }
+    return from_cuda(launch_backward(k, x, S0, S_fwd, dS, dx, dS0, ws, W, s));
 }
 
 }  // extern "C"

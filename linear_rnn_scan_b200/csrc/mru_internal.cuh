@@ -108,6 +108,15 @@ struct Workspace {
     size_t bytes;        // total
 };
 
+// Backward workspace (mru_scan_backward).
+struct BwdWorkspace {
+    size_t status;       // uint32 status word
+    size_t gloc;         // float [B*H, K, n, n]  local gradient at each chunk's first token
+    size_t wq;           // float [B*H, K, n, n]  W_k - I, W_k = X_{t0+1} ... X_{t1}
+    size_t gin;          // float [B*H, K, n, n]  gradient entering each chunk from the right
+    size_t bytes;
+};
+
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Benchmark hook (mru_api.cu): records the caller's event for kernel slot
@@ -152,6 +161,8 @@ cudaError_t launch_build_states(const KParams& p, const void* x, float* X_out, i
 cudaError_t launch_scan(const KParams& p, const void* src, const float* S0, const float* u,
                         int64_t snap_every, float* S_out, float* o_out, float* snaps,
                         void* ws_base, const Workspace& W, cudaStream_t s, int* launches);
+cudaError_t launch_backward(const KParams& p, const void* x, const float* S0, const float* S_fwd, const float* dS,
+                            float* dx, float* dS0, void* ws_base, const BwdWorkspace& W, cudaStream_t s);
 // Name of the i-th kernel one launch_scan call starts for this problem.
 const char* kernel_name(const KParams& p, bool readout, int i);
 // mru_math the kernels for this problem actually use (MRU_MATH_FP32 for the

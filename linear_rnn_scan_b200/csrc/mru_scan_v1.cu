@@ -531,11 +531,393 @@ k_fixup(KParams p, const float* carry, const float* u, int64_t snap_every, float
     }
 }
 
+// ---- backward (vector-Jacobian product) -------------------------------------
+//
+// With G_t = dL/dS_t (every later state included): G_L = dS_L,
+// G_{t-1} = dS_{t-1} + G_t X_t^T, dL/dX_t = S_{t-1}^T G_t, dL/dS0 = G_1 X_1^T
+// (the chain rule of S_t = S_{t-1} X_t).  Chunked like the forward scan:
+//   k_bwd_local   per chunk [t0, t1) with a zero gradient entering from the
+//                 right: the local G at t0 (g_k) and W_k - I with
+//                 W_k = X_{t0+1} ... X_{t1} (through the next chunk's first
+//                 matrix; split form, left multiplications);
+//   k_bwd_carry   per sequence, right to left in fp64: the gradient entering
+//                 chunk k from the right, Gin_{K-1} = 0,
+//                 Gin_{k-1} = g_k + Gin_k W_k^T;
+//   k_bwd_apply   per chunk: G from Gin_k down to t0 again, dX_t from the
+//                 forward states, and the construction's chain rule to the
+//                 embedding gradient (reshape: alpha dX; determinant-corrected:
+//                 alpha c (dX - <dX, Xr> Xr^-T / n); LDU: through L, D, U).
+
+// C = A B^T (trans) or A B of N x N matrices in shared memory, each thread
+// its outputs e = tid + r * kThreads; the whole CTA calls it.
+template <int N, bool BT>
+__device__ __forceinline__ void cta_product(const float* A, const float* Bm, float (&acc)[(N * N + kThreads - 1) / kThreads])
+{
+    constexpr int NN = N * N;
+    constexpr int PER = (NN + kThreads - 1) / kThreads;
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+        const int e = threadIdx.x + r * kThreads;
+        float a = 0.0f;
+        if (e < NN) {
+            const int i = e / N, j = e % N;
+#pragma unroll 8
+            for (int k = 0; k < N; ++k) a = fmaf(A[i * N + k], BT ? Bm[j * N + k] : Bm[k * N + j], a);
+        }
+        acc[r] = a;
+    }
+}
+
+// Xr^-1 by Gauss-Jordan elimination with partial pivoting on [sA | sI] in
+// shared memory (sA destroyed, sI ends as the inverse).  The whole CTA calls
+// it; sets the flag slot of sAux when a pivot column is zero.
+template <int N>
+__device__ void cta_inverse(float* sA, float* sI, float* sAux)
+{
+    constexpr int NN = N * N;
+    int* sPiv = aux_piv<N>(sAux);
+    for (int e = threadIdx.x; e < NN; e += kThreads) sI[e] = (e / N == e % N) ? 1.0f : 0.0f;
+    if (threadIdx.x == 0) *aux_flag<N>(sAux) = 0.0f;
+    __syncthreads();
+    for (int k = 0; k < N; ++k) {
+        if (threadIdx.x < 32) {
+            float best = -1.0f;
+            int bi = k;
+            for (int i = k + threadIdx.x; i < N; i += 32) {
+                const float a = fabsf(sA[i * N + k]);
+                if (a > best) { best = a; bi = i; }
+            }
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ob = __shfl_down_sync(0xffffffffu, best, o);
+                const int oi = __shfl_down_sync(0xffffffffu, bi, o);
+                if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+            }
+            if (threadIdx.x == 0) {
+                *sPiv = bi;
+                if (!(best > 0.0f)) *aux_flag<N>(sAux) = 1.0f;
+            }
+        }
+        __syncthreads();
+        const int piv = *sPiv;
+        if (piv != k)
+            for (int j = threadIdx.x; j < N; j += kThreads) {
+                float a = sA[k * N + j]; sA[k * N + j] = sA[piv * N + j]; sA[piv * N + j] = a;
+                a = sI[k * N + j]; sI[k * N + j] = sI[piv * N + j]; sI[piv * N + j] = a;
+            }
+        __syncthreads();
+        const float pk = sA[k * N + k];
+        const float r = (pk != 0.0f) ? 1.0f / pk : 0.0f;
+        __syncthreads();
+        for (int j = threadIdx.x; j < N; j += kThreads) {
+            sA[k * N + j] *= r;
+            sI[k * N + j] *= r;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < NN; e += kThreads) {
+            const int i = e / N, j = e % N;
+            if (i == k) continue;
+            const float f = sA[i * N + k];
+            sI[e] = fmaf(-f, sI[k * N + j], sI[e]);
+        }
+        for (int e = threadIdx.x; e < NN; e += kThreads) {
+            const int i = e / N, j = e % N;
+            if (i == k || j == k) continue;
+            sA[e] = fmaf(-sA[i * N + k], sA[k * N + j], sA[e]);
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < N; i += kThreads)
+            if (i != k) sA[i * N + k] = 0.0f;
+        __syncthreads();
+    }
+}
+
+template <int N>
+__global__ void __launch_bounds__(kThreads)
+k_bwd_local(KParams p, const void* src, const float* __restrict__ dS, float* __restrict__ gloc,
+            float* __restrict__ Wq, uint32_t* status)
+{
+    constexpr int NN = N * N;
+    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    extern __shared__ float smem[];
+    float* sG = smem;
+    float* sR = sG + NN;
+    float* sF = sR + NN;
+    float* sM = sF + NN;
+    float* sW = sM + NN;
+    float* sAux = sW + NN;
+    const int tid = threadIdx.x;
+    const int64_t chain = blockIdx.x;
+    const int64_t k = chain % p.K, bh = chain / p.K;
+    const int64_t h = bh % p.H, b = bh / p.H;
+    const int64_t t0 = k * p.chunk;
+    const int64_t t1 = (t0 + p.chunk < p.L) ? t0 + p.chunk : p.L;
+    const bool more = t1 < p.L;                     // a chunk follows: W_k is needed
+    for (int e = tid; e < NN; e += kThreads) sG[e] = dS[((b * p.L + t1 - 1) * p.H + h) * NN + e];
+    if (more) {
+        cta_construct<N>(p, src, ((b * p.L + t1) * p.H + h) * NN, sF, sM, sW, sAux, status);
+        for (int e = tid; e < NN; e += kThreads) sR[e] = sF[e];
+    }
+    __syncthreads();
+    for (int64_t q = t1 - 1; q > t0; --q) {
+        cta_construct<N>(p, src, ((b * p.L + q) * p.H + h) * NN, sF, sM, sW, sAux, status);
+        float ag[PER], ar[PER];
+        cta_product<N, true>(sG, sF, ag);           // G F^T
+        if (more) cta_product<N, false>(sF, sR, ar);  // F R
+        __syncthreads();
+        const float* ds = dS + ((b * p.L + q - 1) * p.H + h) * NN;
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            if (e < NN) {
+                sG[e] = ds[e] + (sG[e] + ag[r]);     // dS_{q-1} + G X_q^T
+                if (more) sR[e] = sR[e] + (sF[e] + ar[r]);    // X_q W - I
+            }
+        }
+        __syncthreads();
+    }
+    for (int e = tid; e < NN; e += kThreads) {
+        gloc[chain * NN + e] = sG[e];
+        Wq[chain * NN + e] = more ? sR[e] : 0.0f;
+    }
+}
+
+template <int N>
+__global__ void __launch_bounds__(kThreads)
+k_bwd_carry(KParams p, const float* __restrict__ gloc, const float* __restrict__ Wq, float* __restrict__ Gin)
+{
+    constexpr int NN = N * N;
+    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    extern __shared__ double dsm[];
+    double* sGin = dsm;
+    double* sW = sGin + NN;
+    const int tid = threadIdx.x;
+    const int64_t seq = blockIdx.x;
+    for (int e = tid; e < NN; e += kThreads) sGin[e] = 0.0;
+    __syncthreads();
+    for (int64_t k = p.K - 1; k >= 0; --k) {
+        const int64_t chain = seq * p.K + k;
+        for (int e = tid; e < NN; e += kThreads) {
+            Gin[chain * NN + e] = (float)sGin[e];
+            sW[e] = (double)Wq[chain * NN + e];
+        }
+        __syncthreads();
+        if (k == 0) break;
+        double acc[PER];
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            double a = 0.0;
+            if (e < NN) {
+                const int i = e / N, j = e % N;
+                for (int q = 0; q < N; ++q) a = fma(sGin[i * N + q], sW[j * N + q], a);   // Gin Wq^T
+            }
+            acc[r] = a;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            if (e < NN) sGin[e] = (double)gloc[chain * NN + e] + (sGin[e] + acc[r]);
+        }
+        __syncthreads();
+    }
+}
+
+template <int N>
+__global__ void __launch_bounds__(kThreads)
+k_bwd_apply(KParams p, const void* src, const float* __restrict__ S0, const float* __restrict__ S_fwd,
+            const float* __restrict__ dS, const float* __restrict__ Gin, float* __restrict__ dx,
+            float* __restrict__ dS0, uint32_t* status)
+{
+    constexpr int NN = N * N;
+    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    extern __shared__ float smem[];
+    float* sG = smem;
+    float* sF = sG + NN;
+    float* sM = sF + NN;
+    float* sW = sM + NN;
+    float* sS = sW + NN;
+    float* sD = sS + NN;
+    float* sA = sD + NN;
+    float* sAux = sA + NN;
+    float* sRed = sAux + 4 * N + 8;                 // kThreads / 32 partial sums
+    const int tid = threadIdx.x;
+    const int64_t chain = blockIdx.x;
+    const int64_t k = chain % p.K, bh = chain / p.K;
+    const int64_t h = bh % p.H, b = bh / p.H;
+    const int64_t t0 = k * p.chunk;
+    const int64_t t1 = (t0 + p.chunk < p.L) ? t0 + p.chunk : p.L;
+    for (int e = tid; e < NN; e += kThreads) sG[e] = dS[((b * p.L + t1 - 1) * p.H + h) * NN + e];
+    if (t1 < p.L) {
+        // G_{t1-1} = dS_{t1-1} + Gin X_{t1}^T with X_{t1} = I + F
+        cta_construct<N>(p, src, ((b * p.L + t1) * p.H + h) * NN, sF, sM, sW, sAux, status);
+        for (int e = tid; e < NN; e += kThreads) sS[e] = Gin[chain * NN + e];
+        __syncthreads();
+        float ag[PER];
+        cta_product<N, true>(sS, sF, ag);
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            if (e < NN) sG[e] += sS[e] + ag[r];
+        }
+    }
+    __syncthreads();
+    for (int64_t t = t1 - 1; t >= t0; --t) {
+        const int64_t row = (b * p.L + t) * p.H + h;
+        cta_construct<N>(p, src, row * NN, sF, sM, sW, sAux, status);
+        // S_{t-1} (the state before this token)
+        for (int e = tid; e < NN; e += kThreads) {
+            float v;
+            if (t > 0) v = S_fwd[((b * p.L + t - 1) * p.H + h) * NN + e];
+            else v = S0 ? S0[bh * NN + e] : ((e / N == e % N) ? 1.0f : 0.0f);
+            sS[e] = v;
+        }
+        __syncthreads();
+        // dX = S_{t-1}^T G
+        {
+            float acc[PER];
+#pragma unroll
+            for (int r = 0; r < PER; ++r) {
+                const int e = tid + r * kThreads;
+                float a = 0.0f;
+                if (e < NN) {
+                    const int i = e / N, j = e % N;
+#pragma unroll 8
+                    for (int q = 0; q < N; ++q) a = fmaf(sS[q * N + i], sG[q * N + j], a);
+                }
+                acc[r] = a;
+            }
+#pragma unroll
+            for (int r = 0; r < PER; ++r) {
+                const int e = tid + r * kThreads;
+                if (e < NN) sD[e] = acc[r];
+            }
+        }
+        __syncthreads();
+        float* out = dx + row * NN;
+        if (p.mode == MRU_MODE_RESHAPE) {
+            for (int e = tid; e < NN; e += kThreads) out[e] = p.alpha * sD[e];
+        } else if (p.mode == MRU_MODE_DETNORM) {
+            // dXr = c (dX - <dX, Xr> Xr^-T / N), dM = alpha dXr
+            const float c = aux_c<N>(sAux)[0];
+            float part = 0.0f;
+            for (int e = tid; e < NN; e += kThreads) {
+                float xr = p.alpha * sM[e];
+                if (p.add_identity && e / N == e % N) xr += 1.0f;
+                sA[e] = xr;
+                part = fmaf(sD[e], xr, part);
+            }
+            for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+            if ((tid & 31) == 0) sRed[tid >> 5] = part;
+            __syncthreads();
+            float inner = 0.0f;
+            for (int w = 0; w < kThreads / 32; ++w) inner += sRed[w];
+            cta_inverse<N>(sA, sW, sAux);             // sW = Xr^-1
+            const float f = inner / N;
+            for (int e = tid; e < NN; e += kThreads) {
+                const int i = e / N, j = e % N;
+                out[e] = (c == 0.0f) ? 0.0f : p.alpha * c * fmaf(-f, sW[j * N + i], sD[e]);
+            }
+        } else {
+            // LDU: D_i = sAux[i] (and D_i - 1 = sAux[N + i]) from the construction
+            const float a = p.ldu_a;
+            for (int e = tid; e < NN; e += kThreads) {
+                const int i = e / N, j = e % N;
+                float v;
+                if (i > j) {
+                    // dL_ij = sum_{q >= j} dX_iq D_j U_jq (U_jj = 1)
+                    float s2 = sD[i * N + j];
+                    for (int q = j + 1; q < N; ++q) s2 = fmaf(sD[i * N + q], a * sM[j * N + q], s2);
+                    v = a * sAux[j] * s2;
+                } else {
+                    // d(DU)_ij = sum_{q >= i} L_qi dX_qj (L_ii = 1)
+                    float s2 = sD[i * N + j];
+                    for (int q = i + 1; q < N; ++q) s2 = fmaf(a * sM[q * N + i], sD[q * N + j], s2);
+                    v = (i < j) ? a * sAux[i] * s2 : s2;   // diagonal: d(DU)_ii, finished below
+                }
+                sA[e] = v;
+            }
+            __syncthreads();
+            for (int e = tid; e < NN; e += kThreads) {
+                const int i = e / N, j = e % N;
+                if (i != j) { out[e] = sA[e]; continue; }
+                // dD_i = sum_j d(DU)_ij U_ij = d(DU)_ii + sum_{j > i} (dM_ij / (a D_i)) a M_ij
+                float dD = sA[e];
+                for (int q = i + 1; q < N; ++q) {
+                    // d(DU)_iq = dM_iq / (a D_i)
+                    float s2 = sD[i * N + q];
+                    for (int r2 = i + 1; r2 < N; ++r2) s2 = fmaf(a * sM[r2 * N + i], sD[r2 * N + q], s2);
+                    dD = fmaf(s2, a * sM[i * N + q], dD);
+                }
+                const float th = tanhf(sM[e]);
+                out[e] = dD * sAux[i] * p.ldu_d * (1.0f - th * th);
+            }
+        }
+        __syncthreads();
+        // dS0 = G X_1^T, or G_{t-1} = dS_{t-1} + G X_t^T
+        float ag[PER];
+        cta_product<N, true>(sG, sF, ag);
+        __syncthreads();
+        if (t == 0) {
+            if (dS0)
+#pragma unroll
+                for (int r = 0; r < PER; ++r) {
+                    const int e = tid + r * kThreads;
+                    if (e < NN) dS0[bh * NN + e] = sG[e] + ag[r];
+                }
+        } else if (t > t0) {
+            const float* ds = dS + ((b * p.L + t - 1) * p.H + h) * NN;
+#pragma unroll
+            for (int r = 0; r < PER; ++r) {
+                const int e = tid + r * kThreads;
+                if (e < NN) sG[e] = ds[e] + (sG[e] + ag[r]);
+            }
+        }
+        __syncthreads();
+    }
+}
+
+template <int N>
+cudaError_t backward_n(const KParams& p, const void* src, const float* S0, const float* S_fwd, const float* dS,
+                       float* dx, float* dS0, char* ws, const BwdWorkspace& W, cudaStream_t s);
+
 template <typename K>
 cudaError_t set_smem(K kernel, size_t bytes)
 {
     if (bytes <= 48 * 1024) return cudaSuccess;
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int N>
+cudaError_t backward_n(const KParams& p, const void* src, const float* S0, const float* S_fwd, const float* dS,
+                       float* dx, float* dS0, char* ws, const BwdWorkspace& W, cudaStream_t s)
+{
+    constexpr int NN = N * N;
+    uint32_t* status = reinterpret_cast<uint32_t*>(ws + W.status);
+    float* gloc = reinterpret_cast<float*>(ws + W.gloc);
+    float* Wq = reinterpret_cast<float*>(ws + W.wq);
+    float* Gin = reinterpret_cast<float*>(ws + W.gin);
+    const int64_t BH = p.B * p.H;
+    const int64_t chains = BH * p.K;
+    if (chains == 0) return cudaSuccess;
+    cudaError_t e;
+    const size_t sm_local = sizeof(float) * (5 * NN + 4 * N + 8);
+    const size_t sm_carry = sizeof(double) * 2 * NN;
+    const size_t sm_apply = sizeof(float) * (7 * NN + 4 * N + 8 + kThreads / 32);
+    if ((e = set_smem(k_bwd_local<N>, sm_local)) != cudaSuccess) return e;
+    if ((e = set_smem(k_bwd_carry<N>, sm_carry)) != cudaSuccess) return e;
+    if ((e = set_smem(k_bwd_apply<N>, sm_apply)) != cudaSuccess) return e;
+    profile_mark(0, 0, s);
+    k_bwd_local<N><<<(unsigned)chains, kThreads, sm_local, s>>>(p, src, dS, gloc, Wq, status);
+    profile_mark(0, 1, s);
+    profile_mark(1, 0, s);
+    k_bwd_carry<N><<<(unsigned)BH, kThreads, sm_carry, s>>>(p, gloc, Wq, Gin);
+    profile_mark(1, 1, s);
+    profile_mark(2, 0, s);
+    k_bwd_apply<N><<<(unsigned)chains, kThreads, sm_apply, s>>>(p, src, S0, S_fwd, dS, Gin, dx, dS0, status);
+    profile_mark(2, 1, s);
+    return cudaGetLastError();
 }
 
 template <int N>
@@ -687,6 +1069,20 @@ cudaError_t launch_scan(const KParams& p, const void* src, const float* S0, cons
         case 16: return scan_n<16>(p, src, S0, u, snap_every, S_out, o_out, snaps, ws, W, s, launches);
         case 32: return scan_n<32>(p, src, S0, u, snap_every, S_out, o_out, snaps, ws, W, s, launches);
         case 64: return scan_n<64>(p, src, S0, u, snap_every, S_out, o_out, snaps, ws, W, s, launches);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_backward(const KParams& p, const void* x, const float* S0, const float* S_fwd, const float* dS,
+                            float* dx, float* dS0, void* ws_base, const BwdWorkspace& W, cudaStream_t s)
+{
+    char* ws = reinterpret_cast<char*>(ws_base);
+    switch (p.n) {
+        case 4: return backward_n<4>(p, x, S0, S_fwd, dS, dx, dS0, ws, W, s);
+        case 8: return backward_n<8>(p, x, S0, S_fwd, dS, dx, dS0, ws, W, s);
+        case 16: return backward_n<16>(p, x, S0, S_fwd, dS, dx, dS0, ws, W, s);
+        case 32: return backward_n<32>(p, x, S0, S_fwd, dS, dx, dS0, ws, W, s);
+        case 64: return backward_n<64>(p, x, S0, S_fwd, dS, dx, dS0, ws, W, s);
         default: return cudaErrorInvalidValue;
     }
 }

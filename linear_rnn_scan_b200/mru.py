@@ -30,7 +30,8 @@ MATH = {"auto": 0, "fp32": 1, "tf32": 2, "tf32x3": 3, "bf16x3": 4}
 # Every symbol include/mru.h declares.
 EXPORTS = ["mru_workspace_size", "mru_build_states", "mru_scan", "mru_scan_fused",
            "mru_last_device_status", "mru_status_string", "mru_chosen_chunk", "mru_launch_count",
-           "mru_set_profile_events", "mru_scan_fused_noalloc", "mru_kernel_name", "mru_effective_math"]
+           "mru_set_profile_events", "mru_scan_fused_noalloc", "mru_kernel_name", "mru_effective_math",
+           "mru_backward_workspace_size", "mru_scan_backward"]
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -92,6 +93,10 @@ def load(path: str = LIB_PATH):
             lib.mru_kernel_name.restype = ctypes.c_char_p
             lib.mru_effective_math.argtypes = [P, ctypes.c_int32]
             lib.mru_effective_math.restype = ctypes.c_int32
+            lib.mru_backward_workspace_size.argtypes = [P]
+            lib.mru_backward_workspace_size.restype = sz
+            lib.mru_scan_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            lib.mru_scan_backward.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -162,6 +167,15 @@ def scan_fused_noalloc(p: Problem, x: int, S0: int | None, readout: Readout | No
     device array (for callers that may not allocate device memory)."""
     ro = ctypes.byref(readout) if readout is not None else None
     return load().mru_scan_fused_noalloc(ctypes.byref(p), x, S0, ro, S_out, o_out, status_out, stream)
+
+
+def backward_workspace_size(p: Problem) -> int:
+    return load().mru_backward_workspace_size(ctypes.byref(p))
+
+
+def scan_backward(p: Problem, x: int, S0: int | None, S_fwd: int, dS: int, dx: int, dS0: int | None, ws: int,
+                  ws_bytes: int, stream: int = 0) -> int:
+    return load().mru_scan_backward(ctypes.byref(p), x, S0, S_fwd, dS, dx, dS0, ws, ws_bytes, stream)
 
 
 def last_device_status(ws: int, stream: int = 0) -> int:
@@ -243,6 +257,26 @@ def scan_fused_t(p: Problem, x, *, S0=None, u=None, snapshot_every: int = 0, out
                     ws.data_ptr(), ws.numel(), s)
     _check(rc, "mru_scan_fused")
     return o_out, snapshots
+
+
+def scan_backward_t(p: Problem, x, S_fwd, dS, *, S0=None, dx=None, dS0=None, ws=None, stream=None):
+    """Gradients of sum <dS, S> with respect to the embeddings (dx [B, L, H*n*n]
+    fp32) and, with S0, to S0 (dS0 [B, H, n, n]); S_fwd is the forward's S."""
+    torch = _torch()
+    dev = x.device
+    if ws is None:
+        nbytes = backward_workspace_size(p)
+        if nbytes == 0:
+            raise MruError(ERR_INVALID_ARG, "backward_workspace_size")
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    if dx is None:
+        dx = torch.empty((p.B, p.L, p.H * p.n * p.n), dtype=torch.float32, device=dev)
+    if S0 is not None and dS0 is None:
+        dS0 = torch.empty((p.B, p.H, p.n, p.n), dtype=torch.float32, device=dev)
+    rc = scan_backward(p, _dev_ptr(x, "x"), _dev_ptr(S0, "S0"), _dev_ptr(S_fwd, "S_fwd"), _dev_ptr(dS, "dS"),
+                       _dev_ptr(dx, "dx"), _dev_ptr(dS0, "dS0"), ws.data_ptr(), ws.numel(), _stream(stream))
+    _check(rc, "mru_scan_backward")
+    return dx, dS0, ws
 
 
 def scan_t(p: Problem, X, *, S0=None, out=None, ws=None, stream=None):

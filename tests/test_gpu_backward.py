@@ -1,0 +1,114 @@
+"""GPU backward (mru_scan_backward) against the oracle's fp64 backward on the
+same inputs and upstream gradients: every n, every construction mode, f32
+and bf16 inputs, with S0 and several chunks (ragged last chunk), plus the
+full-size default workload on sampled sequences."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+from linear_rnn_scan_b200 import inputs as gen
+from linear_rnn_scan_b200 import mru
+
+from gpu_helpers import oracle_problem, to_device_x, torch
+
+pytestmark = pytest.mark.gpu
+
+# Relative Frobenius gate per token-head for the fp32 backward (max over every
+# compared (b, t, h)): the forward's fp32 gate.  Measured on B200: below 1e-6
+# near the identity; 1.8e-5 for the determinant-corrected mode without the
+# identity, whose chain rule subtracts <dX, Xr> Xr^-T / n from dX.
+TOL_BWD = 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch().cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    mru.load()
+    yield
+
+
+def _rel(a, b, axis):
+    num = np.sqrt(np.sum((a - b) ** 2, axis=axis))
+    den = np.sqrt(np.sum(b ** 2, axis=axis))
+    return num / np.maximum(den, 1e-300)
+
+
+def _run(w, x, S0, dS, chunk):
+    t = torch()
+    p = mru.problem_from_workload(w, chunk=chunk)
+    xd = to_device_x(x)
+    S0d = t.from_numpy(np.ascontiguousarray(S0, np.float32)).cuda()
+    S = mru.scan_fused_t(p, xd, S0=S0d)
+    dx, dS0, ws = mru.scan_backward_t(p, xd, S, t.from_numpy(np.ascontiguousarray(dS, np.float32)).cuda(), S0=S0d)
+    st = mru.last_device_status(ws.data_ptr(), t.cuda.current_stream().cuda_stream)
+    return dx.cpu().numpy().astype(np.float64), dS0.cpu().numpy().astype(np.float64), st
+
+
+CASES = []
+for n in (4, 8, 16, 32, 64):
+    CASES += [(n, gen.MODE_RESHAPE, 1, "f32"), (n, gen.MODE_DETNORM, 1, "f32"), (n, gen.MODE_LDU, 1, "bf16")]
+CASES += [(16, gen.MODE_RESHAPE, 0, "f32"), (8, gen.MODE_DETNORM, 0, "f32"), (16, gen.MODE_LDU, 1, "f32")]
+
+
+@pytest.mark.parametrize("n,mode,add_identity,dtype", CASES)
+def test_backward_small(n, mode, add_identity, dtype):
+    """fp32 arithmetic (fp64 only for the right-to-left scan of the chunk
+    gradients); the measured errors are in the assertion message."""
+    rng = np.random.default_rng(500 + 10 * n + mode + 3 * add_identity)
+    if mode == gen.MODE_LDU:
+        alpha = 1.0
+    elif add_identity:
+        alpha = 0.3 / np.sqrt(n)
+    else:
+        alpha = 1.0 / np.sqrt(n)
+    L = 37 if add_identity else 13
+    w = gen.Workload(f"b{n}", B=2, H=2, L=L, n=n, x_dtype=dtype, mode=mode, alpha=float(alpha),
+                     add_identity=add_identity, seed=600 + n)
+    x = gen.make_x(w)
+    S0 = gen.make_S0(w, seed=601)
+    dS = rng.standard_normal((w.B, w.L, w.H, n, n)).astype(np.float32)
+    dx, dS0, st = _run(w, x, S0, dS, chunk=8)
+    assert st == mru.OK
+    dx_o, dS0_o = oracle.backward(oracle_problem(w), x, dS.astype(np.float64), S0=S0.astype(np.float64))
+    e_dx = _rel(dx.reshape(w.B, w.L, w.H, n * n), dx_o.reshape(w.B, w.L, w.H, n * n), axis=-1)
+    e_s0 = _rel(dS0.reshape(w.B, w.H, n * n), dS0_o.reshape(w.B, w.H, n * n), axis=-1)
+    assert e_dx.max() <= TOL_BWD and e_s0.max() <= TOL_BWD, (e_dx.max(), np.median(e_dx), e_s0.max())
+
+
+@pytest.mark.parametrize("chunk", [1, 5, 16, 64])
+def test_backward_chunk_sizes_agree(chunk):
+    w = gen.Workload("bc", B=1, H=2, L=50, n=16, x_dtype="f32", mode=gen.MODE_DETNORM, alpha=0.05 / 4, seed=77)
+    x = gen.make_x(w)
+    S0 = gen.make_S0(w, seed=78)
+    dS = np.random.default_rng(79).standard_normal((w.B, w.L, w.H, 16, 16)).astype(np.float32)
+    dx, dS0, st = _run(w, x, S0, dS, chunk=chunk)
+    assert st == mru.OK
+    dx_o, dS0_o = oracle.backward(oracle_problem(w), x, dS.astype(np.float64), S0=S0.astype(np.float64))
+    e = _rel(dx.reshape(w.B, w.L, w.H, 256), dx_o.reshape(w.B, w.L, w.H, 256), axis=-1)
+    assert e.max() <= TOL_BWD, e.max()
+
+
+def test_backward_default_workload_sampled():
+    """The bench's default workload (B8 H8 L4096, n = 16, determinant
+    corrected) end to end; the oracle recomputes two sequences."""
+    t = torch()
+    w = gen.WORKLOADS["n16_detnorm_b8h8l4096"]
+    x = gen.make_x(w)
+    rng = np.random.default_rng(5)
+    dS = rng.standard_normal((w.B, w.L, w.H, 16, 16)).astype(np.float32)
+    p = mru.problem_from_workload(w)
+    xd = to_device_x(x)
+    S = mru.scan_fused_t(p, xd)
+    dx, _, ws = mru.scan_backward_t(p, xd, S, t.from_numpy(dS).cuda())
+    assert mru.last_device_status(ws.data_ptr(), t.cuda.current_stream().cuda_stream) == mru.OK
+    dx = dx.cpu().numpy().astype(np.float64).reshape(w.B, w.L, w.H, 256)
+    for b, h in [(0, 0), (7, 5)]:
+        ws1 = gen.Workload("one", B=1, H=1, L=w.L, n=16, x_dtype="f32", mode=w.mode, alpha=w.alpha, seed=0)
+        x1 = np.ascontiguousarray(x.reshape(w.B, w.L, w.H, 256)[b:b + 1, :, h])
+        dS1 = dS[b:b + 1, :, h:h + 1].astype(np.float64)
+        dx_o, _ = oracle.backward(oracle_problem(ws1), x1, dS1)
+        e = _rel(dx[b, :, h], dx_o.reshape(w.L, 256), axis=-1)
+        assert e.max() <= TOL_BWD, (b, h, e.max(), np.median(e))
