@@ -162,10 +162,23 @@ def read_peaks():
                 "source": "fallback"}
 
 
-def csrc_hash() -> str:
+KERNEL_SOURCES = {"k16_": "mru_n16.cu", "k32_": "mru_n32.cu", "k64_": "mru_n64.cu",
+                  "k_level": "mru_carry.cu", "k_top": "mru_carry.cu", "k_down": "mru_carry.cu"}
+
+
+def kernel_source(kernel: str) -> str:
+    for prefix, f in KERNEL_SOURCES.items():
+        if kernel.startswith(prefix):
+            return f
+    return "mru_scan_v1.cu"
+
+
+def csrc_hash(kernel: str) -> str:
+    """sha256 of the source file that holds the kernel and the shared
+    internal header (a capture stays valid while neither changes)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "linear_rnn_scan_b200", "csrc")
-    for name in sorted(os.listdir(d)):
+    for name in (kernel_source(kernel), "mru_internal.cuh"):
         with open(os.path.join(d, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -181,7 +194,7 @@ def recorded_traffic(workload: str, kernel: str):
             rows = json.load(f)
     except Exception:
         return None
-    cur = csrc_hash()
+    cur = csrc_hash(kernel)
     for r in rows:
         if r.get("workload") == workload and r.get("kernel") == kernel and r.get("csrc_sha256") == cur:
             return float(r["dram_bytes_per_launch"])
