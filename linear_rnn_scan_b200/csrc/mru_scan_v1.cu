@@ -324,6 +324,83 @@ k_chunk_prefix(KParams p, const void* src, const float* u, int64_t snap_every, f
     for (int e = tid; e < NN; e += kThreads) totals[chain * NN + e] = sQ[e];
 }
 
+// fp64 products of the chunk-total scan.  n >= 32: the CTA's 8 warps on the
+// fp64 tensor cores (mma.sync m8n8k4) from shared-memory tiles with rows
+// padded to n + 4 doubles (the fragment reads of a half-warp then hit 16
+// distinct 8-byte banks); warp w computes rows 8 MT (w / 2) ... and columns
+// 8 NT (w % 2) ..., MT x NT tiles of 8 x 8.  n < 32: one output element per
+// thread on the SIMT fp64 pipe.
+template <int N>
+struct CarryMul {
+    static constexpr bool kTensor = N >= 32;
+    static constexpr int SP = kTensor ? N + 4 : N;            // shared-memory row stride
+    static constexpr int PER = (N * N + kThreads - 1) / kThreads;
+    static constexpr int MT = kTensor ? N / 32 : 1, NT = kTensor ? N / 16 : 1;   // tiles per warp (tensor path)
+
+    __device__ static void pos(int r, int& row, int& col)
+    {
+        if constexpr (kTensor) {
+            const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+            const int tile = r >> 1, mt = tile / NT, nt = tile % NT;
+            row = 8 * MT * (w >> 1) + 8 * mt + (lane >> 2);
+            col = 8 * NT * (w & 1) + 8 * nt + 2 * (lane & 3) + (r & 1);
+        } else {
+            const int e = threadIdx.x + r * kThreads;
+            row = e / N;
+            col = e % N;
+        }
+    }
+    __device__ static bool valid(int r) { return kTensor || threadIdx.x + r * kThreads < N * N; }
+
+    // acc[r] = (A B)[pos(r)], A and B N x N fp64 in shared memory (stride SP).
+    __device__ static void mul(const double* A, const double* Bm, double (&acc)[PER])
+    {
+        if constexpr (kTensor) {
+            const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+            const int r0 = 8 * MT * (w >> 1), c0 = 8 * NT * (w & 1);
+            double d[2][MT][NT][2];
+#pragma unroll
+            for (int i = 0; i < 2 * MT * NT * 2; ++i) (&d[0][0][0][0])[i] = 0.0;
+#pragma unroll 4
+            for (int kk = 0; kk < N / 4; ++kk) {
+                double av[MT], bv[NT];
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) av[mt] = A[(r0 + 8 * mt + g) * SP + 4 * kk + t];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) bv[nt] = Bm[(4 * kk + t) * SP + c0 + 8 * nt + g];
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        double (&dd)[2] = d[kk & 1][mt][nt];
+                        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};\n"
+                                     : "+d"(dd[0]), "+d"(dd[1])
+                                     : "d"(av[mt]), "d"(bv[nt]));
+                    }
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) acc[2 * (mt * NT + nt) + h] = d[0][mt][nt][h] + d[1][mt][nt][h];
+        } else {
+#pragma unroll
+            for (int r = 0; r < PER; ++r) {
+                const int e = threadIdx.x + r * kThreads;
+                double a = 0.0;
+                if (e < N * N) {
+                    const int i = e / N, c = e % N;
+                    for (int q = 0; q < N; ++q) a = fma(A[i * SP + q], Bm[q * SP + c], a);
+                }
+                acc[r] = a;
+            }
+        }
+    }
+};
+static_assert(CarryMul<64>::PER == 2 * CarryMul<64>::MT * CarryMul<64>::NT, "tile outputs per thread");
+static_assert(CarryMul<32>::PER == 2 * CarryMul<32>::MT * CarryMul<32>::NT, "tile outputs per thread");
+
 // In-group inclusive prefixes of the chunk totals, fp64, split form:
 // R_j = R_{j-1} + T_j + R_{j-1} T_j.
 template <int N>
@@ -331,35 +408,31 @@ __global__ void __launch_bounds__(kThreads)
 k_carry_local(KParams p, const float* totals, double* local)
 {
     constexpr int NN = N * N;
-    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    using CM = CarryMul<N>;
+    constexpr int SP = CM::SP, PER = CM::PER;
     extern __shared__ double dsm[];
     double* sR = dsm;
-    double* sT = sR + NN;
+    double* sT = sR + N * SP;
     const int tid = threadIdx.x;
     const int64_t bh = blockIdx.x / p.NG, g = blockIdx.x % p.NG;
     const int64_t j0 = g * p.group;
     const int64_t j1 = (j0 + p.group < p.K) ? j0 + p.group : p.K;
-    for (int e = tid; e < NN; e += kThreads) sR[e] = 0.0;
+    for (int e = tid; e < N * SP; e += kThreads) sR[e] = 0.0;
     for (int64_t j = j0; j < j1; ++j) {
         const int64_t base = (bh * p.K + j) * NN;
-        for (int e = tid; e < NN; e += kThreads) sT[e] = (double)totals[base + e];
+        for (int e = tid; e < NN; e += kThreads) sT[(e / N) * SP + e % N] = (double)totals[base + e];
         __syncthreads();
         double acc[PER];
-#pragma unroll
-        for (int r = 0; r < PER; ++r) {
-            const int e = tid + r * kThreads;
-            if (e < NN) {
-                const int i = e / N, c = e % N;
-                double a = 0.0;
-                for (int q = 0; q < N; ++q) a = fma(sR[i * N + q], sT[q * N + c], a);
-                acc[r] = sR[e] + (sT[e] + a);
-            }
-        }
+        CM::mul(sR, sT, acc);
         __syncthreads();
 #pragma unroll
         for (int r = 0; r < PER; ++r) {
-            const int e = tid + r * kThreads;
-            if (e < NN) { sR[e] = acc[r]; local[base + e] = acc[r]; }
+            if (!CM::valid(r)) continue;
+            int row, col;
+            CM::pos(r, row, col);
+            const double v = sR[row * SP + col] + (sT[row * SP + col] + acc[r]);
+            sR[row * SP + col] = v;
+            local[base + row * N + col] = v;
         }
     }
 }
@@ -371,38 +444,32 @@ __global__ void __launch_bounds__(kThreads)
 k_carry_groups(KParams p, const float* S0, const double* local, double* gcarry)
 {
     constexpr int NN = N * N;
-    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    using CM = CarryMul<N>;
+    constexpr int SP = CM::SP, PER = CM::PER;
     extern __shared__ double dsm[];
     double* sG = dsm;
-    double* sT = sG + NN;
+    double* sT = sG + N * SP;
     const int tid = threadIdx.x;
     const int64_t bh = blockIdx.x;
     for (int e = tid; e < NN; e += kThreads)
-        sG[e] = S0 ? (double)S0[bh * NN + e] : ((e / N) == (e % N) ? 1.0 : 0.0);
+        sG[(e / N) * SP + e % N] = S0 ? (double)S0[bh * NN + e] : ((e / N) == (e % N) ? 1.0 : 0.0);
     for (int64_t g = 0; g < p.NG; ++g) {
         const int64_t last = ((g + 1) * p.group < p.K ? (g + 1) * p.group : p.K) - 1;
         __syncthreads();
         for (int e = tid; e < NN; e += kThreads) {
-            gcarry[(bh * p.NG + g) * NN + e] = sG[e];
-            sT[e] = local[(bh * p.K + last) * NN + e];
+            gcarry[(bh * p.NG + g) * NN + e] = sG[(e / N) * SP + e % N];
+            sT[(e / N) * SP + e % N] = local[(bh * p.K + last) * NN + e];
         }
         __syncthreads();
         double acc[PER];
-#pragma unroll
-        for (int r = 0; r < PER; ++r) {
-            const int e = tid + r * kThreads;
-            if (e < NN) {
-                const int i = e / N, c = e % N;
-                double a = 0.0;
-                for (int q = 0; q < N; ++q) a = fma(sG[i * N + q], sT[q * N + c], a);
-                acc[r] = sG[e] + a;
-            }
-        }
+        CM::mul(sG, sT, acc);
         __syncthreads();
 #pragma unroll
         for (int r = 0; r < PER; ++r) {
-            const int e = tid + r * kThreads;
-            if (e < NN) sG[e] = acc[r];
+            if (!CM::valid(r)) continue;
+            int row, col;
+            CM::pos(r, row, col);
+            sG[row * SP + col] += acc[r];
         }
     }
 }
@@ -413,24 +480,28 @@ __global__ void __launch_bounds__(kThreads)
 k_carry_final(KParams p, const double* local, const double* gcarry, float* carry)
 {
     constexpr int NN = N * N;
+    using CM = CarryMul<N>;
+    constexpr int SP = CM::SP, PER = CM::PER;
     extern __shared__ double dsm[];
     double* sG = dsm;
-    double* sT = sG + NN;
+    double* sT = sG + N * SP;
     const int tid = threadIdx.x;
     const int64_t bh = blockIdx.x / p.K, k = blockIdx.x % p.K;
     const int64_t g = k / p.group;
     const bool first = (k == g * p.group);
     for (int e = tid; e < NN; e += kThreads) {
-        sG[e] = gcarry[(bh * p.NG + g) * NN + e];
-        sT[e] = first ? 0.0 : local[(bh * p.K + k - 1) * NN + e];
+        sG[(e / N) * SP + e % N] = gcarry[(bh * p.NG + g) * NN + e];
+        sT[(e / N) * SP + e % N] = first ? 0.0 : local[(bh * p.K + k - 1) * NN + e];
     }
     __syncthreads();
-    for (int e = tid; e < NN; e += kThreads) {
-        const int i = e / N, c = e % N;
-        double a = 0.0;
-        if (!first)
-            for (int q = 0; q < N; ++q) a = fma(sG[i * N + q], sT[q * N + c], a);
-        carry[(bh * p.K + k) * NN + e] = (float)(sG[e] + a);
+    double acc[PER];
+    if (!first) CM::mul(sG, sT, acc);
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+        if (!CM::valid(r)) continue;
+        int row, col;
+        CM::pos(r, row, col);
+        carry[(bh * p.K + k) * NN + row * N + col] = (float)(sG[row * SP + col] + (first ? 0.0 : acc[r]));
     }
 }
 
@@ -951,7 +1022,7 @@ cudaError_t scan_n(const KParams& p, const void* src, const float* S0, const flo
     cudaError_t e;
 
     const size_t sm_chunk = sizeof(float) * (4 * NN + 5 * N + 8);
-    const size_t sm_d = sizeof(double) * 2 * NN;
+    const size_t sm_d = sizeof(double) * 2 * N * CarryMul<N>::SP;
     const size_t sm_fix = sizeof(float) * (2 * NN + 2 * N);
     if ((e = set_smem(k_chunk_prefix<N>, sm_chunk)) != cudaSuccess) return e;
     if ((e = set_smem(k_carry_local<N>, sm_d)) != cudaSuccess) return e;
