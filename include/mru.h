@@ -57,7 +57,7 @@ typedef enum {
     MRU_ERR_WORKSPACE = 3,    /* workspace smaller than mru_workspace_size() */
     MRU_ERR_CUDA = 4,         /* a CUDA launch or copy failed */
     MRU_ERR_SINGULAR = 5,     /* DETNORM met det = 0 or a non-finite determinant */
-    MRU_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up */
+    MRU_ERR_TIMEOUT = 6       /* reserved: a bounded device-side wait gave up (no current kernel waits) */
 } mru_status;
 
 typedef enum { MRU_MODE_RESHAPE = 0, MRU_MODE_DETNORM = 1, MRU_MODE_LDU = 2 } mru_mode;
@@ -144,7 +144,7 @@ mru_status mru_scan_backward(const mru_problem* p, const void* x, const float* S
                              void* stream);
 
 /* Synchronises `stream` and returns the device-detected status of the last
- * call that used this workspace (MRU_OK, MRU_ERR_SINGULAR, MRU_ERR_TIMEOUT). */
+ * call that used this workspace (MRU_OK or MRU_ERR_SINGULAR). */
 mru_status mru_last_device_status(const void* ws, void* stream);
 
 /* Static string for a status code. */

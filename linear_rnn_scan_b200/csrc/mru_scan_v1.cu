@@ -400,6 +400,9 @@ struct CarryMul {
 };
 static_assert(CarryMul<64>::PER == 2 * CarryMul<64>::MT * CarryMul<64>::NT, "tile outputs per thread");
 static_assert(CarryMul<32>::PER == 2 * CarryMul<32>::MT * CarryMul<32>::NT, "tile outputs per thread");
+static_assert(CarryMul<16>::MT * CarryMul<16>::NT == 1 && CarryMul<8>::MT * CarryMul<8>::NT == 1 &&
+                  CarryMul<4>::MT * CarryMul<4>::NT == 1,
+              "the SIMT path keeps one tile");
 
 // In-group inclusive prefixes of the chunk totals, fp64, split form:
 // R_j = R_{j-1} + T_j + R_{j-1} T_j.
