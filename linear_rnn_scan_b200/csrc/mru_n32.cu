@@ -70,6 +70,16 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D = A B (+ 0).
+__device__ __forceinline__ void mma_bf16_first(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};\n"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
 // bf16 pair of (lo_elem, hi_elem), round to nearest.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
@@ -141,23 +151,20 @@ __device__ __forceinline__ void tri_product(const uint32_t (&ah)[2][2][4], const
                                             const uint32_t (&bm)[2][4][2], int d, State& acc)
 {
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.0f;
-#pragma unroll
     for (int kt = 0; kt < 2; ++kt)
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
             // the tile holds k in [16 kt, 16 kt + 15], n in [8 nt, 8 nt + 7]
             if (LOWER && 16 * kt + 15 <= 8 * nt) continue;      // no k > n
             if (!LOWER && 16 * kt >= 8 * nt + 7) continue;      // no k < n
+            // the first tile a column tile meets starts its accumulator at zero
+            const bool first = kt == 0 || (LOWER ? 15 <= 8 * nt : 0 >= 8 * nt + 7);   // tile (0, nt) skipped
             const uint32_t b0 = tri_mask(bm[kt][nt][0], 16 * kt - 8 * nt, d, LOWER);
             const uint32_t b1 = tri_mask(bm[kt][nt][1], 16 * kt + 8 - 8 * nt, d, LOWER);
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
-                mma_bf16(acc[mt][nt], al[mt][kt], b0, b1);
+                if (first) mma_bf16_first(acc[mt][nt], al[mt][kt], b0, b1);
+                else mma_bf16(acc[mt][nt], al[mt][kt], b0, b1);
                 mma_bf16(acc[mt][nt], ah[mt][kt], b0, b1);
             }
         }
