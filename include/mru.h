@@ -25,8 +25,9 @@
  *   X, F     [B, L, H, n, n] float32                                 device
  *   S0       [B, H, n, n]    float32, or NULL for the identity       device
  *   S_out    [B, L, H, n, n] float32; memory position t holds S_{t+1} device
- *   u        [n]             float32, shared by every (b, h)          device
- *   o_out    [B, L, H, n]    float32, o_t = S_t . u                   device
+ *   u        [n, q], or [H, n, q] with u_per_head: the readout's query
+ *            columns U (q = 1: one vector u), float32                device
+ *   o_out    [B, L, H, n, q] float32, o_t = S_t . U (the head's U)    device
  *   snapshots [B, L/every, H, n, n] float32, S_t at 1-based t = k*every device
  *
  * Ownership and execution: the caller owns every buffer (the library never
@@ -86,10 +87,18 @@ typedef struct {
     int32_t chunk;              /* tokens per scan chunk; 0 = library choice, else >= 1 */
 } mru_problem;
 
+/* The readout ("dimension reduction": the state matrix turned back into a
+ * vector, "MRU Update: An independent developer's alternative to Attention
+ * is now running successfully", section "What MRU Actually Does").  The
+ * pages leave its form open; here it is a set of q query columns,
+ * o_t = S_t U (n x q per token and head), one U for all heads or one per
+ * head.  q = 1 is the single readout vector o_t = S_t u. */
 typedef struct {
-    const float* u;             /* [n] readout vector (device) */
+    const float* u;             /* [n, q], or [H, n, q] with u_per_head: query columns U (device) */
     int64_t snapshot_every;     /* 0: no snapshots; else > 0, floor(L/every) snapshots per (b, h) */
     float* snapshots;           /* [B, L/every, H, n, n] (device), ignored when every == 0 */
+    int32_t q;                  /* query columns, 1 <= q <= n; 0 is read as 1 */
+    int32_t u_per_head;         /* 0: one U shared by every head; 1: U[h] for head h */
 } mru_readout;
 
 /* Bytes of device workspace a call on this problem needs (>= 256: the first
@@ -109,8 +118,10 @@ mru_status mru_scan(const mru_problem* p, const float* X, const float* S0, float
 
 /* Lift + scan fused: construction from x happens inside the scan.  With
  * ro == NULL every state is written to S_out (o_out unused, may be NULL).
- * With ro != NULL the states are reduced instead: o_out[b,t,h] = S_t . u, and
- * S_t is stored to ro->snapshots at t = every, 2*every, ... (S_out unused). */
+ * With ro != NULL the states are reduced instead: o_out[b,t,h] = S_t . U
+ * ([n, q] per token and head), and S_t is stored to ro->snapshots at
+ * t = every, 2*every, ... (S_out unused).  q outside [0, n] or u_per_head
+ * outside {0, 1} is MRU_ERR_INVALID_ARG. */
 mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0,
                           const mru_readout* ro, float* S_out, float* o_out,
                           void* ws, size_t ws_bytes, void* stream);

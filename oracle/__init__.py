@@ -66,11 +66,12 @@ def _load():
             lib.mro_lift.restype = ctypes.c_int
             lib.mro_scan.argtypes = [P(Problem), vp, dp, dp, ctypes.c_int]
             lib.mro_scan.restype = ctypes.c_int
-            lib.mro_readout.argtypes = [P(Problem), vp, dp, dp, dp, ctypes.c_int64, dp, ctypes.c_int]
+            ci = ctypes.c_int
+            lib.mro_readout.argtypes = [P(Problem), vp, dp, dp, ci, ci, dp, ctypes.c_int64, dp, ci]
             lib.mro_readout.restype = ctypes.c_int
             lib.mro_compare.argtypes = [P(Problem), vp, dp, i64p, ctypes.c_int64, ctypes.c_int64,
-                                        fp, dp, dp, dp, fp, dp, dp, ctypes.c_int64, fp, dp, dp,
-                                        ctypes.c_int]
+                                        fp, dp, dp, dp, ci, ci, fp, dp, dp, ctypes.c_int64, fp, dp, dp,
+                                        ci]
             lib.mro_compare.restype = ctypes.c_int
             lib.mro_backward.argtypes = [P(Problem), vp, dp, dp, dp, dp, ctypes.c_int]
             lib.mro_backward.restype = ctypes.c_int
@@ -151,21 +152,44 @@ def backward(p: Problem, x: np.ndarray, dS: np.ndarray, S0: np.ndarray | None = 
     return dx, dS0
 
 
+def query_columns(p: Problem, u: np.ndarray):
+    """The readout's query columns as (U fp64 contiguous, q, per_head):
+    u of shape [n] is one vector (q = 1), [n, q] one U for every head,
+    [H, n, q] one U per head."""
+    u = np.asarray(u, np.float64)
+    if u.ndim == 1:
+        u, per_head = u.reshape(p.n, 1), 0
+    elif u.ndim == 2:
+        per_head = 0
+    elif u.ndim == 3:
+        if u.shape[0] != p.H:
+            raise ValueError("per-head query columns must be [H, n, q]")
+        per_head = 1
+    else:
+        raise ValueError("u must be [n], [n, q] or [H, n, q]")
+    if u.shape[-2] != p.n or not 1 <= u.shape[-1] <= p.n:
+        raise ValueError("query columns must be n x q with 1 <= q <= n")
+    return np.ascontiguousarray(u), int(u.shape[-1]), per_head
+
+
 def readout(p: Problem, x: np.ndarray, u: np.ndarray, snapshot_every: int = 0,
             S0: np.ndarray | None = None, nthreads: int = 0):
-    """(o [B, L, H, n], snapshots [B, L//every, H, n, n] or None), fp64."""
+    """(o, snapshots [B, L//every, H, n, n] or None), fp64; o is
+    [B, L, H, n] for a single vector u and [B, L, H, n, q] for query columns
+    U ([n, q] or [H, n, q]): o_t = S_t U."""
     x = _check_x(p, x)
-    u = np.ascontiguousarray(u, np.float64).reshape(p.n)
+    U, q, per_head = query_columns(p, u)
     S0 = None if S0 is None else np.ascontiguousarray(S0, np.float64).reshape(p.B, p.H, p.n, p.n)
-    o = np.empty((p.B, p.L, p.H, p.n), np.float64)
+    o = np.empty((p.B, p.L, p.H, p.n, q), np.float64)
     snaps = None
     if snapshot_every > 0:
         snaps = np.empty((p.B, p.L // snapshot_every, p.H, p.n, p.n), np.float64)
     rc = _load().mro_readout(ctypes.byref(p), x.ctypes.data, _ptr(S0, ctypes.c_double),
-                             _ptr(u, ctypes.c_double), _ptr(o, ctypes.c_double), int(snapshot_every),
-                             _ptr(snaps, ctypes.c_double), nthreads or os.cpu_count() or 1)
+                             _ptr(U, ctypes.c_double), q, per_head, _ptr(o, ctypes.c_double),
+                             int(snapshot_every), _ptr(snaps, ctypes.c_double),
+                             nthreads or os.cpu_count() or 1)
     _raise(rc, "readout")
-    return o, snaps
+    return (o[..., 0] if np.ndim(u) == 1 else o), snaps
 
 
 def compare(p: Problem, x: np.ndarray, *, S0=None, bh=None, t_end=None, S_gpu=None,
@@ -191,12 +215,15 @@ def compare(p: Problem, x: np.ndarray, *, S0=None, bh=None, t_end=None, S_gpu=No
         S_gpu = np.ascontiguousarray(S_gpu, np.float32).reshape(p.B, p.L, p.H, p.n, p.n)
         dS, rS = pair((p.B, p.L, p.H))
         out["S"] = (dS, rS)
+    q = per_head = 0
+    if u is not None:
+        u, q, per_head = query_columns(p, u)
     if o_gpu is not None:
-        o_gpu = np.ascontiguousarray(o_gpu, np.float32).reshape(p.B, p.L, p.H, p.n)
+        if u is None:
+            raise ValueError("o_gpu needs the query columns u")
+        o_gpu = np.ascontiguousarray(o_gpu, np.float32).reshape(p.B, p.L, p.H, p.n, q)
         dO, rO = pair((p.B, p.L, p.H))
         out["o"] = (dO, rO)
-    if u is not None:
-        u = np.ascontiguousarray(u, np.float64).reshape(p.n)
     if snap_gpu is not None:
         ls = p.L // snapshot_every
         snap_gpu = np.ascontiguousarray(snap_gpu, np.float32).reshape(p.B, ls, p.H, p.n, p.n)
@@ -206,7 +233,7 @@ def compare(p: Problem, x: np.ndarray, *, S0=None, bh=None, t_end=None, S_gpu=No
     rc = _load().mro_compare(
         ctypes.byref(p), x.ctypes.data, _ptr(S0, d), _ptr(bh, ctypes.c_int64), len(bh), t_end,
         _ptr(S_gpu, f), _ptr(dS, d), _ptr(rS, d),
-        _ptr(u, d), _ptr(o_gpu, f), _ptr(dO, d), _ptr(rO, d),
+        _ptr(u, d), q, per_head, _ptr(o_gpu, f), _ptr(dO, d), _ptr(rO, d),
         int(snapshot_every), _ptr(snap_gpu, f), _ptr(dP, d), _ptr(rP, d),
         nthreads or os.cpu_count() or 1)
     _raise(rc, "compare")

@@ -175,9 +175,11 @@ typedef struct {
     double* S_all;           /* [B,L,H,n,n] or NULL */
     /* comparison targets (all optional) */
     const float* S_gpu;      /* [B,L,H,n,n] */
-    const double* u;         /* [n] readout vector */
-    const float* o_gpu;      /* [B,L,H,n] */
-    double* o_all;           /* [B,L,H,n] oracle readout, optional */
+    const double* u;         /* readout query columns U: [n,q], or [H,n,q] per head */
+    int q;                   /* columns of U */
+    int u_per_head;
+    const float* o_gpu;      /* [B,L,H,n,q] */
+    double* o_all;           /* [B,L,H,n,q] oracle readout, optional */
     int64_t snap_every;      /* 0: none */
     const float* snap_gpu;   /* [B,L/snap_every,H,n,n] */
     double* snap_all;        /* oracle snapshots, optional */
@@ -230,17 +232,21 @@ static void run_sequence(job_t* J, int64_t bh_idx)
             J->rS[row] = r2;
         }
         if (J->u && (J->o_gpu || J->o_all)) {
+            const int q = J->q;
+            const double* U = J->u + (J->u_per_head ? h * n * q : 0);
+            const int64_t base = row * n * q;
             double d2 = 0.0, r2 = 0.0;
-            for (int i = 0; i < n; ++i) {
-                double o = 0.0;                    /* o_t = S_t . u */
-                for (int j = 0; j < n; ++j) o += S[i * n + j] * J->u[j];
-                if (J->o_all) J->o_all[row * n + i] = o;
-                if (J->o_gpu) {
-                    double df = (double)J->o_gpu[row * n + i] - o;
-                    d2 += df * df;
-                    r2 += o * o;
+            for (int i = 0; i < n; ++i)
+                for (int c = 0; c < q; ++c) {
+                    double o = 0.0;                /* o_t = S_t . U */
+                    for (int j = 0; j < n; ++j) o += S[i * n + j] * U[j * q + c];
+                    if (J->o_all) J->o_all[base + i * q + c] = o;
+                    if (J->o_gpu) {
+                        double df = (double)J->o_gpu[base + i * q + c] - o;
+                        d2 += df * df;
+                        r2 += o * o;
+                    }
                 }
-            }
             if (J->o_gpu) { J->dO[row] = d2; J->rO[row] = r2; }
         }
         if (J->snap_every > 0 && ((t + 1) % J->snap_every) == 0) {
@@ -319,18 +325,20 @@ int mro_scan(const mro_problem* p, const void* x, const double* S0, double* S_al
     return rc;
 }
 
-/* Readout o_t = S_t . u for every (b,t,h) ([B,L,H,n]) and snapshots S_t at
- * 1-based t = every, 2*every, ... ([B, L/every, H, n, n]); either may be NULL. */
+/* Readout o_t = S_t . U for every (b,t,h) ([B,L,H,n,q]; U is [n,q], or
+ * [H,n,q] when u_per_head) and snapshots S_t at 1-based t = every, 2*every,
+ * ... ([B, L/every, H, n, n]); either output may be NULL. */
 int mro_readout(const mro_problem* p, const void* x, const double* S0, const double* u,
-                double* o_all, int64_t snap_every, double* snap_all, int nthreads)
+                int q, int u_per_head, double* o_all, int64_t snap_every, double* snap_all,
+                int nthreads)
 {
-    if (check_problem(p) != MRO_OK || !u) return MRO_ERR_ARG;
+    if (check_problem(p) != MRO_OK || !u || q < 1) return MRO_ERR_ARG;
     const int64_t nbh = p->B * p->H;
     int64_t* bh = malloc(sizeof(int64_t) * (nbh > 0 ? nbh : 1));
     for (int64_t i = 0; i < nbh; ++i) bh[i] = i;
     job_t J;
     memset(&J, 0, sizeof J);
-    J.p = p; J.x = x; J.S0 = S0; J.u = u; J.o_all = o_all;
+    J.p = p; J.x = x; J.S0 = S0; J.u = u; J.q = q; J.u_per_head = u_per_head; J.o_all = o_all;
     J.snap_every = snap_every; J.snap_all = snap_all;
     J.t_end = p->L; J.bh = bh; J.n_bh = nbh;
     int rc = run_job(&J, nthreads);
@@ -346,14 +354,14 @@ int mro_readout(const mro_problem* p, const void* x, const double* S0, const dou
 int mro_compare(const mro_problem* p, const void* x, const double* S0,
                 const int64_t* bh, int64_t n_bh, int64_t t_end,
                 const float* S_gpu, double* dS, double* rS,
-                const double* u, const float* o_gpu, double* dO, double* rO,
+                const double* u, int q, int u_per_head, const float* o_gpu, double* dO, double* rO,
                 int64_t snap_every, const float* snap_gpu, double* dP, double* rP,
                 int nthreads)
 {
     if (check_problem(p) != MRO_OK) return MRO_ERR_ARG;
     if (t_end < 0 || t_end > p->L) return MRO_ERR_ARG;
     if (S_gpu && (!dS || !rS)) return MRO_ERR_ARG;
-    if (o_gpu && (!u || !dO || !rO)) return MRO_ERR_ARG;
+    if (o_gpu && (!u || q < 1 || !dO || !rO)) return MRO_ERR_ARG;
     if (snap_gpu && (snap_every <= 0 || !dP || !rP)) return MRO_ERR_ARG;
     for (int64_t i = 0; i < n_bh; ++i)
         if (bh[i] < 0 || bh[i] >= p->B * p->H) return MRO_ERR_ARG;
@@ -361,7 +369,7 @@ int mro_compare(const mro_problem* p, const void* x, const double* S0,
     memset(&J, 0, sizeof J);
     J.p = p; J.x = x; J.S0 = S0;
     J.S_gpu = S_gpu; J.dS = dS; J.rS = rS;
-    J.u = u; J.o_gpu = o_gpu; J.dO = dO; J.rO = rO;
+    J.u = u; J.q = q; J.u_per_head = u_per_head; J.o_gpu = o_gpu; J.dO = dO; J.rO = rO;
     J.snap_every = snap_gpu ? snap_every : 0; J.snap_gpu = snap_gpu; J.dP = dP; J.rP = rP;
     J.t_end = t_end; J.bh = bh; J.n_bh = n_bh;
     return run_job(&J, nthreads);

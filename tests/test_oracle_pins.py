@@ -447,3 +447,37 @@ def test_compare_reports_errors_where_planted(oracle_mod):
     res = oracle_mod.compare(p, x, S_gpu=g, bh=[3], t_end=6)
     d2 = res["S"][0]
     assert np.isnan(d2[0]).all() and not np.isnan(d2[1, :6, 1]).any() and np.isnan(d2[1, 6:, 1]).all()
+
+
+def test_readout_query_columns(oracle_mod):
+    """Query columns U ([n, q] shared or [H, n, q] per head): o_t = S_t U.
+    Identity columns return S_t itself and unit columns pick columns of S_t
+    (both exact: every product has one non-zero term); general U agrees with
+    numpy's product of the scanned states, head by head."""
+    B, H, L, n, every = 2, 3, 12, 8, 3
+    x = gen.randn_f32((B, L, H * n * n), 21)
+    p = oracle_mod.make_problem(B, H, L, n, mode=1, alpha=0.05, add_identity=1)
+    S = oracle_mod.scan(p, x)
+    o, _ = oracle_mod.readout(p, x, np.eye(n))
+    assert o.shape == (B, L, H, n, n)
+    np.testing.assert_array_equal(o, S)
+    cols = [5, 0, 5]
+    o, _ = oracle_mod.readout(p, x, np.eye(n)[:, cols])
+    np.testing.assert_array_equal(o, S[..., cols])
+    rng = np.random.default_rng(22)
+    U = rng.standard_normal((H, n, 3))
+    o, snaps = oracle_mod.readout(p, x, U, every)
+    for h in range(H):
+        np.testing.assert_allclose(o[:, :, h], S[:, :, h] @ U[h], rtol=1e-12, atol=1e-14)
+    assert np.abs(o[:, :, 0] - S[:, :, 0] @ U[1]).max() > 1e-2       # heads are not interchangeable
+    o1, _ = oracle_mod.readout(p, x, U[0])
+    np.testing.assert_allclose(o1, S @ U[0], rtol=1e-12, atol=1e-14)
+    # the streaming comparison locates a planted error in one query column
+    g = o.astype(np.float32)
+    st = oracle_mod.error_stats(*oracle_mod.compare(p, x, u=U, o_gpu=g)["o"])
+    assert st["count"] == B * L * H and st["max"] < 1e-6
+    g[1, 4, 2, 6, 1] += 1e-2
+    st = oracle_mod.error_stats(*oracle_mod.compare(p, x, u=U, o_gpu=g)["o"])
+    assert st["max"] > 1e-3 and np.unravel_index(st["argmax"], (B, L, H)) == (1, 4, 2)
+    with pytest.raises(ValueError):
+        oracle_mod.readout(p, x, np.zeros((n, n + 1)))
