@@ -31,7 +31,7 @@ _LIB = os.path.join(_HERE, "libmru_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-MODE_RESHAPE, MODE_DETNORM, MODE_LDU = 0, 1, 2
+MODE_RESHAPE, MODE_DETNORM, MODE_LDU, MODE_CAYLEY, MODE_EXPM = 0, 1, 2, 3, 4
 DTYPE_F32, DTYPE_BF16 = 0, 1
 OK, ERR_ARG, ERR_SINGULAR = 0, 1, 5
 

@@ -22,7 +22,11 @@
  *       read here as X = Xr / |det Xr|^(1/n) (sign of det kept);
  *     - LDU factor filling: X = L . D . U with L unit lower, U unit upper,
  *       D diagonal; read here as L = I + a*strict_lower(M),
- *       U = I + a*strict_upper(M), D = diag(exp(d*tanh(M_ii))).
+ *       U = I + a*strict_upper(M), D = diag(exp(d*tanh(M_ii)));
+ *     - orthogonal constructions, the Cayley map and the matrix exponential
+ *       of a skew-symmetric matrix; read here with A = alpha (M - M^T) / 2
+ *       (the skew-symmetric part of alpha M) as X = (I - A)^-1 (I + A) and
+ *       X = exp(A).
  *
  * The oracle is the plain definition written out: every X_t is built in fp64
  * from the widened input, and S_t is the serial left-to-right product with a
@@ -39,8 +43,10 @@ typedef struct {
     int64_t B, H, L;
     int32_t n;
     int32_t x_dtype;      /* 0: float32, 1: bfloat16 (raw 16-bit patterns) */
-    int32_t mode;         /* 0: reshape, 1: determinant-corrected, 2: LDU fill */
-    float alpha;          /* Xr = add_identity*I + alpha*M (modes 0 and 1) */
+    int32_t mode;         /* 0: reshape, 1: determinant-corrected, 2: LDU fill,
+                             3: Cayley map, 4: matrix exponential */
+    float alpha;          /* Xr = add_identity*I + alpha*M (modes 0 and 1);
+                             A = alpha (M - M^T) / 2 (modes 3 and 4) */
     int32_t add_identity;
     float ldu_offdiag;    /* a in L = I + a*strict_lower(M), U = I + a*strict_upper(M) */
     float ldu_diag;       /* d in D = diag(exp(d*tanh(M_ii))) */
@@ -117,6 +123,79 @@ static int log_abs_det(int n, double* A, double* logabs, int* sign)
     return 1;
 }
 
+static void transpose(int n, const double* A, double* T)
+{
+    for (int i = 0; i < n; ++i)
+        for (int j = 0; j < n; ++j) T[j * n + i] = A[i * n + j];
+}
+
+/* A^-1 into Ai by Gauss-Jordan elimination with partial pivoting on [A | I]
+ * (A is destroyed).  Returns 0 when A is singular. */
+static int invert(int n, double* A, double* Ai)
+{
+    set_identity(n, Ai);
+    for (int k = 0; k < n; ++k) {
+        int piv = k;
+        double best = fabs(A[k * n + k]);
+        for (int i = k + 1; i < n; ++i)
+            if (fabs(A[i * n + k]) > best) { best = fabs(A[i * n + k]); piv = i; }
+        if (best == 0.0) return 0;
+        if (piv != k)
+            for (int j = 0; j < n; ++j) {
+                double t = A[k * n + j]; A[k * n + j] = A[piv * n + j]; A[piv * n + j] = t;
+                t = Ai[k * n + j]; Ai[k * n + j] = Ai[piv * n + j]; Ai[piv * n + j] = t;
+            }
+        const double pk = A[k * n + k];
+        for (int j = 0; j < n; ++j) { A[k * n + j] /= pk; Ai[k * n + j] /= pk; }
+        for (int i = 0; i < n; ++i) {
+            if (i == k) continue;
+            const double f = A[i * n + k];
+            if (f == 0.0) continue;
+            for (int j = 0; j < n; ++j) { A[i * n + j] -= f * A[k * n + j]; Ai[i * n + j] -= f * Ai[k * n + j]; }
+        }
+    }
+    return 1;
+}
+
+/* X = exp(A) by scaling and squaring (Moler and Van Loan, "Nineteen dubious
+ * ways to compute the exponential of a matrix", 1978): with B = A / 2^s and
+ * ||B||_1 <= 1/2, exp(B) is its power series summed until the terms vanish
+ * in fp64, and exp(A) = exp(B)^(2^s).  A is overwritten by B; term and tmp
+ * are n x n scratch.  Returns 0 for a non-finite A. */
+static int expm_inplace(int n, double* A, double* X, double* term, double* tmp)
+{
+    const int64_t nn = (int64_t)n * n;
+    double norm = 0.0;
+    for (int j = 0; j < n; ++j) {
+        double c = 0.0;
+        for (int i = 0; i < n; ++i) c += fabs(A[i * n + j]);
+        if (c > norm) norm = c;
+    }
+    if (!isfinite(norm)) return 0;
+    int sq = 0;
+    double scale = 1.0;
+    while (norm * scale > 0.5) { scale *= 0.5; ++sq; }
+    for (int64_t e = 0; e < nn; ++e) A[e] *= scale;
+    set_identity(n, X);
+    set_identity(n, term);
+    for (int k = 1; k <= 60; ++k) {
+        matmul(n, term, A, tmp);                       /* term <- term B / k */
+        double big = 0.0, xbig = 0.0;
+        for (int64_t e = 0; e < nn; ++e) {
+            term[e] = tmp[e] / k;
+            X[e] += term[e];
+            if (fabs(term[e]) > big) big = fabs(term[e]);
+            if (fabs(X[e]) > xbig) xbig = fabs(X[e]);
+        }
+        if (big <= 1e-18 * xbig) break;
+    }
+    for (int r = 0; r < sq; ++r) {
+        matmul(n, X, X, tmp);
+        memcpy(X, tmp, sizeof(double) * (size_t)nn);
+    }
+    return 1;
+}
+
 /* ---- step 1: lift one token-head embedding slice to X_t ----------------
  * The slice of head h is x[b, t, h*n*n : (h+1)*n*n], viewed row-major as
  * n x n: M[i][j] = x[... + i*n + j].  work must hold 3*n*n doubles. */
@@ -161,6 +240,28 @@ int mro_lift(const mro_problem* p, const void* x, int64_t b, int64_t t, int64_t 
             for (int j = 0; j < n; ++j) DU[i * n + j] *= Di;
         }
         matmul(n, Lm, DU, X);
+        return MRO_OK;
+    }
+    if (p->mode == 3 || p->mode == 4) {
+        const double a = (double)p->alpha;
+        double* A = work + nn;                     /* skew-symmetric part of alpha M */
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j) A[i * n + j] = 0.5 * a * (M[i * n + j] - M[j * n + i]);
+        if (p->mode == 3) {
+            /* Cayley map: X = (I - A)^-1 (I + A).  I - A is never singular
+             * for a real skew-symmetric A (its eigenvalues are 1 - i lambda). */
+            double* W = work;                      /* M is no longer needed */
+            double* Wi = work + 2 * nn;
+            for (int64_t e = 0; e < nn; ++e) W[e] = -A[e];
+            for (int i = 0; i < n; ++i) W[i * n + i] += 1.0;
+            if (!invert(n, W, Wi)) return MRO_ERR_SINGULAR;
+            for (int64_t e = 0; e < nn; ++e) W[e] = A[e];
+            for (int i = 0; i < n; ++i) W[i * n + i] += 1.0;
+            matmul(n, Wi, W, X);
+            return MRO_OK;
+        }
+        /* matrix exponential */
+        if (!expm_inplace(n, A, X, work + 2 * nn, work)) return MRO_ERR_ARG;   /* M is no longer needed */
         return MRO_OK;
     }
     return MRO_ERR_ARG;
@@ -304,7 +405,7 @@ static int check_problem(const mro_problem* p)
 {
     if (!p || p->B < 0 || p->H < 0 || p->L < 0 || p->n < 1) return MRO_ERR_ARG;
     if (p->x_dtype != 0 && p->x_dtype != 1) return MRO_ERR_ARG;
-    if (p->mode < 0 || p->mode > 2) return MRO_ERR_ARG;
+    if (p->mode < 0 || p->mode > 4) return MRO_ERR_ARG;
     return MRO_OK;
 }
 
@@ -392,42 +493,8 @@ int mro_compare(const mro_problem* p, const void* x, const double* S0,
  *              dM_ii = dD_i D_i d (1 - tanh^2 M_ii).
  * The inverse is textbook Gauss-Jordan with partial pivoting. */
 
-static void transpose(int n, const double* A, double* T)
-{
-    for (int i = 0; i < n; ++i)
-        for (int j = 0; j < n; ++j) T[j * n + i] = A[i * n + j];
-}
-
-/* A^-1 into Ai by Gauss-Jordan elimination with partial pivoting on [A | I]
- * (A is destroyed).  Returns 0 when A is singular. */
-static int invert(int n, double* A, double* Ai)
-{
-    set_identity(n, Ai);
-    for (int k = 0; k < n; ++k) {
-        int piv = k;
-        double best = fabs(A[k * n + k]);
-        for (int i = k + 1; i < n; ++i)
-            if (fabs(A[i * n + k]) > best) { best = fabs(A[i * n + k]); piv = i; }
-        if (best == 0.0) return 0;
-        if (piv != k)
-            for (int j = 0; j < n; ++j) {
-                double t = A[k * n + j]; A[k * n + j] = A[piv * n + j]; A[piv * n + j] = t;
-                t = Ai[k * n + j]; Ai[k * n + j] = Ai[piv * n + j]; Ai[piv * n + j] = t;
-            }
-        const double pk = A[k * n + k];
-        for (int j = 0; j < n; ++j) { A[k * n + j] /= pk; Ai[k * n + j] /= pk; }
-        for (int i = 0; i < n; ++i) {
-            if (i == k) continue;
-            const double f = A[i * n + k];
-            if (f == 0.0) continue;
-            for (int j = 0; j < n; ++j) { A[i * n + j] -= f * A[k * n + j]; Ai[i * n + j] -= f * Ai[k * n + j]; }
-        }
-    }
-    return 1;
-}
-
 /* dM from dX for one token-head (the construction's chain rule above).
- * work holds 6 n*n doubles. */
+ * work holds 7 n*n doubles. */
 static int lift_vjp(const mro_problem* p, const void* x, int64_t b, int64_t t, int64_t h,
                     const double* dX, double* dM, double* work)
 {
@@ -461,6 +528,54 @@ static int lift_vjp(const mro_problem* p, const void* x, int64_t b, int64_t t, i
                 const double dXr = c * (dX[i * n + j] - inner * Ai[j * n + i] / n);   /* Xr^-T */
                 dM[i * n + j] = a * dXr;
             }
+        return MRO_OK;
+    }
+    if (p->mode == 3 || p->mode == 4) {
+        const double a = (double)p->alpha;
+        double* A = work + nn;
+        double* Ab = work + 2 * nn;                /* dL/dA */
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j) A[i * n + j] = 0.5 * a * (M[i * n + j] - M[j * n + i]);
+        if (p->mode == 3) {
+            /* X = 2 W^-1 - I with W = I - A, so dX = 2 W^-1 dA W^-1 and
+             * dA = 2 W^-T dX W^-T */
+            double* W = work + 3 * nn;
+            double* Wi = work + 4 * nn;
+            double* WiT = work + 5 * nn;
+            double* T = work + 6 * nn;
+            for (int64_t e = 0; e < nn; ++e) W[e] = -A[e];
+            for (int i = 0; i < n; ++i) W[i * n + i] += 1.0;
+            if (!invert(n, W, Wi)) return MRO_ERR_SINGULAR;
+            transpose(n, Wi, WiT);
+            matmul(n, WiT, dX, T);
+            matmul(n, T, WiT, Ab);
+            for (int64_t e = 0; e < nn; ++e) Ab[e] *= 2.0;
+        } else {
+            /* The adjoint of the Frechet derivative of exp at A is the
+             * derivative at A^T: dA = L(A^T, dX), the upper right block of
+             * exp([[A^T, dX], [0, A^T]]) (Van Loan, "Computing integrals
+             * involving the matrix exponential", 1978). */
+            const int m = 2 * n;
+            const int64_t mm = (int64_t)m * m;
+            double* Z = malloc(sizeof(double) * 4 * mm);
+            if (!Z) return MRO_ERR_ARG;
+            double* EZ = Z + mm;
+            for (int64_t e = 0; e < mm; ++e) Z[e] = 0.0;
+            for (int i = 0; i < n; ++i)
+                for (int j = 0; j < n; ++j) {
+                    Z[i * m + j] = A[j * n + i];
+                    Z[(i + n) * m + (j + n)] = A[j * n + i];
+                    Z[i * m + (j + n)] = dX[i * n + j];
+                }
+            const int ok = expm_inplace(m, Z, EZ, Z + 2 * mm, Z + 3 * mm);
+            for (int i = 0; i < n; ++i)
+                for (int j = 0; j < n; ++j) Ab[i * n + j] = EZ[i * m + (j + n)];
+            free(Z);
+            if (!ok) return MRO_ERR_ARG;
+        }
+        /* A = alpha (M - M^T) / 2 */
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j) dM[i * n + j] = 0.5 * a * (Ab[i * n + j] - Ab[j * n + i]);
         return MRO_OK;
     }
     if (p->mode == 2) {
@@ -513,7 +628,7 @@ static int backward_sequence(const mro_problem* p, const void* x, const double* 
     const int64_t b = bh / p->H, h = bh % p->H;
     double* X = malloc(sizeof(double) * (size_t)(L * nn + 1));
     double* S = malloc(sizeof(double) * (size_t)((L + 1) * nn));
-    double* work = malloc(sizeof(double) * (size_t)(11 * nn));    /* 5 n*n here + 6 n*n for lift_vjp */
+    double* work = malloc(sizeof(double) * (size_t)(12 * nn));    /* 5 n*n here + 7 n*n for lift_vjp */
     int rc = MRO_OK;
     if (!X || !S || !work) { rc = MRO_ERR_ARG; goto done; }
     /* forward: S[0] = S0 (or I), S[t+1] = S[t] X_{t+1} */

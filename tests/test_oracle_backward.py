@@ -16,6 +16,9 @@ MODES = [  # (mode, n, add_identity, alpha)
     (oracle.MODE_DETNORM, 3, 1, 0.25),
     (oracle.MODE_DETNORM, 4, 0, 0.5),
     (oracle.MODE_LDU, 4, 1, 1.0),
+    (oracle.MODE_CAYLEY, 4, 1, 0.6),
+    (oracle.MODE_EXPM, 4, 1, 0.6),
+    (oracle.MODE_EXPM, 3, 1, 2.5),      # scaling and squaring in the forward
 ]
 
 

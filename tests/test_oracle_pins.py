@@ -7,7 +7,8 @@ lift each token's embedding to a matrix X_t, multiply S_t = S_{t-1} X_t along
 the sequence (the product is associative, which the parallel scan relies on),
 reduce S_t to a vector.  Construction variants ("Improving Matrix Recurrent
 Units as an Attention Alternative", "Key Points" and "Technical Deep Dive"):
-determinant-correcting scalar and LDU factor filling.
+determinant-correcting scalar and LDU factor filling, and the orthogonal
+constructions (Cayley map, matrix exponential) that the pages report tried.
 
 Every pin is written as a check that takes an oracle (``scan`` and ``lift``
 callables).  The real C oracle must pass every pin; an independent numpy
@@ -72,6 +73,24 @@ class NumpyTwin:
         M = xs[b, t, h].reshape(n, n)
         if self.mistake == "column_major_reshape":
             M = M.T
+        if P["mode"] in (3, 4):
+            a = float(P["alpha"])
+            A = 0.5 * a * (M - M.T)
+            if self.mistake == "skew_sign":
+                A = -A
+            if self.mistake == "skew_no_half":
+                A = 2.0 * A
+            if self.mistake == "skew_from_upper":
+                A = a * (np.triu(M, 1) - np.triu(M, 1).T)
+            I = np.eye(n)
+            if P["mode"] == 3:
+                if self.mistake == "cayley_swapped":
+                    return np.linalg.solve(I + A, I - A)
+                return np.linalg.solve(I - A, I + A)
+            if self.mistake == "expm_first_order":
+                return I + A
+            import scipy.linalg
+            return scipy.linalg.expm(A)
         if P["mode"] in (0, 1):
             X = float(P["alpha"]) * M
             if P["add_identity"] and self.mistake != "drop_identity":
@@ -117,7 +136,8 @@ class NumpyTwin:
 
 MISTAKES = ["left_multiply", "column_major_reshape", "drop_identity", "det_exponent_sign",
             "det_power_not_root", "ldu_swap_triangles", "ldu_diag_no_tanh", "ldu_order_udl",
-            "exclusive_output"]
+            "exclusive_output", "skew_sign", "skew_no_half", "skew_from_upper", "cayley_swapped",
+            "expm_first_order"]
 
 
 # ------------------------------------------------------------------- pins ---
@@ -357,9 +377,62 @@ def pin_initial_state_and_resume(o):
     np.testing.assert_allclose(whole, S, rtol=1e-13, atol=1e-14)
 
 
+def pin_orthogonal_2x2_closed_forms(o):
+    """n = 2: the skew-symmetric part of alpha M is A = [[0, a], [-a, 0]] with
+    a = alpha (M01 - M10) / 2.  Cayley map: X = [[1 - a^2, 2a], [-2a, 1 - a^2]]
+    / (1 + a^2); matrix exponential: the rotation [[cos a, sin a],
+    [-sin a, cos a]] (closed forms; the larger alpha needs the squaring)."""
+    L = 8
+    x = gen.randn_f32((1, L, 4), 31) * np.float32(2.0)
+    for alpha in (0.3, 2.5):
+        al = float(np.float32(alpha))
+        for mode in (3, 4):
+            P = params(1, 1, L, 2, mode=mode, alpha=alpha)
+            for t in range(L):
+                M = x[0, t].astype(np.float64).reshape(2, 2)
+                a = 0.5 * al * (M[0, 1] - M[1, 0])
+                if mode == 3:
+                    ref = np.array([[1 - a * a, 2 * a], [-2 * a, 1 - a * a]]) / (1 + a * a)
+                else:
+                    ref = np.array([[math.cos(a), math.sin(a)], [-math.sin(a), math.cos(a)]])
+                np.testing.assert_allclose(o.lift(P, x, 0, t, 0), ref, rtol=0, atol=1e-13)
+
+
+def pin_orthogonal_modes(o):
+    """Cayley map and matrix exponential: X_t is orthogonal with det +1, it
+    depends only on the skew-symmetric part of M (adding a symmetric matrix
+    to M changes nothing, bit for bit: the inputs are dyadic, so every sum is
+    exact), it agrees with numpy.linalg.solve(I - A, I + A) and
+    scipy.linalg.expm(A), and every S_t stays orthogonal along the sequence."""
+    import scipy.linalg
+    n, L = 8, 30
+    r = _rng(32)
+    M = (np.round(r.standard_normal((L, n, n)) * 256) / 256).astype(np.float32)
+    Y = np.round(r.standard_normal((L, n, n)) * 64) / 64
+    Msym = (M + (Y + np.swapaxes(Y, 1, 2))).astype(np.float32)
+    x1, x2 = M.reshape(1, L, n * n), Msym.reshape(1, L, n * n)
+    for alpha in (0.05, 0.7):
+        al = float(np.float32(alpha))
+        for mode in (3, 4):
+            P = params(1, 1, L, n, mode=mode, alpha=alpha)
+            for t in range(0, L, 7):
+                X = o.lift(P, x1, 0, t, 0)
+                assert np.array_equal(X, o.lift(P, x2, 0, t, 0)), (mode, t)
+                assert np.abs(X.T @ X - np.eye(n)).max() < 1e-13
+                assert abs(np.linalg.det(X) - 1.0) < 1e-12
+                Mt = M[t].astype(np.float64)
+                A = 0.5 * al * (Mt - Mt.T)
+                ref = (np.linalg.solve(np.eye(n) - A, np.eye(n) + A) if mode == 3 else scipy.linalg.expm(A))
+                np.testing.assert_allclose(X, ref, rtol=0, atol=1e-13)
+            S = o.scan(P, x1)[0, :, 0]
+            for t in range(L):
+                assert np.abs(S[t].T @ S[t] - np.eye(n)).max() < 1e-12, (mode, t)
+
+
 PINS = [pin_identity_inputs, pin_diagonal_reshape, pin_diagonal_detnorm, pin_permutations_exact,
         pin_integer_shears_exact, pin_bruteforce_exact, pin_detnorm_unit_det,
-        pin_detnorm_product_det, pin_ldu_factors, pin_initial_state_and_resume]
+        pin_detnorm_product_det, pin_ldu_factors, pin_initial_state_and_resume,
+        pin_orthogonal_2x2_closed_forms, pin_orthogonal_modes]
 
 
 # ------------------------------------------------------------------ tests ---
