@@ -103,7 +103,7 @@ def step_bytes(w: gen.Workload) -> dict:
     xb = 2 if w.x_dtype == "bf16" else 4
     x_bytes = w.token_heads * nn * xb
     if w.readout:
-        out = w.token_heads * w.n * 4
+        out = w.token_heads * w.n * max(w.queries, 1) * 4
         if w.snapshot_every:
             out += w.B * (w.L // w.snapshot_every) * w.H * nn * 4
     else:
@@ -338,8 +338,9 @@ def run_reference(args, w):
 def workload_config(w, chunk):
     sb = step_bytes(w)
     return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "n": w.n, "x_dtype": w.x_dtype,
-            "mode": ["reshape", "detnorm", "ldu"][w.mode], "readout": w.readout,
+            "mode": ["reshape", "detnorm", "ldu", "cayley", "expm"][w.mode], "readout": w.readout,
             "snapshot_every": w.snapshot_every, "chunk": chunk,
+            **({"query_columns": w.queries} if w.queries else {}),
             "l2": ("inputs larger than L2: x %.0f MiB in, %.0f MiB out per step" %
                    (sb["in"] / 2 ** 20, sb["out"] / 2 ** 20)) if sb["total"] > L2_BYTES
             else "inputs smaller than L2: L2 flushed (252 MiB written) between timed steps, outside the events",
@@ -384,10 +385,12 @@ def run_ours(args, w):
     ws = mru.workspace_t(p, dev)
     if w.readout:
         u = torch.from_numpy(gen.make_u(w)).to(dev)
-        o = torch.empty((w.B, w.L, w.H, w.n), dtype=torch.float32, device=dev)
+        o = torch.empty((w.B, w.L, w.H, w.n) + ((w.queries,) if w.queries else ()), dtype=torch.float32,
+                        device=dev)
         snaps = (torch.empty((w.B, w.L // w.snapshot_every, w.H, w.n, w.n), dtype=torch.float32, device=dev)
                  if w.snapshot_every else None)
-        ro = mru.Readout(u.data_ptr(), w.snapshot_every, snaps.data_ptr() if snaps is not None else None)
+        ro = mru.Readout(u.data_ptr(), w.snapshot_every, snaps.data_ptr() if snaps is not None else None,
+                         w.queries, 1 if w.queries else 0)
         out_main = o
         outs_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True)]
         outs_dev = [o]

@@ -17,7 +17,13 @@
  *            sign of det Xr is kept; det Xr = 0 or not finite is an error);
  *   LDU      X = L D U, L = I + ldu_offdiag*strict_lower(M),
  *            U = I + ldu_offdiag*strict_upper(M),
- *            D = diag(exp(ldu_diag*tanh(M_ii))).
+ *            D = diag(exp(ldu_diag*tanh(M_ii)));
+ *   CAYLEY   X = (I - A)^-1 (I + A), and
+ *   EXPM     X = exp(A), with A = alpha (M - M^T) / 2, the skew-symmetric
+ *            part of alpha M (the orthogonal constructions the pages report
+ *            tried, "Key Points"); X is orthogonal with det X = 1.
+ *            add_identity is not used.  These two run on the generic fp32
+ *            kernels for every n.
  * M is the head's slice x[b, t, h*n*n : (h+1)*n*n] viewed row-major as n x n.
  *
  * Layouts (all row-major, contiguous, C order):
@@ -61,7 +67,11 @@ typedef enum {
     MRU_ERR_TIMEOUT = 6       /* reserved: a bounded device-side wait gave up (no current kernel waits) */
 } mru_status;
 
-typedef enum { MRU_MODE_RESHAPE = 0, MRU_MODE_DETNORM = 1, MRU_MODE_LDU = 2 } mru_mode;
+typedef enum {
+    MRU_MODE_RESHAPE = 0, MRU_MODE_DETNORM = 1, MRU_MODE_LDU = 2,
+    MRU_MODE_CAYLEY = 3,  /* X = (I - A)^-1 (I + A), A = alpha (M - M^T) / 2 */
+    MRU_MODE_EXPM = 4     /* X = exp(A),             A = alpha (M - M^T) / 2 */
+} mru_mode;
 typedef enum { MRU_F32 = 0, MRU_BF16 = 1 } mru_dtype;
 typedef enum {
     MRU_MATH_AUTO = 0,    /* library choice per n and dtype (fp32-accurate) */
@@ -137,7 +147,9 @@ mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0,
  *   dL/dX_t = S_{t-1}^T G_t,  dL/dS0 = G_1 X_1^T,
  * then through the construction of X_t from the embedding slice M:
  *   reshape: alpha dX;  determinant-corrected (X = c Xr):
- *   alpha c (dX - <dX, Xr> Xr^-T / n);  LDU: through L, D and U.
+ *   alpha c (dX - <dX, Xr> Xr^-T / n);  LDU: through L, D and U;
+ *   Cayley: dA = 2 W^-T dX W^-T (W = I - A);  exponential: dA = L(A^T, dX),
+ *   the Frechet derivative of exp at A^T;  then dM = alpha (dA - dA^T) / 2.
  *   x      [B, L, H*n*n] the forward's embeddings (f32 or bf16)
  *   S0     [B, H, n, n] fp32 or NULL (identity), as in the forward
  *   S_fwd  [B, L, H, n, n] fp32, the forward's states (mru_scan_fused output)

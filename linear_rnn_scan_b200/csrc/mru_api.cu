@@ -62,7 +62,7 @@ mru_status check_problem(const mru_problem* p)
     if (!p) return MRU_ERR_INVALID_ARG;
     if (p->B < 0 || p->H < 0 || p->L < 0 || p->chunk < 0) return MRU_ERR_INVALID_ARG;
     if (p->x_dtype != MRU_F32 && p->x_dtype != MRU_BF16) return MRU_ERR_INVALID_ARG;
-    if (p->mode < MRU_MODE_RESHAPE || p->mode > MRU_MODE_LDU) return MRU_ERR_INVALID_ARG;
+    if (p->mode < MRU_MODE_RESHAPE || p->mode > MRU_MODE_EXPM) return MRU_ERR_INVALID_ARG;
     if (p->math < MRU_MATH_AUTO || p->math > MRU_MATH_BF16X3) return MRU_ERR_INVALID_ARG;
     if (p->add_identity != 0 && p->add_identity != 1) return MRU_ERR_INVALID_ARG;
     if (!supported_n(p->n)) return MRU_ERR_UNSUPPORTED;
@@ -84,6 +84,7 @@ KParams make_params(const mru_problem& p, int32_t src, bool readout)
     k.NG = k.K > 0 ? ceil_div(k.K, k.group) : 0;
     fastdiv_magic(k.H, k.h_mul, k.h_shr);
     fastdiv_magic(k.K, k.k_mul, k.k_shr);
+    k.rq = 1;
     return k;
 }
 
@@ -264,6 +265,7 @@ mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0, 
     float* snaps = nullptr;
     if (ro) {
         if (!ro->u || !o_out || !aligned16(o_out) || ro->snapshot_every < 0) return MRU_ERR_INVALID_ARG;
+        if (ro->q < 0 || ro->q > p->n || (ro->u_per_head != 0 && ro->u_per_head != 1)) return MRU_ERR_INVALID_ARG;
         every = ro->snapshot_every;
         if (every > 0) {
             snaps = ro->snapshots;
@@ -274,6 +276,10 @@ mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0, 
         if (!S_out || !aligned16(S_out) || (const void*)S_out == x) return MRU_ERR_INVALID_ARG;
     }
     KParams k = make_params(*p, SRC_EMBEDDING, ro != nullptr);
+    if (ro) {
+        k.rq = ro->q == 0 ? 1 : ro->q;
+        k.u_hs = ro->u_per_head ? (int64_t)p->n * k.rq : 0;
+    }
     Workspace W = layout(k, ro != nullptr);
     if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -37,6 +37,10 @@ struct KParams {
     int64_t NG;          // carry groups per sequence, ceil(K / G)
     // q = (umulhi(i, mul) + i) >> shr is i / H (i / K) for 0 <= i < 2^31
     uint32_t h_mul, h_shr, k_mul, k_shr;
+    // readout: query columns of U (o_t = S_t U, [n, rq] per token and head)
+    // and the distance between heads' U in floats (0: one U for all heads)
+    int32_t rq;
+    int64_t u_hs;
 };
 
 // Multiplier and shift of the division by d (>= 1) for 31-bit dividends:

@@ -1,5 +1,5 @@
 // mru_n64.cu -- n = 64 determinant-corrected scan with the readout
-// (o_t = S_t u, snapshots), chunk phase on the tensor cores.
+// (o_t = S_t U, snapshots), chunk phase on the tensor cores.
 //
 // One CTA of 4 warps per chain (b, h, chunk); warp w owns rows 16w..16w+15
 // of the 64 x 64 state Q = P - I, held in mma accumulator registers.  Per
@@ -17,9 +17,10 @@
 //     workload's tf32 arithmetic; the identity split keeps the implicit 1 out
 //     of the tf32 operands); the contraction index is permuted so that the
 //     accumulator tile j is the A fragment of k-tile j,
-//   * v_t = Q_t u (the readout of the local prefix) is written where o_t goes,
-//     and Q_t where a snapshot is due; the chunk total goes to the workspace.
-// The carry scan and the fix-up o_t = C u + C v_t are the generic kernels.
+//   * V_t = Q_t U (the readout of the local prefix, U the head's q query
+//     columns) is written where o_t goes, and Q_t where a snapshot is due;
+//     the chunk total goes to the workspace.
+// The carry scan and the fix-up o_t = C U + C V_t are the generic kernels.
 #include "mru_internal.cuh"
 
 namespace mru {
@@ -35,7 +36,7 @@ struct Smem {
     float x[N * ROWW];               // 17,408 bytes: the token's slice
     float prow[2][N];                // pivot row, double-buffered by step parity
     float pcol[2][N];                // pivot column
-    float u[N];
+    float ut[N * N];                 // the head's query columns U, transposed: ut[c][j] = U[j][c]
     double dsum;                     // pivoted fallback: log|det|
     int flag;
     int piv;
@@ -204,14 +205,12 @@ k64_chunk_readout(KParams p, const float* __restrict__ x, const float* __restric
     const int64_t tok = p.H * NN;
     const float* xb = x + (b * p.L * p.H + h) * NN;
 
-    if (tid < N) sm.u[tid] = u[tid];
-    __syncthreads();
-    float ur[8][2];                                  // u at this lane's columns 8 nt + 2 q, + 1
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-        ur[nt][0] = sm.u[8 * nt + 2 * q];
-        ur[nt][1] = sm.u[8 * nt + 2 * q + 1];
+    const int rq = p.rq;
+    for (int e = tid; e < N * rq; e += THREADS) {
+        const int j = e / rq, c = e - j * rq;
+        sm.ut[c * N + j] = u[h * p.u_hs + e];
     }
+    __syncthreads();
     const int r0 = 16 * warp;                        // this warp's rows
     float Qd[8][4];
 #pragma unroll
@@ -287,19 +286,29 @@ k64_chunk_readout(KParams p, const float* __restrict__ x, const float* __restric
                 Qd[nt][2 * h8] += f0 + acc[nt][2 * h8];
                 Qd[nt][2 * h8 + 1] += f1 + acc[nt][2 * h8 + 1];
             }
-        // ---- readout of the local prefix: v_t = Q_t u ----
+        // ---- readout of the local prefix: V_t = Q_t U (rq columns; the loop
+        // bound is uniform over the CTA, so every lane reaches the shuffles) ----
         const int64_t row_bth = (b * p.L + t) * p.H + h;
-#pragma unroll
-        for (int h8 = 0; h8 < 2; ++h8) {
-            float s = 0.0f;
+        for (int c = 0; c < rq; ++c) {
+            float ur[8][2];                          // U[:, c] at this lane's columns 8 nt + 2 q, + 1
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
-                s = fmaf(Qd[nt][2 * h8], ur[nt][0], s);
-                s = fmaf(Qd[nt][2 * h8 + 1], ur[nt][1], s);
+                const float2 v = *reinterpret_cast<const float2*>(sm.ut + c * N + 8 * nt + 2 * q);
+                ur[nt][0] = v.x;
+                ur[nt][1] = v.y;
             }
-            s += __shfl_xor_sync(0xffffffffu, s, 1);
-            s += __shfl_xor_sync(0xffffffffu, s, 2);
-            if (q == 0) o_out[row_bth * N + r0 + g + 8 * h8] = s;
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+                float s = 0.0f;
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) {
+                    s = fmaf(Qd[nt][2 * h8], ur[nt][0], s);
+                    s = fmaf(Qd[nt][2 * h8 + 1], ur[nt][1], s);
+                }
+                s += __shfl_xor_sync(0xffffffffu, s, 1);
+                s += __shfl_xor_sync(0xffffffffu, s, 2);
+                if (q == 0) o_out[(row_bth * N + r0 + g + 8 * h8) * rq + c] = s;
+            }
         }
         if (snap_every > 0 && ((t + 1) % snap_every) == 0) {
             const int64_t srow = (b * (p.L / snap_every) + (t + 1) / snap_every - 1) * p.H + h;

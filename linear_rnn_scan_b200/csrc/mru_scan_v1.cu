@@ -103,6 +103,140 @@ __device__ void cta_logabsdet_pivoted(float* sW, float* sAux)
     }
 }
 
+// D = (A + A Y) * scale = A (I + Y) * scale for N x N matrices in shared
+// memory (D distinct from A and Y); ends with a barrier.  The product term
+// is accumulated on its own before A is added.
+template <int N>
+__device__ __forceinline__ void cta_mul_plus(const float* A, const float* Y, float* D, float scale)
+{
+    for (int e = threadIdx.x; e < N * N; e += kThreads) {
+        const int i = e / N, j = e % N;
+        float a = 0.0f;
+#pragma unroll 8
+        for (int q = 0; q < N; ++q) a = fmaf(A[i * N + q], Y[q * N + j], a);
+        D[e] = (A[e] + a) * scale;
+    }
+    __syncthreads();
+}
+
+// Scaling and Taylor degree of exp(A) for the N x N matrix A in shared
+// memory: the least s >= 0 with ||A||_1 / 2^s <= 1/2, and the least degree m
+// (1 <= m <= 12) whose next Taylor term ||B||^(m+1) / (m+1)! of B = A / 2^s
+// is below 2^-26 ||B||.  The whole CTA calls it; the results are uniform.
+template <int N>
+__device__ void expm_plan(const float* A, float* sAux, int& m, int& sq)
+{
+    for (int j = threadIdx.x; j < N; j += kThreads) {
+        float c = 0.0f;
+        for (int i = 0; i < N; ++i) c += fabsf(A[i * N + j]);
+        sAux[j] = c;
+    }
+    __syncthreads();
+    int* cfg = reinterpret_cast<int*>(sAux + 4 * N);
+    if (threadIdx.x == 0) {
+        float nrm = 0.0f;
+        for (int j = 0; j < N; ++j) nrm = fmaxf(nrm, sAux[j]);
+        int s2 = 0;
+        while (nrm > 0.5f && s2 < 64) { nrm *= 0.5f; ++s2; }     // nrm = ||B||_1 <= 1/2 (finite input)
+        int d = 1;
+        float term = nrm;                     // ||B||^d / d!
+        while (d < 12 && term * nrm / (float)(d + 1) > 1.4901161e-8f * nrm) {
+            term = term * nrm / (float)(d + 1);
+            ++d;
+        }
+        cfg[0] = d;
+        cfg[1] = s2;
+    }
+    __syncthreads();
+    m = cfg[0];
+    sq = cfg[1];
+    __syncthreads();
+}
+
+// Orthogonal constructions of the skew-symmetric part A = alpha (M - M^T) / 2
+// of the slice M (in sM), written as F = X - I into sF:
+//   Cayley map   X = (I - A)^-1 (I + A), so F = 2 (I - A)^-1 A: Gauss-Jordan
+//                elimination of I - A (kept as I + E, E = -A) applied to 2A.
+//                The symmetric part of I - A is I, so every pivot is at
+//                least 1 and no pivoting is needed;
+//   exponential  X = exp(A) by scaling and squaring: B = A / 2^s with
+//                ||B||_1 <= 1/2, exp(B) - I from its Taylor polynomial of
+//                degree m (Horner, Y_m = B / m, Y_k = B (I + Y_{k+1}) / k,
+//                F = Y_1; m is the least degree whose next term
+//                ||B||^(m+1) / (m+1)! is below 2^-26 ||B||), then s
+//                squarings (I + F)^2 - I = 2F + F F.
+// sW and sAux are scratch, and so is sM in the exponential mode (the slice is
+// not kept); the whole CTA calls it; ends with a barrier.
+template <int N>
+__device__ void cta_orthogonal(const KParams& p, float* sF, float* sM, float* sW, float* sAux)
+{
+    constexpr int NN = N * N;
+    const int tid = threadIdx.x;
+    const float ha = 0.5f * p.alpha;
+    if (p.mode == MRU_MODE_CAYLEY) {
+        for (int e = tid; e < NN; e += kThreads) {
+            const int i = e / N, j = e % N;
+            const float a = ha * (sM[e] - sM[j * N + i]);
+            sW[e] = -a;                       // I - A = I + E
+            sF[e] = 2.0f * a;                 // right-hand side 2A
+        }
+        __syncthreads();
+        for (int k = 0; k < N; ++k) {
+            const float r = 1.0f / (1.0f + sW[k * N + k]);
+            for (int i = tid; i < N; i += kThreads) sAux[i] = sW[i * N + k] * r;
+            __syncthreads();
+            for (int e = tid; e < NN; e += kThreads) {
+                const int i = e / N, j = e % N;
+                if (i == k) continue;             // the pivot row stays as it is
+                const float f = sAux[i];
+                sF[e] = fmaf(-f, sF[k * N + j], sF[e]);
+                if (j > k) sW[e] = fmaf(-f, sW[k * N + j], sW[e]);
+            }
+            __syncthreads();
+        }
+        for (int e = tid; e < NN; e += kThreads) {
+            const int i = e / N;
+            sF[e] = sF[e] / (1.0f + sW[i * N + i]);
+        }
+        __syncthreads();
+        return;
+    }
+    // exponential
+    for (int e = tid; e < NN; e += kThreads) {
+        const int i = e / N, j = e % N;
+        sW[e] = ha * (sM[e] - sM[j * N + i]);
+    }
+    __syncthreads();
+    int m, sq;
+    expm_plan<N>(sW, sAux, m, sq);
+    const float scale = ldexpf(1.0f, -sq);
+    for (int e = tid; e < NN; e += kThreads) sW[e] *= scale;             // B
+    __syncthreads();
+    float* cur = sF;
+    float* nxt = sM;                                                     // M is no longer needed
+    for (int e = tid; e < NN; e += kThreads) cur[e] = sW[e] * (1.0f / (float)m);
+    __syncthreads();
+    for (int k = m - 1; k >= 1; --k) {
+        cta_mul_plus<N>(sW, cur, nxt, 1.0f / (float)k);
+        float* t = cur; cur = nxt; nxt = t;
+    }
+    for (int r = 0; r < sq; ++r) {
+        for (int e = tid; e < NN; e += kThreads) {
+            const int i = e / N, j = e % N;
+            float a = 0.0f;
+#pragma unroll 8
+            for (int q = 0; q < N; ++q) a = fmaf(cur[i * N + q], cur[q * N + j], a);
+            nxt[e] = 2.0f * cur[e] + a;
+        }
+        __syncthreads();
+        float* t = cur; cur = nxt; nxt = t;
+    }
+    if (cur != sF) {
+        for (int e = tid; e < NN; e += kThreads) sF[e] = cur[e];
+        __syncthreads();
+    }
+}
+
 // Lift one token-head slice into F = X - I (shared memory, sF).  The whole
 // CTA calls it; it ends with a barrier.  sM, sW: N*N floats of scratch;
 // sAux: 4N + 8 floats of scratch.
@@ -137,6 +271,11 @@ __device__ void cta_construct(const KParams& p, const void* src, int64_t off, fl
             sF[e] = v;
         }
         __syncthreads();
+        return;
+    }
+
+    if (p.mode == MRU_MODE_CAYLEY || p.mode == MRU_MODE_EXPM) {
+        cta_orthogonal<N>(p, sF, sM, sW, sAux);
         return;
     }
 
@@ -276,9 +415,10 @@ k_chunk_prefix(KParams p, const void* src, const float* u, int64_t snap_every, f
     const int64_t t1 = (t0 + p.chunk < p.L) ? t0 + p.chunk : p.L;
     const bool readout = o_out != nullptr;
 
+    const int rq = p.rq;                    // readout query columns
     for (int e = tid; e < NN; e += kThreads) sQ[e] = 0.0f;
     if (readout)
-        for (int i = tid; i < N; i += kThreads) sU[i] = u[i];
+        for (int e = tid; e < N * rq; e += kThreads) sU[e] = u[h * p.u_hs + e];
     __syncthreads();
 
     for (int64_t t = t0; t < t1; ++t) {
@@ -310,10 +450,11 @@ k_chunk_prefix(KParams p, const void* src, const float* u, int64_t snap_every, f
         }
         __syncthreads();
         if (readout) {
-            for (int i = tid; i < N; i += kThreads) {
+            for (int e = tid; e < N * rq; e += kThreads) {
+                const int i = e / rq, c = e - i * rq;
                 float v = 0.0f;
-                for (int j = 0; j < N; ++j) v = fmaf(sQ[i * N + j], sU[j], v);
-                o_out[row * N + i] = v;                    // Q_t u, fixed up later
+                for (int j = 0; j < N; ++j) v = fmaf(sQ[i * N + j], sU[j * rq + c], v);
+                o_out[row * N * rq + e] = v;               // Q_t U, fixed up later
             }
             if (snap_every > 0 && ((t + 1) % snap_every) == 0) {
                 const int64_t srow = (b * (p.L / snap_every) + (t + 1) / snap_every - 1) * p.H + h;
@@ -508,7 +649,7 @@ k_carry_final(KParams p, const double* local, const double* gcarry, float* carry
     }
 }
 
-// S_t = carry (I + Q_t) = carry + carry Q_t, in place; readout: o_t = carry (u + Q_t u).
+// S_t = carry (I + Q_t) = carry + carry Q_t, in place; readout: o_t = carry (U + Q_t U).
 template <int N>
 __global__ void __launch_bounds__(kThreads)
 k_fixup(KParams p, const float* carry, const float* u, int64_t snap_every, float* S_out,
@@ -557,37 +698,40 @@ k_fixup(KParams p, const float* carry, const float* u, int64_t snap_every, float
         for (int64_t t = t0; t < t1; ++t) fix_matrix(S_out + ((b * p.L + t) * p.H + h) * NN);
         return;
     }
-    // readout: o_t = C u + C v_t for every token of the chunk, N tokens at a
-    // time as one small product with C transposed in shared memory
-    // (thread i reads column entries C[i][j] at consecutive addresses) and
-    // the v_t tile staged in sQ
+    // readout: o_t = C U + C V_t (V_t = Q_t U, n x q) for every token of the
+    // chunk, N / q tokens at a time as one small product with C transposed
+    // in shared memory (thread i reads column entries C[i][j] at consecutive
+    // addresses) and the V_t tile staged in sQ
+    const int rq = p.rq, nq = N * rq;
+    const float* uh = u + h * p.u_hs;
     float* sCt = sQ;                        // first C transposed, then reused
     for (int e = tid; e < NN; e += kThreads) sCt[(e % N) * N + e / N] = sC[e];
     __syncthreads();
-    for (int i = tid; i < N; i += kThreads) {
+    for (int e = tid; e < nq; e += kThreads) {
+        const int i = e / rq, c = e - i * rq;
         float a = 0.0f;
-        for (int j = 0; j < N; ++j) a = fmaf(sCt[j * N + i], u[j], a);
-        sCu[i] = a;
+        for (int j = 0; j < N; ++j) a = fmaf(sCt[j * N + i], uh[j * rq + c], a);
+        sCu[e] = a;
     }
     __syncthreads();
     for (int e = tid; e < NN; e += kThreads) sC[e] = sCt[e];     // sC now holds C transposed
     __syncthreads();
-    constexpr int TT = NN / N;              // tokens per tile (sQ holds TT rows of N)
+    const int TT = N / rq;                  // tokens per tile (sQ holds TT blocks of N x q)
     float* sVt = sQ;
     for (int64_t tb = t0; tb < t1; tb += TT) {
         const int nt = (int)((t1 - tb < TT) ? t1 - tb : TT);
-        for (int e = tid; e < nt * N; e += kThreads) {
-            const int tt = e / N, j = e % N;
-            sVt[e] = o_out[((b * p.L + tb + tt) * p.H + h) * N + j];
+        for (int e = tid; e < nt * nq; e += kThreads) {
+            const int tt = e / nq, r = e - tt * nq;
+            sVt[e] = o_out[((b * p.L + tb + tt) * p.H + h) * nq + r];
         }
         __syncthreads();
-        for (int e = tid; e < nt * N; e += kThreads) {
-            const int tt = e / N, i = e % N;
-            const float* v = sVt + tt * N;
+        for (int e = tid; e < nt * nq; e += kThreads) {
+            const int tt = e / nq, r = e - tt * nq, i = r / rq, c = r - i * rq;
+            const float* v = sVt + tt * nq + c;
             float a = 0.0f;
 #pragma unroll 8
-            for (int j = 0; j < N; ++j) a = fmaf(sC[j * N + i], v[j], a);
-            o_out[((b * p.L + tb + tt) * p.H + h) * N + i] = sCu[i] + a;
+            for (int j = 0; j < N; ++j) a = fmaf(sC[j * N + i], v[j * rq], a);
+            o_out[((b * p.L + tb + tt) * p.H + h) * nq + r] = sCu[r] + a;
         }
         __syncthreads();
     }
@@ -797,6 +941,90 @@ k_bwd_carry(KParams p, const float* __restrict__ gloc, const float* __restrict__
     }
 }
 
+// dA = L(A^T, dX), the adjoint of the Frechet derivative of exp at A (the
+// derivative at A^T), for A = alpha (M - M^T) / 2 of the slice at src + off;
+// with C = A^T = -A: B = C / 2^s, the Taylor part differentiates Horner's
+// recurrence (Y_k = B (I + Y_{k+1}) / k, so
+// dY_k = (E (I + Y_{k+1}) + B dY_{k+1}) / k with E = dX / 2^s, dY_m = E / m),
+// and every squaring X' = X X adds L' = X L + L X = 2L + Y L + L Y (X = I + Y).
+// The same s and m as the forward.  dX comes in sD, dA goes out in sD;
+// sM, sW, sS, sA, sX and sAux are scratch.  The whole CTA calls it.
+template <int N>
+__device__ void expm_vjp(const KParams& p, const void* src, int64_t off, float* sD, float* sM, float* sW,
+                         float* sS, float* sA, float* sX, float* sAux)
+{
+    constexpr int NN = N * N;
+    const int tid = threadIdx.x;
+    for (int e = tid; e < NN; e += kThreads) sM[e] = load_elem(src, off + e, p.x_dtype);
+    __syncthreads();
+    const float ha = 0.5f * p.alpha;
+    for (int e = tid; e < NN; e += kThreads) {
+        const int i = e / N, j = e % N;
+        sA[e] = ha * (sM[j * N + i] - sM[e]);                 // C = A^T
+    }
+    __syncthreads();
+    int m, sq;
+    expm_plan<N>(sA, sAux, m, sq);
+    const float scale = ldexpf(1.0f, -sq);
+    float* B = sA;
+    float* E = sM;
+    float* Y = sW;
+    float* Yn = sS;
+    float* dY = sD;
+    float* dYn = sX;
+    for (int e = tid; e < NN; e += kThreads) {
+        B[e] *= scale;
+        E[e] = sD[e] * scale;
+    }
+    __syncthreads();
+    const float rm = 1.0f / (float)m;
+    for (int e = tid; e < NN; e += kThreads) {
+        Y[e] = B[e] * rm;
+        dY[e] = E[e] * rm;
+    }
+    __syncthreads();
+    for (int k = m - 1; k >= 1; --k) {
+        const float rk = 1.0f / (float)k;
+        for (int e = tid; e < NN; e += kThreads) {
+            const int i = e / N, j = e % N;
+            float a1 = 0.0f, a2 = 0.0f;
+#pragma unroll 4
+            for (int q = 0; q < N; ++q) {
+                const float y = Y[q * N + j];
+                a1 = fmaf(B[i * N + q], y, a1);
+                a2 = fmaf(E[i * N + q], y, a2);
+                a2 = fmaf(B[i * N + q], dY[q * N + j], a2);
+            }
+            Yn[e] = (B[e] + a1) * rk;
+            dYn[e] = (E[e] + a2) * rk;
+        }
+        __syncthreads();
+        float* t = Y; Y = Yn; Yn = t;
+        t = dY; dY = dYn; dYn = t;
+    }
+    for (int r = 0; r < sq; ++r) {
+        for (int e = tid; e < NN; e += kThreads) {
+            const int i = e / N, j = e % N;
+            float a1 = 0.0f, a2 = 0.0f;
+#pragma unroll 4
+            for (int q = 0; q < N; ++q) {
+                a1 = fmaf(Y[i * N + q], Y[q * N + j], a1);
+                a2 = fmaf(Y[i * N + q], dY[q * N + j], a2);
+                a2 = fmaf(dY[i * N + q], Y[q * N + j], a2);
+            }
+            Yn[e] = 2.0f * Y[e] + a1;
+            dYn[e] = 2.0f * dY[e] + a2;
+        }
+        __syncthreads();
+        float* t = Y; Y = Yn; Yn = t;
+        t = dY; dY = dYn; dYn = t;
+    }
+    if (dY != sD) {
+        for (int e = tid; e < NN; e += kThreads) sD[e] = dY[e];
+        __syncthreads();
+    }
+}
+
 template <int N>
 __global__ void __launch_bounds__(kThreads)
 k_bwd_apply(KParams p, const void* src, const float* __restrict__ S0, const float* __restrict__ S_fwd,
@@ -813,7 +1041,8 @@ k_bwd_apply(KParams p, const void* src, const float* __restrict__ S0, const floa
     float* sS = sW + NN;
     float* sD = sS + NN;
     float* sA = sD + NN;
-    float* sAux = sA + NN;
+    float* sX = sA + NN;
+    float* sAux = sX + NN;
     float* sRed = sAux + 4 * N + 8;                 // kThreads / 32 partial sums
     const int tid = threadIdx.x;
     const int64_t chain = blockIdx.x;
@@ -892,6 +1121,37 @@ k_bwd_apply(KParams p, const void* src, const float* __restrict__ S0, const floa
             for (int e = tid; e < NN; e += kThreads) {
                 const int i = e / N, j = e % N;
                 out[e] = (c == 0.0f) ? 0.0f : p.alpha * c * fmaf(-f, sW[j * N + i], sD[e]);
+            }
+        } else if (p.mode == MRU_MODE_CAYLEY) {
+            // X = 2 W^-1 - I with W = I - A, so W^-1 = I + F / 2 and
+            // dA = 2 W^-T dX W^-T = 2 T + T F^T with T = dX + F^T dX / 2
+            for (int e = tid; e < NN; e += kThreads) {
+                const int i = e / N, j = e % N;
+                float a = 0.0f;
+#pragma unroll 8
+                for (int q = 0; q < N; ++q) a = fmaf(sF[q * N + i], sD[q * N + j], a);
+                sA[e] = fmaf(0.5f, a, sD[e]);
+            }
+            __syncthreads();
+            for (int e = tid; e < NN; e += kThreads) {
+                const int i = e / N, j = e % N;
+                float a = 0.0f;
+#pragma unroll 8
+                for (int q = 0; q < N; ++q) a = fmaf(sA[i * N + q], sF[j * N + q], a);
+                sS[e] = 2.0f * sA[e] + a;
+            }
+            __syncthreads();
+            const float ha = 0.5f * p.alpha;       // A = alpha (M - M^T) / 2
+            for (int e = tid; e < NN; e += kThreads) {
+                const int i = e / N, j = e % N;
+                out[e] = ha * (sS[e] - sS[j * N + i]);
+            }
+        } else if (p.mode == MRU_MODE_EXPM) {
+            expm_vjp<N>(p, src, row * NN, sD, sM, sW, sS, sA, sX, sAux);   // dA in sD
+            const float ha = 0.5f * p.alpha;
+            for (int e = tid; e < NN; e += kThreads) {
+                const int i = e / N, j = e % N;
+                out[e] = ha * (sD[e] - sD[j * N + i]);
             }
         } else {
             // LDU: D_i = sAux[i] (and D_i - 1 = sAux[N + i]) from the construction
@@ -978,7 +1238,7 @@ cudaError_t backward_n(const KParams& p, const void* src, const float* S0, const
     cudaError_t e;
     const size_t sm_local = sizeof(float) * (5 * NN + 4 * N + 8);
     const size_t sm_carry = sizeof(double) * 2 * NN;
-    const size_t sm_apply = sizeof(float) * (7 * NN + 4 * N + 8 + kThreads / 32);
+    const size_t sm_apply = sizeof(float) * (8 * NN + 4 * N + 8 + kThreads / 32);
     if ((e = set_smem(k_bwd_local<N>, sm_local)) != cudaSuccess) return e;
     if ((e = set_smem(k_bwd_carry<N>, sm_carry)) != cudaSuccess) return e;
     if ((e = set_smem(k_bwd_apply<N>, sm_apply)) != cudaSuccess) return e;
@@ -1024,9 +1284,9 @@ cudaError_t scan_n(const KParams& p, const void* src, const float* S0, const flo
     if (chains == 0) return cudaSuccess;
     cudaError_t e;
 
-    const size_t sm_chunk = sizeof(float) * (4 * NN + 5 * N + 8);
+    const size_t sm_chunk = sizeof(float) * (4 * NN + 4 * N + 8 + N * p.rq);
     const size_t sm_d = sizeof(double) * 2 * N * CarryMul<N>::SP;
-    const size_t sm_fix = sizeof(float) * (2 * NN + 2 * N);
+    const size_t sm_fix = sizeof(float) * (2 * NN + N * p.rq);
     if ((e = set_smem(k_chunk_prefix<N>, sm_chunk)) != cudaSuccess) return e;
     if ((e = set_smem(k_carry_local<N>, sm_d)) != cudaSuccess) return e;
     if ((e = set_smem(k_carry_groups<N>, sm_d)) != cudaSuccess) return e;

@@ -10,7 +10,9 @@ CPU generator seeded with the workload's seed, laid out [B, L, H*n*n]
 (token-major, heads contiguous inside a token).  bf16 workloads round those
 float32 draws to bf16 (round-to-nearest-even) and hand the raw 16-bit patterns
 around as uint16.  The readout vector u is g/||g||_2 with g ~ N(0, 1)[n] from
-a second generator seeded with seed + 7919.
+a second generator seeded with seed + 7919; a workload with q query columns
+per head draws g ~ N(0, 1)[H, n, q] from that generator instead and scales
+every column to unit length.
 """
 from __future__ import annotations
 
@@ -20,7 +22,7 @@ import math
 import numpy as np
 import torch
 
-MODE_RESHAPE, MODE_DETNORM, MODE_LDU = 0, 1, 2
+MODE_RESHAPE, MODE_DETNORM, MODE_LDU, MODE_CAYLEY, MODE_EXPM = 0, 1, 2, 3, 4
 
 
 @dataclasses.dataclass(frozen=True)
@@ -38,6 +40,7 @@ class Workload:
     ldu_diag: float = 0.1
     readout: bool = False
     snapshot_every: int = 0
+    queries: int = 0      # readout: 0 = one vector u [n]; q >= 1 = query columns U [H, n, q]
     math: str = "auto"    # "auto", "fp32", "tf32", "tf32x3", "bf16x3"
     seed: int = 0
 
@@ -75,6 +78,19 @@ WORKLOADS = {
         "n64_detnorm_readout_b2h4l16384", B=2, H=4, L=16384, n=64, x_dtype="f32",
         mode=MODE_DETNORM, alpha=_alpha(0.03, 64), readout=True, snapshot_every=256,
         math="tf32", seed=1005),
+    # the orthogonal constructions on the default workload's shapes and scale
+    "n16_cayley_b8h8l4096": Workload(
+        "n16_cayley_b8h8l4096", B=8, H=8, L=4096, n=16, x_dtype="f32", mode=MODE_CAYLEY,
+        alpha=_alpha(0.05, 16), seed=1006),
+    "n16_expm_b8h8l4096": Workload(
+        "n16_expm_b8h8l4096", B=8, H=8, L=4096, n=16, x_dtype="f32", mode=MODE_EXPM,
+        alpha=_alpha(0.05, 16), seed=1007),
+    # the readout generalised to several query columns per head (o_t = S_t U,
+    # U [H, 64, 8]) on the same sequences
+    "n64_detnorm_readout_q8_b2h4l16384": Workload(
+        "n64_detnorm_readout_q8_b2h4l16384", B=2, H=4, L=16384, n=64, x_dtype="f32",
+        mode=MODE_DETNORM, alpha=_alpha(0.03, 64), readout=True, snapshot_every=256,
+        queries=8, math="tf32", seed=1005),
 }
 
 # Workload order as listed by the method's measurement plan (small case first).
@@ -105,8 +121,13 @@ def make_x(w: Workload, seed: int | None = None) -> np.ndarray:
 
 
 def make_u(w: Workload, seed: int | None = None) -> np.ndarray:
-    """Readout vector u = g / ||g||_2 (float32 [n])."""
-    g = randn_f32((w.n,), (w.seed if seed is None else seed) + 7919).astype(np.float64)
+    """Readout vector u = g / ||g||_2 (float32 [n]), or with w.queries = q
+    per-head query columns of unit length (float32 [H, n, q])."""
+    s = (w.seed if seed is None else seed) + 7919
+    if w.queries:
+        g = randn_f32((w.H, w.n, w.queries), s).astype(np.float64)
+        return (g / np.linalg.norm(g, axis=1, keepdims=True)).astype(np.float32)
+    g = randn_f32((w.n,), s).astype(np.float64)
     return (g / np.linalg.norm(g)).astype(np.float32)
 
 

@@ -23,7 +23,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libmru.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_SINGULAR, ERR_TIMEOUT = range(7)
-MODE_RESHAPE, MODE_DETNORM, MODE_LDU = 0, 1, 2
+MODE_RESHAPE, MODE_DETNORM, MODE_LDU, MODE_CAYLEY, MODE_EXPM = 0, 1, 2, 3, 4
 F32, BF16 = 0, 1
 MATH = {"auto": 0, "fp32": 1, "tf32": 2, "tf32x3": 3, "bf16x3": 4}
 
@@ -46,7 +46,8 @@ class Problem(ctypes.Structure):
 
 
 class Readout(ctypes.Structure):
-    _fields_ = [("u", ctypes.c_void_p), ("snapshot_every", ctypes.c_int64), ("snapshots", ctypes.c_void_p)]
+    _fields_ = [("u", ctypes.c_void_p), ("snapshot_every", ctypes.c_int64), ("snapshots", ctypes.c_void_p),
+                ("q", ctypes.c_int32), ("u_per_head", ctypes.c_int32)]
 
 
 class MruError(RuntimeError):
@@ -234,7 +235,10 @@ def check_device_status(ws, stream=None):
 def scan_fused_t(p: Problem, x, *, S0=None, u=None, snapshot_every: int = 0, out=None, o_out=None,
                  snapshots=None, ws=None, stream=None):
     """x: CUDA tensor [B, L, H*n*n] (float32, or bfloat16 when x_dtype is bf16).
-    Without u: returns S [B, L, H, n, n].  With u: returns (o, snapshots)."""
+    Without u: returns S [B, L, H, n, n].  With u: returns (o, snapshots),
+    o = S_t U per token and head: u of shape [n] gives o [B, L, H, n];
+    query columns [n, q] (one U for every head) or [H, n, q] (one per head)
+    give o [B, L, H, n, q]."""
     torch = _torch()
     dev = x.device
     if ws is None:
@@ -248,11 +252,22 @@ def scan_fused_t(p: Problem, x, *, S0=None, u=None, snapshot_every: int = 0, out
                         ws.data_ptr(), ws.numel(), s)
         _check(rc, "mru_scan_fused")
         return out
+    if u.dim() == 1:
+        q, per_head, oshape = 1, 0, (B, L, H, n)
+    elif u.dim() in (2, 3):
+        q, per_head, oshape = int(u.shape[-1]), int(u.dim() == 3), (B, L, H, n, int(u.shape[-1]))
+        if u.shape[-2] != n or (per_head and u.shape[0] != H):
+            raise ValueError("query columns must be [n, q] or [H, n, q]")
+    else:
+        raise ValueError("u must be [n], [n, q] or [H, n, q]")
+    if u.dtype != torch.float32 or not u.is_contiguous():
+        raise ValueError("u must be a contiguous float32 tensor")
     if o_out is None:
-        o_out = torch.empty((B, L, H, n), dtype=torch.float32, device=dev)
+        o_out = torch.empty(oshape, dtype=torch.float32, device=dev)
     if snapshot_every > 0 and snapshots is None:
         snapshots = torch.empty((B, L // snapshot_every, H, n, n), dtype=torch.float32, device=dev)
-    ro = Readout(_dev_ptr(u, "u"), int(snapshot_every), _dev_ptr(snapshots, "snapshots") if snapshot_every > 0 else None)
+    ro = Readout(_dev_ptr(u, "u"), int(snapshot_every), _dev_ptr(snapshots, "snapshots") if snapshot_every > 0 else None,
+                 q, per_head)
     rc = scan_fused(p, _dev_ptr(x, "x"), _dev_ptr(S0, "S0"), ro, None, _dev_ptr(o_out, "o_out"),
                     ws.data_ptr(), ws.numel(), s)
     _check(rc, "mru_scan_fused")

@@ -100,6 +100,9 @@ def test_invalid_arguments_rejected_before_any_launch(lib):
     assert mru.scan_fused(p, fake, None, ro, None, 2 * fake, 3 * fake, nb) == mru.ERR_INVALID_ARG  # u null
     ro = mru.Readout(4 * fake, 4, None)
     assert mru.scan_fused(p, fake, None, ro, None, 2 * fake, 3 * fake, nb) == mru.ERR_INVALID_ARG  # snaps null
+    for q, per_head in ((17, 0), (-1, 0), (2, 2)):                 # q outside [0, n], bad per-head flag
+        ro = mru.Readout(4 * fake, 0, None, q, per_head)
+        assert mru.scan_fused(p, fake, None, ro, None, 2 * fake, 3 * fake, nb) == mru.ERR_INVALID_ARG
     assert mru.scan(p, fake, None, fake, 3 * fake, nb) == mru.ERR_INVALID_ARG                  # X aliases S
     assert mru.build_states(p, 0, fake, 3 * fake, nb) == mru.ERR_INVALID_ARG
     assert mru.last_device_status(0) == mru.ERR_INVALID_ARG

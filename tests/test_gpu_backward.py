@@ -51,6 +51,10 @@ CASES = []
 for n in (4, 8, 16, 32, 64):
     CASES += [(n, gen.MODE_RESHAPE, 1, "f32"), (n, gen.MODE_DETNORM, 1, "f32"), (n, gen.MODE_LDU, 1, "bf16")]
 CASES += [(16, gen.MODE_RESHAPE, 0, "f32"), (8, gen.MODE_DETNORM, 0, "f32"), (16, gen.MODE_LDU, 1, "f32")]
+for n in (4, 16, 64):
+    CASES += [(n, gen.MODE_CAYLEY, 1, "f32"), (n, gen.MODE_EXPM, 1, "f32")]
+# orthogonal modes with the larger alpha (the exponential squares twice)
+CASES += [(8, gen.MODE_CAYLEY, 0, "f32"), (8, gen.MODE_EXPM, 0, "bf16"), (32, gen.MODE_EXPM, 0, "f32")]
 
 
 @pytest.mark.parametrize("n,mode,add_identity,dtype", CASES)

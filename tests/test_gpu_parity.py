@@ -3,7 +3,8 @@ the same seeded inputs.  Bit-exact where the arithmetic is exact (integer
 permutation and shear products check indexing, layout, chunking and carries),
 within the relative Frobenius gate elsewhere (1e-4 fp32, 1e-2 tensor-core
 paths), over several chunks and ragged tails, every n, every construction
-mode, both input dtypes, with and without S0, and with the readout."""
+mode, both input dtypes, with and without S0, and with the readout (one
+vector or q query columns)."""
 from __future__ import annotations
 
 import numpy as np
@@ -91,7 +92,7 @@ def test_exact_with_initial_state(n):
 
 # --------------------------------------------------------------- parity ---
 
-MODES = [gen.MODE_RESHAPE, gen.MODE_DETNORM, gen.MODE_LDU]
+MODES = [gen.MODE_RESHAPE, gen.MODE_DETNORM, gen.MODE_LDU, gen.MODE_CAYLEY, gen.MODE_EXPM]
 
 
 @pytest.mark.parametrize("n", NS)
@@ -143,6 +144,23 @@ def test_chunk_sizes_agree(chunk):
 
 
 @pytest.mark.parametrize("n", NS)
+@pytest.mark.parametrize("mode", [gen.MODE_CAYLEY, gen.MODE_EXPM])
+def test_parity_orthogonal_large_alpha(n, mode):
+    """Cayley map and exponential far from the identity (the exponential
+    scales and squares, with Taylor degrees up to the cap): the states stay
+    orthogonal, so the fp32 gate holds over the whole sequence."""
+    for alpha in (1.0, 4.0):
+        w = small(n, mode, B=1, H=2, L=40, alpha=alpha, seed=420 + n)
+        x = gen.make_x(w)
+        S, st = run_fused(w, x, chunk=16)
+        assert st == mru.OK
+        e = compare_S(w, x, S)
+        assert e["max"] <= TOL_FP32, (alpha, e)
+        G = np.einsum("...ki,...kj->...ij", S.astype(np.float64), S.astype(np.float64))
+        assert np.abs(G - np.eye(n)).max() < 1e-4
+
+
+@pytest.mark.parametrize("n", NS)
 def test_readout_and_snapshots(n):
     w = small(n, gen.MODE_DETNORM, B=2, H=2, L=70, seed=600 + n).with_(readout=True, snapshot_every=8)
     x = gen.make_x(w)
@@ -156,6 +174,40 @@ def test_readout_and_snapshots(n):
         assert e["o"]["max"] <= tol and e["snap"]["max"] <= tol, e
     (o, snaps), st = run_fused(w, x, u=u, every=0, chunk=16)
     assert snaps is None and compare_readout(w, x, o, None, u, 0)["o"]["max"] <= tol
+
+
+@pytest.mark.parametrize("n", NS)
+@pytest.mark.parametrize("q,per_head,chunk", [(1, False, 16), (3, True, 16), (0, False, 16), (0, True, 0)])
+def test_readout_query_columns(n, q, per_head, chunk):
+    """o_t = S_t U with q query columns (q = 0 here: q = n), one U for all
+    heads or one per head, over chunk boundaries and a ragged tail."""
+    q = q or n
+    w = small(n, gen.MODE_DETNORM, B=2, H=3, L=53, seed=640 + n + q).with_(readout=True, snapshot_every=8)
+    x = gen.make_x(w)
+    rng = np.random.default_rng(641 + n + q)
+    U = (rng.standard_normal((w.H, n, q) if per_head else (n, q)) / np.sqrt(n)).astype(np.float32)
+    (o, snaps), st = run_fused(w, x, u=U, every=8, chunk=chunk)
+    assert st == mru.OK and o.shape == (w.B, w.L, w.H, n, q)
+    e = compare_readout(w, x, o, snaps, U, 8)
+    tol = tol_for_problem(w, chunk=chunk)
+    assert e["o"]["count"] == w.B * w.L * w.H
+    assert e["o"]["max"] <= tol and e["snap"]["max"] <= tol, e
+
+
+@pytest.mark.parametrize("n", NS)
+def test_readout_unit_columns_exact(n):
+    """Permutation products read out through unit query columns (a different
+    column set per head) are picked columns of S_t, exactly."""
+    B, H, L = 2, 2, 37
+    w = small(n, gen.MODE_RESHAPE, B=B, H=H, L=L, alpha=1.0, add_identity=0).with_(readout=True)
+    x = _perm_inputs(B, H, L, n, seed=650 + n)
+    S_ref = oracle.scan(oracle_problem(w), x)
+    cols = [[n - 1, 0, n // 2], [1, 1, n - 2]]
+    U = np.stack([np.eye(n, dtype=np.float32)[:, c] for c in cols])
+    (o, _), st = run_fused(w, x, u=U, chunk=16)
+    assert st == mru.OK
+    for h in range(H):
+        assert np.array_equal(o[:, :, h].astype(np.float64), S_ref[:, :, h][..., cols[h]])
 
 
 @pytest.mark.parametrize("n", [4, 16, 32])

@@ -17,7 +17,8 @@ pytestmark = pytest.mark.gpu
 
 # sequences compared per workload (None = all)
 SAMPLE = {"n4_reshape_l1024": None, "n16_detnorm_b8h8l4096": None, "n32_ldu_bf16_b4h16l8192": 16,
-          "n16_detnorm_b1h8l262144": None, "n64_detnorm_readout_b2h4l16384": 2}
+          "n16_detnorm_b1h8l262144": None, "n64_detnorm_readout_b2h4l16384": 2,
+          "n64_detnorm_readout_q8_b2h4l16384": 2, "n16_cayley_b8h8l4096": 8, "n16_expm_b8h8l4096": 8}
 
 
 @pytest.mark.parametrize("name", gen.WORKLOAD_ORDER)
