@@ -493,21 +493,30 @@ def run_ours(args, w):
     path["frac_of_hbm_peak"] = path["achieved_gbs"] / peaks["hbm_gbs"]
     kernels_ms = {names[i]: round(per_kernel[i], 5) for i in range(n_k)}
 
-    # e2e: public API with host buffers; H2D of x and D2H of every output inside the region
+    # e2e: the C-ABI call with HOST buffers (mru_scan_fused_host): the upload
+    # of x, the scan and the download of every output, pipelined over pieces
+    # of the batch on three streams, all inside the timed region
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     h2d = x_pin.numel() * x_pin.element_size()
     d2h = sum(t.numel() * t.element_size() for t in outs_host)
+    s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ro_h = ro if w.readout else None
+    snaps_host = outs_host[1].data_ptr() if len(outs_host) > 1 else None
+
+    def call_host():
+        rc = mru.scan_fused_host(p, x_pin.data_ptr(), None, ro_h, outs_host[0].data_ptr(), snaps_host,
+                                 x_dev.data_ptr(), outs_dev[0].data_ptr(), ws.data_ptr(), ws.numel(), 0,
+                                 s_handle, s_h2d.cuda_stream, s_d2h.cuda_stream)
+        if rc != mru.OK:
+            raise mru.MruError(rc, "mru_scan_fused_host")
+
+    call_host()                                   # warm-up of the pipelined path
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        x_dev.copy_(x_pin, non_blocking=True)
-        rc = call(x_dev)
-        if rc != mru.OK:
-            raise mru.MruError(rc, "mru_scan_fused")
-        for hd, dd in zip(outs_host, outs_dev):
-            hd.copy_(dd, non_blocking=True)
+        call_host()
     e1.record(stream)
     e1.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
@@ -524,6 +533,8 @@ def run_ours(args, w):
             "config": cfg, "clocks": clocks.summary(),
             "e2e": {"value": aggregate_rate(world, w.token_heads, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "api": "mru_scan_fused_host (pinned host buffers; upload, scan and download "
+                           "pipelined over pieces of the batch on three streams)",
                     "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
             "roofline": roofline, "path_roofline": path, "kernels_ms": kernels_ms,
@@ -623,6 +634,108 @@ def run_backward(args, w):
     return 0
 
 
+def run_decode(args, w):
+    """One step = one decode token for every (b, h) sequence of the workload:
+    mru_scan_fused with L = 1 started from the previous step's state (S0),
+    the single-launch path.  Reports the device time per step."""
+    import torch
+
+    from linear_rnn_scan_b200 import mru
+
+    if w.readout:
+        print(json.dumps({"impl": "ours", "direction": "decode", "unavailable":
+                          "decode is timed on the full-state output"}), flush=True)
+        return 0
+    local = env_int("LOCAL_RANK", 0)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks("nccl", dev)
+    wd = w.with_(L=1)
+    p = mru.problem_from_workload(wd)
+    total = args.warmup + args.steps
+    xs = gen.make_x(w.with_(L=total), seed=w.seed + ranks.rank)      # one token per step, [B, total, D]
+    if w.x_dtype == "bf16":
+        xt = torch.from_numpy(xs.view(np.int16)).view(torch.bfloat16)
+    else:
+        xt = torch.from_numpy(xs)
+    x_steps = [xt[:, t:t + 1].contiguous().to(dev) for t in range(total)]
+    state = [torch.empty((w.B, 1, w.H, w.n, w.n), dtype=torch.float32, device=dev) for _ in range(2)]
+    state[0].copy_(torch.eye(w.n, device=dev).expand(w.B, 1, w.H, w.n, w.n))
+    ws = mru.workspace_t(p, dev)
+    stream = torch.cuda.current_stream()
+
+    def step(t):
+        src, dst = state[t % 2], state[(t + 1) % 2]
+        rc = mru.scan_fused(p, x_steps[t].data_ptr(), src.data_ptr(), None, dst.data_ptr(), None,
+                            ws.data_ptr(), ws.numel(), stream.cuda_stream)
+        if rc != mru.OK:
+            raise mru.MruError(rc, "mru_scan_fused (decode)")
+
+    for t in range(args.warmup):
+        step(t)
+    torch.cuda.synchronize()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for t in range(args.warmup, total):
+            step(t)
+        ev1.record(stream)
+        ev1.synchronize()
+    torch.cuda.synchronize()
+    ranks.barrier()
+    ms = ranks.max(ev0.elapsed_time(ev1) / args.steps)
+    st = mru.last_device_status(ws.data_ptr(), stream.cuda_stream)
+    if st != mru.OK:
+        raise mru.MruError(st, "device status after decode timing")
+    # the same steps captured once in a CUDA graph and replayed: the device
+    # time per step without the host's per-call cost
+    graph_ms, graph_err = None, None
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                cap = torch.cuda.current_stream().cuda_stream
+                for t in range(args.warmup, total):
+                    src, dst = state[t % 2], state[(t + 1) % 2]
+                    rc = mru.scan_fused(p, x_steps[t].data_ptr(), src.data_ptr(), None, dst.data_ptr(), None,
+                                        ws.data_ptr(), ws.numel(), cap)
+                    if rc != mru.OK:
+                        raise mru.MruError(rc, "mru_scan_fused (graph capture)")
+        stream.wait_stream(side)
+        g.replay()
+        torch.cuda.synchronize()
+        ranks.barrier()
+        ev0.record(stream)
+        g.replay()
+        ev1.record(stream)
+        ev1.synchronize()
+        graph_ms = ranks.max(ev0.elapsed_time(ev1) / args.steps)
+        del g
+    except (RuntimeError, mru.MruError) as exc:       # capture refused: report the eager figure only
+        graph_err = str(exc).splitlines()[0][:200]
+        ranks.max(0.0)
+    if ranks.printer:
+        units = w.B * w.H
+        print(json.dumps({
+            "metric": "MRU decode token·heads/s (one token per (b,h) sequence per step, from S0), 1×B200",
+            "direction": "decode", "value": aggregate_rate(ranks.world, units, ms), "unit": UNIT,
+            "n_gpus": ranks.world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "us_per_step": ms * 1e3,
+            "graph": ({"us_per_step": graph_ms * 1e3, "value": aggregate_rate(ranks.world, units, graph_ms)}
+                      if graph_ms else {"unavailable": graph_err}),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic (seeded N(0,1) embeddings)",
+            "config": dict(workload_config(wd, mru.chosen_chunk(p)), sequences=units),
+            "clocks": clocks.summary(), "gpu_launches": mru.launch_count(p) * args.steps,
+            "kernels": mru.kernel_names(p)}), flush=True)
+    ranks.close()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -634,6 +747,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward", action="store_true", help="time mru_scan_backward instead (not the default)")
+    ap.add_argument("--decode", action="store_true",
+                    help="time single-token decode steps from S0 instead (not the default)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)      # at least 3 untimed warm-up steps, always
     w = gen.WORKLOADS[args.workload]
@@ -641,6 +756,8 @@ def main(argv=None):
         return run_reference(args, w)
     if args.backward:
         return run_backward(args, w)
+    if args.decode:
+        return run_decode(args, w)
     return run_ours(args, w)
 
 

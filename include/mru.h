@@ -136,6 +136,32 @@ mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0,
                           const mru_readout* ro, float* S_out, float* o_out,
                           void* ws, size_t ws_bytes, void* stream);
 
+/* mru_scan_fused from and to HOST buffers, the upload, the scan and the
+ * download pipelined: the problem is cut into `pieces` parts (0: the
+ * library's choice, 8), along the batch when B >= 2, else along the sequence
+ * in whole chunks (each part started from the previous part's last state;
+ * with the readout and B = 1 there is one part).  Part i's upload runs on
+ * h2d_stream while part i - 1 is scanned on compute_stream and part i - 2
+ * downloads on d2h_stream, so that the two copy directions and the kernels
+ * overlap.  Work queued on compute_stream before the call finishes before the
+ * first copy starts, and the call is complete (outputs in host memory) when
+ * compute_stream reaches its end: synchronise that stream before reading.
+ *   x_host     [B, L, H*n*n] host (pinned memory for full speed), as x
+ *   out_host   [B, L, H, n, n] (ro == NULL) or [B, L, H, n, q] (ro) host
+ *   snaps_host [B, L/every, H, n, n] host when ro->snapshot_every > 0,
+ *              downloaded from ro->snapshots (device staging), else unused
+ *   x_dev      device staging of x's size; out_dev device staging of
+ *              out_host's size (16-byte aligned, distinct)
+ *   S0, ro->u  device, as in mru_scan_fused
+ * The three streams may be the same (no overlap then).  Events are created
+ * and released inside the call; no memory is allocated.  Results are
+ * bit-identical to mru_scan_fused when the cut is along the batch; along the
+ * sequence the parts' boundaries round the state to fp32 once more. */
+mru_status mru_scan_fused_host(const mru_problem* p, const void* x_host, const float* S0, const mru_readout* ro,
+                               float* out_host, float* snaps_host, void* x_dev, float* out_dev, void* ws,
+                               size_t ws_bytes, int32_t pieces, void* compute_stream, void* h2d_stream,
+                               void* d2h_stream);
+
 /* Backward (vector-Jacobian product) of mru_scan_fused without the readout.
  * The pages train the MRU but print no gradient: this is the chain rule of
  * the forward definition ("MRU Update: An independent developer's

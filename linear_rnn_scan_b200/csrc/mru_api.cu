@@ -201,6 +201,7 @@ const char* mru_kernel_name(const mru_problem* p, int32_t readout, int32_t i)
     const KParams k = make_params(*p, SRC_EMBEDDING, readout != 0);
     const Workspace W = layout(k, readout != 0);
     if (!W.fast) return kernel_name(k, readout != 0, i);
+    if (k.K == 1) return i == 0 ? (W.fast_n == 16 ? "k16_apply" : "k32_apply") : "";
     if (W.fast_n == 16) return i == 0 ? "k16_reduce" : i == 1 ? "k16_carry" : i == 2 ? "k16_apply" : "";
     const int lv = W.plan.levels;
     const bool n32k = W.fast_n == 32;
@@ -218,6 +219,7 @@ int32_t mru_launch_count(const mru_problem* p, int32_t readout)
     if (p->B * p->H * p->L == 0) return 0;
     const KParams k = make_params(*p, SRC_EMBEDDING, readout != 0);
     const Workspace W = layout(k, readout != 0);
+    if (k.K == 1) return 1;                  // single chunk: one kernel, from S0
     if (W.fast) return W.fast_n == 16 ? 3 : 2 + carry::launches(W.plan);
     return 5;
 }
@@ -287,6 +289,121 @@ mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0, 
     if (p->B * p->H * p->L == 0) return MRU_OK;
     return from_cuda(launch_scan(k, x, S0, ro ? ro->u : nullptr, every, ro ? nullptr : S_out,
                                  ro ? o_out : nullptr, snaps, ws, W, s, nullptr));
+}
+
+mru_status mru_scan_fused_host(const mru_problem* p, const void* x_host, const float* S0, const mru_readout* ro,
+                               float* out_host, float* snaps_host, void* x_dev, float* out_dev, void* ws,
+                               size_t ws_bytes, int32_t pieces, void* compute_stream, void* h2d_stream,
+                               void* d2h_stream)
+{
+    mru_status st = check_problem(p);
+    if (st != MRU_OK) return st;
+    if (!x_host || !out_host || !x_dev || !out_dev || !ws || pieces < 0) return MRU_ERR_INVALID_ARG;
+    if (!aligned16(x_dev) || !aligned16(out_dev) || !aligned16(ws) || (S0 && !aligned16(S0)))
+        return MRU_ERR_INVALID_ARG;
+    if ((const void*)out_dev == x_dev) return MRU_ERR_INVALID_ARG;
+    int64_t every = 0;
+    if (ro) {
+        if (!ro->u || ro->snapshot_every < 0) return MRU_ERR_INVALID_ARG;
+        if (ro->q < 0 || ro->q > p->n || (ro->u_per_head != 0 && ro->u_per_head != 1)) return MRU_ERR_INVALID_ARG;
+        every = ro->snapshot_every;
+        if (every > 0 && (!ro->snapshots || !aligned16(ro->snapshots) || !snaps_host)) return MRU_ERR_INVALID_ARG;
+    }
+    const bool readout = ro != nullptr;
+    KParams k = make_params(*p, SRC_EMBEDDING, readout);
+    if (ro) {
+        k.rq = ro->q == 0 ? 1 : ro->q;
+        k.u_hs = ro->u_per_head ? (int64_t)p->n * k.rq : 0;
+    }
+    const Workspace W = layout(k, readout);
+    if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
+    cudaStream_t sc = reinterpret_cast<cudaStream_t>(compute_stream);
+    cudaStream_t si = reinterpret_cast<cudaStream_t>(h2d_stream);
+    cudaStream_t so = reinterpret_cast<cudaStream_t>(d2h_stream);
+    if ((st = reset_status(ws, sc)) != MRU_OK) return st;
+    if (p->B * p->H * p->L == 0) return MRU_OK;
+
+    // Pieces: along the batch when there are several sequences per head,
+    // else along the sequence (each piece started from the previous piece's
+    // last state), never finer than one chunk; one piece with the readout
+    // of a single batch (its states are not kept).
+    const bool along_b = p->B >= 2;
+    int64_t np = pieces == 0 ? 8 : pieces;
+    if (along_b) np = np < p->B ? np : p->B;
+    else if (readout) np = 1;
+    else np = np < k.K ? np : k.K;
+    if (np > 64) np = 64;
+    if (np < 1) np = 1;
+
+    const int64_t nn = (int64_t)p->n * p->n;
+    const size_t xb = p->x_dtype == MRU_BF16 ? 2 : 4;
+    const int64_t out_tok = readout ? p->H * p->n * k.rq : p->H * nn;   // floats per (b, t)
+    const int64_t ls = every > 0 ? p->L / every : 0;
+    cudaEvent_t ev[2 * 64 + 2];
+    int nev = 0;
+    for (int i = 0; i < 2 * np + 2; ++i) {
+        if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) break;
+        ++nev;
+    }
+    cudaError_t e = nev == 2 * np + 2 ? cudaSuccess : cudaErrorMemoryAllocation;
+    // the copies start after the work already queued on the compute stream
+    if (e == cudaSuccess) e = cudaEventRecord(ev[0], sc);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(si, ev[0], 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(so, ev[0], 0);
+    const char* xh = reinterpret_cast<const char*>(x_host);
+    char* xd = reinterpret_cast<char*>(x_dev);
+    for (int64_t i = 0; i < np && e == cudaSuccess; ++i) {
+        mru_problem sub = *p;
+        sub.chunk = k.chunk;                  // the whole problem's chunk: the workspace fits every piece
+        int64_t xoff, ooff, soff = 0, nx, no, ns = 0;
+        const float* s0 = S0;
+        if (along_b) {
+            const int64_t b0 = p->B * i / np, b1 = p->B * (i + 1) / np;
+            sub.B = b1 - b0;
+            xoff = b0 * p->L * p->H * nn;
+            nx = sub.B * p->L * p->H * nn;
+            ooff = b0 * p->L * out_tok;
+            no = sub.B * p->L * out_tok;
+            soff = b0 * ls * p->H * nn;
+            ns = sub.B * ls * p->H * nn;
+            if (S0) s0 = S0 + b0 * p->H * nn;
+        } else {
+            const int64_t c0 = k.K * i / np, c1 = k.K * (i + 1) / np;    // whole chunks per piece
+            const int64_t t0 = c0 * k.chunk, t1 = c1 * k.chunk < p->L ? c1 * k.chunk : p->L;
+            sub.L = t1 - t0;
+            xoff = t0 * p->H * nn;
+            nx = sub.L * p->H * nn;
+            ooff = t0 * out_tok;
+            no = sub.L * out_tok;
+            if (i > 0) s0 = out_dev + (t0 - 1) * out_tok;               // the previous piece's last state
+        }
+        if ((e = cudaMemcpyAsync(xd + xoff * xb, xh + xoff * xb, (size_t)nx * xb, cudaMemcpyHostToDevice, si)) !=
+            cudaSuccess)
+            break;
+        if ((e = cudaEventRecord(ev[1 + 2 * i], si)) != cudaSuccess) break;
+        if ((e = cudaStreamWaitEvent(sc, ev[1 + 2 * i], 0)) != cudaSuccess) break;
+        KParams ki = make_params(sub, SRC_EMBEDDING, readout);
+        ki.rq = k.rq;
+        ki.u_hs = k.u_hs;
+        const Workspace Wi = layout(ki, readout);
+        e = launch_scan(ki, xd + xoff * xb, s0, ro ? ro->u : nullptr, every, readout ? nullptr : out_dev + ooff,
+                        readout ? out_dev + ooff : nullptr, every > 0 ? ro->snapshots + soff : nullptr, ws, Wi, sc,
+                        nullptr);
+        if (e != cudaSuccess) break;
+        if ((e = cudaEventRecord(ev[2 + 2 * i], sc)) != cudaSuccess) break;
+        if ((e = cudaStreamWaitEvent(so, ev[2 + 2 * i], 0)) != cudaSuccess) break;
+        if ((e = cudaMemcpyAsync(out_host + ooff, out_dev + ooff, (size_t)no * sizeof(float), cudaMemcpyDeviceToHost,
+                                 so)) != cudaSuccess)
+            break;
+        if (ns > 0 && (e = cudaMemcpyAsync(snaps_host + soff, ro->snapshots + soff, (size_t)ns * sizeof(float),
+                                           cudaMemcpyDeviceToHost, so)) != cudaSuccess)
+            break;
+    }
+    // the call is complete once the compute stream passes this point
+    if (e == cudaSuccess) e = cudaEventRecord(ev[2 * np + 1], so);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev[2 * np + 1], 0);
+    for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);     // released once they complete
+    return from_cuda(e);
 }
 
 mru_status mru_last_device_status(const void* ws, void* stream)

@@ -138,8 +138,10 @@ cudaError_t launch_reduce(const KParams& p, const float* x, float* totals, const
                           uint32_t* status, cudaStream_t s);
 cudaError_t launch_carry(const KParams& p, const float* totals, const CarryPlan& cp, char* ws, const float* S0,
                          cudaStream_t s);
+// direct: a single-chunk problem (K = 1), run by the apply pass alone with
+// the carry S0 (or I when S0 is null); no reduce or carry launch precedes it.
 cudaError_t launch_apply(const KParams& p, const float* x, const CarryPlan& cp, const char* ws, float* S_out,
-                         uint32_t* status, cudaStream_t s);
+                         uint32_t* status, const float* S0, bool direct, cudaStream_t s);
 }  // namespace n16
 
 // n = 32 LDU tensor-core kernels (mru_n32.cu).
@@ -148,7 +150,7 @@ bool supports(const KParams& p, bool readout);
 int32_t preferred_chunk(int64_t token_heads);
 cudaError_t launch_reduce(const KParams& p, const void* x, float* totals, cudaStream_t s);
 cudaError_t launch_apply(const KParams& p, const void* x, const carry::Plan& pl, const char* ws, float* S_out,
-                         cudaStream_t s);
+                         const float* S0, bool direct, cudaStream_t s);
 }  // namespace n32
 
 // n = 64 readout chunk kernel on the tensor cores (mru_n64.cu); the carry

@@ -738,6 +738,11 @@ struct Feed {
     const double* E;
     const void* Rf[kCarryLevels];
     bool carry_next;
+    // single-chunk problems (one chain per sequence): the carry is S0 (fp32)
+    // or I, read directly; no carry scan ran
+    bool direct;
+    const float* s0;
+    const float* s0row;
 
     __device__ __forceinline__ void set(const KParams& p, const float* x, const CarryPlan& cp, const char* ws)
     {
@@ -746,7 +751,10 @@ struct Feed {
         xb = x + (c.b * p.L * p.H + c.h) * NN;
         t = c.tbeg;
         tend = c.tend;
-        if (Apply) {
+        if (Apply && direct) {
+            s0row = s0 ? s0 + (c.b * p.H + c.h) * NN : nullptr;
+            carry_next = true;
+        } else if (Apply) {
             const int64_t seq = c.b * p.H + c.h;
             int64_t i = c.k;
 #pragma unroll
@@ -771,7 +779,13 @@ struct Feed {
                                           const CarryPlan& cp, const char* ws)
     {
         if (chain < nchains) {
-            if (Apply && carry_next) {
+            if (Apply && carry_next && direct) {
+                if (s0row) {
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) cp_async16(dst + CF_E + 4 * (lane + 32 * i), s0row + 4 * (lane + 32 * i));
+                }
+                carry_next = false;
+            } else if (Apply && carry_next) {
                 const char* E8 = reinterpret_cast<const char*>(E);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) cp_async16(dst + CF_E + 4 * (lane + 32 * i), E8 + 16 * (lane + 32 * i));
@@ -848,6 +862,21 @@ __device__ __forceinline__ void form_carry(const float* in, const CarryPlan& cp,
         for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
             for (int h = 0; h < 2; ++h) Sd[nb][2 * mt + h] = (float)C.m[mt][nb][h];
+}
+
+// The carry of a single-chunk problem: S0 as staged (fp32, row-major) or I.
+__device__ __forceinline__ void direct_carry(const float* in, bool has_s0, int lane, float (&Sd)[2][4])
+{
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int row = 8 * mt + g, col = 8 * nb + 2 * t + h;
+                Sd[nb][2 * mt + h] = has_s0 ? in[CF_E + row * N + col] : (row == col ? 1.0f : 0.0f);
+            }
 }
 
 // ---- kernels ----------------------------------------------------------------
@@ -927,9 +956,10 @@ k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, u
 // Apply pass: per chain the carry from the carry scan's factors, then
 // S_t = S_{t-1} + S_{t-1} F_t from S = carry, every S_t written, with the
 // per-token determinant scales factorised here.
+template <bool Direct>
 __global__ void __launch_bounds__(AWARPS * 32, 3)
 k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, float* __restrict__ S_out,
-          uint32_t* status)
+          uint32_t* status, const float* __restrict__ S0)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -945,6 +975,8 @@ k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, 
     feed.stride = stride;
     feed.nchains = nchains;
     feed.tok = tok;
+    feed.direct = Direct;
+    feed.s0 = S0;
     feed.set(p, x, cp, ws);
 #pragma unroll
     for (int s = 0; s < ANS - 1; ++s) feed.issue(sm.stage[s], lane, p, x, cp, ws);
@@ -956,7 +988,8 @@ k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, 
         ps = (ps + 1 == ANS) ? 0 : ps + 1;
         cp_async_wait<ANS - 1>();
         __syncwarp();
-        form_carry(sm.stage[cs], cp, c.k, lane, Sd);
+        if (Direct) direct_carry(sm.stage[cs], S0 != nullptr, lane, Sd);
+        else form_carry(sm.stage[cs], cp, c.k, lane, Sd);
         __syncwarp();
         cs = (cs + 1 == ANS) ? 0 : cs + 1;
         float* ob = S_out + (c.b * p.L * p.H + c.h) * NN;
@@ -991,7 +1024,7 @@ k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, 
 
 // CTAs of a persistent launch: resident CTAs per SM times the SM count,
 // cached per device and kernel slot; no more than the chains need.
-std::atomic<int> g_resident[64][3];
+std::atomic<int> g_resident[64][4];
 
 cudaError_t persistent_grid(int slot, const void* kern, int threads, size_t smem, int warps, int64_t nchains,
                             unsigned& grid)
@@ -1102,18 +1135,20 @@ cudaError_t launch_carry(const KParams& p, const float* totals, const CarryPlan&
 }
 
 cudaError_t launch_apply(const KParams& p, const float* x, const CarryPlan& cp, const char* ws, float* S_out,
-                         uint32_t* status, cudaStream_t s)
+                         uint32_t* status, const float* S0, bool direct, cudaStream_t s)
 {
     const int64_t nchains = p.B * p.H * p.K;
     if (nchains == 0) return cudaSuccess;
     if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const size_t sm = sizeof(ASmem) * AWARPS;
-    cudaError_t e = cudaFuncSetAttribute(k16_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    auto kern = direct ? k16_apply<true> : k16_apply<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     unsigned grid = 0;
-    if ((e = persistent_grid(2, (const void*)k16_apply, AWARPS * 32, sm, AWARPS, nchains, grid)) != cudaSuccess)
+    if ((e = persistent_grid(direct ? 3 : 2, (const void*)kern, AWARPS * 32, sm, AWARPS, nchains, grid)) !=
+        cudaSuccess)
         return e;
-    k16_apply<<<grid, AWARPS * 32, sm, s>>>(p, x, cp, ws, S_out, status);
+    kern<<<grid, AWARPS * 32, sm, s>>>(p, x, cp, ws, S_out, status, direct ? S0 : nullptr);
     return cudaGetLastError();
 }
 

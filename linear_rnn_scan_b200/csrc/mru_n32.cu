@@ -417,9 +417,27 @@ __device__ __forceinline__ void form_carry(const double* e1, const float* rp, in
             }
 }
 
+// The carry of a single-chunk problem: S0 (fp32, from L2) or I.
+__device__ __forceinline__ void direct_carry(const float* s0, int lane, State& st)
+{
+    const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int row = 16 * mt + g + 8 * h, col = 8 * nt + 2 * q;
+                float2 v = make_float2(row == col ? 1.0f : 0.0f, row == col + 1 ? 1.0f : 0.0f);
+                if (s0) v = *reinterpret_cast<const float2*>(s0 + row * N + col);
+                st[mt][nt][2 * h] = v.x;
+                st[mt][nt][2 * h + 1] = v.y;
+            }
+}
+
 __global__ void __launch_bounds__(THREADS, 4)
 k32_apply(KParams p, const uint16_t* __restrict__ x, const float* __restrict__ R0, const double* __restrict__ E1,
-          int G, float* __restrict__ S_out)
+          int G, float* __restrict__ S_out, const float* __restrict__ S0, int direct)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -442,7 +460,11 @@ k32_apply(KParams p, const uint16_t* __restrict__ x, const float* __restrict__ R
         const Chain c = chain_at(p, chain);
         const int64_t seq = c.b * p.H + c.h;
         State st;
-        form_carry(E1 + (seq * n1 + c.k / G) * NN, (c.k % G) ? R0 + (seq * p.K + c.k - 1) * NN : nullptr, lane, st);
+        if (direct)
+            direct_carry(S0 ? S0 + seq * NN : nullptr, lane, st);
+        else
+            form_carry(E1 + (seq * n1 + c.k / G) * NN, (c.k % G) ? R0 + (seq * p.K + c.k - 1) * NN : nullptr, lane,
+                       st);
         float* ob = S_out + (c.b * p.L * p.H + c.h) * NN;
         for (int64_t t0 = c.tbeg; t0 < c.tend; t0 += ST) {
             feed.issue(ws.x[ps], lane, p, x);
@@ -516,7 +538,7 @@ cudaError_t launch_reduce(const KParams& p, const void* x, float* totals, cudaSt
 }
 
 cudaError_t launch_apply(const KParams& p, const void* x, const carry::Plan& pl, const char* ws, float* S_out,
-                         cudaStream_t s)
+                         const float* S0, bool direct, cudaStream_t s)
 {
     const int64_t nchains = p.B * p.H * p.K;
     if (nchains == 0) return cudaSuccess;
@@ -528,7 +550,8 @@ cudaError_t launch_apply(const KParams& p, const void* x, const carry::Plan& pl,
     if ((e = persistent_grid(1, (const void*)k32_apply, nchains, grid)) != cudaSuccess) return e;
     k32_apply<<<grid, THREADS, sm, s>>>(p, reinterpret_cast<const uint16_t*>(x),
                                         reinterpret_cast<const float*>(ws + pl.R[0]),
-                                        reinterpret_cast<const double*>(ws + pl.E[1]), pl.G, S_out);
+                                        reinterpret_cast<const double*>(ws + pl.E[1]), pl.G, S_out,
+                                        direct ? S0 : nullptr, direct ? 1 : 0);
     return cudaGetLastError();
 }
 

@@ -335,7 +335,7 @@ k64_chunk_readout(KParams p, const float* __restrict__ x, const float* __restric
 
 bool supports(const KParams& p, bool readout)
 {
-    return p.n == N && p.src == SRC_EMBEDDING && p.x_dtype == MRU_F32 && readout &&
+    return p.n == N && p.src == SRC_EMBEDDING && p.x_dtype == MRU_F32 && readout && p.K > 1 &&
            (p.mode == MRU_MODE_DETNORM || p.mode == MRU_MODE_RESHAPE) &&
            (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32);
 }

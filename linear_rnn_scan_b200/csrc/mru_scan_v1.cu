@@ -395,7 +395,7 @@ k_build_states(KParams p, const void* src, float* X_out, int store_minus_identit
 template <int N>
 __global__ void __launch_bounds__(kThreads)
 k_chunk_prefix(KParams p, const void* src, const float* u, int64_t snap_every, float* S_out,
-               float* o_out, float* snaps, float* totals, uint32_t* status)
+               float* o_out, float* snaps, float* totals, uint32_t* status, const float* S0, int direct)
 {
     constexpr int NN = N * N;
     constexpr int PER = (NN + kThreads - 1) / kThreads;
@@ -416,7 +416,11 @@ k_chunk_prefix(KParams p, const void* src, const float* u, int64_t snap_every, f
     const bool readout = o_out != nullptr;
 
     const int rq = p.rq;                    // readout query columns
-    for (int e = tid; e < NN; e += kThreads) sQ[e] = 0.0f;
+    // direct (one chunk per sequence): the chain starts from S0 (or I), and
+    // every output is final; otherwise from I, fixed up later
+    for (int e = tid; e < NN; e += kThreads)
+        sQ[e] = (direct && S0) ? S0[bh * NN + e] - ((e / N == e % N) ? 1.0f : 0.0f) : 0.0f;
+    const float one = direct ? 1.0f : 0.0f;
     if (readout)
         for (int e = tid; e < N * rq; e += kThreads) sU[e] = u[h * p.u_hs + e];
     __syncthreads();
@@ -445,7 +449,7 @@ k_chunk_prefix(KParams p, const void* src, const float* u, int64_t snap_every, f
             const int e = tid + r * kThreads;
             if (e < NN) {
                 sQ[e] = acc[r];
-                if (!readout) S_out[row * NN + e] = acc[r];
+                if (!readout) S_out[row * NN + e] = acc[r] + ((e / N == e % N) ? one : 0.0f);
             }
         }
         __syncthreads();
@@ -454,15 +458,17 @@ k_chunk_prefix(KParams p, const void* src, const float* u, int64_t snap_every, f
                 const int i = e / rq, c = e - i * rq;
                 float v = 0.0f;
                 for (int j = 0; j < N; ++j) v = fmaf(sQ[i * N + j], sU[j * rq + c], v);
-                o_out[row * N * rq + e] = v;               // Q_t U, fixed up later
+                o_out[row * N * rq + e] = v + one * sU[i * rq + c];   // Q_t U (+ U when final)
             }
             if (snap_every > 0 && ((t + 1) % snap_every) == 0) {
                 const int64_t srow = (b * (p.L / snap_every) + (t + 1) / snap_every - 1) * p.H + h;
-                for (int e = tid; e < NN; e += kThreads) snaps[srow * NN + e] = sQ[e];
+                for (int e = tid; e < NN; e += kThreads)
+                    snaps[srow * NN + e] = sQ[e] + ((e / N == e % N) ? one : 0.0f);
             }
         }
     }
-    for (int e = tid; e < NN; e += kThreads) totals[chain * NN + e] = sQ[e];
+    if (!direct)
+        for (int e = tid; e < NN; e += kThreads) totals[chain * NN + e] = sQ[e];
 }
 
 // fp64 products of the chunk-total scan.  n >= 32: the CTA's 8 warps on the
@@ -1293,13 +1299,22 @@ cudaError_t scan_n(const KParams& p, const void* src, const float* S0, const flo
     if ((e = set_smem(k_carry_final<N>, sm_d)) != cudaSuccess) return e;
     if ((e = set_smem(k_fixup<N>, sm_fix)) != cudaSuccess) return e;
     profile_mark(0, 0, s);
+    if (p.K == 1) {
+        // one chunk per sequence: the chunk kernel starts from S0 and its
+        // outputs are final (the decode / short-segment latency path)
+        k_chunk_prefix<N><<<(unsigned)chains, kThreads, sm_chunk, s>>>(p, src, u, snap_every, S_out, o_out,
+                                                                        snaps, totals, status, S0, 1);
+        profile_mark(0, 1, s);
+        if (launches) *launches = 1;
+        return cudaGetLastError();
+    }
     if (N == 64 && o_out != nullptr && n64::supports(p, true)) {
         if ((e = n64::launch_chunk_readout(p, reinterpret_cast<const float*>(src), u, snap_every, o_out, snaps,
                                            totals, status, s)) != cudaSuccess)
             return e;
     } else {
         k_chunk_prefix<N><<<(unsigned)chains, kThreads, sm_chunk, s>>>(p, src, u, snap_every, S_out, o_out,
-                                                                        snaps, totals, status);
+                                                                        snaps, totals, status, nullptr, 0);
     }
     profile_mark(0, 1, s);
     profile_mark(1, 0, s);
@@ -1326,6 +1341,14 @@ cudaError_t scan_fast16(const KParams& p, const void* src, const float* S0, floa
     const float* x = reinterpret_cast<const float*>(src);
     if (p.B * p.H * p.K == 0) return cudaSuccess;
     cudaError_t e;
+    if (p.K == 1) {
+        // one chunk per sequence: the apply pass alone, from S0
+        profile_mark(0, 0, s);
+        if ((e = n16::launch_apply(p, x, W.c16, ws, S_out, status, S0, true, s)) != cudaSuccess) return e;
+        profile_mark(0, 1, s);
+        if (launches) *launches = 1;
+        return cudaGetLastError();
+    }
     profile_mark(0, 0, s);
     if ((e = n16::launch_reduce(p, x, totals, W.c16, ws, status, s)) != cudaSuccess) return e;
     profile_mark(0, 1, s);
@@ -1333,7 +1356,7 @@ cudaError_t scan_fast16(const KParams& p, const void* src, const float* S0, floa
     if ((e = n16::launch_carry(p, totals, W.c16, ws, S0, s)) != cudaSuccess) return e;
     profile_mark(1, 1, s);
     profile_mark(2, 0, s);
-    if ((e = n16::launch_apply(p, x, W.c16, ws, S_out, status, s)) != cudaSuccess) return e;
+    if ((e = n16::launch_apply(p, x, W.c16, ws, S_out, status, nullptr, false, s)) != cudaSuccess) return e;
     profile_mark(2, 1, s);
     if (launches) *launches = 3;
     return cudaGetLastError();
@@ -1346,12 +1369,19 @@ cudaError_t scan_fast32(const KParams& p, const void* src, const float* S0, floa
     if (p.B * p.H * p.K == 0) return cudaSuccess;
     cudaError_t e;
     int slot = 0;
+    if (p.K == 1) {
+        profile_mark(0, 0, s);
+        if ((e = n32::launch_apply(p, src, W.plan, ws, S_out, S0, true, s)) != cudaSuccess) return e;
+        profile_mark(0, 1, s);
+        if (launches) *launches = 1;
+        return cudaGetLastError();
+    }
     profile_mark(slot, 0, s);
     if ((e = n32::launch_reduce(p, src, totals, s)) != cudaSuccess) return e;
     profile_mark(slot++, 1, s);
     if ((e = carry::run_n32(W.plan, totals, S0, ws, s, slot)) != cudaSuccess) return e;
     profile_mark(slot, 0, s);
-    if ((e = n32::launch_apply(p, src, W.plan, ws, S_out, s)) != cudaSuccess) return e;
+    if ((e = n32::launch_apply(p, src, W.plan, ws, S_out, nullptr, false, s)) != cudaSuccess) return e;
     profile_mark(slot++, 1, s);
     if (launches) *launches = slot;
     return cudaGetLastError();
@@ -1371,7 +1401,7 @@ const char* kernel_name(const KParams& p, bool readout, int i)
 {
     static const char* generic[] = {"k_chunk_prefix", "k_carry_local", "k_carry_groups", "k_carry_final",
                                     "k_fixup"};
-    if (i < 0 || i >= 5) return "";
+    if (i < 0 || i >= (p.K == 1 ? 1 : 5)) return "";
     if (i == 0 && n64::supports(p, readout)) return "k64_chunk_readout";
     return generic[i];
 }

@@ -31,7 +31,7 @@ MATH = {"auto": 0, "fp32": 1, "tf32": 2, "tf32x3": 3, "bf16x3": 4}
 EXPORTS = ["mru_workspace_size", "mru_build_states", "mru_scan", "mru_scan_fused",
            "mru_last_device_status", "mru_status_string", "mru_chosen_chunk", "mru_launch_count",
            "mru_set_profile_events", "mru_scan_fused_noalloc", "mru_kernel_name", "mru_effective_math",
-           "mru_backward_workspace_size", "mru_scan_backward"]
+           "mru_backward_workspace_size", "mru_scan_backward", "mru_scan_fused_host"]
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -98,6 +98,9 @@ def load(path: str = LIB_PATH):
             lib.mru_backward_workspace_size.restype = sz
             lib.mru_scan_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
             lib.mru_scan_backward.restype = ctypes.c_int
+            lib.mru_scan_fused_host.argtypes = [P, vp, vp, ctypes.POINTER(Readout), vp, vp, vp, vp, vp, sz,
+                                                ctypes.c_int32, vp, vp, vp]
+            lib.mru_scan_fused_host.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -168,6 +171,16 @@ def scan_fused_noalloc(p: Problem, x: int, S0: int | None, readout: Readout | No
     device array (for callers that may not allocate device memory)."""
     ro = ctypes.byref(readout) if readout is not None else None
     return load().mru_scan_fused_noalloc(ctypes.byref(p), x, S0, ro, S_out, o_out, status_out, stream)
+
+
+def scan_fused_host(p: Problem, x_host: int, S0: int | None, readout: Readout | None, out_host: int,
+                    snaps_host: int | None, x_dev: int, out_dev: int, ws: int, ws_bytes: int, pieces: int = 0,
+                    compute_stream: int = 0, h2d_stream: int = 0, d2h_stream: int = 0) -> int:
+    """mru_scan_fused from and to host buffers, upload / scan / download
+    pipelined over `pieces` parts on the three streams."""
+    ro = ctypes.byref(readout) if readout is not None else None
+    return load().mru_scan_fused_host(ctypes.byref(p), x_host, S0, ro, out_host, snaps_host, x_dev, out_dev, ws,
+                                      ws_bytes, int(pieces), compute_stream, h2d_stream, d2h_stream)
 
 
 def backward_workspace_size(p: Problem) -> int:
@@ -272,6 +285,35 @@ def scan_fused_t(p: Problem, x, *, S0=None, u=None, snapshot_every: int = 0, out
                     ws.data_ptr(), ws.numel(), s)
     _check(rc, "mru_scan_fused")
     return o_out, snapshots
+
+
+def scan_fused_host_t(p: Problem, x_host, *, S0=None, out_host=None, x_dev=None, out_dev=None, ws=None,
+                      pieces: int = 0, streams=None, device="cuda"):
+    """Full-state scan from and to host memory: x_host is a CPU tensor
+    [B, L, H*n*n] (pinned for full speed); returns the CPU tensor S
+    [B, L, H, n, n] (out_host, pinned when allocated here) after the copies
+    completed.  The device staging buffers and the workspace are allocated
+    here when not given; streams = (compute, h2d, d2h) torch streams."""
+    torch = _torch()
+    B, L, H, n = p.B, p.L, p.H, p.n
+    if x_host.device.type != "cpu" or not x_host.is_contiguous():
+        raise ValueError("x_host must be a contiguous CPU tensor")
+    if out_host is None:
+        out_host = torch.empty((B, L, H, n, n), dtype=torch.float32, pin_memory=True)
+    if x_dev is None:
+        x_dev = torch.empty(x_host.shape, dtype=x_host.dtype, device=device)
+    if out_dev is None:
+        out_dev = torch.empty((B, L, H, n, n), dtype=torch.float32, device=device)
+    if ws is None:
+        ws = workspace_t(p, device)
+    if streams is None:
+        streams = (torch.cuda.current_stream(), torch.cuda.Stream(), torch.cuda.Stream())
+    sc, si, so = (st.cuda_stream for st in streams)
+    rc = scan_fused_host(p, x_host.data_ptr(), _dev_ptr(S0, "S0"), None, out_host.data_ptr(), None,
+                         x_dev.data_ptr(), out_dev.data_ptr(), ws.data_ptr(), ws.numel(), pieces, sc, si, so)
+    _check(rc, "mru_scan_fused_host")
+    streams[0].synchronize()
+    return out_host
 
 
 def scan_backward_t(p: Problem, x, S_fwd, dS, *, S0=None, dx=None, dS0=None, ws=None, stream=None):

@@ -117,3 +117,42 @@ def test_binding_fails_loudly_without_library(tmp_path):
             mru.load(missing)
     finally:
         mru._lib = saved
+
+
+def test_single_chunk_problems_take_one_launch(lib):
+    """A problem of one chunk per sequence (L <= chunk: decode steps, short
+    segments) runs one kernel from S0; longer ones run the full pass order."""
+    cases = [(mru.problem(8, 8, 1, 16, mode=mru.MODE_DETNORM, alpha=0.0125), ["k16_apply"]),
+             (mru.problem(4, 16, 1, 32, x_dtype="bf16", mode=mru.MODE_LDU), ["k32_apply"]),
+             (mru.problem(2, 3, 5, 8, mode=mru.MODE_CAYLEY, alpha=0.1), ["k_chunk_prefix"]),
+             (mru.problem(2, 4, 16, 64, mode=mru.MODE_DETNORM, alpha=0.01, chunk=16), ["k_chunk_prefix"])]
+    for p, names in cases:
+        assert mru.launch_count(p) == 1 and mru.kernel_names(p) == names
+    p = mru.problem(8, 8, 4096, 16, mode=mru.MODE_DETNORM, alpha=0.0125)
+    assert mru.kernel_names(p) == ["k16_reduce", "k16_carry", "k16_apply"]
+    p = mru.problem(2, 4, 16, 64, mode=mru.MODE_DETNORM, alpha=0.01, chunk=16)
+    assert mru.kernel_names(p, True) == ["k_chunk_prefix"]
+    p = mru.problem(2, 4, 4096, 64, mode=mru.MODE_DETNORM, alpha=0.01, math="tf32")
+    assert mru.kernel_names(p, True)[0] == "k64_chunk_readout" and mru.launch_count(p, True) == 5
+
+
+def test_host_entry_rejects_bad_arguments(lib):
+    p = mru.problem(2, 2, 8, 16)
+    nb = mru.workspace_size(p)
+    fake = 1 << 20
+    ok = dict(x_host=fake, out_host=2 * fake, x_dev=3 * fake, out_dev=4 * fake, ws=5 * fake)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return mru.scan_fused_host(p, a["x_host"], None, None, a["out_host"], None, a["x_dev"], a["out_dev"],
+                                   a["ws"], nb, kw.get("pieces", 0))
+    assert call(x_host=0) == mru.ERR_INVALID_ARG
+    assert call(out_host=0) == mru.ERR_INVALID_ARG
+    assert call(x_dev=3 * fake + 8) == mru.ERR_INVALID_ARG          # misaligned staging
+    assert call(out_dev=3 * fake) == mru.ERR_INVALID_ARG            # staging buffers alias
+    assert call(pieces=-1) == mru.ERR_INVALID_ARG
+    ro = mru.Readout(6 * fake, 4, None)                              # snapshots without a staging buffer
+    assert mru.scan_fused_host(p, fake, None, ro, 2 * fake, None, 3 * fake, 4 * fake, 5 * fake, nb) == \
+        mru.ERR_INVALID_ARG
+    assert mru.scan_fused_host(p, fake, None, None, 2 * fake, None, 3 * fake, 4 * fake, 5 * fake, 255) == \
+        mru.ERR_WORKSPACE

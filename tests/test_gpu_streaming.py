@@ -11,7 +11,7 @@ import pytest
 from linear_rnn_scan_b200 import inputs as gen
 from linear_rnn_scan_b200 import mru
 
-from gpu_helpers import compare_S, run_fused, tol_for_problem, torch
+from gpu_helpers import compare_readout, compare_S, run_fused, tol_for_problem, torch
 
 pytestmark = pytest.mark.gpu
 
@@ -76,3 +76,21 @@ def test_token_by_token_decode(n, mode, dtype, alpha):
     e = compare_S(w, x, np.concatenate(steps, axis=1))
     assert e["count"] == w.B * w.H * w.L
     assert e["max"] <= tol_for_problem(w), e
+
+
+@pytest.mark.parametrize("n", [4, 8, 16, 32, 64])
+def test_single_chunk_readout_from_S0(n):
+    """A segment no longer than one chunk runs as one launch started from S0
+    (the decode path); with the readout its outputs are final there too:
+    o_t = S_t U with S_t = S0 X_1 ... X_t, and the snapshots."""
+    w = _workload(n, gen.MODE_DETNORM, "f32", 0.3 / np.sqrt(n), B=2, H=3, L=12, seed=1400 + n)
+    w = w.with_(readout=True, snapshot_every=4)
+    x = gen.make_x(w)
+    S0 = gen.make_S0(w, seed=1401)
+    U = (np.random.default_rng(1402).standard_normal((w.H, n, 3)) / np.sqrt(n)).astype(np.float32)
+    p = mru.problem_from_workload(w, chunk=16)
+    assert mru.launch_count(p, True) == 1 and mru.kernel_names(p, True) == ["k_chunk_prefix"]
+    (o, snaps), st = run_fused(w, x, S0=S0, u=U, every=4, chunk=16)
+    assert st == mru.OK
+    e = compare_readout(w, x, o, snaps, U, 4, S0=S0)
+    assert e["o"]["max"] <= tol_for_problem(w, chunk=16) and e["snap"]["max"] <= tol_for_problem(w, chunk=16), e
