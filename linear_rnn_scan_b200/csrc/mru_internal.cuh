@@ -142,6 +142,14 @@ cudaError_t launch_carry(const KParams& p, const float* totals, const CarryPlan&
 // the carry S0 (or I when S0 is null); no reduce or carry launch precedes it.
 cudaError_t launch_apply(const KParams& p, const float* x, const CarryPlan& cp, const char* ws, float* S_out,
                          uint32_t* status, const float* S0, bool direct, cudaStream_t s);
+// Backward passes on the tensor cores (fp32 embeddings, reshape, and the
+// determinant-corrected mode with the identity); the generic fp64 scan of
+// the chunk gradients runs between them.
+bool supports_backward(const KParams& p);
+cudaError_t launch_bwd_local(const KParams& p, const float* x, const float* dS, float* gloc, float* Wq,
+                             uint32_t* status, cudaStream_t s);
+cudaError_t launch_bwd_apply(const KParams& p, const float* x, const float* S0, const float* S_fwd, const float* dS,
+                             const float* Gin, float* dx, float* dS0, uint32_t* status, cudaStream_t s);
 }  // namespace n16
 
 // n = 32 LDU tensor-core kernels (mru_n32.cu).

@@ -1022,9 +1022,545 @@ k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, 
     }
 }
 
+// ---- backward (vector-Jacobian product) on the tensor cores ----------------
+//
+// G_t = dL/dS_t (later states included): G_{t-1} = dS_{t-1} + G_t X_t^T and
+// dL/dX_t = S_{t-1}^T G_t, the chain rule of S_t = S_{t-1} X_t.  Chunked as
+// the generic backward is: a local pass per chunk [t0, t1) (the gradient at
+// t0 with nothing entering from the right, and W - I with
+// W = X_{t0+1} ... X_{t1}), the generic fp64 right-to-left scan of the chunk
+// gradients, and an apply pass per chunk (G from the gradient entering from
+// the right down to t0, dX_t, and the construction's chain rule).
+// Persistent warps, one chunk at a time, the chunk's tokens in reverse order
+// through a cp.async pipeline of 2-token stages (x_t, S_{t-1}, dS_{t-1}); per
+// stage the two tokens' determinant scales (16 lanes per LU).  Split-tf32
+// products with the matrices in the accumulators:
+//   G <- dS_{t-1} + G + G F_t^T        B = F_t^T, read transposed from x_t
+//   W^T <- W^T + F_t^T + W^T F_t^T     (local pass; W^T keeps the left
+//                                       multiplications of W on the right)
+//   dX = S_{t-1}^T G                   G staged through shared memory
+// Determinant-corrected chain rule: dXr = c (dX - <dX, Xr> Xr^-T / 16),
+// dM = alpha dXr, with Xr^-T = (I + E^T)^-1 (E = alpha M) by Newton-Schulz in
+// split form: Y = I + Z, R = I - Y (I + E^T) = -(Z + E^T + Z E^T),
+// Z <- Z + R + R Z, from Z = -E^T.  The residual squares every step, from
+// at most |E|_F^2, so the least k with (|E|_F^2)^(2^k) <= 2^-20 steps are
+// run; all but the last in single tf32 (the iteration corrects what they
+// round), the last with Z E^T in split tf32.  |E|_F^2 > 0.8 (far from the
+// identity): Gauss-Jordan elimination with partial pivoting on the lanes.
+
+constexpr int BST = 2, BNS = 3, BWARPS = 4;
+
+template <bool Apply>
+struct BSmem {
+    float x[BNS][BST * NN];                           // slices x_t (swizzled)
+    float ds[BNS][BST * NN];                          // dS_{t-1}
+    float s[Apply ? BNS : 1][Apply ? BST * NN : 4];   // S_{t-1} (apply pass)
+    float stg[NN];                                    // a staged accumulator matrix (swizzled)
+    float2 cd[BST];                                   // per token: (c alpha, diagonal term of F)
+};
+
+// tf32 of v, rounded to nearest (the high part of split_tf32).
+__device__ __forceinline__ uint32_t tf32_rn(float v) { return (__float_as_uint(v) + 0x1000u) & 0xffffe000u; }
+
+// B fragments (split) of F^T for F = ca M + dv I, with the contraction index
+// permuted as in make_frag_f, and F^T at this lane's accumulator positions.
+__device__ __forceinline__ void make_frag_ft(const float* xs, float ca, float d0, float d1, int g, int q, FragF& f,
+                                             bool want_fd)
+{
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const float v0 = fmaf(ca, xs[swz(8 * nt + g, 8 * kt + 2 * q)], kt == nt ? d0 : 0.0f);
+            const float v1 = fmaf(ca, xs[swz(8 * nt + g, 8 * kt + 2 * q + 1)], kt == nt ? d1 : 0.0f);
+            split_tf32(v0, f.bh[kt][nt][0], f.bl[kt][nt][0]);
+            split_tf32(v1, f.bh[kt][nt][1], f.bl[kt][nt][1]);
+        }
+    if (want_fd) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+                f.fd[nt][2 * h8 + 0] = fmaf(ca, xs[swz(8 * nt + 2 * q, g + 8 * h8)], h8 == nt ? d0 : 0.0f);
+                f.fd[nt][2 * h8 + 1] = fmaf(ca, xs[swz(8 * nt + 2 * q + 1, g + 8 * h8)], h8 == nt ? d1 : 0.0f);
+            }
+    }
+}
+
+// acc = A B in single tf32: A the accumulator-resident matrix (permuted
+// contraction), b its partner's fragments.
+__device__ __forceinline__ void product_tf32(const float (&Ad)[2][4], const uint32_t (&b)[2][2][2], float (&acc)[2][4])
+{
+    uint32_t a[2][4];
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt) {
+        a[kt][0] = tf32_rn(Ad[kt][0]);
+        a[kt][1] = tf32_rn(Ad[kt][2]);
+        a[kt][2] = tf32_rn(Ad[kt][1]);
+        a[kt][3] = tf32_rn(Ad[kt][3]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        mma_tf32_first(acc[nt], a[0], b[0][nt]);
+        mma_tf32(acc[nt], a[1], b[1][nt]);
+    }
+}
+
+// An accumulator matrix into a swizzled shared tile, and back.
+__device__ __forceinline__ void stage_acc(float* t, const float (&Ad)[2][4], int g, int q)
+{
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8)
+            *reinterpret_cast<float2*>(t + swz(g + 8 * h8, 8 * nt + 2 * q)) = make_float2(Ad[nt][2 * h8], Ad[nt][2 * h8 + 1]);
+}
+__device__ __forceinline__ void unstage_acc(const float* t, float (&Ad)[2][4], int g, int q)
+{
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+            const float2 v = *reinterpret_cast<const float2*>(t + swz(g + 8 * h8, 8 * nt + 2 * q));
+            Ad[nt][2 * h8] = v.x;
+            Ad[nt][2 * h8 + 1] = v.y;
+        }
+}
+// A 16 x 16 row-major matrix in global memory into / out of accumulator layout.
+__device__ __forceinline__ void load_acc(float (&Ad)[2][4], const float* src, int g, int q)
+{
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+            const float2 v = *reinterpret_cast<const float2*>(src + (g + 8 * h8) * N + 8 * nt + 2 * q);
+            Ad[nt][2 * h8] = v.x;
+            Ad[nt][2 * h8 + 1] = v.y;
+        }
+}
+
+// dX = S^T G: A = S^T read from the swizzled tile ss (contraction in natural
+// order), B = G from the staging tile gs; split tf32, fp32 accumulation.
+__device__ __forceinline__ void st_times_g(const float* ss, const float* gs, int g, int q, float (&acc)[2][4])
+{
+    uint32_t ah[2][4], al[2][4], bh[2][2][2], bl[2][2][2];
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt) {
+        split_tf32(ss[swz(8 * kt + q, g)], ah[kt][0], al[kt][0]);
+        split_tf32(ss[swz(8 * kt + q, g + 8)], ah[kt][1], al[kt][1]);
+        split_tf32(ss[swz(8 * kt + q + 4, g)], ah[kt][2], al[kt][2]);
+        split_tf32(ss[swz(8 * kt + q + 4, g + 8)], ah[kt][3], al[kt][3]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            split_tf32(gs[swz(8 * kt + q, 8 * nt + g)], bh[kt][nt][0], bl[kt][nt][0]);
+            split_tf32(gs[swz(8 * kt + q + 4, 8 * nt + g)], bh[kt][nt][1], bl[kt][nt][1]);
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        mma_tf32_first(acc[nt], al[0], bh[0][nt]);
+        mma_tf32(acc[nt], al[1], bh[1][nt]);
+    }
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) mma_tf32(acc[nt], ah[kt], bl[kt][nt]);
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) mma_tf32(acc[nt], ah[kt], bh[kt][nt]);
+}
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);   // every lane ends with the same sum
+    return v;
+}
+
+// Z = Xr^-T - I for Xr = I + alpha M (the slice xs) by Gauss-Jordan
+// elimination with partial pivoting on [Xr^T | I]: lane i (and i + 16) holds
+// row i; Z goes to the accumulator positions through stg.  For tokens far
+// from the identity; kept out of line.
+__device__ __noinline__ void inverse_t_pivoted(const float* xs, float alpha, float* stg, int lane, float (&Z)[2][4])
+{
+    const int r = lane & 15, g = lane >> 2, q = lane & 3;
+    float a[N], b[N];
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+        a[j] = fmaf(alpha, xs[swz(j, r)], j == r ? 1.0f : 0.0f);    // Xr^T[r][j] = Xr[j][r]
+        b[j] = j == r ? 1.0f : 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < N; ++k) {
+        float best = r >= k ? fabsf(a[k]) : -1.0f;
+        int bi = r;
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) {
+            const float ob = __shfl_xor_sync(FULL, best, o, 16);
+            const int oi = __shfl_xor_sync(FULL, bi, o, 16);
+            if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+        }
+#pragma unroll
+        for (int j = 0; j < N; ++j) {                                 // swap rows k and bi
+            const float ak = __shfl_sync(FULL, a[j], k, 16), ap = __shfl_sync(FULL, a[j], bi, 16);
+            const float bk = __shfl_sync(FULL, b[j], k, 16), bp = __shfl_sync(FULL, b[j], bi, 16);
+            if (r == k) { a[j] = ap; b[j] = bp; } else if (r == bi) { a[j] = ak; b[j] = bk; }
+        }
+        const float pk = __shfl_sync(FULL, a[k], k, 16);
+        const float rp = pk != 0.0f ? 1.0f / pk : 0.0f;
+        const float f = a[k];
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            const float ak = __shfl_sync(FULL, a[j], k, 16) * rp, bk = __shfl_sync(FULL, b[j], k, 16) * rp;
+            if (r == k) { a[j] = ak; b[j] = bk; } else { a[j] = fmaf(-f, ak, a[j]); b[j] = fmaf(-f, bk, b[j]); }
+        }
+    }
+    __syncwarp();
+    if (lane < 16)
+#pragma unroll
+        for (int j = 0; j < N; ++j) stg[swz(r, j)] = b[j] - (j == r ? 1.0f : 0.0f);
+    __syncwarp();
+    unstage_acc(stg, Z, g, q);
+    __syncwarp();
+}
+
+// Z = (I + E^T)^-1 - I at the accumulator positions, fe = E^T's fragments and
+// values, fro2 = |E|_F^2 (the same on every lane); Newton-Schulz as above.
+__device__ __forceinline__ void inverse_t_ns(const FragF& fe, float fro2, float* stg, int g, int q, float (&Z)[2][4])
+{
+    const float l = -log2f(fmaxf(fro2, 1e-30f));
+    int k = 1;
+    while (k < 6 && (float)(1 << k) * l < 20.0f) ++k;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) Z[nt][i] = -fe.fd[nt][i];
+    for (int it = 1; it <= k; ++it) {
+        float P[2][4], R[2][4], Qz[2][4];
+        if (it == k) chain_product<true>(Z, fe, P);
+        else product_tf32(Z, fe.bh, P);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) R[nt][i] = -((Z[nt][i] + fe.fd[nt][i]) + P[nt][i]);
+        stage_acc(stg, Z, g, q);
+        __syncwarp();
+        uint32_t zb[2][2][2];
+#pragma unroll
+        for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                zb[kt][nt][0] = tf32_rn(stg[swz(8 * kt + 2 * q, 8 * nt + g)]);
+                zb[kt][nt][1] = tf32_rn(stg[swz(8 * kt + 2 * q + 1, 8 * nt + g)]);
+            }
+        __syncwarp();
+        product_tf32(R, zb, Qz);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) Z[nt][i] += R[nt][i] + Qz[nt][i];
+    }
+}
+
+// The producer side of a backward warp's pipeline: the next stage of items
+// along the warp's chains.  Items of a chunk [t0, t1): the token after it
+// when there is one (only its matrix is used), then t1 - 1 down to t0 (apply)
+// or t0 + 1 (local).
+template <bool Apply>
+struct BFeed {
+    int64_t chain, stride, nchains, tok;
+    int64_t t, lo, base;
+
+    __device__ __forceinline__ void set(const KParams& p)
+    {
+        while (chain < nchains) {
+            const Chain c = chain_at(p, chain);
+            const int64_t hi = c.tend < p.L ? c.tend : c.tend - 1;
+            const int64_t l = Apply ? c.tbeg : c.tbeg + 1;
+            if (hi >= l) {
+                t = hi;
+                lo = l;
+                base = (c.b * p.L * p.H + c.h) * NN;
+                return;
+            }
+            chain += stride;                 // no items (a one-token chunk at the end, local pass)
+        }
+    }
+
+    __device__ __forceinline__ void issue(BSmem<Apply>& sm, int slot, int lane, const KParams& p, const float* x,
+                                          const float* S, const float* dS)
+    {
+        if (chain < nchains) {
+            const int nt = (t - lo + 1 < BST) ? (int)(t - lo + 1) : BST;
+#pragma unroll
+            for (int i = 0; i < BST * 2; ++i) {       // 64 granules a tile, 2 per lane
+                const int gi = lane + 32 * i;
+                const int j = gi >> 6, gr = gi & 63, row = gr >> 2, c4 = gr & 3;
+                if (j < nt) {
+                    const int64_t tau = t - j;
+                    const int so = j * NN + swz(row, 4 * c4);
+                    const int64_t go = base + row * N + 4 * c4;
+                    cp_async16(&sm.x[slot][so], x + go + tau * tok);
+                    if (tau >= 1) {
+                        cp_async16(&sm.ds[slot][so], dS + go + (tau - 1) * tok);
+                        if (Apply) cp_async16(&sm.s[slot][so], S + go + (tau - 1) * tok);
+                    }
+                }
+            }
+            t -= BST;
+            if (t < lo) {
+                chain += stride;
+                set(p);
+            }
+        }
+        cp_async_commit();
+    }
+};
+
+// dS_{t-1} (a staged tile) added to the accumulator matrix: G = ds + (G + a).
+__device__ __forceinline__ void add_ds(const float* dst, const float (&a)[2][4], float (&G)[2][4], int g, int q)
+{
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+            const float2 v = *reinterpret_cast<const float2*>(dst + swz(g + 8 * h8, 8 * nt + 2 * q));
+            G[nt][2 * h8] = v.x + (G[nt][2 * h8] + a[nt][2 * h8]);
+            G[nt][2 * h8 + 1] = v.y + (G[nt][2 * h8 + 1] + a[nt][2 * h8 + 1]);
+        }
+}
+
+// Local pass: per chunk the gradient at t0 with nothing entering from the
+// right (gloc) and W - I (Wq; zero for the last chunk of a sequence).
+__global__ void __launch_bounds__(BWARPS * 32, 2)
+k16b_local(KParams p, const float* __restrict__ x, const float* __restrict__ dS, float* __restrict__ gloc,
+           float* __restrict__ Wq, uint32_t* status)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    BSmem<false>& sm = reinterpret_cast<BSmem<false>*>(smem_raw)[warp];
+    const int64_t nchains = p.B * p.H * p.K;
+    const int64_t first = (int64_t)blockIdx.x * BWARPS + warp, stride = (int64_t)gridDim.x * BWARPS;
+    const int64_t tok = p.H * NN;
+    const int g = lane >> 2, q = lane & 3;
+    const float m0 = (g == 2 * q) ? 1.0f : 0.0f, m1 = (g == 2 * q + 1) ? 1.0f : 0.0f;
+    BFeed<false> feed;
+    feed.chain = first;
+    feed.stride = stride;
+    feed.nchains = nchains;
+    feed.tok = tok;
+    feed.set(p);
+#pragma unroll
+    for (int s = 0; s < BNS - 1; ++s) feed.issue(sm, s, lane, p, x, nullptr, dS);
+    int cs = 0, ps = BNS - 1;
+    for (int64_t chain = first; chain < nchains; chain += stride) {
+        const Chain c = chain_at(p, chain);
+        const int64_t base = (c.b * p.L * p.H + c.h) * NN;
+        const bool more = c.tend < p.L;
+        float G[2][4], Wt[2][4];
+        load_acc(G, dS + base + (c.tend - 1) * tok, g, q);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) Wt[nt][i] = 0.0f;
+        const int64_t hi = more ? c.tend : c.tend - 1, lo = c.tbeg + 1;
+        for (int64_t ts = hi; ts >= lo; ts -= BST) {
+            feed.issue(sm, ps, lane, p, x, nullptr, dS);
+            ps = (ps + 1 == BNS) ? 0 : ps + 1;
+            cp_async_wait<BNS - 1>();
+            __syncwarp();
+            const int nt = (ts - lo + 1 < BST) ? (int)(ts - lo + 1) : BST;
+            stage_scalars<BST>(p, sm.cd, sm.x[cs], nt, lane, status);
+#pragma unroll
+            for (int j = 0; j < BST; ++j) {
+                if (j < nt) {
+                    const int64_t tau = ts - j;
+                    const float2 cdj = sm.cd[j];
+                    FragF ft;
+                    make_frag_ft(sm.x[cs] + j * NN, cdj.x, m0 * cdj.y, m1 * cdj.y, g, q, ft, more);
+                    if (tau == c.tend) {
+#pragma unroll
+                        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) Wt[n2][i] = ft.fd[n2][i];     // W^T = F_{t1}^T
+                    } else {
+                        float a[2][4];
+                        chain_product<true>(G, ft, a);
+                        add_ds(sm.ds[cs] + j * NN, a, G, g, q);
+                        if (more) {
+                            chain_product<false>(Wt, ft, a);                       // F^T + W^T F^T
+#pragma unroll
+                            for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) Wt[n2][i] += a[n2][i];
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            cs = (cs + 1 == BNS) ? 0 : cs + 1;
+        }
+        // the chunk-gradient scan indexes chunks sequence-major: (b H + h) K + k
+        const int64_t wchain = (c.b * p.H + c.h) * p.K + c.k;
+        store_d(gloc + wchain * NN, G, g, q);
+        float* w = Wq + wchain * NN;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {                 // W = (W^T)^T
+                w[(8 * nt + 2 * q) * N + g + 8 * h8] = Wt[nt][2 * h8];
+                w[(8 * nt + 2 * q + 1) * N + g + 8 * h8] = Wt[nt][2 * h8 + 1];
+            }
+    }
+}
+
+// Apply pass: per chunk G from the gradient entering from the right (Gin)
+// down to t0, every dL/dx_t, and dL/dS0 from the first chunk.
+__global__ void __launch_bounds__(BWARPS * 32, 2)
+k16b_apply(KParams p, const float* __restrict__ x, const float* __restrict__ S0, const float* __restrict__ S_fwd,
+           const float* __restrict__ dS, const float* __restrict__ Gin, float* __restrict__ dx,
+           float* __restrict__ dS0, uint32_t* status)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    BSmem<true>& sm = reinterpret_cast<BSmem<true>*>(smem_raw)[warp];
+    const int64_t nchains = p.B * p.H * p.K;
+    const int64_t first = (int64_t)blockIdx.x * BWARPS + warp, stride = (int64_t)gridDim.x * BWARPS;
+    const int64_t tok = p.H * NN;
+    const int g = lane >> 2, q = lane & 3;
+    const float m0 = (g == 2 * q) ? 1.0f : 0.0f, m1 = (g == 2 * q + 1) ? 1.0f : 0.0f;
+    const bool detnorm = p.mode == MRU_MODE_DETNORM;
+    BFeed<true> feed;
+    feed.chain = first;
+    feed.stride = stride;
+    feed.nchains = nchains;
+    feed.tok = tok;
+    feed.set(p);
+#pragma unroll
+    for (int s = 0; s < BNS - 1; ++s) feed.issue(sm, s, lane, p, x, S_fwd, dS);
+    int cs = 0, ps = BNS - 1;
+    for (int64_t chain = first; chain < nchains; chain += stride) {
+        const Chain c = chain_at(p, chain);
+        const int64_t seq = c.b * p.H + c.h;
+        const int64_t base = (c.b * p.L * p.H + c.h) * NN;
+        const bool boundary = c.tend < p.L;
+        float G[2][4];
+        if (boundary) load_acc(G, Gin + (seq * p.K + c.k) * NN, g, q);   // sequence-major chunk index
+        else load_acc(G, dS + base + (c.tend - 1) * tok, g, q);
+        const int64_t hi = boundary ? c.tend : c.tend - 1, lo = c.tbeg;
+        for (int64_t ts = hi; ts >= lo; ts -= BST) {
+            feed.issue(sm, ps, lane, p, x, S_fwd, dS);
+            ps = (ps + 1 == BNS) ? 0 : ps + 1;
+            cp_async_wait<BNS - 1>();
+            __syncwarp();
+            const int nt = (ts - lo + 1 < BST) ? (int)(ts - lo + 1) : BST;
+            stage_scalars<BST>(p, sm.cd, sm.x[cs], nt, lane, status);
+#pragma unroll
+            for (int j = 0; j < BST; ++j) {
+                if (j < nt) {
+                    const int64_t tau = ts - j;
+                    const float* xs = sm.x[cs] + j * NN;
+                    const float2 cdj = sm.cd[j];
+                    FragF ft;
+                    make_frag_ft(xs, cdj.x, m0 * cdj.y, m1 * cdj.y, g, q, ft, false);
+                    float a[2][4];
+                    if (tau == c.tend) {                       // G_{t1-1} = dS_{t1-1} + Gin X_{t1}^T
+                        chain_product<true>(G, ft, a);
+                        add_ds(sm.ds[cs] + j * NN, a, G, g, q);
+                        continue;
+                    }
+                    // dX = S_{t-1}^T G (S_{-1} = S0 or I)
+                    float dX[2][4];
+                    stage_acc(sm.stg, G, g, q);
+                    __syncwarp();
+                    if (tau >= 1) {
+                        st_times_g(sm.s[cs] + j * NN, sm.stg, g, q, dX);
+                    } else if (S0) {
+                        float* s0t = sm.s[cs] + j * NN;    // S0 into the (unused) S tile of this token
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const int gr = lane + 32 * i, row = gr >> 2, c4 = gr & 3;
+                            *reinterpret_cast<float4*>(s0t + swz(row, 4 * c4)) =
+                                *reinterpret_cast<const float4*>(S0 + seq * NN + row * N + 4 * c4);
+                        }
+                        __syncwarp();
+                        st_times_g(s0t, sm.stg, g, q, dX);
+                    } else {
+#pragma unroll
+                        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) dX[n2][i] = G[n2][i];
+                    }
+                    __syncwarp();
+                    // the construction's chain rule
+                    float out[2][4];
+                    if (!detnorm) {
+#pragma unroll
+                        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) out[n2][i] = p.alpha * dX[n2][i];
+                    } else {
+                        // <dX, Xr> with Xr = I + alpha M at the accumulator positions
+                        float part = 0.0f;
+#pragma unroll
+                        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                            for (int h8 = 0; h8 < 2; ++h8) {
+                                const float2 v = *reinterpret_cast<const float2*>(xs + swz(g + 8 * h8, 8 * n2 + 2 * q));
+                                part = fmaf(dX[n2][2 * h8], fmaf(p.alpha, v.x, h8 == n2 ? m0 : 0.0f), part);
+                                part = fmaf(dX[n2][2 * h8 + 1], fmaf(p.alpha, v.y, h8 == n2 ? m1 : 0.0f), part);
+                            }
+                        const float s = warp_sum(part) * (1.0f / N);
+                        FragF fe;
+                        make_frag_ft(xs, p.alpha, 0.0f, 0.0f, g, q, fe, true);
+                        float f2 = 0.0f;
+#pragma unroll
+                        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) f2 = fmaf(fe.fd[n2][i], fe.fd[n2][i], f2);
+                        const float fro2 = warp_sum(f2);
+                        float Z[2][4];
+                        if (fro2 <= 0.8f) inverse_t_ns(fe, fro2, sm.stg, g, q, Z);
+                        else inverse_t_pivoted(xs, p.alpha, sm.stg, lane, Z);
+                        const float c1 = 1.0f + cdj.y;       // c (dv = c - 1)
+                        const float ac = cdj.x == 0.0f ? 0.0f : p.alpha * c1;   // singular token: zero
+#pragma unroll
+                        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                            for (int h8 = 0; h8 < 2; ++h8) {
+                                const float i0 = h8 == n2 ? m0 : 0.0f, i1 = h8 == n2 ? m1 : 0.0f;
+                                out[n2][2 * h8] = ac * fmaf(-s, Z[n2][2 * h8] + i0, dX[n2][2 * h8]);
+                                out[n2][2 * h8 + 1] = ac * fmaf(-s, Z[n2][2 * h8 + 1] + i1, dX[n2][2 * h8 + 1]);
+                            }
+                    }
+                    store_d(dx + base + tau * tok, out, g, q);
+                    // G_{t-1} = dS_{t-1} + G X_t^T, or dS0 = G X_1^T at the first token
+                    if (tau > lo || tau == 0) {
+                        chain_product<true>(G, ft, a);
+                        if (tau == 0) {
+                            if (dS0) {
+#pragma unroll
+                                for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                                    for (int i = 0; i < 4; ++i) a[n2][i] += G[n2][i];
+                                store_d(dS0 + seq * NN, a, g, q);
+                            }
+                        } else {
+                            add_ds(sm.ds[cs] + j * NN, a, G, g, q);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            cs = (cs + 1 == BNS) ? 0 : cs + 1;
+        }
+    }
+}
+
 // CTAs of a persistent launch: resident CTAs per SM times the SM count,
 // cached per device and kernel slot; no more than the chains need.
-std::atomic<int> g_resident[64][4];
+std::atomic<int> g_resident[64][6];
 
 cudaError_t persistent_grid(int slot, const void* kern, int threads, size_t smem, int warps, int64_t nchains,
                             unsigned& grid)
@@ -1131,6 +1667,45 @@ cudaError_t launch_carry(const KParams& p, const float* totals, const CarryPlan&
     cudaError_t e = cudaFuncSetAttribute(k16_carry, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     k16_carry<<<(unsigned)((units + CWARPS - 1) / CWARPS), CWARPS * 32, sm, s>>>(p, totals, cp, ws, S0);
+    return cudaGetLastError();
+}
+
+bool supports_backward(const KParams& p)
+{
+    return p.n == N && p.src == SRC_EMBEDDING && p.x_dtype == MRU_F32 &&
+           (p.mode == MRU_MODE_RESHAPE || (p.mode == MRU_MODE_DETNORM && p.add_identity)) &&
+           (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32X3) && p.chunk > 0;
+}
+
+cudaError_t launch_bwd_local(const KParams& p, const float* x, const float* dS, float* gloc, float* Wq,
+                             uint32_t* status, cudaStream_t s)
+{
+    const int64_t nchains = p.B * p.H * p.K;
+    if (nchains == 0) return cudaSuccess;
+    if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    const size_t sm = sizeof(BSmem<false>) * BWARPS;
+    cudaError_t e = cudaFuncSetAttribute(k16b_local, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    unsigned grid = 0;
+    if ((e = persistent_grid(4, (const void*)k16b_local, BWARPS * 32, sm, BWARPS, nchains, grid)) != cudaSuccess)
+        return e;
+    k16b_local<<<grid, BWARPS * 32, sm, s>>>(p, x, dS, gloc, Wq, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_apply(const KParams& p, const float* x, const float* S0, const float* S_fwd, const float* dS,
+                             const float* Gin, float* dx, float* dS0, uint32_t* status, cudaStream_t s)
+{
+    const int64_t nchains = p.B * p.H * p.K;
+    if (nchains == 0) return cudaSuccess;
+    if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    const size_t sm = sizeof(BSmem<true>) * BWARPS;
+    cudaError_t e = cudaFuncSetAttribute(k16b_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    unsigned grid = 0;
+    if ((e = persistent_grid(5, (const void*)k16b_apply, BWARPS * 32, sm, BWARPS, nchains, grid)) != cudaSuccess)
+        return e;
+    k16b_apply<<<grid, BWARPS * 32, sm, s>>>(p, x, S0, S_fwd, dS, Gin, dx, dS0, status);
     return cudaGetLastError();
 }
 

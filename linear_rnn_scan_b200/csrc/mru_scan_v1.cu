@@ -1282,8 +1282,22 @@ cudaError_t backward_n(const KParams& p, const void* src, const float* S0, const
     const size_t sm_carry = sizeof(double) * 2 * NN;
     const size_t sm_apply = sizeof(float) * gfl_apply * GPB;
     const unsigned grid = (unsigned)((chains + GPB - 1) / GPB);
-    if ((e = set_smem(k_bwd_local<N, Grp>, sm_local)) != cudaSuccess) return e;
     if ((e = set_smem(k_bwd_carry<N>, sm_carry)) != cudaSuccess) return e;
+    if (N == 16 && n16::supports_backward(p)) {
+        // n = 16 on the tensor cores; the chunk-gradient scan stays generic
+        const float* x = reinterpret_cast<const float*>(src);
+        profile_mark(0, 0, s);
+        if ((e = n16::launch_bwd_local(p, x, dS, gloc, Wq, status, s)) != cudaSuccess) return e;
+        profile_mark(0, 1, s);
+        profile_mark(1, 0, s);
+        k_bwd_carry<N><<<(unsigned)BH, kThreads, sm_carry, s>>>(p, gloc, Wq, Gin);
+        profile_mark(1, 1, s);
+        profile_mark(2, 0, s);
+        if ((e = n16::launch_bwd_apply(p, x, S0, S_fwd, dS, Gin, dx, dS0, status, s)) != cudaSuccess) return e;
+        profile_mark(2, 1, s);
+        return cudaGetLastError();
+    }
+    if ((e = set_smem(k_bwd_local<N, Grp>, sm_local)) != cudaSuccess) return e;
     if ((e = set_smem(k_bwd_apply<N, Grp>, sm_apply)) != cudaSuccess) return e;
     profile_mark(0, 0, s);
     k_bwd_local<N, Grp><<<grid, kThreads, sm_local, s>>>(p, src, dS, gloc, Wq, status, gfl_local);

@@ -116,3 +116,23 @@ def test_backward_default_workload_sampled():
         dx_o, _ = oracle.backward(oracle_problem(ws1), x1, dS1)
         e = _rel(dx[b, :, h], dx_o.reshape(w.L, 256), axis=-1)
         assert e.max() <= TOL_BWD, (b, h, e.max(), np.median(e))
+
+
+@pytest.mark.parametrize("alpha", [0.002, 0.0125, 0.04, 0.055, 0.1])
+def test_backward_n16_inverse_regimes(alpha):
+    """n = 16 determinant-corrected backward on the tensor cores: the Xr^-T of
+    its chain rule takes 1 to 6 Newton-Schulz steps as |alpha M|_F grows, and
+    Gauss-Jordan with pivoting beyond (alpha 0.1: |alpha M|_F near 1.6).  (At
+    alpha 0.2 some I + alpha M are ill-conditioned enough that the fp32
+    inverse alone moves dx by about 1e-4, on any path.)"""
+    rng = np.random.default_rng(int(alpha * 1e4))
+    w = gen.Workload("ns", B=1, H=2, L=37, n=16, x_dtype="f32", mode=gen.MODE_DETNORM, alpha=alpha, seed=610)
+    x = gen.make_x(w)
+    S0 = gen.make_S0(w, seed=611)
+    dS = rng.standard_normal((w.B, w.L, w.H, 16, 16)).astype(np.float32)
+    dx, dS0, st = _run(w, x, S0, dS, chunk=8)
+    assert st == mru.OK
+    dx_o, dS0_o = oracle.backward(oracle_problem(w), x, dS.astype(np.float64), S0=S0.astype(np.float64))
+    e_dx = _rel(dx.reshape(w.B, w.L, w.H, 256), dx_o.reshape(w.B, w.L, w.H, 256), axis=-1)
+    e_s0 = _rel(dS0.reshape(w.B, w.H, 256), dS0_o.reshape(w.B, w.H, 256), axis=-1)
+    assert e_dx.max() <= TOL_BWD and e_s0.max() <= TOL_BWD, (e_dx.max(), np.median(e_dx), e_s0.max())
