@@ -1,6 +1,6 @@
 // mru_n16.cu -- n = 16 scan kernels on the tensor cores (fp32 embeddings,
-// reshape and determinant-corrected modes): two launches, two passes over
-// the embeddings.
+// reshape and determinant-corrected modes): three launches, two passes over
+// the embeddings; and the backward's two passes (at the end of the file).
 //
 // Both passes run persistent warps: warp w of W takes the chains (b, h,
 // chunk of C tokens) w, w + W, w + 2W, ... (a CTA's warps hold neighbouring
@@ -20,14 +20,13 @@
 //                  multiplicative, so the product of the corrected matrices
 //                  is gamma P~ with gamma = |det P~|^(-1/16), one 16 x 16
 //                  factorisation per chunk.
-//                  Carry scan, in the same launch: after writing a chunk
-//                  total the warp counts itself in at the chunk's group of G
-//                  totals (an atomic counter); the last of a group scans the
-//                  group (inclusive in-group prefixes and the group total, in
-//                  fp64 on the tensor cores, mma.sync m8n8k4) and counts the
-//                  group total in one level up; the last at the top level
-//                  scans the top from S0 into exclusive carries.  No warp
-//                  waits for another: whoever completes a group does its scan.
+//  * carry scan    its own launch between the passes: a warp per group of G
+//                  chunk totals scans the group (inclusive in-group prefixes
+//                  and the group total, fp64 on the tensor cores, mma.sync
+//                  m8n8k4) and counts the group total in one level up (an
+//                  atomic counter); the last warp of a group there scans that
+//                  one, up to the top, which is scanned from S0 into
+//                  exclusive carries.  No warp waits for another.
 //  * apply pass    each chain's first stage brings the chain's carry factors
 //                  (the top carry and one in-group prefix per level), their
 //                  product is formed in fp64; per stage of 8 tokens the
