@@ -373,7 +373,7 @@ def run_ours(args, w):
                "seconds": round(el, 2)}
 
     p = mru.problem_from_workload(w)
-    chunk = mru.chosen_chunk(p)
+    chunk = mru.chosen_chunk(p, w.readout)
     stream = torch.cuda.current_stream()
     s_handle = stream.cuda_stream
     if w.x_dtype == "bf16":
@@ -729,7 +729,7 @@ def run_decode(args, w):
                       if graph_ms else {"unavailable": graph_err}),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic (seeded N(0,1) embeddings)",
-            "config": dict(workload_config(wd, mru.chosen_chunk(p)), sequences=units),
+            "config": dict(workload_config(wd, mru.chosen_chunk(p, wd.readout)), sequences=units),
             "clocks": clocks.summary(), "gpu_launches": mru.launch_count(p) * args.steps,
             "kernels": mru.kernel_names(p)}), flush=True)
     ranks.close()

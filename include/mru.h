@@ -204,8 +204,9 @@ const char* mru_status_string(mru_status s);
  * MRU_MATH_BF16X3 for the tensor-core kernels); -1 if p is invalid. */
 int32_t mru_effective_math(const mru_problem* p, int32_t readout);
 
-/* Chunk length the library would use for this problem (0 if invalid). */
-int32_t mru_chosen_chunk(const mru_problem* p);
+/* Chunk length the library would use for this problem, with the readout
+ * (readout != 0) or with every state written (0 if p is invalid). */
+int32_t mru_chosen_chunk(const mru_problem* p, int32_t readout);
 
 /* Number of kernel launches one call of mru_scan_fused makes for p. */
 int32_t mru_launch_count(const mru_problem* p, int32_t readout);

@@ -33,10 +33,11 @@ constexpr int ROWW = 68;             // padded shared-memory row stride in words
 constexpr int THREADS = 128;
 
 struct Smem {
-    float x[N * ROWW];               // 17,408 bytes: the token's slice
+    float x[2][N * ROWW];            // 2 x 17,408 bytes: this token's slice and the next one's
     float prow[2][N];                // pivot row, double-buffered by step parity
     float pcol[2][N];                // pivot column
     float ut[N * N];                 // the head's query columns U, transposed: ut[c][j] = U[j][c]
+    float red[4][8];                 // per-warp partial traces and norms
     double dsum;                     // pivoted fallback: log|det|
     int flag;
     int piv;
@@ -49,12 +50,11 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::); }
 
-__device__ __forceinline__ uint32_t to_tf32(float v)
-{
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(v));
-    return r;
-}
+// v rounded to the nearest tf32, ties away from zero (the magnitude bits plus
+// half a unit of the 10th mantissa bit, then truncated): two integer
+// operations on the ALU pipe, the same value cvt.rna.tf32.f32 gives for
+// finite v.
+__device__ __forceinline__ uint32_t to_tf32(float v) { return (__float_as_uint(v) + 0x1000u) & 0xffffe000u; }
 
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
@@ -70,13 +70,13 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 // Thread (br, bc) updates its whole 4 x 8 block at every step where the block
 // reaches below and right of the pivot: entries in eliminated rows or columns
 // are never read again, so they need no masking.
-__device__ float absdet_near_identity(Smem& sm, float alpha, bool& ok)
+__device__ float absdet_near_identity(Smem& sm, const float* xs, float alpha, bool& ok)
 {
     const int t = threadIdx.x, br = t >> 3, bc = t & 7;
     float e[4][8];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const float4* row = reinterpret_cast<const float4*>(sm.x + (4 * br + r) * ROWW + 8 * bc);
+        const float4* row = reinterpret_cast<const float4*>(xs + (4 * br + r) * ROWW + 8 * bc);
         const float4 v0 = row[0], v1 = row[1];
         e[r][0] = alpha * v0.x; e[r][1] = alpha * v0.y; e[r][2] = alpha * v0.z; e[r][3] = alpha * v0.w;
         e[r][4] = alpha * v1.x; e[r][5] = alpha * v1.y; e[r][6] = alpha * v1.z; e[r][7] = alpha * v1.w;
@@ -123,10 +123,9 @@ __device__ float absdet_near_identity(Smem& sm, float alpha, bool& ok)
 // log|det(W)|, W = add_identity I + alpha M, by LU with partial pivoting on
 // a copy in shared memory (the slice buffer is overwritten; it is reloaded
 // afterwards).  Returns NaN when a pivot column is zero.
-__device__ double logdet_pivoted(Smem& sm, float alpha, int add_identity)
+__device__ double logdet_pivoted(Smem& sm, float* W, float alpha, int add_identity)
 {
     const int t = threadIdx.x;
-    float* W = sm.x;
     for (int e = t; e < NN; e += THREADS) {
         const int i = e / N, j = e % N;
         float v = alpha * W[i * ROWW + j];
@@ -178,14 +177,42 @@ __device__ double logdet_pivoted(Smem& sm, float alpha, int add_identity)
     return bad ? __longlong_as_double(0x7ff8000000000000ll) : ld;
 }
 
-__device__ __forceinline__ void load_slice(Smem& sm, const float* src)
+// Copies a token's slice into a slice buffer (cp.async, committed as one group).
+__device__ __forceinline__ void issue_slice(float* xs, const float* src)
 {
     for (int g = threadIdx.x; g < NN / 4; g += THREADS) {
         const int row = g >> 4, c4 = g & 15;
-        cp_async16(sm.x + row * ROWW + 4 * c4, src + row * N + 4 * c4);
+        cp_async16(xs + row * ROWW + 4 * c4, src + row * N + 4 * c4);
     }
-    cp_async_wait_all();
+    asm volatile("cp.async.commit_group;\n" ::);
+}
+
+// Plain reload of a slice (after the pivoted fallback has overwritten it).
+__device__ __forceinline__ void reload_slice(float* xs, const float* src)
+{
+    for (int g = threadIdx.x; g < NN / 4; g += THREADS) {
+        const int row = g >> 4, c4 = g & 15;
+        *reinterpret_cast<float4*>(xs + row * ROWW + 4 * c4) = *reinterpret_cast<const float4*>(src + row * N + 4 * c4);
+    }
     __syncthreads();
+}
+
+// B fragment of the raw slice M for k-tile kt and column tile nt, the
+// contraction index permuted as for the accumulator-resident A operands
+// (slot q <-> row 8 kt + 2 q, slot q + 4 <-> row 8 kt + 2 q + 1).
+__device__ __forceinline__ void frag_m(const float* xs, int kt, int nt, int g, int q, uint32_t& b0, uint32_t& b1)
+{
+    const float* base = xs + (8 * kt + 2 * q) * ROWW + 8 * nt + g;
+    b0 = to_tf32(base[0]);
+    b1 = to_tf32(base[ROWW]);
+}
+
+// Sum over the warp, the same value in every lane.
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
 }
 
 __global__ void __launch_bounds__(THREADS, 4)
@@ -218,29 +245,147 @@ k64_chunk_readout(KParams p, const float* __restrict__ x, const float* __restric
 #pragma unroll
         for (int i = 0; i < 4; ++i) Qd[nt][i] = 0.0f;
 
+    // the determinant scale by the trace series (see series_logdet) where its
+    // certificate holds; the near-identity LU otherwise
+    const bool detnorm = p.mode == MRU_MODE_DETNORM;
+    const bool series = detnorm && p.add_identity != 0;
+    issue_slice(sm.x[0], xb + t0 * tok);
     for (int64_t t = t0; t < t1; ++t) {
-        const float* src = xb + t * tok;
-        load_slice(sm, src);
+        const int cur = (int)((t - t0) & 1);
+        float* xs = sm.x[cur];
+        if (t + 1 < t1) issue_slice(sm.x[cur ^ 1], xb + (t + 1) * tok);
+        else asm volatile("cp.async.commit_group;\n" ::);
+        asm volatile("cp.async.wait_group 1;\n" ::);
+        __syncthreads();
+
+        // ---- for the series: M2 = M M over this warp's rows ----
+        float M2[8][4];
+        if (series) {
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) M2[nt][i] = 0.0f;
+#pragma unroll
+            for (int kt = 0; kt < 8; ++kt) {
+                uint32_t am[4];
+                const float2 m0 = *reinterpret_cast<const float2*>(xs + (r0 + g) * ROWW + 8 * kt + 2 * q);
+                const float2 m1 = *reinterpret_cast<const float2*>(xs + (r0 + g + 8) * ROWW + 8 * kt + 2 * q);
+                am[0] = to_tf32(m0.x);
+                am[1] = to_tf32(m1.x);
+                am[2] = to_tf32(m0.y);
+                am[3] = to_tf32(m1.y);
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) {
+                    uint32_t b0, b1;
+                    frag_m(xs, kt, nt, g, q, b0, b1);
+                    mma_tf32(M2[nt], am, b0, b1);
+                }
+            }
+        }
+
         // ---- determinant scale ----
         float ca = p.alpha, dv = p.add_identity ? 0.0f : -1.0f;
-        if (p.mode == MRU_MODE_DETNORM) {
-            // near the identity: |det| = prod (1 + delta_k) in fp32 (64
-            // factors near 1, relative error about 2e-7), c - 1 =
-            // expm1(-log1p(|det| - 1) / 64); otherwise the pivoted LU's fp64 sum
+        if (detnorm) {
+            bool ok = false;
             float cm1 = 0.0f;
-            bool ok = p.add_identity != 0;
-            if (ok) cm1 = expm1f(-log1pf(absdet_near_identity(sm, p.alpha, ok) - 1.0f) * (1.0f / N));
-            __syncthreads();
-            const bool retry = __syncthreads_or(!ok);
-            bool bad = false;
-            if (retry) {
-                const double ld = logdet_pivoted(sm, p.alpha, p.add_identity);
-                load_slice(sm, src);                 // the fallback overwrote the slice
-                bad = !isfinite(ld);
-                cm1 = (float)expm1(-ld / N);
+            if (series) {
+                // log det(I + E), E = alpha M, by its trace series
+                //   tr E - tr E^2 / 2 + tr E^3 / 3 - tr E^4 / 4 + R,
+                // tr E^k = <E^(k-1), E^T> from M2 = M M and M3 = M2 M (tf32
+                // products on the tensor cores).  Since tr E^k = <E^(k-3), (E^3)^T>
+                // and |E^m|_F <= |E^2|_F |E|_F^(m-2),
+                //   |R| <= |E^3|_F |E^2|_F / (5 (1 - |E|_F))   (|E|_F < 1),
+                // the series is taken when that bound is at most 1e-6 (the scale
+                // c = exp(-log det / 64) then good to 1.6e-8; the tf32 rounding of
+                // M2 and M3 adds about 1e-8 to log det at the workload's alpha).
+                float tr1 = 0.0f, tr2 = 0.0f, tr3 = 0.0f, tr4 = 0.0f, n1 = 0.0f, n2 = 0.0f, n3 = 0.0f;
+                if (lane < 16) tr1 = xs[(r0 + lane) * ROWW + r0 + lane];
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                    for (int h8 = 0; h8 < 2; ++h8) {
+                        const int row = r0 + g + 8 * h8, col = 8 * nt + 2 * q;
+                        const float2 mv = *reinterpret_cast<const float2*>(xs + row * ROWW + col);
+                        const float mt0 = xs[col * ROWW + row], mt1 = xs[(col + 1) * ROWW + row];   // M^T here
+                        tr2 = fmaf(mv.x, mt0, fmaf(mv.y, mt1, tr2));
+                        tr3 = fmaf(M2[nt][2 * h8], mt0, fmaf(M2[nt][2 * h8 + 1], mt1, tr3));
+                        n1 = fmaf(mv.x, mv.x, fmaf(mv.y, mv.y, n1));
+                        n2 = fmaf(M2[nt][2 * h8], M2[nt][2 * h8], fmaf(M2[nt][2 * h8 + 1], M2[nt][2 * h8 + 1], n2));
+                    }
+                // M3 = M2 M, four column tiles at a time
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float M3[4][4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) M3[j][i] = 0.0f;
+#pragma unroll
+                    for (int kt = 0; kt < 8; ++kt) {
+                        uint32_t a[4];
+                        a[0] = to_tf32(M2[kt][0]);
+                        a[1] = to_tf32(M2[kt][2]);
+                        a[2] = to_tf32(M2[kt][1]);
+                        a[3] = to_tf32(M2[kt][3]);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint32_t b0, b1;
+                            frag_m(xs, kt, 4 * hh + j, g, q, b0, b1);
+                            mma_tf32(M3[j], a, b0, b1);
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+#pragma unroll
+                        for (int h8 = 0; h8 < 2; ++h8) {
+                            const int row = r0 + g + 8 * h8, col = 8 * (4 * hh + j) + 2 * q;
+                            const float mt0 = xs[col * ROWW + row], mt1 = xs[(col + 1) * ROWW + row];
+                            tr4 = fmaf(M3[j][2 * h8], mt0, fmaf(M3[j][2 * h8 + 1], mt1, tr4));
+                            n3 = fmaf(M3[j][2 * h8], M3[j][2 * h8], fmaf(M3[j][2 * h8 + 1], M3[j][2 * h8 + 1], n3));
+                        }
+                }
+                tr1 = warp_sum(tr1);
+                tr2 = warp_sum(tr2);
+                tr3 = warp_sum(tr3);
+                tr4 = warp_sum(tr4);
+                n1 = warp_sum(n1);
+                n2 = warp_sum(n2);
+                n3 = warp_sum(n3);
+                if (lane == 0) {
+                    float* rd = sm.red[warp];
+                    rd[0] = tr1; rd[1] = tr2; rd[2] = tr3; rd[3] = tr4; rd[4] = n1; rd[5] = n2; rd[6] = n3;
+                }
+                __syncthreads();
+                float v[7];
+#pragma unroll
+                for (int i = 0; i < 7; ++i) v[i] = (sm.red[0][i] + sm.red[1][i]) + (sm.red[2][i] + sm.red[3][i]);
+                const float a = p.alpha, a2 = a * a;
+                const float ld = a * v[0] - a2 * (0.5f * v[1]) + a2 * a * (v[2] * (1.0f / 3.0f)) -
+                                 a2 * a2 * (0.25f * v[3]);
+                const float fe = a * sqrtf(v[4]), fe2 = a2 * sqrtf(v[5]), fe3 = a2 * a * sqrtf(v[6]);
+                const float bound = fe3 * fe2 / (5.0f * (1.0f - fe));
+                ok = fe < 1.0f && bound <= 1e-6f;      // false for non-finite inputs too
+                if (ok) cm1 = expm1f(-ld * (1.0f / N));
+            }
+            if (!ok) {
+                // near the identity: |det| = prod (1 + delta_k) in fp32 (64
+                // factors near 1, relative error about 2e-7), c - 1 =
+                // expm1(-log1p(|det| - 1) / 64); otherwise the pivoted LU's fp64 sum
+                bool near = p.add_identity != 0;
+                if (near) cm1 = expm1f(-log1pf(absdet_near_identity(sm, xs, p.alpha, near) - 1.0f) * (1.0f / N));
+                __syncthreads();
+                const bool retry = __syncthreads_or(!near);
+                bool bad = false;
+                if (retry) {
+                    const double ld = logdet_pivoted(sm, xs, p.alpha, p.add_identity);
+                    reload_slice(xs, xb + t * tok);      // the fallback overwrote the slice
+                    bad = !isfinite(ld);
+                    cm1 = (float)expm1(-ld / N);
+                }
+                ok = !bad;
             }
             const float c = 1.0f + cm1;
-            if (bad || !isfinite(cm1) || !(c > 0.0f)) {
+            if (!ok || !isfinite(cm1) || !(c > 0.0f)) {
                 if (tid == 0) atomicOr(status, STATUS_SINGULAR);
                 ca = 0.0f;
                 dv = 0.0f;
@@ -249,29 +394,24 @@ k64_chunk_readout(KParams p, const float* __restrict__ x, const float* __restric
                 dv = p.add_identity ? cm1 : -1.0f;
             }
         }
-        // ---- Q_t = Q + (F + Q F), 1xTF32 ----
-        float acc[8][4];
+        // ---- Q_t = Q + (F + Q F), Q F = ca Q M + dv Q, F = ca M + dv I ----
+        float P[8][4];
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+            for (int i = 0; i < 4; ++i) P[nt][i] = 0.0f;
 #pragma unroll
         for (int kt = 0; kt < 8; ++kt) {
-            uint32_t a[4];
-            a[0] = to_tf32(Qd[kt][0]);
-            a[1] = to_tf32(Qd[kt][2]);
-            a[2] = to_tf32(Qd[kt][1]);
-            a[3] = to_tf32(Qd[kt][3]);
+            uint32_t aq[4];
+            aq[0] = to_tf32(Qd[kt][0]);
+            aq[1] = to_tf32(Qd[kt][2]);
+            aq[2] = to_tf32(Qd[kt][1]);
+            aq[3] = to_tf32(Qd[kt][3]);
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
-                // B fragment, contraction index permuted: slot q <-> row 8kt + 2q
-                const float* base = sm.x + (8 * kt + 2 * q) * ROWW + 8 * nt + g;
-                float v0 = ca * base[0], v1 = ca * base[ROWW];
-                if (kt == nt) {
-                    if (g == 2 * q) v0 += dv;
-                    if (g == 2 * q + 1) v1 += dv;
-                }
-                mma_tf32(acc[nt], a, to_tf32(v0), to_tf32(v1));
+                uint32_t b0, b1;
+                frag_m(xs, kt, nt, g, q, b0, b1);
+                mma_tf32(P[nt], aq, b0, b1);
             }
         }
 #pragma unroll
@@ -279,12 +419,14 @@ k64_chunk_readout(KParams p, const float* __restrict__ x, const float* __restric
 #pragma unroll
             for (int h8 = 0; h8 < 2; ++h8) {
                 const int row = r0 + g + 8 * h8, col = 8 * nt + 2 * q;
-                const float2 xv = *reinterpret_cast<const float2*>(sm.x + row * ROWW + col);
+                const float2 xv = *reinterpret_cast<const float2*>(xs + row * ROWW + col);
                 float f0 = ca * xv.x, f1 = ca * xv.y;
                 if (row == col) f0 += dv;
                 if (row == col + 1) f1 += dv;
-                Qd[nt][2 * h8] += f0 + acc[nt][2 * h8];
-                Qd[nt][2 * h8 + 1] += f1 + acc[nt][2 * h8 + 1];
+                const float q0 = fmaf(ca, P[nt][2 * h8], dv * Qd[nt][2 * h8]);
+                const float q1 = fmaf(ca, P[nt][2 * h8 + 1], dv * Qd[nt][2 * h8 + 1]);
+                Qd[nt][2 * h8] += f0 + q0;
+                Qd[nt][2 * h8 + 1] += f1 + q1;
             }
         // ---- readout of the local prefix: V_t = Q_t U (rq columns; the loop
         // bound is uniform over the CTA, so every lane reaches the shuffles) ----

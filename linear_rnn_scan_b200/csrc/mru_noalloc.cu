@@ -57,7 +57,7 @@ extern "C" mru_status mru_scan_fused_noalloc(const mru_problem* p, const void* x
     // Pick the chunk: the caller's, else the library's choice doubled until
     // the workspace fits the fixed scratch.
     if (q.chunk == 0) {
-        q.chunk = mru_chosen_chunk(&q);
+        q.chunk = mru_chosen_chunk(&q, ro != nullptr);
         while (mru_workspace_size(&q) > MRU_NOALLOC_SCRATCH_BYTES && (int64_t)q.chunk < q.L &&
                q.chunk < (1 << 30))
             q.chunk *= 2;

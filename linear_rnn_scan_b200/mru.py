@@ -82,7 +82,7 @@ def load(path: str = LIB_PATH):
             lib.mru_last_device_status.restype = ctypes.c_int
             lib.mru_status_string.argtypes = [ctypes.c_int]
             lib.mru_status_string.restype = ctypes.c_char_p
-            lib.mru_chosen_chunk.argtypes = [P]
+            lib.mru_chosen_chunk.argtypes = [P, ctypes.c_int32]
             lib.mru_chosen_chunk.restype = ctypes.c_int32
             lib.mru_launch_count.argtypes = [P, ctypes.c_int32]
             lib.mru_launch_count.restype = ctypes.c_int32
@@ -126,8 +126,8 @@ def workspace_size(p: Problem) -> int:
     return int(load().mru_workspace_size(ctypes.byref(p)))
 
 
-def chosen_chunk(p: Problem) -> int:
-    return int(load().mru_chosen_chunk(ctypes.byref(p)))
+def chosen_chunk(p: Problem, readout: bool = False) -> int:
+    return int(load().mru_chosen_chunk(ctypes.byref(p), 1 if readout else 0))
 
 
 def launch_count(p: Problem, readout: bool = False) -> int:

@@ -71,7 +71,10 @@ def test_workspace_size(lib):
 
 def test_chunk_override(lib):
     p = mru.problem(2, 3, 100, 16, chunk=7)
-    assert mru.chosen_chunk(p) == 7
+    assert mru.chosen_chunk(p) == 7 and mru.chosen_chunk(p, readout=True) == 7
+    # the n = 64 readout path takes longer chunks than the state-writing one
+    p64 = mru.problem_from_workload(gen.WORKLOADS["n64_detnorm_readout_b2h4l16384"])
+    assert mru.chosen_chunk(p64, readout=True) == 128 and mru.chosen_chunk(p64) == 32
     assert mru.launch_count(p) >= 1
     assert mru.launch_count(mru.problem(0, 3, 100, 16)) == 0
 

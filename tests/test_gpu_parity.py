@@ -210,6 +210,28 @@ def test_readout_unit_columns_exact(n):
         assert np.array_equal(o[:, :, h].astype(np.float64), S_ref[:, :, h][..., cols[h]])
 
 
+@pytest.mark.parametrize("chunk", [16, 32])
+def test_n64_determinant_series_and_lu_tokens_mixed(chunk):
+    """n = 64 readout in the determinant-corrected mode near the identity:
+    most tokens take the scale from the trace series on the tensor cores;
+    tokens t = 1 mod 3 (slice scaled by 6, |E|_F about 1.4) fail the series'
+    certificate and are factorised instead, tokens t = 2 mod 5 (scaled by
+    60, pivots far from 1) need the pivoted LU."""
+    n = 64
+    w = small(n, gen.MODE_DETNORM, B=1, H=2, L=90, alpha=0.03 / np.sqrt(n), seed=660).with_(readout=True,
+                                                                                          snapshot_every=8)
+    x = gen.make_x(w).reshape(w.B, w.L, w.H * n * n).copy()
+    x[:, 1::3] *= 6.0
+    x[:, 2::5] *= 60.0
+    u = gen.make_u(w)
+    (o, snaps), st = run_fused(w, x, u=u, every=8, chunk=chunk)
+    assert st == mru.OK
+    e = compare_readout(w, x, o, snaps, u, 8)
+    tol = tol_for_problem(w, chunk=chunk)
+    assert e["o"]["count"] == w.B * w.L * w.H
+    assert e["o"]["max"] <= tol and e["snap"]["max"] <= tol, e
+
+
 @pytest.mark.parametrize("n", [4, 16, 32])
 @pytest.mark.parametrize("mode", MODES)
 def test_unfused_build_then_scan(n, mode):
