@@ -547,6 +547,19 @@ def run_ours(args, w):
     return 0
 
 
+def bwd_kernel_names(w):
+    """The three launches of mru_scan_backward for this workload: the tensor-core
+    passes where the library has them (n = 16 fp32 reshape / corrected with the
+    identity, n = 32 LDU bf16), the generic kernels otherwise; the chunk-gradient
+    scan between them is always the generic one."""
+    if w.n == 16 and w.x_dtype == "f32" and (w.mode == gen.MODE_RESHAPE or
+                                              (w.mode == gen.MODE_DETNORM and w.add_identity)):
+        return ["k16b_local", "k_bwd_carry", "k16b_apply"]
+    if w.n == 32 and w.x_dtype == "bf16" and w.mode == gen.MODE_LDU:
+        return ["k32b_local", "k_bwd_carry", "k32b_apply"]
+    return ["k_bwd_local", "k_bwd_carry", "k_bwd_apply"]
+
+
 def run_backward(args, w):
     """One step = one mru_scan_backward over the whole workload (gradients of
     sum <dS, S> with respect to the embeddings), with x, the forward states
@@ -601,7 +614,7 @@ def run_backward(args, w):
     torch.cuda.synchronize()
     ranks.barrier()
     ms = ranks.max(ev0.elapsed_time(ev1) / args.steps)
-    names = ["k_bwd_local", "k_bwd_carry", "k_bwd_apply"]
+    names = bwd_kernel_names(w)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
     for e in evs:
         e.record(stream)

@@ -159,6 +159,13 @@ int32_t preferred_chunk(int64_t token_heads);
 cudaError_t launch_reduce(const KParams& p, const void* x, float* totals, cudaStream_t s);
 cudaError_t launch_apply(const KParams& p, const void* x, const carry::Plan& pl, const char* ws, float* S_out,
                          const float* S0, bool direct, cudaStream_t s);
+// Backward of the LDU scan (bf16 embeddings): local pass and apply pass; the
+// chunk-gradient scan between them is the generic one.
+bool supports_backward(const KParams& p);
+cudaError_t launch_bwd_local(const KParams& p, const void* x, const float* dS, float* gloc, float* Wq,
+                             cudaStream_t s);
+cudaError_t launch_bwd_apply(const KParams& p, const void* x, const float* S0, const float* S_fwd, const float* dS,
+                             const float* Gin, float* dx, float* dS0, cudaStream_t s);
 }  // namespace n32
 
 // n = 64 readout chunk kernel on the tensor cores (mru_n64.cu); the carry

@@ -18,6 +18,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "mru_internal.cuh"
 
@@ -50,6 +51,14 @@ template <int Pending>
 __device__ __forceinline__ void cp_async_wait()
 {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(Pending));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* smem_row)
+{
+    const unsigned a = static_cast<unsigned>(__cvta_generic_to_shared(smem_row));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(a));
 }
 
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* smem_row)
@@ -134,6 +143,25 @@ __device__ __forceinline__ void load_m_frags(const unsigned char* xs, int lane, 
         }
 }
 
+// B fragments of M^T (B[k][n] = M[n][k]) for all (kt, nt), in the layout of
+// load_m_frags: bm[kt][nt][h] holds M[8 nt + g][16 kt + 8 h + 2 q], + 1
+// (ldmatrix without transposition on rows of M).
+__device__ __forceinline__ void load_mt_frags(const unsigned char* xs, int lane, uint32_t (&bm)[2][4][2])
+{
+    const int r = lane & 7, kh = (lane >> 3) & 1, np2 = lane >> 4;
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {
+            uint32_t v[4];
+            ldsm_x4(v, xs + (8 * (2 * np + np2) + r) * ROWB + (16 * kt + 8 * kh) * 2);
+            bm[kt][2 * np][0] = v[0];
+            bm[kt][2 * np][1] = v[1];
+            bm[kt][2 * np + 1][0] = v[2];
+            bm[kt][2 * np + 1][1] = v[3];
+        }
+}
+
 // Keep the bf16 halves of a B register whose (k, n) satisfy k > n (lower)
 // or k < n (upper).  c = 16 kt + 8 h - 8 nt is the tile offset, d = 2 q - g.
 __device__ __forceinline__ uint32_t tri_mask(uint32_t v, int c, int d, bool lower)
@@ -170,6 +198,55 @@ __device__ __forceinline__ void tri_product(const uint32_t (&ah)[2][2][4], const
         }
 }
 
+// Three-term split of a pair (x ~ hi + mid + lo, the residual below 2^-26 |x|).
+__device__ __forceinline__ void split_pair3(float x0, float x1, uint32_t& hi, uint32_t& mid, uint32_t& lo)
+{
+    hi = pack_bf16(x0, x1);
+    const float r0 = x0 - bf16_lo(hi), r1 = x1 - bf16_hi(hi);
+    mid = pack_bf16(r0, r1);
+    lo = pack_bf16(r0 - bf16_lo(mid), r1 - bf16_hi(mid));
+}
+
+// A fragments (hi, mid, lo) of the state, as state_frags.
+__device__ __forceinline__ void state_frags3(const State& st, uint32_t (&ah)[2][2][4], uint32_t (&am)[2][2][4],
+                                             uint32_t (&al)[2][2][4])
+{
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int kt = 0; kt < 2; ++kt) {
+            split_pair3(st[mt][2 * kt][0], st[mt][2 * kt][1], ah[mt][kt][0], am[mt][kt][0], al[mt][kt][0]);
+            split_pair3(st[mt][2 * kt][2], st[mt][2 * kt][3], ah[mt][kt][1], am[mt][kt][1], al[mt][kt][1]);
+            split_pair3(st[mt][2 * kt + 1][0], st[mt][2 * kt + 1][1], ah[mt][kt][2], am[mt][kt][2], al[mt][kt][2]);
+            split_pair3(st[mt][2 * kt + 1][2], st[mt][2 * kt + 1][3], ah[mt][kt][3], am[mt][kt][3], al[mt][kt][3]);
+        }
+}
+
+// tri_product with the state in three terms (smallest first).
+template <bool LOWER>
+__device__ __forceinline__ void tri_product3(const uint32_t (&ah)[2][2][4], const uint32_t (&am)[2][2][4],
+                                             const uint32_t (&al)[2][2][4], const uint32_t (&bm)[2][4][2], int d,
+                                             State& acc)
+{
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            if (LOWER && 16 * kt + 15 <= 8 * nt) continue;
+            if (!LOWER && 16 * kt >= 8 * nt + 7) continue;
+            const bool first = kt == 0 || (LOWER ? 15 <= 8 * nt : 0 >= 8 * nt + 7);
+            const uint32_t b0 = tri_mask(bm[kt][nt][0], 16 * kt - 8 * nt, d, LOWER);
+            const uint32_t b1 = tri_mask(bm[kt][nt][1], 16 * kt + 8 - 8 * nt, d, LOWER);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                if (first) mma_bf16_first(acc[mt][nt], al[mt][kt], b0, b1);
+                else mma_bf16(acc[mt][nt], al[mt][kt], b0, b1);
+                mma_bf16(acc[mt][nt], am[mt][kt], b0, b1);
+                mma_bf16(acc[mt][nt], ah[mt][kt], b0, b1);
+            }
+        }
+}
+
 // M at this lane's accumulator positions, as fp32 pairs (row 16 mt + g + 8 h,
 // columns 8 nt + 2 q, + 1).
 __device__ __forceinline__ void load_m_d(const unsigned char* xs, int g, int q, float (&md)[2][4][4])
@@ -187,31 +264,56 @@ __device__ __forceinline__ void load_m_d(const unsigned char* xs, int g, int q, 
             }
 }
 
-// One token applied to the state.  split: state is Q = P - I (reduce pass)
-// and the factors' identity parts enter as the extra terms; otherwise the
-// state is the full product S (apply pass).
-template <bool SPLIT>
-__device__ __forceinline__ void apply_token(State& st, const unsigned char* xs, const float* Dv, const float* Dm1,
-                                            float a, int lane)
+// M^T at this lane's accumulator positions: element (16 mt + g + 8 h,
+// 8 nt + 2 q + s) of M^T is M[8 nt + 2 q + s][16 mt + g + 8 h].
+__device__ __forceinline__ void load_mt_d(const unsigned char* xs, int g, int q, float (&md)[2][4][4])
 {
-    const int g = lane >> 2, q = lane & 3, d = 2 * q - g;
-    uint32_t bm[2][4][2];
-    load_m_frags(xs, lane, bm);
-    float md[2][4][4];
-    load_m_d(xs, g, q, md);
-    uint32_t ah[2][2][4], al[2][2][4];
-    State acc;
-    // --- P L ---
-    state_frags(st, ah, al);
-    tri_product<true>(ah, al, bm, d, acc);
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int row = 16 * mt + g + 8 * (i >> 1), col = 8 * nt + 2 * q + (i & 1);
-                const float ls = (row > col) ? md[mt][nt][i] : 0.0f;
+                const int row = 8 * nt + 2 * q + (i & 1), col = 16 * mt + g + 8 * (i >> 1);
+                const uint16_t v = *reinterpret_cast<const uint16_t*>(xs + row * ROWB + col * 2);
+                md[mt][nt][i] = __uint_as_float((uint32_t)v << 16);
+            }
+}
+
+// One token applied to the state, from the factor fragments bm (M for
+// state X, M^T for state X^T = U^T D L^T: the lower mask then picks U_s^T,
+// the upper one L_s^T) and the same matrix at the accumulator positions md.
+// split: state is Q = P - I and the factors' identity parts enter as the
+// extra terms; otherwise the state is the full product.
+template <bool SPLIT, int TERMS = 2>
+__device__ __forceinline__ void apply_token_f(State& st, const uint32_t (&bm)[2][4][2], const float (&md)[2][4][4],
+                                              const float* Dv, const float* Dm1, float a, int lane)
+{
+    const int g = lane >> 2, q = lane & 3, d = 2 * q - g;
+    uint32_t ah[2][2][4], al[2][2][4];
+    State acc;
+    auto product = [&](auto lower_tag) {
+        constexpr bool LOWER = decltype(lower_tag)::value;
+        if constexpr (TERMS == 3) {
+            uint32_t am[2][2][4];
+            state_frags3(st, ah, am, al);
+            tri_product3<LOWER>(ah, am, al, bm, d, acc);
+        } else {
+            state_frags(st, ah, al);
+            tri_product<LOWER>(ah, al, bm, d, acc);
+        }
+    };
+    // --- P L ---
+    product(std::true_type{});
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                // 8 x 8 block (2 mt + i / 2, nt): below, above or on the diagonal
+                const int R = 2 * mt + (i >> 1), cs = 2 * q + (i & 1);
+                const float ls = R > nt ? md[mt][nt][i] : R < nt ? 0.0f : (g > cs ? md[mt][nt][i] : 0.0f);
                 st[mt][nt][i] += a * ((SPLIT ? ls : 0.0f) + acc[mt][nt][i]);
             }
     // --- (P L) D ---
@@ -223,25 +325,36 @@ __device__ __forceinline__ void apply_token(State& st, const unsigned char* xs, 
         for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int row = 16 * mt + g + 8 * (i >> 1), col = 8 * nt + 2 * q + (i & 1);
+                const int R = 2 * mt + (i >> 1), cs = 2 * q + (i & 1);
                 float v = st[mt][nt][i] * ((i & 1) ? dv.y : dv.x);
-                if (SPLIT && row == col) v += (i & 1) ? dm.y : dm.x;
+                if (SPLIT && R == nt && g == cs) v += (i & 1) ? dm.y : dm.x;
                 st[mt][nt][i] = v;
             }
     }
     // --- (P L D) U ---
-    state_frags(st, ah, al);
-    tri_product<false>(ah, al, bm, d, acc);
+    product(std::false_type{});
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int row = 16 * mt + g + 8 * (i >> 1), col = 8 * nt + 2 * q + (i & 1);
-                const float us = (row < col) ? md[mt][nt][i] : 0.0f;
+                const int R = 2 * mt + (i >> 1), cs = 2 * q + (i & 1);
+                const float us = R < nt ? md[mt][nt][i] : R > nt ? 0.0f : (g < cs ? md[mt][nt][i] : 0.0f);
                 st[mt][nt][i] += a * ((SPLIT ? us : 0.0f) + acc[mt][nt][i]);
             }
+}
+
+// One token applied to the state (forward: the state times X = L D U).
+template <bool SPLIT>
+__device__ __forceinline__ void apply_token(State& st, const unsigned char* xs, const float* Dv, const float* Dm1,
+                                            float a, int lane)
+{
+    uint32_t bm[2][4][2];
+    load_m_frags(xs, lane, bm);
+    float md[2][4][4];
+    load_m_d(xs, lane >> 2, lane & 3, md);
+    apply_token_f<SPLIT>(st, bm, md, Dv, Dm1, a, lane);
 }
 
 __device__ __forceinline__ void store_state(float* out, const State& st, int g, int q)
@@ -483,9 +596,486 @@ k32_apply(KParams p, const uint16_t* __restrict__ x, const float* __restrict__ R
     }
 }
 
+// ---- backward (vector-Jacobian product) on the tensor cores ----------------
+//
+// G_t = dL/dS_t (later states included): G_{t-1} = dS_{t-1} + G_t X_t^T and
+// dL/dX_t = S_{t-1}^T G_t (the chain rule of S_t = S_{t-1} X_t), chunked as
+// the n = 16 backward: a local pass per chunk [t0, t1) (the gradient at t0
+// with nothing entering from the right, and W - I with W = X_{t0+1} ...
+// X_{t1}), the generic fp64 right-to-left scan of the chunk gradients, and an
+// apply pass (G from the gradient entering from the right down to t0, dX_t,
+// the LDU chain rule).  Right products by X^T = U^T D L^T run as the
+// forward's factor steps with the fragments of M^T (apply_token_f); W is
+// carried as W^T so that its left multiplications become right ones.  The
+// tokens of a chunk stream in reverse order, one per stage: x_t (bf16), and
+// for the apply pass S_{t-1}, and dS_{t-1} (fp32, rows padded so that the
+// fragment reads are free of bank conflicts).
+//
+// dX = S^T G is a full product in split bf16 (S^T hi, lo times G hi, lo, the
+// lo lo term dropped), G's halves staged in shared memory for ldmatrix.trans.
+// Chain rule of X = L D U (L = I + a Ls, U = I + a Us, D_i = exp(d tanh M_ii)):
+//   dM_ij = a D_j (dX U^T)_ij      (i > j;  dX U^T = dX + a dX Us^T)
+//   dM_ij = a D_i (L^T dX)_ij      (i < j;  L^T dX = dX + a Ls^T dX)
+//   dM_ii = D_i d (1 - tanh^2 M_ii) (L^T dX U^T)_ii,
+//           (L^T dX U^T)_ii = (L^T dX)_ii + a sum_{k > i} (L^T dX)_ik M_ik.
+
+constexpr int SROW = 36;             // padded row stride (words) of a staged fp32 S_{t-1}
+constexpr int DROW = 40;             // padded row stride (words) of a staged fp32 dS_{t-1}
+constexpr int BLWARPS = 4;           // local pass: warps per CTA (2 CTAs per SM, 255 registers)
+constexpr int BAWARPS = 2;           // apply pass: warps per CTA (3 CTAs per SM)
+
+template <bool APPLY>
+struct BSmem32 {
+    unsigned char x[2][SLICEB];                      // x_t
+    float ds[2][N * DROW];                           // dS_{t-1}
+    float s[APPLY ? 2 : 1][APPLY ? N * SROW : 4];    // S_{t-1}
+    unsigned char stg[APPLY ? 3 : 1][APPLY ? SLICEB : 16];   // bf16 terms (hi, mid, lo) of a staged matrix
+    float dd[2][3][N];                               // per stage: D_i, D_i - 1, d (1 - tanh^2 M_ii)
+};
+
+// D_i, D_i - 1 and dD_i / dM_ii / D_i of one token (lane i: diagonal entry i).
+__device__ __forceinline__ void stage_dd_b(const KParams& p, const unsigned char* xs, float (&dd)[3][N], int lane)
+{
+    const uint16_t mb = *reinterpret_cast<const uint16_t*>(xs + lane * ROWB + lane * 2);
+    const float th = tanhf(__uint_as_float((uint32_t)mb << 16));
+    const float dm1 = expm1f(p.ldu_d * th);
+    dd[0][lane] = 1.0f + dm1;
+    dd[1][lane] = dm1;
+    dd[2][lane] = p.ldu_d * fmaf(-th, th, 1.0f);
+    __syncwarp();
+}
+
+// A 32 x 32 fp32 matrix in accumulator layout from rows `stride` words apart.
+__device__ __forceinline__ void load_state(State& st, const float* src, int stride, int g, int q)
+{
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float2 v = *reinterpret_cast<const float2*>(src + (16 * mt + g + 8 * h) * stride + 8 * nt + 2 * q);
+                st[mt][nt][2 * h] = v.x;
+                st[mt][nt][2 * h + 1] = v.y;
+            }
+}
+
+// st += the matrix at src (rows `stride` words apart).
+__device__ __forceinline__ void add_state(State& st, const float* src, int stride, int g, int q)
+{
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float2 v = *reinterpret_cast<const float2*>(src + (16 * mt + g + 8 * h) * stride + 8 * nt + 2 * q);
+                st[mt][nt][2 * h] += v.x;
+                st[mt][nt][2 * h + 1] += v.y;
+            }
+}
+
+// The producer side of a backward warp's pipeline: one token per stage, in
+// reverse order along the warp's chains.  Local pass: tokens t1 (when a
+// chunk follows) down to t0 + 1; apply pass: t1 (when a chunk follows, for
+// the gradient entering from the right) down to t0.
+template <bool APPLY>
+struct BFeed32 {
+    int64_t chain, stride, nchains, tok;
+    int64_t tau, lo, base;
+
+    __device__ __forceinline__ void set(const KParams& p)
+    {
+        if (chain >= nchains) return;
+        const Chain c = chain_at(p, chain);
+        base = (c.b * p.L * p.H + c.h) * NN;
+        tau = c.tend < p.L ? c.tend : c.tend - 1;
+        lo = APPLY ? c.tbeg : c.tbeg + 1;
+        if (tau < lo) {                      // nothing to stream for this chain
+            chain += stride;
+            set(p);
+        }
+    }
+    __device__ __forceinline__ void issue(BSmem32<APPLY>& sm, int slot, int lane, const KParams& p,
+                                          const uint16_t* x, const float* S_fwd, const float* dS)
+    {
+        if (chain < nchains) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {          // x_tau: 128 granules of 16 bytes
+                const int gi = lane + 32 * i, row = gi >> 2, c4 = gi & 3;
+                cp_async16(sm.x[slot] + row * ROWB + c4 * 16, x + base + tau * tok + row * N + c4 * 8);
+            }
+            if (tau >= 1) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {      // dS_{tau-1}, and S_{tau-1}: 256 granules each
+                    const int gi = lane + 32 * i, row = gi >> 3, c4 = gi & 7;
+                    cp_async16(sm.ds[slot] + row * DROW + 4 * c4, dS + base + (tau - 1) * tok + row * N + 4 * c4);
+                    if (APPLY)
+                        cp_async16(&sm.s[slot][0] + row * SROW + 4 * c4,
+                                   S_fwd + base + (tau - 1) * tok + row * N + 4 * c4);
+                }
+            }
+            if (--tau < lo) {
+                chain += stride;
+                set(p);
+            }
+        }
+        cp_async_commit();
+    }
+};
+
+// The chunk's chains are counted sequence-major by the chunk-gradient scan:
+// (b H + h) K + k.
+__device__ __forceinline__ int64_t seq_major(const KParams& p, const Chain& c)
+{
+    return (c.b * p.H + c.h) * p.K + c.k;
+}
+
+// Local pass: per chunk, G from dS_{t1-1} down to t0 (nothing entering from
+// the right) and W^T = (X_{t0+1} ... X_{t1})^T - I.
+__global__ void __launch_bounds__(BLWARPS * 32, 2)
+k32b_local(KParams p, const uint16_t* __restrict__ x, const float* __restrict__ dS, float* __restrict__ gloc,
+           float* __restrict__ Wq)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    BSmem32<false>& sm = reinterpret_cast<BSmem32<false>*>(smem_raw)[warp];
+    const int64_t nchains = p.B * p.H * p.K;
+    const int64_t first = (int64_t)blockIdx.x * BLWARPS + warp, stride = (int64_t)gridDim.x * BLWARPS;
+    const int64_t tok = p.H * NN;
+    const int g = lane >> 2, q = lane & 3;
+    BFeed32<false> feed;
+    feed.chain = first;
+    feed.stride = stride;
+    feed.nchains = nchains;
+    feed.tok = tok;
+    feed.set(p);
+    feed.issue(sm, 0, lane, p, x, nullptr, dS);
+    int cs = 0;
+    for (int64_t chain = first; chain < nchains; chain += stride) {
+        const Chain c = chain_at(p, chain);
+        const int64_t base = (c.b * p.L * p.H + c.h) * NN;
+        const bool more = c.tend < p.L;
+        State G, Wt;
+        load_state(G, dS + base + (c.tend - 1) * tok, N, g, q);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) Wt[mt][nt][i] = 0.0f;
+        const int64_t hi = more ? c.tend : c.tend - 1, lo = c.tbeg + 1;
+        for (int64_t tau = hi; tau >= lo; --tau) {
+            feed.issue(sm, cs ^ 1, lane, p, x, nullptr, dS);
+            cp_async_wait<1>();
+            __syncwarp();
+            const unsigned char* xs = sm.x[cs];
+            stage_dd_b(p, xs, sm.dd[cs], lane);
+            uint32_t bm[2][4][2];
+            load_mt_frags(xs, lane, bm);
+            float md[2][4][4];
+            load_mt_d(xs, g, q, md);
+            if (more) apply_token_f<true, 3>(Wt, bm, md, sm.dd[cs][0], sm.dd[cs][1], p.ldu_a, lane);   // W^T X^T
+            if (tau < c.tend) {                                     // G <- dS_{tau-1} + G X_tau^T
+                apply_token_f<false, 3>(G, bm, md, sm.dd[cs][0], sm.dd[cs][1], p.ldu_a, lane);
+                add_state(G, sm.ds[cs], DROW, g, q);
+            }
+            __syncwarp();
+            cs ^= 1;
+        }
+        const int64_t wchain = seq_major(p, c);
+        store_state(gloc + wchain * NN, G, g, q);
+        float* w = Wq + wchain * NN;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {                   // W = (W^T)^T
+                    const int row = 16 * mt + g + 8 * (i >> 1), col = 8 * nt + 2 * q + (i & 1);
+                    w[col * N + row] = more ? Wt[mt][nt][i] : 0.0f;
+                }
+    }
+}
+
+// The bf16 halves (A fragments from state_frags) of a matrix written row-major
+// into stg[0] (hi) and stg[1] (lo), rows padded to ROWB bytes.
+__device__ __forceinline__ void stage_frags(unsigned char (*stg)[SLICEB], const uint32_t (&ah)[2][2][4],
+                                            const uint32_t (&al)[2][2][4], int g, int q)
+{
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int row = 16 * mt + g + 8 * (i & 1), col = 16 * kt + 2 * q + 8 * (i >> 1);
+                *reinterpret_cast<uint32_t*>(stg[0] + row * ROWB + col * 2) = ah[mt][kt][i];
+                *reinterpret_cast<uint32_t*>(stg[1] + row * ROWB + col * 2) = al[mt][kt][i];
+            }
+}
+
+// The three bf16 terms of a matrix (A fragments from state_frags3) written
+// row-major into stg[0..2].
+__device__ __forceinline__ void stage_frags3(unsigned char (*stg)[SLICEB], const uint32_t (&ah)[2][2][4],
+                                             const uint32_t (&am)[2][2][4], const uint32_t (&al)[2][2][4], int g,
+                                             int q)
+{
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int row = 16 * mt + g + 8 * (i & 1), col = 16 * kt + 2 * q + 8 * (i >> 1);
+                *reinterpret_cast<uint32_t*>(stg[0] + row * ROWB + col * 2) = ah[mt][kt][i];
+                *reinterpret_cast<uint32_t*>(stg[1] + row * ROWB + col * 2) = am[mt][kt][i];
+                *reinterpret_cast<uint32_t*>(stg[2] + row * ROWB + col * 2) = al[mt][kt][i];
+            }
+}
+
+// dX = S^T G with both operands in three bf16 terms (S^T from S staged in
+// fp32, rows SROW words apart; G's terms staged in stg[0..2]): the six
+// products down to hi x lo and mid x mid, smallest first (the dropped ones
+// are below 2^-26 of |S| |G|).  dX is the sum of many products of growing
+// states and can be much smaller than |S| |G|, which is why the two-term
+// split is not enough here.  One row tile of dX at a time.
+__device__ __forceinline__ void st_times_g3(const float* sS, const unsigned char (*stg)[SLICEB], int lane, State& dX)
+{
+    const int g = lane >> 2, q = lane & 3;
+    const int r = lane & 15, cg = lane >> 4;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+        uint32_t sh[2][4], sm_[2][4], sl[2][4];
+#pragma unroll
+        for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int m = 16 * mt + g + 8 * (i & 1), k = 16 * kt + 2 * q + 8 * (i >> 1);
+                split_pair3(sS[k * SROW + m], sS[(k + 1) * SROW + m], sh[kt][i], sm_[kt][i], sl[kt][i]);
+            }
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {
+            uint32_t bh[2][4], bm_[2][4], bl[2][4];    // per k-tile: (b0, b1) of column tiles 2 np, 2 np + 1
+#pragma unroll
+            for (int kt = 0; kt < 2; ++kt) {
+                const int off = (16 * kt + r) * ROWB + (8 * (2 * np + cg)) * 2;
+                ldsm_x4_trans(bh[kt], stg[0] + off);
+                ldsm_x4_trans(bm_[kt], stg[1] + off);
+                ldsm_x4_trans(bl[kt], stg[2] + off);
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int nt = 2 * np + j;
+                float (&acc)[4] = dX[mt][nt];
+                mma_bf16_first(acc, sl[0], bh[0][2 * j], bh[0][2 * j + 1]);
+                mma_bf16(acc, sl[1], bh[1][2 * j], bh[1][2 * j + 1]);
+#pragma unroll
+                for (int kt = 0; kt < 2; ++kt) {
+                    mma_bf16(acc, sm_[kt], bm_[kt][2 * j], bm_[kt][2 * j + 1]);
+                    mma_bf16(acc, sh[kt], bl[kt][2 * j], bl[kt][2 * j + 1]);
+                }
+#pragma unroll
+                for (int kt = 0; kt < 2; ++kt) {
+                    mma_bf16(acc, sm_[kt], bh[kt][2 * j], bh[kt][2 * j + 1]);
+                    mma_bf16(acc, sh[kt], bm_[kt][2 * j], bm_[kt][2 * j + 1]);
+                }
+#pragma unroll
+                for (int kt = 0; kt < 2; ++kt) mma_bf16(acc, sh[kt], bh[kt][2 * j], bh[kt][2 * j + 1]);
+            }
+        }
+    }
+}
+
+// A fragments of Ls^T (A[m][k] = M[k][m] for k > m, else 0) by
+// ldmatrix.trans on M, for the tiles kt >= mt (the others are zero).
+__device__ __forceinline__ void load_lst_frags(const unsigned char* xs, int lane, uint32_t (&a)[2][2][4])
+{
+    const int g = lane >> 2, q = lane & 3, d = 2 * q - g;
+    const int r = lane & 7, mh = (lane >> 3) & 1, kh = lane >> 4;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int kt = 0; kt < 2; ++kt) {
+            if (kt < mt) continue;
+            uint32_t v[4];
+            ldsm_x4_trans(v, xs + (16 * kt + 8 * kh + r) * ROWB + (16 * mt + 8 * mh) * 2);
+            if (kt == mt) {
+                // element (m, k) = (16 mt + g + 8 (i & 1), 16 kt + 2 q + s + 8 (i >> 1)): k - m = off + d + s
+                v[0] = tri_mask(v[0], 0, d, true);
+                v[1] = 0u;                                     // k - m <= 7 - 8 < 0
+                v[3] = tri_mask(v[3], 0, d, true);             // v[2]: k - m >= 8 - 7 > 0, kept
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[mt][kt][i] = v[i];
+        }
+}
+
+// Apply pass: per chunk G from the gradient entering from the right (Gin)
+// down to t0, every dL/dx_t, and dL/dS0 from the first chunk.
+__global__ void __launch_bounds__(BAWARPS * 32, 3)
+k32b_apply(KParams p, const uint16_t* __restrict__ x, const float* __restrict__ S0, const float* __restrict__ S_fwd,
+           const float* __restrict__ dS, const float* __restrict__ Gin, float* __restrict__ dx,
+           float* __restrict__ dS0)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    BSmem32<true>& sm = reinterpret_cast<BSmem32<true>*>(smem_raw)[warp];
+    const int64_t nchains = p.B * p.H * p.K;
+    const int64_t first = (int64_t)blockIdx.x * BAWARPS + warp, stride = (int64_t)gridDim.x * BAWARPS;
+    const int64_t tok = p.H * NN;
+    const int g = lane >> 2, q = lane & 3, d = 2 * q - g;
+    const float a = p.ldu_a;
+    BFeed32<true> feed;
+    feed.chain = first;
+    feed.stride = stride;
+    feed.nchains = nchains;
+    feed.tok = tok;
+    feed.set(p);
+    feed.issue(sm, 0, lane, p, x, S_fwd, dS);
+    int cs = 0;
+    for (int64_t chain = first; chain < nchains; chain += stride) {
+        const Chain c = chain_at(p, chain);
+        const int64_t seq = c.b * p.H + c.h;
+        const int64_t base = (c.b * p.L * p.H + c.h) * NN;
+        const bool boundary = c.tend < p.L;
+        State G;
+        if (boundary) load_state(G, Gin + seq_major(p, c) * NN, N, g, q);
+        else load_state(G, dS + base + (c.tend - 1) * tok, N, g, q);
+        const int64_t hi = boundary ? c.tend : c.tend - 1, lo = c.tbeg;
+        for (int64_t tau = hi; tau >= lo; --tau) {
+            feed.issue(sm, cs ^ 1, lane, p, x, S_fwd, dS);
+            cp_async_wait<1>();
+            __syncwarp();
+            const unsigned char* xs = sm.x[cs];
+            stage_dd_b(p, xs, sm.dd[cs], lane);
+            const float* Dv = sm.dd[cs][0];
+            uint32_t bmt[2][4][2];
+            load_mt_frags(xs, lane, bmt);
+            float mdt[2][4][4];
+            load_mt_d(xs, g, q, mdt);
+            if (tau == c.tend) {                       // G_{t1-1} = dS_{t1-1} + Gin X_{t1}^T
+                apply_token_f<false, 3>(G, bmt, mdt, Dv, sm.dd[cs][1], a, lane);
+                add_state(G, sm.ds[cs], DROW, g, q);
+                __syncwarp();
+                cs ^= 1;
+                continue;
+            }
+            // ---- dX = S_{tau-1}^T G (S_{-1} = S0 or I) ----
+            State dX;
+            {
+                uint32_t gh[2][2][4], gm[2][2][4], gl[2][2][4];
+                state_frags3(G, gh, gm, gl);
+                stage_frags3(sm.stg, gh, gm, gl, g, q);
+            }
+            if (tau == 0 && S0) {                      // S0 into the (unused) S tile of this stage
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int gi = lane + 32 * i, row = gi >> 3, c4 = gi & 7;
+                    *reinterpret_cast<float4*>(&sm.s[cs][0] + row * SROW + 4 * c4) =
+                        *reinterpret_cast<const float4*>(S0 + seq * NN + row * N + 4 * c4);
+                }
+            }
+            __syncwarp();
+            if (tau >= 1 || S0) {
+                st_times_g3(&sm.s[cs][0], sm.stg, lane, dX);
+            } else {
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) dX[mt][nt][i] = G[mt][nt][i];
+            }
+            __syncwarp();                              // every lane done with the staged G
+            // ---- the LDU chain rule ----
+            // P1 = dX U^T = dX + a dX Us^T (lower mask on M^T), P2 = L^T dX = dX + a Ls^T dX
+            State acc1, acc2;
+            {
+                uint32_t dh[2][2][4], dl[2][2][4];
+                state_frags(dX, dh, dl);
+                tri_product<true>(dh, dl, bmt, d, acc1);
+                stage_frags(sm.stg, dh, dl, g, q);
+            }
+            __syncwarp();
+            {
+                uint32_t bdh[2][4][2], bdl[2][4][2];
+                load_m_frags(sm.stg[0], lane, bdh);
+                load_m_frags(sm.stg[1], lane, bdl);
+                uint32_t als[2][2][4];
+                load_lst_frags(xs, lane, als);
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt) {
+                        mma_bf16_first(acc2[mt][nt], als[mt][1], bdl[1][nt][0], bdl[1][nt][1]);
+                        if (mt == 0) mma_bf16(acc2[mt][nt], als[mt][0], bdl[0][nt][0], bdl[0][nt][1]);
+                        if (mt == 0) mma_bf16(acc2[mt][nt], als[mt][0], bdh[0][nt][0], bdh[0][nt][1]);
+                        mma_bf16(acc2[mt][nt], als[mt][1], bdh[1][nt][0], bdh[1][nt][1]);
+                    }
+            }
+            float md[2][4][4];
+            load_m_d(xs, g, q, md);
+            // row sums of (L^T dX)_ik M_ik over k > i, for this lane's rows (mt, h)
+            float rs[2][2];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float v = 0.0f;
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                        for (int s2 = 0; s2 < 2; ++s2) {
+                            const int i = 2 * h + s2, R = 2 * mt + h, cs2 = 2 * q + s2;
+                            const bool above = R < nt || (R == nt && cs2 > g);
+                            if (above) v = fmaf(fmaf(a, acc2[mt][nt][i], dX[mt][nt][i]), md[mt][nt][i], v);
+                        }
+                    v += __shfl_xor_sync(0xffffffffu, v, 1);
+                    v += __shfl_xor_sync(0xffffffffu, v, 2);
+                    rs[mt][h] = v;
+                }
+            float* out = dx + base + tau * tok;
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int row = 16 * mt + g + 8 * h, R = 2 * mt + h;
+                        const float dr = Dv[row];
+                        float o[2];
+#pragma unroll
+                        for (int s2 = 0; s2 < 2; ++s2) {
+                            const int i = 2 * h + s2, cs2 = 2 * q + s2, col = 8 * nt + cs2;
+                            const float p1 = fmaf(a, acc1[mt][nt][i], dX[mt][nt][i]);
+                            const float p2 = fmaf(a, acc2[mt][nt][i], dX[mt][nt][i]);
+                            const bool below = R > nt || (R == nt && g > cs2);
+                            const bool diag = R == nt && g == cs2;
+                            if (below) o[s2] = a * p1 * Dv[col];
+                            else if (diag) o[s2] = fmaf(a, rs[mt][h], p2) * dr * sm.dd[cs][2][row];
+                            else o[s2] = a * dr * p2;
+                        }
+                        *reinterpret_cast<float2*>(out + row * N + 8 * nt + 2 * q) = make_float2(o[0], o[1]);
+                    }
+            // ---- G_{tau-1} = dS_{tau-1} + G X_tau^T, or dS0 = G X_0^T at the first token ----
+            if (tau > lo || tau == 0) {
+                apply_token_f<false, 3>(G, bmt, mdt, Dv, sm.dd[cs][1], a, lane);
+                if (tau == 0) {
+                    if (dS0) store_state(dS0 + seq * NN, G, g, q);
+                } else {
+                    add_state(G, sm.ds[cs], DROW, g, q);
+                }
+            }
+            __syncwarp();
+            cs ^= 1;
+        }
+    }
+}
+
 // CTAs of a persistent launch: resident CTAs per SM times the SM count,
 // cached per device and kernel slot; no more than the chains need.
-std::atomic<int> g_resident[64][2];
+std::atomic<int> g_resident[64][4];
 
 cudaError_t persistent_grid(int slot, const void* kern, int64_t nchains, unsigned& grid)
 {
@@ -504,6 +1094,28 @@ cudaError_t persistent_grid(int slot, const void* kern, int64_t nchains, unsigne
         if (dev >= 0 && dev < 64) g_resident[dev][slot].store(res, std::memory_order_relaxed);
     }
     const int64_t need = (nchains + WARPS - 1) / WARPS;
+    grid = (unsigned)(need < res ? need : res);
+    return cudaSuccess;
+}
+
+// The same for a kernel with its own block shape (backward kernels).
+cudaError_t persistent_grid_w(int slot, const void* kern, int threads, size_t smem, int warps, int64_t nchains,
+                              unsigned& grid)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int res = (dev >= 0 && dev < 64) ? g_resident[dev][slot].load(std::memory_order_relaxed) : 0;
+    if (res <= 0) {
+        int sms = 0, per_sm = 0;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem)) != cudaSuccess)
+            return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+        res = sms * per_sm;
+        if (dev >= 0 && dev < 64) g_resident[dev][slot].store(res, std::memory_order_relaxed);
+    }
+    const int64_t need = (nchains + warps - 1) / warps;
     grid = (unsigned)(need < res ? need : res);
     return cudaSuccess;
 }
@@ -552,6 +1164,44 @@ cudaError_t launch_apply(const KParams& p, const void* x, const carry::Plan& pl,
                                         reinterpret_cast<const float*>(ws + pl.R[0]),
                                         reinterpret_cast<const double*>(ws + pl.E[1]), pl.G, S_out,
                                         direct ? S0 : nullptr, direct ? 1 : 0);
+    return cudaGetLastError();
+}
+
+bool supports_backward(const KParams& p)
+{
+    return p.n == N && p.src == SRC_EMBEDDING && p.x_dtype == MRU_BF16 && p.mode == MRU_MODE_LDU &&
+           (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_BF16X3) && p.chunk > 0;
+}
+
+cudaError_t launch_bwd_local(const KParams& p, const void* x, const float* dS, float* gloc, float* Wq,
+                             cudaStream_t s)
+{
+    const int64_t nchains = p.B * p.H * p.K;
+    if (nchains == 0) return cudaSuccess;
+    if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    const size_t sm = sizeof(BSmem32<false>) * BLWARPS;
+    cudaError_t e = cudaFuncSetAttribute(k32b_local, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    unsigned grid = 0;
+    if ((e = persistent_grid_w(2, (const void*)k32b_local, BLWARPS * 32, sm, BLWARPS, nchains, grid)) != cudaSuccess)
+        return e;
+    k32b_local<<<grid, BLWARPS * 32, sm, s>>>(p, reinterpret_cast<const uint16_t*>(x), dS, gloc, Wq);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_apply(const KParams& p, const void* x, const float* S0, const float* S_fwd, const float* dS,
+                             const float* Gin, float* dx, float* dS0, cudaStream_t s)
+{
+    const int64_t nchains = p.B * p.H * p.K;
+    if (nchains == 0) return cudaSuccess;
+    if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    const size_t sm = sizeof(BSmem32<true>) * BAWARPS;
+    cudaError_t e = cudaFuncSetAttribute(k32b_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    unsigned grid = 0;
+    if ((e = persistent_grid_w(3, (const void*)k32b_apply, BAWARPS * 32, sm, BAWARPS, nchains, grid)) != cudaSuccess)
+        return e;
+    k32b_apply<<<grid, BAWARPS * 32, sm, s>>>(p, reinterpret_cast<const uint16_t*>(x), S0, S_fwd, dS, Gin, dx, dS0);
     return cudaGetLastError();
 }
 

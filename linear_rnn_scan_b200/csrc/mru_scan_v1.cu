@@ -1297,6 +1297,19 @@ cudaError_t backward_n(const KParams& p, const void* src, const float* S0, const
         profile_mark(2, 1, s);
         return cudaGetLastError();
     }
+    if (N == 32 && n32::supports_backward(p)) {
+        // n = 32 LDU on the tensor cores; the chunk-gradient scan stays generic
+        profile_mark(0, 0, s);
+        if ((e = n32::launch_bwd_local(p, src, dS, gloc, Wq, s)) != cudaSuccess) return e;
+        profile_mark(0, 1, s);
+        profile_mark(1, 0, s);
+        k_bwd_carry<N><<<(unsigned)BH, kThreads, sm_carry, s>>>(p, gloc, Wq, Gin);
+        profile_mark(1, 1, s);
+        profile_mark(2, 0, s);
+        if ((e = n32::launch_bwd_apply(p, src, S0, S_fwd, dS, Gin, dx, dS0, s)) != cudaSuccess) return e;
+        profile_mark(2, 1, s);
+        return cudaGetLastError();
+    }
     if ((e = set_smem(k_bwd_local<N, Grp>, sm_local)) != cudaSuccess) return e;
     if ((e = set_smem(k_bwd_apply<N, Grp>, sm_apply)) != cudaSuccess) return e;
     profile_mark(0, 0, s);

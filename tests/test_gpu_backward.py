@@ -136,3 +136,56 @@ def test_backward_n16_inverse_regimes(alpha):
     e_dx = _rel(dx.reshape(w.B, w.L, w.H, 256), dx_o.reshape(w.B, w.L, w.H, 256), axis=-1)
     e_s0 = _rel(dS0.reshape(w.B, w.H, 256), dS0_o.reshape(w.B, w.H, 256), axis=-1)
     assert e_dx.max() <= TOL_BWD and e_s0.max() <= TOL_BWD, (e_dx.max(), np.median(e_dx), e_s0.max())
+
+
+@pytest.mark.parametrize("chunk", [1, 3, 8, 16])
+@pytest.mark.parametrize("with_s0", [False, True])
+def test_backward_n32_ldu_tensor_cores(chunk, with_s0):
+    """The n = 32 LDU backward on the tensor cores (bf16 embeddings): chunks
+    of 1, 3, 8 and 16 tokens over L = 45 (a ragged last chunk), with and
+    without S0 (then the first token's S_{-1} is I and no dS0 is asked)."""
+    t = torch()
+    n = 32
+    w = gen.Workload("b32", B=2, H=2, L=45, n=n, x_dtype="bf16", mode=gen.MODE_LDU, alpha=1.0, seed=620)
+    x = gen.make_x(w)
+    S0 = gen.make_S0(w, seed=621) if with_s0 else None
+    dS = np.random.default_rng(622 + chunk).standard_normal((w.B, w.L, w.H, n, n)).astype(np.float32)
+    p = mru.problem_from_workload(w, chunk=chunk)
+    xd = to_device_x(x)
+    S0d = None if S0 is None else t.from_numpy(np.ascontiguousarray(S0, np.float32)).cuda()
+    S = mru.scan_fused_t(p, xd, S0=S0d)
+    dx, dS0, ws = mru.scan_backward_t(p, xd, S, t.from_numpy(dS).cuda(), S0=S0d)
+    assert mru.last_device_status(ws.data_ptr(), t.cuda.current_stream().cuda_stream) == mru.OK
+    dx_o, dS0_o = oracle.backward(oracle_problem(w), x, dS.astype(np.float64),
+                                  S0=None if S0 is None else S0.astype(np.float64))
+    dx = dx.cpu().numpy().astype(np.float64)
+    e_dx = _rel(dx.reshape(w.B, w.L, w.H, n * n), dx_o.reshape(w.B, w.L, w.H, n * n), axis=-1)
+    assert e_dx.max() <= TOL_BWD, (e_dx.max(), np.median(e_dx))
+    if with_s0:
+        e_s0 = _rel(dS0.cpu().numpy().astype(np.float64).reshape(w.B, w.H, n * n), dS0_o.reshape(w.B, w.H, n * n),
+                    axis=-1)
+        assert e_s0.max() <= TOL_BWD, e_s0.max()
+
+
+def test_backward_n32_ldu_workload_sampled():
+    """The n = 32 LDU workload (B4 H16 L8192, bf16) end to end on the tensor
+    cores; the oracle recomputes two sequences."""
+    t = torch()
+    w = gen.WORKLOADS["n32_ldu_bf16_b4h16l8192"]
+    n = w.n
+    x = gen.make_x(w)
+    dS = np.random.default_rng(6).standard_normal((w.B, w.L, w.H, n, n)).astype(np.float32)
+    p = mru.problem_from_workload(w)
+    xd = to_device_x(x)
+    S = mru.scan_fused_t(p, xd)
+    dx, _, ws = mru.scan_backward_t(p, xd, S, t.from_numpy(dS).cuda())
+    assert mru.last_device_status(ws.data_ptr(), t.cuda.current_stream().cuda_stream) == mru.OK
+    dx = dx.cpu().numpy().astype(np.float64).reshape(w.B, w.L, w.H, n * n)
+    for b, h in [(0, 0), (3, 11)]:
+        w1 = gen.Workload("one", B=1, H=1, L=w.L, n=n, x_dtype=w.x_dtype, mode=w.mode, alpha=w.alpha,
+                          ldu_offdiag=w.ldu_offdiag, ldu_diag=w.ldu_diag, seed=0)
+        x1 = np.ascontiguousarray(x.reshape(w.B, w.L, w.H, n * n)[b:b + 1, :, h])
+        dS1 = dS[b:b + 1, :, h:h + 1].astype(np.float64)
+        dx_o, _ = oracle.backward(oracle_problem(w1), x1, dS1)
+        e = _rel(dx[b, :, h], dx_o.reshape(w.L, n * n), axis=-1)
+        assert e.max() <= TOL_BWD, (b, h, e.max(), np.median(e))
