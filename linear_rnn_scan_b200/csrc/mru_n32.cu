@@ -686,14 +686,12 @@ struct BFeed32 {
 
     __device__ __forceinline__ void set(const KParams& p)
     {
-        if (chain >= nchains) return;
-        const Chain c = chain_at(p, chain);
-        base = (c.b * p.L * p.H + c.h) * NN;
-        tau = c.tend < p.L ? c.tend : c.tend - 1;
-        lo = APPLY ? c.tbeg : c.tbeg + 1;
-        if (tau < lo) {                      // nothing to stream for this chain
-            chain += stride;
-            set(p);
+        for (; chain < nchains; chain += stride) {      // skips chains with nothing to stream
+            const Chain c = chain_at(p, chain);
+            base = (c.b * p.L * p.H + c.h) * NN;
+            tau = c.tend < p.L ? c.tend : c.tend - 1;
+            lo = APPLY ? c.tbeg : c.tbeg + 1;
+            if (tau >= lo) return;
         }
     }
     __device__ __forceinline__ void issue(BSmem32<APPLY>& sm, int slot, int lane, const KParams& p,
