@@ -162,7 +162,8 @@ def read_peaks():
                 "source": "fallback"}
 
 
-KERNEL_SOURCES = {"k16_": "mru_n16.cu", "k32_": "mru_n32.cu", "k64_": "mru_n64.cu",
+KERNEL_SOURCES = {"k16_": "mru_n16.cu", "k16b_": "mru_n16.cu", "k32_": "mru_n32.cu", "k32b_": "mru_n32.cu",
+                  "k64_": "mru_n64.cu",
                   "k_level": "mru_carry.cu", "k_top": "mru_carry.cu", "k_down": "mru_carry.cu"}
 
 

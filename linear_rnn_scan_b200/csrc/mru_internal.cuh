@@ -174,6 +174,9 @@ namespace n64 {
 bool supports(const KParams& p, bool readout);
 cudaError_t launch_chunk_readout(const KParams& p, const float* x, const float* u, int64_t snap_every,
                                  float* o_out, float* snaps, float* totals, uint32_t* status, cudaStream_t s);
+// o_t = C U + C V_t and the snapshots C + C Q_t from the chains' carries C.
+cudaError_t launch_fixup_readout(const KParams& p, const float* carry, const float* u, int64_t snap_every,
+                                 float* o_out, float* snaps, cudaStream_t s);
 }  // namespace n64
 
 // Launchers (mru_scan_v1.cu).

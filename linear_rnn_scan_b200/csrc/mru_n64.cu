@@ -473,6 +473,141 @@ k64_chunk_readout(KParams p, const float* __restrict__ x, const float* __restric
                 make_float2(Qd[nt][2 * h8], Qd[nt][2 * h8 + 1]);
 }
 
+// ---- fix-up of the readout on the tensor cores ------------------------------
+//
+// Per chain (one CTA of 4 warps, warp w owns rows 16 w .. 16 w + 15 of the
+// chain's carry C): o_t = C U + C V_t for every token of the chunk (V_t the
+// chunk kernel's local readout, written where o_t goes), as products of C
+// with blocks of the matrix [V_t0 .. V_t1-1] (64 rows, q columns per token)
+// staged in shared memory two blocks at a time; C U once per chain; and the
+// snapshots S_t = C + C Q_t.  tf32 mma.sync with fp32 accumulation, the
+// chunk kernel's arithmetic.
+
+constexpr int FX_COLS = 64;                      // columns of a staged block
+constexpr int FX_BUF = N * (N + 4);              // floats per staging buffer (fits a padded 64 x 64 Q_t too)
+
+// acc = C W for column tile nt of a staged block: C in A fragments ca (plain
+// contraction order), W column col at offset boff of the buffer, entries
+// `ld` words apart.
+__device__ __forceinline__ void fx_tile(const uint32_t (&ca)[8][4], const float* buf, int boff, int ld, int qq,
+                                        float (&acc)[4])
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = 0.0f;
+#pragma unroll
+    for (int kt = 0; kt < 8; ++kt)
+        mma_tf32(acc, ca[kt], to_tf32(buf[boff + (8 * kt + qq) * ld]), to_tf32(buf[boff + (8 * kt + qq + 4) * ld]));
+}
+
+__global__ void __launch_bounds__(THREADS, 4)
+k64_fixup(KParams p, const float* __restrict__ carry, const float* __restrict__ u, int64_t snap_every,
+          float* __restrict__ o_out, float* __restrict__ snaps)
+{
+    extern __shared__ __align__(16) float fsm[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, qq = lane & 3;
+    const int q = p.rq, nq = N * q;
+    const int tpb = FX_COLS / q > 0 ? FX_COLS / q : 1;      // tokens per staged block
+    const int TS = nq + 4;                                  // padded words per staged token
+    float* sCU = fsm + 2 * FX_BUF;                          // C U, [64][q]
+    const int64_t chain = blockIdx.x;
+    const int64_t k = chain % p.K, bh = chain / p.K;
+    const int64_t h = bh % p.H, b = bh / p.H;
+    const int64_t t0 = k * p.chunk;
+    const int64_t t1 = (t0 + p.chunk < p.L) ? t0 + p.chunk : p.L;
+    const int r0 = 16 * warp;
+    const float* C = carry + chain * NN;
+    uint32_t ca[8][4];
+#pragma unroll
+    for (int kt = 0; kt < 8; ++kt) {
+        ca[kt][0] = to_tf32(C[(r0 + g) * N + 8 * kt + qq]);
+        ca[kt][1] = to_tf32(C[(r0 + g + 8) * N + 8 * kt + qq]);
+        ca[kt][2] = to_tf32(C[(r0 + g) * N + 8 * kt + qq + 4]);
+        ca[kt][3] = to_tf32(C[(r0 + g + 8) * N + 8 * kt + qq + 4]);
+    }
+    auto issue = [&](float* dst, int64_t tb) {          // the block of tokens tb .. (cp.async)
+        const int ntok = (int)((t1 - tb < tpb) ? t1 - tb : tpb);
+        const int gran = nq / 4;                          // 16-byte granules a token
+        for (int i = tid; i < ntok * gran; i += THREADS) {
+            const int tt = i / gran, gg = i - tt * gran;
+            cp_async16(dst + tt * TS + 4 * gg, o_out + ((b * p.L + tb + tt) * p.H + h) * nq + 4 * gg);
+        }
+        asm volatile("cp.async.commit_group;\n" ::);
+    };
+    if (t0 < t1) issue(fsm + FX_BUF, t0);
+    // C U (U staged as one token of the block layout in the first buffer)
+    for (int e = tid; e < nq; e += THREADS) fsm[e] = u[h * p.u_hs + e];
+    __syncthreads();
+    for (int nt = 0; nt * 8 < q; ++nt) {
+        const int cb = 8 * nt + g;
+        float acc[4];
+        fx_tile(ca, fsm, cb < q ? cb : 0, q, qq, acc);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int row = r0 + g + 8 * (i >> 1), c = 8 * nt + 2 * qq + (i & 1);
+            if (c < q) sCU[row * q + c] = acc[i];
+        }
+    }
+    __syncthreads();
+    // the chunk's tokens, a block at a time: o = C U + C V
+    int cur = 1;
+    for (int64_t tb = t0; tb < t1; tb += tpb) {
+        const int64_t tn = tb + tpb;
+        if (tn < t1) issue(fsm + (cur ^ 1) * FX_BUF, tn);
+        else asm volatile("cp.async.commit_group;\n" ::);
+        asm volatile("cp.async.wait_group 1;\n" ::);
+        __syncthreads();
+        const float* w = fsm + cur * FX_BUF;
+        const int ncol = (int)((t1 - tb < tpb) ? t1 - tb : tpb) * q;
+        for (int nt = 0; nt * 8 < ncol; ++nt) {
+            const int cb = 8 * nt + g;
+            const int boff = cb < ncol ? (cb / q) * TS + cb % q : 0;
+            float acc[4];
+            fx_tile(ca, w, boff, q, qq, acc);
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2) {
+                const int col = 8 * nt + 2 * qq + s2;
+                if (col < ncol) {
+                    const int tt = col / q, c = col - tt * q;
+                    float* dst = o_out + ((b * p.L + tb + tt) * p.H + h) * nq;
+#pragma unroll
+                    for (int h8 = 0; h8 < 2; ++h8) {
+                        const int row = r0 + g + 8 * h8;
+                        dst[row * q + c] = sCU[row * q + c] + acc[2 * h8 + s2];
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        cur ^= 1;
+    }
+    // snapshots: S_t = C + C Q_t, Q_t staged with rows padded to N + 4 words
+    if (snap_every > 0) {
+        const int64_t first = ((t0 + snap_every) / snap_every) * snap_every;   // 1-based
+        for (int64_t t1b = first; t1b <= t1; t1b += snap_every) {
+            float* sp = snaps + ((b * (p.L / snap_every) + t1b / snap_every - 1) * p.H + h) * NN;
+            for (int e = tid; e < NN / 4; e += THREADS) {
+                const int row = e >> 4, c4 = e & 15;
+                *reinterpret_cast<float4*>(fsm + row * (N + 4) + 4 * c4) =
+                    *reinterpret_cast<const float4*>(sp + row * N + 4 * c4);
+            }
+            __syncthreads();
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                float acc[4];
+                fx_tile(ca, fsm, 8 * nt + g, N + 4, qq, acc);
+#pragma unroll
+                for (int h8 = 0; h8 < 2; ++h8) {
+                    const int row = r0 + g + 8 * h8, col = 8 * nt + 2 * qq;
+                    const float2 cv = *reinterpret_cast<const float2*>(C + row * N + col);
+                    *reinterpret_cast<float2*>(sp + row * N + col) =
+                        make_float2(cv.x + acc[2 * h8], cv.y + acc[2 * h8 + 1]);
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
 }  // namespace
 
 bool supports(const KParams& p, bool readout)
@@ -490,6 +625,18 @@ cudaError_t launch_chunk_readout(const KParams& p, const float* x, const float* 
     cudaError_t e = cudaFuncSetAttribute(k64_chunk_readout, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     k64_chunk_readout<<<(unsigned)chains, THREADS, sm, s>>>(p, x, u, snap_every, o_out, snaps, totals, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fixup_readout(const KParams& p, const float* carry, const float* u, int64_t snap_every,
+                                 float* o_out, float* snaps, cudaStream_t s)
+{
+    const int64_t chains = p.B * p.H * p.K;
+    if (chains == 0) return cudaSuccess;
+    const size_t sm = sizeof(float) * (2 * FX_BUF + N * p.rq);
+    cudaError_t e = cudaFuncSetAttribute(k64_fixup, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    k64_fixup<<<(unsigned)chains, THREADS, sm, s>>>(p, carry, u, snap_every, o_out, snaps);
     return cudaGetLastError();
 }
 

@@ -1397,7 +1397,11 @@ cudaError_t scan_n(const KParams& p, const void* src, const float* S0, const flo
     k_carry_final<N><<<(unsigned)chains, kThreads, sm_d, s>>>(p, local, gcarry, carry);
     profile_mark(3, 1, s);
     profile_mark(4, 0, s);
-    k_fixup<N><<<(unsigned)chains, kThreads, sm_fix, s>>>(p, carry, u, snap_every, S_out, o_out, snaps);
+    if (N == 64 && o_out != nullptr && n64::supports(p, true)) {
+        if ((e = n64::launch_fixup_readout(p, carry, u, snap_every, o_out, snaps, s)) != cudaSuccess) return e;
+    } else {
+        k_fixup<N><<<(unsigned)chains, kThreads, sm_fix, s>>>(p, carry, u, snap_every, S_out, o_out, snaps);
+    }
     profile_mark(4, 1, s);
     if (launches) *launches = 5;
     return cudaGetLastError();
@@ -1473,6 +1477,7 @@ const char* kernel_name(const KParams& p, bool readout, int i)
                                     "k_fixup"};
     if (i < 0 || i >= (p.K == 1 ? 1 : 5)) return "";
     if (i == 0 && n64::supports(p, readout)) return "k64_chunk_readout";
+    if (i == 4 && n64::supports(p, readout)) return "k64_fixup";
     return generic[i];
 }
 
