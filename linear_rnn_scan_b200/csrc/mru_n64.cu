@@ -4,23 +4,25 @@
 // One CTA of 4 warps per chain (b, h, chunk); warp w owns rows 16w..16w+15
 // of the 64 x 64 state Q = P - I, held in mma accumulator registers.  Per
 // token:
-//   * the slice is copied to shared memory (cp.async),
-//   * the determinant scale c = |det(I + alpha M)|^(-1/64) comes from an LU
-//     of E = alpha M in identity-split form (pivots 1 + delta_k), register
-//     blocked: thread (br, bc) owns rows 4br..4br+3, columns 8bc..8bc+7; the
-//     pivot row and column are exchanged through shared memory, one barrier
-//     per step; |det| = prod (1 + delta_k) in fp32, c - 1 by log1p and expm1.
-//     A pivot below 1/2 in magnitude sends the token to a partially pivoted
-//     LU in shared memory,
+//   * the slice arrives in one of two shared-memory buffers (cp.async; the
+//     next token's copy is in flight meanwhile),
+//   * the determinant scale c = |det(I + alpha M)|^(-1/64): from the trace
+//     series of log det (M2 = M M and M3 = M2 M on the tensor cores in bf16,
+//     traces and norms summed over the CTA, a remainder bound deciding), or
+//     where the bound does not certify it from an LU of E = alpha M in
+//     identity-split form (register blocked, one barrier per step), and
+//     far from the identity from a partially pivoted LU in shared memory,
 //   * Q_t = Q_{t-1} + (F_t + Q_{t-1} F_t) with F = c alpha M + (c - 1) I,
-//     the product on mma.sync m16n8k8 tf32 with fp32 accumulation (the
-//     workload's tf32 arithmetic; the identity split keeps the implicit 1 out
-//     of the tf32 operands); the contraction index is permuted so that the
-//     accumulator tile j is the A fragment of k-tile j,
+//     Q F formed as c alpha (Q M) + (c - 1) Q, the product on mma.sync
+//     m16n8k8 tf32 with fp32 accumulation (the workload's tf32 arithmetic;
+//     the identity split keeps the implicit 1 out of the tf32 operands); the
+//     contraction index is permuted so that the accumulator tile j is the A
+//     fragment of k-tile j,
 //   * V_t = Q_t U (the readout of the local prefix, U the head's q query
 //     columns) is written where o_t goes, and Q_t where a snapshot is due;
 //     the chunk total goes to the workspace.
-// The carry scan and the fix-up o_t = C U + C V_t are the generic kernels.
+// The carry scan is the generic one; the fix-up o_t = C U + C V_t (and the
+// snapshots C + C Q_t) is k64_fixup below, on the tensor cores.
 #include "mru_internal.cuh"
 
 namespace mru {
@@ -177,6 +179,33 @@ __device__ double logdet_pivoted(Smem& sm, float* W, float alpha, int add_identi
     return bad ? __longlong_as_double(0x7ff8000000000000ll) : ld;
 }
 
+// D += A B, m16n8k16, bf16 operands, fp32 accumulate (the determinant's series).
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// bf16 pair (lo_elem in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// bf16 B fragment of the raw slice M for k-tile kt (16 rows) and column
+// tile nt: b0 = M[16 kt + 2 q, + 1][8 nt + g], b1 the same 8 rows lower.
+__device__ __forceinline__ void frag_m16(const float* xs, int kt, int nt, int g, int q, uint32_t& b0, uint32_t& b1)
+{
+    const float* base = xs + (16 * kt + 2 * q) * ROWW + 8 * nt + g;
+    b0 = pack_bf16(base[0], base[ROWW]);
+    b1 = pack_bf16(base[8 * ROWW], base[9 * ROWW]);
+}
+
 // Copies a token's slice into a slice buffer (cp.async, committed as one group).
 __device__ __forceinline__ void issue_slice(float* xs, const float* src)
 {
@@ -266,19 +295,21 @@ k64_chunk_readout(KParams p, const float* __restrict__ x, const float* __restric
 #pragma unroll
                 for (int i = 0; i < 4; ++i) M2[nt][i] = 0.0f;
 #pragma unroll
-            for (int kt = 0; kt < 8; ++kt) {
+            for (int kt = 0; kt < 4; ++kt) {                // bf16 m16n8k16: 16 contraction rows a step
                 uint32_t am[4];
-                const float2 m0 = *reinterpret_cast<const float2*>(xs + (r0 + g) * ROWW + 8 * kt + 2 * q);
-                const float2 m1 = *reinterpret_cast<const float2*>(xs + (r0 + g + 8) * ROWW + 8 * kt + 2 * q);
-                am[0] = to_tf32(m0.x);
-                am[1] = to_tf32(m1.x);
-                am[2] = to_tf32(m0.y);
-                am[3] = to_tf32(m1.y);
+                const float2 m0 = *reinterpret_cast<const float2*>(xs + (r0 + g) * ROWW + 16 * kt + 2 * q);
+                const float2 m1 = *reinterpret_cast<const float2*>(xs + (r0 + g + 8) * ROWW + 16 * kt + 2 * q);
+                const float2 m2 = *reinterpret_cast<const float2*>(xs + (r0 + g) * ROWW + 16 * kt + 8 + 2 * q);
+                const float2 m3 = *reinterpret_cast<const float2*>(xs + (r0 + g + 8) * ROWW + 16 * kt + 8 + 2 * q);
+                am[0] = pack_bf16(m0.x, m0.y);
+                am[1] = pack_bf16(m1.x, m1.y);
+                am[2] = pack_bf16(m2.x, m2.y);
+                am[3] = pack_bf16(m3.x, m3.y);
 #pragma unroll
                 for (int nt = 0; nt < 8; ++nt) {
                     uint32_t b0, b1;
-                    frag_m(xs, kt, nt, g, q, b0, b1);
-                    mma_tf32(M2[nt], am, b0, b1);
+                    frag_m16(xs, kt, nt, g, q, b0, b1);
+                    mma_bf16(M2[nt], am, b0, b1);
                 }
             }
         }
@@ -291,13 +322,14 @@ k64_chunk_readout(KParams p, const float* __restrict__ x, const float* __restric
             if (series) {
                 // log det(I + E), E = alpha M, by its trace series
                 //   tr E - tr E^2 / 2 + tr E^3 / 3 - tr E^4 / 4 + R,
-                // tr E^k = <E^(k-1), E^T> from M2 = M M and M3 = M2 M (tf32
-                // products on the tensor cores).  Since tr E^k = <E^(k-3), (E^3)^T>
+                // tr E^k = <E^(k-1), E^T> from M2 = M M and M3 = M2 M (bf16
+                // products on the tensor cores, m16n8k16).  Since tr E^k = <E^(k-3), (E^3)^T>
                 // and |E^m|_F <= |E^2|_F |E|_F^(m-2),
                 //   |R| <= |E^3|_F |E^2|_F / (5 (1 - |E|_F))   (|E|_F < 1),
                 // the series is taken when that bound is at most 1e-6 (the scale
-                // c = exp(-log det / 64) then good to 1.6e-8; the tf32 rounding of
-                // M2 and M3 adds about 1e-8 to log det at the workload's alpha).
+                // c = exp(-log det / 64) then good to 1.6e-8; the bf16 rounding of
+                // the products' operands adds about 1e-7 to log det at the
+                // workload's alpha).
                 float tr1 = 0.0f, tr2 = 0.0f, tr3 = 0.0f, tr4 = 0.0f, n1 = 0.0f, n2 = 0.0f, n3 = 0.0f;
                 if (lane < 16) tr1 = xs[(r0 + lane) * ROWW + r0 + lane];
 #pragma unroll
@@ -321,17 +353,18 @@ k64_chunk_readout(KParams p, const float* __restrict__ x, const float* __restric
 #pragma unroll
                         for (int i = 0; i < 4; ++i) M3[j][i] = 0.0f;
 #pragma unroll
-                    for (int kt = 0; kt < 8; ++kt) {
+                    for (int kt = 0; kt < 4; ++kt) {
+                        // accumulator tiles 2 kt, 2 kt + 1 are the bf16 A fragment of k-tile kt
                         uint32_t a[4];
-                        a[0] = to_tf32(M2[kt][0]);
-                        a[1] = to_tf32(M2[kt][2]);
-                        a[2] = to_tf32(M2[kt][1]);
-                        a[3] = to_tf32(M2[kt][3]);
+                        a[0] = pack_bf16(M2[2 * kt][0], M2[2 * kt][1]);
+                        a[1] = pack_bf16(M2[2 * kt][2], M2[2 * kt][3]);
+                        a[2] = pack_bf16(M2[2 * kt + 1][0], M2[2 * kt + 1][1]);
+                        a[3] = pack_bf16(M2[2 * kt + 1][2], M2[2 * kt + 1][3]);
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             uint32_t b0, b1;
-                            frag_m(xs, kt, 4 * hh + j, g, q, b0, b1);
-                            mma_tf32(M3[j], a, b0, b1);
+                            frag_m16(xs, kt, 4 * hh + j, g, q, b0, b1);
+                            mma_bf16(M3[j], a, b0, b1);
                         }
                     }
 #pragma unroll

@@ -3,14 +3,14 @@ the tensor cores (no GPU; numpy restatements of the kernel's arithmetic).
 
 For X = I + E, E = alpha M, the kernel takes
     log det X = tr E - tr E^2 / 2 + tr E^3 / 3 - tr E^4 / 4 + R
-with tr E^k = <E^(k-1), E^T> from tf32 products M2 = M M, M3 = M2 M, and
+with tr E^k = <E^(k-1), E^T> from bf16 products M2 = M M, M3 = M2 M, and
 accepts it when the remainder bound
     |R| <= |E^3|_F |E^2|_F / (5 (1 - |E|_F))        (|E|_F < 1)
 is at most 1e-6; otherwise it factorises (LU).  These tests pin the series
 against numpy's slogdet, the bound against the true remainder, the
 acceptance at the benchmark's alpha, the rejection far from the identity,
 and the integer-operation tf32 rounding (round to nearest, ties away) the
-kernels use for the tensor-core operands."""
+kernels use for the chain's tensor-core operands."""
 import numpy as np
 
 N = 64
@@ -31,8 +31,15 @@ def tf32_reference(a):
     return (s * 2.0 ** e).astype(np.float32)
 
 
+def bf16_round(a):
+    """Round to bf16, nearest even (cvt.rn.bf16x2.f32)."""
+    b = np.asarray(a, np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000
+    return b.astype(np.uint32).view(np.float32)
+
+
 def series(M, alpha, rounded=True):
-    r = tf32_round if rounded else (lambda a: a)
+    r = bf16_round if rounded else (lambda a: a)
     M = M.astype(np.float64)
     M2 = r(M).astype(np.float64) @ r(M).astype(np.float64)
     M3 = r(M2).astype(np.float64) @ r(M).astype(np.float64)
@@ -67,7 +74,7 @@ def test_series_matches_slogdet_within_the_bound_exact_products():
             assert abs(ld - true) <= bound
 
 
-def test_series_accepted_at_benchmark_alpha_and_accurate_with_tf32_products():
+def test_series_accepted_at_benchmark_alpha_and_accurate_with_bf16_products():
     rng = np.random.default_rng(13)
     alpha = 0.03 / np.sqrt(N)
     for _ in range(60):
@@ -75,7 +82,7 @@ def test_series_accepted_at_benchmark_alpha_and_accurate_with_tf32_products():
         ld, bound = series(M, alpha)
         assert bound <= TAU
         true = np.linalg.slogdet(np.eye(N) + alpha * M.astype(np.float64))[1]
-        assert abs(ld - true) <= 1e-7        # c = exp(-ld / 64) good to 2e-9
+        assert abs(ld - true) <= 2e-7        # c = exp(-ld / 64) good to 3e-9
 
 
 def test_series_rejected_far_from_identity():
