@@ -622,12 +622,12 @@ k32_apply(KParams p, const uint16_t* __restrict__ x, const float* __restrict__ R
 constexpr int SROW = 36;             // padded row stride (words) of a staged fp32 S_{t-1}
 constexpr int DROW = 40;             // padded row stride (words) of a staged fp32 dS_{t-1}
 constexpr int BLWARPS = 4;           // local pass: warps per CTA (2 CTAs per SM, 255 registers)
-constexpr int BAWARPS = 2;           // apply pass: warps per CTA (3 CTAs per SM)
+constexpr int BAWARPS = 2;           // apply pass: warps per CTA (4 CTAs per SM)
 
 template <bool APPLY>
 struct BSmem32 {
     unsigned char x[2][SLICEB];                      // x_t
-    float ds[2][N * DROW];                           // dS_{t-1}
+    float ds[APPLY ? 1 : 2][N * DROW];               // dS_{t-1} (apply: one buffer, filled as its token starts)
     float s[APPLY ? 2 : 1][APPLY ? N * SROW : 4];    // S_{t-1}
     unsigned char stg[APPLY ? 3 : 1][APPLY ? SLICEB : 16];   // bf16 terms (hi, mid, lo) of a staged matrix
     float dd[2][3][N];                               // per stage: D_i, D_i - 1, d (1 - tanh^2 M_ii)
@@ -705,12 +705,13 @@ struct BFeed32 {
             }
             if (tau >= 1) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {      // dS_{tau-1}, and S_{tau-1}: 256 granules each
+                for (int i = 0; i < 8; ++i) {      // dS_{tau-1} (local pass) or S_{tau-1} (apply): 256 granules
                     const int gi = lane + 32 * i, row = gi >> 3, c4 = gi & 7;
-                    cp_async16(sm.ds[slot] + row * DROW + 4 * c4, dS + base + (tau - 1) * tok + row * N + 4 * c4);
                     if (APPLY)
                         cp_async16(&sm.s[slot][0] + row * SROW + 4 * c4,
                                    S_fwd + base + (tau - 1) * tok + row * N + 4 * c4);
+                    else
+                        cp_async16(sm.ds[slot] + row * DROW + 4 * c4, dS + base + (tau - 1) * tok + row * N + 4 * c4);
                 }
             }
             if (--tau < lo) {
@@ -911,7 +912,7 @@ __device__ __forceinline__ void load_lst_frags(const unsigned char* xs, int lane
 
 // Apply pass: per chunk G from the gradient entering from the right (Gin)
 // down to t0, every dL/dx_t, and dL/dS0 from the first chunk.
-__global__ void __launch_bounds__(BAWARPS * 32, 3)
+__global__ void __launch_bounds__(BAWARPS * 32, 4)
 k32b_apply(KParams p, const uint16_t* __restrict__ x, const float* __restrict__ S0, const float* __restrict__ S_fwd,
            const float* __restrict__ dS, const float* __restrict__ Gin, float* __restrict__ dx,
            float* __restrict__ dS0)
@@ -942,8 +943,16 @@ k32b_apply(KParams p, const uint16_t* __restrict__ x, const float* __restrict__ 
         else load_state(G, dS + base + (c.tend - 1) * tok, N, g, q);
         const int64_t hi = boundary ? c.tend : c.tend - 1, lo = c.tbeg;
         for (int64_t tau = hi; tau >= lo; --tau) {
+            if (tau >= 1) {                              // dS_{tau-1}, used at the end of this token
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int gi = lane + 32 * i, row = gi >> 3, c4 = gi & 7;
+                    cp_async16(sm.ds[0] + row * DROW + 4 * c4, dS + base + (tau - 1) * tok + row * N + 4 * c4);
+                }
+            }
+            cp_async_commit();
             feed.issue(sm, cs ^ 1, lane, p, x, S_fwd, dS);
-            cp_async_wait<1>();
+            cp_async_wait<2>();                          // this token's x and S (the next stage and dS may fly)
             __syncwarp();
             const unsigned char* xs = sm.x[cs];
             stage_dd_b(p, xs, sm.dd[cs], lane);
@@ -954,7 +963,9 @@ k32b_apply(KParams p, const uint16_t* __restrict__ x, const float* __restrict__ 
             load_mt_d(xs, g, q, mdt);
             if (tau == c.tend) {                       // G_{t1-1} = dS_{t1-1} + Gin X_{t1}^T
                 apply_token_f<false, 3>(G, bmt, mdt, Dv, sm.dd[cs][1], a, lane);
-                add_state(G, sm.ds[cs], DROW, g, q);
+                cp_async_wait<1>();                      // dS_{tau-1}
+                __syncwarp();
+                add_state(G, sm.ds[0], DROW, g, q);
                 __syncwarp();
                 cs ^= 1;
                 continue;
@@ -1062,7 +1073,9 @@ k32b_apply(KParams p, const uint16_t* __restrict__ x, const float* __restrict__ 
                 if (tau == 0) {
                     if (dS0) store_state(dS0 + seq * NN, G, g, q);
                 } else {
-                    add_state(G, sm.ds[cs], DROW, g, q);
+                    cp_async_wait<1>();                  // dS_{tau-1}
+                    __syncwarp();
+                    add_state(G, sm.ds[0], DROW, g, q);
                 }
             }
             __syncwarp();
