@@ -1047,7 +1047,7 @@ k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, 
 // round), the last with Z E^T in split tf32.  |E|_F^2 > 0.8 (far from the
 // identity): Gauss-Jordan elimination with partial pivoting on the lanes.
 
-constexpr int BST = 2, BNS = 3, BWARPS = 4;
+constexpr int BST = 2, BNS = 2, BWARPS = 4;
 
 template <bool Apply>
 struct BSmem {
@@ -1416,7 +1416,7 @@ k16b_local(KParams p, const float* __restrict__ x, const float* __restrict__ dS,
 
 // Apply pass: per chunk G from the gradient entering from the right (Gin)
 // down to t0, every dL/dx_t, and dL/dS0 from the first chunk.
-__global__ void __launch_bounds__(BWARPS * 32, 2)
+__global__ void __launch_bounds__(BWARPS * 32, 3)
 k16b_apply(KParams p, const float* __restrict__ x, const float* __restrict__ S0, const float* __restrict__ S_fwd,
            const float* __restrict__ dS, const float* __restrict__ Gin, float* __restrict__ dx,
            float* __restrict__ dS0, uint32_t* status)
