@@ -337,6 +337,76 @@ __device__ __forceinline__ void stage_scalars(const KParams& p, float2* cd, cons
     __syncwarp();
 }
 
+// F = X - I = 2 (I - A)^-1 A of the Cayley map X = (I - A)^-1 (I + A),
+// A = alpha (M - M^T) / 2, for the nt (<= ST) tokens of a stage, written over
+// the tokens' slices (same swizzled layout).  Gauss-Jordan elimination on
+// [I - A | 2A] (rows of 32 entries), 8 lanes per token (lane r: rows r and
+// r + 8), 4 tokens per round; no pivoting: the symmetric part of I - A is I,
+// and every Schur complement keeps a symmetric part of at least I, so each
+// pivot is at least 1.  The right half ends as F.
+template <int ST>
+__device__ __forceinline__ void stage_cayley(float alpha, float* xs, int nt, int lane)
+{
+    static_assert(ST % 4 == 0, "whole rounds of 4 tokens");
+    const int grp = lane >> 3, r = lane & 7;
+    const float ha = 0.5f * alpha;
+#pragma unroll 1
+    for (int rd = 0; rd < ST / 4; ++rd) {
+        const int tk = 4 * rd + grp;
+        float* ms = xs + (tk < nt ? tk : 0) * NN;       // idle groups eliminate token 0's copy, not stored
+        float w[2][2 * N];
+#pragma unroll
+        for (int lr = 0; lr < 2; ++lr) {
+            const int i = r + 8 * lr;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const float4 v = *reinterpret_cast<const float4*>(ms + swz(i, 4 * c4));
+                const float mv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 4 * c4 + e;
+                    const float a = ha * (mv[e] - ms[swz(j, i)]);
+                    w[lr][j] = (i == j ? 1.0f : 0.0f) - a;
+                    w[lr][N + j] = 2.0f * a;
+                }
+            }
+        }
+        __syncwarp();                                    // every read of M before any write of F
+#pragma unroll
+        for (int k = 0; k < N; ++k) {
+            const int kr = k / 8, owner = k % 8;
+            float prow[2 * N];
+#pragma unroll
+            for (int j = k; j < 2 * N; ++j) prow[j] = __shfl_sync(FULL, w[kr][j], owner, 8);
+            const float rk = 1.0f / prow[k];
+#pragma unroll
+            for (int lr = 0; lr < 2; ++lr) {
+                const int i = r + 8 * lr;
+                if (i == k) {
+#pragma unroll
+                    for (int j = k + 1; j < 2 * N; ++j) w[lr][j] = prow[j] * rk;
+                } else {
+                    const float l = w[lr][k] * rk;
+#pragma unroll
+                    for (int j = k + 1; j < 2 * N; ++j) w[lr][j] = fmaf(-l, prow[j], w[lr][j]);
+                }
+            }
+        }
+        if (tk < nt) {
+#pragma unroll
+            for (int lr = 0; lr < 2; ++lr) {
+                const int i = r + 8 * lr;
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4)
+                    *reinterpret_cast<float4*>(ms + swz(i, 4 * c4)) =
+                        make_float4(w[lr][N + 4 * c4], w[lr][N + 4 * c4 + 1], w[lr][N + 4 * c4 + 2],
+                                    w[lr][N + 4 * c4 + 3]);
+            }
+        }
+        __syncwarp();
+    }
+}
+
 // ---- the token chain (tf32 split, accumulator-resident state) -------------
 
 // B fragments (split) of F = ca M + dv I for one token, with the contraction
@@ -886,7 +956,7 @@ __device__ __forceinline__ void direct_carry(const float* in, bool has_s0, int l
 // runs on the uncorrected matrices and the carry kernel applies the
 // determinant correction of each total.  CTA 0 also zeroes the carry scan's
 // counters (the carry kernel runs after this launch).
-template <bool PerToken>
+template <bool PerToken, bool Cayley = false>
 __global__ void __launch_bounds__(RWARPS * 32, 2)
 k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, unsigned* ctr, int64_t nctr,
            uint32_t* status)
@@ -927,6 +997,11 @@ k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, u
             const int nt = (c.tend - t0 < RST) ? (int)(c.tend - t0) : RST;
             float ca = p.alpha, dv = p.add_identity ? 0.0f : -1.0f;
             if (PerToken) stage_scalars<RST>(p, sm.cd, xs, nt, lane, status);
+            if (Cayley) {                                  // F itself now sits where M was
+                stage_cayley<RST>(p.alpha, sm.stage[cs], nt, lane);
+                ca = 1.0f;
+                dv = 0.0f;
+            }
 #pragma unroll
             for (int j = 0; j < RST; ++j) {
                 if (j < nt) {
@@ -955,7 +1030,7 @@ k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, u
 // Apply pass: per chain the carry from the carry scan's factors, then
 // S_t = S_{t-1} + S_{t-1} F_t from S = carry, every S_t written, with the
 // per-token determinant scales factorised here.
-template <bool Direct>
+template <bool Direct, bool Cayley = false>
 __global__ void __launch_bounds__(AWARPS * 32, 3)
 k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, float* __restrict__ S_out,
           uint32_t* status, const float* __restrict__ S0)
@@ -999,7 +1074,13 @@ k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, 
             __syncwarp();
             const float* xs = sm.stage[cs];
             const int nt = (c.tend - t0 < AST) ? (int)(c.tend - t0) : AST;
-            stage_scalars<AST>(p, sm.cd, xs, nt, lane, status);
+            if (Cayley) {                                  // F itself now sits where M was
+                stage_cayley<AST>(p.alpha, sm.stage[cs], nt, lane);
+                if (lane < AST) sm.cd[lane] = make_float2(1.0f, 0.0f);
+                __syncwarp();
+            } else {
+                stage_scalars<AST>(p, sm.cd, xs, nt, lane, status);
+            }
 #pragma unroll
             for (int j = 0; j < AST; ++j) {
                 if (j < nt) {
@@ -1559,7 +1640,7 @@ k16b_apply(KParams p, const float* __restrict__ x, const float* __restrict__ S0,
 
 // CTAs of a persistent launch: resident CTAs per SM times the SM count,
 // cached per device and kernel slot; no more than the chains need.
-std::atomic<int> g_resident[64][6];
+std::atomic<int> g_resident[64][10];
 
 cudaError_t persistent_grid(int slot, const void* kern, int threads, size_t smem, int warps, int64_t nchains,
                             unsigned& grid)
@@ -1587,7 +1668,7 @@ cudaError_t persistent_grid(int slot, const void* kern, int threads, size_t smem
 bool supports(const KParams& p, bool readout)
 {
     return p.n == N && p.src == SRC_EMBEDDING && p.x_dtype == MRU_F32 && !readout &&
-           (p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM) &&
+           (p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM || p.mode == MRU_MODE_CAYLEY) &&
            (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32X3) && p.chunk > 0 && p.chunk % kSub == 0;
 }
 
@@ -1645,11 +1726,13 @@ cudaError_t launch_reduce(const KParams& p, const float* x, float* totals, const
     if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const size_t sm = sizeof(RSmem) * RWARPS;
     const bool per_token = p.mode == MRU_MODE_DETNORM && !p.add_identity;
-    auto kern = per_token ? k16_reduce<true> : k16_reduce<false>;
+    const bool cayley = p.mode == MRU_MODE_CAYLEY;
+    auto kern = cayley ? k16_reduce<false, true> : per_token ? k16_reduce<true> : k16_reduce<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     unsigned grid = 0;
-    if ((e = persistent_grid(per_token ? 1 : 0, (const void*)kern, RWARPS * 32, sm, RWARPS, nchains, grid)) !=
+    if ((e = persistent_grid(cayley ? 6 : per_token ? 1 : 0, (const void*)kern, RWARPS * 32, sm, RWARPS, nchains,
+                             grid)) !=
         cudaSuccess)
         return e;
     kern<<<grid, RWARPS * 32, sm, s>>>(p, x, totals, reinterpret_cast<unsigned*>(ws + cp.ctr_begin),
@@ -1715,11 +1798,14 @@ cudaError_t launch_apply(const KParams& p, const float* x, const CarryPlan& cp, 
     if (nchains == 0) return cudaSuccess;
     if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const size_t sm = sizeof(ASmem) * AWARPS;
-    auto kern = direct ? k16_apply<true> : k16_apply<false>;
+    const bool cayley = p.mode == MRU_MODE_CAYLEY;
+    auto kern = cayley ? (direct ? k16_apply<true, true> : k16_apply<false, true>)
+                       : (direct ? k16_apply<true> : k16_apply<false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     unsigned grid = 0;
-    if ((e = persistent_grid(direct ? 3 : 2, (const void*)kern, AWARPS * 32, sm, AWARPS, nchains, grid)) !=
+    if ((e = persistent_grid(cayley ? (direct ? 8 : 7) : (direct ? 3 : 2), (const void*)kern, AWARPS * 32, sm, AWARPS,
+                             nchains, grid)) !=
         cudaSuccess)
         return e;
     kern<<<grid, AWARPS * 32, sm, s>>>(p, x, cp, ws, S_out, status, direct ? S0 : nullptr);
