@@ -60,9 +60,20 @@ int32_t n64_chunk(int64_t token_heads)
     return c;
 }
 
+// n = 4 without a readout, up to 2^20 tokens in all: the whole sequence is
+// one chunk, run by the one-launch kernel (one CTA per sequence, up to 64
+// tokens per thread).  Larger problems keep the bandwidth-shaped passes.
+bool small_eligible(const mru_problem& p, int32_t src, bool readout)
+{
+    return p.n == 4 && !readout && p.L >= 1 && p.L <= 16384 && p.B * p.H * p.L <= (int64_t(1) << 20) &&
+           (src != SRC_EMBEDDING || p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM ||
+            p.mode == MRU_MODE_LDU);
+}
+
 int32_t choose_chunk(const mru_problem& p, int32_t src, bool readout)
 {
     if (p.chunk > 0) return p.chunk;
+    if (small_eligible(p, src, readout)) return (int32_t)p.L;
     if (src == SRC_EMBEDDING && fast64_eligible(p, readout)) return n64_chunk(p.B * p.H * p.L);
     if (src == SRC_EMBEDDING && fast32_eligible(p, readout)) return n32::preferred_chunk(p.B * p.H * p.L);
     if (src == SRC_EMBEDDING && fast16_eligible(p, readout))

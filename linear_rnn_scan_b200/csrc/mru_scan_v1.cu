@@ -1338,6 +1338,242 @@ cudaError_t build_states_n(const KParams& p, const void* x, float* X_out, int sm
     return cudaGetLastError();
 }
 
+// ---- small problems in one launch (n = 4, the whole sequence one chunk) ------
+//
+// One CTA per sequence; thread i takes the tokens [i T, (i + 1) T) with
+// T = ceil(L / 256), forms their product in registers (fp64), the CTA scans
+// the 256 products in fp64 (shuffles within each warp, then the eight warp
+// totals), and every thread re-runs its tokens in fp32 from its exclusive
+// carry S0 P_0 ... P_{i-1}, writing S_t.  The construction
+// follows cta_construct's arithmetic token by token in the thread.
+
+constexpr int SN = 4, SNN = SN * SN;
+
+// F = X - I of one token into F (fp32).  Returns false for a singular
+// determinant-corrected matrix (F is then 0: X = I, output unspecified).
+__device__ __forceinline__ bool small_construct(const KParams& p, const void* src, int64_t off, float (&F)[SNN])
+{
+    if (p.src != SRC_EMBEDDING) {
+        const float* f = reinterpret_cast<const float*>(src) + off;
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) F[e] = f[e] - ((p.src == SRC_X && e / SN == e % SN) ? 1.0f : 0.0f);
+        return true;
+    }
+    float M[SNN];
+#pragma unroll
+    for (int e = 0; e < SNN; ++e) M[e] = load_elem(src, off + e, p.x_dtype);
+    if (p.mode == MRU_MODE_RESHAPE) {
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) F[e] = p.alpha * M[e] - ((!p.add_identity && e / SN == e % SN) ? 1.0f : 0.0f);
+        return true;
+    }
+    if (p.mode == MRU_MODE_LDU) {
+        float D[SN], Dm1[SN];
+#pragma unroll
+        for (int k = 0; k < SN; ++k) {
+            const double z = (double)p.ldu_d * tanh((double)M[k * SN + k]);
+            D[k] = (float)exp(z);
+            Dm1[k] = (float)expm1(z);
+        }
+        const float a = p.ldu_a;
+#pragma unroll
+        for (int i = 0; i < SN; ++i)
+#pragma unroll
+            for (int j = 0; j < SN; ++j) {
+                const int m = i < j ? i : j;
+                float acc = 0.0f;
+#pragma unroll
+                for (int k = 0; k < m; ++k) acc = fmaf(a * M[i * SN + k] * D[k], a * M[k * SN + j], acc);
+                if (i < j) acc = fmaf(D[i], a * M[i * SN + j], acc);
+                else if (i > j) acc = fmaf(a * M[i * SN + j], D[j], acc);
+                else acc += Dm1[i];
+                F[i * SN + j] = acc;
+            }
+        return true;
+    }
+    // determinant-corrected: X = c Xr, c = |det Xr|^(-1/n)
+    double ld = 0.0;
+    bool pivot = !p.add_identity, singular = false;
+    if (p.add_identity) {                       // near the identity: eliminate E alone
+        float W[SNN];
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) W[e] = p.alpha * M[e];
+        double prod = 1.0;
+#pragma unroll
+        for (int k = 0; k < SN; ++k) {
+            const float d = W[k * SN + k];
+            if (!(fabsf(1.0f + d) >= 0.5f)) pivot = true;
+            prod *= 1.0 + (double)d;
+            const float r = 1.0f / (1.0f + d);
+#pragma unroll
+            for (int i = k + 1; i < SN; ++i)
+#pragma unroll
+                for (int j = k + 1; j < SN; ++j) W[i * SN + j] = fmaf(-W[i * SN + k] * r, W[k * SN + j], W[i * SN + j]);
+        }
+        ld = log(fabs(prod));
+    }
+    if (pivot) {                                // partial pivoting on Xr itself
+        float W[SNN];
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) W[e] = p.alpha * M[e] + ((p.add_identity && e / SN == e % SN) ? 1.0f : 0.0f);
+        ld = 0.0;
+#pragma unroll
+        for (int k = 0; k < SN; ++k) {
+            int piv = k;
+            float best = fabsf(W[k * SN + k]);
+#pragma unroll
+            for (int i = k + 1; i < SN; ++i)
+                if (fabsf(W[i * SN + k]) > best) { best = fabsf(W[i * SN + k]); piv = i; }
+            if (!(best > 0.0f)) singular = true;
+#pragma unroll
+            for (int i = k + 1; i < SN; ++i)   // swap rows k and piv (compile-time registers, selects)
+                if (i == piv)
+#pragma unroll
+                    for (int j = 0; j < SN; ++j) {
+                        const float tmp = W[k * SN + j];
+                        W[k * SN + j] = W[i * SN + j];
+                        W[i * SN + j] = tmp;
+                    }
+            const float pk = W[k * SN + k];
+            ld += log(fabs((double)pk));
+            const float r = pk != 0.0f ? 1.0f / pk : 0.0f;
+#pragma unroll
+            for (int i = k + 1; i < SN; ++i)
+#pragma unroll
+                for (int j = k + 1; j < SN; ++j) W[i * SN + j] = fmaf(-W[i * SN + k] * r, W[k * SN + j], W[i * SN + j]);
+        }
+    }
+    const double cm1 = expm1(-ld / SN);
+    float c = (float)(1.0 + cm1), cm1f = (float)cm1;
+    if (singular || !isfinite(ld) || !isfinite(c) || c == 0.0f) {
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) F[e] = 0.0f;
+        return false;
+    }
+#pragma unroll
+    for (int e = 0; e < SNN; ++e)
+        F[e] = c * (p.alpha * M[e]) + ((e / SN == e % SN) ? (p.add_identity ? cm1f : -1.0f) : 0.0f);
+    return true;
+}
+
+__device__ __forceinline__ void d4_mul(const double (&A)[SNN], const double (&B)[SNN], double (&C)[SNN])
+{
+#pragma unroll
+    for (int i = 0; i < SN; ++i)
+#pragma unroll
+        for (int j = 0; j < SN; ++j) {
+            double a = 0.0;
+#pragma unroll
+            for (int k = 0; k < SN; ++k) a = fma(A[i * SN + k], B[k * SN + j], a);
+            C[i * SN + j] = a;
+        }
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_small_scan(KParams p, const void* src, float* __restrict__ S_out, const float* __restrict__ S0, uint32_t* status)
+{
+    __shared__ double wtot[kThreads / 32][SNN];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t bh = blockIdx.x, h = bh % p.H, b = bh / p.H;
+    const int64_t T = (p.L + kThreads - 1) / kThreads;
+    const int64_t t0 = tid * T < p.L ? tid * T : p.L, t1 = t0 + T < p.L ? t0 + T : p.L;
+    bool bad = false;
+    // segment product in fp64, P <- P + P F, so that the carries hold little
+    // more than the rounding of each token's F (fp32 segment products gave
+    // 3.5x the worst-token error on rotated near-permutation chains)
+    double P[SNN];
+#pragma unroll
+    for (int e = 0; e < SNN; ++e) P[e] = (e / SN == e % SN) ? 1.0 : 0.0;
+    for (int64_t t = t0; t < t1; ++t) {
+        float F[SNN];
+        bad |= !small_construct(p, src, ((b * p.L + t) * p.H + h) * SNN, F);
+        double PF[SNN];
+#pragma unroll
+        for (int i = 0; i < SN; ++i)
+#pragma unroll
+            for (int j = 0; j < SN; ++j) {
+                double a = P[i * SN + j];
+#pragma unroll
+                for (int k = 0; k < SN; ++k) a = fma(P[i * SN + k], (double)F[k * SN + j], a);
+                PF[i * SN + j] = a;
+            }
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) P[e] = PF[e];
+    }
+    if (bad) atomicOr(status, STATUS_SINGULAR);
+    // inclusive scan of the segment products over the warp, fp64, in order
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        double O[SNN], R[SNN];
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) O[e] = __shfl_up_sync(0xffffffffu, P[e], d);
+        d4_mul(O, P, R);
+        if (lane >= d) {
+#pragma unroll
+            for (int e = 0; e < SNN; ++e) P[e] = R[e];
+        }
+    }
+    if (lane == 31) {
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) wtot[warp][e] = P[e];
+    }
+    __syncthreads();
+    // exclusive carry: S0 (or I), the earlier warps' totals, this warp's lanes before
+    double C[SNN], R[SNN];
+#pragma unroll
+    for (int e = 0; e < SNN; ++e) C[e] = S0 ? (double)S0[bh * SNN + e] : ((e / SN == e % SN) ? 1.0 : 0.0);
+    for (int w = 0; w < warp; ++w) {
+        double Wt[SNN];
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) Wt[e] = wtot[w][e];
+        d4_mul(C, Wt, R);
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) C[e] = R[e];
+    }
+    {
+        double O[SNN];
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) O[e] = __shfl_up_sync(0xffffffffu, P[e], 1);
+        if (lane > 0) {
+            d4_mul(C, O, R);
+#pragma unroll
+            for (int e = 0; e < SNN; ++e) C[e] = R[e];
+        }
+    }
+    // re-run from the carry: S <- S + S F, every S_t written
+    float S[SNN];
+#pragma unroll
+    for (int e = 0; e < SNN; ++e) S[e] = (float)C[e];
+    for (int64_t t = t0; t < t1; ++t) {
+        const int64_t row = ((b * p.L + t) * p.H + h) * SNN;
+        float F[SNN];
+        small_construct(p, src, row, F);
+        float SF[SNN];
+#pragma unroll
+        for (int i = 0; i < SN; ++i)
+#pragma unroll
+            for (int j = 0; j < SN; ++j) {
+                float a = 0.0f;
+#pragma unroll
+                for (int k = 0; k < SN; ++k) a = fmaf(S[i * SN + k], F[k * SN + j], a);
+                SF[i * SN + j] = a;
+            }
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) S[e] += SF[e];
+        float4* o = reinterpret_cast<float4*>(S_out + row);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) o[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+    }
+}
+
+// Whether a problem runs on k_small_scan (its chunk is the whole sequence).
+bool small_scan_ok(const KParams& p, bool readout)
+{
+    return p.n == SN && !readout && p.K == 1 &&
+           (p.src != SRC_EMBEDDING || p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM ||
+            p.mode == MRU_MODE_LDU);
+}
+
 template <int N>
 cudaError_t scan_n(const KParams& p, const void* src, const float* S0, const float* u, int64_t snap_every,
                    float* S_out, float* o_out, float* snaps, char* ws, const Workspace& W, cudaStream_t s,
@@ -1369,6 +1605,12 @@ cudaError_t scan_n(const KParams& p, const void* src, const float* S0, const flo
     if ((e = set_smem(k_carry_final<N>, sm_d)) != cudaSuccess) return e;
     if ((e = set_smem(k_fixup<N>, sm_fix)) != cudaSuccess) return e;
     profile_mark(0, 0, s);
+    if (N == SN && small_scan_ok(p, o_out != nullptr)) {
+        k_small_scan<<<(unsigned)BH, kThreads, 0, s>>>(p, src, S_out, S0, status);
+        profile_mark(0, 1, s);
+        if (launches) *launches = 1;
+        return cudaGetLastError();
+    }
     if (p.K == 1) {
         // one chunk per sequence: the chunk kernel starts from S0 and its
         // outputs are final (the decode / short-segment latency path)
@@ -1476,6 +1718,7 @@ const char* kernel_name(const KParams& p, bool readout, int i)
     static const char* generic[] = {"k_chunk_prefix", "k_carry_local", "k_carry_groups", "k_carry_final",
                                     "k_fixup"};
     if (i < 0 || i >= (p.K == 1 ? 1 : 5)) return "";
+    if (i == 0 && small_scan_ok(p, readout)) return "k_small_scan";
     if (i == 0 && n64::supports(p, readout)) return "k64_chunk_readout";
     if (i == 4 && n64::supports(p, readout)) return "k64_fixup";
     return generic[i];

@@ -139,6 +139,19 @@ def test_single_chunk_problems_take_one_launch(lib):
     assert mru.kernel_names(p, True)[0] == "k64_chunk_readout" and mru.launch_count(p, True) == 5
 
 
+def test_small_problems_choose_one_launch(lib):
+    """n = 4 without a readout, up to 2^20 tokens, automatic chunk: the whole
+    sequence is one chunk on the one-launch kernel; otherwise the passes."""
+    for p in (mru.problem(1, 1, 1024, 4), mru.problem(2, 3, 16384, 4, mode=mru.MODE_DETNORM, alpha=0.1),
+              mru.problem(64, 16, 1024, 4, x_dtype="bf16", mode=mru.MODE_LDU)):
+        assert mru.kernel_names(p) == ["k_small_scan"] and mru.chosen_chunk(p) == p.L
+    assert mru.kernel_names(mru.problem(1, 1, 1024, 4), True) == ["k_chunk_prefix", "k_carry_local",
+                                                                  "k_carry_groups", "k_carry_final", "k_fixup"]
+    for p in (mru.problem(1, 1, 16385, 4), mru.problem(128, 16, 1024, 4), mru.problem(1, 1, 1024, 8),
+              mru.problem(1, 1, 1024, 4, mode=mru.MODE_CAYLEY, alpha=0.1), mru.problem(1, 1, 1024, 4, chunk=16)):
+        assert "k_small_scan" not in mru.kernel_names(p)
+
+
 def test_host_entry_rejects_bad_arguments(lib):
     p = mru.problem(2, 2, 8, 16)
     nb = mru.workspace_size(p)

@@ -232,6 +232,70 @@ def test_n64_determinant_series_and_lu_tokens_mixed(chunk):
     assert e["o"]["max"] <= tol and e["snap"]["max"] <= tol, e
 
 
+def _near_permutation_x(w, seed, with_identity):
+    """Embeddings whose X~ = I + 0.03 N(0, 1), with the rows of every fifth
+    token rotated by one (a zero-ish diagonal: the construction must pivot);
+    with_identity=False stores X~ - I (for add_identity = 1).  Products stay
+    within fp32 range over thousands of tokens, unlike Gaussian X~."""
+    r = np.random.default_rng(seed)
+    n = w.n
+    X = np.eye(n) + 0.03 * r.standard_normal((w.B, w.L, w.H, n, n))
+    rot = np.arange(w.L) % 5 == 3
+    X[:, rot] = np.roll(X[:, rot], 1, axis=-2)
+    if not with_identity:
+        X -= np.eye(n)
+    x = X.astype(np.float32).reshape(w.B, w.L, w.H * n * n)
+    return gen.f32_to_bf16_bits(x) if w.x_dtype == "bf16" else x
+
+
+# (mode, add_identity, alpha, embeddings): Gaussian near the identity, or the
+# rotated near-permutations above for the pivoting constructions
+SMALL_CASES = [(gen.MODE_RESHAPE, 1, 0.05, "gauss"), (gen.MODE_RESHAPE, 0, 1.0, "perm"),
+               (gen.MODE_DETNORM, 1, 0.05, "gauss"), (gen.MODE_DETNORM, 0, 1.0, "perm"),
+               (gen.MODE_DETNORM, 1, 1.0, "perm"), (gen.MODE_LDU, 1, 0.05, "gauss")]
+
+
+@pytest.mark.parametrize("mode,add_id,alpha,emb", SMALL_CASES)
+@pytest.mark.parametrize("L", [1, 255, 257, 1000, 4099])
+@pytest.mark.parametrize("x_dtype,with_s0", [("f32", False), ("bf16", True)])
+def test_small_problems_one_launch(mode, add_id, alpha, emb, L, x_dtype, with_s0):
+    """n = 4 with the automatic chunk runs in one launch (each thread a
+    segment of tokens, the segment products scanned across the CTA): every
+    construction it takes (near-identity and pivoted determinant correction
+    included), segments that are full, partial and empty, with and without
+    S0, against the oracle over every token."""
+    w = small(4, mode, B=2, H=3, L=L, x_dtype=x_dtype, alpha=alpha, add_identity=add_id, seed=900 + L)
+    p = mru.problem_from_workload(w)
+    assert mru.launch_count(p) == 1 and mru.kernel_names(p) == ["k_small_scan"]
+    x = gen.make_x(w) if emb == "gauss" else _near_permutation_x(w, 902 + L, with_identity=not add_id)
+    S0 = gen.make_S0(w, seed=901) if with_s0 else None
+    S, st = run_fused(w, x, S0=S0)
+    assert st == mru.OK
+    e = compare_S(w, x, S, S0=S0)
+    assert e["count"] == w.B * w.L * w.H
+    assert e["max"] <= TOL_FP32, e
+
+
+def test_small_problems_singular_and_lifted_input():
+    """The one-launch path reports a singular determinant-corrected matrix
+    (the other heads stay within tolerance), and scans lifted matrices X
+    (mru_scan)."""
+    t = torch()
+    w = small(4, gen.MODE_DETNORM, B=1, H=2, L=300, alpha=1.0, add_identity=0, seed=950)
+    x = _near_permutation_x(w, 950, with_identity=True)
+    x[0, 123, 16:32] = 0.0                      # head 1, token 123: X~ = 0
+    S, st = run_fused(w, x)
+    assert st == mru.ERR_SINGULAR and np.isfinite(S).all()
+    assert compare_S(w, x, S, bh=[0])["max"] <= TOL_FP32
+    w = small(4, gen.MODE_LDU, B=2, H=2, L=700, seed=951)
+    x = gen.make_x(w)
+    for smi in (0, 1):
+        p = mru.problem_from_workload(w, store_minus_identity=smi)
+        assert mru.kernel_names(p) == ["k_small_scan"]
+        S = mru.scan_t(p, mru.build_states_t(p, to_device_x(x))).cpu().numpy()
+        assert compare_S(w, x, S)["max"] <= TOL_FP32
+
+
 @pytest.mark.parametrize("n", [4, 16, 32])
 @pytest.mark.parametrize("mode", MODES)
 def test_unfused_build_then_scan(n, mode):
