@@ -60,12 +60,15 @@ int32_t n64_chunk(int64_t token_heads)
     return c;
 }
 
-// n = 4 without a readout, up to 2^20 tokens in all: the whole sequence is
-// one chunk, run by the one-launch kernel (one CTA per sequence, up to 64
-// tokens per thread).  Larger problems keep the bandwidth-shaped passes.
+// n = 4 without a readout, sequences of up to 16384 tokens, and either at
+// most 2^20 tokens in all or at least one sequence per SM: the whole
+// sequence is one chunk, run by the one-launch kernel (one CTA per
+// sequence, up to 64 tokens per thread; 18x faster than the passes at
+// 1024 sequences of 1024 tokens).  Few long sequences keep the passes.
 bool small_eligible(const mru_problem& p, int32_t src, bool readout)
 {
-    return p.n == 4 && !readout && p.L >= 1 && p.L <= 16384 && p.B * p.H * p.L <= (int64_t(1) << 20) &&
+    return p.n == 4 && !readout && p.L >= 1 && p.L <= 16384 &&
+           (p.B * p.H * p.L <= (int64_t(1) << 20) || p.B * p.H >= 148) &&
            (src != SRC_EMBEDDING || p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM ||
             p.mode == MRU_MODE_LDU);
 }

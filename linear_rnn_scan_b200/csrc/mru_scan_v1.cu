@@ -1349,19 +1349,43 @@ cudaError_t build_states_n(const KParams& p, const void* x, float* X_out, int sm
 
 constexpr int SN = 4, SNN = SN * SN;
 
-// F = X - I of one token into F (fp32).  Returns false for a singular
-// determinant-corrected matrix (F is then 0: X = I, output unspecified).
-__device__ __forceinline__ bool small_construct(const KParams& p, const void* src, int64_t off, float (&F)[SNN])
+// The 16 values of one token (its embedding slice, or X or F for lifted
+// input) as fp32, in 16-byte loads: the boundary takes 16-byte aligned
+// buffers only and a token starts at a multiple of 16 elements.
+__device__ __forceinline__ void small_load(const KParams& p, const void* src, int64_t off, float (&M)[SNN])
+{
+    if (p.src == SRC_EMBEDDING && p.x_dtype == MRU_BF16) {
+        const uint4* q = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(src) + off);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const uint4 v = __ldg(q + r);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {      // element 2k in the low half of word k
+                M[8 * r + 2 * k] = __uint_as_float(w[k] << 16);
+                M[8 * r + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+            }
+        }
+        return;
+    }
+    const float4* q = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(src) + off);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const float4 v = __ldg(q + r);
+        M[4 * r] = v.x; M[4 * r + 1] = v.y; M[4 * r + 2] = v.z; M[4 * r + 3] = v.w;
+    }
+}
+
+// F = X - I of one token from its loaded values M.  Returns false for a
+// singular determinant-corrected matrix (F is then 0: X = I, output
+// unspecified).
+__device__ __forceinline__ bool small_construct(const KParams& p, const float (&M)[SNN], float (&F)[SNN])
 {
     if (p.src != SRC_EMBEDDING) {
-        const float* f = reinterpret_cast<const float*>(src) + off;
 #pragma unroll
-        for (int e = 0; e < SNN; ++e) F[e] = f[e] - ((p.src == SRC_X && e / SN == e % SN) ? 1.0f : 0.0f);
+        for (int e = 0; e < SNN; ++e) F[e] = M[e] - ((p.src == SRC_X && e / SN == e % SN) ? 1.0f : 0.0f);
         return true;
     }
-    float M[SNN];
-#pragma unroll
-    for (int e = 0; e < SNN; ++e) M[e] = load_elem(src, off + e, p.x_dtype);
     if (p.mode == MRU_MODE_RESHAPE) {
 #pragma unroll
         for (int e = 0; e < SNN; ++e) F[e] = p.alpha * M[e] - ((!p.add_identity && e / SN == e % SN) ? 1.0f : 0.0f);
@@ -1481,12 +1505,21 @@ k_small_scan(KParams p, const void* src, float* __restrict__ S_out, const float*
     // segment product in fp64, P <- P + P F, so that the carries hold little
     // more than the rounding of each token's F (fp32 segment products gave
     // 3.5x the worst-token error on rotated near-permutation chains)
+    // tokens are loaded two ahead of their use (ring of three)
+    const int64_t stride = p.H * SNN, base = (b * p.L * p.H + h) * SNN;
+    float M0[SNN] = {}, M1[SNN] = {};
+    if (t0 < t1) small_load(p, src, base + t0 * stride, M0);
+    if (t0 + 1 < t1) small_load(p, src, base + (t0 + 1) * stride, M1);
     double P[SNN];
 #pragma unroll
     for (int e = 0; e < SNN; ++e) P[e] = (e / SN == e % SN) ? 1.0 : 0.0;
     for (int64_t t = t0; t < t1; ++t) {
+        float M2[SNN] = {};
+        if (t + 2 < t1) small_load(p, src, base + (t + 2) * stride, M2);
         float F[SNN];
-        bad |= !small_construct(p, src, ((b * p.L + t) * p.H + h) * SNN, F);
+        bad |= !small_construct(p, M0, F);
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) { M0[e] = M1[e]; M1[e] = M2[e]; }
         double PF[SNN];
 #pragma unroll
         for (int i = 0; i < SN; ++i)
@@ -1544,10 +1577,16 @@ k_small_scan(KParams p, const void* src, float* __restrict__ S_out, const float*
     float S[SNN];
 #pragma unroll
     for (int e = 0; e < SNN; ++e) S[e] = (float)C[e];
+    if (t0 < t1) small_load(p, src, base + t0 * stride, M0);
+    if (t0 + 1 < t1) small_load(p, src, base + (t0 + 1) * stride, M1);
     for (int64_t t = t0; t < t1; ++t) {
-        const int64_t row = ((b * p.L + t) * p.H + h) * SNN;
+        const int64_t row = base + t * stride;
+        float M2[SNN] = {};
+        if (t + 2 < t1) small_load(p, src, base + (t + 2) * stride, M2);
         float F[SNN];
-        small_construct(p, src, row, F);
+        small_construct(p, M0, F);
+#pragma unroll
+        for (int e = 0; e < SNN; ++e) { M0[e] = M1[e]; M1[e] = M2[e]; }
         float SF[SNN];
 #pragma unroll
         for (int i = 0; i < SN; ++i)

@@ -140,14 +140,16 @@ def test_single_chunk_problems_take_one_launch(lib):
 
 
 def test_small_problems_choose_one_launch(lib):
-    """n = 4 without a readout, up to 2^20 tokens, automatic chunk: the whole
+    """n = 4 without a readout, automatic chunk, sequences of up to 16384
+    tokens and either up to 2^20 tokens or at least 148 sequences: the whole
     sequence is one chunk on the one-launch kernel; otherwise the passes."""
     for p in (mru.problem(1, 1, 1024, 4), mru.problem(2, 3, 16384, 4, mode=mru.MODE_DETNORM, alpha=0.1),
-              mru.problem(64, 16, 1024, 4, x_dtype="bf16", mode=mru.MODE_LDU)):
+              mru.problem(64, 16, 1024, 4, x_dtype="bf16", mode=mru.MODE_LDU), mru.problem(128, 16, 1024, 4),
+              mru.problem(148, 1, 16384, 4)):
         assert mru.kernel_names(p) == ["k_small_scan"] and mru.chosen_chunk(p) == p.L
     assert mru.kernel_names(mru.problem(1, 1, 1024, 4), True) == ["k_chunk_prefix", "k_carry_local",
                                                                   "k_carry_groups", "k_carry_final", "k_fixup"]
-    for p in (mru.problem(1, 1, 16385, 4), mru.problem(128, 16, 1024, 4), mru.problem(1, 1, 1024, 8),
+    for p in (mru.problem(1, 1, 16385, 4), mru.problem(147, 1, 16384, 4), mru.problem(1, 1, 1024, 8),
               mru.problem(1, 1, 1024, 4, mode=mru.MODE_CAYLEY, alpha=0.1), mru.problem(1, 1, 1024, 4, chunk=16)):
         assert "k_small_scan" not in mru.kernel_names(p)
 
