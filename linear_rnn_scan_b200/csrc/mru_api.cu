@@ -67,7 +67,7 @@ int32_t n64_chunk(int64_t token_heads)
 // 1024 sequences of 1024 tokens).  Few long sequences keep the passes.
 bool small_eligible(const mru_problem& p, int32_t src, bool readout)
 {
-    return p.n == 4 && !readout && p.L >= 1 && p.L <= 16384 &&
+    return p.n == 4 && !readout && p.L >= 1 && p.L <= 16384 && p.B * p.H < (int64_t(1) << 31) &&
            (p.B * p.H * p.L <= (int64_t(1) << 20) || p.B * p.H >= 148) &&
            (src != SRC_EMBEDDING || p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM ||
             p.mode == MRU_MODE_LDU);
