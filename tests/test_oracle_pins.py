@@ -55,6 +55,9 @@ class COracle:
     def lift(self, P, x, b, t, h):
         return self.m.lift(self._p(P), x, b, t, h)
 
+    def readout(self, P, x, U, every=0):
+        return self.m.readout(self._p(P), x, U, every)
+
 
 class NumpyTwin:
     """Independent numpy restatement of the definition; ``mistake`` plants one
@@ -133,11 +136,28 @@ class NumpyTwin:
                     out[b, t, h] = S
         return out
 
+    def readout(self, P, x, U, every=0):
+        """o_t = S_t U (U [n, q] shared or [H, n, q] per head) and the
+        snapshots S_t at 1-based t = every, 2 every, ..."""
+        S = self.scan(P, x)
+        H, L = P["H"], P["L"]
+        U = np.asarray(U, np.float64)
+        Uh = [U] * H if U.ndim == 2 else [U[h] for h in range(H)]
+        if self.mistake == "readout_head_shift":
+            Uh = [Uh[(h + 1) % H] for h in range(H)]
+        St = np.swapaxes(S, -1, -2) if self.mistake == "readout_transposed_state" else S
+        o = np.stack([St[:, :, h] @ Uh[h] for h in range(H)], axis=2)
+        snaps = None
+        if every > 0:
+            first = 0 if self.mistake == "snapshot_zero_based" else every - 1
+            snaps = S[:, first::every][:, :L // every]
+        return o, snaps
+
 
 MISTAKES = ["left_multiply", "column_major_reshape", "drop_identity", "det_exponent_sign",
             "det_power_not_root", "ldu_swap_triangles", "ldu_diag_no_tanh", "ldu_order_udl",
             "exclusive_output", "skew_sign", "skew_no_half", "skew_from_upper", "cayley_swapped",
-            "expm_first_order"]
+            "expm_first_order", "readout_transposed_state", "readout_head_shift", "snapshot_zero_based"]
 
 
 # ------------------------------------------------------------------- pins ---
@@ -429,10 +449,77 @@ def pin_orthogonal_modes(o):
                 assert np.abs(S[t].T @ S[t] - np.eye(n)).max() < 1e-12, (mode, t)
 
 
+# ------------------------------------------------------------ readout pins ---
+# The pages leave the reduction of S_t open; the reading taken is o_t = S_t U
+# with q query columns (one U for every head, or one per head) and full
+# snapshots of S_t at the 1-based steps t = every, 2 every, ...  These pins
+# check an oracle's ``readout(P, x, U, every)`` against integer products
+# computed exactly with Python ints.
+
+def _shear_chains(H, L, n, seed):
+    """Per-head chains of unipotent integer shears (upper and lower mixed)
+    and their exact prefix products as nested Python-int lists."""
+    r = _rng(seed)
+    x = np.zeros((1, L, H * n * n), np.float32)
+    prefix = []
+    for h in range(H):
+        cur = [[int(i == j) for j in range(n)] for i in range(n)]
+        seq = []
+        for t in range(L):
+            A = np.eye(n, dtype=np.int64)
+            k = np.triu_indices(n, 1) if (t + h) % 2 == 0 else np.tril_indices(n, -1)
+            A[k] = r.integers(-2, 3, size=len(k[0]))
+            x[0, t, h * n * n:(h + 1) * n * n] = A.astype(np.float32).ravel()
+            X = A.tolist()
+            cur = [[sum(cur[i][m] * X[m][j] for m in range(n)) for j in range(n)] for i in range(n)]
+            seq.append(cur)
+        prefix.append(seq)
+    return x, prefix
+
+
+def _int_matmul(A, Bm):
+    return [[sum(A[i][m] * Bm[m][j] for m in range(len(Bm))) for j in range(len(Bm[0]))] for i in range(len(A))]
+
+
+def pin_readout_exact_integer(o):
+    """Integer shear chains read out through integer query columns: o_t = S_t U
+    entry for entry, exactly, with one U for every head and with one U per
+    head (each head reads its own)."""
+    n, L, H, q = 4, 9, 3, 2
+    x, prefix = _shear_chains(H, L, n, 31)
+    P = params(1, H, L, n, alpha=1.0, add_identity=0)
+    r = _rng(32)
+    U_shared = r.integers(-3, 4, size=(n, q))
+    U_head = r.integers(-3, 4, size=(H, n, q))
+    for U, per_head in ((U_shared, False), (U_head, True)):
+        out, _ = o.readout(P, x, U.astype(np.float64), 0)
+        out = np.asarray(out).reshape(1, L, H, n, q)
+        for h in range(H):
+            Uh = (U_head[h] if per_head else U_shared).tolist()
+            for t in range(L):
+                ref = _int_matmul(prefix[h][t], Uh)
+                assert max(abs(v) for row in ref for v in row) < 2 ** 53
+                assert np.array_equal(out[0, t, h], np.array(ref, np.float64)), (per_head, h, t)
+
+
+def pin_snapshots_one_based(o):
+    """Snapshots are S_t at 1-based t = every, 2 every, ... (floor(L / every)
+    of them), compared with the exact integer prefix products."""
+    n, L, H, every = 4, 10, 2, 3
+    x, prefix = _shear_chains(H, L, n, 33)
+    P = params(1, H, L, n, alpha=1.0, add_identity=0)
+    _, snaps = o.readout(P, x, np.eye(n)[:, :1], every)
+    snaps = np.asarray(snaps).reshape(1, L // every, H, n, n)
+    for k in range(L // every):
+        for h in range(H):
+            assert np.array_equal(snaps[0, k, h], np.array(prefix[h][(k + 1) * every - 1], np.float64)), (k, h)
+
+
 PINS = [pin_identity_inputs, pin_diagonal_reshape, pin_diagonal_detnorm, pin_permutations_exact,
         pin_integer_shears_exact, pin_bruteforce_exact, pin_detnorm_unit_det,
         pin_detnorm_product_det, pin_ldu_factors, pin_initial_state_and_resume,
-        pin_orthogonal_2x2_closed_forms, pin_orthogonal_modes]
+        pin_orthogonal_2x2_closed_forms, pin_orthogonal_modes, pin_readout_exact_integer,
+        pin_snapshots_one_based]
 
 
 # ------------------------------------------------------------------ tests ---
