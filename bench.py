@@ -118,13 +118,17 @@ def kernel_bytes(name: str, w: gen.Workload, chunk: int) -> int:
     the fix-up reads Q_t and writes S_t.  Two-pass paths: the reduce pass
     reads the embeddings and writes the chunk totals; the apply pass reads
     the embeddings and each chain's carry factors and writes S_t; the carry
-    kernels touch only chunk totals, in-group prefixes and carries."""
+    kernels touch only chunk totals, in-group prefixes and carries.  The
+    one-launch small kernel reads the embeddings and writes S_t (its second
+    pass over a sequence's embeddings is meant to hit L2)."""
     nn = w.n * w.n
     sb = step_bytes(w)
     K = -(-w.L // chunk)
     chains = w.B * w.H * K
     tot = chains * nn                       # elements of all chunk totals
     groups = -(-chains // 16)
+    if name == "k_small_scan":
+        return sb["in"] + sb["out"]
     if "chunk" in name:
         return sb["in"] + sb["out"] + tot * 4
     if "fixup" in name:

@@ -67,3 +67,22 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
     args = bench.argparse.Namespace(gpus=2, steps=1, warmup=3, impl="reference")
     assert bench.run_reference(args, bench.gen.WORKLOADS[bench.DEFAULT_WORKLOAD]) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_every_forward_kernel_has_own_bytes():
+    """Each kernel the library names for a workload's forward step has a
+    byte count of its own design (the roofline's per-kernel figure), at the
+    workloads' sizes and at small sizes that take other paths."""
+    from linear_rnn_scan_b200 import inputs as gen
+    from linear_rnn_scan_b200 import mru
+    mru.load()
+    ws = list(gen.WORKLOADS.values())
+    ws += [w.with_(L=1) for w in ws] + [w.with_(n=8) for w in ws if w.n == 4]
+    for w in ws:
+        for ro in ((False, True) if w.readout else (False,)):
+            p = mru.problem_from_workload(w)
+            chunk = mru.chosen_chunk(p, readout=ro)
+            names = mru.kernel_names(p, ro)
+            assert names, w.name
+            for k in names:
+                assert bench.kernel_bytes(k, w, chunk) > 0, (w.name, k)
