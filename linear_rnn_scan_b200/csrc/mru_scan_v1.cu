@@ -1502,14 +1502,14 @@ k_small_scan(KParams p, const void* src, float* __restrict__ S_out, const float*
     const int64_t T = (p.L + kThreads - 1) / kThreads;
     const int64_t t0 = tid * T < p.L ? tid * T : p.L, t1 = t0 + T < p.L ? t0 + T : p.L;
     bool bad = false;
-    // segment product in fp64, P <- P + P F, so that the carries hold little
-    // more than the rounding of each token's F (fp32 segment products gave
-    // 3.5x the worst-token error on rotated near-permutation chains)
     // tokens are loaded two ahead of their use (ring of three)
     const int64_t stride = p.H * SNN, base = (b * p.L * p.H + h) * SNN;
     float M0[SNN] = {}, M1[SNN] = {};
     if (t0 < t1) small_load(p, src, base + t0 * stride, M0);
     if (t0 + 1 < t1) small_load(p, src, base + (t0 + 1) * stride, M1);
+    // segment product in fp64, P <- P + P F, so that the carries hold little
+    // more than the rounding of each token's F (fp32 segment products gave
+    // 3.5x the worst-token error on rotated near-permutation chains)
     double P[SNN];
 #pragma unroll
     for (int e = 0; e < SNN; ++e) P[e] = (e / SN == e % SN) ? 1.0 : 0.0;
