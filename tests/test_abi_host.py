@@ -174,3 +174,44 @@ def test_host_entry_rejects_bad_arguments(lib):
         mru.ERR_INVALID_ARG
     assert mru.scan_fused_host(p, fake, None, None, 2 * fake, None, 3 * fake, 4 * fake, 5 * fake, 255) == \
         mru.ERR_WORKSPACE
+
+
+def test_plain_c_program_uses_the_library(lib, tmp_path):
+    """A C99 program that includes only include/mru.h and links libmru.so
+    sizes a workspace, picks the chunk and reads status strings, agreeing
+    with the Python binding: the boundary needs no C++ and no torch."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not found")
+    src = tmp_path / "use_mru.c"
+    src.write_text(r'''
+#include "mru.h"
+#include <stdio.h>
+int main(void) {
+    mru_problem p = {0};
+    p.B = 8; p.H = 8; p.L = 4096; p.n = 16;
+    p.x_dtype = MRU_F32; p.mode = MRU_MODE_DETNORM; p.math = MRU_MATH_AUTO;
+    p.alpha = 0.0125f; p.add_identity = 1;
+    printf("%zu %d %s\n", mru_workspace_size(&p), (int)mru_chosen_chunk(&p, 0),
+           mru_status_string(MRU_ERR_WORKSPACE));
+    p.n = 12;
+    printf("%zu\n", mru_workspace_size(&p));
+    return 0;
+}
+''')
+    libdir = os.path.dirname(mru.LIB_PATH)
+    exe = tmp_path / "use_mru"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                        str(src), "-o", str(exe), "-L", libdir, "-l:" + os.path.basename(mru.LIB_PATH),
+                        "-Wl,-rpath," + libdir], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    first, second = out.stdout.strip().splitlines()
+    ws, chunk, msg = first.split(" ", 2)
+    p = mru.problem(8, 8, 4096, 16, mode=mru.MODE_DETNORM, alpha=0.0125)
+    assert int(ws) == mru.workspace_size(p) and int(chunk) == mru.chosen_chunk(p)
+    assert msg == mru.status_string(mru.ERR_WORKSPACE)
+    assert second == "0"
