@@ -86,3 +86,20 @@ def test_every_forward_kernel_has_own_bytes():
             assert names, w.name
             for k in names:
                 assert bench.kernel_bytes(k, w, chunk) > 0, (w.name, k)
+
+
+def test_algorithmic_bytes_per_unit():
+    """The roofline's per-unit bytes (embeddings in, results out): n16 fp32
+    2,048 B; n32 bf16 in 6,144 B; n64 readout 16,384 + 256 B plus the
+    snapshots; n4 128 B."""
+    from linear_rnn_scan_b200 import inputs as gen
+    W = gen.WORKLOADS
+    per_unit = lambda w: bench.step_bytes(w)["total"] / w.token_heads
+    assert per_unit(W["n16_detnorm_b8h8l4096"]) == 2048
+    assert per_unit(W["n16_detnorm_b1h8l262144"]) == 2048
+    assert per_unit(W["n32_ldu_bf16_b4h16l8192"]) == 6144
+    assert per_unit(W["n4_reshape_l1024"]) == 128
+    w = W["n64_detnorm_readout_b2h4l16384"]
+    snaps = w.B * (w.L // 256) * w.H * 64 * 64 * 4
+    assert bench.step_bytes(w)["total"] == w.token_heads * (16384 + 256) + snaps
+    assert snaps == 8388608
