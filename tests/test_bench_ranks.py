@@ -103,3 +103,37 @@ def test_algorithmic_bytes_per_unit():
     snaps = w.B * (w.L // 256) * w.H * 64 * 64 * 4
     assert bench.step_bytes(w)["total"] == w.token_heads * (16384 + 256) + snaps
     assert snaps == 8388608
+
+
+def test_clock_sampler_with_a_fake_nvml(monkeypatch):
+    """The clock record of the timed region, read through a fake NVML (no
+    GPU setting is read or changed): median SM clock, the visible-device
+    index mapped to the physical one, reason bits named (idle left out)."""
+    import types
+    import time as _time
+    calls = {"index": None}
+    clocks = iter([1965, 1965, 1900, 1965, 1500] + [1965] * 10000)
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=1,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByIndex=lambda i: calls.__setitem__("index", i) or "h",
+        nvmlDeviceGetMaxClockInfo=lambda h, c: 1965,
+        nvmlDeviceGetClockInfo=lambda h, c: next(clocks),
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0x1 | 0x4 | 0x8,
+    )
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "5,3")
+    with bench.ClockSampler(1, period_s=0.001) as cs:
+        _time.sleep(0.05)
+    s = cs.summary()
+    assert calls["index"] == 3
+    assert s["sm_max_mhz"] == 1965 and s["samples"] >= 5 and s["sm_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap", "hw_slowdown"] and s["sm_mhz_min"] == 1500
+
+
+def test_clock_sampler_without_nvml(monkeypatch):
+    monkeypatch.setitem(sys.modules, "pynvml", None)      # import fails
+    with bench.ClockSampler(0) as cs:
+        pass
+    s = cs.summary()
+    assert s["samples"] == 0 and s["sm_mhz"] is None and s["note"]
