@@ -137,3 +137,23 @@ def test_clock_sampler_without_nvml(monkeypatch):
         pass
     s = cs.summary()
     assert s["samples"] == 0 and s["sm_mhz"] is None and s["note"]
+
+
+def test_oracle_rate_is_a_bounded_sample():
+    """The CPU baseline times the oracle on a bounded sample: the first
+    t_end tokens of a spread subset of sequences, repeated to about the
+    target time; the rate is the units it ran over the seconds they took."""
+    import time as _time
+    import oracle
+    from linear_rnn_scan_b200 import inputs as gen
+    oracle.build()
+    w = gen.WORKLOADS["n16_detnorm_b8h8l4096"]
+    x = gen.make_x(w)
+    t0 = _time.perf_counter()
+    rate, units, secs, sample = bench.oracle_rate(w, x, 0.3, 2)
+    wall = _time.perf_counter() - t0
+    assert wall < 10.0 and secs >= 0.15 and rate == units / secs
+    assert "of 4096 tokens of 8 of 64 (b,h) sequences" in sample and "2 threads" in sample
+    t_end = int(sample.split()[1])
+    reps = int(sample.split(" x")[1].split(",")[0])
+    assert units == 8 * t_end * reps and 16 <= t_end <= 4096
