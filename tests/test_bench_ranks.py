@@ -157,3 +157,22 @@ def test_oracle_rate_is_a_bounded_sample():
     t_end = int(sample.split()[1])
     reps = int(sample.split(" x")[1].split(",")[0])
     assert units == 8 * t_end * reps and 16 <= t_end <= 4096
+
+
+def test_reference_arm_line_on_rank_0(monkeypatch, capsys):
+    """Rank 0 of the reference arm prints one JSON line with the contract's
+    keys: the oracle's rate as value, cpu_baseline describing the run, e2e
+    with no host-device bytes, at least three warm-up steps."""
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    monkeypatch.setenv("MRU_REF_STEP_SECONDS", "0.2")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0", "--workload",
+                       "n4_reshape_l1024"]) == 0
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["warmup"] == 3 and d["steps"] == 1 and d["n_gpus"] == 1
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["config"]["workload"] == "n4_reshape_l1024"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
