@@ -129,6 +129,11 @@ def kernel_bytes(name: str, w: gen.Workload, chunk: int) -> int:
     groups = -(-chains // 16)
     if name == "k_small_scan":
         return sb["in"] + sb["out"]
+    if name == "k16_fused":
+        # embeddings in once (the apply items read them again from L2), S_t
+        # out, chunk totals and in-group prefixes, per-token scalars
+        cdb = w.token_heads * 8 if w.mode == gen.MODE_DETNORM else 0
+        return sb["in"] + sb["out"] + tot * (4 + 4) + cdb
     if "chunk" in name:
         return sb["in"] + sb["out"] + tot * 4
     if "fixup" in name:

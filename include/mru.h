@@ -64,7 +64,7 @@ typedef enum {
     MRU_ERR_WORKSPACE = 3,    /* workspace smaller than mru_workspace_size() */
     MRU_ERR_CUDA = 4,         /* a CUDA launch or copy failed */
     MRU_ERR_SINGULAR = 5,     /* DETNORM met det = 0 or a non-finite determinant */
-    MRU_ERR_TIMEOUT = 6       /* reserved: a bounded device-side wait gave up (no current kernel waits) */
+    MRU_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up (recorded in the status word) */
 } mru_status;
 
 typedef enum {
@@ -196,8 +196,25 @@ mru_status mru_scan_backward(const mru_problem* p, const void* x, const float* S
                              void* stream);
 
 /* Synchronises `stream` and returns the device-detected status of the last
- * call that used this workspace (MRU_OK or MRU_ERR_SINGULAR). */
+ * call that used this workspace: MRU_OK, MRU_ERR_SINGULAR, or
+ * MRU_ERR_TIMEOUT when a bounded wait of the single-read n = 16 kernel gave
+ * up (its outputs are then unspecified; the CUDA context stays usable). */
 mru_status mru_last_device_status(const void* ws, void* stream);
+
+/* Testing hook for the bounded waits of the single-read n = 16 kernel.  With
+ * MRU_N16_FUSED=1 in the environment (read at each call), mru_scan_fused for
+ * n = 16, fp32, reshape / DETNORM / CAYLEY and more than one chunk per
+ * sequence runs one persistent kernel that reads x from HBM once instead of
+ * the three passes (it is correct but, on B200, still slower; the passes
+ * stay the default).  Its warps wait on one another in two
+ * places only: a group of chunks looking back for the aggregates of the
+ * groups before it, and an apply item waiting for its group's carry; every
+ * wait gives up after a time limit (2 s), records MRU_ERR_TIMEOUT in the
+ * status word and makes the launch end early.  After this call, the next
+ * such launch in the process never publishes the carry of its first group
+ * and uses a limit of `ms` milliseconds (> 0), so that it ends with
+ * MRU_ERR_TIMEOUT without any fault; ms <= 0 cancels a pending request. */
+void mru_debug_stall_next_fused(int32_t ms);
 
 /* Static string for a status code. */
 const char* mru_status_string(mru_status s);

@@ -122,6 +122,16 @@ KParams make_params(const mru_problem& p, int32_t src, bool readout)
     return k;
 }
 
+// The single-read fused n = 16 kernel is opt-in (MRU_N16_FUSED=1 in the
+// environment, read at each call): on B200 it is still slower than the three
+// passes (configuration B8 H8 L4096: 0.34 ms against 0.22 ms), its warps
+// waiting on group carries.
+bool fused16_enabled()
+{
+    const char* v = getenv("MRU_N16_FUSED");
+    return v && v[0] == '1';
+}
+
 Workspace layout(const KParams& k, bool readout)
 {
     Workspace W;
@@ -133,6 +143,12 @@ Workspace layout(const KParams& k, bool readout)
     if (n16::supports(k, readout)) {
         W.fast = true;
         W.fast_n = 16;
+        W.fused = fused16_enabled();
+        if (W.fused) {
+            W.f16 = n16::fused_plan(k, off);
+            W.bytes = W.f16.end;
+            return W;
+        }
         W.totals = off; off = round_up(off + BH * k.K * nn * sizeof(float), 256);
         W.c16 = n16::carry_plan((int64_t)BH, k.K, off);
         W.bytes = W.c16.end > off ? W.c16.end : off;
@@ -236,6 +252,7 @@ const char* mru_kernel_name(const mru_problem* p, int32_t readout, int32_t i)
     const Workspace W = layout(k, readout != 0);
     if (!W.fast) return kernel_name(k, readout != 0, i);
     if (k.K == 1) return i == 0 ? (W.fast_n == 16 ? "k16_apply" : "k32_apply") : "";
+    if (W.fast_n == 16 && W.fused) return i == 0 ? "k16_fused" : "";
     if (W.fast_n == 16) return i == 0 ? "k16_reduce" : i == 1 ? "k16_carry" : i == 2 ? "k16_apply" : "";
     const int lv = W.plan.levels;
     const bool n32k = W.fast_n == 32;
@@ -254,7 +271,7 @@ int32_t mru_launch_count(const mru_problem* p, int32_t readout)
     const KParams k = make_params(*p, SRC_EMBEDDING, readout != 0);
     const Workspace W = layout(k, readout != 0);
     if (k.K == 1) return 1;                  // single chunk: one kernel, from S0
-    if (W.fast) return W.fast_n == 16 ? 3 : 2 + carry::launches(W.plan);
+    if (W.fast) return W.fast_n == 16 ? (W.fused ? 1 : 3) : 2 + carry::launches(W.plan);
     return 5;
 }
 
@@ -451,6 +468,8 @@ mru_status mru_last_device_status(const void* ws, void* stream)
     if (word & STATUS_SINGULAR) return MRU_ERR_SINGULAR;
     return MRU_OK;
 }
+
+void mru_debug_stall_next_fused(int32_t ms) { n16::set_stall_test(ms > 0 ? ms : 0); }
 
 mru_status mru_set_profile_events(void* const* events, int32_t count)
 {

@@ -97,6 +97,18 @@ struct CarryPlan {
     size_t ctr_begin, ctr_bytes;         // the counters (zeroed by every reduce launch)
     size_t end;
 };
+// Workspace of the single-read fused kernel (k16_fused): chunk totals and
+// in-group prefixes per chunk, group aggregates, carries and inclusive
+// prefixes per group of 2^gshift chunks, per-token scalars of the corrected
+// mode, and a control block (tickets, abort flag, group counters and flags)
+// that is zeroed before every launch.
+struct FusedPlan {
+    int32_t gshift;
+    int64_t NG, Lp;                      // groups per sequence; row length of the scalar records
+    size_t tot, R0, agg, incl, excl, cd;
+    size_t ctl, gcnt, gflag, ctl_bytes;  // control block [ctl, ctl + ctl_bytes)
+    size_t end;
+};
 }  // namespace n16
 
 struct Workspace {
@@ -108,7 +120,9 @@ struct Workspace {
     bool fast;           // specialised kernels: chunk totals and a carry plan
     int fast_n;          // 16 or 32: which specialised kernels
     carry::Plan plan;    // n = 32
-    n16::CarryPlan c16;  // n = 16
+    n16::CarryPlan c16;  // n = 16, three launches
+    n16::FusedPlan f16;  // n = 16, the single-read fused launch
+    bool fused;          // n = 16 runs k16_fused
     size_t bytes;        // total
 };
 
@@ -142,6 +156,14 @@ cudaError_t launch_carry(const KParams& p, const float* totals, const CarryPlan&
 // the carry S0 (or I when S0 is null); no reduce or carry launch precedes it.
 cudaError_t launch_apply(const KParams& p, const float* x, const CarryPlan& cp, const char* ws, float* S_out,
                          uint32_t* status, const float* S0, bool direct, cudaStream_t s);
+// The single-read fused scan (one launch after a memset of its control block).
+FusedPlan fused_plan(const KParams& p, size_t off);
+cudaError_t launch_fused(const KParams& p, const FusedPlan& fp, char* ws, const float* x, const float* S0,
+                         float* S_out, uint32_t* status, cudaStream_t s);
+// Testing hook: the next fused launch never publishes its first group's carry
+// and bounds its waits by `ms` milliseconds, so that it ends with
+// STATUS_TIMEOUT.
+void set_stall_test(int32_t ms);
 // Backward passes on the tensor cores (fp32 embeddings, reshape, and the
 // determinant-corrected mode with the identity); the generic fp64 scan of
 // the chunk gradients runs between them.

@@ -38,6 +38,7 @@
 // Split-tf32 ("3xTF32", after Ootomo and Yokota, 2022): x = hi + lo with hi
 // x rounded to tf32 (sign, exponent, 10 mantissa bits) and lo = x - hi exact
 // in fp32; a b ~ a_lo b_hi + a_hi b_lo + a_hi b_hi.
+#include <stdlib.h>
 #include <string.h>
 
 #include <atomic>
@@ -1102,6 +1103,573 @@ k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, 
     }
 }
 
+// ---- single-read fused scan: one persistent launch --------------------------
+//
+// Warps take items, one chain (b, h, chunk of C tokens) each, from two
+// counters that hand them out in chain order (h fastest, then the chunk,
+// then b):
+//  * reduce item   streams the chunk's slices from HBM (under an L2
+//                  evict-last policy, so that the apply item finds them in
+//                  L2), factorises every token's determinant in the corrected
+//                  mode and records the token's (c alpha, c - 1), runs the
+//                  chain on the corrected matrices and writes the chunk total.
+//                  The reduce item that completes a group of G chunks of a
+//                  sequence scans the group in fp64 (inclusive in-group
+//                  prefixes, kept fp32, and the group aggregate), publishes
+//                  the aggregate, finds the group's carry by a decoupled
+//                  look-back (the aggregates of the earlier groups multiplied
+//                  in, from right to left, until an inclusive prefix or S0),
+//                  and publishes the carry and the group's inclusive prefix.
+//  * apply item    taken only once its group's carry is out: the chain's
+//                  carry (group carry times in-group prefix, fp64), then the
+//                  chain from it with the recorded scalars, x read a second
+//                  time (from L2, evict-first), every S_t written
+//                  (evict-first).
+// A warp takes the next apply item in chain order when its group's carry is
+// out, else the next reduce item.  The only waits -- a look-back on a group
+// that no warp has scanned yet, and a warp with nothing to take -- are on
+// items of lower chain order, which running warps hold (items are claimed by
+// running warps only, reduce tickets in order), so they end; each is bounded
+// by a time limit anyway, past which the kernel records STATUS_TIMEOUT,
+// raises an abort flag that every warp reads before it takes an item, and
+// returns.  Per token-head HBM sees x once and S once.
+
+constexpr int FST = 8, FWARPS = 4;
+
+struct FSmem {
+    float stage[2][FST * NN];          // token slices (swizzled), or an apply item's carry factors
+    float2 cd[2][FST];                 // per stage: per-token (c alpha, diagonal term of F)
+};
+// Word offsets of the carry factors in a fused apply stage: the group carry E
+// (fp32, full matrix) and the in-group prefix R (fp32, split form).
+constexpr int FCF_E = 0, FCF_R = NN;
+
+enum : int { FK_REDUCE = 1, FK_APPLY = 2, FK_DONE = 3 };
+
+struct FCtl {
+    unsigned* ctr;        // [0] ticket counter, [1] abort flag
+    unsigned* gcnt;       // [seq][NG] reduce items done per group
+    unsigned* gflag;      // [seq][NG] 0; 1 aggregate out; 2 carry and inclusive prefix out
+    float* tot;           // [seq][K] chunk totals (split form, corrected)
+    float* R0;            // [seq][K] inclusive in-group prefixes (split form)
+    double* agg;          // [seq][NG] group aggregates (split form)
+    double* incl;         // [seq][NG] inclusive prefix through each group (full)
+    float* excl;          // [seq][NG] group carries (full)
+    float2* cd;           // [seq][Lp] per-token (c alpha, c - 1), corrected mode
+    int64_t Lp, NG;
+    int64_t lead;         // reduce items handed out before the first apply item
+    int32_t gshift;
+    uint64_t limit_ns;    // bound on every wait
+    int32_t stall_first;  // testing: group 0's carry is never published
+};
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_last()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t policy_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ void cp_async16_hint(void* smem, const void* gmem, uint64_t pol)
+{
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "l"(pol));
+}
+__device__ __forceinline__ void st_f2_hint(float* p, float a, float b, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(p), "f"(a), "f"(b), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void store_d_hint(float* out, const float (&Ad)[2][4], int g, int q, uint64_t pol)
+{
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8)
+            st_f2_hint(out + (g + 8 * h8) * N + 8 * nt + 2 * q, Ad[nt][2 * h8], Ad[nt][2 * h8 + 1], pol);
+}
+
+// Records a timeout and raises the abort flag.
+__device__ __forceinline__ void fused_abort(const FCtl& f, uint32_t* status)
+{
+    atomicOr(status, STATUS_TIMEOUT);
+    atomicExch(f.ctr + 1, 1u);
+}
+
+// Ticket -> item.  The schedule: the first `lead` reduce items, then an
+// apply item and a reduce item in turn while reduce items remain, then the
+// remaining apply items; apply item i thus comes after reduce item
+// lead + i - 1.  With lead at least a group of chains (G chunks of every
+// head) the apply item's whole group, and every earlier group of its
+// sequence, is handed out before it.
+__device__ __forceinline__ int fused_decode(unsigned t, int64_t nchains, int64_t lead, int64_t& chain)
+{
+    const int64_t u = t;
+    if (u >= 2 * nchains) return FK_DONE;
+    if (u < lead) { chain = u; return FK_REDUCE; }
+    const int64_t pairs = nchains - lead;
+    if (u < lead + 2 * pairs) {
+        const int64_t v = u - lead;
+        chain = (v & 1) ? lead + (v >> 1) : (v >> 1);
+        return (v & 1) ? FK_REDUCE : FK_APPLY;
+    }
+    chain = u - nchains;
+    return FK_APPLY;
+}
+
+__device__ __forceinline__ unsigned* group_flag(const KParams& p, const FCtl& f, const Chain& c)
+{
+    return f.gflag + (c.b * p.H + c.h) * f.NG + (c.k >> f.gshift);
+}
+
+// Waits (lane 0, bounded) until the apply item's group carry is out; false
+// on timeout or when the launch is aborting.  `seen` is a flag value read
+// earlier (0 when none was).
+__device__ bool wait_ready(const unsigned* flag, unsigned seen, const FCtl& f, uint32_t* status)
+{
+    if (seen == 2u) return true;
+    const uint64_t t0 = global_ns();
+    unsigned ns = 64;
+    for (;;) {
+        if (ld_acquire(flag) == 2u) return true;
+        if (ld_acquire(f.ctr + 1)) return false;
+        if (global_ns() - t0 > f.limit_ns) {
+            fused_abort(f, status);
+            return false;
+        }
+        __nanosleep(ns);
+        if (ns < 1024) ns <<= 1;
+    }
+}
+
+// A 16 x 16 matrix from global memory (bypassing L1) in accumulator layout
+// (fp64), full form (plus_i adds I to a split-form matrix).
+template <typename T>
+__device__ __forceinline__ void d16_ld_acc(const T* src, D16& a, int lane, bool plus_i)
+{
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int row = 8 * mt + g, col = 8 * nb + 2 * t + h;
+                a.m[mt][nb][h] = (double)__ldcg(src + row * N + col) + ((plus_i && row == col) ? 1.0 : 0.0);
+            }
+}
+// The same as the B operand.
+template <typename T>
+__device__ __forceinline__ void d16_ld_b(const T* src, B16& b, int lane)
+{
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) b.b[kk][nb] = (double)__ldcg(src + (8 * (kk >> 1) + 2 * t + (kk & 1)) * N + 8 * nb + g);
+}
+
+// The group scan: R_j = R_{j-1} + (T_j + R_{j-1} T_j) over the m chunk totals
+// at tot (fp64; R_j kept fp32 at R), the last one, the aggregate, to agg.
+// Operands come straight from L2, two items ahead of the products.
+__device__ __noinline__ void fused_group_scan(const float* tot, float* R, double* agg, int m, int lane)
+{
+    const int g = lane >> 2, t = lane & 3;
+    float rb[2][8], ra[2][8];
+    auto fetch = [&](int j, float (&b)[8], float (&a)[8]) {
+        const float* it = tot + (int64_t)j * NN;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) b[2 * kk + nb] = __ldcg(it + (8 * (kk >> 1) + 2 * t + (kk & 1)) * N + 8 * nb + g);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+                const float2 v = __ldcg(reinterpret_cast<const float2*>(it + (8 * mt + g) * N + 8 * nb + 2 * t));
+                a[4 * mt + 2 * nb] = v.x;
+                a[4 * mt + 2 * nb + 1] = v.y;
+            }
+    };
+    fetch(0, rb[0], ra[0]);
+    if (m > 1) fetch(1, rb[1], ra[1]);
+    D16 st, acc;
+    d16_zero(st);
+    for (int j = 0; j < m; ++j) {
+        B16 Bf;
+        const int s = j & 1;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) Bf.b[kk][nb] = (double)rb[s][2 * kk + nb];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) acc.m[mt][nb][h] = (double)ra[s][4 * mt + 2 * nb + h];
+        if (j + 2 < m) fetch(j + 2, rb[s], ra[s]);
+        d16_mac(st, Bf, acc);                          // T_j + R_{j-1} T_j
+#pragma unroll
+        for (int i = 0; i < 8; ++i) (&st.m[0][0][0])[i] += (&acc.m[0][0][0])[i];
+        store_acc(R + (int64_t)j * NN, st, lane);
+    }
+    store_acc(agg, st, lane);
+}
+
+// The decoupled look-back of group gi of one sequence: the carry
+// E = E_0 (I + A_0) ... (I + A_{gi-1}), E_0 = S0 (or I), taken from the
+// first group j < gi (right to left) whose inclusive prefix is out, the
+// aggregates A of the groups in between multiplied in; then the group's
+// carry (fp32) and inclusive prefix E (I + A_gi) (fp64) are written and
+// published.  pf: 2 KB of this warp's shared memory.  False when a wait ran
+// out (or the launch is aborting).
+__device__ __noinline__ bool fused_lookback(const FCtl f, int64_t seq, int64_t gi, const float* s0, double* pf,
+                                            uint32_t* status, int lane)
+{
+    const int64_t base = seq * f.NG;
+    // P = (I + A_{j+1}) ... (I + A_{gi-1}), full form, in registers and in pf
+    D16 P, acc, E;
+    {
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) P.m[mt][nb][h] = (8 * mt + g == 8 * nb + 2 * t + h) ? 1.0 : 0.0;
+    }
+    store_acc(pf, P, lane);
+    __syncwarp();
+    bool found = false;
+    for (int64_t j = gi - 1; j >= 0; --j) {
+        unsigned fl = 0;
+        if (lane == 0) {
+            const uint64_t t0 = global_ns();
+            unsigned ns = 32;
+            for (;;) {
+                fl = ld_acquire(f.gflag + base + j);
+                if (fl >= 1u || ld_acquire(f.ctr + 1)) break;
+                if (global_ns() - t0 > f.limit_ns) {
+                    fused_abort(f, status);
+                    break;
+                }
+                __nanosleep(ns);
+                if (ns < 1024) ns <<= 1;
+            }
+        }
+        fl = __shfl_sync(FULL, fl, 0);
+        if (fl == 0u) return false;
+        B16 Pb;
+        d16_load(pf, Pb, lane);
+        if (fl == 2u) {                                    // E = incl_j P
+            D16 Ij;
+            d16_ld_acc(f.incl + (base + j) * NN, Ij, lane, false);
+            d16_zero(E);
+            d16_mac(Ij, Pb, E);
+            found = true;
+            break;
+        }
+        D16 Aj;                                            // P <- (I + A_j) P = P + A_j P
+        d16_ld_acc(f.agg + (base + j) * NN, Aj, lane, false);
+        acc = P;
+        d16_mac(Aj, Pb, acc);
+        P = acc;
+        __syncwarp();
+        store_acc(pf, P, lane);
+        __syncwarp();
+    }
+    if (!found) {                                          // E = E_0 P
+        if (s0) {
+            D16 Z;
+            B16 Pb;
+            d16_load(pf, Pb, lane);
+            d16_ld_acc(s0, Z, lane, false);
+            d16_zero(E);
+            d16_mac(Z, Pb, E);
+        } else {
+            E = P;
+        }
+    }
+    // the group's carry (fp32) and its inclusive prefix E + E A_gi (fp64)
+    store_acc(f.excl + (base + gi) * NN, E, lane);
+    B16 Ab;
+    d16_ld_b(f.agg + (base + gi) * NN, Ab, lane);
+    acc = E;
+    d16_mac(E, Ab, acc);
+    store_acc(f.incl + (base + gi) * NN, acc, lane);
+    __threadfence();
+    __syncwarp();
+    if (lane == 0 && !(f.stall_first && gi == 0)) st_release(f.gflag + base + gi, 2u);
+    return true;
+}
+
+// The carry of an apply item, C = E (I + R) in fp64 (R absent for the first
+// chunk of a group), rounded to fp32 into accumulator layout.
+__device__ __forceinline__ void fused_carry(const float* in, bool has_r, int lane, float (&Sd)[2][4])
+{
+    D16 C;
+    {
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+                const float2 v = *reinterpret_cast<const float2*>(in + FCF_E + (8 * mt + g) * N + 8 * nb + 2 * t);
+                C.m[mt][nb][0] = v.x;
+                C.m[mt][nb][1] = v.y;
+            }
+    }
+    if (has_r) {
+        D16 acc = C;
+        F16<float> Rb;
+        d16_load(in + FCF_R, Rb, lane);
+        d16_mac(C, Rb, acc);
+        C = acc;
+    }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) Sd[nb][2 * mt + h] = (float)C.m[mt][nb][h];
+}
+
+// Stage `s` of item (kind, chain) into buf / cdbuf: for an apply item stage 0
+// is the carry factors, then the token stages of FST tokens.
+__device__ __forceinline__ void fused_issue(const KParams& p, const FCtl& f, const float* x, int kind,
+                                            const Chain& c, int s, float* buf, float2* cdbuf, int lane,
+                                            uint64_t pol_x)
+{
+    const int64_t seq = c.b * p.H + c.h;
+    if (kind == FK_APPLY && s == 0) {
+        const int64_t gi = c.k >> f.gshift;
+        const float* E = f.excl + (seq * f.NG + gi) * NN;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) cp_async16(buf + FCF_E + 4 * (lane + 32 * i), E + 4 * (lane + 32 * i));
+        if (c.k & ((1 << f.gshift) - 1)) {
+            const float* R = f.R0 + (seq * p.K + c.k - 1) * NN;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) cp_async16(buf + FCF_R + 4 * (lane + 32 * i), R + 4 * (lane + 32 * i));
+        }
+        return;
+    }
+    const int64_t t0 = c.tbeg + (int64_t)(s - (kind == FK_APPLY ? 1 : 0)) * FST;
+    const int nt = (c.tend - t0 < FST) ? (int)(c.tend - t0) : FST;
+    const float* xb = x + ((c.b * p.L + t0) * p.H + c.h) * NN;
+    const int64_t tok = p.H * NN;
+#pragma unroll
+    for (int i = 0; i < FST * 2; ++i) {                    // 64 granules a slice, 2 per lane
+        const int gi = lane + 32 * i;
+        const int j = gi >> 6, gr = gi & 63, row = gr >> 2, c4 = gr & 3;
+        if (j < nt) cp_async16_hint(buf + j * NN + swz(row, 4 * c4), xb + j * tok + row * N + 4 * c4, pol_x);
+    }
+    if (kind == FK_APPLY && p.mode == MRU_MODE_DETNORM && lane < FST / 2)
+        cp_async16(cdbuf + 2 * lane, f.cd + seq * f.Lp + t0 + 2 * lane);
+}
+
+template <bool Cayley>
+__global__ void __launch_bounds__(FWARPS * 32, 3)
+k16_fused(KParams p, FCtl f, const float* __restrict__ x, const float* __restrict__ S0, float* __restrict__ S_out,
+          uint32_t* status)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    FSmem& sm = reinterpret_cast<FSmem*>(smem_raw)[warp];
+    const int64_t nchains = p.B * p.H * p.K;
+    const int g = lane >> 2, q = lane & 3;
+    const float m0 = (g == 2 * q) ? 1.0f : 0.0f;
+    const float m1 = (g == 2 * q + 1) ? 1.0f : 0.0f;
+    const int G = 1 << f.gshift;
+    const bool detnorm = p.mode == MRU_MODE_DETNORM && !Cayley;
+    const uint64_t pol_keep = policy_evict_last(), pol_drop = policy_evict_first();
+    const int64_t tok = p.H * NN;
+
+    // the first item
+    unsigned tk = 0;
+    if (lane == 0) tk = atomicAdd(f.ctr, 1u);
+    tk = __shfl_sync(FULL, tk, 0);
+    int64_t chain = 0;
+    int kind = fused_decode(tk, nchains, f.lead, chain);
+    if (kind == FK_DONE) return;
+    Chain c = chain_at(p, chain);
+    if (kind == FK_APPLY) {
+        bool ok = true;
+        if (lane == 0) ok = wait_ready(group_flag(p, f, c), 0u, f, status);
+        if (!__shfl_sync(FULL, (int)ok, 0)) return;
+        __syncwarp();
+    }
+    unsigned slot = 0;                                     // stream position: stage buffers alternate
+    fused_issue(p, f, x, kind, c, 0, sm.stage[0], sm.cd[0], lane, kind == FK_APPLY ? pol_drop : pol_keep);
+    cp_async_commit();
+    for (;;) {
+        // claim the next item now; its ticket is read one stage later and
+        // (for an apply item) its group flag at the last stage
+        unsigned tk_next = 0, fl_next = 0;
+        if (lane == 0) tk_next = atomicAdd(f.ctr, 1u);
+        int nkind = FK_DONE;
+        int64_t nchain = 0;
+        Chain nc = c;
+        bool decoded = false, deferred = false;
+        const int ntok = (int)(c.tend - c.tbeg);
+        const int nst = (ntok + FST - 1) / FST + (kind == FK_APPLY ? 1 : 0);
+        const int64_t seq = c.b * p.H + c.h;
+        float St[2][4];                                    // the chain's state: Q (reduce) or S (apply)
+#pragma unroll
+        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) St[n2][i] = 0.0f;
+        for (int s = 0; s < nst; ++s) {
+            const unsigned cur = slot & 1u, nxt = cur ^ 1u;
+            if (s + 1 < nst) {
+                fused_issue(p, f, x, kind, c, s + 1, sm.stage[nxt], sm.cd[nxt], lane,
+                            kind == FK_APPLY ? pol_drop : pol_keep);
+            } else {
+                if (!decoded) {
+                    nkind = fused_decode(__shfl_sync(FULL, tk_next, 0), nchains, f.lead, nchain);
+                    if (nkind != FK_DONE) nc = chain_at(p, nchain);
+                }
+                // an apply item's carry factors are fetched now only if its
+                // group carry is out already; otherwise after this item is
+                // finished (waiting here could wait on this very item)
+                if (nkind == FK_APPLY) {
+                    int ready = 0;
+                    if (lane == 0) ready = fl_next == 2u || ld_acquire(group_flag(p, f, nc)) == 2u;
+                    deferred = !__shfl_sync(FULL, ready, 0);
+                    __syncwarp();
+                }
+                if (nkind != FK_DONE && !deferred)
+                    fused_issue(p, f, x, nkind, nc, 0, sm.stage[nxt], sm.cd[nxt], lane,
+                                nkind == FK_APPLY ? pol_drop : pol_keep);
+            }
+            cp_async_commit();
+            cp_async_wait<1>();
+            __syncwarp();
+            ++slot;
+            float* xs = sm.stage[cur];
+            if (kind == FK_APPLY && s == 0) {
+                fused_carry(xs, (c.k & (G - 1)) != 0, lane, St);
+            } else {
+                const int64_t t0 = c.tbeg + (int64_t)(s - (kind == FK_APPLY ? 1 : 0)) * FST;
+                const int nt = (c.tend - t0 < FST) ? (int)(c.tend - t0) : FST;
+                float2* cdv = sm.cd[cur];
+                if (Cayley) {
+                    stage_cayley<FST>(p.alpha, xs, nt, lane);
+                    if (lane < FST) cdv[lane] = make_float2(1.0f, 0.0f);
+                    __syncwarp();
+                } else if (kind == FK_REDUCE) {
+                    stage_scalars<FST>(p, cdv, xs, nt, lane, status);
+                    if (detnorm && lane < nt) f.cd[seq * f.Lp + t0 + lane] = cdv[lane];
+                } else if (!detnorm) {
+                    if (lane < FST) cdv[lane] = make_float2(p.alpha, p.add_identity ? 0.0f : -1.0f);
+                    __syncwarp();
+                }
+                // One copy of each chain loop, not unrolled over the stage's
+                // tokens (the kernel's code must stay small enough for the
+                // instruction cache); the next token's fragments are formed
+                // while this token's products run.
+                if (kind == FK_REDUCE) {
+                    FragF fr;
+                    float2 cdj = cdv[0];
+                    make_frag_f(xs, cdj.x, m0 * cdj.y, m1 * cdj.y, g, q, fr, true);
+#pragma unroll 1
+                    for (int j = 0; j < nt; ++j) {
+                        float acc[2][4];
+                        chain_product<false>(St, fr, acc);        // F + Q F
+                        if (j + 1 < nt) {
+                            cdj = cdv[j + 1];
+                            make_frag_f(xs + (j + 1) * NN, cdj.x, m0 * cdj.y, m1 * cdj.y, g, q, fr, true);
+                        }
+#pragma unroll
+                        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) St[n2][i] += acc[n2][i];
+                    }
+                } else {
+                    float* ob = S_out + ((c.b * p.L + t0) * p.H + c.h) * NN;
+                    FragF fr;
+                    float2 cdj = cdv[0];
+                    make_frag_f(xs, cdj.x, m0 * cdj.y, m1 * cdj.y, g, q, fr, false);
+#pragma unroll 1
+                    for (int j = 0; j < nt; ++j) {
+                        float acc[2][4];
+                        chain_product<true>(St, fr, acc);         // S F
+                        if (j + 1 < nt) {
+                            cdj = cdv[j + 1];
+                            make_frag_f(xs + (j + 1) * NN, cdj.x, m0 * cdj.y, m1 * cdj.y, g, q, fr, false);
+                        }
+#pragma unroll
+                        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) St[n2][i] += acc[n2][i];
+                        store_d_hint(ob + j * tok, St, g, q, pol_drop);
+                    }
+                }
+            }
+            __syncwarp();
+            if (s == 0 && nst > 1) {
+                // the next ticket has had this stage to arrive: decode it, and
+                // start reading an apply item's group flag
+                nkind = fused_decode(__shfl_sync(FULL, tk_next, 0), nchains, f.lead, nchain);
+                decoded = true;
+                if (nkind != FK_DONE) {
+                    nc = chain_at(p, nchain);
+                    if (nkind == FK_APPLY && lane == 0) fl_next = ld_acquire(group_flag(p, f, nc));
+                }
+            }
+            if (s + 1 == nst && kind == FK_REDUCE) {
+                // the chunk total, then the group's count; the last one scans
+                store_d(f.tot + (seq * p.K + c.k) * NN, St, g, q);
+                const int64_t gi = c.k >> f.gshift;
+                const int64_t first = gi << f.gshift;
+                const int m = (p.K - first < G) ? (int)(p.K - first) : G;
+                if (arrive(f.gcnt + seq * f.NG + gi, (unsigned)m, lane)) {
+                    fused_group_scan(f.tot + (seq * p.K + first) * NN, f.R0 + (seq * p.K + first) * NN,
+                                     f.agg + (seq * f.NG + gi) * NN, m, lane);
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) st_release(f.gflag + seq * f.NG + gi, 1u);
+                    fused_lookback(f, seq, gi, S0 ? S0 + seq * NN : nullptr, reinterpret_cast<double*>(xs),
+                                   status, lane);
+                }
+            }
+        }
+        if (nkind == FK_DONE) break;
+        if (deferred) {                                    // this item is done: wait for the carry
+            bool ok = true;
+            if (lane == 0) ok = wait_ready(group_flag(p, f, nc), 0u, f, status);
+            if (!__shfl_sync(FULL, (int)ok, 0)) break;
+            __syncwarp();
+            fused_issue(p, f, x, nkind, nc, 0, sm.stage[slot & 1u], sm.cd[slot & 1u], lane, pol_drop);
+            cp_async_commit();
+        }
+        kind = nkind;
+        c = nc;
+    }
+    cp_async_wait<0>();
+}
+
 // ---- backward (vector-Jacobian product) on the tensor cores ----------------
 //
 // G_t = dL/dS_t (later states included): G_{t-1} = dS_{t-1} + G_t X_t^T and
@@ -1640,7 +2208,7 @@ k16b_apply(KParams p, const float* __restrict__ x, const float* __restrict__ S0,
 
 // CTAs of a persistent launch: resident CTAs per SM times the SM count,
 // cached per device and kernel slot; no more than the chains need.
-std::atomic<int> g_resident[64][10];
+std::atomic<int> g_resident[64][12];
 
 cudaError_t persistent_grid(int slot, const void* kern, int threads, size_t smem, int warps, int64_t nchains,
                             unsigned& grid)
@@ -1749,6 +2317,99 @@ cudaError_t launch_carry(const KParams& p, const float* totals, const CarryPlan&
     cudaError_t e = cudaFuncSetAttribute(k16_carry, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     k16_carry<<<(unsigned)((units + CWARPS - 1) / CWARPS), CWARPS * 32, sm, s>>>(p, totals, cp, ws, S0);
+    return cudaGetLastError();
+}
+
+// Chunk totals, in-group prefixes, group aggregates, carries and inclusive
+// prefixes, per-token scalars, then the control block, laid out from byte
+// offset off.  Groups of 16 chunks, or the smallest power of two with at
+// most 4096 groups per sequence (the look-back multiplies one aggregate per
+// group it passes; fewer, longer groups keep that chain short).
+FusedPlan fused_plan(const KParams& p, size_t off)
+{
+    FusedPlan fp;
+    memset(&fp, 0, sizeof fp);
+    const int64_t nseq = p.B * p.H;
+    fp.gshift = 4;
+    while (p.K > ((int64_t)4096 << fp.gshift) && fp.gshift < 10) ++fp.gshift;
+    fp.NG = p.K > 0 ? (p.K + (1 << fp.gshift) - 1) >> fp.gshift : 0;
+    fp.Lp = (p.L + 7) / 8 * 8;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = (off + bytes + 255) / 256 * 256;
+        return o;
+    };
+    fp.tot = take((size_t)nseq * p.K * NN * sizeof(float));
+    fp.R0 = take((size_t)nseq * p.K * NN * sizeof(float));
+    fp.agg = take((size_t)nseq * fp.NG * NN * sizeof(double));
+    fp.incl = take((size_t)nseq * fp.NG * NN * sizeof(double));
+    fp.excl = take((size_t)nseq * fp.NG * NN * sizeof(float));
+    fp.cd = take(p.mode == MRU_MODE_DETNORM ? (size_t)nseq * fp.Lp * sizeof(float2) : 0);
+    fp.ctl = off;
+    fp.gcnt = fp.ctl + 16;
+    fp.gflag = fp.gcnt + (size_t)nseq * fp.NG * sizeof(unsigned);
+    take(16 + 2 * (size_t)nseq * fp.NG * sizeof(unsigned));
+    fp.ctl_bytes = off - fp.ctl;
+    fp.end = off;
+    return fp;
+}
+
+namespace {
+std::atomic<int32_t> g_stall_ms{0};
+
+// Reduce items handed out before the first apply item: about 64 MB of
+// embeddings between a chain's reduce and its apply (measured on B200 for
+// B8 H8 L4096 with 32-token chunks: 16 MB 0.49 ms, 32 MB 0.45, 64 MB 0.38),
+// and at least a group of chains of every head plus one row of heads, which
+// the waits need (see fused_decode).
+int64_t fused_lead(const KParams& p, const FusedPlan& fp)
+{
+    const int64_t nchains = p.B * p.H * p.K;
+    const int64_t chain_bytes = (int64_t)p.chunk * NN * (int64_t)sizeof(float);
+    int64_t lead = ((int64_t)64 << 20) / (chain_bytes > 0 ? chain_bytes : 1);
+    const int64_t need = ((int64_t)1 << fp.gshift) * p.H + p.H;
+    if (lead < need) lead = need;
+    return lead < nchains ? lead : nchains;
+}
+}
+
+void set_stall_test(int32_t ms) { g_stall_ms.store(ms, std::memory_order_relaxed); }
+
+cudaError_t launch_fused(const KParams& p, const FusedPlan& fp, char* ws, const float* x, const float* S0,
+                         float* S_out, uint32_t* status, cudaStream_t s)
+{
+    const int64_t nchains = p.B * p.H * p.K;
+    if (nchains == 0) return cudaSuccess;
+    if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    FCtl f;
+    f.ctr = reinterpret_cast<unsigned*>(ws + fp.ctl);
+    f.gcnt = reinterpret_cast<unsigned*>(ws + fp.gcnt);
+    f.gflag = reinterpret_cast<unsigned*>(ws + fp.gflag);
+    f.tot = reinterpret_cast<float*>(ws + fp.tot);
+    f.R0 = reinterpret_cast<float*>(ws + fp.R0);
+    f.agg = reinterpret_cast<double*>(ws + fp.agg);
+    f.incl = reinterpret_cast<double*>(ws + fp.incl);
+    f.excl = reinterpret_cast<float*>(ws + fp.excl);
+    f.cd = reinterpret_cast<float2*>(ws + fp.cd);
+    f.Lp = fp.Lp;
+    f.NG = fp.NG;
+    f.gshift = fp.gshift;
+    f.lead = fused_lead(p, fp);
+    const int32_t stall = g_stall_ms.exchange(0, std::memory_order_relaxed);
+    f.stall_first = stall > 0;
+    f.limit_ns = stall > 0 ? (uint64_t)stall * 1000000ull : 2000000000ull;     // 2 s unless testing
+    cudaError_t e = cudaMemsetAsync(ws + fp.ctl, 0, fp.ctl_bytes, s);
+    if (e != cudaSuccess) return e;
+    const bool cayley = p.mode == MRU_MODE_CAYLEY;
+    auto kern = cayley ? k16_fused<true> : k16_fused<false>;
+    const size_t sm = sizeof(FSmem) * FWARPS;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)) != cudaSuccess)
+        return e;
+    unsigned grid = 0;
+    if ((e = persistent_grid(cayley ? 10 : 9, (const void*)kern, FWARPS * 32, sm, FWARPS, nchains, grid)) !=
+        cudaSuccess)
+        return e;
+    kern<<<grid, FWARPS * 32, sm, s>>>(p, f, x, S0, S_out, status);
     return cudaGetLastError();
 }
 

@@ -1704,6 +1704,13 @@ cudaError_t scan_fast16(const KParams& p, const void* src, const float* S0, floa
         if (launches) *launches = 1;
         return cudaGetLastError();
     }
+    if (W.fused) {
+        profile_mark(0, 0, s);
+        if ((e = n16::launch_fused(p, W.f16, ws, x, S0, S_out, status, s)) != cudaSuccess) return e;
+        profile_mark(0, 1, s);
+        if (launches) *launches = 1;
+        return cudaGetLastError();
+    }
     profile_mark(0, 0, s);
     if ((e = n16::launch_reduce(p, x, totals, W.c16, ws, status, s)) != cudaSuccess) return e;
     profile_mark(0, 1, s);

@@ -31,7 +31,8 @@ MATH = {"auto": 0, "fp32": 1, "tf32": 2, "tf32x3": 3, "bf16x3": 4}
 EXPORTS = ["mru_workspace_size", "mru_build_states", "mru_scan", "mru_scan_fused",
            "mru_last_device_status", "mru_status_string", "mru_chosen_chunk", "mru_launch_count",
            "mru_set_profile_events", "mru_scan_fused_noalloc", "mru_kernel_name", "mru_effective_math",
-           "mru_backward_workspace_size", "mru_scan_backward", "mru_scan_fused_host"]
+           "mru_backward_workspace_size", "mru_scan_backward", "mru_scan_fused_host",
+           "mru_debug_stall_next_fused"]
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -101,6 +102,8 @@ def load(path: str = LIB_PATH):
             lib.mru_scan_fused_host.argtypes = [P, vp, vp, ctypes.POINTER(Readout), vp, vp, vp, vp, vp, sz,
                                                 ctypes.c_int32, vp, vp, vp]
             lib.mru_scan_fused_host.restype = ctypes.c_int
+            lib.mru_debug_stall_next_fused.argtypes = [ctypes.c_int32]
+            lib.mru_debug_stall_next_fused.restype = None
             _lib = lib
     return _lib
 
@@ -194,6 +197,13 @@ def scan_backward(p: Problem, x: int, S0: int | None, S_fwd: int, dS: int, dx: i
 
 def last_device_status(ws: int, stream: int = 0) -> int:
     return load().mru_last_device_status(ws, stream)
+
+
+def debug_stall_next_fused(ms: int) -> None:
+    """Testing hook: the next single-read n = 16 launch withholds its first
+    group's carry and bounds its waits by `ms` milliseconds, so that it ends
+    with ERR_TIMEOUT in the status word."""
+    load().mru_debug_stall_next_fused(int(ms))
 
 
 def set_profile_events(handles) -> int:

@@ -124,7 +124,8 @@ def test_binding_fails_loudly_without_library(tmp_path):
 
 def test_single_chunk_problems_take_one_launch(lib):
     """A problem of one chunk per sequence (L <= chunk: decode steps, short
-    segments) runs one kernel from S0; longer ones run the full pass order."""
+    segments) runs one kernel from S0; longer ones run the full pass order
+    (for n = 16 the three passes, or the single-read kernel when asked for)."""
     cases = [(mru.problem(8, 8, 1, 16, mode=mru.MODE_DETNORM, alpha=0.0125), ["k16_apply"]),
              (mru.problem(4, 16, 1, 32, x_dtype="bf16", mode=mru.MODE_LDU), ["k32_apply"]),
              (mru.problem(2, 3, 5, 8, mode=mru.MODE_CAYLEY, alpha=0.1), ["k_chunk_prefix"]),
@@ -133,6 +134,11 @@ def test_single_chunk_problems_take_one_launch(lib):
         assert mru.launch_count(p) == 1 and mru.kernel_names(p) == names
     p = mru.problem(8, 8, 4096, 16, mode=mru.MODE_DETNORM, alpha=0.0125)
     assert mru.kernel_names(p) == ["k16_reduce", "k16_carry", "k16_apply"]
+    os.environ["MRU_N16_FUSED"] = "1"
+    try:
+        assert mru.kernel_names(p) == ["k16_fused"] and mru.launch_count(p) == 1
+    finally:
+        os.environ.pop("MRU_N16_FUSED", None)
     p = mru.problem(2, 4, 16, 64, mode=mru.MODE_DETNORM, alpha=0.01, chunk=16)
     assert mru.kernel_names(p, True) == ["k_chunk_prefix"]
     p = mru.problem(2, 4, 4096, 64, mode=mru.MODE_DETNORM, alpha=0.01, math="tf32")
