@@ -6,9 +6,12 @@
 
 One step = one call of mru_scan_fused over the whole workload (lift + chunk
 prefixes + chunk-total scan + fix-up, every kernel of the path) with the
-embeddings already resident in HBM.  The default workload is the n = 16,
-B8 H8 L4096 determinant-corrected scan (x [8, 4096, 2048] fp32 in, every
-S_t [8, 4096, 8, 16, 16] fp32 out).  Rank 0 prints one JSON line.
+embeddings already resident in HBM.  The default workload is the largest
+single-GPU configuration the metric is quoted on: the n = 16, B1 H8 L262144
+determinant-corrected scan (x [1, 262144, 2048] fp32 in, every S_t
+[1, 262144, 8, 16, 16] fp32 out).  Rank 0 prints one JSON line; at N = 1 it
+also carries `per_workload`, the same measurement for each of the five
+configurations (n4, n16 B8, n32 LDU, n16 long, n64 readout).
 
 Multi-GPU (torchrun, one process per GPU): the (b, h) sequences are
 independent, so every rank scans its own replica of the workload with no
@@ -40,7 +43,7 @@ from linear_rnn_scan_b200 import inputs as gen  # noqa: E402
 
 METRIC = "MRU scan tokens·heads/s and achieved % of HBM/tensor roofline, 1×B200"
 UNIT = "token·heads/s"
-DEFAULT_WORKLOAD = "n16_detnorm_b8h8l4096"
+DEFAULT_WORKLOAD = "n16_detnorm_b1h8l262144"
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -359,6 +362,203 @@ def workload_config(w, chunk):
 
 # ------------------------------------------------------------------- ours ---
 
+# The five workloads the benchmark's metric is quoted on (n4, n16 B8, n32
+# LDU, n16 long, n64 readout), reported together in `per_workload`.
+BASELINE_WORKLOADS = ["n4_reshape_l1024", "n16_detnorm_b8h8l4096", "n32_ldu_bf16_b4h16l8192",
+                      "n16_detnorm_b1h8l262144", "n64_detnorm_readout_b2h4l16384"]
+
+# Tensor pipe each workload's products run on and its peak in TFLOP/s: the
+# contraction's own dtype, from MEASURED_PEAKS.json's bf16 figure times the
+# nominal dense ratio (tf32 1.1 / bf16 2.25 PFLOP/s).  The kernels issue
+# mma.sync, whose measured ceiling on this part is lower (tf32 279, bf16
+# 557 TFLOP/s); every workload is bound by HBM either way.
+NOMINAL_TF32_OVER_BF16 = 1.1 / 2.25
+
+
+def flop_side(w: gen.Workload, peaks) -> dict:
+    """Algorithmic scan FLOPs (2 n^3 per token-head) over the peak of the
+    pipe the path's products use."""
+    flops = 2.0 * w.n ** 3 * w.token_heads
+    if w.n == 32 and w.x_dtype == "bf16":
+        pipe, tf = "bf16 tensor (split bf16)", peaks["bf16_tflops"]
+    elif w.n in (16, 64):
+        pipe, tf = "tf32 tensor", peaks["bf16_tflops"] * NOMINAL_TF32_OVER_BF16
+    else:
+        pipe, tf = "fp32 FMA (SIMT, nominal 74.4)", 74.4
+    return {"flops_per_step": flops, "pipe": pipe, "peak_tflops": tf, "min_ms": flops / (tf * 1e12) * 1e3}
+
+
+def roofline_min_ms(w: gen.Workload, peaks) -> dict:
+    """The slower of the bytes at HBM peak and the scan FLOPs at the pipe's
+    peak: the roofline time of one step."""
+    sb = step_bytes(w)
+    hbm_ms = sb["total"] / (peaks["hbm_gbs"] * 1e9) * 1e3
+    fl = flop_side(w, peaks)
+    bound = "hbm" if hbm_ms >= fl["min_ms"] else "tensor"
+    return {"bytes_per_step": sb["total"], "hbm_min_ms": hbm_ms, "flop": fl, "bound": bound,
+            "min_ms": max(hbm_ms, fl["min_ms"])}
+
+
+class Case:
+    """One workload resident on the device: inputs, outputs, workspace and
+    the call, through the C-ABI."""
+
+    def __init__(self, w, dev, stream, seed_offset=0, x_np=None):
+        import torch
+
+        from linear_rnn_scan_b200 import mru
+        self.w, self.mru = w, mru
+        self.p = mru.problem_from_workload(w)
+        self.chunk = mru.chosen_chunk(self.p, w.readout)
+        self.stream = stream
+        if x_np is None:
+            x_np = gen.make_x(w, seed=w.seed + seed_offset)
+        if w.x_dtype == "bf16":
+            x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16)
+        else:
+            x_host = torch.from_numpy(x_np)
+        self.x_pin = x_host.pin_memory()
+        self.x_dev = self.x_pin.to(dev)
+        self.ws = mru.workspace_t(self.p, dev)
+        self.ro = None
+        if w.readout:
+            self.u = torch.from_numpy(gen.make_u(w)).to(dev)
+            o = torch.empty((w.B, w.L, w.H, w.n) + ((w.queries,) if w.queries else ()), dtype=torch.float32,
+                            device=dev)
+            snaps = (torch.empty((w.B, w.L // w.snapshot_every, w.H, w.n, w.n), dtype=torch.float32, device=dev)
+                     if w.snapshot_every else None)
+            self.ro = mru.Readout(self.u.data_ptr(), w.snapshot_every,
+                                  snaps.data_ptr() if snaps is not None else None, w.queries, 1 if w.queries else 0)
+            self.outs_dev = [o] + ([snaps] if snaps is not None else [])
+        else:
+            self.outs_dev = [torch.empty((w.B, w.L, w.H, w.n, w.n), dtype=torch.float32, device=dev)]
+        self.names = mru.kernel_names(self.p, w.readout)
+        self.launches = mru.launch_count(self.p, w.readout)
+
+    def step(self):
+        mru, o = self.mru, self.outs_dev[0]
+        if self.ro is not None:
+            rc = mru.scan_fused(self.p, self.x_dev.data_ptr(), None, self.ro, None, o.data_ptr(), self.ws.data_ptr(),
+                                self.ws.numel(), self.stream.cuda_stream)
+        else:
+            rc = mru.scan_fused(self.p, self.x_dev.data_ptr(), None, None, o.data_ptr(), None, self.ws.data_ptr(),
+                                self.ws.numel(), self.stream.cuda_stream)
+        if rc != mru.OK:
+            raise mru.MruError(rc, "mru_scan_fused")
+
+    def check_status(self, what):
+        st = self.mru.last_device_status(self.ws.data_ptr(), self.stream.cuda_stream)
+        if st != self.mru.OK:
+            raise self.mru.MruError(st, what)
+
+    def time_steps(self, steps, dev, clocks=None):
+        """Device time of `steps` calls (CUDA events on the launching
+        stream); workloads smaller than L2 get an L2 flush (a write of twice
+        its size) between steps, outside the per-step events."""
+        import torch
+        stream = self.stream
+        if step_bytes(self.w)["total"] > L2_BYTES:
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            for _ in range(steps):
+                self.step()
+            ev1.record(stream)
+            ev1.synchronize()
+            return ev0.elapsed_time(ev1) / steps
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for a, b in pairs:
+            flush.zero_()
+            a.record(stream)
+            self.step()
+            b.record(stream)
+        pairs[-1][1].synchronize()
+        return sum(a.elapsed_time(b) for a, b in pairs) / steps
+
+    def kernel_times(self, steps):
+        """Mean device time of each of the call's launches over `steps`
+        calls, from the library's event hook."""
+        import torch
+        n_k = self.launches
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_k)] for _ in range(steps)]
+        for row in evs:
+            for e in row:
+                e.record(self.stream)           # creates the handles
+        torch.cuda.synchronize()
+        for row in evs:
+            self.mru.set_profile_events([e.cuda_event for e in row])
+            self.step()
+        self.mru.set_profile_events(None)
+        torch.cuda.synchronize()
+        return [statistics.mean(row[2 * i].elapsed_time(row[2 * i + 1]) for row in evs) for i in range(n_k)]
+
+
+def roofline_entry(w, ms, per_kernel, names, chunk, peaks):
+    """The dominant kernel's roofline (algorithmic bytes of the whole step,
+    which that kernel's launch processes, over its launch time) and the whole
+    call's fraction of the step's roofline time."""
+    rl = roofline_min_ms(w, peaks)
+    dom = int(np.argmax(per_kernel))
+    dom_name = names[dom]
+    sb = step_bytes(w)
+    achieved = sb["total"] / (per_kernel[dom] / 1e3) / 1e9
+    whole = rl["min_ms"] / ms
+    roof = {"bound": rl["bound"], "kernel": dom_name, "achieved": achieved, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+            "frac_whole_call": whole,
+            "traffic": recorded_traffic(w.name, dom_name),
+            "algorithmic_bytes_per_launch": sb["total"], "avg_launch_ms": per_kernel[dom],
+            "kernel_own_bytes_per_launch": kernel_bytes(dom_name, w, chunk),
+            "flop_side": {"flops_per_step": rl["flop"]["flops_per_step"], "pipe": rl["flop"]["pipe"],
+                          "peak_tflops": round(rl["flop"]["peak_tflops"], 1),
+                          "achieved_tflops": rl["flop"]["flops_per_step"] / (ms / 1e3) / 1e12,
+                          "min_ms": rl["flop"]["min_ms"]},
+            "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] == "measured"
+            else "fallback 6.65 TB/s"}
+    path = {"algorithmic_bytes_per_step": sb["total"], "achieved_gbs": sb["total"] / (ms / 1e3) / 1e9,
+            "frac_of_hbm_peak": sb["total"] / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "roofline_ms": rl["min_ms"], "frac_of_roofline": whole}
+    return roof, path
+
+
+def measure_case(case, args, dev, clocks=None):
+    """Warm-up, the timed region (K steps), then the per-kernel split."""
+    for _ in range(args.warmup):
+        case.step()
+    case.check_status("device status after warm-up")
+    import torch
+    torch.cuda.synchronize()
+    ms = case.time_steps(args.steps, dev)
+    case.check_status("device status after timing")
+    per_kernel = case.kernel_times(min(args.steps, 10))
+    return ms, per_kernel
+
+
+def per_workload_lines(args, dev, stream, peaks, skip_name, skip_entry):
+    """Every workload the metric is quoted on, one entry each (rank 0 at
+    N = 1): step time, throughput, the whole call's fraction of its roofline,
+    the dominant kernel and its fraction, and the per-kernel split."""
+    import torch
+    out = {}
+    for name in BASELINE_WORKLOADS:
+        if name == skip_name:
+            out[name] = skip_entry
+            continue
+        w = gen.WORKLOADS[name]
+        case = Case(w, dev, stream)
+        ms, per_kernel = measure_case(case, args, dev)
+        roof, path = roofline_entry(w, ms, per_kernel, case.names, case.chunk, peaks)
+        out[name] = {"ms_per_step": ms, "value": w.token_heads / (ms / 1e3), "unit": UNIT,
+                     "frac_whole_call": roof["frac_whole_call"], "bound": roof["bound"],
+                     "dominant_kernel": roof["kernel"], "dominant_kernel_frac": roof["frac"],
+                     "roofline_ms": path["roofline_ms"], "chunk": case.chunk,
+                     "kernels_ms": {case.names[i]: round(per_kernel[i], 5) for i in range(len(per_kernel))}}
+        del case
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, w):
     import torch
 
@@ -372,8 +572,8 @@ def run_ours(args, w):
     barrier, max_over_ranks = ranks.barrier, ranks.max
 
     # CPU baseline first (rank 0, one GPU), before any CUDA work.
-    x_np = gen.make_x(w, seed=w.seed + rank)
     cpu = None
+    x_np = gen.make_x(w, seed=w.seed + rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
@@ -382,141 +582,44 @@ def run_ours(args, w):
         cpu = {"value": r, "unit": UNIT, "cores": nthreads, "kind": "oracle", "sample": sample,
                "seconds": round(el, 2)}
 
-    p = mru.problem_from_workload(w)
-    chunk = mru.chosen_chunk(p, w.readout)
     stream = torch.cuda.current_stream()
-    s_handle = stream.cuda_stream
-    if w.x_dtype == "bf16":
-        x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16)
-    else:
-        x_host = torch.from_numpy(x_np)
-    x_pin = x_host.pin_memory()
-    x_dev = x_pin.to(dev)
-    ws = mru.workspace_t(p, dev)
-    if w.readout:
-        u = torch.from_numpy(gen.make_u(w)).to(dev)
-        o = torch.empty((w.B, w.L, w.H, w.n) + ((w.queries,) if w.queries else ()), dtype=torch.float32,
-                        device=dev)
-        snaps = (torch.empty((w.B, w.L // w.snapshot_every, w.H, w.n, w.n), dtype=torch.float32, device=dev)
-                 if w.snapshot_every else None)
-        ro = mru.Readout(u.data_ptr(), w.snapshot_every, snaps.data_ptr() if snaps is not None else None,
-                         w.queries, 1 if w.queries else 0)
-        out_main = o
-        outs_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True)]
-        outs_dev = [o]
-        if snaps is not None:
-            outs_host.append(torch.empty(snaps.shape, dtype=snaps.dtype, pin_memory=True))
-            outs_dev.append(snaps)
-
-        def call(xd):
-            return mru.scan_fused(p, xd.data_ptr(), None, ro, None, o.data_ptr(), ws.data_ptr(), ws.numel(),
-                                  s_handle)
-    else:
-        S = torch.empty((w.B, w.L, w.H, w.n, w.n), dtype=torch.float32, device=dev)
-        out_main = S
-        outs_host = [torch.empty(S.shape, dtype=S.dtype, pin_memory=True)]
-        outs_dev = [S]
-
-        def call(xd):
-            return mru.scan_fused(p, xd.data_ptr(), None, None, S.data_ptr(), None, ws.data_ptr(), ws.numel(),
-                                  s_handle)
-
-    launches_per_step = mru.launch_count(p, w.readout)
-    names = mru.kernel_names(p, w.readout)
-
-    def step():
-        rc = call(x_dev)
-        if rc != mru.OK:
-            raise mru.MruError(rc, "mru_scan_fused")
-
-    # warm-up
+    case = Case(w, dev, stream, x_np=x_np)
+    del x_np
+    peaks = read_peaks()
     for _ in range(args.warmup):
-        step()
-    st = mru.last_device_status(ws.data_ptr(), s_handle)
-    if st != mru.OK:
-        raise mru.MruError(st, "device status after warm-up")
+        case.step()
+    case.check_status("device status after warm-up")
 
-    # timed region: exactly K steps, device-resident inputs.  Workloads
-    # smaller than L2 get an L2 flush (a write of twice its size) between
-    # steps, outside the per-step events.
-    flush = None
-    if step_bytes(w)["total"] <= L2_BYTES:
-        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    # timed region: exactly K steps, device-resident inputs
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        if flush is None:
-            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            ev0.record(stream)
-            for _ in range(args.steps):
-                step()
-            ev1.record(stream)
-            ev1.synchronize()
-            ms = ev0.elapsed_time(ev1) / args.steps
-        else:
-            pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                     for _ in range(args.steps)]
-            for a, b in pairs:
-                flush.zero_()
-                a.record(stream)
-                step()
-                b.record(stream)
-            pairs[-1][1].synchronize()
-            ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+        ms = case.time_steps(args.steps, dev)
     torch.cuda.synchronize()
     barrier()
     ms = max_over_ranks(ms)
     value = aggregate_rate(world, w.token_heads, ms)
+    case.check_status("device status after timing")
 
-    # per-kernel durations: the same K steps again with the library's event hook
-    n_k = launches_per_step
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_k)] for _ in range(args.steps)]
-    for row in evs:
-        for e in row:
-            e.record(stream)           # creates the handles
-    torch.cuda.synchronize()
-    for row in evs:
-        mru.set_profile_events([e.cuda_event for e in row])
-        step()
-    mru.set_profile_events(None)
-    torch.cuda.synchronize()
-    per_kernel = []
-    for i in range(n_k):
-        per_kernel.append(statistics.mean(row[2 * i].elapsed_time(row[2 * i + 1]) for row in evs))
-    dom = int(np.argmax(per_kernel))
-    dom_name = names[dom]
-    peaks = read_peaks()
-    # achieved: the path's algorithmic bytes per unit (embeddings in + results
-    # out) x the units one launch processes, over the kernel's launch time
-    sb = step_bytes(w)
-    dom_bytes = sb["total"]
-    achieved = dom_bytes / (per_kernel[dom] / 1e3) / 1e9
-    roofline = {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                "traffic": recorded_traffic(w.name, dom_name),
-                "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_ms": per_kernel[dom],
-                "kernel_own_bytes_per_launch": kernel_bytes(dom_name, w, chunk),
-                "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] == "measured"
-                else "fallback 6.65 TB/s"}
-    path = {"algorithmic_bytes_per_step": sb["total"], "achieved_gbs": sb["total"] / (ms / 1e3) / 1e9}
-    path["frac_of_hbm_peak"] = path["achieved_gbs"] / peaks["hbm_gbs"]
-    kernels_ms = {names[i]: round(per_kernel[i], 5) for i in range(n_k)}
+    per_kernel = case.kernel_times(min(args.steps, 10))
+    roofline, path = roofline_entry(w, ms, per_kernel, case.names, case.chunk, peaks)
+    kernels_ms = {case.names[i]: round(per_kernel[i], 5) for i in range(len(per_kernel))}
 
     # e2e: the C-ABI call with HOST buffers (mru_scan_fused_host): the upload
     # of x, the scan and the download of every output, pipelined over pieces
-    # of the batch on three streams, all inside the timed region
+    # on three streams, all inside the timed region
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    h2d = x_pin.numel() * x_pin.element_size()
+    outs_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in case.outs_dev]
+    h2d = case.x_pin.numel() * case.x_pin.element_size()
     d2h = sum(t.numel() * t.element_size() for t in outs_host)
     s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ro_h = ro if w.readout else None
     snaps_host = outs_host[1].data_ptr() if len(outs_host) > 1 else None
 
     def call_host():
-        rc = mru.scan_fused_host(p, x_pin.data_ptr(), None, ro_h, outs_host[0].data_ptr(), snaps_host,
-                                 x_dev.data_ptr(), outs_dev[0].data_ptr(), ws.data_ptr(), ws.numel(), 0,
-                                 s_handle, s_h2d.cuda_stream, s_d2h.cuda_stream)
+        rc = mru.scan_fused_host(case.p, case.x_pin.data_ptr(), None, case.ro, outs_host[0].data_ptr(), snaps_host,
+                                 case.x_dev.data_ptr(), case.outs_dev[0].data_ptr(), case.ws.data_ptr(),
+                                 case.ws.numel(), 0, stream.cuda_stream, s_h2d.cuda_stream, s_d2h.cuda_stream)
         if rc != mru.OK:
             raise mru.MruError(rc, "mru_scan_fused_host")
 
@@ -530,29 +633,44 @@ def run_ours(args, w):
     e1.record(stream)
     e1.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
-    st = mru.last_device_status(ws.data_ptr(), s_handle)
-    if st != mru.OK:
-        raise mru.MruError(st, "device status after timing")
+    case.check_status("device status after the end-to-end timing")
+    launches = case.launches
+    chunk = case.chunk
+    del case, outs_host
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    per_workload = None
+    if world == 1 and not args.no_per_workload:
+        head = {"ms_per_step": ms, "value": value, "unit": UNIT, "frac_whole_call": roofline["frac_whole_call"],
+                "bound": roofline["bound"], "dominant_kernel": roofline["kernel"],
+                "dominant_kernel_frac": roofline["frac"], "roofline_ms": path["roofline_ms"], "chunk": chunk,
+                "kernels_ms": kernels_ms}
+        per_workload = per_workload_lines(args, dev, stream, peaks, w.name, head)
 
     if rank == 0:
         cfg = workload_config(w, chunk)
+        clk = clocks.summary()
+        if clk.get("sm_mhz"):
+            clk["ms_x_sm_mhz"] = ms * clk["sm_mhz"]
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded N(0,1) embeddings)",
-            "config": cfg, "clocks": clocks.summary(),
+            "config": cfg, "clocks": clk,
             "e2e": {"value": aggregate_rate(world, w.token_heads, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                     "api": "mru_scan_fused_host (pinned host buffers; upload, scan and download "
-                           "pipelined over pieces of the batch on three streams)",
+                           "pipelined over pieces on three streams)",
                     "ms_per_step": e2e_ms},
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": launches * args.steps,
             "roofline": roofline, "path_roofline": path, "kernels_ms": kernels_ms,
         }
+        if per_workload is not None:
+            line["per_workload"] = per_workload
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
-    del out_main
     ranks.close()
     return 0
 
@@ -762,13 +880,15 @@ def run_decode(args, w):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(gen.WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the per_workload entries (the other configurations the metric is quoted on)")
     ap.add_argument("--backward", action="store_true", help="time mru_scan_backward instead (not the default)")
     ap.add_argument("--decode", action="store_true",
                     help="time single-token decode steps from S0 instead (not the default)")

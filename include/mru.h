@@ -259,12 +259,14 @@ mru_status mru_set_profile_events(void* const* events, int32_t count);
  * allocates nothing (no cudaMalloc, no cudaFree, no allocating library call).
  *
  *   - Size limit: with p->chunk == 0 the chunk is the library's choice,
- *     doubled until the workspace (mru_workspace_size) fits the scratch; a
+ *     doubled until the workspace this call needs (its output form and
+ *     readout layout; at most mru_workspace_size) fits the scratch; a
  *     problem that does not fit even then, or whose explicit p->chunk does not
  *     fit, is rejected with MRU_ERR_WORKSPACE before anything is launched.
- *   - Set-up: the first call on each device looks up the scratch's device
- *     address (cudaGetSymbolAddress, with that device current) and caches
- *     it; make that first call before any stream capture.
+ *   - Set-up: every call looks up the scratch's device address on the
+ *     current device (cudaGetSymbolAddress; nothing is cached, so the lookup
+ *     stays right after a device reset); the first call on a device also
+ *     loads the module there, so make it before any stream capture.
  *   - Sharing: every call on a device uses the same scratch, which keeps the
  *     last call's contents; the call clears what must start at zero itself.
  *     Calls whose executions overlap on the GPU (on different streams, or

@@ -207,6 +207,32 @@ mru_status reset_status(void* ws, cudaStream_t s)
 
 }  // namespace
 
+namespace {
+// Kernel parameters and workspace layout of one mru_scan_fused call: the
+// embedding source, and the readout's query columns when there is one.
+void fused_call_plan(const mru_problem& p, const mru_readout* ro, KParams& k, Workspace& W)
+{
+    k = make_params(p, SRC_EMBEDDING, ro != nullptr);
+    if (ro) {
+        k.rq = ro->q == 0 ? 1 : ro->q;
+        k.u_hs = ro->u_per_head ? (int64_t)p.n * k.rq : 0;
+    }
+    W = layout(k, ro != nullptr);
+}
+}  // namespace
+
+// Workspace bytes mru_scan_fused needs for this problem with this output
+// form (the readout's query-column count and per-head layout included);
+// 0 for an invalid problem.
+size_t fused_workspace_bytes(const mru_problem& p, const mru_readout* ro)
+{
+    if (check_problem(&p) != MRU_OK) return 0;
+    KParams k;
+    Workspace W;
+    fused_call_plan(p, ro, k, W);
+    return W.bytes;
+}
+
 void profile_mark(int kernel, int after, cudaStream_t s)
 {
     const int slot = 2 * kernel + after;
@@ -328,12 +354,9 @@ mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0, 
     } else {
         if (!S_out || !aligned16(S_out) || (const void*)S_out == x) return MRU_ERR_INVALID_ARG;
     }
-    KParams k = make_params(*p, SRC_EMBEDDING, ro != nullptr);
-    if (ro) {
-        k.rq = ro->q == 0 ? 1 : ro->q;
-        k.u_hs = ro->u_per_head ? (int64_t)p->n * k.rq : 0;
-    }
-    Workspace W = layout(k, ro != nullptr);
+    KParams k;
+    Workspace W;
+    fused_call_plan(*p, ro, k, W);
     if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = reset_status(ws, s)) != MRU_OK) return st;

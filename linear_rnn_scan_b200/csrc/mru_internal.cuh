@@ -137,6 +137,10 @@ struct BwdWorkspace {
 
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Workspace bytes mru_scan_fused needs for this problem and output form
+// (mru_api.cu); 0 for an invalid problem.
+size_t fused_workspace_bytes(const mru_problem& p, const mru_readout* ro);
+
 // Benchmark hook (mru_api.cu): records the caller's event for kernel slot
 // `kernel`, before (after = 0) or after (after = 1) its launch; no-op when
 // no events are registered.

@@ -4,7 +4,6 @@
 // every device allocation, or a service that reserves its whole memory budget
 // at start-up and forbids allocation afterwards).  Its scratch lives in one
 // fixed-size, file-scope __device__ array instead.
-#include <mutex>
 #include <string.h>
 
 #include "mru_internal.cuh"
@@ -15,27 +14,17 @@ namespace {
 // context loads this library holds these bytes until the process exits.
 __device__ __align__(256) unsigned char g_noalloc_scratch[MRU_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch per device.  In host code the symbol is
-// only a host-side stand-in, so the address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, and reused afterwards.
-constexpr int kMaxDevices = 128;
-void* g_scratch_addr[kMaxDevices] = {};
-std::mutex g_scratch_lock;
-
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the symbol is only a host-side stand-in, so the address is asked for with
+// cudaGetSymbolAddress, with the device current, on every call (a cheap
+// lookup); nothing is cached, so a context torn down and created again
+// (cudaDeviceReset) gets the address of its own copy of the array.
 cudaError_t scratch_address(void** out)
 {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> g(g_scratch_lock);
-    if (!g_scratch_addr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return cudaSuccess;
 }
 
@@ -46,24 +35,22 @@ extern "C" mru_status mru_scan_fused_noalloc(const mru_problem* p, const void* x
                                              uint32_t* status_out, void* stream)
 {
     using namespace mru;
-    // The same checks as mru_scan_fused, before any CUDA call.
     if (!p) return MRU_ERR_INVALID_ARG;
     mru_problem q = *p;
-    const size_t need_default = mru_workspace_size(&q);
-    if (need_default == 0) {
+    if (fused_workspace_bytes(q, ro) == 0) {
         // invalid problem: let the shared validation name the error
         return mru_scan_fused(&q, x, S0, ro, S_out, o_out, nullptr, 0, stream);
     }
     // Pick the chunk: the caller's, else the library's choice doubled until
-    // the workspace fits the fixed scratch.
+    // the workspace of this very call (its source, output form and readout
+    // layout) fits the fixed scratch.
     if (q.chunk == 0) {
         q.chunk = mru_chosen_chunk(&q, ro != nullptr);
-        while (mru_workspace_size(&q) > MRU_NOALLOC_SCRATCH_BYTES && (int64_t)q.chunk < q.L &&
+        while (fused_workspace_bytes(q, ro) > MRU_NOALLOC_SCRATCH_BYTES && (int64_t)q.chunk < q.L &&
                q.chunk < (1 << 30))
             q.chunk *= 2;
     }
-    const size_t need = mru_workspace_size(&q);
-    if (need > MRU_NOALLOC_SCRATCH_BYTES) return MRU_ERR_WORKSPACE;
+    if (fused_workspace_bytes(q, ro) > MRU_NOALLOC_SCRATCH_BYTES) return MRU_ERR_WORKSPACE;
     if (status_out && (reinterpret_cast<uintptr_t>(status_out) & 3u)) return MRU_ERR_INVALID_ARG;
 
     void* ws = nullptr;

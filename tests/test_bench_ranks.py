@@ -176,3 +176,26 @@ def test_reference_arm_line_on_rank_0(monkeypatch, capsys):
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_roofline_sides_of_the_quoted_workloads():
+    """Both sides of the step roofline for the five workloads the metric is
+    quoted on: bytes at the HBM peak and 2 n^3 scan FLOPs per token-head at
+    the peak of the pipe the products use (tf32 for n = 16 and 64, bf16 for
+    the n = 32 LDU path); HBM binds every one of them."""
+    from linear_rnn_scan_b200 import inputs as gen
+    peaks = {"hbm_gbs": 6549.4, "bf16_tflops": 1657.1, "bf16_tflops_sustained": 1394.4, "source": "measured"}
+    assert len(bench.BASELINE_WORKLOADS) == 5
+    assert bench.DEFAULT_WORKLOAD in bench.BASELINE_WORKLOADS
+    for name in bench.BASELINE_WORKLOADS:
+        w = gen.WORKLOADS[name]
+        r = bench.roofline_min_ms(w, peaks)
+        assert r["flop"]["flops_per_step"] == 2 * w.n ** 3 * w.token_heads
+        assert r["bound"] == "hbm", (name, r)
+        assert abs(r["hbm_min_ms"] - bench.step_bytes(w)["total"] / 6549.4e9 * 1e3) < 1e-12
+    w2 = gen.WORKLOADS["n16_detnorm_b8h8l4096"]
+    assert abs(bench.roofline_min_ms(w2, peaks)["min_ms"] - 536870912 / 6549.4e9 * 1e3) < 1e-9
+    w5 = gen.WORKLOADS["n64_detnorm_readout_b2h4l16384"]
+    f5 = bench.flop_side(w5, peaks)
+    assert f5["pipe"].startswith("tf32") and abs(f5["peak_tflops"] - 1657.1 * 1.1 / 2.25) < 1e-6
+    assert bench.flop_side(gen.WORKLOADS["n32_ldu_bf16_b4h16l8192"], peaks)["pipe"].startswith("bf16")

@@ -3,12 +3,14 @@ device memory (a plugin inside a framework that owns every device
 allocation, a service that reserves its memory budget at start-up).  Its
 scratch is the library's fixed device array instead of a caller workspace.
 
-The GPU test calls it through the C-ABI twice in a row, on two different
-inputs, and checks each result against mru_scan_fused (which uses a caller
-workspace) on the same input, within the fp32 relative Frobenius gate of the
-other parity tests.  The second call shows that nothing the first call left
-in the shared scratch leaks into the next result.  This file is collected
-last on purpose.
+The GPU tests call it through the C-ABI twice in a row, on two different
+inputs, and check each result against the fp64 oracle and against
+mru_scan_fused (which uses a caller workspace) on the same input, within the
+fp32 relative Frobenius gate of the other parity tests.  The second call
+shows that nothing the first call left in the shared scratch leaks into the
+next result.  One case is too large for the scratch at the library's chunk:
+the entry point doubles the chunk, and its result equals mru_scan_fused's at
+that chunk bit for bit.  This file is collected last on purpose.
 """
 import numpy as np
 import pytest
@@ -16,7 +18,7 @@ import pytest
 from linear_rnn_scan_b200 import inputs as gen
 from linear_rnn_scan_b200 import mru
 
-from gpu_helpers import TOL_FP32, to_device_x, torch
+from gpu_helpers import TOL_FP32, compare_S, to_device_x, torch
 
 
 def _rel_frobenius(a, b):
@@ -47,6 +49,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
         got, ref = S.cpu().numpy(), S_ref.cpu().numpy()
         assert np.isfinite(got).all()
         assert _rel_frobenius(got, ref) <= TOL_FP32
+        e = compare_S(w, gen.make_x(w, seed=seed), got)            # and against the oracle directly
+        assert e["count"] == w.B * w.L * w.H and e["max"] <= TOL_FP32, e
 
     # the readout form, twice as well (o_t = S_t u and snapshots)
     wr = w.with_(readout=True, snapshot_every=32)
@@ -64,6 +68,43 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
         rel_o = np.linalg.norm(o_h - or_h, axis=-1) / np.linalg.norm(or_h, axis=-1)
         assert float(rel_o.max()) <= TOL_FP32
         assert _rel_frobenius(sn.cpu().numpy(), sn_ref.cpu().numpy()) <= TOL_FP32
+
+
+@pytest.mark.gpu
+def test_noalloc_doubles_the_chunk_when_the_default_does_not_fit():
+    """B4 H8 L4096, n = 16: at the library's chunk (16 tokens, 8192 chains)
+    the call's own workspace is about 17 MB, above the 16 MiB scratch.  The
+    entry point doubles the chunk until it fits, so its result equals
+    mru_scan_fused run with that chunk exactly (same kernels, same chunking),
+    and the oracle within the fp32 gate; twice in a row."""
+    t = torch()
+    if not t.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    w = gen.Workload("noalloc_big", B=4, H=8, L=4096, n=16, x_dtype="f32", mode=gen.MODE_DETNORM,
+                     alpha=0.05 / 4, seed=9005)
+    p = mru.problem_from_workload(w)
+    c0 = mru.chosen_chunk(p)
+    assert mru.workspace_size(mru.problem_from_workload(w, chunk=c0)) > mru.NOALLOC_SCRATCH_BYTES
+    stream = t.cuda.current_stream().cuda_stream
+    for seed in (9005, 9006):
+        x_np = gen.make_x(w, seed=seed)
+        x = to_device_x(x_np)
+        S = t.full((w.B, w.L, w.H, 16, 16), float("nan"), device="cuda")
+        status = t.full((1,), 7, dtype=t.int32, device="cuda")
+        rc = mru.scan_fused_noalloc(p, x.data_ptr(), None, None, S.data_ptr(), None, status.data_ptr(), stream)
+        assert rc == mru.OK, mru.status_string(rc)
+        t.cuda.synchronize()
+        assert int(status.item()) == 0
+        got = S.cpu().numpy()
+        used = None
+        for c in (2 * c0, 4 * c0, 8 * c0):
+            ref = mru.scan_fused_t(mru.problem_from_workload(w, chunk=c), x).cpu().numpy()
+            if np.array_equal(got, ref):
+                used = c
+                break
+        assert used is not None, "no doubled chunk reproduces the no-alloc result"
+        e = compare_S(w, x_np, got)
+        assert e["count"] == w.B * w.L * w.H and e["max"] <= TOL_FP32, e
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch():
