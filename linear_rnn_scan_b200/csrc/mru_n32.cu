@@ -100,10 +100,18 @@ __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v 
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
 // Split a pair of fp32 values into bf16 hi and lo parts (x ~ hi + lo).
+// PK: the residual by one packed subtraction (same values).
+template <bool PK = true>
 __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo)
 {
     hi = pack_bf16(x0, x1);
-    lo = pack_bf16(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
+    if (PK) {
+        float r0, r1;
+        f2::up(f2::sub(f2::pk(x0, x1), f2::pk(bf16_lo(hi), bf16_hi(hi))), r0, r1);
+        lo = pack_bf16(r0, r1);
+    } else {
+        lo = pack_bf16(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
+    }
 }
 
 // The state: 32 x 32 fp32 in accumulator layout, st[mt][nt][i] holds
@@ -112,16 +120,17 @@ using State = float[2][4][4];
 
 // A fragments (hi, lo) of the state: the accumulator tile (mt, 2 kt) and
 // (mt, 2 kt + 1) are exactly the A fragment (mt, kt) of m16n8k16.
+template <bool PK = true>
 __device__ __forceinline__ void state_frags(const State& st, uint32_t (&ah)[2][2][4], uint32_t (&al)[2][2][4])
 {
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
         for (int kt = 0; kt < 2; ++kt) {
-            split_pair(st[mt][2 * kt][0], st[mt][2 * kt][1], ah[mt][kt][0], al[mt][kt][0]);
-            split_pair(st[mt][2 * kt][2], st[mt][2 * kt][3], ah[mt][kt][1], al[mt][kt][1]);
-            split_pair(st[mt][2 * kt + 1][0], st[mt][2 * kt + 1][1], ah[mt][kt][2], al[mt][kt][2]);
-            split_pair(st[mt][2 * kt + 1][2], st[mt][2 * kt + 1][3], ah[mt][kt][3], al[mt][kt][3]);
+            split_pair<PK>(st[mt][2 * kt][0], st[mt][2 * kt][1], ah[mt][kt][0], al[mt][kt][0]);
+            split_pair<PK>(st[mt][2 * kt][2], st[mt][2 * kt][3], ah[mt][kt][1], al[mt][kt][1]);
+            split_pair<PK>(st[mt][2 * kt + 1][0], st[mt][2 * kt + 1][1], ah[mt][kt][2], al[mt][kt][2]);
+            split_pair<PK>(st[mt][2 * kt + 1][2], st[mt][2 * kt + 1][3], ah[mt][kt][3], al[mt][kt][3]);
         }
 }
 
@@ -166,6 +175,11 @@ __device__ __forceinline__ void load_mt_frags(const unsigned char* xs, int lane,
 // or k < n (upper).  c = 16 kt + 8 h - 8 nt is the tile offset, d = 2 q - g.
 __device__ __forceinline__ uint32_t tri_mask(uint32_t v, int c, int d, bool lower)
 {
+    // k - n = c + d (+ 1) with |d| <= 7 and c a multiple of 8: off the
+    // diagonal 8 x 8 blocks every entry of the register has the sign of c
+    // (c is a compile-time constant at every use, so these fold away)
+    if (c >= 8) return lower ? v : 0u;
+    if (c <= -8) return lower ? 0u : v;
     const int lo_kn = c + d, hi_kn = c + d + 1;    // k - n of the two halves
     const bool keep_lo = lower ? lo_kn > 0 : lo_kn < 0;
     const bool keep_hi = lower ? hi_kn > 0 : hi_kn < 0;
@@ -202,9 +216,12 @@ __device__ __forceinline__ void tri_product(const uint32_t (&ah)[2][2][4], const
 __device__ __forceinline__ void split_pair3(float x0, float x1, uint32_t& hi, uint32_t& mid, uint32_t& lo)
 {
     hi = pack_bf16(x0, x1);
-    const float r0 = x0 - bf16_lo(hi), r1 = x1 - bf16_hi(hi);
+    const uint64_t r = f2::sub(f2::pk(x0, x1), f2::pk(bf16_lo(hi), bf16_hi(hi)));
+    float r0, r1;
+    f2::up(r, r0, r1);
     mid = pack_bf16(r0, r1);
-    lo = pack_bf16(r0 - bf16_lo(mid), r1 - bf16_hi(mid));
+    f2::up(f2::sub(r, f2::pk(bf16_lo(mid), bf16_hi(mid))), r0, r1);
+    lo = pack_bf16(r0, r1);
 }
 
 // A fragments (hi, mid, lo) of the state, as state_frags.
@@ -290,6 +307,7 @@ __device__ __forceinline__ void apply_token_f(State& st, const uint32_t (&bm)[2]
                                               const float* Dv, const float* Dm1, float a, int lane)
 {
     const int g = lane >> 2, q = lane & 3, d = 2 * q - g;
+    constexpr bool PK = SPLIT || TERMS == 3;
     uint32_t ah[2][2][4], al[2][2][4];
     State acc;
     auto product = [&](auto lower_tag) {
@@ -299,50 +317,79 @@ __device__ __forceinline__ void apply_token_f(State& st, const uint32_t (&bm)[2]
             state_frags3(st, ah, am, al);
             tri_product3<LOWER>(ah, am, al, bm, d, acc);
         } else {
-            state_frags(st, ah, al);
+            state_frags<PK>(st, ah, al);
             tri_product<LOWER>(ah, al, bm, d, acc);
         }
     };
+    // The element updates run on packed pairs (columns 2 q, 2 q + 1 of a
+    // row), with the scalar rounding of every operation: fewer issue slots
+    // for the split-form reduce chain and the backward's three-term chains;
+    // the forward apply pass, bound by memory, keeps the scalar form
+    // (measured on B200: packed there made it 4 % slower).
+    const uint64_t a2 = f2::pk(a, a);
+    auto update = [&](auto lower_tag) {
+        constexpr bool LOWER = decltype(lower_tag)::value;
+        if constexpr (!PK) {
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) st[mt][nt][i] += a * acc[mt][nt][i];
+            return;
+        }
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    // 8 x 8 block (2 mt + h, nt): below, above or on the diagonal
+                    const int R = 2 * mt + h;
+                    float t[2];
+#pragma unroll
+                    for (int s2 = 0; s2 < 2; ++s2) {
+                        const int cs = 2 * q + s2;
+                        const float m = md[mt][nt][2 * h + s2];
+                        t[s2] = LOWER ? (R > nt ? m : R < nt ? 0.0f : (g > cs ? m : 0.0f))
+                                      : (R < nt ? m : R > nt ? 0.0f : (g < cs ? m : 0.0f));
+                    }
+                    const uint64_t ac = f2::pk(acc[mt][nt][2 * h], acc[mt][nt][2 * h + 1]);
+                    const uint64_t sv = f2::pk(st[mt][nt][2 * h], st[mt][nt][2 * h + 1]);
+                    f2::up(f2::fma(a2, SPLIT ? f2::add(f2::pk(t[0], t[1]), ac) : ac, sv), st[mt][nt][2 * h],
+                           st[mt][nt][2 * h + 1]);
+                }
+    };
     // --- P L ---
     product(std::true_type{});
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                // 8 x 8 block (2 mt + i / 2, nt): below, above or on the diagonal
-                const int R = 2 * mt + (i >> 1), cs = 2 * q + (i & 1);
-                const float ls = R > nt ? md[mt][nt][i] : R < nt ? 0.0f : (g > cs ? md[mt][nt][i] : 0.0f);
-                st[mt][nt][i] += a * ((SPLIT ? ls : 0.0f) + acc[mt][nt][i]);
-            }
+    update(std::true_type{});
     // --- (P L) D ---
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
         const float2 dv = *reinterpret_cast<const float2*>(Dv + 8 * nt + 2 * q);
         const float2 dm = *reinterpret_cast<const float2*>(Dm1 + 8 * nt + 2 * q);
+        const uint64_t dv2 = f2::pk(dv.x, dv.y);
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int R = 2 * mt + (i >> 1), cs = 2 * q + (i & 1);
-                float v = st[mt][nt][i] * ((i & 1) ? dv.y : dv.x);
-                if (SPLIT && R == nt && g == cs) v += (i & 1) ? dm.y : dm.x;
-                st[mt][nt][i] = v;
+            for (int h = 0; h < 2; ++h) {
+                const int R = 2 * mt + h;
+                float v0, v1;
+                if (PK) {
+                    f2::up(f2::mul(f2::pk(st[mt][nt][2 * h], st[mt][nt][2 * h + 1]), dv2), v0, v1);
+                } else {
+                    v0 = st[mt][nt][2 * h] * dv.x;
+                    v1 = st[mt][nt][2 * h + 1] * dv.y;
+                }
+                if (SPLIT && R == nt && g == 2 * q) v0 += dm.x;
+                if (SPLIT && R == nt && g == 2 * q + 1) v1 += dm.y;
+                st[mt][nt][2 * h] = v0;
+                st[mt][nt][2 * h + 1] = v1;
             }
     }
     // --- (P L D) U ---
     product(std::false_type{});
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int R = 2 * mt + (i >> 1), cs = 2 * q + (i & 1);
-                const float us = R < nt ? md[mt][nt][i] : R > nt ? 0.0f : (g < cs ? md[mt][nt][i] : 0.0f);
-                st[mt][nt][i] += a * ((SPLIT ? us : 0.0f) + acc[mt][nt][i]);
-            }
+    update(std::false_type{});
 }
 
 // One token applied to the state (forward: the state times X = L D U).
