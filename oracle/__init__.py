@@ -75,6 +75,9 @@ def _load():
             lib.mro_compare.restype = ctypes.c_int
             lib.mro_backward.argtypes = [P(Problem), vp, dp, dp, dp, dp, ctypes.c_int]
             lib.mro_backward.restype = ctypes.c_int
+            lib.mro_backward_readout.argtypes = [P(Problem), vp, dp, dp, ci, ci, dp, ctypes.c_int64, dp, dp, dp,
+                                                 ci]
+            lib.mro_backward_readout.restype = ctypes.c_int
             lib.mro_bf16_to_double.argtypes = [ctypes.c_uint16]
             lib.mro_bf16_to_double.restype = ctypes.c_double
             _lib = lib
@@ -149,6 +152,29 @@ def backward(p: Problem, x: np.ndarray, dS: np.ndarray, S0: np.ndarray | None = 
                               _ptr(dS, ctypes.c_double), _ptr(dx, ctypes.c_double), _ptr(dS0, ctypes.c_double),
                               nthreads or os.cpu_count() or 1)
     _raise(rc, "backward")
+    return dx, dS0
+
+
+def backward_readout(p: Problem, x: np.ndarray, u: np.ndarray, d_o: np.ndarray, snapshot_every: int = 0,
+                     d_snap: np.ndarray | None = None, S0: np.ndarray | None = None, nthreads: int = 0):
+    """Vector-Jacobian product of the readout form: (dx [B, L, H*n*n], dS0
+    [B, H, n, n] or None) from the gradients of o_t = S_t U (d_o shaped like
+    o: [B, L, H, n] for one vector u, [B, L, H, n, q] for query columns) and
+    of the snapshots (d_snap [B, L//every, H, n, n] or None), fp64."""
+    x = _check_x(p, x)
+    U, q, per_head = query_columns(p, u)
+    d_o = np.ascontiguousarray(d_o, np.float64).reshape(p.B, p.L, p.H, p.n, q)
+    if d_snap is not None:
+        d_snap = np.ascontiguousarray(d_snap, np.float64).reshape(p.B, p.L // snapshot_every, p.H, p.n, p.n)
+    S0 = None if S0 is None else np.ascontiguousarray(S0, np.float64).reshape(p.B, p.H, p.n, p.n)
+    dx = np.empty((p.B, p.L, p.H * p.n * p.n), np.float64)
+    dS0 = None if S0 is None else np.empty((p.B, p.H, p.n, p.n), np.float64)
+    rc = _load().mro_backward_readout(ctypes.byref(p), x.ctypes.data, _ptr(S0, ctypes.c_double),
+                                      _ptr(U, ctypes.c_double), q, per_head, _ptr(d_o, ctypes.c_double),
+                                      int(snapshot_every if d_snap is not None else 0),
+                                      _ptr(d_snap, ctypes.c_double), _ptr(dx, ctypes.c_double),
+                                      _ptr(dS0, ctypes.c_double), nthreads or os.cpu_count() or 1)
+    _raise(rc, "backward_readout")
     return dx, dS0
 
 

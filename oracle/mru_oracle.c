@@ -618,17 +618,60 @@ static int lift_vjp(const mro_problem* p, const void* x, int64_t b, int64_t t, i
     return MRO_ERR_ARG;
 }
 
-/* Backward of one (b, h) sequence.  dS: [B,L,H,n,n]; dx: [B,L,H*n*n];
- * dS0: [B,H,n,n] or NULL.  Holds every X_t and S_t of the sequence. */
+/* Upstream gradient of the readout form: o_t = S_t U (and the snapshots
+ * S_t at 1-based t = k * every) are the outputs, so
+ *   dL/dS_t = do_t U^T  (+ dP_k when t = k * every),
+ * with U the head's [n, q] query columns.  Written for position t (0-based)
+ * of sequence (b, h) into G. */
+typedef struct {
+    const double* u;        /* [n, q], or [H, n, q] with u_per_head */
+    int q, u_per_head;
+    const double* d_o;      /* [B, L, H, n, q] */
+    int64_t snap_every;     /* 0: no snapshots */
+    const double* d_snap;   /* [B, L/every, H, n, n] or NULL */
+} readout_grad_t;
+
+static void readout_dS(const mro_problem* p, const readout_grad_t* R, int64_t b, int64_t t, int64_t h,
+                       double* G)
+{
+    const int n = p->n, q = R->q;
+    const double* U = R->u + (R->u_per_head ? h * n * q : 0);
+    const double* dO = R->d_o + ((b * p->L + t) * p->H + h) * (int64_t)n * q;
+    for (int i = 0; i < n; ++i)
+        for (int j = 0; j < n; ++j) {
+            double a = 0.0;                       /* (do_t U^T)_ij = sum_c do_t[i][c] U[j][c] */
+            for (int c = 0; c < q; ++c) a += dO[i * q + c] * U[j * q + c];
+            G[i * n + j] = a;
+        }
+    if (R->snap_every > 0 && R->d_snap && (t + 1) % R->snap_every == 0) {
+        const int64_t L_s = p->L / R->snap_every, k = (t + 1) / R->snap_every - 1;
+        const double* dP = R->d_snap + ((b * L_s + k) * p->H + h) * (int64_t)n * n;
+        for (int e = 0; e < n * n; ++e) G[e] += dP[e];
+    }
+}
+
+/* dL/dS_t for position t: from the dense array dS, or from the readout's
+ * gradients. */
+static void upstream(const mro_problem* p, const double* dS, const readout_grad_t* R, int64_t b, int64_t t,
+                     int64_t h, double* G)
+{
+    const int64_t nn = (int64_t)p->n * p->n;
+    if (R) readout_dS(p, R, b, t, h, G);
+    else memcpy(G, dS + ((b * p->L + t) * p->H + h) * nn, (size_t)nn * sizeof(double));
+}
+
+/* Backward of one (b, h) sequence.  dS: [B,L,H,n,n] (or, with R, the
+ * readout's gradients); dx: [B,L,H*n*n]; dS0: [B,H,n,n] or NULL.  Holds
+ * every X_t and S_t of the sequence. */
 static int backward_sequence(const mro_problem* p, const void* x, const double* S0, const double* dS,
-                             double* dx, double* dS0, int64_t bh)
+                             const readout_grad_t* R, double* dx, double* dS0, int64_t bh)
 {
     const int n = p->n;
     const int64_t nn = (int64_t)n * n, L = p->L;
     const int64_t b = bh / p->H, h = bh % p->H;
     double* X = malloc(sizeof(double) * (size_t)(L * nn + 1));
     double* S = malloc(sizeof(double) * (size_t)((L + 1) * nn));
-    double* work = malloc(sizeof(double) * (size_t)(12 * nn));    /* 5 n*n here + 7 n*n for lift_vjp */
+    double* work = malloc(sizeof(double) * (size_t)(13 * nn));    /* 6 n*n here + 7 n*n for lift_vjp */
     int rc = MRO_OK;
     if (!X || !S || !work) { rc = MRO_ERR_ARG; goto done; }
     /* forward: S[0] = S0 (or I), S[t+1] = S[t] X_{t+1} */
@@ -644,16 +687,17 @@ static int backward_sequence(const mro_problem* p, const void* x, const double* 
     double* Xt = work + 2 * nn;
     double* dX = work + 3 * nn;
     double* St = work + 4 * nn;
-    if (L > 0) memcpy(G, dS + ((b * L + (L - 1)) * p->H + h) * nn, (size_t)nn * sizeof(double));
+    double* ds = work + 5 * nn;
+    if (L > 0) upstream(p, dS, R, b, L - 1, h, G);
     for (int64_t t = L - 1; t >= 0; --t) {
         transpose(n, S + t * nn, St);                 /* S_{t-1}^T (position t holds X_{t+1}) */
         matmul(n, St, G, dX);
-        if ((rc = lift_vjp(p, x, b, t, h, dX, dx + ((b * L + t) * p->H + h) * nn, work + 5 * nn)) != MRO_OK)
+        if ((rc = lift_vjp(p, x, b, t, h, dX, dx + ((b * L + t) * p->H + h) * nn, work + 6 * nn)) != MRO_OK)
             goto done;
         transpose(n, X + t * nn, Xt);
         matmul(n, G, Xt, Gn);                         /* G_t X_t^T */
         if (t > 0) {
-            const double* ds = dS + ((b * L + (t - 1)) * p->H + h) * nn;
+            upstream(p, dS, R, b, t - 1, h, ds);
             for (int64_t e = 0; e < nn; ++e) G[e] = ds[e] + Gn[e];
         } else if (dS0) {
             memcpy(dS0 + bh * nn, Gn, (size_t)nn * sizeof(double));
@@ -672,6 +716,7 @@ typedef struct {
     const void* x;
     const double* S0;
     const double* dS;
+    const readout_grad_t* R;
     double* dx;
     double* dS0;
     int64_t next;
@@ -687,7 +732,7 @@ static void* bwd_worker(void* arg)
         const int64_t i = J->next++;
         pthread_mutex_unlock(&J->lock);
         if (i >= J->p->B * J->p->H) break;
-        const int rc = backward_sequence(J->p, J->x, J->S0, J->dS, J->dx, J->dS0, i);
+        const int rc = backward_sequence(J->p, J->x, J->S0, J->dS, J->R, J->dx, J->dS0, i);
         if (rc != MRO_OK) {
             pthread_mutex_lock(&J->lock);
             J->status = rc;
@@ -707,6 +752,33 @@ int mro_backward(const mro_problem* p, const void* x, const double* S0, const do
     bwd_job_t J;
     memset(&J, 0, sizeof J);
     J.p = p; J.x = x; J.S0 = S0; J.dS = dS; J.dx = dx; J.dS0 = dS0;
+    pthread_mutex_init(&J.lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    pthread_t th[256];
+    if (nthreads > 256) nthreads = 256;
+    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, bwd_worker, &J);
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    pthread_mutex_destroy(&J.lock);
+    return J.status;
+}
+
+/* Backward of the readout form: dx [B,L,H*n*n] and dS0 [B,H,n,n] (may be
+ * NULL) from the gradients of the readout outputs, d_o [B,L,H,n,q] (with o_t
+ * = S_t U, U [n,q] or [H,n,q] when u_per_head) and d_snap [B,L/every,H,n,n]
+ * of the snapshots S_t at 1-based t = k * every (NULL or every == 0: none).
+ * The chain rule of o_t = S_t U gives dL/dS_t = do_t U^T, then the scan's
+ * backward as in mro_backward. */
+int mro_backward_readout(const mro_problem* p, const void* x, const double* S0, const double* u, int q,
+                         int u_per_head, const double* d_o, int64_t snap_every, const double* d_snap,
+                         double* dx, double* dS0, int nthreads)
+{
+    if (check_problem(p) != MRO_OK || !u || q < 1 || !d_o || !dx || snap_every < 0) return MRO_ERR_ARG;
+    if (p->mode == 2 && p->n > 512) return MRO_ERR_ARG;
+    readout_grad_t R;
+    R.u = u; R.q = q; R.u_per_head = u_per_head; R.d_o = d_o; R.snap_every = snap_every; R.d_snap = d_snap;
+    bwd_job_t J;
+    memset(&J, 0, sizeof J);
+    J.p = p; J.x = x; J.S0 = S0; J.R = &R; J.dx = dx; J.dS0 = dS0;
     pthread_mutex_init(&J.lock, NULL);
     if (nthreads < 1) nthreads = 1;
     pthread_t th[256];

@@ -102,3 +102,54 @@ def test_backward_bf16_equals_widened_f32():
         pf = oracle.make_problem(B, H, L, n, x_dtype="f32", mode=mode, alpha=0.2)
         assert np.array_equal(oracle.backward(pb, bits, dS, nthreads=1)[0],
                               oracle.backward(pf, widened, dS, nthreads=1)[0])
+
+
+def _J_readout(p, x, S0, u, d_o, every, d_snap):
+    o, snaps = oracle.readout(p, x, u, snapshot_every=every, S0=S0, nthreads=1)
+    j = float(np.sum(o * d_o))
+    if every:
+        j += float(np.sum(snaps * d_snap))
+    return j
+
+
+@pytest.mark.parametrize("mode,n,add_identity,alpha,ushape,every", [
+    (oracle.MODE_RESHAPE, 3, 1, 0.3, "vector", 2),
+    (oracle.MODE_DETNORM, 3, 1, 0.25, "shared", 3),
+    (oracle.MODE_LDU, 3, 1, 1.0, "per_head", 2),
+    (oracle.MODE_CAYLEY, 3, 1, 0.6, "shared", 0),
+])
+def test_backward_readout_matches_finite_differences(mode, n, add_identity, alpha, ushape, every):
+    """The readout form's VJP (gradients of o_t = S_t U and of the snapshots
+    given, no state stored) against central finite differences of
+    J = sum_t <do_t, o_t> + sum_k <dP_k, P_k> computed with the oracle's
+    readout forward, with respect to every embedding value and to S0."""
+    rng = np.random.default_rng(70 + 5 * mode + n)
+    B, H, L = 1, 2, 6
+    p = oracle.make_problem(B, H, L, n, mode=mode, alpha=alpha, add_identity=add_identity,
+                            ldu_offdiag=0.3, ldu_diag=0.5)
+    x = _dyadic(rng, (B, L, H * n * n), lim=1.0)
+    S0 = np.eye(n)[None, None] + 0.3 * rng.standard_normal((B, H, n, n))
+    q = 2
+    u = {"vector": rng.standard_normal(n), "shared": rng.standard_normal((n, q)),
+         "per_head": rng.standard_normal((H, n, q))}[ushape]
+    o, _ = oracle.readout(p, x, u, S0=S0, nthreads=1)
+    d_o = rng.standard_normal(o.shape)
+    d_snap = rng.standard_normal((B, L // every, H, n, n)) if every else None
+    dx, dS0 = oracle.backward_readout(p, x, u, d_o, snapshot_every=every, d_snap=d_snap, S0=S0, nthreads=1)
+    h = 2.0 ** -11
+    worst, scale = 0.0, np.abs(dx).max()
+    for idx in np.ndindex(x.shape):
+        def f(e, idx=idx):
+            xe = x.copy()
+            xe[idx] = np.float32(x[idx] + e)
+            return _J_readout(p, xe, S0, u, d_o, every, d_snap)
+        worst = max(worst, abs(_fd(f, h) - dx[idx]) / scale)
+    assert worst < 1e-7, worst
+    worst, scale = 0.0, np.abs(dS0).max()
+    for idx in np.ndindex(S0.shape):
+        def g(e, idx=idx):
+            Se = S0.copy()
+            Se[idx] += e
+            return _J_readout(p, x, Se, u, d_o, every, d_snap)
+        worst = max(worst, abs(_fd(g, 1e-4) - dS0[idx]) / scale)
+    assert worst < 1e-8, worst
