@@ -697,9 +697,7 @@ def run_backward(args, w):
     from linear_rnn_scan_b200 import mru
 
     if w.readout:
-        print(json.dumps({"impl": "ours", "direction": "backward", "unavailable":
-                          "the backward covers the full-state output, not the readout"}), flush=True)
-        return 0
+        return run_backward_readout(args, w)
     local = env_int("LOCAL_RANK", 0)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -771,6 +769,88 @@ def run_backward(args, w):
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                          "algorithmic_bytes_per_launch": unit_bytes * w.token_heads}}), flush=True)
+    ranks.close()
+    return 0
+
+
+def run_backward_readout(args, w):
+    """One step = one mru_scan_backward_readout over the whole workload: the
+    gradients of the readout outputs (o_t = S_t U, and the snapshots) to the
+    embeddings, no forward state kept by the caller (the call recomputes the
+    states in its workspace).  Not part of the default run."""
+    import torch
+
+    from linear_rnn_scan_b200 import mru
+
+    local = env_int("LOCAL_RANK", 0)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks("nccl", dev)
+    p = mru.problem_from_workload(w)
+    x_np = gen.make_x(w, seed=w.seed + ranks.rank)
+    if w.x_dtype == "bf16":
+        x = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(dev)
+    else:
+        x = torch.from_numpy(x_np).to(dev)
+    del x_np
+    u = torch.from_numpy(gen.make_u(w)).to(dev)
+    q = max(w.queries, 1)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 17)
+    d_o = torch.randn((w.B, w.L, w.H, w.n, q), generator=g, device=dev, dtype=torch.float32)
+    d_sn = (torch.randn((w.B, w.L // w.snapshot_every, w.H, w.n, w.n), generator=g, device=dev,
+                        dtype=torch.float32) if w.snapshot_every else None)
+    dx = torch.empty((w.B, w.L, w.H * w.n * w.n), dtype=torch.float32, device=dev)
+    ws = torch.empty(mru.backward_readout_workspace_size(p), dtype=torch.uint8, device=dev)
+    ro = mru.Readout(u.data_ptr(), w.snapshot_every, None, w.queries, 1 if w.queries else 0)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        rc = mru.scan_backward_readout(p, x.data_ptr(), None, ro, d_o.data_ptr(),
+                                       d_sn.data_ptr() if d_sn is not None else None, dx.data_ptr(), None,
+                                       ws.data_ptr(), ws.numel(), stream.cuda_stream)
+        if rc != mru.OK:
+            raise mru.MruError(rc, "mru_scan_backward_readout")
+
+    for _ in range(args.warmup):
+        step()
+    st = mru.last_device_status(ws.data_ptr(), stream.cuda_stream)
+    if st != mru.OK:
+        raise mru.MruError(st, "device status after warm-up")
+    torch.cuda.synchronize()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        ev1.synchronize()
+    torch.cuda.synchronize()
+    ranks.barrier()
+    ms = ranks.max(ev0.elapsed_time(ev1) / args.steps)
+    # algorithmic bytes per token-head: x in, the readout gradient in, dx out
+    nn = w.n * w.n
+    xb = 2 if w.x_dtype == "bf16" else 4
+    unit_bytes = nn * xb + w.n * q * 4 + nn * 4
+    snap_bytes = (w.B * (w.L // w.snapshot_every) * w.H * nn * 4) if w.snapshot_every else 0
+    algo = unit_bytes * w.token_heads + snap_bytes
+    peaks = read_peaks()
+    achieved = algo / (ms / 1e3) / 1e9
+    if ranks.printer:
+        print(json.dumps({
+            "metric": "MRU readout backward token·heads/s, 1×B200", "direction": "backward_readout",
+            "value": aggregate_rate(ranks.world, w.token_heads, ms), "unit": UNIT, "n_gpus": ranks.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded N(0,1) embeddings and readout gradients)", "config": workload_config(w, None),
+            "clocks": clocks.summary(),
+            "roofline": {"bound": "hbm", "scope": "whole call", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "algorithmic_bytes_per_step": algo,
+                         "note": "the call recomputes every state into its workspace (the forward's full-state "
+                                 "scan), forms dL/dS_t = do_t U^T there, and runs the scan's backward"}}),
+              flush=True)
     ranks.close()
     return 0
 

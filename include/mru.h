@@ -195,6 +195,34 @@ mru_status mru_scan_backward(const mru_problem* p, const void* x, const float* S
                              const float* dS, float* dx, float* dS0, void* ws, size_t ws_bytes,
                              void* stream);
 
+/* Backward of mru_scan_fused WITH the readout: the gradient with respect to
+ * the embeddings (and S0) of a loss of the readout's outputs, given their
+ * gradients, without any state stored by the caller.  The readout maps the
+ * state back to vectors ("MRU Update: An independent developer's alternative
+ * to Attention is now running successfully", section "What MRU Actually
+ * Does", step 3); its chain rule, o_t = S_t U, gives every state the upstream
+ * gradient
+ *   dL/dS_t = do_t U^T  (+ dP_k at 1-based t = k * every),
+ * and the scan's backward (mru_scan_backward) takes it from there.  The
+ * call recomputes the states with the forward scan into the workspace, forms
+ * those gradients there, and runs the backward.
+ *   x      [B, L, H*n*n] the forward's embeddings (f32 or bf16)
+ *   S0     [B, H, n, n] fp32 or NULL (identity), as in the forward
+ *   ro     the forward's readout: u, q, u_per_head, snapshot_every
+ *          (ro->snapshots is not used)
+ *   d_o    [B, L, H, n, q] fp32 gradients of the readout outputs o_t
+ *   d_snaps [B, L/every, H, n, n] fp32 gradients of the snapshots, or NULL
+ *          (no snapshot term; ignored when ro->snapshot_every == 0)
+ *   dx     [B, L, H*n*n] fp32 out;  dS0 [B, H, n, n] fp32 out, or NULL
+ * Every pointer 16-byte aligned; dx and dS0 alias no input.  The workspace
+ * holds mru_backward_readout_workspace_size(p) bytes (twice the states'
+ * size plus the backward's own); the status word is at its start, as for
+ * every other call.  Arithmetic as mru_scan_backward's. */
+size_t mru_backward_readout_workspace_size(const mru_problem* p);
+mru_status mru_scan_backward_readout(const mru_problem* p, const void* x, const float* S0, const mru_readout* ro,
+                                     const float* d_o, const float* d_snaps, float* dx, float* dS0, void* ws,
+                                     size_t ws_bytes, void* stream);
+
 /* Synchronises `stream` and returns the device-detected status of the last
  * call that used this workspace: MRU_OK, MRU_ERR_SINGULAR, or
  * MRU_ERR_TIMEOUT when a bounded wait of the single-read n = 16 kernel gave

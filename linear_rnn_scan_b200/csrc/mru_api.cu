@@ -518,6 +518,80 @@ const char* mru_status_string(mru_status s)
     }
 }
 
+namespace {
+// The readout backward's workspace: one region shared by the forward
+// recomputation and the backward (the status word at its start, where
+// mru_last_device_status reads it), then the recomputed states and their
+// upstream gradients (each [B, L, H, n, n] fp32).
+struct ReadoutBwdLayout {
+    size_t S, dS, region, region_bytes, bytes;
+};
+ReadoutBwdLayout readout_bwd_layout(const mru_problem& p)
+{
+    ReadoutBwdLayout R;
+    const size_t states = (size_t)(p.B * p.L * p.H) * (size_t)p.n * p.n * sizeof(float);
+    const size_t fwd = layout(make_params(p, SRC_EMBEDDING, false), false).bytes;
+    const size_t bwd = bwd_layout(make_bwd_params(p)).bytes;
+    R.region = 0;
+    R.region_bytes = fwd > bwd ? fwd : bwd;
+    R.S = round_up(R.region_bytes, 256);
+    R.dS = R.S + round_up(states, 256);
+    R.bytes = R.dS + round_up(states, 256);
+    return R;
+}
+}  // namespace
+
+size_t mru_backward_readout_workspace_size(const mru_problem* p)
+{
+    if (check_problem(p) != MRU_OK) return 0;
+    return readout_bwd_layout(*p).bytes;
+}
+
+mru_status mru_scan_backward_readout(const mru_problem* p, const void* x, const float* S0, const mru_readout* ro,
+                                     const float* d_o, const float* d_snaps, float* dx, float* dS0, void* ws,
+                                     size_t ws_bytes, void* stream)
+{
+    mru_status st = check_problem(p);
+    if (st != MRU_OK) return st;
+    if (!x || !ro || !ro->u || !d_o || !dx || !ws) return MRU_ERR_INVALID_ARG;
+    if (ro->q < 0 || ro->q > p->n || (ro->u_per_head != 0 && ro->u_per_head != 1) || ro->snapshot_every < 0)
+        return MRU_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dx) || !aligned16(ws) || !aligned16(d_o) || (S0 && !aligned16(S0)) ||
+        (dS0 && !aligned16(dS0)) || (d_snaps && !aligned16(d_snaps)))
+        return MRU_ERR_INVALID_ARG;
+    if ((const void*)dx == x || (const void*)dx == (const void*)d_o) return MRU_ERR_INVALID_ARG;
+    if (dS0 && ((const void*)dS0 == (const void*)S0 || (const void*)dS0 == (const void*)dx)) return MRU_ERR_INVALID_ARG;
+    const ReadoutBwdLayout R = readout_bwd_layout(*p);
+    if (ws_bytes < R.bytes) return MRU_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* base = reinterpret_cast<char*>(ws);
+    char* region = base + R.region;
+    if ((st = reset_status(region, s)) != MRU_OK) return st;
+    if (p->B * p->H * p->L == 0) {
+        if (dS0 && p->B * p->H > 0)
+            return from_cuda(cudaMemsetAsync(dS0, 0, sizeof(float) * (size_t)(p->B * p->H * p->n * p->n), s));
+        return MRU_OK;
+    }
+    float* S_buf = reinterpret_cast<float*>(base + R.S);
+    float* dS_buf = reinterpret_cast<float*>(base + R.dS);
+    cudaError_t e;
+    // 1. the states, recomputed by the fused forward (all of them, into the workspace)
+    const KParams kf = make_params(*p, SRC_EMBEDDING, false);
+    const Workspace Wf = layout(kf, false);
+    if ((e = launch_scan(kf, x, S0, nullptr, 0, S_buf, nullptr, nullptr, region, Wf, s, nullptr)) != cudaSuccess)
+        return MRU_ERR_CUDA;
+    // 2. their upstream gradients from the readout's
+    const int q = ro->q == 0 ? 1 : ro->q;
+    const int64_t u_hs = ro->u_per_head ? (int64_t)p->n * q : 0;
+    if ((e = launch_readout_grad(kf, ro->u, q, u_hs, d_o, ro->snapshot_every, ro->snapshot_every > 0 ? d_snaps : nullptr,
+                                 dS_buf, s)) != cudaSuccess)
+        return MRU_ERR_CUDA;
+    // 3. the scan's backward
+    const KParams kb = make_bwd_params(*p);
+    const BwdWorkspace Wb = bwd_layout(kb);
+    return from_cuda(launch_backward(kb, x, S0, S_buf, dS_buf, dx, dS0, region, Wb, s));
+}
+
 size_t mru_backward_workspace_size(const mru_problem* p)
 {
     if (check_problem(p) != MRU_OK) return 0;

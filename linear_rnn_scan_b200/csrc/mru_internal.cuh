@@ -254,6 +254,10 @@ cudaError_t launch_scan(const KParams& p, const void* src, const float* S0, cons
                         void* ws_base, const Workspace& W, cudaStream_t s, int* launches);
 cudaError_t launch_backward(const KParams& p, const void* x, const float* S0, const float* S_fwd, const float* dS,
                             float* dx, float* dS0, void* ws_base, const BwdWorkspace& W, cudaStream_t s);
+// dL/dS_t = do_t U^T (+ the snapshot's gradient at 1-based t = k * every)
+// for every state, the upstream gradient of the readout form (mru_readout_bwd.cu).
+cudaError_t launch_readout_grad(const KParams& p, const float* u, int q, int64_t u_hs, const float* d_o,
+                                int64_t every, const float* d_snap, float* dS, cudaStream_t s);
 // Name of the i-th kernel one launch_scan call starts for this problem.
 const char* kernel_name(const KParams& p, bool readout, int i);
 // mru_math the kernels for this problem actually use (MRU_MATH_FP32 for the

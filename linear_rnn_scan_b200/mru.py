@@ -32,7 +32,7 @@ EXPORTS = ["mru_workspace_size", "mru_build_states", "mru_scan", "mru_scan_fused
            "mru_last_device_status", "mru_status_string", "mru_chosen_chunk", "mru_launch_count",
            "mru_set_profile_events", "mru_scan_fused_noalloc", "mru_kernel_name", "mru_effective_math",
            "mru_backward_workspace_size", "mru_scan_backward", "mru_scan_fused_host",
-           "mru_debug_stall_next_fused"]
+           "mru_debug_stall_next_fused", "mru_backward_readout_workspace_size", "mru_scan_backward_readout"]
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -102,6 +102,11 @@ def load(path: str = LIB_PATH):
             lib.mru_scan_fused_host.argtypes = [P, vp, vp, ctypes.POINTER(Readout), vp, vp, vp, vp, vp, sz,
                                                 ctypes.c_int32, vp, vp, vp]
             lib.mru_scan_fused_host.restype = ctypes.c_int
+            lib.mru_backward_readout_workspace_size.argtypes = [P]
+            lib.mru_backward_readout_workspace_size.restype = sz
+            lib.mru_scan_backward_readout.argtypes = [P, vp, vp, ctypes.POINTER(Readout), vp, vp, vp, vp, vp, sz,
+                                                      vp]
+            lib.mru_scan_backward_readout.restype = ctypes.c_int
             lib.mru_debug_stall_next_fused.argtypes = [ctypes.c_int32]
             lib.mru_debug_stall_next_fused.restype = None
             _lib = lib
@@ -193,6 +198,16 @@ def backward_workspace_size(p: Problem) -> int:
 def scan_backward(p: Problem, x: int, S0: int | None, S_fwd: int, dS: int, dx: int, dS0: int | None, ws: int,
                   ws_bytes: int, stream: int = 0) -> int:
     return load().mru_scan_backward(ctypes.byref(p), x, S0, S_fwd, dS, dx, dS0, ws, ws_bytes, stream)
+
+
+def backward_readout_workspace_size(p: Problem) -> int:
+    return load().mru_backward_readout_workspace_size(ctypes.byref(p))
+
+
+def scan_backward_readout(p: Problem, x: int, S0: int | None, readout: Readout, d_o: int, d_snaps: int | None,
+                          dx: int, dS0: int | None, ws: int, ws_bytes: int, stream: int = 0) -> int:
+    return load().mru_scan_backward_readout(ctypes.byref(p), x, S0, ctypes.byref(readout), d_o, d_snaps, dx, dS0,
+                                            ws, ws_bytes, stream)
 
 
 def last_device_status(ws: int, stream: int = 0) -> int:
@@ -343,6 +358,30 @@ def scan_backward_t(p: Problem, x, S_fwd, dS, *, S0=None, dx=None, dS0=None, ws=
     rc = scan_backward(p, _dev_ptr(x, "x"), _dev_ptr(S0, "S0"), _dev_ptr(S_fwd, "S_fwd"), _dev_ptr(dS, "dS"),
                        _dev_ptr(dx, "dx"), _dev_ptr(dS0, "dS0"), ws.data_ptr(), ws.numel(), _stream(stream))
     _check(rc, "mru_scan_backward")
+    return dx, dS0, ws
+
+
+def scan_backward_readout_t(p: Problem, x, u, d_o, *, snapshot_every: int = 0, d_snaps=None, S0=None,
+                            q: int = 0, u_per_head: int = 0, dx=None, dS0=None, ws=None, stream=None):
+    """Gradients of a loss of the readout's outputs (d_o [B, L, H, n, q],
+    and d_snaps [B, L//every, H, n, n] or None) with respect to the
+    embeddings (dx) and, with S0, to S0 (dS0); no forward state is needed."""
+    torch = _torch()
+    dev = x.device
+    if ws is None:
+        nbytes = backward_readout_workspace_size(p)
+        if nbytes == 0:
+            raise MruError(ERR_INVALID_ARG, "backward_readout_workspace_size")
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    if dx is None:
+        dx = torch.empty((p.B, p.L, p.H * p.n * p.n), dtype=torch.float32, device=dev)
+    if S0 is not None and dS0 is None:
+        dS0 = torch.empty((p.B, p.H, p.n, p.n), dtype=torch.float32, device=dev)
+    ro = Readout(_dev_ptr(u, "u"), int(snapshot_every), None, int(q), int(u_per_head))
+    rc = scan_backward_readout(p, _dev_ptr(x, "x"), _dev_ptr(S0, "S0"), ro, _dev_ptr(d_o, "d_o"),
+                               _dev_ptr(d_snaps, "d_snaps"), _dev_ptr(dx, "dx"), _dev_ptr(dS0, "dS0"),
+                               ws.data_ptr(), ws.numel(), _stream(stream))
+    _check(rc, "mru_scan_backward_readout")
     return dx, dS0, ws
 
 

@@ -189,3 +189,48 @@ def test_backward_n32_ldu_workload_sampled():
         dx_o, _ = oracle.backward(oracle_problem(w1), x1, dS1)
         e = _rel(dx[b, :, h], dx_o.reshape(w.L, n * n), axis=-1)
         assert e.max() <= TOL_BWD, (b, h, e.max(), np.median(e))
+
+
+READOUT_CASES = [  # n, mode, x_dtype, ushape, every, with_s0
+    (4, gen.MODE_RESHAPE, "f32", "vector", 8, False),
+    (16, gen.MODE_DETNORM, "f32", "shared", 16, True),
+    (16, gen.MODE_CAYLEY, "f32", "per_head", 0, False),
+    (32, gen.MODE_LDU, "bf16", "vector", 16, True),
+    (64, gen.MODE_DETNORM, "f32", "per_head", 8, False),
+]
+
+
+@pytest.mark.parametrize("n,mode,x_dtype,ushape,every,with_s0", READOUT_CASES)
+def test_backward_readout_against_oracle(n, mode, x_dtype, ushape, every, with_s0):
+    """mru_scan_backward_readout: gradients of the readout's outputs (o_t =
+    S_t U with one vector, shared or per-head query columns; snapshots every
+    `every` steps) to the embeddings and S0, through the C-ABI, against the
+    oracle's readout backward; several chunks with a ragged tail."""
+    t = torch()
+    B, H, L = 2, 3, 53
+    alpha = 0.3 / np.sqrt(n) if mode != gen.MODE_LDU else 1.0
+    w = gen.Workload("bro", B=B, H=H, L=L, n=n, x_dtype=x_dtype, mode=mode, alpha=float(alpha), seed=31 + n)
+    x = gen.make_x(w)
+    r = np.random.default_rng(n + every)
+    q = 1 if ushape == "vector" else 3
+    u = {"vector": r.standard_normal(n), "shared": r.standard_normal((n, q)),
+         "per_head": r.standard_normal((H, n, q))}[ushape].astype(np.float32)
+    d_o = r.standard_normal((B, L, H, n, q)).astype(np.float32)
+    d_snap = r.standard_normal((B, L // every, H, n, n)).astype(np.float32) if every else None
+    S0 = (np.eye(n) + 0.1 * r.standard_normal((B, H, n, n))).astype(np.float32) if with_s0 else None
+    p = mru.problem_from_workload(w, chunk=16)
+    dx, dS0, ws = mru.scan_backward_readout_t(
+        p, to_device_x(x), t.from_numpy(u).cuda(), t.from_numpy(d_o).cuda(), snapshot_every=every,
+        d_snaps=None if d_snap is None else t.from_numpy(d_snap).cuda(),
+        S0=None if S0 is None else t.from_numpy(S0).cuda(), q=0 if ushape == "vector" else q,
+        u_per_head=1 if ushape == "per_head" else 0)
+    assert mru.last_device_status(ws.data_ptr(), t.cuda.current_stream().cuda_stream) == mru.OK
+    dx_o, dS0_o = oracle.backward_readout(oracle_problem(w), x, u.astype(np.float64) if ushape != "vector" else
+                                          u.astype(np.float64), d_o[..., 0] if ushape == "vector" else d_o,
+                                          snapshot_every=every, d_snap=d_snap,
+                                          S0=None if S0 is None else S0.astype(np.float64))
+    e = _rel(dx.cpu().numpy().astype(np.float64).reshape(B, L, H, n * n), dx_o.reshape(B, L, H, n * n), axis=-1)
+    assert e.max() <= TOL_BWD, (e.max(), np.median(e))
+    if with_s0:
+        e0 = _rel(dS0.cpu().numpy().astype(np.float64).reshape(B, H, n * n), dS0_o.reshape(B, H, n * n), axis=-1)
+        assert e0.max() <= TOL_BWD, e0.max()
