@@ -31,7 +31,8 @@ int32_t generic_chunk(const mru_problem& p)
 bool fast16_eligible(const mru_problem& p, bool readout)
 {
     return p.n == 16 && p.x_dtype == MRU_F32 && !readout &&
-           (p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM || p.mode == MRU_MODE_CAYLEY) &&
+           (p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM || p.mode == MRU_MODE_CAYLEY ||
+            p.mode == MRU_MODE_EXPM) &&
            (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32X3) && p.chunk % n16::kSub == 0;
 }
 

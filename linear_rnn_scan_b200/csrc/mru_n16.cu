@@ -308,17 +308,18 @@ __device__ __forceinline__ float det_scale_m1(const float* src, int stride, int 
     return cm1;
 }
 
-// The per-token scalars of F = ca M + dv I for the nt (<= ST) tokens of a
-// stage, written to cd: one LU factorisation per token, 32 / ST lanes each,
-// in the determinant-corrected mode; the constants (alpha, 0 or -1)
-// otherwise.  A singular token sets the status bit and keeps X = I.
+// The per-token scalars of F = ca M + dv I for the live slots of a stage
+// (bit s of live_mask: slot s holds a token), written to cd: one LU
+// factorisation per slot, 32 / ST lanes each, in the determinant-corrected
+// mode; the constants (alpha, 0 or -1) otherwise.  A singular token sets the
+// status bit and keeps X = I.
 template <int ST>
-__device__ __forceinline__ void stage_scalars(const KParams& p, float2* cd, const float* xs, int nt, int lane,
-                                              uint32_t* status)
+__device__ __forceinline__ void stage_scalars(const KParams& p, float2* cd, const float* xs, unsigned live_mask,
+                                              int lane, uint32_t* status)
 {
     constexpr int R = N * ST / 32, W = N / R;
     const int grp = lane / W, r = lane % W;
-    const bool live = grp < nt;
+    const bool live = (live_mask >> grp) & 1u;
     float ca = p.alpha, dv = p.add_identity ? 0.0f : -1.0f;
     if (p.mode == MRU_MODE_DETNORM) {
         // idle groups factorise I (scale 0, plus I)
@@ -339,14 +340,15 @@ __device__ __forceinline__ void stage_scalars(const KParams& p, float2* cd, cons
 }
 
 // F = X - I = 2 (I - A)^-1 A of the Cayley map X = (I - A)^-1 (I + A),
-// A = alpha (M - M^T) / 2, for the nt (<= ST) tokens of a stage, written over
-// the tokens' slices (same swizzled layout).  Gauss-Jordan elimination on
+// A = alpha (M - M^T) / 2, for the live slots of a stage (bit s of live_mask:
+// slot s holds a token; slot 0 always does), written over the slots' slices
+// (same swizzled layout).  Gauss-Jordan elimination on
 // [I - A | 2A] (rows of 32 entries), 8 lanes per token (lane r: rows r and
 // r + 8), 4 tokens per round; no pivoting: the symmetric part of I - A is I,
 // and every Schur complement keeps a symmetric part of at least I, so each
 // pivot is at least 1.  The right half ends as F.
 template <int ST>
-__device__ __forceinline__ void stage_cayley(float alpha, float* xs, int nt, int lane)
+__device__ __forceinline__ void stage_cayley(float alpha, float* xs, unsigned live_mask, int lane)
 {
     static_assert(ST % 4 == 0, "whole rounds of 4 tokens");
     const int grp = lane >> 3, r = lane & 7;
@@ -354,7 +356,8 @@ __device__ __forceinline__ void stage_cayley(float alpha, float* xs, int nt, int
 #pragma unroll 1
     for (int rd = 0; rd < ST / 4; ++rd) {
         const int tk = 4 * rd + grp;
-        float* ms = xs + (tk < nt ? tk : 0) * NN;       // idle groups eliminate token 0's copy, not stored
+        const bool live = (live_mask >> tk) & 1u;
+        float* ms = xs + (live ? tk : 0) * NN;          // idle groups eliminate slot 0's copy, not stored
         float w[2][2 * N];
 #pragma unroll
         for (int lr = 0; lr < 2; ++lr) {
@@ -393,7 +396,7 @@ __device__ __forceinline__ void stage_cayley(float alpha, float* xs, int nt, int
                 }
             }
         }
-        if (tk < nt) {
+        if (live) {
 #pragma unroll
             for (int lr = 0; lr < 2; ++lr) {
                 const int i = r + 8 * lr;
@@ -477,6 +480,150 @@ __device__ __forceinline__ void chain_product(const float (&Ad)[2][4], const Fra
     for (int kt = 0; kt < 2; ++kt)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) mma_tf32(acc[nt], ah[kt], f.bh[kt][nt]);
+}
+
+// ---- the exponential map on the tensor cores -------------------------------
+
+// 1 / k! for k = 0 .. 13.
+__constant__ float kInvFact[14] = {1.0f, 1.0f, 0.5f, (float)(1.0 / 6.0), (float)(1.0 / 24.0),
+                                   (float)(1.0 / 120.0), (float)(1.0 / 720.0), (float)(1.0 / 5040.0),
+                                   (float)(1.0 / 40320.0), (float)(1.0 / 362880.0), (float)(1.0 / 3628800.0),
+                                   (float)(1.0 / 39916800.0), (float)(1.0 / 479001600.0),
+                                   (float)(1.0 / 6227020800.0)};
+
+// B fragments (split, contraction index permuted as in make_frag_f) of a
+// symmetric (sign = 1) or skew-symmetric (sign = -1) 16 x 16 matrix held in
+// accumulator layout: the fragment needs element (8 kt + 2 q + e, 8 nt + g),
+// which is sign times the lane's own (8 nt + g, 8 kt + 2 q + e).
+__device__ __forceinline__ void frag_from_acc(const float (&Ad)[2][4], float sign, FragF& f)
+{
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) split_tf32(sign * Ad[kt][2 * nt + e], f.bh[kt][nt][e], f.bl[kt][nt][e]);
+}
+
+// A 16 x 16 matrix in accumulator layout written to a swizzled slice.
+__device__ __forceinline__ void store_acc_swz(float* ms, const float (&Ad)[2][4], int g, int q)
+{
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8)
+            *reinterpret_cast<float2*>(ms + swz(g + 8 * h8, 8 * nt + 2 * q)) =
+                make_float2(Ad[nt][2 * h8], Ad[nt][2 * h8 + 1]);
+}
+
+// F = X - I of the exponential map X = exp(A), A = alpha (M - M^T) / 2, for
+// the live slots of a stage (bit s of live_mask: slot s holds a token),
+// written over the slots' slices in the same swizzled layout.  The whole warp
+// works on one token at a time, its 16 x 16 products on the tensor cores in
+// split tf32 (the chain's chain_product).
+//
+// Scaling and squaring (Moler and Van Loan, 1978), with s and the Taylor
+// degree m chosen as the generic kernels choose them: B = A / 2^s with
+// ||A||_1 / 2^s <= 1/2, m the least degree (at most 12) whose next term
+// ||B||^(m+1) / (m+1)! is below 2^-26 ||B||.  exp(B) - I = sum_k B^k / k!
+// (k = 1..m) in Horner form over B^2, pairs of odd and even terms:
+// H = c_{2p-1} B + c_{2p} B^2, then H <- c_{2i+1} B + c_{2i+2} B^2 + H B^2
+// for i = p-2 .. 0 (p = ceil(m / 2), c_k = 1 / k!, c_k = 0 above m), so
+// every product has B^2 as its right operand.  B is skew-symmetric and B^2
+// symmetric: each lane's accumulator fragment of B (B^2) gives it its
+// B-operand fragments of B (B^2) by transposition, with no data exchange.
+// The s squarings (I + F)^2 - I = 2 F + F F take F's B-operand fragments
+// through the token's own slice (M is no longer needed there).
+template <int ST>
+__device__ __forceinline__ void stage_expm(float alpha, float* xs, unsigned live_mask, int lane)
+{
+    const int g = lane >> 2, q = lane & 3;
+    const float ha = 0.5f * alpha;
+#pragma unroll 1
+    for (int tk = 0; tk < ST; ++tk) {
+        if (!((live_mask >> tk) & 1u)) continue;
+        float* ms = xs + tk * NN;
+        float Bd[2][4];                                  // A at this lane's accumulator positions
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+                const int r = g + 8 * h8, c = 8 * nt + 2 * q;
+                const float2 v = *reinterpret_cast<const float2*>(ms + swz(r, c));
+                Bd[nt][2 * h8] = ha * (v.x - ms[swz(c, r)]);
+                Bd[nt][2 * h8 + 1] = ha * (v.y - ms[swz(c + 1, r)]);
+            }
+        __syncwarp();                                    // every read of M before the slice is reused
+        // ||A||_1: the lane's share of 4 column sums (rows g and g + 8),
+        // summed over g, then the largest column
+        float cs[4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) cs[2 * nt + e] = fabsf(Bd[nt][e]) + fabsf(Bd[nt][2 + e]);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) cs[i] += __shfl_xor_sync(FULL, cs[i], o);
+        float nrm = fmaxf(fmaxf(cs[0], cs[1]), fmaxf(cs[2], cs[3]));
+        nrm = fmaxf(nrm, __shfl_xor_sync(FULL, nrm, 1));
+        nrm = fmaxf(nrm, __shfl_xor_sync(FULL, nrm, 2));
+        int s2 = 0;
+        while (nrm > 0.5f && s2 < 64) { nrm *= 0.5f; ++s2; }     // uniform across the warp
+        int m = 1;
+        float term = nrm;
+        while (m < 12 && term * nrm / (float)(m + 1) > 1.4901161e-8f * nrm) {
+            term = term * nrm / (float)(m + 1);
+            ++m;
+        }
+        const float sc = ldexpf(1.0f, -s2);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) (&Bd[0][0])[i] *= sc;
+        FragF f;
+        frag_from_acc(Bd, -1.0f, f);
+        float P[2][4];                                   // B^2
+        chain_product<true>(Bd, f, P);
+        frag_from_acc(P, 1.0f, f);
+        const int pp = (m + 1) >> 1;
+        float H[2][4];
+        {
+            const float c1 = kInvFact[2 * pp - 1], c2 = 2 * pp <= m ? kInvFact[2 * pp] : 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) (&H[0][0])[i] = fmaf(c1, (&Bd[0][0])[i], c2 * (&P[0][0])[i]);
+        }
+#pragma unroll 1
+        for (int k = pp - 2; k >= 0; --k) {
+            float acc[2][4];
+            chain_product<true>(H, f, acc);              // H B^2
+            const float c1 = kInvFact[2 * k + 1], c2 = kInvFact[2 * k + 2];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                (&H[0][0])[i] = fmaf(c1, (&Bd[0][0])[i], c2 * (&P[0][0])[i]) + (&acc[0][0])[i];
+        }
+#pragma unroll 1
+        for (int r = 0; r < s2; ++r) {
+            store_acc_swz(ms, H, g, q);
+            __syncwarp();
+            FragF fh;
+            make_frag_f(ms, 1.0f, 0.0f, 0.0f, g, q, fh, false);
+            __syncwarp();                                // every read before the next write
+            float acc[2][4];
+            chain_product<true>(H, fh, acc);             // F F
+#pragma unroll
+            for (int i = 0; i < 8; ++i) (&H[0][0])[i] = fmaf(2.0f, (&H[0][0])[i], (&acc[0][0])[i]);
+        }
+        store_acc_swz(ms, H, g, q);
+    }
+    __syncwarp();
+}
+
+// F = X - I of the orthogonal constructions over the slots' slices: Tr = 1
+// the Cayley map, Tr = 2 the exponential map.
+template <int Tr, int ST>
+__device__ __forceinline__ void stage_transform(float alpha, float* xs, unsigned live_mask, int lane)
+{
+    if (Tr == 1) stage_cayley<ST>(alpha, xs, live_mask, lane);
+    else stage_expm<ST>(alpha, xs, live_mask, lane);
 }
 
 __device__ __forceinline__ void store_d(float* out, const float (&Ad)[2][4], int g, int q)
@@ -957,7 +1104,7 @@ __device__ __forceinline__ void direct_carry(const float* in, bool has_s0, int l
 // runs on the uncorrected matrices and the carry kernel applies the
 // determinant correction of each total.  CTA 0 also zeroes the carry scan's
 // counters (the carry kernel runs after this launch).
-template <bool PerToken, bool Cayley = false>
+template <bool PerToken, int Tr = 0>
 __global__ void __launch_bounds__(RWARPS * 32, 2)
 k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, unsigned* ctr, int64_t nctr,
            uint32_t* status)
@@ -997,9 +1144,9 @@ k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, u
             const float* xs = sm.stage[cs];
             const int nt = (c.tend - t0 < RST) ? (int)(c.tend - t0) : RST;
             float ca = p.alpha, dv = p.add_identity ? 0.0f : -1.0f;
-            if (PerToken) stage_scalars<RST>(p, sm.cd, xs, nt, lane, status);
-            if (Cayley) {                                  // F itself now sits where M was
-                stage_cayley<RST>(p.alpha, sm.stage[cs], nt, lane);
+            if (PerToken) stage_scalars<RST>(p, sm.cd, xs, (1u << nt) - 1u, lane, status);
+            if (Tr != 0) {                                 // F itself now sits where M was
+                stage_transform<Tr, RST>(p.alpha, sm.stage[cs], (1u << nt) - 1u, lane);
                 ca = 1.0f;
                 dv = 0.0f;
             }
@@ -1031,7 +1178,7 @@ k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, u
 // Apply pass: per chain the carry from the carry scan's factors, then
 // S_t = S_{t-1} + S_{t-1} F_t from S = carry, every S_t written, with the
 // per-token determinant scales factorised here.
-template <bool Direct, bool Cayley = false>
+template <bool Direct, int Tr = 0>
 __global__ void __launch_bounds__(AWARPS * 32, 3)
 k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, float* __restrict__ S_out,
           uint32_t* status, const float* __restrict__ S0)
@@ -1075,12 +1222,12 @@ k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, 
             __syncwarp();
             const float* xs = sm.stage[cs];
             const int nt = (c.tend - t0 < AST) ? (int)(c.tend - t0) : AST;
-            if (Cayley) {                                  // F itself now sits where M was
-                stage_cayley<AST>(p.alpha, sm.stage[cs], nt, lane);
+            if (Tr != 0) {                                 // F itself now sits where M was
+                stage_transform<Tr, AST>(p.alpha, sm.stage[cs], (1u << nt) - 1u, lane);
                 if (lane < AST) sm.cd[lane] = make_float2(1.0f, 0.0f);
                 __syncwarp();
             } else {
-                stage_scalars<AST>(p, sm.cd, xs, nt, lane, status);
+                stage_scalars<AST>(p, sm.cd, xs, (1u << nt) - 1u, lane, status);
             }
 #pragma unroll
             for (int j = 0; j < AST; ++j) {
@@ -1489,7 +1636,7 @@ __device__ __forceinline__ void fused_issue(const KParams& p, const FCtl& f, con
         cp_async16(cdbuf + 2 * lane, f.cd + seq * f.Lp + t0 + 2 * lane);
 }
 
-template <bool Cayley>
+template <int Tr>
 __global__ void __launch_bounds__(FWARPS * 32, 3)
 k16_fused(KParams p, FCtl f, const float* __restrict__ x, const float* __restrict__ S0, float* __restrict__ S_out,
           uint32_t* status)
@@ -1502,7 +1649,7 @@ k16_fused(KParams p, FCtl f, const float* __restrict__ x, const float* __restric
     const float m0 = (g == 2 * q) ? 1.0f : 0.0f;
     const float m1 = (g == 2 * q + 1) ? 1.0f : 0.0f;
     const int G = 1 << f.gshift;
-    const bool detnorm = p.mode == MRU_MODE_DETNORM && !Cayley;
+    const bool detnorm = p.mode == MRU_MODE_DETNORM && Tr == 0;
     const uint64_t pol_keep = policy_evict_last(), pol_drop = policy_evict_first();
     const int64_t tok = p.H * NN;
 
@@ -1574,12 +1721,12 @@ k16_fused(KParams p, FCtl f, const float* __restrict__ x, const float* __restric
                 const int64_t t0 = c.tbeg + (int64_t)(s - (kind == FK_APPLY ? 1 : 0)) * FST;
                 const int nt = (c.tend - t0 < FST) ? (int)(c.tend - t0) : FST;
                 float2* cdv = sm.cd[cur];
-                if (Cayley) {
-                    stage_cayley<FST>(p.alpha, xs, nt, lane);
+                if (Tr != 0) {
+                    stage_transform<Tr, FST>(p.alpha, xs, (1u << nt) - 1u, lane);
                     if (lane < FST) cdv[lane] = make_float2(1.0f, 0.0f);
                     __syncwarp();
                 } else if (kind == FK_REDUCE) {
-                    stage_scalars<FST>(p, cdv, xs, nt, lane, status);
+                    stage_scalars<FST>(p, cdv, xs, (1u << nt) - 1u, lane, status);
                     if (detnorm && lane < nt) f.cd[seq * f.Lp + t0 + lane] = cdv[lane];
                 } else if (!detnorm) {
                     if (lane < FST) cdv[lane] = make_float2(p.alpha, p.add_identity ? 0.0f : -1.0f);
@@ -2019,7 +2166,7 @@ k16b_local(KParams p, const float* __restrict__ x, const float* __restrict__ dS,
             cp_async_wait<BNS - 1>();
             __syncwarp();
             const int nt = (ts - lo + 1 < BST) ? (int)(ts - lo + 1) : BST;
-            stage_scalars<BST>(p, sm.cd, sm.x[cs], nt, lane, status);
+            stage_scalars<BST>(p, sm.cd, sm.x[cs], (1u << nt) - 1u, lane, status);
 #pragma unroll
             for (int j = 0; j < BST; ++j) {
                 if (j < nt) {
@@ -2103,7 +2250,7 @@ k16b_apply(KParams p, const float* __restrict__ x, const float* __restrict__ S0,
             cp_async_wait<BNS - 1>();
             __syncwarp();
             const int nt = (ts - lo + 1 < BST) ? (int)(ts - lo + 1) : BST;
-            stage_scalars<BST>(p, sm.cd, sm.x[cs], nt, lane, status);
+            stage_scalars<BST>(p, sm.cd, sm.x[cs], (1u << nt) - 1u, lane, status);
 #pragma unroll
             for (int j = 0; j < BST; ++j) {
                 if (j < nt) {
@@ -2208,7 +2355,14 @@ k16b_apply(KParams p, const float* __restrict__ x, const float* __restrict__ S0,
 
 // CTAs of a persistent launch: resident CTAs per SM times the SM count,
 // cached per device and kernel slot; no more than the chains need.
-std::atomic<int> g_resident[64][12];
+std::atomic<int> g_resident[64][16];
+
+// The orthogonal construction the passes apply to each slice: 0 none, 1 the
+// Cayley map, 2 the exponential map.
+int transform_of(const KParams& p)
+{
+    return p.mode == MRU_MODE_CAYLEY ? 1 : p.mode == MRU_MODE_EXPM ? 2 : 0;
+}
 
 cudaError_t persistent_grid(int slot, const void* kern, int threads, size_t smem, int warps, int64_t nchains,
                             unsigned& grid)
@@ -2236,7 +2390,8 @@ cudaError_t persistent_grid(int slot, const void* kern, int threads, size_t smem
 bool supports(const KParams& p, bool readout)
 {
     return p.n == N && p.src == SRC_EMBEDDING && p.x_dtype == MRU_F32 && !readout &&
-           (p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM || p.mode == MRU_MODE_CAYLEY) &&
+           (p.mode == MRU_MODE_RESHAPE || p.mode == MRU_MODE_DETNORM || p.mode == MRU_MODE_CAYLEY ||
+            p.mode == MRU_MODE_EXPM) &&
            (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32X3) && p.chunk > 0 && p.chunk % kSub == 0;
 }
 
@@ -2294,12 +2449,14 @@ cudaError_t launch_reduce(const KParams& p, const float* x, float* totals, const
     if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const size_t sm = sizeof(RSmem) * RWARPS;
     const bool per_token = p.mode == MRU_MODE_DETNORM && !p.add_identity;
-    const bool cayley = p.mode == MRU_MODE_CAYLEY;
-    auto kern = cayley ? k16_reduce<false, true> : per_token ? k16_reduce<true> : k16_reduce<false>;
+    const int tr = transform_of(p);
+    auto kern = tr == 1 ? k16_reduce<false, 1> : tr == 2 ? k16_reduce<false, 2>
+                        : per_token ? k16_reduce<true> : k16_reduce<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     unsigned grid = 0;
-    if ((e = persistent_grid(cayley ? 6 : per_token ? 1 : 0, (const void*)kern, RWARPS * 32, sm, RWARPS, nchains,
+    if ((e = persistent_grid(tr == 1 ? 6 : tr == 2 ? 11 : per_token ? 1 : 0, (const void*)kern, RWARPS * 32, sm,
+                             RWARPS, nchains,
                              grid)) !=
         cudaSuccess)
         return e;
@@ -2400,13 +2557,13 @@ cudaError_t launch_fused(const KParams& p, const FusedPlan& fp, char* ws, const 
     f.limit_ns = stall > 0 ? (uint64_t)stall * 1000000ull : 2000000000ull;     // 2 s unless testing
     cudaError_t e = cudaMemsetAsync(ws + fp.ctl, 0, fp.ctl_bytes, s);
     if (e != cudaSuccess) return e;
-    const bool cayley = p.mode == MRU_MODE_CAYLEY;
-    auto kern = cayley ? k16_fused<true> : k16_fused<false>;
+    const int tr = transform_of(p);
+    auto kern = tr == 1 ? k16_fused<1> : tr == 2 ? k16_fused<2> : k16_fused<0>;
     const size_t sm = sizeof(FSmem) * FWARPS;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)) != cudaSuccess)
         return e;
     unsigned grid = 0;
-    if ((e = persistent_grid(cayley ? 10 : 9, (const void*)kern, FWARPS * 32, sm, FWARPS, nchains, grid)) !=
+    if ((e = persistent_grid(9 + tr, (const void*)kern, FWARPS * 32, sm, FWARPS, nchains, grid)) !=
         cudaSuccess)
         return e;
     kern<<<grid, FWARPS * 32, sm, s>>>(p, f, x, S0, S_out, status);
@@ -2459,13 +2616,15 @@ cudaError_t launch_apply(const KParams& p, const float* x, const CarryPlan& cp, 
     if (nchains == 0) return cudaSuccess;
     if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const size_t sm = sizeof(ASmem) * AWARPS;
-    const bool cayley = p.mode == MRU_MODE_CAYLEY;
-    auto kern = cayley ? (direct ? k16_apply<true, true> : k16_apply<false, true>)
-                       : (direct ? k16_apply<true> : k16_apply<false>);
+    const int tr = transform_of(p);
+    auto kern = tr == 1   ? (direct ? k16_apply<true, 1> : k16_apply<false, 1>)
+                : tr == 2 ? (direct ? k16_apply<true, 2> : k16_apply<false, 2>)
+                          : (direct ? k16_apply<true> : k16_apply<false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     unsigned grid = 0;
-    if ((e = persistent_grid(cayley ? (direct ? 8 : 7) : (direct ? 3 : 2), (const void*)kern, AWARPS * 32, sm, AWARPS,
+    const int slot = tr == 1 ? (direct ? 8 : 7) : tr == 2 ? (direct ? 13 : 12) : (direct ? 3 : 2);
+    if ((e = persistent_grid(slot, (const void*)kern, AWARPS * 32, sm, AWARPS,
                              nchains, grid)) !=
         cudaSuccess)
         return e;

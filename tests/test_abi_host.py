@@ -134,6 +134,10 @@ def test_single_chunk_problems_take_one_launch(lib):
         assert mru.launch_count(p) == 1 and mru.kernel_names(p) == names
     p = mru.problem(8, 8, 4096, 16, mode=mru.MODE_DETNORM, alpha=0.0125)
     assert mru.kernel_names(p) == ["k16_reduce", "k16_carry", "k16_apply"]
+    for mode in (mru.MODE_CAYLEY, mru.MODE_EXPM):           # orthogonal maps on the same passes
+        q = mru.problem(8, 8, 4096, 16, mode=mode, alpha=0.0125)
+        assert mru.kernel_names(q) == ["k16_reduce", "k16_carry", "k16_apply"]
+        assert mru.effective_math(q) == "tf32x3"
     os.environ["MRU_N16_FUSED"] = "1"
     try:
         assert mru.kernel_names(p) == ["k16_fused"] and mru.launch_count(p) == 1
