@@ -239,6 +239,9 @@ cudaError_t launch_bwd_apply(const KParams& p, const void* x, const float* S0, c
 // scan and fix-up are the generic kernels.
 namespace n64 {
 bool supports(const KParams& p, bool readout);
+// The chunk phase on tcgen05 (k64_chunk_readout_tc) instead of mma.sync:
+// MRU_N64_TCGEN05=1 in the environment, read at every call.
+bool use_tcgen05();
 cudaError_t launch_chunk_readout(const KParams& p, const float* x, const float* u, int64_t snap_every,
                                  float* o_out, float* snaps, float* totals, uint32_t* status, cudaStream_t s);
 // o_t = C U + C V_t and the snapshots C + C Q_t from the chains' carries C.

@@ -1765,7 +1765,7 @@ const char* kernel_name(const KParams& p, bool readout, int i)
                                     "k_fixup"};
     if (i < 0 || i >= (p.K == 1 ? 1 : 5)) return "";
     if (i == 0 && small_scan_ok(p, readout)) return "k_small_scan";
-    if (i == 0 && n64::supports(p, readout)) return "k64_chunk_readout";
+    if (i == 0 && n64::supports(p, readout)) return n64::use_tcgen05() ? "k64_chunk_readout_tc" : "k64_chunk_readout";
     if (i == 4 && n64::supports(p, readout)) return "k64_fixup";
     return generic[i];
 }

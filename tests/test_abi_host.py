@@ -147,6 +147,11 @@ def test_single_chunk_problems_take_one_launch(lib):
     assert mru.kernel_names(p, True) == ["k_chunk_prefix"]
     p = mru.problem(2, 4, 4096, 64, mode=mru.MODE_DETNORM, alpha=0.01, math="tf32")
     assert mru.kernel_names(p, True)[0] == "k64_chunk_readout" and mru.launch_count(p, True) == 5
+    os.environ["MRU_N64_TCGEN05"] = "1"
+    try:
+        assert mru.kernel_names(p, True)[0] == "k64_chunk_readout_tc" and mru.launch_count(p, True) == 5
+    finally:
+        os.environ.pop("MRU_N64_TCGEN05", None)
 
 
 def test_small_problems_choose_one_launch(lib):
