@@ -131,7 +131,11 @@ mru_status mru_scan(const mru_problem* p, const float* X, const float* S0, float
  * With ro != NULL the states are reduced instead: o_out[b,t,h] = S_t . U
  * ([n, q] per token and head), and S_t is stored to ro->snapshots at
  * t = every, 2*every, ... (S_out unused).  q outside [0, n] or u_per_head
- * outside {0, 1} is MRU_ERR_INVALID_ARG. */
+ * outside {0, 1} is MRU_ERR_INVALID_ARG.
+ * With MRU_N64_TCGEN05=1 in the environment (read at each call) the n = 64
+ * readout path runs its chunk phase on the fifth-generation tensor cores
+ * (tcgen05.mma into tensor memory) instead of mma.sync: the same results
+ * within the tf32 gate, slower on B200, so not the default. */
 mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0,
                           const mru_readout* ro, float* S_out, float* o_out,
                           void* ws, size_t ws_bytes, void* stream);
@@ -225,13 +229,15 @@ mru_status mru_scan_backward_readout(const mru_problem* p, const void* x, const 
 
 /* Synchronises `stream` and returns the device-detected status of the last
  * call that used this workspace: MRU_OK, MRU_ERR_SINGULAR, or
- * MRU_ERR_TIMEOUT when a bounded wait of the single-read n = 16 kernel gave
- * up (its outputs are then unspecified; the CUDA context stays usable). */
+ * MRU_ERR_TIMEOUT when a bounded wait of one of the opt-in kernels gave up
+ * (the single-read n = 16 kernel's carry waits, the n = 64 tcgen05 kernel's
+ * tensor-core waits; outputs are then unspecified, the CUDA context stays
+ * usable). */
 mru_status mru_last_device_status(const void* ws, void* stream);
 
 /* Testing hook for the bounded waits of the single-read n = 16 kernel.  With
  * MRU_N16_FUSED=1 in the environment (read at each call), mru_scan_fused for
- * n = 16, fp32, reshape / DETNORM / CAYLEY and more than one chunk per
+ * n = 16, fp32, reshape / DETNORM / CAYLEY / EXPM and more than one chunk per
  * sequence runs one persistent kernel that reads x from HBM once instead of
  * the three passes (it is correct but, on B200, still slower; the passes
  * stay the default).  Its warps wait on one another in two
