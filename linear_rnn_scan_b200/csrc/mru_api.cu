@@ -133,7 +133,10 @@ bool fused16_enabled()
     return v && v[0] == '1';
 }
 
-Workspace layout(const KParams& k, bool readout)
+// fstore_ok: the n = 16 passes of the Cayley map and the exponential may keep
+// every token's F = X - I in the workspace (written by the reduce pass, read
+// by the apply pass instead of forming F again); off, they form it twice.
+Workspace layout(const KParams& k, bool readout, bool fstore_ok = true)
 {
     Workspace W;
     memset(&W, 0, sizeof W);
@@ -152,7 +155,13 @@ Workspace layout(const KParams& k, bool readout)
         }
         W.totals = off; off = round_up(off + BH * k.K * nn * sizeof(float), 256);
         W.c16 = n16::carry_plan((int64_t)BH, k.K, off);
-        W.bytes = W.c16.end > off ? W.c16.end : off;
+        off = W.c16.end > off ? W.c16.end : off;
+        if (fstore_ok && k.K > 1 && (k.mode == MRU_MODE_CAYLEY || k.mode == MRU_MODE_EXPM)) {
+            W.fstore = true;
+            W.fbuf = off;
+            off = round_up(off + (size_t)k.B * (size_t)k.L * (size_t)k.H * nn * sizeof(float), 256);
+        }
+        W.bytes = off;
         return W;
     }
     if (n32::supports(k, readout)) {
@@ -210,27 +219,30 @@ mru_status reset_status(void* ws, cudaStream_t s)
 
 namespace {
 // Kernel parameters and workspace layout of one mru_scan_fused call: the
-// embedding source, and the readout's query columns when there is one.
-void fused_call_plan(const mru_problem& p, const mru_readout* ro, KParams& k, Workspace& W)
+// embedding source, and the readout's query columns when there is one.  The
+// layout that keeps F in the workspace is taken when ws_bytes holds it, else
+// the one that forms F twice.
+void fused_call_plan(const mru_problem& p, const mru_readout* ro, KParams& k, Workspace& W, size_t ws_bytes)
 {
     k = make_params(p, SRC_EMBEDDING, ro != nullptr);
     if (ro) {
         k.rq = ro->q == 0 ? 1 : ro->q;
         k.u_hs = ro->u_per_head ? (int64_t)p.n * k.rq : 0;
     }
-    W = layout(k, ro != nullptr);
+    W = layout(k, ro != nullptr, true);
+    if (W.bytes > ws_bytes) W = layout(k, ro != nullptr, false);
 }
 }  // namespace
 
-// Workspace bytes mru_scan_fused needs for this problem with this output
-// form (the readout's query-column count and per-head layout included);
-// 0 for an invalid problem.
+// The least workspace mru_scan_fused accepts for this problem with this
+// output form (the readout's query-column count and per-head layout
+// included); 0 for an invalid problem.
 size_t fused_workspace_bytes(const mru_problem& p, const mru_readout* ro)
 {
     if (check_problem(&p) != MRU_OK) return 0;
     KParams k;
     Workspace W;
-    fused_call_plan(p, ro, k, W);
+    fused_call_plan(p, ro, k, W, 0);
     return W.bytes;
 }
 
@@ -357,7 +369,7 @@ mru_status mru_scan_fused(const mru_problem* p, const void* x, const float* S0, 
     }
     KParams k;
     Workspace W;
-    fused_call_plan(*p, ro, k, W);
+    fused_call_plan(*p, ro, k, W, ws_bytes);
     if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = reset_status(ws, s)) != MRU_OK) return st;
@@ -390,7 +402,8 @@ mru_status mru_scan_fused_host(const mru_problem* p, const void* x_host, const f
         k.rq = ro->q == 0 ? 1 : ro->q;
         k.u_hs = ro->u_per_head ? (int64_t)p->n * k.rq : 0;
     }
-    const Workspace W = layout(k, readout);
+    Workspace W = layout(k, readout, true);
+    if (ws_bytes < W.bytes) W = layout(k, readout, false);
     if (ws_bytes < W.bytes) return MRU_ERR_WORKSPACE;
     cudaStream_t sc = reinterpret_cast<cudaStream_t>(compute_stream);
     cudaStream_t si = reinterpret_cast<cudaStream_t>(h2d_stream);
@@ -460,7 +473,7 @@ mru_status mru_scan_fused_host(const mru_problem* p, const void* x_host, const f
         KParams ki = make_params(sub, SRC_EMBEDDING, readout);
         ki.rq = k.rq;
         ki.u_hs = k.u_hs;
-        const Workspace Wi = layout(ki, readout);
+        const Workspace Wi = layout(ki, readout, W.fstore);
         e = launch_scan(ki, xd + xoff * xb, s0, ro ? ro->u : nullptr, every, readout ? nullptr : out_dev + ooff,
                         readout ? out_dev + ooff : nullptr, every > 0 ? ro->snapshots + soff : nullptr, ws, Wi, sc,
                         nullptr);

@@ -123,6 +123,8 @@ struct Workspace {
     n16::CarryPlan c16;  // n = 16, three launches
     n16::FusedPlan f16;  // n = 16, the single-read fused launch
     bool fused;          // n = 16 runs k16_fused
+    size_t fbuf;         // float [B, L, H, n, n]: F = X - I of an orthogonal construction, written by the
+    bool fstore;         // reduce pass and read by the apply pass (n = 16, Cayley or exponential)
     size_t bytes;        // total
 };
 
@@ -193,14 +195,17 @@ constexpr int kSub = 8;           // chunks of the specialised kernels are multi
 bool supports(const KParams& p, bool readout);
 int32_t preferred_chunk(int64_t token_heads);
 CarryPlan carry_plan(int64_t nseq, int64_t K, size_t off);
+// fout: for the Cayley map and the exponential, where every token's F = X - I
+// goes (x's layout) for the apply pass to read, or null.
 cudaError_t launch_reduce(const KParams& p, const float* x, float* totals, const CarryPlan& cp, char* ws,
-                          uint32_t* status, cudaStream_t s);
+                          uint32_t* status, float* fout, cudaStream_t s);
 cudaError_t launch_carry(const KParams& p, const float* totals, const CarryPlan& cp, char* ws, const float* S0,
                          cudaStream_t s);
 // direct: a single-chunk problem (K = 1), run by the apply pass alone with
 // the carry S0 (or I when S0 is null); no reduce or carry launch precedes it.
+// pre_transformed: x holds the F = X - I the reduce pass wrote (not direct).
 cudaError_t launch_apply(const KParams& p, const float* x, const CarryPlan& cp, const char* ws, float* S_out,
-                         uint32_t* status, const float* S0, bool direct, cudaStream_t s);
+                         uint32_t* status, const float* S0, bool direct, bool pre_transformed, cudaStream_t s);
 // The single-read fused scan (one launch after a memset of its control block).
 FusedPlan fused_plan(const KParams& p, size_t off);
 cudaError_t launch_fused(const KParams& p, const FusedPlan& fp, char* ws, const float* x, const float* S0,

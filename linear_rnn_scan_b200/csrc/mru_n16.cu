@@ -1102,12 +1102,15 @@ __device__ __forceinline__ void direct_carry(const float* in, bool has_s0, int l
 // without the identity, whose uncorrected products alpha M could leave the
 // fp32 range) the chain takes every token's scale as it goes; otherwise it
 // runs on the uncorrected matrices and the carry kernel applies the
-// determinant correction of each total.  CTA 0 also zeroes the carry scan's
-// counters (the carry kernel runs after this launch).
+// determinant correction of each total.  With an orthogonal construction
+// (Tr 1 or 2) and fout non-null, every token's F = X - I is also written to
+// fout (x's layout), so that the apply pass reads F instead of forming it
+// again.  CTA 0 also zeroes the carry scan's counters (the carry kernel runs
+// after this launch).
 template <bool PerToken, int Tr = 0>
 __global__ void __launch_bounds__(RWARPS * 32, 2)
 k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, unsigned* ctr, int64_t nctr,
-           uint32_t* status)
+           uint32_t* status, float* __restrict__ fout)
 {
     if (blockIdx.x == 0)
         for (int64_t i = threadIdx.x; i < nctr; i += blockDim.x) ctr[i] = 0u;
@@ -1149,6 +1152,17 @@ k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, u
                 stage_transform<Tr, RST>(p.alpha, sm.stage[cs], (1u << nt) - 1u, lane);
                 ca = 1.0f;
                 dv = 0.0f;
+                if (fout) {                                // F to HBM, x's layout (one copy per slice)
+                    float* fb = fout + (c.b * p.L * p.H + c.h) * NN + t0 * feed.tok;
+#pragma unroll
+                    for (int i = 0; i < RST * 2; ++i) {
+                        const int gi = lane + 32 * i;
+                        const int j = gi >> 6, gr = gi & 63, row = gr >> 2, c4 = gr & 3;
+                        if (j < nt)
+                            *reinterpret_cast<float4*>(fb + j * feed.tok + row * N + 4 * c4) =
+                                *reinterpret_cast<const float4*>(xs + j * NN + swz(row, 4 * c4));
+                    }
+                }
             }
 #pragma unroll
             for (int j = 0; j < RST; ++j) {
@@ -1177,7 +1191,9 @@ k16_reduce(KParams p, const float* __restrict__ x, float* __restrict__ totals, u
 
 // Apply pass: per chain the carry from the carry scan's factors, then
 // S_t = S_{t-1} + S_{t-1} F_t from S = carry, every S_t written, with the
-// per-token determinant scales factorised here.
+// per-token determinant scales factorised here.  Tr = 3: x holds F = X - I
+// already (the reduce pass wrote it), taken with scale 1 and no diagonal
+// term.
 template <bool Direct, int Tr = 0>
 __global__ void __launch_bounds__(AWARPS * 32, 3)
 k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, float* __restrict__ S_out,
@@ -1222,8 +1238,11 @@ k16_apply(KParams p, const float* __restrict__ x, CarryPlan cp, const char* ws, 
             __syncwarp();
             const float* xs = sm.stage[cs];
             const int nt = (c.tend - t0 < AST) ? (int)(c.tend - t0) : AST;
-            if (Tr != 0) {                                 // F itself now sits where M was
+            if (Tr == 1 || Tr == 2) {                      // F itself now sits where M was
                 stage_transform<Tr, AST>(p.alpha, sm.stage[cs], (1u << nt) - 1u, lane);
+                if (lane < AST) sm.cd[lane] = make_float2(1.0f, 0.0f);
+                __syncwarp();
+            } else if (Tr == 3) {
                 if (lane < AST) sm.cd[lane] = make_float2(1.0f, 0.0f);
                 __syncwarp();
             } else {
@@ -2442,7 +2461,7 @@ CarryPlan carry_plan(int64_t nseq, int64_t K, size_t off)
 }
 
 cudaError_t launch_reduce(const KParams& p, const float* x, float* totals, const CarryPlan& cp, char* ws,
-                          uint32_t* status, cudaStream_t s)
+                          uint32_t* status, float* fout, cudaStream_t s)
 {
     const int64_t nchains = p.B * p.H * p.K;
     if (nchains == 0) return cudaSuccess;
@@ -2461,7 +2480,7 @@ cudaError_t launch_reduce(const KParams& p, const float* x, float* totals, const
         cudaSuccess)
         return e;
     kern<<<grid, RWARPS * 32, sm, s>>>(p, x, totals, reinterpret_cast<unsigned*>(ws + cp.ctr_begin),
-                                       (int64_t)(cp.ctr_bytes / sizeof(unsigned)), status);
+                                       (int64_t)(cp.ctr_bytes / sizeof(unsigned)), status, tr != 0 ? fout : nullptr);
     return cudaGetLastError();
 }
 
@@ -2610,20 +2629,21 @@ cudaError_t launch_bwd_apply(const KParams& p, const float* x, const float* S0, 
 }
 
 cudaError_t launch_apply(const KParams& p, const float* x, const CarryPlan& cp, const char* ws, float* S_out,
-                         uint32_t* status, const float* S0, bool direct, cudaStream_t s)
+                         uint32_t* status, const float* S0, bool direct, bool pre_transformed, cudaStream_t s)
 {
     const int64_t nchains = p.B * p.H * p.K;
     if (nchains == 0) return cudaSuccess;
     if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const size_t sm = sizeof(ASmem) * AWARPS;
-    const int tr = transform_of(p);
+    const int tr = pre_transformed && !direct ? 3 : transform_of(p);
     auto kern = tr == 1   ? (direct ? k16_apply<true, 1> : k16_apply<false, 1>)
                 : tr == 2 ? (direct ? k16_apply<true, 2> : k16_apply<false, 2>)
+                : tr == 3 ? k16_apply<false, 3>
                           : (direct ? k16_apply<true> : k16_apply<false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     unsigned grid = 0;
-    const int slot = tr == 1 ? (direct ? 8 : 7) : tr == 2 ? (direct ? 13 : 12) : (direct ? 3 : 2);
+    const int slot = tr == 1 ? (direct ? 8 : 7) : tr == 2 ? (direct ? 13 : 12) : tr == 3 ? 14 : (direct ? 3 : 2);
     if ((e = persistent_grid(slot, (const void*)kern, AWARPS * 32, sm, AWARPS,
                              nchains, grid)) !=
         cudaSuccess)

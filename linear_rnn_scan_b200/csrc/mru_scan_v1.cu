@@ -1699,7 +1699,7 @@ cudaError_t scan_fast16(const KParams& p, const void* src, const float* S0, floa
     if (p.K == 1) {
         // one chunk per sequence: the apply pass alone, from S0
         profile_mark(0, 0, s);
-        if ((e = n16::launch_apply(p, x, W.c16, ws, S_out, status, S0, true, s)) != cudaSuccess) return e;
+        if ((e = n16::launch_apply(p, x, W.c16, ws, S_out, status, S0, true, false, s)) != cudaSuccess) return e;
         profile_mark(0, 1, s);
         if (launches) *launches = 1;
         return cudaGetLastError();
@@ -1712,13 +1712,16 @@ cudaError_t scan_fast16(const KParams& p, const void* src, const float* S0, floa
         return cudaGetLastError();
     }
     profile_mark(0, 0, s);
-    if ((e = n16::launch_reduce(p, x, totals, W.c16, ws, status, s)) != cudaSuccess) return e;
+    float* fbuf = W.fstore ? reinterpret_cast<float*>(ws + W.fbuf) : nullptr;
+    if ((e = n16::launch_reduce(p, x, totals, W.c16, ws, status, fbuf, s)) != cudaSuccess) return e;
     profile_mark(0, 1, s);
     profile_mark(1, 0, s);
     if ((e = n16::launch_carry(p, totals, W.c16, ws, S0, s)) != cudaSuccess) return e;
     profile_mark(1, 1, s);
     profile_mark(2, 0, s);
-    if ((e = n16::launch_apply(p, x, W.c16, ws, S_out, status, nullptr, false, s)) != cudaSuccess) return e;
+    if ((e = n16::launch_apply(p, fbuf ? fbuf : x, W.c16, ws, S_out, status, nullptr, false, fbuf != nullptr, s)) !=
+        cudaSuccess)
+        return e;
     profile_mark(2, 1, s);
     if (launches) *launches = 3;
     return cudaGetLastError();

@@ -118,3 +118,34 @@ def test_noalloc_rejects_problems_beyond_the_scratch():
     assert rc == mru.ERR_WORKSPACE
     bad = mru.problem(1, 1, 8, 12)
     assert mru.scan_fused_noalloc(bad, fake, None, None, 2 * fake, None, None, 0) == mru.ERR_UNSUPPORTED
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mode", [gen.MODE_CAYLEY, gen.MODE_EXPM])
+def test_orthogonal_maps_form_F_once_or_twice_alike(mode):
+    """At n = 16 the Cayley map and the exponential keep every token's
+    F = X - I in the workspace when it fits (the reduce pass writes it, the
+    apply pass reads it); in the fixed scratch it does not fit here (32 MiB
+    of F), so the passes form F twice.  Both form it with the same code on
+    the same slice: the states agree bit for bit, and with the oracle."""
+    t = torch()
+    if not t.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    w = gen.Workload("noalloc_orth", B=4, H=4, L=2048, n=16, x_dtype="f32", mode=mode, alpha=0.0125, seed=9101)
+    p = mru.problem_from_workload(w, chunk=32)
+    assert w.B * w.L * w.H * 16 * 16 * 4 > mru.NOALLOC_SCRATCH_BYTES
+    x_np = gen.make_x(w)
+    x = to_device_x(x_np)
+    S_ref = mru.scan_fused_t(p, x)                 # caller workspace: F kept
+    S = t.full_like(S_ref, float("nan"))
+    status = t.full((1,), 7, dtype=t.int32, device="cuda")
+    stream = t.cuda.current_stream().cuda_stream
+    rc = mru.scan_fused_noalloc(p, x.data_ptr(), None, None, S.data_ptr(), None, status.data_ptr(), stream)
+    assert rc == mru.OK, mru.status_string(rc)
+    t.cuda.synchronize()
+    assert int(status.item()) == 0
+    got, ref = S.cpu().numpy(), S_ref.cpu().numpy()
+    assert np.array_equal(got, ref)
+    bh = np.array([0, 7, 15])
+    e = compare_S(w, x_np, got, bh=bh)
+    assert e["max"] <= TOL_FP32, e
