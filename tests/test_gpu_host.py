@@ -12,7 +12,7 @@ import pytest
 from linear_rnn_scan_b200 import inputs as gen
 from linear_rnn_scan_b200 import mru
 
-from gpu_helpers import compare_S, run_fused, to_device_x, tol_for_problem, torch
+from gpu_helpers import compare_readout, compare_S, run_fused, to_device_x, tol_for_problem, torch
 
 pytestmark = pytest.mark.gpu
 
@@ -72,6 +72,8 @@ def test_along_batch_matches_device_call_exactly(n, mode, dtype, pieces):
     S_host, _, st = _run_host(w, x, pieces, S0=S0)
     assert st == mru.OK
     assert np.array_equal(S_host, S_dev)
+    e = compare_S(w, x, S_host, S0=S0)                 # and against the oracle directly
+    assert e["count"] == w.B * w.H * w.L and e["max"] <= tol_for_problem(w), e
 
 
 @pytest.mark.parametrize("n,mode", [(16, gen.MODE_DETNORM), (4, gen.MODE_RESHAPE), (32, gen.MODE_EXPM)])
@@ -95,6 +97,9 @@ def test_readout_along_batch_matches_device_call_exactly():
     o_host, sn_host, st = _run_host(w, x, 0, u=U, every=128)
     assert st == mru.OK
     assert np.array_equal(o_host, o_dev) and np.array_equal(sn_host, sn_dev)
+    e = compare_readout(w, x, o_host, sn_host, U, 128)  # and against the oracle directly
+    tol = tol_for_problem(w)
+    assert e["o"]["max"] <= tol and e["snap"]["max"] <= tol, e
 
 
 def test_single_batch_readout_is_one_piece():
