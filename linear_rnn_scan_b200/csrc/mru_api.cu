@@ -201,6 +201,17 @@ BwdWorkspace bwd_layout(const KParams& k)
     W.gloc = off; off = round_up(off + chains * nn * sizeof(float), 256);
     W.wq = off;   off = round_up(off + chains * nn * sizeof(float), 256);
     W.gin = off;  off = round_up(off + chains * nn * sizeof(float), 256);
+    // groups of about sqrt(K) chunks: the serial steps are G within the groups
+    // and NG across them
+    W.gshift = 0;
+    while (((int64_t)1 << (2 * W.gshift)) < k.K) ++W.gshift;
+    W.NG = k.K > 0 ? (k.K + ((int64_t)1 << W.gshift) - 1) >> W.gshift : 0;
+    const size_t groups = (size_t)(k.B * k.H) * (size_t)W.NG;
+    W.sg = off;   off = round_up(off + chains * nn * sizeof(double), 256);
+    W.sw = off;   off = round_up(off + chains * nn * sizeof(double), 256);
+    W.gg = off;   off = round_up(off + groups * nn * sizeof(double), 256);
+    W.gw = off;   off = round_up(off + groups * nn * sizeof(double), 256);
+    W.ginr = off; off = round_up(off + groups * nn * sizeof(double), 256);
     W.bytes = off;
     return W;
 }

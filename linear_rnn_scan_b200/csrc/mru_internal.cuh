@@ -134,6 +134,14 @@ struct BwdWorkspace {
     size_t gloc;         // float [B*H, K, n, n]  local gradient at each chunk's first token
     size_t wq;           // float [B*H, K, n, n]  W_k - I, W_k = X_{t0+1} ... X_{t1}
     size_t gin;          // float [B*H, K, n, n]  gradient entering each chunk from the right
+    // The chunk-gradient scan in groups of G = 2^gshift chunks (NG per
+    // sequence): per chunk the composition of the maps of the later chunks of
+    // its group (g part, W part in split form), per group its whole
+    // composition and the gradient entering its last chunk (all fp64).
+    int32_t gshift;
+    int64_t NG;
+    size_t sg, sw;       // double [B*H, K, n, n]
+    size_t gg, gw, ginr; // double [B*H, NG, n, n]
     size_t bytes;
 };
 

@@ -785,9 +785,10 @@ k_fixup(KParams p, const float* carry, const float* u, int64_t snap_every, float
 //                 right: the local G at t0 (g_k) and W_k - I with
 //                 W_k = X_{t0+1} ... X_{t1} (through the next chunk's first
 //                 matrix; split form, left multiplications);
-//   k_bwd_carry   per sequence, right to left in fp64: the gradient entering
-//                 chunk k from the right, Gin_{K-1} = 0,
-//                 Gin_{k-1} = g_k + Gin_k W_k^T;
+//   k_bwd_carry, or k_bwd_group / k_bwd_top / k_bwd_fix for larger
+//                 problems: right to left in fp64 (serially, or in groups of
+//                 about sqrt(K) chunks), the gradient entering chunk k from
+//                 the right, Gin_{K-1} = 0, Gin_{k-1} = g_k + Gin_k W_k^T;
 //   k_bwd_apply   per chunk: G from Gin_k down to t0 again, dX_t from the
 //                 forward states, and the construction's chain rule to the
 //                 embedding gradient (reshape: alpha dX; determinant-corrected:
@@ -929,6 +930,161 @@ k_bwd_local(KParams p, const void* src, const float* __restrict__ dS, float* __r
     }
 }
 
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes)
+{
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+// ---- the chunk-gradient scan, in groups --------------------------------------
+//
+// Chunk k's map is A_k(G) = g_k + G W_k^T (g_k = gloc_k, W_k = I + Wq_k);
+// the gradient entering chunk k from the right is
+// Gin_k = (A_{k+1} o ... o A_{K-1})(0).  The maps compose associatively,
+// (g_a, W_a) o (g_b, W_b) = (g_a + g_b W_a^T, W_a W_b), so the right-to-left
+// scan runs in groups of G chunks: k_bwd_group walks each group from its
+// right end and records for every chunk the composition of the group's later
+// chunks (the identity for the last) and the group's whole composition;
+// k_bwd_top walks the groups from the right (the gradient entering each
+// group's last chunk); k_bwd_fix applies each chunk's recorded composition
+// to its group's entering gradient.  W parts in split form (W - I), all in
+// fp64; the serial steps are G + NG instead of K.
+
+template <int N>
+__global__ void __launch_bounds__(kThreads)
+k_bwd_group(KParams p, const float* __restrict__ gloc, const float* __restrict__ Wq, int gshift, int64_t NG,
+            double* __restrict__ sg, double* __restrict__ sw, double* __restrict__ gg, double* __restrict__ gw)
+{
+    constexpr int NN = N * N;
+    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    extern __shared__ double dsm[];
+    double* cg = dsm;                       // the running composition's g part
+    double* cw = cg + NN;                   // its W part, W - I
+    double* sq = cw + NN;                   // Q_k = W_k - I of the chunk at hand
+    const int tid = threadIdx.x;
+    const int64_t seq = blockIdx.x / NG, grp = blockIdx.x - seq * NG;
+    const int64_t k0 = grp << gshift;
+    const int64_t k1 = (k0 + ((int64_t)1 << gshift) < p.K) ? k0 + ((int64_t)1 << gshift) : p.K;
+    for (int e = tid; e < NN; e += kThreads) {
+        cg[e] = 0.0;
+        cw[e] = 0.0;
+    }
+    __syncthreads();
+    for (int64_t k = k1 - 1; k >= k0; --k) {
+        const int64_t chain = seq * p.K + k;
+        for (int e = tid; e < NN; e += kThreads) {
+            sg[chain * NN + e] = cg[e];
+            sw[chain * NN + e] = cw[e];
+            sq[e] = (double)Wq[chain * NN + e];
+        }
+        __syncthreads();
+        double ag[PER], aw[PER];
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            double a = 0.0, w = 0.0;
+            if (e < NN) {
+                const int i = e / N, j = e % N;
+                for (int q = 0; q < N; ++q) {
+                    a = fma(cg[i * N + q], sq[j * N + q], a);     // cg Q^T
+                    w = fma(sq[i * N + q], cw[q * N + j], w);     // Q cw
+                }
+            }
+            ag[r] = a;
+            aw[r] = w;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            if (e < NN) {
+                cg[e] = (double)gloc[chain * NN + e] + (cg[e] + ag[r]);   // g_k + cg (I + Q)^T
+                cw[e] = sq[e] + (cw[e] + aw[r]);                         // (I + Q)(I + cw) - I
+            }
+        }
+        __syncthreads();
+    }
+    for (int e = tid; e < NN; e += kThreads) {
+        gg[blockIdx.x * (int64_t)NN + e] = cg[e];
+        gw[blockIdx.x * (int64_t)NN + e] = cw[e];
+    }
+}
+
+template <int N>
+__global__ void __launch_bounds__(kThreads)
+k_bwd_top(int64_t NG, const double* __restrict__ gg, const double* __restrict__ gw, double* __restrict__ ginr)
+{
+    constexpr int NN = N * N;
+    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    extern __shared__ double dsm[];
+    double* cur = dsm;
+    double* w = cur + NN;
+    const int tid = threadIdx.x;
+    const int64_t base = (int64_t)blockIdx.x * NG;
+    for (int e = tid; e < NN; e += kThreads) cur[e] = 0.0;
+    __syncthreads();
+    for (int64_t grp = NG - 1; grp >= 0; --grp) {
+        const int64_t gi = (base + grp) * NN;
+        for (int e = tid; e < NN; e += kThreads) {
+            ginr[gi + e] = cur[e];
+            w[e] = gw[gi + e];
+        }
+        __syncthreads();
+        double acc[PER];
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            double a = 0.0;
+            if (e < NN) {
+                const int i = e / N, j = e % N;
+                for (int q = 0; q < N; ++q) a = fma(cur[i * N + q], w[j * N + q], a);   // cur W_G^T (split)
+            }
+            acc[r] = a;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int e = tid + r * kThreads;
+            if (e < NN) cur[e] = gg[gi + e] + (cur[e] + acc[r]);
+        }
+        __syncthreads();
+    }
+}
+
+template <int N>
+__global__ void __launch_bounds__(kThreads)
+k_bwd_fix(KParams p, int gshift, int64_t NG, const double* __restrict__ sg, const double* __restrict__ sw,
+          const double* __restrict__ ginr, float* __restrict__ Gin)
+{
+    constexpr int NN = N * N;
+    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    extern __shared__ double dsm[];
+    double* gr = dsm;
+    double* w = gr + NN;
+    const int tid = threadIdx.x;
+    const int64_t chain = blockIdx.x;
+    const int64_t seq = chain / p.K, k = chain - seq * p.K;
+    const int64_t gi = (seq * NG + (k >> gshift)) * NN;
+    for (int e = tid; e < NN; e += kThreads) {
+        gr[e] = ginr[gi + e];
+        w[e] = sw[chain * NN + e];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+        const int e = tid + r * kThreads;
+        if (e < NN) {
+            const int i = e / N, j = e % N;
+            double a = 0.0;
+            for (int q = 0; q < N; ++q) a = fma(gr[i * N + q], w[j * N + q], a);       // Ginr W_suf^T (split)
+            Gin[chain * NN + e] = (float)(sg[chain * NN + e] + (gr[e] + a));
+        }
+    }
+}
+
+// The same scan serially, one CTA per sequence right to left (fewer
+// launches and no per-chunk records: the choice for small problems).
 template <int N>
 __global__ void __launch_bounds__(kThreads)
 k_bwd_carry(KParams p, const float* __restrict__ gloc, const float* __restrict__ Wq, float* __restrict__ Gin)
@@ -969,6 +1125,41 @@ k_bwd_carry(KParams p, const float* __restrict__ gloc, const float* __restrict__
         }
         __syncthreads();
     }
+}
+
+// The chunk-gradient scan: Gin from gloc, Wq.  Serially per sequence while
+// K n^3 is at most 2^20 (measured on B200: B8 H8 L4096, n = 16, K = 128 takes
+// 0.082 ms serially, 0.105 ms in groups), else in groups (B1 H8 L262144,
+// n = 16: 0.63 ms serially, 0.14 ms in groups; n = 32, K = 128: 0.33 and
+// 0.27 ms).
+template <int N>
+cudaError_t bwd_carry_scan(const KParams& p, const float* gloc, const float* Wq, float* Gin, char* ws,
+                           const BwdWorkspace& W, cudaStream_t s)
+{
+    constexpr int NN = N * N;
+    const int64_t BH = p.B * p.H, chains = BH * p.K;
+    if (chains == 0) return cudaSuccess;
+    if (p.K * (int64_t)N * N * N <= ((int64_t)1 << 20)) {
+        const size_t sm_carry = sizeof(double) * 2 * NN;
+        cudaError_t e = set_smem(k_bwd_carry<N>, sm_carry);
+        if (e != cudaSuccess) return e;
+        k_bwd_carry<N><<<(unsigned)BH, kThreads, sm_carry, s>>>(p, gloc, Wq, Gin);
+        return cudaGetLastError();
+    }
+    double* sg = reinterpret_cast<double*>(ws + W.sg);
+    double* sw = reinterpret_cast<double*>(ws + W.sw);
+    double* gg = reinterpret_cast<double*>(ws + W.gg);
+    double* gw = reinterpret_cast<double*>(ws + W.gw);
+    double* ginr = reinterpret_cast<double*>(ws + W.ginr);
+    const size_t sm3 = sizeof(double) * 3 * NN, sm2 = sizeof(double) * 2 * NN;
+    cudaError_t e;
+    if ((e = set_smem(k_bwd_group<N>, sm3)) != cudaSuccess) return e;
+    if ((e = set_smem(k_bwd_top<N>, sm2)) != cudaSuccess) return e;
+    if ((e = set_smem(k_bwd_fix<N>, sm2)) != cudaSuccess) return e;
+    k_bwd_group<N><<<(unsigned)(BH * W.NG), kThreads, sm3, s>>>(p, gloc, Wq, W.gshift, W.NG, sg, sw, gg, gw);
+    k_bwd_top<N><<<(unsigned)BH, kThreads, sm2, s>>>(W.NG, gg, gw, ginr);
+    k_bwd_fix<N><<<(unsigned)chains, kThreads, sm2, s>>>(p, W.gshift, W.NG, sg, sw, ginr, Gin);
+    return cudaGetLastError();
 }
 
 // dA = L(A^T, dX), the adjoint of the Frechet derivative of exp at A (the
@@ -1252,12 +1443,6 @@ template <int N>
 cudaError_t backward_n(const KParams& p, const void* src, const float* S0, const float* S_fwd, const float* dS,
                        float* dx, float* dS0, char* ws, const BwdWorkspace& W, cudaStream_t s);
 
-template <typename K>
-cudaError_t set_smem(K kernel, size_t bytes)
-{
-    if (bytes <= 48 * 1024) return cudaSuccess;
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-}
 
 template <int N>
 cudaError_t backward_n(const KParams& p, const void* src, const float* S0, const float* S_fwd, const float* dS,
@@ -1279,10 +1464,8 @@ cudaError_t backward_n(const KParams& p, const void* src, const float* S0, const
     const int gfl_local = 5 * NN + 4 * N + 8;
     const int gfl_apply = 8 * NN + 4 * N + 8 + kThreads / 32;
     const size_t sm_local = sizeof(float) * gfl_local * GPB;
-    const size_t sm_carry = sizeof(double) * 2 * NN;
     const size_t sm_apply = sizeof(float) * gfl_apply * GPB;
     const unsigned grid = (unsigned)((chains + GPB - 1) / GPB);
-    if ((e = set_smem(k_bwd_carry<N>, sm_carry)) != cudaSuccess) return e;
     if (N == 16 && n16::supports_backward(p)) {
         // n = 16 on the tensor cores; the chunk-gradient scan stays generic
         const float* x = reinterpret_cast<const float*>(src);
@@ -1290,7 +1473,7 @@ cudaError_t backward_n(const KParams& p, const void* src, const float* S0, const
         if ((e = n16::launch_bwd_local(p, x, dS, gloc, Wq, status, s)) != cudaSuccess) return e;
         profile_mark(0, 1, s);
         profile_mark(1, 0, s);
-        k_bwd_carry<N><<<(unsigned)BH, kThreads, sm_carry, s>>>(p, gloc, Wq, Gin);
+        if ((e = bwd_carry_scan<N>(p, gloc, Wq, Gin, ws, W, s)) != cudaSuccess) return e;
         profile_mark(1, 1, s);
         profile_mark(2, 0, s);
         if ((e = n16::launch_bwd_apply(p, x, S0, S_fwd, dS, Gin, dx, dS0, status, s)) != cudaSuccess) return e;
@@ -1303,7 +1486,7 @@ cudaError_t backward_n(const KParams& p, const void* src, const float* S0, const
         if ((e = n32::launch_bwd_local(p, src, dS, gloc, Wq, s)) != cudaSuccess) return e;
         profile_mark(0, 1, s);
         profile_mark(1, 0, s);
-        k_bwd_carry<N><<<(unsigned)BH, kThreads, sm_carry, s>>>(p, gloc, Wq, Gin);
+        if ((e = bwd_carry_scan<N>(p, gloc, Wq, Gin, ws, W, s)) != cudaSuccess) return e;
         profile_mark(1, 1, s);
         profile_mark(2, 0, s);
         if ((e = n32::launch_bwd_apply(p, src, S0, S_fwd, dS, Gin, dx, dS0, s)) != cudaSuccess) return e;
@@ -1316,7 +1499,7 @@ cudaError_t backward_n(const KParams& p, const void* src, const float* S0, const
     k_bwd_local<N, Grp><<<grid, kThreads, sm_local, s>>>(p, src, dS, gloc, Wq, status, gfl_local);
     profile_mark(0, 1, s);
     profile_mark(1, 0, s);
-    k_bwd_carry<N><<<(unsigned)BH, kThreads, sm_carry, s>>>(p, gloc, Wq, Gin);
+    if ((e = bwd_carry_scan<N>(p, gloc, Wq, Gin, ws, W, s)) != cudaSuccess) return e;
     profile_mark(1, 1, s);
     profile_mark(2, 0, s);
     k_bwd_apply<N, Grp><<<grid, kThreads, sm_apply, s>>>(p, src, S0, S_fwd, dS, Gin, dx, dS0, status, gfl_apply);

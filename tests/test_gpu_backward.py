@@ -234,3 +234,29 @@ def test_backward_readout_against_oracle(n, mode, x_dtype, ushape, every, with_s
     if with_s0:
         e0 = _rel(dS0.cpu().numpy().astype(np.float64).reshape(B, H, n * n), dS0_o.reshape(B, H, n * n), axis=-1)
         assert e0.max() <= TOL_BWD, e0.max()
+
+
+@pytest.mark.parametrize("n,mode,dtype,L,chunk", [
+    (16, gen.MODE_DETNORM, "f32", 530 * 2 + 3, 2),   # K = 532: groups of 32, the last one ragged
+    (8, gen.MODE_DETNORM, "f32", 4200, 1),           # K = 4200 at n = 8: groups of 128
+    (32, gen.MODE_LDU, "bf16", 77 * 2, 2),           # K = 77 at n = 32: groups of 16, the last one ragged
+])
+def test_backward_grouped_chunk_gradient_scan(n, mode, dtype, L, chunk):
+    """Problems large enough (K n^3 > 2^20) for the chunk-gradient scan to run
+    in groups (group suffix compositions, a scan over the groups, a fix-up per
+    chunk) instead of serially: the gradients still match the oracle's fp64
+    backward, with S0, over ragged last groups (determinant-corrected, alpha
+    small: the states stay in range over thousands of tokens)."""
+    alpha = 1.0 if mode == gen.MODE_LDU else 0.05 / np.sqrt(n)
+    w = gen.Workload(f"g{n}", B=1, H=2, L=L, n=n, x_dtype=dtype, mode=mode, alpha=float(alpha), seed=900 + n)
+    K = -(-L // chunk)
+    assert K * n ** 3 > 2 ** 20
+    x = gen.make_x(w)
+    S0 = gen.make_S0(w, seed=901)
+    dS = np.random.default_rng(902).standard_normal((w.B, w.L, w.H, n, n)).astype(np.float32)
+    dx, dS0, st = _run(w, x, S0, dS, chunk=chunk)
+    assert st == mru.OK
+    dx_o, dS0_o = oracle.backward(oracle_problem(w), x, dS.astype(np.float64), S0=S0.astype(np.float64))
+    e_dx = _rel(dx.reshape(w.B, w.L, w.H, n * n), dx_o.reshape(w.B, w.L, w.H, n * n), axis=-1)
+    e_s0 = _rel(dS0.reshape(w.B, w.H, n * n), dS0_o.reshape(w.B, w.H, n * n), axis=-1)
+    assert e_dx.max() <= TOL_BWD and e_s0.max() <= TOL_BWD, (e_dx.max(), np.median(e_dx), e_s0.max())
