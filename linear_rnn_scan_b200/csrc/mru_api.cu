@@ -47,11 +47,12 @@ bool fast32_eligible(const mru_problem& p, bool readout)
 // longer chunks mean fewer chunk totals for the carry scan and the fix-up.
 // Measured on B200 for B2 H4 L16384: 32 -> 2.56 ms, 64 -> 2.25, 128 -> 2.15,
 // 256 -> 2.34.
+// Every state (no readout) takes the same path when tf32 is asked for
+// explicitly (the fix-up writes each token's state as a snapshot).
 bool fast64_eligible(const mru_problem& p, bool readout)
 {
-    return p.n == 64 && p.x_dtype == MRU_F32 && readout &&
-           (p.mode == MRU_MODE_DETNORM || p.mode == MRU_MODE_RESHAPE) &&
-           (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32);
+    return p.n == 64 && p.x_dtype == MRU_F32 && (p.mode == MRU_MODE_DETNORM || p.mode == MRU_MODE_RESHAPE) &&
+           (readout ? (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32) : p.math == MRU_MATH_TF32);
 }
 
 int32_t n64_chunk(int64_t token_heads)

@@ -543,8 +543,8 @@ k64_fixup(KParams p, const float* __restrict__ carry, const float* __restrict__ 
 {
     extern __shared__ __align__(16) float fsm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, qq = lane & 3;
-    const int q = p.rq, nq = N * q;
-    const int tpb = FX_COLS / q > 0 ? FX_COLS / q : 1;      // tokens per staged block
+    const int q = p.rq, nq = N * q;                         // q = 0: snapshots only (full states)
+    const int tpb = q > 0 && FX_COLS / q > 0 ? FX_COLS / q : 1;   // tokens per staged block
     const int TS = nq + 4;                                  // padded words per staged token
     float* sCU = fsm + 2 * FX_BUF;                          // C U, [64][q]
     const int64_t chain = blockIdx.x;
@@ -571,7 +571,7 @@ k64_fixup(KParams p, const float* __restrict__ carry, const float* __restrict__ 
         }
         asm volatile("cp.async.commit_group;\n" ::);
     };
-    if (t0 < t1) issue(fsm + FX_BUF, t0);
+    if (q > 0 && t0 < t1) issue(fsm + FX_BUF, t0);
     // C U (U staged as one token of the block layout in the first buffer)
     for (int e = tid; e < nq; e += THREADS) fsm[e] = u[h * p.u_hs + e];
     __syncthreads();
@@ -588,7 +588,7 @@ k64_fixup(KParams p, const float* __restrict__ carry, const float* __restrict__ 
     __syncthreads();
     // the chunk's tokens, a block at a time: o = C U + C V
     int cur = 1;
-    for (int64_t tb = t0; tb < t1; tb += tpb) {
+    for (int64_t tb = t0; q > 0 && tb < t1; tb += tpb) {
         const int64_t tn = tb + tpb;
         if (tn < t1) issue(fsm + (cur ^ 1) * FX_BUF, tn);
         else asm volatile("cp.async.commit_group;\n" ::);
@@ -1246,11 +1246,14 @@ bool use_tcgen05()
     return v != nullptr && v[0] == '1' && v[1] == 0;
 }
 
+// The readout form (tf32 unless another arithmetic is asked for), and every
+// state when tf32 is asked for explicitly: the chunk kernel then records each
+// Q_t as a snapshot and the fix-up writes S_t = C + C Q_t for every token.
 bool supports(const KParams& p, bool readout)
 {
-    return p.n == N && p.src == SRC_EMBEDDING && p.x_dtype == MRU_F32 && readout && p.K > 1 &&
+    return p.n == N && p.src == SRC_EMBEDDING && p.x_dtype == MRU_F32 && p.K > 1 &&
            (p.mode == MRU_MODE_DETNORM || p.mode == MRU_MODE_RESHAPE) &&
-           (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32);
+           (readout ? (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32) : p.math == MRU_MATH_TF32);
 }
 
 cudaError_t launch_chunk_readout(const KParams& p, const float* x, const float* u, int64_t snap_every,

@@ -1842,9 +1842,14 @@ cudaError_t scan_n(const KParams& p, const void* src, const float* S0, const flo
         if (launches) *launches = 1;
         return cudaGetLastError();
     }
-    if (N == 64 && o_out != nullptr && n64::supports(p, true)) {
-        if ((e = n64::launch_chunk_readout(p, reinterpret_cast<const float*>(src), u, snap_every, o_out, snaps,
-                                           totals, status, s)) != cudaSuccess)
+    // n = 64 on the tensor cores: the readout form, or every state as a
+    // snapshot at every token (no query columns)
+    const bool fast64 = N == 64 && n64::supports(p, o_out != nullptr);
+    KParams p64 = p;
+    if (fast64 && o_out == nullptr) p64.rq = 0;
+    if (fast64) {
+        if ((e = n64::launch_chunk_readout(p64, reinterpret_cast<const float*>(src), u, o_out ? snap_every : 1,
+                                           o_out, o_out ? snaps : S_out, totals, status, s)) != cudaSuccess)
             return e;
     } else {
         k_chunk_prefix<N, Grp><<<grid_chunk, kThreads, sm_chunk, s>>>(p, src, u, snap_every, S_out, o_out,
@@ -1861,8 +1866,10 @@ cudaError_t scan_n(const KParams& p, const void* src, const float* S0, const flo
     k_carry_final<N><<<(unsigned)chains, kThreads, sm_d, s>>>(p, local, gcarry, carry);
     profile_mark(3, 1, s);
     profile_mark(4, 0, s);
-    if (N == 64 && o_out != nullptr && n64::supports(p, true)) {
-        if ((e = n64::launch_fixup_readout(p, carry, u, snap_every, o_out, snaps, s)) != cudaSuccess) return e;
+    if (fast64) {
+        if ((e = n64::launch_fixup_readout(p64, carry, u, o_out ? snap_every : 1, o_out, o_out ? snaps : S_out, s)) !=
+            cudaSuccess)
+            return e;
     } else {
         k_fixup<N><<<(unsigned)chains, kThreads, sm_fix, s>>>(p, carry, u, snap_every, S_out, o_out, snaps);
     }

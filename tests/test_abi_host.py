@@ -72,9 +72,13 @@ def test_workspace_size(lib):
 def test_chunk_override(lib):
     p = mru.problem(2, 3, 100, 16, chunk=7)
     assert mru.chosen_chunk(p) == 7 and mru.chosen_chunk(p, readout=True) == 7
-    # the n = 64 readout path takes longer chunks than the state-writing one
+    # the n = 64 tensor-core path (the readout, and every state when tf32 is
+    # asked for, as this workload does) takes longer chunks than the generic
+    # state-writing one (fp32)
     p64 = mru.problem_from_workload(gen.WORKLOADS["n64_detnorm_readout_b2h4l16384"])
-    assert mru.chosen_chunk(p64, readout=True) == 128 and mru.chosen_chunk(p64) == 32
+    assert mru.chosen_chunk(p64, readout=True) == 128 and mru.chosen_chunk(p64) == 128
+    p64f = mru.problem_from_workload(gen.WORKLOADS["n64_detnorm_readout_b2h4l16384"], math="auto")
+    assert mru.chosen_chunk(p64f, readout=True) == 128 and mru.chosen_chunk(p64f) == 32
     assert mru.launch_count(p) >= 1
     assert mru.launch_count(mru.problem(0, 3, 100, 16)) == 0
 
@@ -152,6 +156,13 @@ def test_single_chunk_problems_take_one_launch(lib):
         assert mru.kernel_names(p, True)[0] == "k64_chunk_readout_tc" and mru.launch_count(p, True) == 5
     finally:
         os.environ.pop("MRU_N64_TCGEN05", None)
+    # every state at n = 64: the tensor-core path when tf32 is asked for, fp32 generic otherwise
+    p = mru.problem(2, 4, 4096, 64, mode=mru.MODE_DETNORM, alpha=0.01, math="tf32")
+    assert mru.kernel_names(p) == ["k64_chunk_readout", "k_carry_local", "k_carry_groups", "k_carry_final",
+                                   "k64_fixup"]
+    assert mru.effective_math(p) == "tf32"
+    p = mru.problem(2, 4, 4096, 64, mode=mru.MODE_DETNORM, alpha=0.01)
+    assert mru.kernel_names(p)[0] == "k_chunk_prefix" and mru.effective_math(p) == "fp32"
 
 
 def test_small_problems_choose_one_launch(lib):

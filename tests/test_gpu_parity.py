@@ -418,3 +418,22 @@ def test_parity_n16_carry_levels(B, H, L, chunk, mode, add_identity):
     e = compare_S(w, x, S, S0=S0)
     assert e["count"] == B * H * L
     assert e["max"] <= TOL_FP32, e
+
+
+@pytest.mark.parametrize("mode,add_id,L,chunk", [(gen.MODE_DETNORM, 1, 130, 16), (gen.MODE_RESHAPE, 1, 53, 16),
+                                                 (gen.MODE_DETNORM, 1, 257, 0)])
+@pytest.mark.parametrize("with_s0", [False, True])
+def test_n64_every_state_on_the_tensor_cores(mode, add_id, L, chunk, with_s0):
+    """n = 64 without the readout, tf32 asked for: the readout path's chunk
+    kernel records every Q_t as a snapshot and its fix-up writes
+    S_t = C + C Q_t for every token.  Every state within the tf32 gate."""
+    w = small(64, mode, B=2, H=3, L=L, add_identity=add_id, alpha=0.03 / 8, seed=770 + L).with_(math="tf32")
+    p = mru.problem_from_workload(w, chunk=chunk)
+    assert mru.kernel_names(p)[0] == "k64_chunk_readout"
+    x = gen.make_x(w)
+    S0 = gen.make_S0(w, seed=771) if with_s0 else None
+    S, st = run_fused(w, x, S0=S0, chunk=chunk)
+    assert st == mru.OK
+    e = compare_S(w, x, S, S0=S0)
+    assert e["count"] == w.B * w.L * w.H
+    assert e["max"] <= tol_for_problem(w, chunk=chunk), e
