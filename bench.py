@@ -175,7 +175,7 @@ def read_peaks():
 
 
 KERNEL_SOURCES = {"k16_": "mru_n16.cu", "k16b_": "mru_n16.cu", "k32_": "mru_n32.cu", "k32b_": "mru_n32.cu",
-                  "k64_": "mru_n64.cu",
+                  "k64_": "mru_n64.cu", "k64b_": "mru_n64_bwd.cu",
                   "k_level": "mru_carry.cu", "k_top": "mru_carry.cu", "k_down": "mru_carry.cu"}
 
 
@@ -678,7 +678,8 @@ def run_ours(args, w):
 def bwd_kernel_names(w):
     """The three launches of mru_scan_backward for this workload: the tensor-core
     passes where the library has them (n = 16 fp32 reshape / corrected with the
-    identity, n = 32 LDU bf16), the generic kernels otherwise; the chunk-gradient
+    identity, n = 32 LDU bf16, n = 64 fp32 reshape / corrected in tf32), the
+    generic kernels otherwise; the chunk-gradient
     scan between them is always the generic one ("chunk_scan": k_bwd_carry
     serially, or k_bwd_group, k_bwd_top and k_bwd_fix in groups for larger
     problems)."""
@@ -687,6 +688,8 @@ def bwd_kernel_names(w):
         return ["k16b_local", "chunk_scan", "k16b_apply"]
     if w.n == 32 and w.x_dtype == "bf16" and w.mode == gen.MODE_LDU:
         return ["k32b_local", "chunk_scan", "k32b_apply"]
+    if w.n == 64 and w.x_dtype == "f32" and w.math == "tf32" and w.mode in (gen.MODE_RESHAPE, gen.MODE_DETNORM):
+        return ["k64b_local", "chunk_scan", "k64b_apply"]
     return ["k_bwd_local", "chunk_scan", "k_bwd_apply"]
 
 

@@ -189,10 +189,13 @@ mru_status mru_scan_fused_host(const mru_problem* p, const void* x_host, const f
  *   dS0    [B, H, n, n] fp32 out, or NULL
  * Every pointer 16-byte aligned; dx and dS0 alias no input.  The workspace
  * holds mru_backward_workspace_size(p) bytes.  fp32-accurate arithmetic for
- * every n and mode: fp32 on the generic kernels, split tf32 on the tensor
- * cores for n = 16 (fp32 embeddings, reshape or corrected with the
- * identity), three-term split bf16 for n = 32 LDU (bf16 embeddings, exact
- * in bf16); fp64 for the right-to-left scan of the chunk gradients.  A
+ * every n and mode unless tf32 is asked for: fp32 on the generic kernels,
+ * split tf32 on the tensor cores for n = 16 (fp32 embeddings, reshape or
+ * corrected with the identity), three-term split bf16 for n = 32 LDU (bf16
+ * embeddings, exact in bf16).  n = 64 with p->math = MRU_MATH_TF32 (fp32
+ * embeddings, reshape or determinant-corrected): tf32 products on the
+ * tensor cores, the forward's tf32 arithmetic (chunks of 64 tokens by
+ * default).  fp64 for the right-to-left scan of the chunk gradients.  A
  * singular matrix sets MRU_ERR_SINGULAR in the workspace status word. */
 size_t mru_backward_workspace_size(const mru_problem* p);
 mru_status mru_scan_backward(const mru_problem* p, const void* x, const float* S0, const float* S_fwd,

@@ -260,6 +260,14 @@ cudaError_t launch_chunk_readout(const KParams& p, const float* x, const float* 
 // o_t = C U + C V_t and the snapshots C + C Q_t from the chains' carries C.
 cudaError_t launch_fixup_readout(const KParams& p, const float* carry, const float* u, int64_t snap_every,
                                  float* o_out, float* snaps, cudaStream_t s);
+// Backward on the tensor cores (mru_n64_bwd.cu) when tf32 is asked for:
+// local pass and apply pass; the chunk-gradient scan between them is the
+// generic one.
+bool supports_backward(const KParams& p);
+cudaError_t launch_bwd_local(const KParams& p, const float* x, const float* dS, float* gloc, float* Wq,
+                             uint32_t* status, cudaStream_t s);
+cudaError_t launch_bwd_apply(const KParams& p, const float* x, const float* S0, const float* S_fwd, const float* dS,
+                             const float* Gin, float* dx, float* dS0, uint32_t* status, cudaStream_t s);
 }  // namespace n64
 
 // Launchers (mru_scan_v1.cu).

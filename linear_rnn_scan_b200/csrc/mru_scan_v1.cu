@@ -949,7 +949,9 @@ cudaError_t set_smem(K kernel, size_t bytes)
 // k_bwd_top walks the groups from the right (the gradient entering each
 // group's last chunk); k_bwd_fix applies each chunk's recorded composition
 // to its group's entering gradient.  W parts in split form (W - I), all in
-// fp64; the serial steps are G + NG instead of K.
+// fp64 (the products by CarryMul: on the fp64 tensor cores for n >= 32, W
+// parts stored transposed where they multiply from the right); the serial
+// steps are G + NG instead of K.
 
 template <int N>
 __global__ void __launch_bounds__(kThreads)
@@ -957,16 +959,18 @@ k_bwd_group(KParams p, const float* __restrict__ gloc, const float* __restrict__
             double* __restrict__ sg, double* __restrict__ sw, double* __restrict__ gg, double* __restrict__ gw)
 {
     constexpr int NN = N * N;
-    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    using CM = CarryMul<N>;
+    constexpr int SP = CM::SP, PER = CM::PER;
     extern __shared__ double dsm[];
     double* cg = dsm;                       // the running composition's g part
-    double* cw = cg + NN;                   // its W part, W - I
-    double* sq = cw + NN;                   // Q_k = W_k - I of the chunk at hand
+    double* cw = cg + N * SP;               // its W part, W - I
+    double* sq = cw + N * SP;               // Q_k = W_k - I of the chunk at hand
+    double* sqt = sq + N * SP;              // Q_k^T
     const int tid = threadIdx.x;
     const int64_t seq = blockIdx.x / NG, grp = blockIdx.x - seq * NG;
     const int64_t k0 = grp << gshift;
     const int64_t k1 = (k0 + ((int64_t)1 << gshift) < p.K) ? k0 + ((int64_t)1 << gshift) : p.K;
-    for (int e = tid; e < NN; e += kThreads) {
+    for (int e = tid; e < N * SP; e += kThreads) {
         cg[e] = 0.0;
         cw[e] = 0.0;
     }
@@ -974,40 +978,33 @@ k_bwd_group(KParams p, const float* __restrict__ gloc, const float* __restrict__
     for (int64_t k = k1 - 1; k >= k0; --k) {
         const int64_t chain = seq * p.K + k;
         for (int e = tid; e < NN; e += kThreads) {
-            sg[chain * NN + e] = cg[e];
-            sw[chain * NN + e] = cw[e];
-            sq[e] = (double)Wq[chain * NN + e];
+            const int i = e / N, j = e % N;
+            sg[chain * NN + e] = cg[i * SP + j];
+            sw[chain * NN + e] = cw[i * SP + j];
+            const double qv = (double)Wq[chain * NN + e];
+            sq[i * SP + j] = qv;
+            sqt[j * SP + i] = qv;
         }
         __syncthreads();
         double ag[PER], aw[PER];
-#pragma unroll
-        for (int r = 0; r < PER; ++r) {
-            const int e = tid + r * kThreads;
-            double a = 0.0, w = 0.0;
-            if (e < NN) {
-                const int i = e / N, j = e % N;
-                for (int q = 0; q < N; ++q) {
-                    a = fma(cg[i * N + q], sq[j * N + q], a);     // cg Q^T
-                    w = fma(sq[i * N + q], cw[q * N + j], w);     // Q cw
-                }
-            }
-            ag[r] = a;
-            aw[r] = w;
-        }
+        CM::mul(cg, sqt, ag);               // cg Q^T
+        CM::mul(sq, cw, aw);                // Q cw
         __syncthreads();
 #pragma unroll
         for (int r = 0; r < PER; ++r) {
-            const int e = tid + r * kThreads;
-            if (e < NN) {
-                cg[e] = (double)gloc[chain * NN + e] + (cg[e] + ag[r]);   // g_k + cg (I + Q)^T
-                cw[e] = sq[e] + (cw[e] + aw[r]);                         // (I + Q)(I + cw) - I
-            }
+            if (!CM::valid(r)) continue;
+            int row, col;
+            CM::pos(r, row, col);
+            const int e = row * SP + col;
+            cg[e] = (double)gloc[chain * NN + row * N + col] + (cg[e] + ag[r]);   // g_k + cg (I + Q)^T
+            cw[e] = sq[e] + (cw[e] + aw[r]);                                       // (I + Q)(I + cw) - I
         }
         __syncthreads();
     }
     for (int e = tid; e < NN; e += kThreads) {
-        gg[blockIdx.x * (int64_t)NN + e] = cg[e];
-        gw[blockIdx.x * (int64_t)NN + e] = cw[e];
+        const int i = e / N, j = e % N;
+        gg[blockIdx.x * (int64_t)NN + e] = cg[i * SP + j];
+        gw[blockIdx.x * (int64_t)NN + e] = cw[i * SP + j];
     }
 }
 
@@ -1016,37 +1013,32 @@ __global__ void __launch_bounds__(kThreads)
 k_bwd_top(int64_t NG, const double* __restrict__ gg, const double* __restrict__ gw, double* __restrict__ ginr)
 {
     constexpr int NN = N * N;
-    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    using CM = CarryMul<N>;
+    constexpr int SP = CM::SP, PER = CM::PER;
     extern __shared__ double dsm[];
     double* cur = dsm;
-    double* w = cur + NN;
+    double* wt = cur + N * SP;              // (W_G - I)^T of the group at hand
     const int tid = threadIdx.x;
     const int64_t base = (int64_t)blockIdx.x * NG;
-    for (int e = tid; e < NN; e += kThreads) cur[e] = 0.0;
+    for (int e = tid; e < N * SP; e += kThreads) cur[e] = 0.0;
     __syncthreads();
     for (int64_t grp = NG - 1; grp >= 0; --grp) {
         const int64_t gi = (base + grp) * NN;
         for (int e = tid; e < NN; e += kThreads) {
-            ginr[gi + e] = cur[e];
-            w[e] = gw[gi + e];
+            const int i = e / N, j = e % N;
+            ginr[gi + e] = cur[i * SP + j];
+            wt[j * SP + i] = gw[gi + e];
         }
         __syncthreads();
         double acc[PER];
-#pragma unroll
-        for (int r = 0; r < PER; ++r) {
-            const int e = tid + r * kThreads;
-            double a = 0.0;
-            if (e < NN) {
-                const int i = e / N, j = e % N;
-                for (int q = 0; q < N; ++q) a = fma(cur[i * N + q], w[j * N + q], a);   // cur W_G^T (split)
-            }
-            acc[r] = a;
-        }
+        CM::mul(cur, wt, acc);              // cur W_G^T (split)
         __syncthreads();
 #pragma unroll
         for (int r = 0; r < PER; ++r) {
-            const int e = tid + r * kThreads;
-            if (e < NN) cur[e] = gg[gi + e] + (cur[e] + acc[r]);
+            if (!CM::valid(r)) continue;
+            int row, col;
+            CM::pos(r, row, col);
+            cur[row * SP + col] = gg[gi + row * N + col] + (cur[row * SP + col] + acc[r]);
         }
         __syncthreads();
     }
@@ -1058,28 +1050,30 @@ k_bwd_fix(KParams p, int gshift, int64_t NG, const double* __restrict__ sg, cons
           const double* __restrict__ ginr, float* __restrict__ Gin)
 {
     constexpr int NN = N * N;
-    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    using CM = CarryMul<N>;
+    constexpr int SP = CM::SP, PER = CM::PER;
     extern __shared__ double dsm[];
     double* gr = dsm;
-    double* w = gr + NN;
+    double* wt = gr + N * SP;
     const int tid = threadIdx.x;
     const int64_t chain = blockIdx.x;
     const int64_t seq = chain / p.K, k = chain - seq * p.K;
     const int64_t gi = (seq * NG + (k >> gshift)) * NN;
     for (int e = tid; e < NN; e += kThreads) {
-        gr[e] = ginr[gi + e];
-        w[e] = sw[chain * NN + e];
+        const int i = e / N, j = e % N;
+        gr[i * SP + j] = ginr[gi + e];
+        wt[j * SP + i] = sw[chain * NN + e];
     }
     __syncthreads();
+    double acc[PER];
+    CM::mul(gr, wt, acc);                   // Ginr W_suf^T (split)
 #pragma unroll
     for (int r = 0; r < PER; ++r) {
-        const int e = tid + r * kThreads;
-        if (e < NN) {
-            const int i = e / N, j = e % N;
-            double a = 0.0;
-            for (int q = 0; q < N; ++q) a = fma(gr[i * N + q], w[j * N + q], a);       // Ginr W_suf^T (split)
-            Gin[chain * NN + e] = (float)(sg[chain * NN + e] + (gr[e] + a));
-        }
+        if (!CM::valid(r)) continue;
+        int row, col;
+        CM::pos(r, row, col);
+        const int64_t e = chain * NN + row * N + col;
+        Gin[e] = (float)(sg[e] + (gr[row * SP + col] + acc[r]));
     }
 }
 
@@ -1090,38 +1084,33 @@ __global__ void __launch_bounds__(kThreads)
 k_bwd_carry(KParams p, const float* __restrict__ gloc, const float* __restrict__ Wq, float* __restrict__ Gin)
 {
     constexpr int NN = N * N;
-    constexpr int PER = (NN + kThreads - 1) / kThreads;
+    using CM = CarryMul<N>;
+    constexpr int SP = CM::SP, PER = CM::PER;
     extern __shared__ double dsm[];
     double* sGin = dsm;
-    double* sW = sGin + NN;
+    double* sWt = sGin + N * SP;            // (W_k - I)^T
     const int tid = threadIdx.x;
     const int64_t seq = blockIdx.x;
-    for (int e = tid; e < NN; e += kThreads) sGin[e] = 0.0;
+    for (int e = tid; e < N * SP; e += kThreads) sGin[e] = 0.0;
     __syncthreads();
     for (int64_t k = p.K - 1; k >= 0; --k) {
         const int64_t chain = seq * p.K + k;
         for (int e = tid; e < NN; e += kThreads) {
-            Gin[chain * NN + e] = (float)sGin[e];
-            sW[e] = (double)Wq[chain * NN + e];
+            const int i = e / N, j = e % N;
+            Gin[chain * NN + e] = (float)sGin[i * SP + j];
+            sWt[j * SP + i] = (double)Wq[chain * NN + e];
         }
         __syncthreads();
         if (k == 0) break;
         double acc[PER];
-#pragma unroll
-        for (int r = 0; r < PER; ++r) {
-            const int e = tid + r * kThreads;
-            double a = 0.0;
-            if (e < NN) {
-                const int i = e / N, j = e % N;
-                for (int q = 0; q < N; ++q) a = fma(sGin[i * N + q], sW[j * N + q], a);   // Gin Wq^T
-            }
-            acc[r] = a;
-        }
+        CM::mul(sGin, sWt, acc);            // Gin Wq^T
         __syncthreads();
 #pragma unroll
         for (int r = 0; r < PER; ++r) {
-            const int e = tid + r * kThreads;
-            if (e < NN) sGin[e] = (double)gloc[chain * NN + e] + (sGin[e] + acc[r]);
+            if (!CM::valid(r)) continue;
+            int row, col;
+            CM::pos(r, row, col);
+            sGin[row * SP + col] = (double)gloc[chain * NN + row * N + col] + (sGin[row * SP + col] + acc[r]);
         }
         __syncthreads();
     }
@@ -1136,11 +1125,11 @@ template <int N>
 cudaError_t bwd_carry_scan(const KParams& p, const float* gloc, const float* Wq, float* Gin, char* ws,
                            const BwdWorkspace& W, cudaStream_t s)
 {
-    constexpr int NN = N * N;
     const int64_t BH = p.B * p.H, chains = BH * p.K;
     if (chains == 0) return cudaSuccess;
+    constexpr int SP = CarryMul<N>::SP;
     if (p.K * (int64_t)N * N * N <= ((int64_t)1 << 20)) {
-        const size_t sm_carry = sizeof(double) * 2 * NN;
+        const size_t sm_carry = sizeof(double) * 2 * N * SP;
         cudaError_t e = set_smem(k_bwd_carry<N>, sm_carry);
         if (e != cudaSuccess) return e;
         k_bwd_carry<N><<<(unsigned)BH, kThreads, sm_carry, s>>>(p, gloc, Wq, Gin);
@@ -1151,7 +1140,7 @@ cudaError_t bwd_carry_scan(const KParams& p, const float* gloc, const float* Wq,
     double* gg = reinterpret_cast<double*>(ws + W.gg);
     double* gw = reinterpret_cast<double*>(ws + W.gw);
     double* ginr = reinterpret_cast<double*>(ws + W.ginr);
-    const size_t sm3 = sizeof(double) * 3 * NN, sm2 = sizeof(double) * 2 * NN;
+    const size_t sm3 = sizeof(double) * 4 * N * SP, sm2 = sizeof(double) * 2 * N * SP;
     cudaError_t e;
     if ((e = set_smem(k_bwd_group<N>, sm3)) != cudaSuccess) return e;
     if ((e = set_smem(k_bwd_top<N>, sm2)) != cudaSuccess) return e;
@@ -1490,6 +1479,20 @@ cudaError_t backward_n(const KParams& p, const void* src, const float* S0, const
         profile_mark(1, 1, s);
         profile_mark(2, 0, s);
         if ((e = n32::launch_bwd_apply(p, src, S0, S_fwd, dS, Gin, dx, dS0, s)) != cudaSuccess) return e;
+        profile_mark(2, 1, s);
+        return cudaGetLastError();
+    }
+    if (N == 64 && n64::supports_backward(p)) {
+        // n = 64 in tf32 on the tensor cores; the chunk-gradient scan stays generic
+        const float* x = reinterpret_cast<const float*>(src);
+        profile_mark(0, 0, s);
+        if ((e = n64::launch_bwd_local(p, x, dS, gloc, Wq, status, s)) != cudaSuccess) return e;
+        profile_mark(0, 1, s);
+        profile_mark(1, 0, s);
+        if ((e = bwd_carry_scan<N>(p, gloc, Wq, Gin, ws, W, s)) != cudaSuccess) return e;
+        profile_mark(1, 1, s);
+        profile_mark(2, 0, s);
+        if ((e = n64::launch_bwd_apply(p, x, S0, S_fwd, dS, Gin, dx, dS0, status, s)) != cudaSuccess) return e;
         profile_mark(2, 1, s);
         return cudaGetLastError();
     }

@@ -260,3 +260,73 @@ def test_backward_grouped_chunk_gradient_scan(n, mode, dtype, L, chunk):
     e_dx = _rel(dx.reshape(w.B, w.L, w.H, n * n), dx_o.reshape(w.B, w.L, w.H, n * n), axis=-1)
     e_s0 = _rel(dS0.reshape(w.B, w.H, n * n), dS0_o.reshape(w.B, w.H, n * n), axis=-1)
     assert e_dx.max() <= TOL_BWD and e_s0.max() <= TOL_BWD, (e_dx.max(), np.median(e_dx), e_s0.max())
+
+
+# n = 64 on the tensor cores when tf32 is asked for (k64b_local / k64b_apply):
+# the tf32 gate of the forward.
+TOL_BWD_TF32 = 1e-2
+
+N64_TC_CASES = [  # mode, add_identity, alpha, with_s0, L, chunk
+    (gen.MODE_DETNORM, 1, 0.03 / 8, True, 53, 16),    # trace series and its three-term inverse
+    (gen.MODE_DETNORM, 1, 0.03 / 8, False, 40, 1),    # one-token chunks
+    (gen.MODE_DETNORM, 1, 0.3 / 8, False, 37, 8),     # far from the identity: pivoted elimination
+    (gen.MODE_DETNORM, 0, 1.0 / 8, True, 21, 8),      # no identity: pivoted elimination
+    (gen.MODE_RESHAPE, 1, 0.3 / 8, True, 53, 16),
+    (gen.MODE_RESHAPE, 0, 1.0 / 8, False, 13, 4),
+]
+
+
+@pytest.mark.parametrize("mode,add_identity,alpha,with_s0,L,chunk", N64_TC_CASES)
+def test_backward_n64_tensor_cores(mode, add_identity, alpha, with_s0, L, chunk):
+    """mru_scan_backward at n = 64 with math = tf32 (the tensor-core local and
+    apply passes) against the oracle's fp64 backward: several chunks with a
+    ragged tail, with and without S0, near and far from the identity."""
+    t = torch()
+    n = 64
+    w = gen.Workload("b64tc", B=2, H=2, L=L, n=n, x_dtype="f32", mode=mode, alpha=float(alpha),
+                     add_identity=add_identity, math="tf32", seed=640 + L)
+    x = gen.make_x(w)
+    S0 = gen.make_S0(w, seed=641) if with_s0 else None
+    dS = np.random.default_rng(642 + L).standard_normal((w.B, w.L, w.H, n, n)).astype(np.float32)
+    p = mru.problem_from_workload(w, chunk=chunk)
+    xd = to_device_x(x)
+    S0d = None if S0 is None else t.from_numpy(np.ascontiguousarray(S0, np.float32)).cuda()
+    S = mru.scan_fused_t(p, xd, S0=S0d)
+    dx, dS0, ws = mru.scan_backward_t(p, xd, S, t.from_numpy(dS).cuda(), S0=S0d)
+    assert mru.last_device_status(ws.data_ptr(), t.cuda.current_stream().cuda_stream) == mru.OK
+    dx_o, dS0_o = oracle.backward(oracle_problem(w), x, dS.astype(np.float64),
+                                  S0=None if S0 is None else S0.astype(np.float64))
+    e = _rel(dx.cpu().numpy().astype(np.float64).reshape(w.B, w.L, w.H, n * n), dx_o.reshape(w.B, w.L, w.H, n * n),
+             axis=-1)
+    print("n64 tensor-core backward: max", e.max(), "median", np.median(e))
+    assert e.max() <= TOL_BWD_TF32, (e.max(), np.median(e))
+    if with_s0:
+        e0 = _rel(dS0.cpu().numpy().astype(np.float64).reshape(w.B, w.H, n * n), dS0_o.reshape(w.B, w.H, n * n),
+                  axis=-1)
+        assert e0.max() <= TOL_BWD_TF32, e0.max()
+
+
+def test_backward_readout_n64_tensor_cores_workload_shape():
+    """The readout backward of the n = 64 workload's construction (alpha =
+    0.03 / 8, corrected with the identity, one query vector, snapshots every
+    256 steps, tf32) on a shorter sequence (automatic chunking):
+    k64b_local / k64b_apply behind mru_scan_backward_readout, against the
+    oracle's readout backward."""
+    t = torch()
+    B, H, L, n = 1, 2, 1024, 64
+    w = gen.Workload("bro64", B=B, H=H, L=L, n=n, x_dtype="f32", mode=gen.MODE_DETNORM, alpha=0.03 / 8,
+                     math="tf32", seed=1005)
+    x = gen.make_x(w)
+    r = np.random.default_rng(77)
+    u = r.standard_normal(n).astype(np.float32)
+    d_o = r.standard_normal((B, L, H, n, 1)).astype(np.float32)
+    d_snap = r.standard_normal((B, L // 256, H, n, n)).astype(np.float32)
+    p = mru.problem_from_workload(w)
+    dx, _, ws = mru.scan_backward_readout_t(p, to_device_x(x), t.from_numpy(u).cuda(), t.from_numpy(d_o).cuda(),
+                                            snapshot_every=256, d_snaps=t.from_numpy(d_snap).cuda())
+    assert mru.last_device_status(ws.data_ptr(), t.cuda.current_stream().cuda_stream) == mru.OK
+    dx_o, _ = oracle.backward_readout(oracle_problem(w), x, u.astype(np.float64), d_o[..., 0],
+                                      snapshot_every=256, d_snap=d_snap)
+    e = _rel(dx.cpu().numpy().astype(np.float64).reshape(B, L, H, n * n), dx_o.reshape(B, L, H, n * n), axis=-1)
+    print("n64 tensor-core readout backward: max", e.max(), "median", np.median(e))
+    assert e.max() <= TOL_BWD_TF32, (e.max(), np.median(e))
