@@ -977,9 +977,15 @@ def main(argv=None):
     ap.add_argument("--backward", action="store_true", help="time mru_scan_backward instead (not the default)")
     ap.add_argument("--decode", action="store_true",
                     help="time single-token decode steps from S0 instead (not the default)")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="run the workload with this sequence length instead of its own (small cases for "
+                         "profiler captures; the workload's name gets the suffix _l<L>)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)      # at least 3 untimed warm-up steps, always
     w = gen.WORKLOADS[args.workload]
+    if args.seq_len > 0:
+        import dataclasses
+        w = dataclasses.replace(w, L=args.seq_len, name=f"{w.name}_l{args.seq_len}")
     if args.impl == "reference":
         return run_reference(args, w)
     if args.backward:
