@@ -619,14 +619,7 @@ k64b_apply(KParams p, const float* __restrict__ x, const float* __restrict__ S0,
                     dsr[nt][h8] = tau > t0 ? *reinterpret_cast<const float2*>(d0 + (r0 + g + 8 * h8) * N + 8 * nt + 2 * q)
                                            : make_float2(0.0f, 0.0f);
         }
-        // ---- the determinant scale and the inverse's series terms ----
-        float Y[8][4];
-        Series sr;
-        sr.ok = !detnorm;
-        sr.inv_ok = !detnorm;
-        sr.cm1 = 0.0f;
-        if (series) sr = det_series<true>(sm.c, xs, p.alpha, warp, lane, Y);
-        // ---- dX = S_{tau-1}^T G ----
+        // ---- dX = S_{tau-1}^T G, and this warp's part of <dX, Xr> ----
         float D[8][4];
         if (out_tok) {
             zero(D);
@@ -662,8 +655,17 @@ k64b_apply(KParams p, const float* __restrict__ x, const float* __restrict__ S0,
                 part = warp_sum(part);
                 if (lane == 0) sm.c.red2[warp] = part;
             }
-            __syncthreads();                         // every warp has read S and G
         }
+        // ---- the determinant scale and the inverse's series terms; its barrier
+        // (or the one in its place) also publishes the parts of <dX, Xr> and
+        // ends every warp's reads of S and G ----
+        float Y[8][4];
+        Series sr;
+        sr.ok = !detnorm;
+        sr.inv_ok = !detnorm;
+        sr.cm1 = 0.0f;
+        if (series) sr = det_series<true>(sm.c, xs, p.alpha, warp, lane, Y);
+        else if (out_tok) __syncthreads();
         // ---- where the series does not serve: the pivoted elimination ----
         const bool elim = detnorm && (!sr.ok || (out_tok && !sr.inv_ok));     // uniform over the CTA
         float cm1 = sr.cm1;
