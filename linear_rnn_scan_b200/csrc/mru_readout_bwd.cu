@@ -6,37 +6,72 @@
 namespace mru {
 namespace {
 
-// dS[b, t, h] = do_t U_h^T (+ dP_k at 1-based t = k * every): one CTA per
-// token-head row at a time (grid-stride over the B L H rows), do_t ([n, q])
-// and the head's U_h ([n, q], u + h * u_hs) staged in shared memory, the
-// row's n * n outputs written by consecutive threads.
+// dS[b, t, h] = do_t U_h^T (+ dP_k at 1-based t = k * every): each thread
+// writes float4 runs of one token-head row; a block takes one row at a time
+// for n >= 32 and 256 / (n^2 / 4) rows at once below.  do_t ([n, q]) comes
+// through the read-only cache (at most two rows i per warp: broadcasts).
+// StageU: the heads' U_h ([n, q] = u + h * u_hs; one U when u_hs = 0) are
+// staged transposed in shared memory once per block, [head][c][j], so each
+// column c is a float4 read; otherwise U is read through the read-only cache
+// (the heads' U too large to stage).
+template <bool StageU>
 __global__ void __launch_bounds__(256)
 k_readout_grad(int64_t B, int64_t L, int64_t H, int n, int q, int64_t u_hs, const float* __restrict__ u,
                const float* __restrict__ d_o, int64_t every, const float* __restrict__ d_snap, float* __restrict__ dS)
 {
-    extern __shared__ float rsm[];
-    float* sO = rsm;                                         // do_t, [n][q]
-    float* sU = rsm + n * q;                                 // U_h, [n][q]
-    const int nn = n * n, nq = n * q, ln = __ffs(n) - 1;  // n is a power of two
-    const int64_t rows = B * L * H, L_s = every > 0 ? L / every : 0;
-    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {   // row = (b L + t) H + h
-        const int64_t h = row % H, bt = row / H, t = bt % L, b = bt / L;
-        __syncthreads();                                     // the previous row's reads are done
-        for (int e = threadIdx.x; e < nq; e += blockDim.x) {
-            sO[e] = d_o[row * nq + e];
-            sU[e] = u[h * u_hs + e];
+    extern __shared__ __align__(16) float sUt[];
+    const int nn = n * n, nq = n * q, ln = __ffs(n) - 1;   // n is a power of two, at least 4
+    if constexpr (StageU) {
+        const int heads = u_hs == 0 ? 1 : (int)H;
+        for (int e = threadIdx.x; e < heads * nq; e += blockDim.x) {
+            const int hh = e / nq, r = e - hh * nq, c = r >> ln, j = r & (n - 1);
+            sUt[e] = u[hh * u_hs + j * q + c];
         }
         __syncthreads();
-        const float* snap = (d_snap && every > 0 && (t + 1) % every == 0)
-                                ? d_snap + ((b * L_s + (t + 1) / every - 1) * H + h) * nn
-                                : nullptr;
-        float* out = dS + row * nn;
-        for (int e = threadIdx.x; e < nn; e += blockDim.x) {
-            const int i = e >> ln, j = e & (n - 1);
-            float a = 0.0f;
-            for (int c = 0; c < q; ++c) a = fmaf(sO[i * q + c], sU[j * q + c], a);
-            if (snap) a += snap[e];
-            out[e] = a;
+    }
+    const int per_row = nn >> 2;                             // float4 runs of a row
+    const int rpi = per_row >= 256 ? 1 : 256 / per_row;      // rows a block takes at a time
+    const int lr = per_row >= 256 ? 0 : (int)threadIdx.x / per_row;
+    const int e4_0 = per_row >= 256 ? (int)threadIdx.x : (int)threadIdx.x % per_row;
+    const int e4_step = per_row >= 256 ? 256 : per_row;
+    const int64_t rows = B * L * H, L_s = every > 0 ? L / every : 0;
+    for (int64_t r0 = (int64_t)blockIdx.x * rpi; r0 < rows; r0 += (int64_t)gridDim.x * rpi) {
+        const int64_t row = r0 + lr;                          // row = (b L + t) H + h
+        if (row >= rows) continue;
+        const int64_t h = row % H, bt = row / H, t = bt % L, b = bt / L;
+        const float* dO = d_o + row * nq;
+        const float* U = u + h * u_hs;
+        const float* Ut = sUt + (u_hs == 0 ? 0 : (int)h * nq);
+        const float4* snap = (d_snap && every > 0 && (t + 1) % every == 0)
+                                 ? reinterpret_cast<const float4*>(d_snap + ((b * L_s + (t + 1) / every - 1) * H + h) * nn)
+                                 : nullptr;
+        float4* out = reinterpret_cast<float4*>(dS + row * nn);
+        for (int e4 = e4_0; e4 < per_row; e4 += e4_step) {
+            const int e = e4 << 2, i = e >> ln, j = e & (n - 1);
+            float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+            for (int c = 0; c < q; ++c) {
+                const float d = __ldg(dO + i * q + c);
+                if constexpr (StageU) {
+                    const float4 uv = *reinterpret_cast<const float4*>(Ut + c * n + j);
+                    a0 = fmaf(d, uv.x, a0);
+                    a1 = fmaf(d, uv.y, a1);
+                    a2 = fmaf(d, uv.z, a2);
+                    a3 = fmaf(d, uv.w, a3);
+                } else {
+                    a0 = fmaf(d, __ldg(U + j * q + c), a0);
+                    a1 = fmaf(d, __ldg(U + (j + 1) * q + c), a1);
+                    a2 = fmaf(d, __ldg(U + (j + 2) * q + c), a2);
+                    a3 = fmaf(d, __ldg(U + (j + 3) * q + c), a3);
+                }
+            }
+            if (snap) {
+                const float4 sv = snap[e4];
+                a0 += sv.x;
+                a1 += sv.y;
+                a2 += sv.z;
+                a3 += sv.w;
+            }
+            out[e4] = make_float4(a0, a1, a2, a3);
         }
     }
 }
@@ -53,9 +88,16 @@ cudaError_t launch_readout_grad(const KParams& p, const float* u, int q, int64_t
     if (e != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const int64_t rows = p.B * p.L * p.H;
-    const int64_t blocks = rows < (int64_t)sms * 8 ? rows : (int64_t)sms * 8;
-    const size_t sm = sizeof(float) * 2 * (size_t)p.n * q;
-    k_readout_grad<<<(unsigned)blocks, 256, sm, s>>>(p.B, p.L, p.H, p.n, q, u_hs, u, d_o, every, d_snap, dS);
+    const int per_row = p.n * p.n / 4;
+    const int64_t rpi = per_row >= 256 ? 1 : 256 / per_row;
+    const int64_t need = (rows + rpi - 1) / rpi;
+    const int64_t blocks = need < (int64_t)sms * 8 ? need : (int64_t)sms * 8;
+    const size_t staged = sizeof(float) * (size_t)(u_hs == 0 ? 1 : p.H) * (size_t)p.n * q;
+    if (staged <= 48 * 1024)
+        k_readout_grad<true><<<(unsigned)blocks, 256, staged, s>>>(p.B, p.L, p.H, p.n, q, u_hs, u, d_o, every, d_snap,
+                                                                   dS);
+    else
+        k_readout_grad<false><<<(unsigned)blocks, 256, 0, s>>>(p.B, p.L, p.H, p.n, q, u_hs, u, d_o, every, d_snap, dS);
     return cudaGetLastError();
 }
 

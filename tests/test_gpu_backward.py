@@ -330,3 +330,24 @@ def test_backward_readout_n64_tensor_cores_workload_shape():
     e = _rel(dx.cpu().numpy().astype(np.float64).reshape(B, L, H, n * n), dx_o.reshape(B, L, H, n * n), axis=-1)
     print("n64 tensor-core readout backward: max", e.max(), "median", np.median(e))
     assert e.max() <= TOL_BWD_TF32, (e.max(), np.median(e))
+
+
+def test_backward_readout_many_query_columns():
+    """The readout gradient when the heads' query columns are too many to
+    stage in shared memory (H n q floats above 48 KB: read through the cache
+    instead): 16 heads of n = 32 with 32 columns each, against the oracle."""
+    t = torch()
+    B, H, L, n, q = 1, 16, 9, 32, 32
+    w = gen.Workload("brq", B=B, H=H, L=L, n=n, x_dtype="f32", mode=gen.MODE_DETNORM, alpha=float(0.3 / np.sqrt(n)),
+                     seed=91)
+    x = gen.make_x(w)
+    r = np.random.default_rng(92)
+    u = r.standard_normal((H, n, q)).astype(np.float32)
+    d_o = r.standard_normal((B, L, H, n, q)).astype(np.float32)
+    p = mru.problem_from_workload(w, chunk=4)
+    dx, _, ws = mru.scan_backward_readout_t(p, to_device_x(x), t.from_numpy(u).cuda(), t.from_numpy(d_o).cuda(),
+                                            q=q, u_per_head=1)
+    assert mru.last_device_status(ws.data_ptr(), t.cuda.current_stream().cuda_stream) == mru.OK
+    dx_o, _ = oracle.backward_readout(oracle_problem(w), x, u.astype(np.float64), d_o)
+    e = _rel(dx.cpu().numpy().astype(np.float64).reshape(B, L, H, n * n), dx_o.reshape(B, L, H, n * n), axis=-1)
+    assert e.max() <= TOL_BWD, (e.max(), np.median(e))
