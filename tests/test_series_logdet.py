@@ -10,7 +10,13 @@ is at most 1e-6; otherwise it factorises (LU).  These tests pin the series
 against numpy's slogdet, the bound against the true remainder, the
 acceptance at the benchmark's alpha, the rejection far from the identity,
 and the integer-operation tf32 rounding (round to nearest, ties away) the
-kernels use for the chain's tensor-core operands."""
+kernels use for the chain's tensor-core operands.
+
+The n = 64 backward (k64b_apply) forms the same series from P2 = (M^T)^2 and
+P3 = P2 M^T, and from them the chain rule's inverse
+    Xr^-T = I - E^T + (E^T)^2 - (E^T)^3 + R,  |R|_F <= |E^3|_F |E|_F / (1 - |E|_F),
+taken when that bound is at most 1e-3: the last tests pin the transposed
+traces, the inverse against numpy's, its bound, acceptance and rejection."""
 import numpy as np
 
 N = 64
@@ -108,3 +114,89 @@ def test_series_sign_and_terms_are_all_needed():
         ww = w.copy()
         ww[k] = -ww[k]
         assert abs(ww @ t - true) > 1e-6
+
+
+# ---- the n = 64 backward (k64b_apply): the same series on transposed
+# products, and the chain rule's inverse from them ----
+INV_TAU = 1e-3
+
+
+def transposed_products(M, rounded=True):
+    """P2 = (M^T)^2 and P3 = P2 M^T as the backward kernels form them (bf16
+    operands, wide accumulation)."""
+    r = bf16_round if rounded else (lambda a: a)
+    Mt = r(M.astype(np.float32).T).astype(np.float64)
+    P2 = Mt @ Mt
+    P3 = r(P2).astype(np.float64) @ Mt
+    return P2, P3
+
+
+def inverse_series(M, alpha, rounded=True):
+    """Xr^-T ~ I - E^T + alpha^2 P2 - alpha^3 P3 and the bound on the dropped
+    tail, |E^3|_F |E|_F / (1 - |E|_F)."""
+    P2, P3 = transposed_products(M, rounded)
+    Z = np.eye(N) - alpha * M.astype(np.float64).T + alpha ** 2 * P2 - alpha ** 3 * P3
+    fe = alpha * np.linalg.norm(M.astype(np.float64))
+    bound = (alpha ** 3 * np.linalg.norm(P3)) * fe / (1 - fe) if fe < 1 else np.inf
+    return Z, bound
+
+
+def test_transposed_products_give_the_same_traces_and_norms():
+    """tr M^3 = <P2, M>, tr M^4 = <P3, M>, |M^2|_F = |P2|_F and |M^3|_F =
+    |P3|_F for P2 = (M^T)^2, P3 = (M^T)^3: the backward's series equals the
+    forward's."""
+    rng = np.random.default_rng(21)
+    M = rng.standard_normal((N, N)).astype(np.float32).astype(np.float64)     # exact in fp32, as the slices are
+    P2, P3 = transposed_products(M, rounded=False)
+    M2, M3 = M @ M, M @ M @ M
+    np.testing.assert_allclose(np.sum(P2 * M), np.trace(M3), rtol=1e-10)
+    np.testing.assert_allclose(np.sum(P3 * M), np.trace(M3 @ M), rtol=1e-10)
+    np.testing.assert_allclose(np.linalg.norm(P2), np.linalg.norm(M2), rtol=1e-12)
+    np.testing.assert_allclose(np.linalg.norm(P3), np.linalg.norm(M3), rtol=1e-12)
+    # and not the untransposed pairing: <M2, M> is tr(M^2 M^T), a different number
+    assert abs(np.sum(M2 * M) - np.trace(M3)) > 1e-3 * abs(np.trace(M3)) + 1.0
+
+
+def test_inverse_series_within_its_bound_exact_products():
+    rng = np.random.default_rng(22)
+    for alpha in (0.002, 0.00375, 0.006):
+        for _ in range(20):
+            M = rng.standard_normal((N, N)).astype(np.float32)
+            Z, bound = inverse_series(M, alpha, rounded=False)
+            true = np.linalg.inv(np.eye(N) + alpha * M.astype(np.float64)).T
+            assert np.linalg.norm(Z - true) <= bound
+
+
+def test_inverse_series_accepted_at_benchmark_alpha_and_accurate_with_bf16_products():
+    rng = np.random.default_rng(23)
+    alpha = 0.03 / np.sqrt(N)
+    for _ in range(30):
+        M = rng.standard_normal((N, N)).astype(np.float32)
+        Z, bound = inverse_series(M, alpha)
+        assert bound <= INV_TAU
+        true = np.linalg.inv(np.eye(N) + alpha * M.astype(np.float64)).T
+        assert np.linalg.norm(Z - true) / np.linalg.norm(true) <= 2e-5
+
+
+def test_inverse_series_rejected_far_from_identity():
+    rng = np.random.default_rng(24)
+    for alpha in (0.3 / np.sqrt(N), 0.05, 0.2):
+        M = rng.standard_normal((N, N)).astype(np.float32)
+        _, bound = inverse_series(M, alpha)
+        assert not bound <= INV_TAU
+
+
+def test_inverse_series_each_term_needed():
+    """Dropping or flipping any of the three terms beyond I moves the inverse
+    by more than the bound at the benchmark's alpha."""
+    rng = np.random.default_rng(25)
+    alpha = 0.03 / np.sqrt(N)
+    M = rng.standard_normal((N, N)).astype(np.float32)
+    P2, P3 = transposed_products(M, rounded=False)
+    Mt = M.astype(np.float64).T
+    true = np.linalg.inv(np.eye(N) + alpha * M.astype(np.float64)).T
+    terms = [-alpha * Mt, alpha ** 2 * P2, -alpha ** 3 * P3]
+    _, bound = inverse_series(M, alpha, rounded=False)
+    for k in range(3):
+        Z = np.eye(N) + sum(-t if i == k else t for i, t in enumerate(terms))
+        assert np.linalg.norm(Z - true) > bound
