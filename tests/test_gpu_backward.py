@@ -273,6 +273,9 @@ N64_TC_CASES = [  # mode, add_identity, alpha, with_s0, L, chunk
     (gen.MODE_DETNORM, 0, 1.0 / 8, True, 21, 8),      # no identity: pivoted elimination
     (gen.MODE_RESHAPE, 1, 0.3 / 8, True, 53, 16),
     (gen.MODE_RESHAPE, 0, 1.0 / 8, False, 13, 4),
+    (gen.MODE_DETNORM, 1, 0.03 / 8, True, 1, 64),     # a single token
+    (gen.MODE_DETNORM, 1, 0.03 / 8, True, 5, 0),      # a single chunk (the default chunk for this size)
+    (gen.MODE_RESHAPE, 1, 0.3 / 8, False, 2, 1),      # two one-token chunks
 ]
 
 
