@@ -678,12 +678,13 @@ def run_ours(args, w):
 def bwd_kernel_names(w):
     """The three launches of mru_scan_backward for this workload: the tensor-core
     passes where the library has them (n = 16 fp32 reshape / corrected with the
-    identity, n = 32 LDU bf16, n = 64 fp32 reshape / corrected in tf32), the
+    identity / Cayley map, n = 32 LDU bf16, n = 64 fp32 reshape / corrected in
+    tf32), the
     generic kernels otherwise; the chunk-gradient
     scan between them is always the generic one ("chunk_scan": k_bwd_carry
     serially, or k_bwd_group, k_bwd_top and k_bwd_fix in groups for larger
     problems)."""
-    if w.n == 16 and w.x_dtype == "f32" and (w.mode == gen.MODE_RESHAPE or
+    if w.n == 16 and w.x_dtype == "f32" and (w.mode in (gen.MODE_RESHAPE, gen.MODE_CAYLEY) or
                                               (w.mode == gen.MODE_DETNORM and w.add_identity)):
         return ["k16b_local", "chunk_scan", "k16b_apply"]
     if w.n == 32 and w.x_dtype == "bf16" and w.mode == gen.MODE_LDU:

@@ -190,8 +190,8 @@ mru_status mru_scan_fused_host(const mru_problem* p, const void* x_host, const f
  * Every pointer 16-byte aligned; dx and dS0 alias no input.  The workspace
  * holds mru_backward_workspace_size(p) bytes.  fp32-accurate arithmetic for
  * every n and mode unless tf32 is asked for: fp32 on the generic kernels,
- * split tf32 on the tensor cores for n = 16 (fp32 embeddings, reshape or
- * corrected with the identity), three-term split bf16 for n = 32 LDU (bf16
+ * split tf32 on the tensor cores for n = 16 (fp32 embeddings, reshape,
+ * corrected with the identity, or the Cayley map), three-term split bf16 for n = 32 LDU (bf16
  * embeddings, exact in bf16).  n = 64 with p->math = MRU_MATH_TF32 (fp32
  * embeddings, reshape or determinant-corrected): tf32 products on the
  * tensor cores, the forward's tf32 arithmetic (chunks of 64 tokens by

@@ -2145,9 +2145,30 @@ __device__ __forceinline__ void add_ds(const float* dst, const float (&a)[2][4],
         }
 }
 
+// The per-token scalars of a backward stage (F = c alpha M + dv I); for the
+// Cayley map F itself, formed over the stage's slices (stage_cayley in rounds
+// of 4 tokens: the slots beyond the stage's 2 are never live and only read
+// slot 0), with the scalars (1, 0).
+template <bool Cay>
+__device__ __forceinline__ void stage_scalars_or_cayley(const KParams& p, float2* cd, float* xs, unsigned live,
+                                                        int lane, uint32_t* status)
+{
+    if constexpr (Cay) {
+        stage_cayley<4>(p.alpha, xs, live, lane);
+        if (lane < BST) cd[lane] = make_float2(1.0f, 0.0f);
+        __syncwarp();
+    } else {
+        stage_scalars<BST>(p, cd, xs, live, lane, status);
+    }
+}
+
 // Local pass: per chunk the gradient at t0 with nothing entering from the
-// right (gloc) and W - I (Wq; zero for the last chunk of a sequence).
-__global__ void __launch_bounds__(BWARPS * 32, 2)
+// right (gloc) and W - I (Wq; zero for the last chunk of a sequence).  Cay:
+// the Cayley map, its own instantiation (the elimination's registers would
+// otherwise cost the other modes a CTA per SM), capped for three CTAs per SM
+// (153 registers, no spills).
+template <bool Cay>
+__global__ void __launch_bounds__(BWARPS * 32, Cay ? 3 : 2)
 k16b_local(KParams p, const float* __restrict__ x, const float* __restrict__ dS, float* __restrict__ gloc,
            float* __restrict__ Wq, uint32_t* status)
 {
@@ -2185,7 +2206,7 @@ k16b_local(KParams p, const float* __restrict__ x, const float* __restrict__ dS,
             cp_async_wait<BNS - 1>();
             __syncwarp();
             const int nt = (ts - lo + 1 < BST) ? (int)(ts - lo + 1) : BST;
-            stage_scalars<BST>(p, sm.cd, sm.x[cs], (1u << nt) - 1u, lane, status);
+            stage_scalars_or_cayley<Cay>(p, sm.cd, sm.x[cs], (1u << nt) - 1u, lane, status);
 #pragma unroll
             for (int j = 0; j < BST; ++j) {
                 if (j < nt) {
@@ -2231,6 +2252,7 @@ k16b_local(KParams p, const float* __restrict__ x, const float* __restrict__ dS,
 
 // Apply pass: per chunk G from the gradient entering from the right (Gin)
 // down to t0, every dL/dx_t, and dL/dS0 from the first chunk.
+template <bool Cay>
 __global__ void __launch_bounds__(BWARPS * 32, 3)
 k16b_apply(KParams p, const float* __restrict__ x, const float* __restrict__ S0, const float* __restrict__ S_fwd,
            const float* __restrict__ dS, const float* __restrict__ Gin, float* __restrict__ dx,
@@ -2245,6 +2267,7 @@ k16b_apply(KParams p, const float* __restrict__ x, const float* __restrict__ S0,
     const int g = lane >> 2, q = lane & 3;
     const float m0 = (g == 2 * q) ? 1.0f : 0.0f, m1 = (g == 2 * q + 1) ? 1.0f : 0.0f;
     const bool detnorm = p.mode == MRU_MODE_DETNORM;
+    constexpr bool cayley = Cay;
     BFeed<true> feed;
     feed.chain = first;
     feed.stride = stride;
@@ -2269,7 +2292,7 @@ k16b_apply(KParams p, const float* __restrict__ x, const float* __restrict__ S0,
             cp_async_wait<BNS - 1>();
             __syncwarp();
             const int nt = (ts - lo + 1 < BST) ? (int)(ts - lo + 1) : BST;
-            stage_scalars<BST>(p, sm.cd, sm.x[cs], (1u << nt) - 1u, lane, status);
+            stage_scalars_or_cayley<Cay>(p, sm.cd, sm.x[cs], (1u << nt) - 1u, lane, status);
 #pragma unroll
             for (int j = 0; j < BST; ++j) {
                 if (j < nt) {
@@ -2309,7 +2332,37 @@ k16b_apply(KParams p, const float* __restrict__ x, const float* __restrict__ S0,
                     __syncwarp();
                     // the construction's chain rule
                     float out[2][4];
-                    if (!detnorm) {
+                    if constexpr (cayley) {
+                        // X = 2 W^-1 - I, W = I - A, A = alpha (M - M^T) / 2: with
+                        // W^-1 = I + F / 2, dA = 2 W^-T dX W^-T = 2 T + T F^T for
+                        // T = dX + F^T dX / 2 (xs holds F), dM = alpha (dA - dA^T) / 2
+                        stage_acc(sm.stg, dX, g, q);
+                        __syncwarp();
+                        float T[2][4], a2[2][4];
+                        st_times_g(xs, sm.stg, g, q, T);      // F^T dX
+#pragma unroll
+                        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) T[n2][i] = fmaf(0.5f, T[n2][i], dX[n2][i]);
+                        chain_product<true>(T, ft, a2);       // T F^T
+#pragma unroll
+                        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) a2[n2][i] = fmaf(2.0f, T[n2][i], a2[n2][i]);   // dA
+                        __syncwarp();
+                        stage_acc(sm.stg, a2, g, q);
+                        __syncwarp();
+                        const float ha = 0.5f * p.alpha;
+#pragma unroll
+                        for (int n2 = 0; n2 < 2; ++n2)
+#pragma unroll
+                            for (int h8 = 0; h8 < 2; ++h8)
+#pragma unroll
+                                for (int e = 0; e < 2; ++e)
+                                    out[n2][2 * h8 + e] =
+                                        ha * (a2[n2][2 * h8 + e] - sm.stg[swz(8 * n2 + 2 * q + e, g + 8 * h8)]);
+                        __syncwarp();
+                    } else if (!detnorm) {
 #pragma unroll
                         for (int n2 = 0; n2 < 2; ++n2)
 #pragma unroll
@@ -2373,8 +2426,11 @@ k16b_apply(KParams p, const float* __restrict__ x, const float* __restrict__ S0,
 }
 
 // CTAs of a persistent launch: resident CTAs per SM times the SM count,
-// cached per device and kernel slot; no more than the chains need.
-std::atomic<int> g_resident[64][16];
+// cached per device and kernel slot (one slot per kernel instantiation:
+// reduce 0, 1, 6, 11; apply 2, 3, 7, 8, 12, 13, 14; backward 4, 5, and 16, 17
+// for the Cayley map; single-read 9, 10, 15); no more than the chains need.
+constexpr int kSlots = 18;
+std::atomic<int> g_resident[64][kSlots];
 
 // The orthogonal construction the passes apply to each slice: 0 none, 1 the
 // Cayley map, 2 the exponential map.
@@ -2389,6 +2445,7 @@ cudaError_t persistent_grid(int slot, const void* kern, int threads, size_t smem
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    if (slot < 0 || slot >= kSlots) return cudaErrorInvalidValue;
     int res = (dev >= 0 && dev < 64) ? g_resident[dev][slot].load(std::memory_order_relaxed) : 0;
     if (res <= 0) {
         int sms = 0, per_sm = 0;
@@ -2582,7 +2639,7 @@ cudaError_t launch_fused(const KParams& p, const FusedPlan& fp, char* ws, const 
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)) != cudaSuccess)
         return e;
     unsigned grid = 0;
-    if ((e = persistent_grid(9 + tr, (const void*)kern, FWARPS * 32, sm, FWARPS, nchains, grid)) !=
+    if ((e = persistent_grid(tr == 2 ? 15 : 9 + tr, (const void*)kern, FWARPS * 32, sm, FWARPS, nchains, grid)) !=
         cudaSuccess)
         return e;
     kern<<<grid, FWARPS * 32, sm, s>>>(p, f, x, S0, S_out, status);
@@ -2592,7 +2649,8 @@ cudaError_t launch_fused(const KParams& p, const FusedPlan& fp, char* ws, const 
 bool supports_backward(const KParams& p)
 {
     return p.n == N && p.src == SRC_EMBEDDING && p.x_dtype == MRU_F32 &&
-           (p.mode == MRU_MODE_RESHAPE || (p.mode == MRU_MODE_DETNORM && p.add_identity)) &&
+           (p.mode == MRU_MODE_RESHAPE || (p.mode == MRU_MODE_DETNORM && p.add_identity) ||
+            p.mode == MRU_MODE_CAYLEY) &&
            (p.math == MRU_MATH_AUTO || p.math == MRU_MATH_TF32X3) && p.chunk > 0;
 }
 
@@ -2603,12 +2661,14 @@ cudaError_t launch_bwd_local(const KParams& p, const float* x, const float* dS, 
     if (nchains == 0) return cudaSuccess;
     if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const size_t sm = sizeof(BSmem<false>) * BWARPS;
-    cudaError_t e = cudaFuncSetAttribute(k16b_local, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    const bool cay = p.mode == MRU_MODE_CAYLEY;
+    auto kern = cay ? k16b_local<true> : k16b_local<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     unsigned grid = 0;
-    if ((e = persistent_grid(4, (const void*)k16b_local, BWARPS * 32, sm, BWARPS, nchains, grid)) != cudaSuccess)
+    if ((e = persistent_grid(cay ? 16 : 4, (const void*)kern, BWARPS * 32, sm, BWARPS, nchains, grid)) != cudaSuccess)
         return e;
-    k16b_local<<<grid, BWARPS * 32, sm, s>>>(p, x, dS, gloc, Wq, status);
+    kern<<<grid, BWARPS * 32, sm, s>>>(p, x, dS, gloc, Wq, status);
     return cudaGetLastError();
 }
 
@@ -2619,12 +2679,14 @@ cudaError_t launch_bwd_apply(const KParams& p, const float* x, const float* S0, 
     if (nchains == 0) return cudaSuccess;
     if (nchains >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     const size_t sm = sizeof(BSmem<true>) * BWARPS;
-    cudaError_t e = cudaFuncSetAttribute(k16b_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    const bool cay = p.mode == MRU_MODE_CAYLEY;
+    auto kern = cay ? k16b_apply<true> : k16b_apply<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     unsigned grid = 0;
-    if ((e = persistent_grid(5, (const void*)k16b_apply, BWARPS * 32, sm, BWARPS, nchains, grid)) != cudaSuccess)
+    if ((e = persistent_grid(cay ? 17 : 5, (const void*)kern, BWARPS * 32, sm, BWARPS, nchains, grid)) != cudaSuccess)
         return e;
-    k16b_apply<<<grid, BWARPS * 32, sm, s>>>(p, x, S0, S_fwd, dS, Gin, dx, dS0, status);
+    kern<<<grid, BWARPS * 32, sm, s>>>(p, x, S0, S_fwd, dS, Gin, dx, dS0, status);
     return cudaGetLastError();
 }
 

@@ -354,3 +354,57 @@ def test_backward_readout_many_query_columns():
     dx_o, _ = oracle.backward_readout(oracle_problem(w), x, u.astype(np.float64), d_o)
     e = _rel(dx.cpu().numpy().astype(np.float64).reshape(B, L, H, n * n), dx_o.reshape(B, L, H, n * n), axis=-1)
     assert e.max() <= TOL_BWD, (e.max(), np.median(e))
+
+
+@pytest.mark.parametrize("alpha,chunk,with_s0", [(0.0125, 8, True), (0.3 / 4, 16, False), (1.0 / 4, 1, True),
+                                                 (0.0125, 3, False)])
+def test_backward_n16_cayley_tensor_cores(alpha, chunk, with_s0):
+    """The n = 16 Cayley map's backward on the tensor cores: F formed per
+    stage as in the forward, dA = 2 T + T F^T with T = dX + F^T dX / 2, dM =
+    alpha (dA - dA^T) / 2, all in split tf32; chunks of 1, 3, 8 and 16 over
+    L = 45 (ragged), near and far from the identity, with and without S0."""
+    t = torch()
+    n = 16
+    w = gen.Workload("b16c", B=2, H=2, L=45, n=n, x_dtype="f32", mode=gen.MODE_CAYLEY, alpha=float(alpha), seed=630)
+    x = gen.make_x(w)
+    S0 = gen.make_S0(w, seed=631) if with_s0 else None
+    dS = np.random.default_rng(632 + chunk).standard_normal((w.B, w.L, w.H, n, n)).astype(np.float32)
+    p = mru.problem_from_workload(w, chunk=chunk)
+    xd = to_device_x(x)
+    S0d = None if S0 is None else t.from_numpy(np.ascontiguousarray(S0, np.float32)).cuda()
+    S = mru.scan_fused_t(p, xd, S0=S0d)
+    dx, dS0, ws = mru.scan_backward_t(p, xd, S, t.from_numpy(dS).cuda(), S0=S0d)
+    assert mru.last_device_status(ws.data_ptr(), t.cuda.current_stream().cuda_stream) == mru.OK
+    dx_o, dS0_o = oracle.backward(oracle_problem(w), x, dS.astype(np.float64),
+                                  S0=None if S0 is None else S0.astype(np.float64))
+    e = _rel(dx.cpu().numpy().astype(np.float64).reshape(w.B, w.L, w.H, n * n), dx_o.reshape(w.B, w.L, w.H, n * n),
+             axis=-1)
+    print("n16 Cayley backward: max", e.max(), "median", np.median(e))
+    assert e.max() <= TOL_BWD, (e.max(), np.median(e))
+    if with_s0:
+        e0 = _rel(dS0.cpu().numpy().astype(np.float64).reshape(w.B, w.H, n * n), dS0_o.reshape(w.B, w.H, n * n),
+                  axis=-1)
+        assert e0.max() <= TOL_BWD, e0.max()
+
+
+def test_backward_n16_cayley_workload_sampled():
+    """The n = 16 Cayley workload (B8 H8 L4096) end to end on the tensor
+    cores; the oracle recomputes two sequences."""
+    t = torch()
+    w = gen.WORKLOADS["n16_cayley_b8h8l4096"]
+    x = gen.make_x(w)
+    dS = np.random.default_rng(7).standard_normal((w.B, w.L, w.H, 16, 16)).astype(np.float32)
+    p = mru.problem_from_workload(w)
+    xd = to_device_x(x)
+    S = mru.scan_fused_t(p, xd)
+    dx, _, ws = mru.scan_backward_t(p, xd, S, t.from_numpy(dS).cuda())
+    assert mru.last_device_status(ws.data_ptr(), t.cuda.current_stream().cuda_stream) == mru.OK
+    dx = dx.cpu().numpy().astype(np.float64).reshape(w.B, w.L, w.H, 256)
+    for b, h in [(0, 0), (6, 3)]:
+        w1 = gen.Workload("one", B=1, H=1, L=w.L, n=16, x_dtype="f32", mode=w.mode, alpha=w.alpha, seed=0)
+        x1 = np.ascontiguousarray(x.reshape(w.B, w.L, w.H, 256)[b:b + 1, :, h])
+        dS1 = dS[b:b + 1, :, h:h + 1].astype(np.float64)
+        dx_o, _ = oracle.backward(oracle_problem(w1), x1, dS1)
+        e = _rel(dx[b, :, h], dx_o.reshape(w.L, 256), axis=-1)
+        print("n16 Cayley workload backward:", b, h, e.max(), np.median(e))
+        assert e.max() <= TOL_BWD, (b, h, e.max(), np.median(e))
