@@ -408,3 +408,28 @@ def test_backward_n16_cayley_workload_sampled():
         e = _rel(dx[b, :, h], dx_o.reshape(w.L, 256), axis=-1)
         print("n16 Cayley workload backward:", b, h, e.max(), np.median(e))
         assert e.max() <= TOL_BWD, (b, h, e.max(), np.median(e))
+
+
+def test_backward_readout_n64_tensor_cores_long_sequence():
+    """The n = 64 readout backward in tf32 with the workload's construction
+    and default chunking over one sequence of 4096 tokens (64 chunks): the
+    tf32 rounding of the gradient chains accumulated over a quarter of the
+    workload's length, against the oracle."""
+    t = torch()
+    B, H, L, n = 1, 1, 4096, 64
+    w = gen.Workload("bro64l", B=B, H=H, L=L, n=n, x_dtype="f32", mode=gen.MODE_DETNORM, alpha=0.03 / 8,
+                     math="tf32", seed=1007)
+    x = gen.make_x(w)
+    r = np.random.default_rng(78)
+    u = r.standard_normal(n).astype(np.float32)
+    d_o = r.standard_normal((B, L, H, n, 1)).astype(np.float32)
+    d_snap = r.standard_normal((B, L // 256, H, n, n)).astype(np.float32)
+    p = mru.problem_from_workload(w)
+    dx, _, ws = mru.scan_backward_readout_t(p, to_device_x(x), t.from_numpy(u).cuda(), t.from_numpy(d_o).cuda(),
+                                            snapshot_every=256, d_snaps=t.from_numpy(d_snap).cuda())
+    assert mru.last_device_status(ws.data_ptr(), t.cuda.current_stream().cuda_stream) == mru.OK
+    dx_o, _ = oracle.backward_readout(oracle_problem(w), x, u.astype(np.float64), d_o[..., 0],
+                                      snapshot_every=256, d_snap=d_snap)
+    e = _rel(dx.cpu().numpy().astype(np.float64).reshape(B, L, H, n * n), dx_o.reshape(B, L, H, n * n), axis=-1)
+    print("n64 tensor-core readout backward, L = 4096: max", e.max(), "median", np.median(e))
+    assert e.max() <= TOL_BWD_TF32, (e.max(), np.median(e))
