@@ -169,7 +169,7 @@ struct Series {
 //   |R| <= |E^3|_F |E^2|_F / (5 (1 - |E|_F)),
 // taken when that bound is at most 1e-6, like the forward kernel.  The
 // products are P2 = (M^T)^2 and P3 = P2 M^T (bf16 operands, fp32 accumulate):
-// tr M^3 = <P2, M> and tr M^4 = <P3, M>.  With WantY, Y = E2^T - E3^T =
+// tr M^3 = <P2, M> and tr M^4 = <P3, M>.  With WantY, Y = (E^T)^2 - (E^T)^3 =
 // alpha^2 P2 - alpha^3 P3 at this thread's accumulator positions when
 // inv_ok: the inverse's terms beyond I - E^T, the dropped tail bounded by
 // |E^3|_F |E|_F / (1 - |E|_F) <= 1e-3.
@@ -364,16 +364,15 @@ __device__ __forceinline__ void reload_slice(float* xs, const float* src)
     __syncthreads();
 }
 
-// F = ca M + dv I for this token: the scale of the construction (the
-// determinant's c from the series, else from the pivoted elimination),
-// SINGULAR recorded where it does not exist.  `xs` may be overwritten and
-// reloaded from `src`; Winv (apply pass, output tokens) receives Xr^-1 when
-// the elimination runs.  Returns whether the elimination ran.
+// A token's F = ca M + dv I and the determinant scale c.
 struct Scale {
     float ca, dv;                    // F = ca M + dv I
     float c;                         // determinant scale (1 for reshape, 0 when singular)
 };
 
+// The scale from c - 1 (cm1, from the series or the pivoted elimination;
+// good: the elimination found no zero pivot); SINGULAR is recorded, and F = 0,
+// where c does not exist.
 __device__ __forceinline__ Scale finish_scale(const KParams& p, bool detnorm, float cm1, bool good, uint32_t* status)
 {
     Scale s;
